@@ -1,0 +1,263 @@
+/*
+ * tp_layer.h -- C ABI of the B200 (sm_100a) tensor-parallel transformer
+ * sublayer library (libtplayer.so).
+ *
+ * The method is Megatron-LM's intra-layer (tensor) model parallelism
+ * (Shoeybi et al., 2019), as described on the pages
+ *   "Megatron-LM: what the tensor parallelism paper actually says"
+ *     - "How transformer layers actually decompose"  (MLP: W1 column split,
+ *       local GeLU, W2 row split, partial outputs summed),
+ *     - "The attention heads split" (Q/K/V split by head, local attention,
+ *       row-split output projection, partial outputs summed),
+ *     - "The layernorm placement the paper flags as critical" (pre-LN);
+ *   "Megatron-LM interactive explainer" - "One Idea, Two Insertions" (one
+ *       reduction in the forward and one in the backward of each pair).
+ * All t shards run on ONE GPU: the cross-shard all-reduce of the forward is
+ * the fp32 accumulation of the t partial products inside the row-parallel
+ * GEMM, and the backward reduction of input gradients is the same walk in
+ * the input-gradient GEMM.  No collective is issued.
+ *
+ * Conventions for every entry point
+ *  - Element type: bf16, passed as raw 16-bit patterns (tp_bf16).  fp32 where
+ *    stated.  Accumulation is fp32; outputs are rounded to nearest even once.
+ *  - Pointers: DEVICE pointers owned by the caller, 16-byte aligned, dense
+ *    row-major, unless stated otherwise.  The library allocates nothing and
+ *    keeps no state apart from cached per-device attributes.
+ *  - Shapes: T = batch*seq tokens (batch outer), D = hidden, F = ffn,
+ *    H = heads, dh = head_dim (D = H*dh), t = tensor-parallel degree,
+ *    Ft = F/t, Dt = D/t.  Activations x, y: [T][D].
+ *  - Shard-packed weights (each shard's block contiguous, the way one GPU
+ *    of a t-GPU group would hold it; tp_shard_* convert):
+ *      W1   [t][D][Ft]    column shards of W1 [D][F]
+ *      W2   [t][Ft][D]    row shards of W2 [F][D] (byte-identical to W2)
+ *      Wqkv [t][D][3*Dt]  shard i = [Wq_i | Wk_i | Wv_i], the columns of heads
+ *                         i*H/t .. (i+1)*H/t-1 of Wq, Wk, Wv [D][D]
+ *      Wout [t][Dt][D]    row shards of Wout [D][D]
+ *    Biases follow their matrix: b1 [t][Ft], bqkv [t][3*Dt], b2/bout [D].
+ *    The bias of a row-parallel product is added once, after the shard sum.
+ *  - Streams: every call only enqueues work on `stream` (a cudaStream_t, or
+ *    NULL for the legacy default stream) and returns; it never synchronises.
+ *  - Errors: no exception crosses the ABI.  Arguments are validated on the
+ *    host before anything is launched; on failure nothing is enqueued and a
+ *    status != TP_OK is returned.  Launch failures return TP_ERR_CUDA.  A
+ *    device-side wait that exceeds its bound (about 2 s) records a code in
+ *    the library's device error word and the kernel returns early; read it
+ *    with tp_check_error after synchronising.
+ */
+#ifndef TP_LAYER_H
+#define TP_LAYER_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t tp_bf16;  /* raw bfloat16 bits */
+typedef void* tp_stream;   /* cudaStream_t */
+
+typedef enum {
+  TP_OK = 0,
+  TP_ERR_INVALID_ARG = 1,  /* null pointer, non-positive size, t not dividing H or F, D != H*dh */
+  TP_ERR_UNSUPPORTED = 2,  /* valid but not provided: t not in {1,2,4,8}, dh not in {64,128} */
+  TP_ERR_MISALIGNED = 3,   /* pointer not 16-byte aligned or a row not a multiple of 8 elements */
+  TP_ERR_WORKSPACE = 4,    /* workspace pointer null or smaller than tp_workspace_size */
+  TP_ERR_CUDA = 5,         /* a CUDA runtime call or kernel launch failed */
+  TP_ERR_TIMEOUT = 6       /* a bounded device wait expired (from tp_check_error) */
+} tp_status;
+
+/* Sizes of one problem.  Fields an operation does not use are ignored
+ * (e.g. heads/head_dim for the MLP, ffn for attention). */
+typedef struct {
+  int batch;     /* B >= 1 */
+  int seq;       /* S >= 1; T = B*S */
+  int hidden;    /* D, multiple of 8*t */
+  int ffn;       /* F, multiple of 8*t */
+  int heads;     /* H, multiple of t */
+  int head_dim;  /* dh in {64, 128}, D = H*dh */
+  int t;         /* tensor-parallel degree in {1, 2, 4, 8} */
+  int causal;    /* attention mask: 1 = key s' visible to query s iff s' <= s; 0 = none */
+  float ln_eps;  /* LayerNorm epsilon (pre-LN layer only), > 0 */
+} tp_dims;
+
+typedef enum {
+  TP_OP_MLP_FWD = 0,
+  TP_OP_MLP_BWD = 1,
+  TP_OP_ATTN_FWD = 2,
+  TP_OP_ATTN_BWD = 3,
+  TP_OP_LAYER_FWD = 4,
+  TP_OP_LAYER_BWD = 5
+} tp_op;
+
+/* Version string of the library. */
+const char* tp_version(void);
+
+/* Human-readable name of a status code (static storage). */
+const char* tp_status_string(tp_status s);
+
+/* Bytes of device workspace operation `op` needs for `dims` (0 if none, or
+ * if the dims are invalid).  The workspace is scratch: its contents on entry
+ * are ignored and on return are unspecified.  Calls that may run at the same
+ * time need distinct workspaces. */
+size_t tp_workspace_size(int op, const tp_dims* dims);
+
+/* Synchronises the current device, then reads and clears the library's
+ * device error word.  TP_ERR_TIMEOUT if a bounded wait expired since the
+ * last call (the code is stored in *code if code != NULL), TP_ERR_CUDA if
+ * the synchronisation failed, TP_OK otherwise. */
+tp_status tp_check_error(unsigned int* code);
+
+/* ------------------------------------------------------------------ layout
+ * Slicing exactly as "How transformer layers actually decompose" and "The
+ * attention heads split" define it; bit-exact copies.  All on device,
+ * enqueued on `stream`; `src` and `dst` must not overlap. */
+
+/* W [rows][cols] -> [t][rows][cols/t]; shard i holds columns i*cols/t .. (i+1)*cols/t-1. */
+tp_status tp_shard_cols(const tp_bf16* w, int rows, int cols, int t, tp_bf16* out, tp_stream stream);
+/* Inverse of tp_shard_cols. */
+tp_status tp_unshard_cols(const tp_bf16* packed, int rows, int cols, int t, tp_bf16* w, tp_stream stream);
+/* W [rows][cols] -> [t][rows/t][cols]; shard i holds rows i*rows/t .. (i+1)*rows/t-1.
+ * The packed layout is byte-identical to W; this is a copy. */
+tp_status tp_shard_rows(const tp_bf16* w, int rows, int cols, int t, tp_bf16* out, tp_stream stream);
+/* Inverse of tp_shard_rows (a copy). */
+tp_status tp_unshard_rows(const tp_bf16* packed, int rows, int cols, int t, tp_bf16* w, tp_stream stream);
+/* Fused QKV matrix (or bias, rows = 1) [rows][3*hidden] = [Wq | Wk | Wv] ->
+ * [t][rows][3*hidden/t], shard i = [Wq_i | Wk_i | Wv_i] holding the columns of
+ * heads i*heads/t .. (i+1)*heads/t-1.  heads % t == 0 and hidden % heads == 0. */
+tp_status tp_shard_qkv_heads(const tp_bf16* w, int rows, int hidden, int heads, int t, tp_bf16* out,
+                             tp_stream stream);
+/* Inverse of tp_shard_qkv_heads. */
+tp_status tp_unshard_qkv_heads(const tp_bf16* packed, int rows, int hidden, int heads, int t,
+                               tp_bf16* w, tp_stream stream);
+
+/* ------------------------------------------------------------------ MLP
+ * "How transformer layers actually decompose": output = GeLU(x W1) W2 with
+ * W1 split by columns and W2 by rows; GeLU is the tanh form
+ * 0.5 a (1 + tanh(sqrt(2/pi) (a + 0.044715 a^3))).
+ *
+ * tp_mlp_fwd:
+ *   a_save[i] = x W1_i + b1_i             [t][T][Ft]   (pre-activation, saved)
+ *   h_save[i] = GeLU(a_save[i])          [t][T][Ft]   (activation, saved)
+ *   y = sum_{i=0..t-1} h_save[i] W2_i + b2 (+ resid)   [T][D]
+ * The shard sum is accumulated in fp32 in shard order and rounded once.
+ * b1, b2, resid may be NULL (zero).  Uses dims: batch, seq, hidden, ffn, t.
+ * No workspace (pass NULL, 0). */
+tp_status tp_mlp_fwd(const tp_dims* dims, const tp_bf16* x, const tp_bf16* w1, const tp_bf16* b1,
+                     const tp_bf16* w2, const tp_bf16* b2, const tp_bf16* resid, tp_bf16* y,
+                     tp_bf16* a_save, tp_bf16* h_save, void* ws, size_t ws_bytes, tp_stream stream);
+
+/* tp_mlp_bwd: vector-Jacobian product of tp_mlp_fwd for upstream gradient dy [T][D]:
+ *   dA_i  = (dy W2_i^T) * GeLU'(a_save[i])          (workspace)
+ *   dw2_i = h_save[i]^T dy       [t][Ft][D]
+ *   dw1_i = x^T dA_i             [t][D][Ft]
+ *   dx    = sum_i dA_i W1_i^T (+ dres)   [T][D]     (backward shard reduction)
+ *   db1   = column sums of dA [t][Ft], db2 = column sums of dy [D]
+ * dres (the gradient arriving through a residual branch) and db1/db2 may be
+ * NULL.  Workspace: tp_workspace_size(TP_OP_MLP_BWD, dims) bytes. */
+tp_status tp_mlp_bwd(const tp_dims* dims, const tp_bf16* x, const tp_bf16* w1, const tp_bf16* w2,
+                     const tp_bf16* a_save, const tp_bf16* h_save, const tp_bf16* dy,
+                     const tp_bf16* dres, tp_bf16* dx, tp_bf16* dw1, tp_bf16* dw2, tp_bf16* db1,
+                     tp_bf16* db2, void* ws, size_t ws_bytes, tp_stream stream);
+
+/* ------------------------------------------------------------------ attention
+ * "The attention heads split": shard i owns heads i*H/t .. (i+1)*H/t-1.
+ *
+ * tp_attn_fwd:
+ *   qkv_save[i] = x Wqkv_i + bqkv_i        [t][T][3*Dt]; within shard i, columns
+ *                 [0,Dt) are q, [Dt,2Dt) k, [2Dt,3Dt) v, local head j at j*dh
+ *   per head:  O = softmax(q k^T / sqrt(dh) + mask) v, softmax in fp32;
+ *              lse_save = log-sum-exp of the scaled masked scores, fp32 [B][H][S]
+ *   o_save[i]   = the shard's head outputs  [t][T][Dt]
+ *   y = sum_i o_save[i] Wout_i + bout (+ resid)      [T][D]
+ * bqkv, bout, resid may be NULL.  Uses batch, seq, hidden, heads, head_dim, t,
+ * causal.  No workspace. */
+tp_status tp_attn_fwd(const tp_dims* dims, const tp_bf16* x, const tp_bf16* wqkv,
+                      const tp_bf16* bqkv, const tp_bf16* wout, const tp_bf16* bout,
+                      const tp_bf16* resid, tp_bf16* y, tp_bf16* qkv_save, tp_bf16* o_save,
+                      float* lse_save, void* ws, size_t ws_bytes, tp_stream stream);
+
+/* tp_attn_bwd: vector-Jacobian product of tp_attn_fwd for dy [T][D]:
+ *   dO_i = dy Wout_i^T; dwout_i = o_save[i]^T dy   [t][Dt][D]
+ *   per head: dv = P^T dO, dP = dO v^T, dS = P * (dP - rowsum(dO * O)),
+ *             dq = dS k / sqrt(dh), dk = dS^T q / sqrt(dh)     (P recomputed from lse)
+ *   dwqkv_i = x^T dqkv_i  [t][D][3*Dt];  dx = sum_i dqkv_i Wqkv_i^T (+ dres)
+ *   dbqkv = column sums of dqkv [t][3*Dt], dbout = column sums of dy [D]
+ * dres, dbqkv, dbout may be NULL.  Workspace: tp_workspace_size(TP_OP_ATTN_BWD). */
+tp_status tp_attn_bwd(const tp_dims* dims, const tp_bf16* x, const tp_bf16* wqkv,
+                      const tp_bf16* wout, const tp_bf16* qkv_save, const tp_bf16* o_save,
+                      const float* lse_save, const tp_bf16* dy, const tp_bf16* dres, tp_bf16* dx,
+                      tp_bf16* dwqkv, tp_bf16* dbqkv, tp_bf16* dwout, tp_bf16* dbout, void* ws,
+                      size_t ws_bytes, tp_stream stream);
+
+/* ------------------------------------------------------------------ pre-LN layer
+ * "The layernorm placement the paper flags as critical":
+ *   h = x + Attn(LN1(x));  y = h + MLP(LN2(h))
+ * LayerNorm: biased variance over D, eps = dims->ln_eps, affine gamma/beta
+ * (bf16); mean and rstd saved in fp32.  Dropout is not applied. */
+typedef struct {
+  const tp_bf16 *ln1_g, *ln1_b;   /* [D] */
+  const tp_bf16 *wqkv, *bqkv;     /* [t][D][3Dt], [t][3Dt] (bqkv may be NULL) */
+  const tp_bf16 *wout, *bout;     /* [t][Dt][D], [D] (bout may be NULL) */
+  const tp_bf16 *ln2_g, *ln2_b;   /* [D] */
+  const tp_bf16 *w1, *b1;         /* [t][D][Ft], [t][Ft] (b1 may be NULL) */
+  const tp_bf16 *w2, *b2;         /* [t][Ft][D], [D] (b2 may be NULL) */
+} tp_layer_params;
+
+/* Activations saved by tp_layer_fwd for tp_layer_bwd (all caller-owned). */
+typedef struct {
+  tp_bf16* u1;            /* LN1(x) [T][D] */
+  float *mean1, *rstd1;   /* [T] */
+  tp_bf16* qkv;           /* [t][T][3Dt] */
+  tp_bf16* o;             /* [t][T][Dt] */
+  float* lse;             /* [B][H][S] */
+  tp_bf16* h;             /* x + attention output [T][D] */
+  tp_bf16* u2;            /* LN2(h) [T][D] */
+  float *mean2, *rstd2;   /* [T] */
+  tp_bf16* a;             /* MLP pre-activation [t][T][Ft] */
+  tp_bf16* hact;          /* MLP activation [t][T][Ft] */
+} tp_layer_acts;
+
+/* Parameter gradients written by tp_layer_bwd (same layouts as the parameters;
+ * any bias / LayerNorm gradient pointer may be NULL to skip it). */
+typedef struct {
+  tp_bf16 *dln1_g, *dln1_b, *dwqkv, *dbqkv, *dwout, *dbout;
+  tp_bf16 *dln2_g, *dln2_b, *dw1, *db1, *dw2, *db2;
+} tp_layer_grads;
+
+/* tp_layer_fwd: x [T][D] -> y [T][D], filling every field of *acts.
+ * No workspace. */
+tp_status tp_layer_fwd(const tp_dims* dims, const tp_bf16* x, const tp_layer_params* params,
+                       const tp_layer_acts* acts, tp_bf16* y, void* ws, size_t ws_bytes,
+                       tp_stream stream);
+
+/* tp_layer_bwd: dy [T][D] -> dx [T][D] and *grads, from the activations that
+ * tp_layer_fwd saved for the same x and params.
+ *   dh = dy + LN2^T(MLP^T(dy));  dx = dh + LN1^T(Attn^T(dh))
+ * Workspace: tp_workspace_size(TP_OP_LAYER_BWD, dims) bytes. */
+tp_status tp_layer_bwd(const tp_dims* dims, const tp_bf16* x, const tp_layer_params* params,
+                       const tp_layer_acts* acts, const tp_bf16* dy, tp_bf16* dx,
+                       const tp_layer_grads* grads, void* ws, size_t ws_bytes, tp_stream stream);
+
+/* ------------------------------------------------------------------ LayerNorm
+ * The pre-LN building block on its own ("The layernorm placement the paper
+ * flags as critical"), exposed for tests and for callers composing layers.
+ *   tp_layernorm_fwd: y = (x - mean) * rstd * gamma + beta per row of x [rows][D];
+ *                     mean, rstd fp32 [rows].  No workspace.
+ *   tp_layernorm_bwd: dx = rstd (g - mean(g) - xhat mean(g xhat)) (+ dres),
+ *                     g = dy * gamma; dgamma = sum_rows dy*xhat, dbeta = sum_rows dy.
+ *                     dres, dgamma, dbeta may be NULL.
+ *                     Workspace: tp_layernorm_bwd_workspace_size(rows, D). */
+tp_status tp_layernorm_fwd(const tp_bf16* x, const tp_bf16* gamma, const tp_bf16* beta, int rows,
+                           int D, float eps, tp_bf16* y, float* mean, float* rstd, tp_stream stream);
+size_t tp_layernorm_bwd_workspace_size(int rows, int D);
+tp_status tp_layernorm_bwd(const tp_bf16* dy, const tp_bf16* x, const tp_bf16* gamma,
+                           const float* mean, const float* rstd, const tp_bf16* dres, int rows,
+                           int D, tp_bf16* dx, tp_bf16* dgamma, tp_bf16* dbeta, void* ws,
+                           size_t ws_bytes, tp_stream stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TP_LAYER_H */

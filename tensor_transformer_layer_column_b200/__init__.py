@@ -1,0 +1,267 @@
+"""Python binding of libtplayer.so, the B200 tensor-parallel sublayer library.
+
+Argument marshalling only: every entry point forwards device pointers and
+sizes to the C ABI declared in include/tp_layer.h, and every step of the
+computation runs in the library's CUDA kernels.  There is no CPU fallback:
+if the shared library is missing, calling any entry point raises.
+
+Tensors are ``torch`` CUDA tensors (bf16 unless stated) or raw integer
+device addresses; ``None`` passes NULL.  The stream defaults to torch's
+current stream of the tensors' device.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+__all__ = [
+    "TpError", "Dims", "LayerParams", "LayerActs", "LayerGrads", "lib", "lib_path",
+    "OP_MLP_FWD", "OP_MLP_BWD", "OP_ATTN_FWD", "OP_ATTN_BWD", "OP_LAYER_FWD", "OP_LAYER_BWD",
+    "workspace_size", "check_error", "version", "EXPORTED_SYMBOLS",
+    "shard_cols", "unshard_cols", "shard_rows", "unshard_rows", "shard_qkv_heads",
+    "unshard_qkv_heads", "mlp_fwd", "mlp_bwd", "attn_fwd", "attn_bwd", "layer_fwd", "layer_bwd",
+    "layernorm_fwd", "layernorm_bwd", "layernorm_bwd_workspace_size",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+lib_path = os.path.join(_HERE, "libtplayer.so")
+
+OP_MLP_FWD, OP_MLP_BWD, OP_ATTN_FWD, OP_ATTN_BWD, OP_LAYER_FWD, OP_LAYER_BWD = range(6)
+
+STATUS_NAMES = {0: "TP_OK", 1: "TP_ERR_INVALID_ARG", 2: "TP_ERR_UNSUPPORTED",
+                3: "TP_ERR_MISALIGNED", 4: "TP_ERR_WORKSPACE", 5: "TP_ERR_CUDA",
+                6: "TP_ERR_TIMEOUT"}
+
+
+class TpError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS_NAMES.get(status, status)}")
+
+
+class Dims(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int), ("seq", ctypes.c_int), ("hidden", ctypes.c_int),
+                ("ffn", ctypes.c_int), ("heads", ctypes.c_int), ("head_dim", ctypes.c_int),
+                ("t", ctypes.c_int), ("causal", ctypes.c_int), ("ln_eps", ctypes.c_float)]
+
+    @classmethod
+    def of(cls, batch, seq, hidden, ffn=0, heads=0, head_dim=0, t=1, causal=1, ln_eps=1e-5):
+        return cls(batch, seq, hidden, ffn, heads, head_dim, t, causal, ln_eps)
+
+
+_P = ctypes.c_void_p
+
+
+class LayerParams(ctypes.Structure):
+    _fields_ = [(n, _P) for n in ("ln1_g", "ln1_b", "wqkv", "bqkv", "wout", "bout",
+                                  "ln2_g", "ln2_b", "w1", "b1", "w2", "b2")]
+
+
+class LayerActs(ctypes.Structure):
+    _fields_ = [(n, _P) for n in ("u1", "mean1", "rstd1", "qkv", "o", "lse", "h", "u2",
+                                  "mean2", "rstd2", "a", "hact")]
+
+
+class LayerGrads(ctypes.Structure):
+    _fields_ = [(n, _P) for n in ("dln1_g", "dln1_b", "dwqkv", "dbqkv", "dwout", "dbout",
+                                  "dln2_g", "dln2_b", "dw1", "db1", "dw2", "db2")]
+
+
+# name -> argument types (all return tp_status unless listed in _RESTYPES)
+_SIGS = {
+    "tp_version": [],
+    "tp_status_string": [ctypes.c_int],
+    "tp_workspace_size": [ctypes.c_int, ctypes.POINTER(Dims)],
+    "tp_check_error": [ctypes.POINTER(ctypes.c_uint)],
+    "tp_shard_cols": [_P, ctypes.c_int, ctypes.c_int, ctypes.c_int, _P, _P],
+    "tp_unshard_cols": [_P, ctypes.c_int, ctypes.c_int, ctypes.c_int, _P, _P],
+    "tp_shard_rows": [_P, ctypes.c_int, ctypes.c_int, ctypes.c_int, _P, _P],
+    "tp_unshard_rows": [_P, ctypes.c_int, ctypes.c_int, ctypes.c_int, _P, _P],
+    "tp_shard_qkv_heads": [_P, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, _P, _P],
+    "tp_unshard_qkv_heads": [_P, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, _P, _P],
+    "tp_mlp_fwd": [ctypes.POINTER(Dims)] + [_P] * 9 + [_P, ctypes.c_size_t, _P],
+    "tp_mlp_bwd": [ctypes.POINTER(Dims)] + [_P] * 12 + [_P, ctypes.c_size_t, _P],
+    "tp_attn_fwd": [ctypes.POINTER(Dims)] + [_P] * 10 + [_P, ctypes.c_size_t, _P],
+    "tp_attn_bwd": [ctypes.POINTER(Dims)] + [_P] * 13 + [_P, ctypes.c_size_t, _P],
+    "tp_layer_fwd": [ctypes.POINTER(Dims), _P, ctypes.POINTER(LayerParams),
+                     ctypes.POINTER(LayerActs), _P, _P, ctypes.c_size_t, _P],
+    "tp_layer_bwd": [ctypes.POINTER(Dims), _P, ctypes.POINTER(LayerParams),
+                     ctypes.POINTER(LayerActs), _P, _P, ctypes.POINTER(LayerGrads), _P,
+                     ctypes.c_size_t, _P],
+    "tp_layernorm_fwd": [_P, _P, _P, ctypes.c_int, ctypes.c_int, ctypes.c_float, _P, _P, _P, _P],
+    "tp_layernorm_bwd_workspace_size": [ctypes.c_int, ctypes.c_int],
+    "tp_layernorm_bwd": [_P, _P, _P, _P, _P, _P, ctypes.c_int, ctypes.c_int, _P, _P, _P, _P,
+                         ctypes.c_size_t, _P],
+}
+_RESTYPES = {"tp_version": ctypes.c_char_p, "tp_status_string": ctypes.c_char_p,
+             "tp_workspace_size": ctypes.c_size_t,
+             "tp_layernorm_bwd_workspace_size": ctypes.c_size_t}
+EXPORTED_SYMBOLS = tuple(_SIGS)
+
+_lib: Optional[ctypes.CDLL] = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libtplayer.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(lib_path):
+            raise RuntimeError(f"{lib_path} is missing: build it with "
+                               "`python -m tensor_transformer_layer_column_b200.build`")
+        handle = ctypes.CDLL(lib_path)
+        for name, args in _SIGS.items():
+            fn = getattr(handle, name)
+            fn.argtypes = args
+            fn.restype = _RESTYPES.get(name, ctypes.c_int)
+        _lib = handle
+    return _lib
+
+
+def _ptr(x) -> Optional[int]:
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    if not x.is_cuda:
+        raise ValueError("tensor arguments must live on a CUDA device")
+    if not x.is_contiguous():
+        raise ValueError("tensor arguments must be contiguous")
+    return x.data_ptr()
+
+
+def _stream(stream, *tensors) -> Optional[int]:
+    if stream is not None:
+        return stream if isinstance(stream, int) else stream.cuda_stream
+    import torch
+    for t in tensors:
+        if t is not None and not isinstance(t, int):
+            return torch.cuda.current_stream(t.device).cuda_stream
+    return torch.cuda.current_stream().cuda_stream
+
+
+def _check(status: int, where: str):
+    if status != 0:
+        raise TpError(status, where)
+
+
+def version() -> str:
+    return lib().tp_version().decode()
+
+
+def workspace_size(op: int, dims: Dims) -> int:
+    return lib().tp_workspace_size(op, ctypes.byref(dims))
+
+
+def check_error() -> int:
+    """Synchronise and return the device error word (0 if no bounded wait expired)."""
+    code = ctypes.c_uint(0)
+    st = lib().tp_check_error(ctypes.byref(code))
+    if st not in (0, 6):
+        raise TpError(st, "tp_check_error")
+    return code.value
+
+
+def _ws(ws):
+    if ws is None:
+        return None, 0
+    if isinstance(ws, tuple):
+        return ws
+    return ws.data_ptr(), ws.numel() * ws.element_size()
+
+
+# ---------------------------------------------------------------- layout
+def shard_cols(w, rows, cols, t, out, stream=None):
+    _check(lib().tp_shard_cols(_ptr(w), rows, cols, t, _ptr(out), _stream(stream, w)), "tp_shard_cols")
+
+
+def unshard_cols(p, rows, cols, t, out, stream=None):
+    _check(lib().tp_unshard_cols(_ptr(p), rows, cols, t, _ptr(out), _stream(stream, p)), "tp_unshard_cols")
+
+
+def shard_rows(w, rows, cols, t, out, stream=None):
+    _check(lib().tp_shard_rows(_ptr(w), rows, cols, t, _ptr(out), _stream(stream, w)), "tp_shard_rows")
+
+
+def unshard_rows(p, rows, cols, t, out, stream=None):
+    _check(lib().tp_unshard_rows(_ptr(p), rows, cols, t, _ptr(out), _stream(stream, p)), "tp_unshard_rows")
+
+
+def shard_qkv_heads(w, rows, hidden, heads, t, out, stream=None):
+    _check(lib().tp_shard_qkv_heads(_ptr(w), rows, hidden, heads, t, _ptr(out), _stream(stream, w)),
+           "tp_shard_qkv_heads")
+
+
+def unshard_qkv_heads(p, rows, hidden, heads, t, out, stream=None):
+    _check(lib().tp_unshard_qkv_heads(_ptr(p), rows, hidden, heads, t, _ptr(out),
+                                      _stream(stream, p)), "tp_unshard_qkv_heads")
+
+
+# ---------------------------------------------------------------- sublayers
+def mlp_fwd(dims, x, w1, b1, w2, b2, resid, y, a_save, h_save, ws=None, stream=None):
+    wp, wn = _ws(ws)
+    _check(lib().tp_mlp_fwd(ctypes.byref(dims), _ptr(x), _ptr(w1), _ptr(b1), _ptr(w2), _ptr(b2),
+                            _ptr(resid), _ptr(y), _ptr(a_save), _ptr(h_save), wp, wn,
+                            _stream(stream, x)), "tp_mlp_fwd")
+
+
+def mlp_bwd(dims, x, w1, w2, a_save, h_save, dy, dres, dx, dw1, dw2, db1, db2, ws, stream=None):
+    wp, wn = _ws(ws)
+    _check(lib().tp_mlp_bwd(ctypes.byref(dims), _ptr(x), _ptr(w1), _ptr(w2), _ptr(a_save),
+                            _ptr(h_save), _ptr(dy), _ptr(dres), _ptr(dx), _ptr(dw1), _ptr(dw2),
+                            _ptr(db1), _ptr(db2), wp, wn, _stream(stream, x)), "tp_mlp_bwd")
+
+
+def attn_fwd(dims, x, wqkv, bqkv, wout, bout, resid, y, qkv_save, o_save, lse_save, ws=None,
+             stream=None):
+    wp, wn = _ws(ws)
+    _check(lib().tp_attn_fwd(ctypes.byref(dims), _ptr(x), _ptr(wqkv), _ptr(bqkv), _ptr(wout),
+                             _ptr(bout), _ptr(resid), _ptr(y), _ptr(qkv_save), _ptr(o_save),
+                             _ptr(lse_save), wp, wn, _stream(stream, x)), "tp_attn_fwd")
+
+
+def attn_bwd(dims, x, wqkv, wout, qkv_save, o_save, lse_save, dy, dres, dx, dwqkv, dbqkv, dwout,
+             dbout, ws, stream=None):
+    wp, wn = _ws(ws)
+    _check(lib().tp_attn_bwd(ctypes.byref(dims), _ptr(x), _ptr(wqkv), _ptr(wout), _ptr(qkv_save),
+                             _ptr(o_save), _ptr(lse_save), _ptr(dy), _ptr(dres), _ptr(dx),
+                             _ptr(dwqkv), _ptr(dbqkv), _ptr(dwout), _ptr(dbout), wp, wn,
+                             _stream(stream, x)), "tp_attn_bwd")
+
+
+def _struct(cls, d):
+    return cls(**{k: _ptr(v) for k, v in d.items()})
+
+
+def layer_fwd(dims, x, params: dict, acts: dict, y, ws=None, stream=None):
+    wp, wn = _ws(ws)
+    p = _struct(LayerParams, params)
+    a = _struct(LayerActs, acts)
+    _check(lib().tp_layer_fwd(ctypes.byref(dims), _ptr(x), ctypes.byref(p), ctypes.byref(a),
+                              _ptr(y), wp, wn, _stream(stream, x)), "tp_layer_fwd")
+
+
+def layer_bwd(dims, x, params: dict, acts: dict, dy, dx, grads: dict, ws, stream=None):
+    wp, wn = _ws(ws)
+    p = _struct(LayerParams, params)
+    a = _struct(LayerActs, acts)
+    g = _struct(LayerGrads, grads)
+    _check(lib().tp_layer_bwd(ctypes.byref(dims), _ptr(x), ctypes.byref(p), ctypes.byref(a),
+                              _ptr(dy), _ptr(dx), ctypes.byref(g), wp, wn, _stream(stream, x)),
+           "tp_layer_bwd")
+
+
+def layernorm_fwd(x, gamma, beta, rows, D, eps, y, mean, rstd, stream=None):
+    _check(lib().tp_layernorm_fwd(_ptr(x), _ptr(gamma), _ptr(beta), rows, D, eps, _ptr(y),
+                                  _ptr(mean), _ptr(rstd), _stream(stream, x)), "tp_layernorm_fwd")
+
+
+def layernorm_bwd_workspace_size(rows, D) -> int:
+    return lib().tp_layernorm_bwd_workspace_size(rows, D)
+
+
+def layernorm_bwd(dy, x, gamma, mean, rstd, dres, rows, D, dx, dgamma, dbeta, ws, stream=None):
+    wp, wn = _ws(ws)
+    _check(lib().tp_layernorm_bwd(_ptr(dy), _ptr(x), _ptr(gamma), _ptr(mean), _ptr(rstd),
+                                  _ptr(dres), rows, D, _ptr(dx), _ptr(dgamma), _ptr(dbeta), wp,
+                                  wn, _stream(stream, x)), "tp_layernorm_bwd")

@@ -1,0 +1,896 @@
+// Per-head causal attention on tcgen05, over the shard-packed projections.
+//
+// "The attention heads split": shard i owns heads i*H/t .. (i+1)*H/t-1 and
+// runs full attention for them with no communication.  The projections arrive
+// as qkv [t][T][3Dt] (the column-parallel GEMM's output): local head j of
+// shard i has q at columns j*dh, k at Dt + j*dh, v at 2Dt + j*dh of rows
+// b*S + s.  One launch covers every head of every shard.
+//
+// Forward (per 128-query block, head, batch):
+//   S = q k^T (tcgen05, fp32 in TMEM, double-buffered), online softmax in
+//   fp32 by one thread per query row (base-2 exponent, scores pre-scaled by
+//   log2(e)/sqrt(dh)), P rounded to bf16 into swizzled shared memory,
+//   O += P v (tcgen05, fp32 in TMEM, rescaled in place when the row max moves).
+//   Writes O [t][T][Dt] (bf16) and the log-sum-exp [B][H][S] (fp32).
+// Backward (P recomputed from the log-sum-exp; no atomics, deterministic):
+//   prep:   Dv = rowsum(dO * O), lse2 = lse * log2(e)
+//   dK/dV:  per 128-key block, walk 64-query blocks:  S^T = k q^T, dP^T = v dO^T,
+//           P^T, dS^T = P^T * (dP^T - Dv) by one thread per key row,
+//           dV += P^T dO, dK += dS^T q
+//   dQ:     per 128-query block, walk 64-key blocks: S = q k^T, dP = dO v^T,
+//           dS = P * (dP - Dv), dQ += dS k
+// Every wait is bounded (about 2 s); a timeout records an error code and the
+// kernel drains its copies and MMAs, frees TMEM and returns.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+#include "internal.h"
+#include "sm100_ptx.cuh"
+
+namespace tp {
+
+namespace {
+
+enum : unsigned int {
+  ERR_ATTN_FWD_WAIT = 0x201,
+  ERR_ATTN_DKDV_WAIT = 0x202,
+  ERR_ATTN_DQ_WAIT = 0x203,
+};
+
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+struct AttnArgs {
+  int B, S, H, Ht, Dt, t;
+  int causal;
+  long long T;
+  float scale_log2;     // log2(e) / sqrt(dh)
+  float inv_sqrt_dh;
+  uint16_t* out;        // fwd: o_save [t][T][Dt]; bwd: dqkv [t][T][3Dt]
+  float* lse;           // fwd: lse [B][H][S]
+  const float* lse2;    // bwd: lse * log2(e), [B][H][S]
+  const float* dvec;    // bwd: rowsum(dO * O), [B][H][S]
+  unsigned int* err;
+};
+
+struct Ctl {
+  volatile int* abort_flag;
+  unsigned int* err;
+};
+
+__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, const Ctl& c,
+                                         unsigned int code) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*c.abort_flag || globaltimer_ns() - t0 > 2000000000ull) {
+      *c.abort_flag = 1;
+      if (c.err) atomicCAS(c.err, 0u, code);
+      return false;
+    }
+  }
+}
+
+__device__ __forceinline__ uint4 pack8_bf16(const float* v) {
+  uint4 o;
+  o.x = pack_bf16x2(v[0], v[1]);
+  o.y = pack_bf16x2(v[2], v[3]);
+  o.z = pack_bf16x2(v[4], v[5]);
+  o.w = pack_bf16x2(v[6], v[7]);
+  return o;
+}
+
+// K-major operand descriptor for a tile of R rows x (64*chunks) columns, at K step kk (16 cols).
+__device__ __forceinline__ uint64_t kmajor_desc(uint32_t base, int R, int kk) {
+  return smem_desc_sw128(base + (kk >> 2) * R * 128 + (kk & 3) * 32, 16, 1024);
+}
+
+// MN-major operand descriptor: tile rows are the K index (R rows), columns the
+// M/N index in 64-wide chunks of R*128 bytes; K step kk covers rows 16kk..16kk+15.
+__device__ __forceinline__ uint64_t mnmajor_desc(uint32_t base, int R, int kk) {
+  return smem_desc_sw128(base + kk * 2048, R * 128, 1024);
+}
+
+// =====================================================================================
+// Forward
+// =====================================================================================
+template <int DH>
+struct FwdCfg {
+  static constexpr int BM = 128, BN = 128, CH = DH / 64;
+  static constexpr int Q_BYTES = BM * DH * 2;
+  static constexpr int KV_BYTES = BN * DH * 2;
+  static constexpr int P_BYTES = BM * BN * 2;
+  static constexpr int OFF_K = Q_BYTES;                      // K[s] = OFF_K + s*2*KV, V[s] = +KV
+  static constexpr int OFF_P = Q_BYTES + 4 * KV_BYTES;
+  static constexpr int OFF_BAR = OFF_P + P_BYTES;
+  static constexpr int RAW = OFF_BAR + 256 + 1024;
+  // One CTA per SM: the kernel holds all 512 TMEM columns.
+  static constexpr int SMEM = RAW > 120 * 1024 ? RAW : 120 * 1024;
+};
+
+template <int DH>
+__global__ void __launch_bounds__(192, 1)
+attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_qkv, const AttnArgs p) {
+  using C = FwdCfg<DH>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint64_t* q_full = bars + 0;
+  uint64_t* kv_full = bars + 1;     // [2]
+  uint64_t* kv_empty = bars + 3;    // [2]
+  uint64_t* s_full = bars + 5;      // [2]
+  uint64_t* s_free = bars + 7;      // [2]
+  uint64_t* p_full = bars + 9;
+  uint64_t* pv_done = bars + 10;
+  uint64_t* drain = bars + 11;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 12);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nqb = (p.S + C::BM - 1) / C::BM;
+  const int qb = p.causal ? nqb - 1 - (int)blockIdx.x : (int)blockIdx.x;
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int shard = h / p.Ht, hl = h - shard * p.Ht;
+  const int q0 = qb * C::BM;
+  const int nkb = (p.S + C::BN - 1) / C::BN;
+  const int n_kv = p.causal ? min(nkb, qb + 1) : nkb;
+  const int colq = hl * DH, colk = p.Dt + hl * DH, colv = 2 * p.Dt + hl * DH;
+  const Ctl ctl{abort_flag, p.err};
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&kv_full[i], 1);
+      mbar_init(&kv_empty[i], 1);
+      mbar_init(&s_full[i], 1);
+      mbar_init(&s_free[i], 128);
+    }
+    mbar_init(p_full, 128);
+    mbar_init(pv_done, 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tm_qkv);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t t_s0 = tmem, t_o = tmem + 256;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      uint8_t* sq = smem;
+      mbar_arrive_expect_tx(q_full, C::Q_BYTES);
+      for (int c = 0; c < C::CH; ++c)
+        tma_load_4d(sq + c * C::BM * 128, &tm_qkv, q_full, colq + 64 * c, q0, b, shard);
+      int j = 0;
+      for (; j < n_kv; ++j) {
+        const int st = j & 1;
+        const uint32_t u = j >> 1;
+        if (!wait_bar(&kv_empty[st], (u & 1) ^ 1, ctl, ERR_ATTN_FWD_WAIT)) break;
+        uint8_t* sk = smem + C::OFF_K + st * 2 * C::KV_BYTES;
+        uint8_t* sv = sk + C::KV_BYTES;
+        mbar_arrive_expect_tx(&kv_full[st], 2 * C::KV_BYTES);
+        for (int c = 0; c < C::CH; ++c) {
+          tma_load_4d(sk + c * C::BN * 128, &tm_qkv, &kv_full[st], colk + 64 * c, j * C::BN, b, shard);
+          tma_load_4d(sv + c * C::BN * 128, &tm_qkv, &kv_full[st], colv + 64 * c, j * C::BN, b, shard);
+        }
+      }
+      // Let the copies this thread issued land before the CTA may exit.
+      mbar_wait(q_full, 0, 200000000ull);
+      for (int i = j - 1; i >= 0 && i >= j - 2; --i) mbar_wait(&kv_full[i & 1], (i >> 1) & 1, 200000000ull);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t id_qk = idesc_bf16_f32(128, 128, false, false);
+      constexpr uint32_t id_pv = idesc_bf16_f32(128, DH, false, true);
+      const uint32_t sq = smem_u32(smem), sp = smem_u32(smem + C::OFF_P);
+      bool ok = wait_bar(q_full, 0, ctl, ERR_ATTN_FWD_WAIT);
+      for (int j = 0; ok && j <= n_kv; ++j) {
+        if (j < n_kv) {
+          const int st = j & 1;
+          const uint32_t u = j >> 1;
+          if (!wait_bar(&kv_full[st], u & 1, ctl, ERR_ATTN_FWD_WAIT)) break;
+          if (!wait_bar(&s_free[st], (u & 1) ^ 1, ctl, ERR_ATTN_FWD_WAIT)) break;
+          tc_fence_after();
+          const uint32_t sk = smem_u32(smem + C::OFF_K + st * 2 * C::KV_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < DH / 16; ++kk)
+            tc_mma_f16(t_s0 + st * 128, kmajor_desc(sq, C::BM, kk), kmajor_desc(sk, C::BN, kk),
+                       id_qk, kk > 0);
+          tc_commit(&s_full[st]);
+        }
+        if (j > 0) {
+          const int jj = j - 1, st = jj & 1;
+          if (!wait_bar(p_full, jj & 1, ctl, ERR_ATTN_FWD_WAIT)) break;
+          tc_fence_after();
+          const uint32_t sv = smem_u32(smem + C::OFF_K + st * 2 * C::KV_BYTES + C::KV_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < C::BN / 16; ++kk)
+            tc_mma_f16(t_o, kmajor_desc(sp, C::BM, kk), mnmajor_desc(sv, C::BN, kk), id_pv,
+                       (jj | kk) != 0);
+          tc_commit(pv_done);
+          tc_commit(&kv_empty[st]);
+        }
+      }
+      tc_commit(drain);
+      mbar_wait(drain, 0, 200000000ull);
+    }
+  } else {
+    // ---------------------------------------------------------------- softmax warps
+    const int quad = warp & 3;
+    const int r = quad * 32 + lane;
+    const int q = q0 + r;
+    const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+    uint8_t* sp = smem + C::OFF_P;
+    float m = -1e30f, l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < n_kv; ++j) {
+      const int st = j & 1;
+      if (!__all_sync(0xffffffffu, wait_bar(&s_full[st], (j >> 1) & 1, ctl, ERR_ATTN_FWD_WAIT))) { ok = false; break; }
+      tc_fence_after();
+      float s[128];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t rr[32];
+        tmem_ld32(t_s0 + st * 128 + lane_off + c * 32, rr);
+        tc_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) s[c * 32 + e] = __uint_as_float(rr[e]);
+      }
+      tc_fence_before();
+      mbar_arrive(&s_free[st]);
+      const int k0 = j * C::BN;
+      const bool need_mask = (p.causal && k0 + C::BN - 1 > q0) || (k0 + C::BN > p.S);
+      float mx = m;
+#pragma unroll
+      for (int c = 0; c < 128; ++c) {
+        float v = s[c] * p.scale_log2;
+        if (need_mask) {
+          const int kpos = k0 + c;
+          if ((p.causal && kpos > q) || kpos >= p.S) v = -INFINITY;
+        }
+        s[c] = v;
+        mx = fmaxf(mx, v);
+      }
+      const float alpha = fast_exp2(m - mx);
+      m = mx;
+      float sum = 0.f;
+#pragma unroll
+      for (int c = 0; c < 128; ++c) {
+        const float e = fast_exp2(s[c] - m);
+        s[c] = e;
+        sum += e;
+      }
+      l = l * alpha + sum;
+      if (j > 0) {
+        // The previous P V has landed: P's buffer is free and O may be rescaled.
+        if (!__all_sync(0xffffffffu, wait_bar(pv_done, (j - 1) & 1, ctl, ERR_ATTN_FWD_WAIT))) { ok = false; break; }
+        tc_fence_after();
+        if (!__all_sync(0xffffffffu, alpha == 1.0f)) {
+#pragma unroll 1
+          for (int c = 0; c < DH / 32; ++c) {
+            uint32_t rr[32];
+            tmem_ld32(t_o + lane_off + c * 32, rr);
+            tc_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) rr[e] = __float_as_uint(__uint_as_float(rr[e]) * alpha);
+            tmem_st32(t_o + lane_off + c * 32, rr);
+          }
+          tc_wait_st();
+        }
+      }
+#pragma unroll
+      for (int g = 0; g < 16; ++g)
+        *reinterpret_cast<uint4*>(sp + sw128_offset(C::BM, r, g * 8)) = pack8_bf16(&s[g * 8]);
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(p_full);
+    }
+    if (ok && __all_sync(0xffffffffu, wait_bar(pv_done, (n_kv - 1) & 1, ctl, ERR_ATTN_FWD_WAIT))) {
+      tc_fence_after();
+      const float inv_l = 1.0f / l;
+      const bool valid = q < p.S;
+      uint16_t* orow = p.out + (long long)shard * p.T * p.Dt + ((long long)b * p.S + q) * p.Dt + hl * DH;
+#pragma unroll 1
+      for (int c = 0; c < DH / 32; ++c) {
+        uint32_t rr[32];
+        tmem_ld32(t_o + lane_off + c * 32, rr);
+        tc_wait_ld();
+        if (valid) {
+          float v[32];
+#pragma unroll
+          for (int e = 0; e < 32; ++e) v[e] = __uint_as_float(rr[e]) * inv_l;
+#pragma unroll
+          for (int g = 0; g < 4; ++g)
+            *reinterpret_cast<uint4*>(orow + c * 32 + g * 8) = pack8_bf16(&v[g * 8]);
+        }
+      }
+      if (valid) p.lse[((long long)b * p.H + h) * p.S + q] = (m + __log2f(l)) * kLn2;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// =====================================================================================
+// Backward
+// =====================================================================================
+__global__ void attn_bwd_prep_kernel(const uint16_t* __restrict__ o, const uint16_t* __restrict__ dout,
+                                     const float* __restrict__ lse, float* __restrict__ dvec,
+                                     float* __restrict__ lse2, int B, int S, int H, int Ht,
+                                     int dh, int Dt, long long T) {
+  const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= (long long)B * H * S) return;
+  const int s = (int)(idx % S);
+  const int h = (int)((idx / S) % H);
+  const int b = (int)(idx / ((long long)S * H));
+  const int shard = h / Ht, hl = h - shard * Ht;
+  const long long off = (long long)shard * T * Dt + ((long long)b * S + s) * Dt + hl * dh;
+  float acc = 0.f;
+  for (int d = 0; d < dh; d += 8) {
+    const uint4 a = *reinterpret_cast<const uint4*>(o + off + d);
+    const uint4 g = *reinterpret_cast<const uint4*>(dout + off + d);
+    const uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wg[4] = {g.x, g.y, g.z, g.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      acc += bf16_lo(wa[k]) * bf16_lo(wg[k]) + bf16_hi(wa[k]) * bf16_hi(wg[k]);
+  }
+  dvec[idx] = acc;
+  lse2[idx] = lse[idx] * kLog2e;
+}
+
+// ---------------------------------------------------------------- dK / dV
+template <int DH>
+struct DkdvCfg {
+  static constexpr int BK = 128, BQ = 64, CH = DH / 64;
+  static constexpr int K_BYTES = BK * DH * 2;              // K and V tiles, each
+  static constexpr int Q_BYTES = BQ * DH * 2;              // q and dO tiles, each (per stage)
+  static constexpr int OFF_K = 0, OFF_V = K_BYTES;
+  static constexpr int OFF_ST = 2 * K_BYTES;               // stage s: q at +s*2*Q, dO at +Q
+  static constexpr int OFF_PT = OFF_ST + 4 * Q_BYTES;      // P^T  [128 keys][64 queries]
+  static constexpr int OFF_DST = OFF_PT + BK * BQ * 2;     // dS^T [128 keys][64 queries]
+  static constexpr int OFF_BAR = OFF_DST + BK * BQ * 2;
+  static constexpr int RAW = OFF_BAR + 256 + 1024;
+  static constexpr int SMEM = RAW > 120 * 1024 ? RAW : 120 * 1024;
+};
+
+template <int DH>
+__global__ void __launch_bounds__(192, 1)
+attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_kv128,
+                     const __grid_constant__ CUtensorMap tm_q64,
+                     const __grid_constant__ CUtensorMap tm_do64, const AttnArgs p) {
+  using C = DkdvCfg<DH>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint64_t* kv_full = bars + 0;
+  uint64_t* qd_full = bars + 1;    // [2]
+  uint64_t* qd_empty = bars + 3;   // [2]
+  uint64_t* s_full = bars + 5;
+  uint64_t* s_free = bars + 6;
+  uint64_t* p_full = bars + 7;
+  uint64_t* mm2_done = bars + 8;
+  uint64_t* drain = bars + 9;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 10);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int kb = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int shard = h / p.Ht, hl = h - shard * p.Ht;
+  const int k0 = kb * C::BK;
+  const int nqb = (p.S + C::BQ - 1) / C::BQ;
+  const int i0 = p.causal ? k0 / C::BQ : 0;
+  const int nsteps = nqb - i0;
+  const int colq = hl * DH, colk = p.Dt + hl * DH, colv = 2 * p.Dt + hl * DH, cold = hl * DH;
+  const Ctl ctl{abort_flag, p.err};
+
+  if (threadIdx.x == 0) {
+    mbar_init(kv_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&qd_full[i], 1);
+      mbar_init(&qd_empty[i], 1);
+    }
+    mbar_init(s_full, 1);
+    mbar_init(s_free, 128);
+    mbar_init(p_full, 128);
+    mbar_init(mm2_done, 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t t_s = tmem, t_dp = tmem + 64, t_dv = tmem + 128, t_dk = tmem + 128 + DH;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      mbar_arrive_expect_tx(kv_full, 2 * C::K_BYTES);
+      for (int c = 0; c < C::CH; ++c) {
+        tma_load_4d(smem + C::OFF_K + c * C::BK * 128, &tm_kv128, kv_full, colk + 64 * c, k0, b, shard);
+        tma_load_4d(smem + C::OFF_V + c * C::BK * 128, &tm_kv128, kv_full, colv + 64 * c, k0, b, shard);
+      }
+      int k = 0;
+      for (; k < nsteps; ++k) {
+        const int st = k & 1;
+        const uint32_t u = k >> 1;
+        if (!wait_bar(&qd_empty[st], (u & 1) ^ 1, ctl, ERR_ATTN_DKDV_WAIT)) break;
+        uint8_t* sq = smem + C::OFF_ST + st * 2 * C::Q_BYTES;
+        uint8_t* sd = sq + C::Q_BYTES;
+        const int qs = (i0 + k) * C::BQ;
+        mbar_arrive_expect_tx(&qd_full[st], 2 * C::Q_BYTES);
+        for (int c = 0; c < C::CH; ++c) {
+          tma_load_4d(sq + c * C::BQ * 128, &tm_q64, &qd_full[st], colq + 64 * c, qs, b, shard);
+          tma_load_4d(sd + c * C::BQ * 128, &tm_do64, &qd_full[st], cold + 64 * c, qs, b, shard);
+        }
+      }
+      mbar_wait(kv_full, 0, 200000000ull);
+      for (int i = k - 1; i >= 0 && i >= k - 2; --i) mbar_wait(&qd_full[i & 1], (i >> 1) & 1, 200000000ull);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t id_s = idesc_bf16_f32(128, C::BQ, false, false);
+      constexpr uint32_t id_acc = idesc_bf16_f32(128, DH, false, true);
+      const uint32_t sk = smem_u32(smem + C::OFF_K), sv = smem_u32(smem + C::OFF_V);
+      const uint32_t spt = smem_u32(smem + C::OFF_PT), sdst = smem_u32(smem + C::OFF_DST);
+      bool ok = wait_bar(kv_full, 0, ctl, ERR_ATTN_DKDV_WAIT);
+      for (int k = 0; ok && k < nsteps; ++k) {
+        const int st = k & 1;
+        const uint32_t u = k >> 1;
+        if (!wait_bar(&qd_full[st], u & 1, ctl, ERR_ATTN_DKDV_WAIT)) break;
+        if (!wait_bar(s_free, (k & 1) ^ 1, ctl, ERR_ATTN_DKDV_WAIT)) break;
+        tc_fence_after();
+        const uint32_t sq = smem_u32(smem + C::OFF_ST + st * 2 * C::Q_BYTES);
+        const uint32_t sd = sq + C::Q_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < DH / 16; ++kk) {
+          tc_mma_f16(t_s, kmajor_desc(sk, C::BK, kk), kmajor_desc(sq, C::BQ, kk), id_s, kk > 0);
+          tc_mma_f16(t_dp, kmajor_desc(sv, C::BK, kk), kmajor_desc(sd, C::BQ, kk), id_s, kk > 0);
+        }
+        tc_commit(s_full);
+        if (!wait_bar(p_full, k & 1, ctl, ERR_ATTN_DKDV_WAIT)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < C::BQ / 16; ++kk) {
+          tc_mma_f16(t_dv, kmajor_desc(spt, C::BK, kk), mnmajor_desc(sd, C::BQ, kk), id_acc,
+                     (k | kk) != 0);
+          tc_mma_f16(t_dk, kmajor_desc(sdst, C::BK, kk), mnmajor_desc(sq, C::BQ, kk), id_acc,
+                     (k | kk) != 0);
+        }
+        tc_commit(mm2_done);
+        tc_commit(&qd_empty[st]);
+      }
+      tc_commit(drain);
+      mbar_wait(drain, 0, 200000000ull);
+    }
+  } else {
+    const int quad = warp & 3;
+    const int r = quad * 32 + lane;
+    const int kpos = k0 + r;
+    const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+    uint8_t* spt = smem + C::OFF_PT;
+    uint8_t* sdst = smem + C::OFF_DST;
+    const long long hrow = ((long long)b * p.H + h) * p.S;
+    bool ok = true;
+    for (int k = 0; k < nsteps; ++k) {
+      const int qs = (i0 + k) * C::BQ;
+      if (!__all_sync(0xffffffffu, wait_bar(s_full, k & 1, ctl, ERR_ATTN_DKDV_WAIT))) { ok = false; break; }
+      if (k > 0 && !__all_sync(0xffffffffu, wait_bar(mm2_done, (k - 1) & 1, ctl, ERR_ATTN_DKDV_WAIT))) { ok = false; break; }
+      tc_fence_after();
+#pragma unroll 1
+      for (int c = 0; c < C::BQ / 32; ++c) {
+        uint32_t rs[32], rd[32];
+        tmem_ld32(t_s + lane_off + c * 32, rs);
+        tmem_ld32(t_dp + lane_off + c * 32, rd);
+        tc_wait_ld();
+        float pv[32], dsv[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const int q = qs + c * 32 + e;
+          float pe = 0.f, de = 0.f;
+          if (q < p.S && !(p.causal && kpos > q)) {
+            pe = fast_exp2(__uint_as_float(rs[e]) * p.scale_log2 - __ldg(p.lse2 + hrow + q));
+            de = pe * (__uint_as_float(rd[e]) - __ldg(p.dvec + hrow + q));
+          }
+          pv[e] = pe;
+          dsv[e] = de;
+        }
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          const uint32_t off = sw128_offset(C::BK, r, c * 32 + g * 8);
+          *reinterpret_cast<uint4*>(spt + off) = pack8_bf16(&pv[g * 8]);
+          *reinterpret_cast<uint4*>(sdst + off) = pack8_bf16(&dsv[g * 8]);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(s_free);
+      fence_proxy_async_smem();
+      mbar_arrive(p_full);
+    }
+    if (ok && __all_sync(0xffffffffu, wait_bar(mm2_done, (nsteps - 1) & 1, ctl, ERR_ATTN_DKDV_WAIT))) {
+      tc_fence_after();
+      const bool valid = kpos < p.S;
+      const long long w3 = 3LL * p.Dt;
+      uint16_t* row = p.out + (long long)shard * p.T * w3 + ((long long)b * p.S + kpos) * w3;
+#pragma unroll 1
+      for (int c = 0; c < DH / 32; ++c) {
+        uint32_t rv[32], rk[32];
+        tmem_ld32(t_dv + lane_off + c * 32, rv);
+        tmem_ld32(t_dk + lane_off + c * 32, rk);
+        tc_wait_ld();
+        if (valid) {
+          float v[32], kx[32];
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            v[e] = __uint_as_float(rv[e]);
+            kx[e] = __uint_as_float(rk[e]) * p.inv_sqrt_dh;
+          }
+#pragma unroll
+          for (int g = 0; g < 4; ++g) {
+            *reinterpret_cast<uint4*>(row + colv + c * 32 + g * 8) = pack8_bf16(&v[g * 8]);
+            *reinterpret_cast<uint4*>(row + colk + c * 32 + g * 8) = pack8_bf16(&kx[g * 8]);
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------- dQ
+template <int DH>
+struct DqCfg {
+  static constexpr int BQ = 128, BK = 64, CH = DH / 64;
+  static constexpr int Q_BYTES = BQ * DH * 2;                // q and dO tiles, each
+  static constexpr int K_BYTES = BK * DH * 2;                // K and V tiles, each (per stage)
+  static constexpr int OFF_Q = 0, OFF_DO = Q_BYTES;
+  static constexpr int OFF_ST = 2 * Q_BYTES;                 // stage s: k at +s*2*K, v at +K
+  static constexpr int OFF_DS = OFF_ST + 4 * K_BYTES;        // dS [128 queries][64 keys]
+  static constexpr int OFF_BAR = OFF_DS + BQ * BK * 2;
+  static constexpr int RAW = OFF_BAR + 256 + 1024;
+  static constexpr int SMEM = RAW > 120 * 1024 ? RAW : 120 * 1024;
+};
+
+template <int DH>
+__global__ void __launch_bounds__(192, 1)
+attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q128,
+                   const __grid_constant__ CUtensorMap tm_do128,
+                   const __grid_constant__ CUtensorMap tm_kv64, const AttnArgs p) {
+  using C = DqCfg<DH>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint64_t* q_full = bars + 0;
+  uint64_t* kv_full = bars + 1;    // [2]
+  uint64_t* kv_empty = bars + 3;   // [2]
+  uint64_t* s_full = bars + 5;
+  uint64_t* s_free = bars + 6;
+  uint64_t* p_full = bars + 7;
+  uint64_t* mm2_done = bars + 8;
+  uint64_t* drain = bars + 9;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 10);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nqb = (p.S + C::BQ - 1) / C::BQ;
+  const int qb = p.causal ? nqb - 1 - (int)blockIdx.x : (int)blockIdx.x;
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int shard = h / p.Ht, hl = h - shard * p.Ht;
+  const int q0 = qb * C::BQ;
+  const int nkb = (p.S + C::BK - 1) / C::BK;
+  const int nsteps = p.causal ? min(nkb, (q0 + C::BQ) / C::BK) : nkb;
+  const int colq = hl * DH, colk = p.Dt + hl * DH, colv = 2 * p.Dt + hl * DH, cold = hl * DH;
+  const Ctl ctl{abort_flag, p.err};
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&kv_full[i], 1);
+      mbar_init(&kv_empty[i], 1);
+    }
+    mbar_init(s_full, 1);
+    mbar_init(s_free, 128);
+    mbar_init(p_full, 128);
+    mbar_init(mm2_done, 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 256);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t t_s = tmem, t_dp = tmem + 64, t_dq = tmem + 128;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      mbar_arrive_expect_tx(q_full, 2 * C::Q_BYTES);
+      for (int c = 0; c < C::CH; ++c) {
+        tma_load_4d(smem + C::OFF_Q + c * C::BQ * 128, &tm_q128, q_full, colq + 64 * c, q0, b, shard);
+        tma_load_4d(smem + C::OFF_DO + c * C::BQ * 128, &tm_do128, q_full, cold + 64 * c, q0, b, shard);
+      }
+      int k = 0;
+      for (; k < nsteps; ++k) {
+        const int st = k & 1;
+        const uint32_t u = k >> 1;
+        if (!wait_bar(&kv_empty[st], (u & 1) ^ 1, ctl, ERR_ATTN_DQ_WAIT)) break;
+        uint8_t* sk = smem + C::OFF_ST + st * 2 * C::K_BYTES;
+        uint8_t* sv = sk + C::K_BYTES;
+        mbar_arrive_expect_tx(&kv_full[st], 2 * C::K_BYTES);
+        for (int c = 0; c < C::CH; ++c) {
+          tma_load_4d(sk + c * C::BK * 128, &tm_kv64, &kv_full[st], colk + 64 * c, k * C::BK, b, shard);
+          tma_load_4d(sv + c * C::BK * 128, &tm_kv64, &kv_full[st], colv + 64 * c, k * C::BK, b, shard);
+        }
+      }
+      mbar_wait(q_full, 0, 200000000ull);
+      for (int i = k - 1; i >= 0 && i >= k - 2; --i) mbar_wait(&kv_full[i & 1], (i >> 1) & 1, 200000000ull);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t id_s = idesc_bf16_f32(128, C::BK, false, false);
+      constexpr uint32_t id_acc = idesc_bf16_f32(128, DH, false, true);
+      const uint32_t sq = smem_u32(smem + C::OFF_Q), sd = smem_u32(smem + C::OFF_DO);
+      const uint32_t sds = smem_u32(smem + C::OFF_DS);
+      bool ok = wait_bar(q_full, 0, ctl, ERR_ATTN_DQ_WAIT);
+      for (int k = 0; ok && k < nsteps; ++k) {
+        const int st = k & 1;
+        const uint32_t u = k >> 1;
+        if (!wait_bar(&kv_full[st], u & 1, ctl, ERR_ATTN_DQ_WAIT)) break;
+        if (!wait_bar(s_free, (k & 1) ^ 1, ctl, ERR_ATTN_DQ_WAIT)) break;
+        tc_fence_after();
+        const uint32_t sk = smem_u32(smem + C::OFF_ST + st * 2 * C::K_BYTES);
+        const uint32_t sv = sk + C::K_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < DH / 16; ++kk) {
+          tc_mma_f16(t_s, kmajor_desc(sq, C::BQ, kk), kmajor_desc(sk, C::BK, kk), id_s, kk > 0);
+          tc_mma_f16(t_dp, kmajor_desc(sd, C::BQ, kk), kmajor_desc(sv, C::BK, kk), id_s, kk > 0);
+        }
+        tc_commit(s_full);
+        if (!wait_bar(p_full, k & 1, ctl, ERR_ATTN_DQ_WAIT)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < C::BK / 16; ++kk)
+          tc_mma_f16(t_dq, kmajor_desc(sds, C::BQ, kk), mnmajor_desc(sk, C::BK, kk), id_acc,
+                     (k | kk) != 0);
+        tc_commit(mm2_done);
+        tc_commit(&kv_empty[st]);
+      }
+      tc_commit(drain);
+      mbar_wait(drain, 0, 200000000ull);
+    }
+  } else {
+    const int quad = warp & 3;
+    const int r = quad * 32 + lane;
+    const int q = q0 + r;
+    const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+    uint8_t* sds = smem + C::OFF_DS;
+    const long long hrow = ((long long)b * p.H + h) * p.S;
+    const bool qvalid = q < p.S;
+    const float l2 = qvalid ? p.lse2[hrow + q] : 0.f;
+    const float dv = qvalid ? p.dvec[hrow + q] : 0.f;
+    bool ok = true;
+    for (int k = 0; k < nsteps; ++k) {
+      const int ks = k * C::BK;
+      if (!__all_sync(0xffffffffu, wait_bar(s_full, k & 1, ctl, ERR_ATTN_DQ_WAIT))) { ok = false; break; }
+      if (k > 0 && !__all_sync(0xffffffffu, wait_bar(mm2_done, (k - 1) & 1, ctl, ERR_ATTN_DQ_WAIT))) { ok = false; break; }
+      tc_fence_after();
+#pragma unroll 1
+      for (int c = 0; c < C::BK / 32; ++c) {
+        uint32_t rs[32], rd[32];
+        tmem_ld32(t_s + lane_off + c * 32, rs);
+        tmem_ld32(t_dp + lane_off + c * 32, rd);
+        tc_wait_ld();
+        float dsv[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const int kpos = ks + c * 32 + e;
+          float de = 0.f;
+          if (qvalid && kpos < p.S && !(p.causal && kpos > q)) {
+            const float pe = fast_exp2(__uint_as_float(rs[e]) * p.scale_log2 - l2);
+            de = pe * (__uint_as_float(rd[e]) - dv);
+          }
+          dsv[e] = de;
+        }
+#pragma unroll
+        for (int g = 0; g < 4; ++g)
+          *reinterpret_cast<uint4*>(sds + sw128_offset(C::BQ, r, c * 32 + g * 8)) = pack8_bf16(&dsv[g * 8]);
+      }
+      tc_fence_before();
+      mbar_arrive(s_free);
+      fence_proxy_async_smem();
+      mbar_arrive(p_full);
+    }
+    if (ok && nsteps > 0 && __all_sync(0xffffffffu, wait_bar(mm2_done, (nsteps - 1) & 1, ctl, ERR_ATTN_DQ_WAIT))) {
+      tc_fence_after();
+      const long long w3 = 3LL * p.Dt;
+      uint16_t* row = p.out + (long long)shard * p.T * w3 + ((long long)b * p.S + q) * w3 + colq;
+#pragma unroll 1
+      for (int c = 0; c < DH / 32; ++c) {
+        uint32_t rq[32];
+        tmem_ld32(t_dq + lane_off + c * 32, rq);
+        tc_wait_ld();
+        if (qvalid) {
+          float v[32];
+#pragma unroll
+          for (int e = 0; e < 32; ++e) v[e] = __uint_as_float(rq[e]) * p.inv_sqrt_dh;
+#pragma unroll
+          for (int g = 0; g < 4; ++g)
+            *reinterpret_cast<uint4*>(row + c * 32 + g * 8) = pack8_bf16(&v[g * 8]);
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 256);
+  }
+}
+
+// =====================================================================================
+// Host side
+// =====================================================================================
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+// 4-D map over a shard-packed activation [t][B*S][width]: dims (width, S, B, t),
+// box (64, rows, 1, 1), 128-byte swizzle, zero fill past S.
+bool encode_act(CUtensorMap* m, const void* base, long long width, int S, int B, int t,
+                long long T, int rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[4] = {(cuuint64_t)width, (cuuint64_t)S, (cuuint64_t)B, (cuuint64_t)t};
+  const cuuint64_t strides[3] = {(cuuint64_t)width * 2, (cuuint64_t)S * width * 2,
+                                 (cuuint64_t)T * width * 2};
+  const cuuint32_t box[4] = {64, (cuuint32_t)rows, 1, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Opt the kernel into `bytes` of dynamic shared memory once per device.
+bool set_smem(const void* kern, int bytes) {
+  static std::mutex mu;
+  static const void* done[64][8] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  std::lock_guard<std::mutex> lk(mu);
+  if (dev >= 0 && dev < 64)
+    for (int i = 0; i < 8; ++i)
+      if (done[dev][i] == kern) return true;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+    return false;
+  if (dev >= 0 && dev < 64)
+    for (int i = 0; i < 8; ++i)
+      if (!done[dev][i]) { done[dev][i] = kern; break; }
+  return true;
+}
+
+AttnArgs make_args(int B, int S, int H, int dh, int t, int causal) {
+  AttnArgs a{};
+  a.B = B; a.S = S; a.H = H; a.Ht = H / t; a.Dt = (H / t) * dh; a.t = t;
+  a.causal = causal;
+  a.T = (long long)B * S;
+  a.scale_log2 = kLog2e / sqrtf((float)dh);
+  a.inv_sqrt_dh = 1.0f / sqrtf((float)dh);
+  a.err = error_word();
+  return a;
+}
+
+template <int DH>
+tp_status fwd_launch(const uint16_t* qkv, uint16_t* o, float* lse, const AttnArgs& a,
+                     cudaStream_t st) {
+  CUtensorMap tm;
+  if (!encode_act(&tm, qkv, 3LL * a.Dt, a.S, a.B, a.t, a.T, 128)) return TP_ERR_CUDA;
+  AttnArgs p = a;
+  p.out = o;
+  p.lse = lse;
+  auto kern = attn_fwd_kernel<DH>;
+  if (!set_smem((const void*)kern, FwdCfg<DH>::SMEM)) return TP_ERR_CUDA;
+  const dim3 grid((a.S + 127) / 128, a.H, a.B);
+  kern<<<grid, 192, FwdCfg<DH>::SMEM, st>>>(tm, p);
+  return cuda_status(cudaGetLastError());
+}
+
+template <int DH>
+tp_status bwd_launch(const uint16_t* qkv, const uint16_t* o, const float* lse, const uint16_t* dout,
+                     uint16_t* dqkv, const AttnArgs& a, void* scratch, cudaStream_t st) {
+  float* dvec = static_cast<float*>(scratch);
+  float* lse2 = dvec + align_up((size_t)a.B * a.H * a.S, 64);
+  const long long n = (long long)a.B * a.H * a.S;
+  attn_bwd_prep_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(o, dout, lse, dvec, lse2, a.B,
+                                                                     a.S, a.H, a.Ht, DH, a.Dt, a.T);
+  if (cudaGetLastError() != cudaSuccess) return TP_ERR_CUDA;
+  AttnArgs p = a;
+  p.out = dqkv;
+  p.lse2 = lse2;
+  p.dvec = dvec;
+  CUtensorMap kv128, q64, do64, q128, do128, kv64;
+  if (!encode_act(&kv128, qkv, 3LL * a.Dt, a.S, a.B, a.t, a.T, 128) ||
+      !encode_act(&q64, qkv, 3LL * a.Dt, a.S, a.B, a.t, a.T, 64) ||
+      !encode_act(&do64, dout, a.Dt, a.S, a.B, a.t, a.T, 64) ||
+      !encode_act(&q128, qkv, 3LL * a.Dt, a.S, a.B, a.t, a.T, 128) ||
+      !encode_act(&do128, dout, a.Dt, a.S, a.B, a.t, a.T, 128) ||
+      !encode_act(&kv64, qkv, 3LL * a.Dt, a.S, a.B, a.t, a.T, 64))
+    return TP_ERR_CUDA;
+  auto k1 = attn_bwd_dkdv_kernel<DH>;
+  auto k2 = attn_bwd_dq_kernel<DH>;
+  if (!set_smem((const void*)k1, DkdvCfg<DH>::SMEM) || !set_smem((const void*)k2, DqCfg<DH>::SMEM))
+    return TP_ERR_CUDA;
+  k1<<<dim3((a.S + 127) / 128, a.H, a.B), 192, DkdvCfg<DH>::SMEM, st>>>(kv128, q64, do64, p);
+  if (cudaGetLastError() != cudaSuccess) return TP_ERR_CUDA;
+  k2<<<dim3((a.S + 127) / 128, a.H, a.B), 192, DqCfg<DH>::SMEM, st>>>(q128, do128, kv64, p);
+  return cuda_status(cudaGetLastError());
+}
+
+}  // namespace
+
+tp_status launch_attn_fwd(const uint16_t* qkv, uint16_t* o, float* lse, int B, int S, int H,
+                          int dh, int t, int causal, cudaStream_t stream) {
+  if ((long long)B * S == 0) return TP_OK;
+  const AttnArgs a = make_args(B, S, H, dh, t, causal);
+  if (dh == 64) return fwd_launch<64>(qkv, o, lse, a, stream);
+  if (dh == 128) return fwd_launch<128>(qkv, o, lse, a, stream);
+  return TP_ERR_UNSUPPORTED;
+}
+
+size_t attn_bwd_scratch_bytes(int B, int S, int H, int dh) {
+  (void)dh;
+  return 2 * align_up((size_t)B * H * S, 64) * sizeof(float);
+}
+
+tp_status launch_attn_bwd(const uint16_t* qkv, const uint16_t* o, const float* lse,
+                          const uint16_t* dout, uint16_t* dqkv, int B, int S, int H, int dh, int t,
+                          int causal, void* scratch, cudaStream_t stream) {
+  if ((long long)B * S == 0) return TP_OK;
+  const AttnArgs a = make_args(B, S, H, dh, t, causal);
+  if (dh == 64) return bwd_launch<64>(qkv, o, lse, dout, dqkv, a, scratch, stream);
+  if (dh == 128) return bwd_launch<128>(qkv, o, lse, dout, dqkv, a, scratch, stream);
+  return TP_ERR_UNSUPPORTED;
+}
+
+}  // namespace tp

@@ -1,0 +1,100 @@
+// Host side of the tcgen05 GEMM: tensor-map encoding and launch.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+#include "gemm_sm100.cuh"
+#include "internal.h"
+
+namespace tp {
+
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 3-D bf16 tensor map with 128-byte swizzle; out-of-range elements read as 0.
+bool encode_operand(CUtensorMap* map, const OperandDesc& d, uint32_t box_outer) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {(cuuint64_t)d.inner, (cuuint64_t)d.outer, (cuuint64_t)d.shards};
+  const long long shard_stride = d.shards > 1 ? d.shard_stride : d.ld * d.outer;
+  const cuuint64_t strides[2] = {(cuuint64_t)d.ld * 2, (cuuint64_t)shard_stride * 2};
+  const cuuint32_t box[3] = {64, box_outer, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(d.ptr), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <bool A_MN, bool B_MN>
+tp_status launch_inst(const CUtensorMap& ta, const CUtensorMap& tb, const GemmArgs& args,
+                      int grid, cudaStream_t stream) {
+  static bool configured[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  auto kern = gemm_bf16_sm100<A_MN, B_MN>;
+  if (dev < 64 && !configured[dev]) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             GEMM_SMEM_BYTES) != cudaSuccess)
+      return TP_ERR_CUDA;
+    configured[dev] = true;
+  }
+  kern<<<grid, GEMM_THREADS, GEMM_SMEM_BYTES, stream>>>(ta, tb, args);
+  return cuda_status(cudaGetLastError());
+}
+
+}  // namespace
+
+tp_status launch_gemm(const GemmProblem& g, cudaStream_t stream) {
+  if (g.Mt <= 0 || g.Nt <= 0 || g.Kt <= 0) return TP_OK;   // empty product: nothing to do
+  CUtensorMap ta, tb;
+  if (!encode_operand(&ta, g.a, g.a.mn_major ? 64 : GEMM_BM)) return TP_ERR_CUDA;
+  if (!encode_operand(&tb, g.b, g.b.mn_major ? 64 : GEMM_BN)) return TP_ERR_CUDA;
+
+  GemmArgs a{};
+  a.m_shards = g.m_shards;
+  a.n_shards = g.n_shards;
+  a.Mt = g.Mt;
+  a.Nt = g.Nt;
+  a.mb_per_shard = (g.Mt + GEMM_BM - 1) / GEMM_BM;
+  a.nb_per_shard = (g.Nt + GEMM_BN - 1) / GEMM_BN;
+  a.k_shards = g.k_shards;
+  a.kb_per_shard = (g.Kt + GEMM_BK - 1) / GEMM_BK;
+  a.a_src = g.a.src;
+  a.b_src = g.b.src;
+  const long long tiles = (long long)a.m_shards * a.mb_per_shard * a.n_shards * a.nb_per_shard;
+  a.num_tiles = (int)tiles;
+  a.group_m = 16;
+  a.epi = g.epi;
+  a.c = static_cast<__nv_bfloat16*>(g.c);
+  a.c2 = static_cast<__nv_bfloat16*>(g.c2);
+  a.aux = static_cast<const __nv_bfloat16*>(g.aux);
+  a.bias = static_cast<const __nv_bfloat16*>(g.bias);
+  a.c_ms = g.c_ms;
+  a.c_ns = g.c_ns;
+  a.ldc = g.ldc;
+  a.err = error_word();
+  const int grid = (int)(tiles < sm_count() ? tiles : sm_count());
+
+  if (!g.a.mn_major && g.b.mn_major) return launch_inst<false, true>(ta, tb, a, grid, stream);
+  if (!g.a.mn_major && !g.b.mn_major) return launch_inst<false, false>(ta, tb, a, grid, stream);
+  if (g.a.mn_major && g.b.mn_major) return launch_inst<true, true>(ta, tb, a, grid, stream);
+  return launch_inst<true, false>(ta, tb, a, grid, stream);
+}
+
+}  // namespace tp

@@ -1,0 +1,369 @@
+// Persistent, warp-specialised tcgen05 GEMM for the sharded sublayer.
+//
+// C[m, n] = epilogue( sum_k A[m, k] * B[k, n] ), bf16 operands, fp32
+// accumulation in tensor memory, bf16 output.
+//
+// Tensor-parallel structure ("How transformer layers actually decompose",
+// "The attention heads split"): the t shards of a column-parallel product
+// appear as N shards (output [t][M][N/t]); the t partial products of a
+// row-parallel product appear as K shards, walked one after the other into
+// the SAME tensor-memory accumulator, so the cross-shard sum that the pages
+// perform with an all-reduce happens in fp32 inside the MMA, in shard order
+// 0..t-1, with a single bf16 rounding in the epilogue.  Weight-gradient
+// products shard M or N the same way.
+//
+// Roles (192 threads, one CTA per SM):
+//   warp 0      TMA producer: streams A/B k-blocks into a 4-stage ring;
+//   warp 1      TMEM owner and MMA issuer (one thread): 4 x (128x256x16) MMAs
+//               per k-block into one of two 256-column accumulators;
+//   warps 2..5  epilogue: tcgen05.ld of their 32-lane quarter, bias / GeLU /
+//               GeLU-backward / residual, bf16 stores.  The second
+//               accumulator lets the epilogue of tile i overlap the MMAs of
+//               tile i+1.
+// Every wait is bounded; a timeout records an error code and the kernel
+// drains its own copies and MMAs, frees TMEM and returns.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cstdint>
+
+#include "sm100_ptx.cuh"
+
+namespace tp {
+
+constexpr int GEMM_BM = 128;
+constexpr int GEMM_BN = 256;
+constexpr int GEMM_BK = 64;        // one 128-byte swizzle row of bf16
+constexpr int GEMM_STAGES = 4;
+constexpr int GEMM_THREADS = 192;
+constexpr int GEMM_A_BYTES = GEMM_BM * GEMM_BK * 2;   // 16 KiB
+constexpr int GEMM_B_BYTES = GEMM_BN * GEMM_BK * 2;   // 32 KiB
+constexpr int GEMM_STAGE_BYTES = GEMM_A_BYTES + GEMM_B_BYTES;
+constexpr int GEMM_SMEM_BYTES = GEMM_STAGES * GEMM_STAGE_BYTES + 1024 /*align*/ + 256 /*bars*/;
+constexpr uint32_t GEMM_TMEM_COLS = 512;               // two 128x256 fp32 accumulators
+
+enum EpiKind : int {
+  EPI_LINEAR = 0,     // C = acc (+ bias[n]) (+ aux[m, n])
+  EPI_BIAS_GELU = 1,  // C = acc (+ bias[n]);  C2 = GeLU(C)
+  EPI_DGELU = 2,      // C = acc * GeLU'(aux[m, n])
+};
+
+enum ShardSrc : int { SHARD_NONE = 0, SHARD_K = 1, SHARD_MN = 2 };
+
+// Error codes written to the library's device error word.
+enum : unsigned int {
+  ERR_GEMM_PRODUCER_WAIT = 0x101,
+  ERR_GEMM_MMA_WAIT = 0x102,
+  ERR_GEMM_EPI_WAIT = 0x103,
+  ERR_GEMM_DRAIN_WAIT = 0x104,
+};
+
+struct GemmArgs {
+  int m_shards, n_shards;          // output shards along M and along N
+  int Mt, Nt;                      // rows / columns of one output shard
+  int mb_per_shard, nb_per_shard;  // ceil(Mt / BM), ceil(Nt / BN)
+  int k_shards, kb_per_shard;      // K walk: k_shards x ceil(Kt / BK) blocks
+  int a_src, b_src;                // which index selects each operand's shard
+  int num_tiles, group_m;
+  int epi;
+  // C element (ms, m, ns, n) lives at c + ms*c_ms + ns*c_ns + m*ldc + n; aux
+  // (residual or saved pre-activation) and C2 share that layout; bias is
+  // indexed by ns*Nt + n.
+  __nv_bfloat16* c;
+  __nv_bfloat16* c2;
+  const __nv_bfloat16* aux;
+  const __nv_bfloat16* bias;
+  long long c_ms, c_ns, ldc;
+  unsigned int* err;
+};
+
+__device__ __forceinline__ float gelu_tanh_f(float a) {
+  const float k0 = 0.7978845608028654f, k1 = 0.044715f;
+  return 0.5f * a * (1.0f + tanhf(k0 * (a + k1 * a * a * a)));
+}
+
+__device__ __forceinline__ float gelu_tanh_grad_f(float a) {
+  const float k0 = 0.7978845608028654f, k1 = 0.044715f;
+  const float th = tanhf(k0 * (a + k1 * a * a * a));
+  return 0.5f * (1.0f + th) + 0.5f * a * (1.0f - th * th) * k0 * (1.0f + 3.0f * k1 * a * a);
+}
+
+struct TileCoord {
+  int ms, m0, ns, n0;
+};
+
+__device__ __forceinline__ TileCoord gemm_tile(const GemmArgs& p, int tile) {
+  const int mbt = p.m_shards * p.mb_per_shard;
+  const int nbt = p.n_shards * p.nb_per_shard;
+  const int per_group = p.group_m * nbt;
+  const int g = tile / per_group;
+  const int first = g * p.group_m;
+  const int gsize = min(mbt - first, p.group_m);
+  const int r = tile - g * per_group;
+  const int mb = first + r % gsize;
+  const int nb = r / gsize;
+  TileCoord tc;
+  tc.ms = mb / p.mb_per_shard;
+  tc.m0 = (mb - tc.ms * p.mb_per_shard) * GEMM_BM;
+  tc.ns = nb / p.nb_per_shard;
+  tc.n0 = (nb - tc.ns * p.nb_per_shard) * GEMM_BN;
+  return tc;
+}
+
+__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity,
+                                              volatile int* abort_flag) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (globaltimer_ns() - t0 > 2000000000ull) return false;
+  }
+}
+
+__device__ __forceinline__ void record_error(unsigned int* err, volatile int* abort_flag,
+                                             unsigned int code) {
+  *abort_flag = 1;
+  if (err) atomicCAS(err, 0u, code);
+}
+
+template <bool A_MN, bool B_MN>
+__global__ void __launch_bounds__(GEMM_THREADS, 1)
+gemm_bf16_sm100(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                const GemmArgs p) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + GEMM_STAGES * GEMM_STAGE_BYTES);
+  uint64_t* full = bars;                        // [STAGES]
+  uint64_t* empty = bars + GEMM_STAGES;         // [STAGES]
+  uint64_t* tfull = bars + 2 * GEMM_STAGES;     // [2]
+  uint64_t* tempty = tfull + 2;                 // [2]
+  uint64_t* drain = tempty + 2;                 // [1]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < GEMM_STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&tfull[i], 1);
+      mbar_init(&tempty[i], 128);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, GEMM_TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int num_kb = p.k_shards * p.kb_per_shard;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int it = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x) {
+        const TileCoord tc = gemm_tile(p, tile);
+        for (int kb = 0; kb < num_kb; ++kb, ++it) {
+          const int s = it % GEMM_STAGES;
+          const uint32_t round = it / GEMM_STAGES;
+          if (!wait_or_abort(&empty[s], (round & 1) ^ 1, abort_flag)) {
+            record_error(p.err, abort_flag, ERR_GEMM_PRODUCER_WAIT);
+            ok = false;
+            break;
+          }
+          const int ks = kb / p.kb_per_shard;
+          const int k0 = (kb - ks * p.kb_per_shard) * GEMM_BK;
+          const int a_s = p.a_src == SHARD_K ? ks : (p.a_src == SHARD_MN ? tc.ms : 0);
+          const int b_s = p.b_src == SHARD_K ? ks : (p.b_src == SHARD_MN ? tc.ns : 0);
+          uint8_t* sa = smem + s * GEMM_STAGE_BYTES;
+          uint8_t* sb = sa + GEMM_A_BYTES;
+          mbar_arrive_expect_tx(&full[s], GEMM_STAGE_BYTES);
+          if (A_MN) {
+#pragma unroll
+            for (int j = 0; j < GEMM_BM / 64; ++j)
+              tma_load_3d(sa + j * 8192, &tmA, &full[s], tc.m0 + 64 * j, k0, a_s);
+          } else {
+            tma_load_3d(sa, &tmA, &full[s], k0, tc.m0, a_s);
+          }
+          if (B_MN) {
+#pragma unroll
+            for (int j = 0; j < GEMM_BN / 64; ++j)
+              tma_load_3d(sb + j * 8192, &tmB, &full[s], tc.n0 + 64 * j, k0, b_s);
+          } else {
+            tma_load_3d(sb, &tmB, &full[s], k0, tc.n0, b_s);
+          }
+        }
+      }
+      // Let every copy this thread issued land before the CTA can exit.
+      const int issued = it;
+      for (int j = 0; j < GEMM_STAGES && j < issued; ++j) {
+        const int i = issued - 1 - j;
+        mbar_wait(&full[i % GEMM_STAGES], (i / GEMM_STAGES) & 1, 200000000ull);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(GEMM_BM, GEMM_BN, A_MN, B_MN);
+      int it = 0, tcount = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x, ++tcount) {
+        const int acc = tcount & 1;
+        const uint32_t use = tcount >> 1;
+        if (!wait_or_abort(&tempty[acc], (use & 1) ^ 1, abort_flag)) {
+          record_error(p.err, abort_flag, ERR_GEMM_MMA_WAIT);
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * GEMM_BN;
+        for (int kb = 0; kb < num_kb; ++kb, ++it) {
+          const int s = it % GEMM_STAGES;
+          const uint32_t round = it / GEMM_STAGES;
+          if (!wait_or_abort(&full[s], round & 1, abort_flag)) {
+            record_error(p.err, abort_flag, ERR_GEMM_MMA_WAIT);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + s * GEMM_STAGE_BYTES);
+          const uint32_t sb = sa + GEMM_A_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < GEMM_BK / 16; ++kk) {
+            const uint64_t ad = A_MN ? smem_desc_sw128(sa + kk * 2048, 8192, 1024)
+                                     : smem_desc_sw128(sa + kk * 32, 16, 1024);
+            const uint64_t bd = B_MN ? smem_desc_sw128(sb + kk * 2048, 8192, 1024)
+                                     : smem_desc_sw128(sb + kk * 32, 16, 1024);
+            tc_mma_f16(d_tmem, ad, bd, idesc, (kb | kk) != 0);
+          }
+          tc_commit(&empty[s]);   // frees the stage once these MMAs have read it
+        }
+        if (!ok) break;
+        tc_commit(&tfull[acc]);   // accumulator ready for the epilogue
+      }
+      // Drain: every MMA issued above has completed before TMEM is freed.
+      tc_commit(drain);
+      if (!mbar_wait(drain, 0, 200000000ull)) record_error(p.err, abort_flag, ERR_GEMM_DRAIN_WAIT);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int quad = warp & 3;                 // TMEM lane quarter this warp may access
+    const int row = quad * 32 + lane;          // row within the tile
+    int tcount = 0;
+    for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++tcount) {
+      const TileCoord tc = gemm_tile(p, tile);
+      const int acc = tcount & 1;
+      const uint32_t use = tcount >> 1;
+      // Warp-uniform outcome: the tcgen05.ld below is a warp-collective instruction.
+      if (!__all_sync(0xffffffffu, wait_or_abort(&tfull[acc], use & 1, abort_flag))) {
+        record_error(p.err, abort_flag, ERR_GEMM_EPI_WAIT);
+        break;
+      }
+      tc_fence_after();
+      const int m = tc.m0 + row;
+      const bool row_ok = m < p.Mt;
+      const long long base = tc.ms * p.c_ms + tc.ns * p.c_ns + (long long)m * p.ldc;
+      const uint32_t taddr = tmem_base + ((uint32_t)(quad * 32) << 16) + acc * GEMM_BN;
+#pragma unroll 1
+      for (int c = 0; c < GEMM_BN / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld32(taddr + c * 32, r);
+        tc_wait_ld();
+        const int n = tc.n0 + c * 32;
+        if (!row_ok || n >= p.Nt) continue;
+        float v[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+        const int nvalid = min(32, p.Nt - n);   // a multiple of 8
+        if (p.bias != nullptr && p.epi != EPI_DGELU) {
+          const __nv_bfloat16* bp = p.bias + (long long)tc.ns * p.Nt + n;
+#pragma unroll
+          for (int g = 0; g < 4; ++g) {
+            if (g * 8 < nvalid) {
+              const uint4 bv = *reinterpret_cast<const uint4*>(bp + g * 8);
+              const uint32_t w[4] = {bv.x, bv.y, bv.z, bv.w};
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                v[g * 8 + 2 * q] += bf16_lo(w[q]);
+                v[g * 8 + 2 * q + 1] += bf16_hi(w[q]);
+              }
+            }
+          }
+        }
+        if (p.aux != nullptr) {
+          const __nv_bfloat16* xp = p.aux + base + n;
+#pragma unroll
+          for (int g = 0; g < 4; ++g) {
+            if (g * 8 < nvalid) {
+              const uint4 av = *reinterpret_cast<const uint4*>(xp + g * 8);
+              const uint32_t w[4] = {av.x, av.y, av.z, av.w};
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                const float lo = bf16_lo(w[q]), hi = bf16_hi(w[q]);
+                if (p.epi == EPI_DGELU) {
+                  v[g * 8 + 2 * q] *= gelu_tanh_grad_f(lo);
+                  v[g * 8 + 2 * q + 1] *= gelu_tanh_grad_f(hi);
+                } else {
+                  v[g * 8 + 2 * q] += lo;
+                  v[g * 8 + 2 * q + 1] += hi;
+                }
+              }
+            }
+          }
+        }
+        __nv_bfloat16* cp = p.c + base + n;
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          if (g * 8 < nvalid) {
+            uint4 o;
+            o.x = pack_bf16x2(v[g * 8 + 0], v[g * 8 + 1]);
+            o.y = pack_bf16x2(v[g * 8 + 2], v[g * 8 + 3]);
+            o.z = pack_bf16x2(v[g * 8 + 4], v[g * 8 + 5]);
+            o.w = pack_bf16x2(v[g * 8 + 6], v[g * 8 + 7]);
+            *reinterpret_cast<uint4*>(cp + g * 8) = o;
+          }
+        }
+        if (p.epi == EPI_BIAS_GELU) {
+          __nv_bfloat16* hp = p.c2 + base + n;
+#pragma unroll
+          for (int g = 0; g < 4; ++g) {
+            if (g * 8 < nvalid) {
+              uint4 o;
+              o.x = pack_bf16x2(gelu_tanh_f(v[g * 8 + 0]), gelu_tanh_f(v[g * 8 + 1]));
+              o.y = pack_bf16x2(gelu_tanh_f(v[g * 8 + 2]), gelu_tanh_f(v[g * 8 + 3]));
+              o.z = pack_bf16x2(gelu_tanh_f(v[g * 8 + 4]), gelu_tanh_f(v[g * 8 + 5]));
+              o.w = pack_bf16x2(gelu_tanh_f(v[g * 8 + 6]), gelu_tanh_f(v[g * 8 + 7]));
+              *reinterpret_cast<uint4*>(hp + g * 8) = o;
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&tempty[acc]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, GEMM_TMEM_COLS);
+  }
+}
+
+}  // namespace tp

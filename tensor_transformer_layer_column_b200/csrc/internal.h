@@ -1,0 +1,78 @@
+// Declarations shared by the translation units of libtplayer.so (not part of the ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cstddef>
+#include <cstdint>
+
+#include "tp_layer.h"
+
+namespace tp {
+
+// One GEMM operand as a 3-D tensor (inner, outer, shards), row-major, bf16.
+//   K-major operand : inner = K extent, outer = M (or N) extent;
+//   MN-major operand: inner = M (or N) extent, outer = K extent.
+// src selects what indexes the shard dimension: nothing, the K walk, or the
+// operand's own M/N shard.
+struct OperandDesc {
+  const void* ptr;
+  bool mn_major;
+  int src;                   // ShardSrc
+  long long inner, outer, shards;
+  long long ld;              // elements between consecutive outer indices
+  long long shard_stride;    // elements between consecutive shards
+};
+
+struct GemmProblem {
+  int m_shards, n_shards, Mt, Nt;
+  int k_shards, Kt;
+  OperandDesc a, b;
+  int epi;                   // EpiKind
+  void* c;
+  void* c2;
+  const void* aux;
+  const void* bias;
+  long long c_ms, c_ns, ldc;
+};
+
+tp_status launch_gemm(const GemmProblem& g, cudaStream_t stream);
+
+// Device error word of the current device (bounded-wait timeouts).
+unsigned int* error_word();
+int sm_count();
+
+// Column sums of S stacked [rows][cols] bf16 matrices into bf16 out[S][cols]
+// (fp32 accumulation, deterministic two-pass over `partial`, an fp32 scratch
+// of colsum_partial_floats(S, rows, cols) floats).
+size_t colsum_partial_floats(long long S, long long rows, long long cols);
+tp_status launch_colsum_stacked(const uint16_t* x, long long S, long long rows, long long cols,
+                                uint16_t* out, float* partial, cudaStream_t stream);
+
+tp_status launch_layernorm_fwd(const uint16_t* x, const uint16_t* g, const uint16_t* b,
+                               long long rows, int D, float eps, uint16_t* y, float* mean,
+                               float* rstd, cudaStream_t stream);
+size_t layernorm_bwd_partial_floats(long long rows, int D);
+tp_status launch_layernorm_bwd(const uint16_t* dy, const uint16_t* x, const uint16_t* g,
+                               const float* mean, const float* rstd, const uint16_t* dres,
+                               long long rows, int D, uint16_t* dx, uint16_t* dg, uint16_t* db,
+                               float* partial, cudaStream_t stream);
+
+// Per-head causal attention over the shard-packed qkv [t][T][3Dt].
+tp_status launch_attn_fwd(const uint16_t* qkv, uint16_t* o, float* lse, int B, int S, int H,
+                          int dh, int t, int causal, cudaStream_t stream);
+size_t attn_bwd_scratch_bytes(int B, int S, int H, int dh);
+tp_status launch_attn_bwd(const uint16_t* qkv, const uint16_t* o, const float* lse,
+                          const uint16_t* dout, uint16_t* dqkv, int B, int S, int H, int dh, int t,
+                          int causal, void* scratch, cudaStream_t stream);
+
+tp_status launch_shard_cols(const uint16_t* src, int rows, int cols, int t, uint16_t* dst,
+                            bool inverse, cudaStream_t stream);
+tp_status launch_shard_qkv(const uint16_t* src, int rows, int hidden, int t, uint16_t* dst,
+                           bool inverse, cudaStream_t stream);
+tp_status launch_copy(const uint16_t* src, size_t n, uint16_t* dst, cudaStream_t stream);
+
+inline tp_status cuda_status(cudaError_t e) { return e == cudaSuccess ? TP_OK : TP_ERR_CUDA; }
+
+inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+}  // namespace tp

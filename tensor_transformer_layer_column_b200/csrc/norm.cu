@@ -1,0 +1,317 @@
+// HBM-bound row and column kernels: LayerNorm forward / backward (pre-LN,
+// "The layernorm placement the paper flags as critical") and deterministic
+// column sums for bias gradients.  128-bit loads and stores throughout; fp32
+// statistics; every reduction order is fixed, so results repeat bit for bit.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "internal.h"
+
+namespace tp {
+
+namespace {
+
+__device__ __forceinline__ void unpack8(const uint4& u, float (&f)[8]) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    f[2 * q] = __uint_as_float(w[q] << 16);
+    f[2 * q + 1] = __uint_as_float(w[q] & 0xFFFF0000u);
+  }
+}
+
+__device__ __forceinline__ uint4 pack8(const float (&f)[8]) {
+  uint4 u;
+  uint32_t w[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(f[2 * q], f[2 * q + 1]);
+    w[q] = *reinterpret_cast<uint32_t*>(&v);
+  }
+  u.x = w[0]; u.y = w[1]; u.z = w[2]; u.w = w[3];
+  return u;
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// One warp per row; lane owns 8-element chunks lane, lane+32, ...
+template <int CH>
+__global__ void __launch_bounds__(256)
+ln_fwd_kernel(const uint16_t* __restrict__ x, const uint16_t* __restrict__ g,
+              const uint16_t* __restrict__ b, long long rows, int D, float eps,
+              uint16_t* __restrict__ y, float* __restrict__ mean, float* __restrict__ rstd) {
+  const int lane = threadIdx.x & 31;
+  const long long row = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (row >= rows) return;
+  const int nch = D >> 3;
+  const uint16_t* xr = x + row * D;
+  float v[CH][8];
+  float s = 0.f;
+#pragma unroll
+  for (int j = 0; j < CH; ++j) {
+    const int c = lane + 32 * j;
+    if (c < nch) {
+      unpack8(*reinterpret_cast<const uint4*>(xr + c * 8), v[j]);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) s += v[j][e];
+    }
+  }
+  const float mu = warp_sum(s) / D;
+  float ss = 0.f;
+#pragma unroll
+  for (int j = 0; j < CH; ++j) {
+    if (lane + 32 * j < nch) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const float d = v[j][e] - mu;
+        ss += d * d;
+      }
+    }
+  }
+  const float rs = rsqrtf(warp_sum(ss) / D + eps);
+#pragma unroll
+  for (int j = 0; j < CH; ++j) {
+    const int c = lane + 32 * j;
+    if (c < nch) {
+      float gv[8], bv[8], o[8];
+      unpack8(*reinterpret_cast<const uint4*>(g + c * 8), gv);
+      unpack8(*reinterpret_cast<const uint4*>(b + c * 8), bv);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) o[e] = (v[j][e] - mu) * rs * gv[e] + bv[e];
+      *reinterpret_cast<uint4*>(y + row * D + c * 8) = pack8(o);
+    }
+  }
+  if (lane == 0) {
+    mean[row] = mu;
+    rstd[row] = rs;
+  }
+}
+
+constexpr int LNB_THREADS = 256;
+
+// One block walks a contiguous chunk of rows; thread owns 8-element chunks
+// tid, tid+256, ...; per-block dgamma/dbeta partials go to `partial`
+// [gridDim.x][2][D] and are reduced by ln_param_reduce in block order.
+template <int CH>
+__global__ void __launch_bounds__(LNB_THREADS)
+ln_bwd_kernel(const uint16_t* __restrict__ dy, const uint16_t* __restrict__ x,
+              const uint16_t* __restrict__ g, const float* __restrict__ mean,
+              const float* __restrict__ rstd, const uint16_t* __restrict__ dres, long long rows,
+              int D, int rows_per_block, uint16_t* __restrict__ dx, float* __restrict__ partial) {
+  __shared__ float red[2][2][LNB_THREADS / 32];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int nch = D >> 3;
+  float gam[CH][8], adg[CH][8], adb[CH][8];
+#pragma unroll
+  for (int j = 0; j < CH; ++j) {
+    const int c = tid + LNB_THREADS * j;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) adg[j][e] = adb[j][e] = 0.f;
+    if (c < nch) unpack8(*reinterpret_cast<const uint4*>(g + c * 8), gam[j]);
+  }
+  const long long r0 = (long long)blockIdx.x * rows_per_block;
+  const long long r1 = min(rows, r0 + rows_per_block);
+  const float invD = 1.0f / D;
+  int buf = 0;
+  for (long long r = r0; r < r1; ++r, buf ^= 1) {
+    const float mu = mean[r], rs = rstd[r];
+    float xh[CH][8], gv[CH][8];
+    float s1 = 0.f, s2 = 0.f;
+#pragma unroll
+    for (int j = 0; j < CH; ++j) {
+      const int c = tid + LNB_THREADS * j;
+      if (c < nch) {
+        float dv[8];
+        unpack8(*reinterpret_cast<const uint4*>(dy + r * D + c * 8), dv);
+        unpack8(*reinterpret_cast<const uint4*>(x + r * D + c * 8), xh[j]);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          xh[j][e] = (xh[j][e] - mu) * rs;
+          gv[j][e] = dv[e] * gam[j][e];
+          s1 += gv[j][e];
+          s2 += gv[j][e] * xh[j][e];
+          adg[j][e] += dv[e] * xh[j][e];
+          adb[j][e] += dv[e];
+        }
+      }
+    }
+    s1 = warp_sum(s1);
+    s2 = warp_sum(s2);
+    if (lane == 0) {
+      red[buf][0][warp] = s1;
+      red[buf][1][warp] = s2;
+    }
+    __syncthreads();
+    s1 = 0.f;
+    s2 = 0.f;
+#pragma unroll
+    for (int w = 0; w < LNB_THREADS / 32; ++w) {
+      s1 += red[buf][0][w];
+      s2 += red[buf][1][w];
+    }
+    const float m1 = s1 * invD, m2 = s2 * invD;
+#pragma unroll
+    for (int j = 0; j < CH; ++j) {
+      const int c = tid + LNB_THREADS * j;
+      if (c < nch) {
+        float o[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) o[e] = rs * (gv[j][e] - m1 - xh[j][e] * m2);
+        if (dres != nullptr) {
+          float rv[8];
+          unpack8(*reinterpret_cast<const uint4*>(dres + r * D + c * 8), rv);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) o[e] += rv[e];
+        }
+        *reinterpret_cast<uint4*>(dx + r * D + c * 8) = pack8(o);
+      }
+    }
+  }
+  float* pg = partial + (long long)blockIdx.x * 2 * D;
+#pragma unroll
+  for (int j = 0; j < CH; ++j) {
+    const int c = tid + LNB_THREADS * j;
+    if (c < nch) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        pg[c * 8 + e] = adg[j][e];
+        pg[D + c * 8 + e] = adb[j][e];
+      }
+    }
+  }
+}
+
+// out_k[c] = sum over blocks b (in order) of partial[b][k][c], k = 0 (dgamma), 1 (dbeta).
+__global__ void ln_param_reduce(const float* __restrict__ partial, int nblocks, int D,
+                                uint16_t* __restrict__ dg, uint16_t* __restrict__ db) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= 2 * D) return;
+  float s = 0.f;
+  for (int b = 0; b < nblocks; ++b) s += partial[(long long)b * 2 * D + i];
+  uint16_t* out = i < D ? dg : db;
+  if (out == nullptr) return;
+  __nv_bfloat16 v = __float2bfloat16_rn(s);
+  out[i < D ? i : i - D] = *reinterpret_cast<uint16_t*>(&v);
+}
+
+// Column sums of S stacked [rows][cols] matrices, pass 1: block (cx, cy, s)
+// sums rows [cy*rpc, (cy+1)*rpc) of columns [cx*2048, cx*2048+2048) of matrix s.
+__global__ void __launch_bounds__(256)
+colsum_partial_kernel(const uint16_t* __restrict__ x, long long rows, long long cols,
+                      int rows_per_chunk, float* __restrict__ partial) {
+  const long long c = ((long long)blockIdx.x * 256 + threadIdx.x) * 8;
+  if (c >= cols) return;
+  const long long s = blockIdx.z;
+  const long long r0 = (long long)blockIdx.y * rows_per_chunk;
+  const long long r1 = min(rows, r0 + rows_per_chunk);
+  const uint16_t* base = x + s * rows * cols + c;
+  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  for (long long r = r0; r < r1; ++r) {
+    float v[8];
+    unpack8(*reinterpret_cast<const uint4*>(base + r * cols), v);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] += v[e];
+  }
+  float* p = partial + (s * gridDim.y + blockIdx.y) * cols + c;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) p[e] = acc[e];
+}
+
+__global__ void colsum_reduce_kernel(const float* __restrict__ partial, int chunks, long long cols,
+                                     long long S, uint16_t* __restrict__ out) {
+  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= S * cols) return;
+  const long long s = i / cols, c = i - s * cols;
+  float acc = 0.f;
+  for (int k = 0; k < chunks; ++k) acc += partial[(s * chunks + k) * cols + c];
+  __nv_bfloat16 v = __float2bfloat16_rn(acc);
+  out[i] = *reinterpret_cast<uint16_t*>(&v);
+}
+
+int colsum_chunks(long long rows, long long cols, long long S) {
+  const long long colblocks = (cols + 2047) / 2048;
+  long long chunks = (4LL * sm_count()) / (colblocks * S);
+  if (chunks < 1) chunks = 1;
+  if (chunks > rows) chunks = rows;
+  if (chunks > 1024) chunks = 1024;
+  return (int)(chunks < 1 ? 1 : chunks);
+}
+
+int ln_bwd_blocks(long long rows) {
+  long long b = 4LL * sm_count();
+  if (b > rows) b = rows;
+  return (int)(b < 1 ? 1 : b);
+}
+
+}  // namespace
+
+size_t colsum_partial_floats(long long S, long long rows, long long cols) {
+  if (rows < 1) rows = 1;
+  return (size_t)S * (size_t)colsum_chunks(rows, cols, S) * (size_t)cols;
+}
+
+tp_status launch_colsum_stacked(const uint16_t* x, long long S, long long rows, long long cols,
+                                uint16_t* out, float* partial, cudaStream_t stream) {
+  if (out == nullptr || cols == 0 || S == 0) return TP_OK;
+  if (rows == 0) {
+    return cuda_status(cudaMemsetAsync(out, 0, (size_t)(S * cols) * 2, stream));
+  }
+  const int chunks = colsum_chunks(rows, cols, S);
+  const dim3 grid((unsigned)((cols + 2047) / 2048), (unsigned)chunks, (unsigned)S);
+  colsum_partial_kernel<<<grid, 256, 0, stream>>>(x, rows, cols, (int)((rows + chunks - 1) / chunks),
+                                                  partial);
+  const long long n = S * cols;
+  colsum_reduce_kernel<<<(unsigned)((n + 255) / 256), 256, 0, stream>>>(partial, chunks, cols, S, out);
+  return cuda_status(cudaGetLastError());
+}
+
+tp_status launch_layernorm_fwd(const uint16_t* x, const uint16_t* g, const uint16_t* b,
+                               long long rows, int D, float eps, uint16_t* y, float* mean,
+                               float* rstd, cudaStream_t stream) {
+  if (rows == 0) return TP_OK;
+  const unsigned grid = (unsigned)((rows + 7) / 8);
+  const int per_lane = (D / 8 + 31) / 32;
+  if (per_lane <= 1) ln_fwd_kernel<1><<<grid, 256, 0, stream>>>(x, g, b, rows, D, eps, y, mean, rstd);
+  else if (per_lane <= 2) ln_fwd_kernel<2><<<grid, 256, 0, stream>>>(x, g, b, rows, D, eps, y, mean, rstd);
+  else if (per_lane <= 4) ln_fwd_kernel<4><<<grid, 256, 0, stream>>>(x, g, b, rows, D, eps, y, mean, rstd);
+  else if (per_lane <= 8) ln_fwd_kernel<8><<<grid, 256, 0, stream>>>(x, g, b, rows, D, eps, y, mean, rstd);
+  else if (per_lane <= 16) ln_fwd_kernel<16><<<grid, 256, 0, stream>>>(x, g, b, rows, D, eps, y, mean, rstd);
+  else if (per_lane <= 32) ln_fwd_kernel<32><<<grid, 256, 0, stream>>>(x, g, b, rows, D, eps, y, mean, rstd);
+  else return TP_ERR_UNSUPPORTED;
+  return cuda_status(cudaGetLastError());
+}
+
+size_t layernorm_bwd_partial_floats(long long rows, int D) {
+  return (size_t)ln_bwd_blocks(rows < 1 ? 1 : rows) * 2 * (size_t)D;
+}
+
+tp_status launch_layernorm_bwd(const uint16_t* dy, const uint16_t* x, const uint16_t* g,
+                               const float* mean, const float* rstd, const uint16_t* dres,
+                               long long rows, int D, uint16_t* dx, uint16_t* dg, uint16_t* db,
+                               float* partial, cudaStream_t stream) {
+  if (rows == 0) {
+    if (dg) cudaMemsetAsync(dg, 0, (size_t)D * 2, stream);
+    if (db) cudaMemsetAsync(db, 0, (size_t)D * 2, stream);
+    return cuda_status(cudaGetLastError());
+  }
+  const int nb = ln_bwd_blocks(rows);
+  const int rpb = (int)((rows + nb - 1) / nb);
+  const int per_thread = (D / 8 + LNB_THREADS - 1) / LNB_THREADS;
+  if (per_thread <= 1)
+    ln_bwd_kernel<1><<<nb, LNB_THREADS, 0, stream>>>(dy, x, g, mean, rstd, dres, rows, D, rpb, dx, partial);
+  else if (per_thread <= 2)
+    ln_bwd_kernel<2><<<nb, LNB_THREADS, 0, stream>>>(dy, x, g, mean, rstd, dres, rows, D, rpb, dx, partial);
+  else if (per_thread <= 4)
+    ln_bwd_kernel<4><<<nb, LNB_THREADS, 0, stream>>>(dy, x, g, mean, rstd, dres, rows, D, rpb, dx, partial);
+  else
+    return TP_ERR_UNSUPPORTED;
+  if (dg != nullptr || db != nullptr)
+    ln_param_reduce<<<(2 * D + 255) / 256, 256, 0, stream>>>(partial, nb, D, dg, db);
+  return cuda_status(cudaGetLastError());
+}
+
+}  // namespace tp

@@ -1,0 +1,218 @@
+"""torch-facing wrappers of the C ABI: the sharded MLP, attention and pre-LN layer.
+
+Each object takes UNSHARDED bf16 CUDA weights (the orientation of
+``output = GeLU(x W1) W2``: weights are [in, out]), packs them into the
+shard layouts with the library's own layout kernels, and owns the device
+buffers of one forward/backward pass.  torch is used for allocation and
+streams only; all arithmetic happens in libtplayer.so.
+"""
+from __future__ import annotations
+
+from typing import Dict, Optional
+
+import torch
+
+from . import (Dims, OP_ATTN_BWD, OP_LAYER_BWD, OP_MLP_BWD, attn_bwd, attn_fwd, layer_bwd,
+               layer_fwd, mlp_bwd, mlp_fwd, shard_cols, shard_qkv_heads, shard_rows,
+               unshard_cols, unshard_qkv_heads, workspace_size)
+
+BF16 = torch.bfloat16
+
+
+def _empty(shape, dtype=BF16, device="cuda"):
+    return torch.empty(shape, dtype=dtype, device=device)
+
+
+def pack_cols(w: torch.Tensor, t: int) -> torch.Tensor:
+    rows, cols = w.shape
+    out = _empty((t, rows, cols // t), device=w.device)
+    shard_cols(w, rows, cols, t, out)
+    return out
+
+
+def unpack_cols(p: torch.Tensor) -> torch.Tensor:
+    t, rows, ct = p.shape
+    out = _empty((rows, t * ct), device=p.device)
+    unshard_cols(p, rows, t * ct, t, out)
+    return out
+
+
+def pack_rows(w: torch.Tensor, t: int) -> torch.Tensor:
+    rows, cols = w.shape
+    out = _empty((t, rows // t, cols), device=w.device)
+    shard_rows(w, rows, cols, t, out)
+    return out
+
+
+def pack_qkv(w: torch.Tensor, heads: int, t: int) -> torch.Tensor:
+    """[rows, 3D] (or a [3D] bias) -> [t][rows][3D/t]."""
+    w2 = w.reshape(-1, w.shape[-1])
+    rows, c3 = w2.shape
+    out = _empty((t, rows, c3 // t), device=w.device)
+    shard_qkv_heads(w2, rows, c3 // 3, heads, t, out)
+    return out
+
+
+def unpack_qkv(p: torch.Tensor, heads: int) -> torch.Tensor:
+    t, rows, c3t = p.shape
+    out = _empty((rows, c3t * t), device=p.device)
+    unshard_qkv_heads(p, rows, c3t * t // 3, heads, t, out)
+    return out
+
+
+def _ws(op: int, dims: Dims, device) -> Optional[torch.Tensor]:
+    n = workspace_size(op, dims)
+    return torch.empty(max(n, 1), dtype=torch.uint8, device=device) if n else None
+
+
+class ShardedMLP:
+    """Column-parallel W1 + local GeLU, row-parallel W2 + shard sum, on one GPU."""
+
+    def __init__(self, dims: Dims, w1, b1, w2, b2):
+        self.dims = dims
+        t = dims.t
+        self.w1 = pack_cols(w1, t)           # [t][D][Ft]
+        self.w2 = pack_rows(w2, t)           # [t][Ft][D]
+        self.b1 = None if b1 is None else b1.contiguous()   # [F] == [t][Ft]
+        self.b2 = None if b2 is None else b2.contiguous()
+        self.device = w1.device
+        self.ws = None
+
+    def forward(self, x, resid=None, out: Optional[Dict] = None):
+        d = self.dims
+        T, D, F = d.batch * d.seq, d.hidden, d.ffn
+        o = out if out is not None else {
+            "y": _empty((T, D), device=self.device),
+            "a": _empty((d.t, T, F // d.t), device=self.device),
+            "h": _empty((d.t, T, F // d.t), device=self.device)}
+        mlp_fwd(d, x, self.w1, self.b1, self.w2, self.b2, resid, o["y"], o["a"], o["h"])
+        self.saved = (x, o["a"], o["h"])
+        return o
+
+    def backward(self, dy, dres=None, bias_grads=True, out: Optional[Dict] = None):
+        d = self.dims
+        T, D, F = d.batch * d.seq, d.hidden, d.ffn
+        x, a, h = self.saved
+        if self.ws is None:
+            self.ws = _ws(OP_MLP_BWD, d, self.device)
+        g = out if out is not None else {
+            "dx": _empty((T, D), device=self.device),
+            "dw1": _empty((d.t, D, F // d.t), device=self.device),
+            "dw2": _empty((d.t, F // d.t, D), device=self.device),
+            "db1": _empty((F,), device=self.device) if bias_grads else None,
+            "db2": _empty((D,), device=self.device) if bias_grads else None}
+        mlp_bwd(d, x, self.w1, self.w2, a, h, dy, dres, g["dx"], g["dw1"], g["dw2"], g["db1"],
+                g["db2"], self.ws)
+        return g
+
+
+class ShardedAttention:
+    """Q/K/V split by head, local causal attention, row-parallel Wout + shard sum."""
+
+    def __init__(self, dims: Dims, wqkv, bqkv, wout, bout):
+        self.dims = dims
+        t, H = dims.t, dims.heads
+        self.wqkv = pack_qkv(wqkv, H, t)                                  # [t][D][3Dt]
+        self.bqkv = None if bqkv is None else pack_qkv(bqkv, H, t)        # [t][1][3Dt]
+        self.wout = pack_rows(wout, t)                                    # [t][Dt][D]
+        self.bout = None if bout is None else bout.contiguous()
+        self.device = wqkv.device
+        self.ws = None
+
+    def forward(self, x, resid=None, out: Optional[Dict] = None):
+        d = self.dims
+        T, D = d.batch * d.seq, d.hidden
+        o = out if out is not None else {
+            "y": _empty((T, D), device=self.device),
+            "qkv": _empty((d.t, T, 3 * D // d.t), device=self.device),
+            "o": _empty((d.t, T, D // d.t), device=self.device),
+            "lse": _empty((d.batch, d.heads, d.seq), dtype=torch.float32, device=self.device)}
+        attn_fwd(d, x, self.wqkv, self.bqkv, self.wout, self.bout, resid, o["y"], o["qkv"],
+                 o["o"], o["lse"])
+        self.saved = (x, o["qkv"], o["o"], o["lse"])
+        return o
+
+    def backward(self, dy, dres=None, bias_grads=True, out: Optional[Dict] = None):
+        d = self.dims
+        T, D = d.batch * d.seq, d.hidden
+        x, qkv, o, lse = self.saved
+        if self.ws is None:
+            self.ws = _ws(OP_ATTN_BWD, d, self.device)
+        g = out if out is not None else {
+            "dx": _empty((T, D), device=self.device),
+            "dwqkv": _empty((d.t, D, 3 * D // d.t), device=self.device),
+            "dwout": _empty((d.t, D // d.t, D), device=self.device),
+            "dbqkv": _empty((d.t, 1, 3 * D // d.t), device=self.device) if bias_grads else None,
+            "dbout": _empty((D,), device=self.device) if bias_grads else None}
+        attn_bwd(d, x, self.wqkv, self.wout, qkv, o, lse, dy, dres, g["dx"], g["dwqkv"],
+                 g["dbqkv"], g["dwout"], g["dbout"], self.ws)
+        return g
+
+
+LAYER_PARAM_NAMES = ("ln1_g", "ln1_b", "wqkv", "bqkv", "wout", "bout", "ln2_g", "ln2_b",
+                     "w1", "b1", "w2", "b2")
+
+
+class ShardedLayer:
+    """Pre-LN layer: h = x + Attn(LN1(x)); y = h + MLP(LN2(h))."""
+
+    def __init__(self, dims: Dims, p: Dict[str, torch.Tensor]):
+        self.dims = dims
+        t, H = dims.t, dims.heads
+        self.device = p["w1"].device
+        self.p = {
+            "ln1_g": p["ln1_g"].contiguous(), "ln1_b": p["ln1_b"].contiguous(),
+            "wqkv": pack_qkv(p["wqkv"], H, t),
+            "bqkv": None if p.get("bqkv") is None else pack_qkv(p["bqkv"], H, t),
+            "wout": pack_rows(p["wout"], t),
+            "bout": None if p.get("bout") is None else p["bout"].contiguous(),
+            "ln2_g": p["ln2_g"].contiguous(), "ln2_b": p["ln2_b"].contiguous(),
+            "w1": pack_cols(p["w1"], t),
+            "b1": None if p.get("b1") is None else p["b1"].contiguous(),
+            "w2": pack_rows(p["w2"], t),
+            "b2": None if p.get("b2") is None else p["b2"].contiguous(),
+        }
+        self.ws = None
+
+    def alloc_acts(self):
+        d = self.dims
+        T, D, F, t = d.batch * d.seq, d.hidden, d.ffn, d.t
+        f32 = torch.float32
+        dev = self.device
+        return {"u1": _empty((T, D), device=dev), "mean1": _empty((T,), f32, dev),
+                "rstd1": _empty((T,), f32, dev), "qkv": _empty((t, T, 3 * D // t), device=dev),
+                "o": _empty((t, T, D // t), device=dev),
+                "lse": _empty((d.batch, d.heads, d.seq), f32, dev),
+                "h": _empty((T, D), device=dev), "u2": _empty((T, D), device=dev),
+                "mean2": _empty((T,), f32, dev), "rstd2": _empty((T,), f32, dev),
+                "a": _empty((t, T, F // t), device=dev), "hact": _empty((t, T, F // t), device=dev)}
+
+    def alloc_grads(self, bias_grads=True):
+        d = self.dims
+        D, F, t = d.hidden, d.ffn, d.t
+        dev = self.device
+        opt = (lambda s: _empty(s, device=dev)) if bias_grads else (lambda s: None)
+        return {"dln1_g": opt((D,)), "dln1_b": opt((D,)),
+                "dwqkv": _empty((t, D, 3 * D // t), device=dev), "dbqkv": opt((t, 1, 3 * D // t)),
+                "dwout": _empty((t, D // t, D), device=dev), "dbout": opt((D,)),
+                "dln2_g": opt((D,)), "dln2_b": opt((D,)),
+                "dw1": _empty((t, D, F // t), device=dev), "db1": opt((F,)),
+                "dw2": _empty((t, F // t, D), device=dev), "db2": opt((D,))}
+
+    def forward(self, x, acts=None, y=None):
+        d = self.dims
+        acts = acts if acts is not None else self.alloc_acts()
+        y = y if y is not None else _empty((d.batch * d.seq, d.hidden), device=self.device)
+        layer_fwd(d, x, self.p, acts, y)
+        self.saved = (x, acts)
+        return y, acts
+
+    def backward(self, dy, dx=None, grads=None, bias_grads=True):
+        d = self.dims
+        x, acts = self.saved
+        if self.ws is None:
+            self.ws = _ws(OP_LAYER_BWD, d, self.device)
+        dx = dx if dx is not None else torch.empty_like(x)
+        grads = grads if grads is not None else self.alloc_grads(bias_grads)
+        layer_bwd(d, x, self.p, acts, dy, dx, grads, self.ws)
+        return dx, grads

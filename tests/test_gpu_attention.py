@@ -1,0 +1,91 @@
+"""Parity of the CUDA attention sublayer (tp_attn_fwd / tp_attn_bwd) with the fp64 oracle.
+
+"The attention heads split": Q, K, V split column-wise by head, full attention
+per head on its shard, Wout split by rows and the partial outputs summed.
+"""
+import numpy as np
+import pytest
+import torch
+
+from gpu_util import assert_no_device_error, dev, dims_of, require_gpu
+from oracle import attention as oatt
+from oracle import layout as olay
+from parity import check
+from synth import Workload, make_inputs, to_f64, workload
+from tensor_transformer_layer_column_b200.sublayer import ShardedAttention
+
+pytestmark = pytest.mark.gpu
+
+
+def _run(w, inp, backward):
+    d = dims_of(w)
+    g = dev(inp)
+    m = ShardedAttention(d, g["wqkv"], g["bqkv"], g["wout"], g["bout"])
+    o = m.forward(g["x"], resid=g.get("resid"))
+    grads = m.backward(g["dy"]) if backward else None
+    torch.cuda.synchronize()
+    assert_no_device_error()
+    return o, grads
+
+
+def _compare(w, inp, o, grads):
+    t = w.t
+    x, wqkv, bqkv, wout, bout = (to_f64(inp[k]) for k in ("x", "wqkv", "bqkv", "wout", "bout"))
+    resid = to_f64(inp["resid"]) if "resid" in inp else None
+    y, sv = oatt.attn_fwd(x, wqkv, bqkv, wout, bout, w.batch, w.heads, w.causal, resid=resid)
+    check("y", o["y"], y)
+    check("qkv_save", o["qkv"], olay.shard_qkv(sv["qkv"], t))
+    check("o_save", o["o"], olay.shard_cols(sv["o"], t))
+    check("lse", o["lse"], sv["lse"])
+    if grads is not None:
+        g = oatt.attn_bwd(x, wqkv, bqkv, wout, to_f64(inp["dy"]), w.batch, w.heads, w.causal)
+        check("dx", grads["dx"], g["dx"])
+        check("dwqkv", grads["dwqkv"], olay.shard_qkv(g["dwqkv"], t))
+        check("dbqkv", grads["dbqkv"], olay.shard_qkv(g["dbqkv"][None, :], t))
+        check("dwout", grads["dwout"], olay.shard_rows(g["dwout"], t))
+        check("dbout", grads["dbout"], g["dbout"])
+
+
+def test_attn_fwd_workload_B4_S1024_D1024_H16_t4():
+    require_gpu()
+    w = workload("attn_fwd_B4_S1024_D1024_H16_t4")
+    inp = make_inputs(w)
+    o, _ = _run(w, inp, backward=False)
+    _compare(w, inp, o, None)
+
+
+# Sequence lengths that are not multiples of the 128/64 tiles, both head
+# dims, causal and full masks, every t.
+SMALL = [
+    (2, 100, 4, 64, 2, True),
+    (1, 300, 8, 128, 4, True),
+    (2, 64, 2, 64, 1, False),
+    (1, 257, 8, 64, 8, True),
+    (3, 130, 4, 128, 2, False),
+    (2, 512, 4, 128, 4, True),
+    (1, 1, 2, 64, 2, True),
+]
+
+
+@pytest.mark.parametrize("B,S,H,dh,t,causal", SMALL)
+@pytest.mark.parametrize("affine", [False, True])
+def test_attn_fwd_bwd_small(B, S, H, dh, t, causal, affine):
+    require_gpu()
+    w = Workload("attn_test", "attn_fwdbwd", batch=B, seq=S, hidden=H * dh, heads=H,
+                 head_dim=dh, t=t, causal=causal)
+    inp = make_inputs(w, seed=7, random_affine=affine)
+    o, grads = _run(w, inp, backward=True)
+    _compare(w, inp, o, grads)
+
+
+def test_attn_deterministic_run_to_run():
+    require_gpu()
+    w = Workload("attn_test", "attn_fwdbwd", batch=2, seq=384, hidden=512, heads=4, head_dim=128,
+                 t=4)
+    inp = make_inputs(w, seed=9, random_affine=True)
+    o1, g1 = _run(w, inp, True)
+    o2, g2 = _run(w, inp, True)
+    for k in o1:
+        assert torch.equal(o1[k], o2[k]), k
+    for k in g1:
+        assert torch.equal(g1[k], g2[k]), k

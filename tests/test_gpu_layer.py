@@ -1,0 +1,70 @@
+"""Parity of the CUDA pre-LN layer (tp_layer_fwd / tp_layer_bwd) with the fp64 oracle.
+
+"The layernorm placement the paper flags as critical": h = x + Attn(LN1(x));
+y = h + MLP(LN2(h)), with both sublayers tensor-parallel over t shards.
+"""
+import numpy as np
+import pytest
+import torch
+
+from gpu_util import assert_no_device_error, dev, dims_of, require_gpu
+from oracle import layer as olayer
+from oracle import layout as olay
+from parity import check
+from synth import Workload, make_inputs, to_f64, workload
+from tensor_transformer_layer_column_b200.sublayer import ShardedLayer
+
+pytestmark = pytest.mark.gpu
+
+PARAMS = ("ln1_g", "ln1_b", "wqkv", "bqkv", "wout", "bout", "ln2_g", "ln2_b", "w1", "b1", "w2", "b2")
+
+
+def _run_and_compare(w, inp):
+    d = dims_of(w)
+    g = dev(inp)
+    layer = ShardedLayer(d, {k: g[k] for k in PARAMS})
+    y, acts = layer.forward(g["x"])
+    dx, grads = layer.backward(g["dy"])
+    torch.cuda.synchronize()
+    assert_no_device_error()
+    t = w.t
+    p = {k: to_f64(inp[k]) for k in PARAMS}
+    x = to_f64(inp["x"])
+    yr, sv = olayer.layer_fwd(x, p, w.batch, w.heads, w.causal, w.ln_eps)
+    check("y", y, yr)
+    check("h", acts["h"], sv["h"])
+    check("u1", acts["u1"], sv["u1"])
+    check("u2", acts["u2"], sv["u2"])
+    check("o", acts["o"], olay.shard_cols(sv["o"], t))
+    check("lse", acts["lse"], sv["lse"])
+    check("a", acts["a"], olay.shard_cols(sv["a"], t))
+    check("hact", acts["hact"], olay.shard_cols(sv["hact"], t))
+    gr = olayer.layer_bwd(x, p, to_f64(inp["dy"]), w.batch, w.heads, w.causal, w.ln_eps)
+    check("dx", dx, gr["dx"])
+    check("dwqkv", grads["dwqkv"], olay.shard_qkv(gr["dwqkv"], t))
+    check("dbqkv", grads["dbqkv"], olay.shard_qkv(gr["dbqkv"][None, :], t))
+    check("dwout", grads["dwout"], olay.shard_rows(gr["dwout"], t))
+    check("dbout", grads["dbout"], gr["dbout"])
+    check("dw1", grads["dw1"], olay.shard_cols(gr["dw1"], t))
+    check("db1", grads["db1"], gr["db1"])
+    check("dw2", grads["dw2"], olay.shard_rows(gr["dw2"], t))
+    check("db2", grads["db2"], gr["db2"])
+    for k in ("dln1_g", "dln1_b", "dln2_g", "dln2_b"):
+        check(k, grads[k], gr[k])
+
+
+@pytest.mark.parametrize("B,S,H,dh,F,t", [(2, 128, 4, 64, 1024, 2), (1, 200, 2, 128, 1024, 2),
+                                          (2, 96, 8, 64, 2048, 8)])
+@pytest.mark.parametrize("affine", [False, True])
+def test_layer_fwd_bwd_small(B, S, H, dh, F, t, affine):
+    require_gpu()
+    w = Workload("layer_test", "layer_fwdbwd", batch=B, seq=S, hidden=H * dh, ffn=F, heads=H,
+                 head_dim=dh, t=t)
+    _run_and_compare(w, make_inputs(w, seed=13, random_affine=affine))
+
+
+def test_layer_full_size_B4_S2048_D4096_H32_F16384_t8():
+    """The pre-LN GPT layer at full size, every output and gradient against the full oracle."""
+    require_gpu()
+    w = workload("layer_fwdbwd_B4_S2048_D4096_H32_F16384_t8")
+    _run_and_compare(w, make_inputs(w))
