@@ -1,0 +1,367 @@
+"""Benchmark of the sharded pre-LN transformer layer (forward + backward) on B200.
+
+One step = one pass of the whole hot path over one batch of synthetic input:
+tp_layer_fwd followed by tp_layer_bwd of the pre-LN GPT layer
+(batch 4 x seq 2048, hidden 4096, 32 heads x 128, ffn 16384, t = 8 shards on
+one GPU), the workload the headline metric is quoted on.  Prints ONE JSON
+line (rank 0).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+N > 1 (launched with torch.distributed.run): N independent replicas, one per
+GPU, each on its own batch; no collective on the data path (weak scaling);
+the time is the max over ranks.  --impl reference times the fp64 CPU oracle
+on the host cores on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from synth import Workload, make_inputs, to_f64, workload  # noqa: E402
+
+METRIC = "sharded-layer TFLOP/s (bf16 fwd+bwd, 1 B200) and % of dense BF16 peak"
+WORKLOAD = "layer_fwdbwd_B4_S2048_D4096_H32_F16384_t8"
+NOMINAL_BF16_TFLOPS = 2250.0
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+PARAMS = ("ln1_g", "ln1_b", "wqkv", "bqkv", "wout", "bout", "ln2_g", "ln2_b", "w1", "b1", "w2", "b2")
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {k: float(p[k]) for k in FALLBACK_PEAKS}, "measured"
+    except (OSError, KeyError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+# ---------------------------------------------------------------- CPU oracle leg
+def oracle_sample(seq: int):
+    """A bounded sample of the workload: one sequence of `seq` tokens, full widths."""
+    w = workload(WORKLOAD)
+    return Workload("sample", "layer_fwdbwd", batch=1, seq=seq, hidden=w.hidden, ffn=w.ffn,
+                    heads=w.heads, head_dim=w.head_dim, t=w.t)
+
+
+def time_oracle(seq: int, reps: int):
+    """Times the fp64 oracle's layer forward + backward on the sample; returns (TFLOP/s, s/rep)."""
+    from oracle import layer as olayer
+    s = oracle_sample(seq)
+    inp = make_inputs(s)
+    p = {k: to_f64(inp[k]) for k in PARAMS}
+    x, dy = to_f64(inp["x"]), to_f64(inp["dy"])
+    times = []
+    for _ in range(reps):
+        t0 = time.perf_counter()
+        olayer.layer_fwd(x, p, s.batch, s.heads, s.causal, s.ln_eps)
+        olayer.layer_bwd(x, p, dy, s.batch, s.heads, s.causal, s.ln_eps)
+        times.append(time.perf_counter() - t0)
+    sec = statistics.median(times)
+    return s.flops() / sec / 1e12, sec, s
+
+
+def cores_used():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def run_reference(args):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return
+    seq = 256
+    from oracle import layer  # noqa: F401  (import outside the timed region)
+    value, sec, s = None, None, None
+    for _ in range(args.warmup):
+        time_oracle(seq, 1)
+    vals = []
+    for _ in range(args.steps):
+        v, sec, s = time_oracle(seq, 1)
+        vals.append(v)
+    value = statistics.median(vals)
+    sample = (f"one sequence of {seq} tokens of the workload (batch 1, full hidden/ffn/heads), "
+              f"fp64 NumPy oracle layer forward+backward, median of {args.steps} steps")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": sec * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "sample_seq": seq},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores_used(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        return False
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        try:
+            rows = open(self.path).read().strip().splitlines()
+        except OSError:
+            rows = []
+        for row in rows:
+            f = [c.strip() for c in row.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for name, val in zip(names, f[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- our arm
+def build_layer(w: Workload, device):
+    import tensor_transformer_layer_column_b200 as tl
+    from tensor_transformer_layer_column_b200.sublayer import ShardedLayer
+    tl.lib()
+    inp = make_inputs(w)
+    g = {k: v.to(device) for k, v in inp.items()}
+    dims = tl.Dims.of(w.batch, w.seq, w.hidden, w.ffn, w.heads, w.head_dim, w.t, 1, w.ln_eps)
+    layer = ShardedLayer(dims, {k: g[k] for k in PARAMS})
+    return layer, g, inp
+
+
+def run_ours(args):
+    import tensor_transformer_layer_column_b200 as tl
+    world, rank, local = dist_env()
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    device = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(device)
+    w = workload(WORKLOAD)
+    layer, g, host_inp = build_layer(w, device)
+    acts = layer.alloc_acts()
+    grads = layer.alloc_grads()
+    y = torch.empty_like(g["x"])
+    dx = torch.empty_like(g["x"])
+    stream = torch.cuda.current_stream(device)
+
+    def step(x, dy):
+        layer.forward(x, acts=acts, y=y)
+        layer.backward(dy, dx=dx, grads=grads)
+
+    for _ in range(args.warmup):
+        step(g["x"], g["dy"])
+    torch.cuda.synchronize(device)
+    if tl.check_error() != 0:
+        raise RuntimeError("device error word set during warm-up")
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    # ---- device-resident timed region (with the launch trace open)
+    per_step_launches = 64
+    trace = tl.LaunchTrace(per_step_launches * args.steps + 16)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(torch.cuda.current_device() if world == 1 else local) as clocks:
+        barrier()
+        torch.cuda.synchronize(device)
+        with trace:
+            start.record(stream)
+            for _ in range(args.steps):
+                step(g["x"], g["dy"])
+            end.record(stream)
+        torch.cuda.synchronize(device)
+        barrier()
+    ms_total = start.elapsed_time(end)
+    if world > 1:
+        t = torch.tensor([ms_total], device=device)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms_total = float(t.item())
+    clock = clocks.summary()
+    records = trace.records()
+    launches = trace.count
+    ms_step = ms_total / args.steps
+    flops_step = w.flops()
+    value = world * flops_step / (ms_step * 1e-3) / 1e12
+
+    # ---- end to end through the public API with host buffers
+    hx = host_inp["x"].pin_memory()
+    hdy = host_inp["dy"].pin_memory()
+    hy = torch.empty_like(hx).pin_memory()
+    hdx = torch.empty_like(hx).pin_memory()
+    dxin = torch.empty_like(g["x"])
+    dyin = torch.empty_like(g["dy"])
+
+    def e2e_step():
+        dxin.copy_(hx, non_blocking=True)
+        dyin.copy_(hdy, non_blocking=True)
+        step(dxin, dyin)
+        hy.copy_(y, non_blocking=True)
+        hdx.copy_(dx, non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        e2e_step()
+    barrier()
+    torch.cuda.synchronize(device)
+    s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s2.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e2.record(stream)
+    torch.cuda.synchronize(device)
+    barrier()
+    e2e_ms = s2.elapsed_time(e2)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=device)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = world * flops_step / (e2e_ms / args.steps * 1e-3) / 1e12
+    if tl.check_error() != 0:
+        raise RuntimeError("device error word set during the timed region")
+
+    # ---- roofline of the dominant kernel class (live CUDA-event durations)
+    peaks, peak_src = load_peaks()
+    by_kind = {}
+    for kind, fl, ms in records:
+        d = by_kind.setdefault(kind, [0, 0.0, 0.0])
+        d[0] += 1
+        d[1] += fl
+        d[2] += ms
+    dom = max(by_kind, key=lambda k: by_kind[k][2]) if by_kind else None
+    roofline = None
+    if dom is not None:
+        n, fl, ms = by_kind[dom]
+        achieved = fl / (ms * 1e-3) / 1e12 if ms > 0 else 0.0
+        peak = peaks["bf16_tflops_sustained"]
+        roofline = {"bound": "tensor", "kernel": f"{dom} (tcgen05)", "achieved": achieved,
+                    "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                    "peak_source": f"{peak_src} bf16_tflops_sustained", "traffic": None,
+                    "launches": n, "avg_launch_ms": ms / n,
+                    "avg_launch_gflop": fl / n / 1e9}
+    breakdown = {k: {"launches": v[0], "ms_per_step": v[2] / args.steps,
+                     "share": v[2] / max(1e-9, sum(x[2] for x in by_kind.values())),
+                     **({"tflops": v[1] / (v[2] * 1e-3) / 1e12} if v[1] > 0 and v[2] > 0 else {})}
+                 for k, v in sorted(by_kind.items(), key=lambda kv: -kv[1][2])}
+
+    # ---- CPU oracle baseline (rank 0, N = 1 only), after the GPU timing
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        oseq = 512
+        cv, csec, cs = time_oracle(oseq, 2)
+        cpu = {"value": cv, "unit": "TFLOP/s", "cores": cores_used(), "kind": "oracle",
+               "sample": (f"one sequence of {oseq} tokens of the workload (batch 1, full widths), "
+                          f"fp64 NumPy oracle layer forward+backward, median of 2 "
+                          f"({csec:.1f} s each)")}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "batch": w.batch, "seq": w.seq,
+                       "hidden": w.hidden, "ffn": w.ffn, "heads": w.heads,
+                       "head_dim": w.head_dim, "t": w.t, "causal": True,
+                       "flop_per_step": flops_step,
+                       "l2": "inputs larger than L2 (weights 384 MiB, activations > 1 GiB per step)",
+                       "parallelism": f"t{w.t} shards on each GPU; {world} independent replica(s)"},
+            "pct_dense_bf16_peak": 100.0 * value / world / NOMINAL_BF16_TFLOPS,
+            "pct_measured_bf16_peak": 100.0 * value / world / peaks["bf16_tflops"],
+            "peak_source": peak_src,
+            "e2e": {"value": e2e_value, "unit": "TFLOP/s",
+                    "h2d_bytes_per_step": hx.numel() * 2 + hdy.numel() * 2,
+                    "d2h_bytes_per_step": hy.numel() * 2 + hdx.numel() * 2},
+            "gpu_launches": launches,
+            "roofline": roofline,
+            "kernels": breakdown,
+            "clocks": clock,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true",
+                    help="skip the timed CPU oracle sample (for profiler runs)")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -18,8 +18,8 @@
  * the input-gradient GEMM.  No collective is issued.
  *
  * Conventions for every entry point
- *  - Element type: bf16, passed as raw 16-bit patterns (tp_bf16).  fp32 where
- *    stated.  Accumulation is fp32; outputs are rounded to nearest even once.
+ *  - Element type: bf16, passed as raw 16-bit patterns (tp_bf16); fp16 or fp32
+ *    where stated.  Accumulation is fp32; outputs are rounded to nearest even once.
  *  - Pointers: DEVICE pointers owned by the caller, 16-byte aligned, dense
  *    row-major, unless stated otherwise.  The library allocates nothing and
  *    keeps no state apart from cached per-device attributes.
@@ -164,14 +164,20 @@ tp_status tp_mlp_bwd(const tp_dims* dims, const tp_bf16* x, const tp_bf16* w1, c
  * "The attention heads split": shard i owns heads i*H/t .. (i+1)*H/t-1.
  *
  * tp_attn_fwd:
- *   qkv_save[i] = x Wqkv_i + bqkv_i        [t][T][3*Dt]; within shard i, columns
- *                 [0,Dt) are q, [Dt,2Dt) k, [2Dt,3Dt) v, local head j at j*dh
+ *   qkv_save[i] = x Wqkv_i + bqkv_i        [t][T][3*Dt], FP16; within shard i,
+ *                 columns [0,Dt) are q, [Dt,2Dt) k, [2Dt,3Dt) v, local head j at j*dh
  *   per head:  O = softmax(q k^T / sqrt(dh) + mask) v, softmax in fp32;
  *              lse_save = log-sum-exp of the scaled masked scores, fp32 [B][H][S]
- *   o_save[i]   = the shard's head outputs  [t][T][Dt]
+ *   o_save[i]   = the shard's head outputs  [t][T][Dt] (bf16)
  *   y = sum_i o_save[i] Wout_i + bout (+ resid)      [T][D]
+ * Inside the attention sublayer the products run on fp16 operands (x and Wqkv
+ * are converted, q/k/v, P, dO, dS are fp16; fp32 accumulation): with bf16
+ * storage the softmax over long causal rows amplifies the rounding of q and k
+ * to a relative error near 6e-3 in O at S = 2048, with fp16 near 2e-3.  A value
+ * beyond the fp16 range (|v| > 65504) sets device error code 0x301
+ * (tp_check_error reports TP_ERR_TIMEOUT with that code).
  * bqkv, bout, resid may be NULL.  Uses batch, seq, hidden, heads, head_dim, t,
- * causal.  No workspace. */
+ * causal.  Workspace: tp_workspace_size(TP_OP_ATTN_FWD, dims) bytes. */
 tp_status tp_attn_fwd(const tp_dims* dims, const tp_bf16* x, const tp_bf16* wqkv,
                       const tp_bf16* bqkv, const tp_bf16* wout, const tp_bf16* bout,
                       const tp_bf16* resid, tp_bf16* y, tp_bf16* qkv_save, tp_bf16* o_save,
@@ -206,9 +212,9 @@ typedef struct {
 
 /* Activations saved by tp_layer_fwd for tp_layer_bwd (all caller-owned). */
 typedef struct {
-  tp_bf16* u1;            /* LN1(x) [T][D] */
+  tp_bf16* u1;            /* LN1(x) [T][D], FP16 (it feeds only the fp16 attention products) */
   float *mean1, *rstd1;   /* [T] */
-  tp_bf16* qkv;           /* [t][T][3Dt] */
+  tp_bf16* qkv;           /* [t][T][3Dt], FP16 */
   tp_bf16* o;             /* [t][T][Dt] */
   float* lse;             /* [B][H][S] */
   tp_bf16* h;             /* x + attention output [T][D] */
@@ -226,7 +232,7 @@ typedef struct {
 } tp_layer_grads;
 
 /* tp_layer_fwd: x [T][D] -> y [T][D], filling every field of *acts.
- * No workspace. */
+ * Workspace: tp_workspace_size(TP_OP_LAYER_FWD, dims) bytes. */
 tp_status tp_layer_fwd(const tp_dims* dims, const tp_bf16* x, const tp_layer_params* params,
                        const tp_layer_acts* acts, tp_bf16* y, void* ws, size_t ws_bytes,
                        tp_stream stream);
@@ -255,6 +261,24 @@ tp_status tp_layernorm_bwd(const tp_bf16* dy, const tp_bf16* x, const tp_bf16* g
                            const float* mean, const float* rstd, const tp_bf16* dres, int rows,
                            int D, tp_bf16* dx, tp_bf16* dgamma, tp_bf16* dbeta, void* ws,
                            size_t ws_bytes, tp_stream stream);
+
+/* ------------------------------------------------------------------ launch trace
+ * Measurement support (the pages describe no tracing; this exists so that a
+ * bench can time individual kernels inside a longer step on their own stream).
+ * tp_trace_begin: from now on, for the i-th kernel the library enqueues
+ * (i < capacity), record events[2i] on the launch stream just before it and
+ * events[2i+1] just after it, store its class in kinds[i] (0 GEMM, 1 attention
+ * forward, 2 attention-backward prep, 3 attention dK/dV, 4 attention dQ,
+ * 5 LayerNorm forward, 6 LayerNorm backward, 7 LayerNorm parameter reduce,
+ * 8 column sum, 9 layout copy, 10 bf16-to-fp16 conversion) and, if flops != NULL, its algorithmic FLOP
+ * count in flops[i] (0 for non-contraction kernels).  events are cudaEvent_t
+ * handles created by the caller on the current device; arrays are host memory
+ * owned by the caller and must stay valid until tp_trace_end.  capacity 0
+ * closes the trace.  INVALID_ARG on negative capacity or NULL arrays.
+ * tp_trace_end: closes the trace and returns the number of launches seen
+ * since tp_trace_begin (which may exceed capacity). */
+tp_status tp_trace_begin(void* const* events, int* kinds, double* flops, int capacity);
+int tp_trace_end(void);
 
 #ifdef __cplusplus
 }

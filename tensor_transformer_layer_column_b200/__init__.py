@@ -21,7 +21,8 @@ __all__ = [
     "workspace_size", "check_error", "version", "EXPORTED_SYMBOLS",
     "shard_cols", "unshard_cols", "shard_rows", "unshard_rows", "shard_qkv_heads",
     "unshard_qkv_heads", "mlp_fwd", "mlp_bwd", "attn_fwd", "attn_bwd", "layer_fwd", "layer_bwd",
-    "layernorm_fwd", "layernorm_bwd", "layernorm_bwd_workspace_size",
+    "layernorm_fwd", "layernorm_bwd", "layernorm_bwd_workspace_size", "LaunchTrace",
+    "TRACE_KINDS",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -93,10 +94,13 @@ _SIGS = {
     "tp_layernorm_bwd_workspace_size": [ctypes.c_int, ctypes.c_int],
     "tp_layernorm_bwd": [_P, _P, _P, _P, _P, _P, ctypes.c_int, ctypes.c_int, _P, _P, _P, _P,
                          ctypes.c_size_t, _P],
+    "tp_trace_begin": [ctypes.POINTER(ctypes.c_void_p), ctypes.POINTER(ctypes.c_int),
+                       ctypes.POINTER(ctypes.c_double), ctypes.c_int],
+    "tp_trace_end": [],
 }
 _RESTYPES = {"tp_version": ctypes.c_char_p, "tp_status_string": ctypes.c_char_p,
              "tp_workspace_size": ctypes.c_size_t,
-             "tp_layernorm_bwd_workspace_size": ctypes.c_size_t}
+             "tp_layernorm_bwd_workspace_size": ctypes.c_size_t, "tp_trace_end": ctypes.c_int}
 EXPORTED_SYMBOLS = tuple(_SIGS)
 
 _lib: Optional[ctypes.CDLL] = None
@@ -265,3 +269,47 @@ def layernorm_bwd(dy, x, gamma, mean, rstd, dres, rows, D, dx, dgamma, dbeta, ws
     _check(lib().tp_layernorm_bwd(_ptr(dy), _ptr(x), _ptr(gamma), _ptr(mean), _ptr(rstd),
                                   _ptr(dres), rows, D, _ptr(dx), _ptr(dgamma), _ptr(dbeta), wp,
                                   wn, _stream(stream, x)), "tp_layernorm_bwd")
+
+
+TRACE_KINDS = ("gemm", "attn_fwd", "attn_bwd_prep", "attn_bwd_dkdv", "attn_bwd_dq", "ln_fwd",
+               "ln_bwd", "ln_param", "colsum", "layout", "cast")
+
+
+class LaunchTrace:
+    """Context manager around tp_trace_begin / tp_trace_end.
+
+    Inside the block every kernel the library enqueues is bracketed by CUDA
+    events on its own stream; afterwards ``records()`` gives, per launch, its
+    class name, algorithmic FLOPs and device duration in milliseconds.
+    """
+
+    def __init__(self, capacity: int):
+        import torch
+        self.capacity = capacity
+        self._events = [torch.cuda.Event(enable_timing=True) for _ in range(2 * capacity)]
+        for e in self._events:       # materialise the underlying cudaEvent_t handles
+            e.record()
+        torch.cuda.synchronize()
+        self._handles = (ctypes.c_void_p * (2 * capacity))(*[e.cuda_event for e in self._events])
+        self._kinds = (ctypes.c_int * capacity)()
+        self._flops = (ctypes.c_double * capacity)()
+        self.count = 0
+
+    def __enter__(self):
+        _check(lib().tp_trace_begin(self._handles, self._kinds, self._flops, self.capacity),
+               "tp_trace_begin")
+        return self
+
+    def __exit__(self, *exc):
+        self.count = lib().tp_trace_end()
+        return False
+
+    def records(self):
+        import torch
+        torch.cuda.synchronize()
+        n = min(self.count, self.capacity)
+        out = []
+        for i in range(n):
+            ms = self._events[2 * i].elapsed_time(self._events[2 * i + 1])
+            out.append((TRACE_KINDS[self._kinds[i]], float(self._flops[i]), ms))
+        return out

@@ -144,8 +144,8 @@ tp_status check_layer(const tp_dims* d) {
 }
 
 OperandDesc op(const void* p, bool mn, int src, long long inner, long long outer,
-               long long shards, long long ld, long long shard_stride) {
-  return OperandDesc{p, mn, src, inner, outer, shards, ld, shard_stride};
+               long long shards, long long ld, long long shard_stride, bool f16 = false) {
+  return OperandDesc{p, mn, f16, src, inner, outer, shards, ld, shard_stride};
 }
 
 // Workspace carving: consecutive 256-byte aligned slices.
@@ -265,17 +265,20 @@ tp_status mlp_bwd_impl(const Sizes& z, bf16p x, bf16p w1, bf16p w2, bf16p a_save
 }
 
 // ------------------------------------------------------------------ attention
-tp_status attn_fwd_impl(const Sizes& z, int causal, bf16p x, bf16p wqkv, bf16p bqkv, bf16p wout,
-                        bf16p bout, bf16p resid, uint16_t* y, uint16_t* qkv, uint16_t* o,
-                        float* lse, cudaStream_t st) {
+// The attention sublayer runs on fp16 operands internally (see attention.cu
+// for why): its input x16 and the fp16 copy of Wqkv are prepared by the
+// caller of these helpers; qkv is stored fp16, O bf16.
+tp_status attn_fwd_impl(const Sizes& z, int causal, bf16p x16, bf16p wqkv16, bf16p bqkv,
+                        bf16p wout, bf16p bout, bf16p resid, uint16_t* y, uint16_t* qkv,
+                        uint16_t* o, float* lse, cudaStream_t st) {
   if (z.T == 0) return TP_OK;
   const long long w3 = 3 * z.Dt;
   GemmProblem g1{};
   g1.m_shards = 1; g1.n_shards = (int)z.t; g1.Mt = (int)z.T; g1.Nt = (int)w3;
   g1.k_shards = 1; g1.Kt = (int)z.D;
-  g1.a = op(x, false, SHARD_NONE, z.D, z.T, 1, z.D, 0);
-  g1.b = op(wqkv, true, SHARD_MN, w3, z.D, z.t, w3, z.D * w3);
-  g1.epi = EPI_LINEAR; g1.c = qkv; g1.bias = bqkv;
+  g1.a = op(x16, false, SHARD_NONE, z.D, z.T, 1, z.D, 0, true);
+  g1.b = op(wqkv16, true, SHARD_MN, w3, z.D, z.t, w3, z.D * w3, true);
+  g1.epi = EPI_LINEAR; g1.c = qkv; g1.bias = bqkv; g1.out_f16 = true;
   g1.c_ms = 0; g1.c_ns = z.T * w3; g1.ldc = w3;
   tp_status s = launch_gemm(g1, st);
   if (s != TP_OK) return s;
@@ -293,17 +296,18 @@ tp_status attn_fwd_impl(const Sizes& z, int causal, bf16p x, bf16p wqkv, bf16p b
   return launch_gemm(g2, st);
 }
 
-size_t attn_bwd_ws(const Sizes& z) {
+// Workspace of attn_bwd_impl: dO (fp16), dqkv (fp16), attention scratch, colsum partials.
+size_t attn_bwd_core_ws(const Sizes& z) {
   Carver c(nullptr);
-  c.take<uint16_t>((size_t)(z.T * z.D));        // dO
-  c.take<uint16_t>((size_t)(z.T * 3 * z.D));    // dqkv
+  c.take<uint16_t>((size_t)(z.T * z.D));
+  c.take<uint16_t>((size_t)(z.T * 3 * z.D));
   c.take<uint8_t>(attn_bwd_scratch_bytes((int)z.B, (int)z.S, (int)z.H, (int)z.dh));
   c.take<float>(colsum_scratch_floats_max(z.T, {{z.t, 3 * z.Dt}, {1, z.D}}));
   return align_up(c.off, 256);
 }
 
-tp_status attn_bwd_impl(const Sizes& z, int causal, bf16p x, bf16p wqkv, bf16p wout, bf16p qkv,
-                        bf16p o, const float* lse, bf16p dy, bf16p dres, uint16_t* dx,
+tp_status attn_bwd_impl(const Sizes& z, int causal, bf16p x16, bf16p wqkv16, bf16p wout,
+                        bf16p qkv, bf16p o, const float* lse, bf16p dy, bf16p dres, uint16_t* dx,
                         uint16_t* dwqkv, uint16_t* dbqkv, uint16_t* dwout, uint16_t* dbout,
                         void* ws, cudaStream_t st) {
   const long long w3 = 3 * z.Dt;
@@ -320,13 +324,13 @@ tp_status attn_bwd_impl(const Sizes& z, int causal, bf16p x, bf16p wqkv, bf16p w
   void* scratch = c.take<uint8_t>(attn_bwd_scratch_bytes((int)z.B, (int)z.S, (int)z.H, (int)z.dh));
   float* part = c.take<float>(colsum_scratch_floats_max(z.T, {{z.t, w3}, {1, z.D}}));
 
-  // dO_i = dY Wout_i^T: B = Wout_i read as [n = Dt][k = D], K-major, N shards.
+  // dO_i = dY Wout_i^T: B = Wout_i read as [n = Dt][k = D], K-major, N shards; fp16 out.
   GemmProblem g1{};
   g1.m_shards = 1; g1.n_shards = (int)z.t; g1.Mt = (int)z.T; g1.Nt = (int)z.Dt;
   g1.k_shards = 1; g1.Kt = (int)z.D;
   g1.a = op(dy, false, SHARD_NONE, z.D, z.T, 1, z.D, 0);
   g1.b = op(wout, false, SHARD_MN, z.D, z.Dt, z.t, z.D, z.Dt * z.D);
-  g1.epi = EPI_LINEAR; g1.c = dout;
+  g1.epi = EPI_LINEAR; g1.c = dout; g1.out_f16 = true;
   g1.c_ms = 0; g1.c_ns = z.T * z.Dt; g1.ldc = z.Dt;
   tp_status s = launch_gemm(g1, st);
   if (s != TP_OK) return s;
@@ -345,37 +349,55 @@ tp_status attn_bwd_impl(const Sizes& z, int causal, bf16p x, bf16p wqkv, bf16p w
                       causal, scratch, st);
   if (s != TP_OK) return s;
 
-  // dWqkv_i = x^T dqkv_i, N shards.
+  // dWqkv_i = x^T dqkv_i, N shards (fp16 operands).
   GemmProblem g3{};
   g3.m_shards = 1; g3.n_shards = (int)z.t; g3.Mt = (int)z.D; g3.Nt = (int)w3;
   g3.k_shards = 1; g3.Kt = (int)z.T;
-  g3.a = op(x, true, SHARD_NONE, z.D, z.T, 1, z.D, 0);
-  g3.b = op(dqkv, true, SHARD_MN, w3, z.T, z.t, w3, z.T * w3);
+  g3.a = op(x16, true, SHARD_NONE, z.D, z.T, 1, z.D, 0, true);
+  g3.b = op(dqkv, true, SHARD_MN, w3, z.T, z.t, w3, z.T * w3, true);
   g3.epi = EPI_LINEAR; g3.c = dwqkv;
   g3.c_ms = 0; g3.c_ns = z.D * w3; g3.ldc = w3;
   if ((s = launch_gemm(g3, st)) != TP_OK) return s;
 
-  // dX = sum_i dqkv_i Wqkv_i^T (+ dres): the backward shard reduction.
+  // dX = sum_i dqkv_i Wqkv_i^T (+ dres): the backward shard reduction (fp16 operands).
   GemmProblem g4{};
   g4.m_shards = 1; g4.n_shards = 1; g4.Mt = (int)z.T; g4.Nt = (int)z.D;
   g4.k_shards = (int)z.t; g4.Kt = (int)w3;
-  g4.a = op(dqkv, false, SHARD_K, w3, z.T, z.t, w3, z.T * w3);
-  g4.b = op(wqkv, false, SHARD_K, w3, z.D, z.t, w3, z.D * w3);
+  g4.a = op(dqkv, false, SHARD_K, w3, z.T, z.t, w3, z.T * w3, true);
+  g4.b = op(wqkv16, false, SHARD_K, w3, z.D, z.t, w3, z.D * w3, true);
   g4.epi = EPI_LINEAR; g4.c = dx; g4.aux = dres;
   g4.c_ms = 0; g4.c_ns = 0; g4.ldc = z.D;
   if ((s = launch_gemm(g4, st)) != TP_OK) return s;
 
-  if (dbqkv && (s = launch_colsum_stacked(dqkv, z.t, z.T, w3, dbqkv, part, st)) != TP_OK) return s;
+  if (dbqkv && (s = launch_colsum_stacked(dqkv, z.t, z.T, w3, dbqkv, part, st, true)) != TP_OK)
+    return s;
   if (dbout && (s = launch_colsum_stacked(dy, 1, z.T, z.D, dbout, part, st)) != TP_OK) return s;
   return TP_OK;
 }
 
+// Standalone attention: fp16 copies of x and Wqkv, then the core workspace.
+size_t attn_fwd_ws(const Sizes& z) {
+  Carver c(nullptr);
+  c.take<uint16_t>((size_t)(z.T * z.D));
+  c.take<uint16_t>((size_t)(z.D * 3 * z.D));
+  return align_up(c.off, 256);
+}
+
+size_t attn_bwd_ws(const Sizes& z) {
+  return attn_fwd_ws(z) + attn_bwd_core_ws(z);
+}
+
+size_t layer_fwd_ws(const Sizes& z) {
+  return align_up((size_t)(z.D * 3 * z.D) * 2, 256);   // fp16 copy of Wqkv
+}
+
 size_t layer_bwd_ws(const Sizes& z) {
   Carver c(nullptr);
-  c.take<uint16_t>((size_t)(z.T * z.D));   // du
-  c.take<uint16_t>((size_t)(z.T * z.D));   // dh
+  c.take<uint16_t>((size_t)(z.D * 3 * z.D));   // fp16 copy of Wqkv
+  c.take<uint16_t>((size_t)(z.T * z.D));       // du
+  c.take<uint16_t>((size_t)(z.T * z.D));       // dh
   c.take<float>(layernorm_bwd_partial_floats(z.T, (int)z.D));
-  const size_t sub = mlp_bwd_ws(z) > attn_bwd_ws(z) ? mlp_bwd_ws(z) : attn_bwd_ws(z);
+  const size_t sub = mlp_bwd_ws(z) > attn_bwd_core_ws(z) ? mlp_bwd_ws(z) : attn_bwd_core_ws(z);
   c.take<uint8_t>(sub);
   return align_up(c.off, 256);
 }
@@ -411,7 +433,9 @@ const char* tp_status_string(tp_status s) {
 
 size_t tp_workspace_size(int op_, const tp_dims* d) {
   switch (op_) {
-    case TP_OP_MLP_FWD: case TP_OP_ATTN_FWD: case TP_OP_LAYER_FWD: return 0;
+    case TP_OP_MLP_FWD: return 0;
+    case TP_OP_ATTN_FWD: return check_attn(d) == TP_OK ? attn_fwd_ws(sizes_of(*d)) : 0;
+    case TP_OP_LAYER_FWD: return check_layer(d) == TP_OK ? layer_fwd_ws(sizes_of(*d)) : 0;
     case TP_OP_MLP_BWD: return check_mlp(d) == TP_OK ? mlp_bwd_ws(sizes_of(*d)) : 0;
     case TP_OP_ATTN_BWD: return check_attn(d) == TP_OK ? attn_bwd_ws(sizes_of(*d)) : 0;
     case TP_OP_LAYER_BWD: return check_layer(d) == TP_OK ? layer_bwd_ws(sizes_of(*d)) : 0;
@@ -521,7 +545,6 @@ tp_status tp_attn_fwd(const tp_dims* dims, const tp_bf16* x, const tp_bf16* wqkv
                       const tp_bf16* bqkv, const tp_bf16* wout, const tp_bf16* bout,
                       const tp_bf16* resid, tp_bf16* y, tp_bf16* qkv_save, tp_bf16* o_save,
                       float* lse_save, void* ws, size_t ws_bytes, tp_stream s) {
-  (void)ws; (void)ws_bytes;
   tp_status st = check_attn(dims);
   if (st != TP_OK) return st;
   const bool tok = (long long)dims->batch * dims->seq > 0;
@@ -529,8 +552,17 @@ tp_status tp_attn_fwd(const tp_dims* dims, const tp_bf16* x, const tp_bf16* wqkv
     return TP_ERR_INVALID_ARG;
   if (!all_aligned(x, wqkv, bqkv, wout, bout, resid, y, qkv_save, o_save, lse_save))
     return TP_ERR_MISALIGNED;
-  return attn_fwd_impl(sizes_of(*dims), dims->causal, x, wqkv, bqkv, wout, bout, resid, y,
-                       qkv_save, o_save, lse_save, (cudaStream_t)s);
+  const Sizes z = sizes_of(*dims);
+  if (z.T == 0) return TP_OK;
+  if ((st = check_ws(ws, ws_bytes, attn_fwd_ws(z))) != TP_OK) return st;
+  cudaStream_t cs = (cudaStream_t)s;
+  Carver c(ws);
+  uint16_t* x16 = c.take<uint16_t>((size_t)(z.T * z.D));
+  uint16_t* w16 = c.take<uint16_t>((size_t)(z.D * 3 * z.D));
+  if ((st = launch_cast_f16(x, (size_t)(z.T * z.D), x16, cs)) != TP_OK) return st;
+  if ((st = launch_cast_f16(wqkv, (size_t)(z.D * 3 * z.D), w16, cs)) != TP_OK) return st;
+  return attn_fwd_impl(z, dims->causal, x16, w16, bqkv, wout, bout, resid, y, qkv_save, o_save,
+                       lse_save, cs);
 }
 
 tp_status tp_attn_bwd(const tp_dims* dims, const tp_bf16* x, const tp_bf16* wqkv,
@@ -549,8 +581,18 @@ tp_status tp_attn_bwd(const tp_dims* dims, const tp_bf16* x, const tp_bf16* wqkv
     return TP_ERR_MISALIGNED;
   const Sizes z = sizes_of(*dims);
   if ((st = check_ws(ws, ws_bytes, z.T ? attn_bwd_ws(z) : 0)) != TP_OK) return st;
-  return attn_bwd_impl(z, dims->causal, x, wqkv, wout, qkv_save, o_save, lse_save, dy, dres, dx,
-                       dwqkv, dbqkv, dwout, dbout, ws, (cudaStream_t)s);
+  cudaStream_t cs = (cudaStream_t)s;
+  if (z.T == 0)
+    return attn_bwd_impl(z, dims->causal, nullptr, nullptr, wout, nullptr, nullptr, nullptr,
+                         nullptr, nullptr, nullptr, dwqkv, dbqkv, dwout, dbout, nullptr, cs);
+  Carver c(ws);
+  uint16_t* x16 = c.take<uint16_t>((size_t)(z.T * z.D));
+  uint16_t* w16 = c.take<uint16_t>((size_t)(z.D * 3 * z.D));
+  void* core = c.take<uint8_t>(attn_bwd_core_ws(z));
+  if ((st = launch_cast_f16(x, (size_t)(z.T * z.D), x16, cs)) != TP_OK) return st;
+  if ((st = launch_cast_f16(wqkv, (size_t)(z.D * 3 * z.D), w16, cs)) != TP_OK) return st;
+  return attn_bwd_impl(z, dims->causal, x16, w16, wout, qkv_save, o_save, lse_save, dy, dres, dx,
+                       dwqkv, dbqkv, dwout, dbout, core, cs);
 }
 
 // ------------------------------------------------------------------ LayerNorm
@@ -599,7 +641,6 @@ static tp_status check_layer_ptrs(const tp_layer_params* p, const tp_layer_acts*
 
 tp_status tp_layer_fwd(const tp_dims* dims, const tp_bf16* x, const tp_layer_params* p,
                        const tp_layer_acts* a, tp_bf16* y, void* ws, size_t ws_bytes, tp_stream s) {
-  (void)ws; (void)ws_bytes;
   tp_status st = check_layer(dims);
   if (st != TP_OK) return st;
   if (!x || !y) return TP_ERR_INVALID_ARG;
@@ -608,10 +649,14 @@ tp_status tp_layer_fwd(const tp_dims* dims, const tp_bf16* x, const tp_layer_par
   const Sizes z = sizes_of(*dims);
   cudaStream_t cs = (cudaStream_t)s;
   if (z.T == 0) return TP_OK;
+  if ((st = check_ws(ws, ws_bytes, layer_fwd_ws(z))) != TP_OK) return st;
+  uint16_t* w16 = static_cast<uint16_t*>(ws);
+  if ((st = launch_cast_f16(p->wqkv, (size_t)(z.D * 3 * z.D), w16, cs)) != TP_OK) return st;
+  // LN1 writes u1 in fp16: it only feeds the attention sublayer's fp16 products.
   if ((st = launch_layernorm_fwd(x, p->ln1_g, p->ln1_b, z.T, (int)z.D, dims->ln_eps, a->u1,
-                                 a->mean1, a->rstd1, cs)) != TP_OK)
+                                 a->mean1, a->rstd1, cs, true)) != TP_OK)
     return st;
-  if ((st = attn_fwd_impl(z, dims->causal, a->u1, p->wqkv, p->bqkv, p->wout, p->bout, x, a->h,
+  if ((st = attn_fwd_impl(z, dims->causal, a->u1, w16, p->bqkv, p->wout, p->bout, x, a->h,
                           a->qkv, a->o, a->lse, cs)) != TP_OK)
     return st;
   if ((st = launch_layernorm_fwd(a->h, p->ln2_g, p->ln2_b, z.T, (int)z.D, dims->ln_eps, a->u2,
@@ -645,11 +690,13 @@ tp_status tp_layer_bwd(const tp_dims* dims, const tp_bf16* x, const tp_layer_par
     return cuda_status(cudaGetLastError());
   }
   Carver c(ws);
+  uint16_t* w16 = c.take<uint16_t>((size_t)(z.D * 3 * z.D));
   uint16_t* du = c.take<uint16_t>((size_t)(z.T * z.D));
   uint16_t* dh = c.take<uint16_t>((size_t)(z.T * z.D));
   float* lnp = c.take<float>(layernorm_bwd_partial_floats(z.T, (int)z.D));
-  const size_t sub = mlp_bwd_ws(z) > attn_bwd_ws(z) ? mlp_bwd_ws(z) : attn_bwd_ws(z);
+  const size_t sub = mlp_bwd_ws(z) > attn_bwd_core_ws(z) ? mlp_bwd_ws(z) : attn_bwd_core_ws(z);
   void* subws = c.take<uint8_t>(sub);
+  if ((st = launch_cast_f16(p->wqkv, (size_t)(z.D * 3 * z.D), w16, cs)) != TP_OK) return st;
 
   // y = h + MLP(LN2(h)):  du2 = MLP^T(dy);  dh = dy + LN2^T(du2).
   if ((st = mlp_bwd_impl(z, a->u2, p->w1, p->w2, a->a, a->hact, dy, nullptr, du, g->dw1, g->dw2,
@@ -659,7 +706,7 @@ tp_status tp_layer_bwd(const tp_dims* dims, const tp_bf16* x, const tp_layer_par
                                  g->dln2_g, g->dln2_b, lnp, cs)) != TP_OK)
     return st;
   // h = x + Attn(LN1(x)):  du1 = Attn^T(dh);  dx = dh + LN1^T(du1).
-  if ((st = attn_bwd_impl(z, dims->causal, a->u1, p->wqkv, p->wout, a->qkv, a->o, a->lse, dh,
+  if ((st = attn_bwd_impl(z, dims->causal, a->u1, w16, p->wout, a->qkv, a->o, a->lse, dh,
                           nullptr, du, g->dwqkv, g->dbqkv, g->dwout, g->dbout, subws, cs)) != TP_OK)
     return st;
   return launch_layernorm_bwd(du, x, p->ln1_g, a->mean1, a->rstd1, dh, z.T, (int)z.D, dx,

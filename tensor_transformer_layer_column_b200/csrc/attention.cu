@@ -2,17 +2,24 @@
 //
 // "The attention heads split": shard i owns heads i*H/t .. (i+1)*H/t-1 and
 // runs full attention for them with no communication.  The projections arrive
-// as qkv [t][T][3Dt] (the column-parallel GEMM's output): local head j of
-// shard i has q at columns j*dh, k at Dt + j*dh, v at 2Dt + j*dh of rows
+// as qkv [t][T][3Dt] (the column-parallel GEMM's output, fp16): local head j
+// of shard i has q at columns j*dh, k at Dt + j*dh, v at 2Dt + j*dh of rows
 // b*S + s.  One launch covers every head of every shard.
+//
+// Operand precision: q, k, v, P, dO and dS are fp16 (10-bit mantissa) rather
+// than bf16.  Over long causal rows the softmax amplifies the storage
+// rounding of q and k (and of the LayerNorm output they come from); with
+// bf16 storage that alone puts the relative L2 error of O and of dWout near
+// 6e-3 at S = 2048, with fp16 near 2e-3.  The tensor-core rate is the same.
 //
 // Forward (per 128-query block, head, batch):
 //   S = q k^T (tcgen05, fp32 in TMEM, double-buffered), online softmax in
 //   fp32 by one thread per query row (base-2 exponent, scores pre-scaled by
-//   log2(e)/sqrt(dh)), P rounded to bf16 into swizzled shared memory,
+//   log2(e)/sqrt(dh)), P rounded to fp16 into swizzled shared memory,
 //   O += P v (tcgen05, fp32 in TMEM, rescaled in place when the row max moves).
 //   Writes O [t][T][Dt] (bf16) and the log-sum-exp [B][H][S] (fp32).
-// Backward (P recomputed from the log-sum-exp; no atomics, deterministic):
+// Backward (P recomputed from the log-sum-exp; no atomics, deterministic;
+// dO in and dqkv out are fp16):
 //   prep:   Dv = rowsum(dO * O), lse2 = lse * log2(e)
 //   dK/dV:  per 128-key block, walk 64-query blocks:  S^T = k q^T, dP^T = v dO^T,
 //           P^T, dS^T = P^T * (dP^T - Dv) by one thread per key row,
@@ -73,6 +80,15 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, const C
       return false;
     }
   }
+}
+
+__device__ __forceinline__ uint4 pack8_f16(const float* v) {
+  uint4 o;
+  o.x = pack_f16x2(v[0], v[1]);
+  o.y = pack_f16x2(v[2], v[3]);
+  o.z = pack_f16x2(v[4], v[5]);
+  o.w = pack_f16x2(v[6], v[7]);
+  return o;
 }
 
 __device__ __forceinline__ uint4 pack8_bf16(const float* v) {
@@ -192,8 +208,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_qkv, const AttnArgs p) {
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      constexpr uint32_t id_qk = idesc_bf16_f32(128, 128, false, false);
-      constexpr uint32_t id_pv = idesc_bf16_f32(128, DH, false, true);
+      constexpr uint32_t id_qk = idesc_f32acc(128, 128, false, false, true);
+      constexpr uint32_t id_pv = idesc_f32acc(128, DH, false, true, true);
       const uint32_t sq = smem_u32(smem), sp = smem_u32(smem + C::OFF_P);
       bool ok = wait_bar(q_full, 0, ctl, ERR_ATTN_FWD_WAIT);
       for (int j = 0; ok && j <= n_kv; ++j) {
@@ -292,7 +308,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_qkv, const AttnArgs p) {
       }
 #pragma unroll
       for (int g = 0; g < 16; ++g)
-        *reinterpret_cast<uint4*>(sp + sw128_offset(C::BM, r, g * 8)) = pack8_bf16(&s[g * 8]);
+        *reinterpret_cast<uint4*>(sp + sw128_offset(C::BM, r, g * 8)) = pack8_f16(&s[g * 8]);
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(p_full);
@@ -348,7 +364,7 @@ __global__ void attn_bwd_prep_kernel(const uint16_t* __restrict__ o, const uint1
     const uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wg[4] = {g.x, g.y, g.z, g.w};
 #pragma unroll
     for (int k = 0; k < 4; ++k)
-      acc += bf16_lo(wa[k]) * bf16_lo(wg[k]) + bf16_hi(wa[k]) * bf16_hi(wg[k]);
+      acc += bf16_lo(wa[k]) * f16_lo(wg[k]) + bf16_hi(wa[k]) * f16_hi(wg[k]);
   }
   dvec[idx] = acc;
   lse2[idx] = lse[idx] * kLog2e;
@@ -450,8 +466,8 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_kv128,
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      constexpr uint32_t id_s = idesc_bf16_f32(128, C::BQ, false, false);
-      constexpr uint32_t id_acc = idesc_bf16_f32(128, DH, false, true);
+      constexpr uint32_t id_s = idesc_f32acc(128, C::BQ, false, false, true);
+      constexpr uint32_t id_acc = idesc_f32acc(128, DH, false, true, true);
       const uint32_t sk = smem_u32(smem + C::OFF_K), sv = smem_u32(smem + C::OFF_V);
       const uint32_t spt = smem_u32(smem + C::OFF_PT), sdst = smem_u32(smem + C::OFF_DST);
       bool ok = wait_bar(kv_full, 0, ctl, ERR_ATTN_DKDV_WAIT);
@@ -519,8 +535,8 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_kv128,
 #pragma unroll
         for (int g = 0; g < 4; ++g) {
           const uint32_t off = sw128_offset(C::BK, r, c * 32 + g * 8);
-          *reinterpret_cast<uint4*>(spt + off) = pack8_bf16(&pv[g * 8]);
-          *reinterpret_cast<uint4*>(sdst + off) = pack8_bf16(&dsv[g * 8]);
+          *reinterpret_cast<uint4*>(spt + off) = pack8_f16(&pv[g * 8]);
+          *reinterpret_cast<uint4*>(sdst + off) = pack8_f16(&dsv[g * 8]);
         }
       }
       tc_fence_before();
@@ -541,16 +557,19 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_kv128,
         tc_wait_ld();
         if (valid) {
           float v[32], kx[32];
+          bool over = false;
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
             v[e] = __uint_as_float(rv[e]);
             kx[e] = __uint_as_float(rk[e]) * p.inv_sqrt_dh;
+            over |= fabsf(v[e]) > 65504.0f || fabsf(kx[e]) > 65504.0f;
           }
 #pragma unroll
           for (int g = 0; g < 4; ++g) {
-            *reinterpret_cast<uint4*>(row + colv + c * 32 + g * 8) = pack8_bf16(&v[g * 8]);
-            *reinterpret_cast<uint4*>(row + colk + c * 32 + g * 8) = pack8_bf16(&kx[g * 8]);
+            *reinterpret_cast<uint4*>(row + colv + c * 32 + g * 8) = pack8_f16(&v[g * 8]);
+            *reinterpret_cast<uint4*>(row + colk + c * 32 + g * 8) = pack8_f16(&kx[g * 8]);
           }
+          if (over && p.err) atomicCAS(p.err, 0u, 0x301u);
         }
       }
     }
@@ -658,8 +677,8 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q128,
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      constexpr uint32_t id_s = idesc_bf16_f32(128, C::BK, false, false);
-      constexpr uint32_t id_acc = idesc_bf16_f32(128, DH, false, true);
+      constexpr uint32_t id_s = idesc_f32acc(128, C::BK, false, false, true);
+      constexpr uint32_t id_acc = idesc_f32acc(128, DH, false, true, true);
       const uint32_t sq = smem_u32(smem + C::OFF_Q), sd = smem_u32(smem + C::OFF_DO);
       const uint32_t sds = smem_u32(smem + C::OFF_DS);
       bool ok = wait_bar(q_full, 0, ctl, ERR_ATTN_DQ_WAIT);
@@ -724,7 +743,7 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q128,
         }
 #pragma unroll
         for (int g = 0; g < 4; ++g)
-          *reinterpret_cast<uint4*>(sds + sw128_offset(C::BQ, r, c * 32 + g * 8)) = pack8_bf16(&dsv[g * 8]);
+          *reinterpret_cast<uint4*>(sds + sw128_offset(C::BQ, r, c * 32 + g * 8)) = pack8_f16(&dsv[g * 8]);
       }
       tc_fence_before();
       mbar_arrive(s_free);
@@ -742,11 +761,16 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q128,
         tc_wait_ld();
         if (qvalid) {
           float v[32];
+          bool over = false;
 #pragma unroll
-          for (int e = 0; e < 32; ++e) v[e] = __uint_as_float(rq[e]) * p.inv_sqrt_dh;
+          for (int e = 0; e < 32; ++e) {
+            v[e] = __uint_as_float(rq[e]) * p.inv_sqrt_dh;
+            over |= fabsf(v[e]) > 65504.0f;
+          }
 #pragma unroll
           for (int g = 0; g < 4; ++g)
-            *reinterpret_cast<uint4*>(row + c * 32 + g * 8) = pack8_bf16(&v[g * 8]);
+            *reinterpret_cast<uint4*>(row + c * 32 + g * 8) = pack8_f16(&v[g * 8]);
+          if (over && p.err) atomicCAS(p.err, 0u, 0x301u);
         }
       }
     }
@@ -776,7 +800,7 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// 4-D map over a shard-packed activation [t][B*S][width]: dims (width, S, B, t),
+// 4-D map over a shard-packed fp16 activation [t][B*S][width]: dims (width, S, B, t),
 // box (64, rows, 1, 1), 128-byte swizzle, zero fill past S.
 bool encode_act(CUtensorMap* m, const void* base, long long width, int S, int B, int t,
                 long long T, int rows) {
@@ -787,7 +811,7 @@ bool encode_act(CUtensorMap* m, const void* base, long long width, int S, int B,
                                  (cuuint64_t)T * width * 2};
   const cuuint32_t box[4] = {64, (cuuint32_t)rows, 1, 1};
   const cuuint32_t estr[4] = {1, 1, 1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box,
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4, const_cast<void*>(base), dims, strides, box,
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -808,6 +832,12 @@ bool set_smem(const void* kern, int bytes) {
     for (int i = 0; i < 8; ++i)
       if (!done[dev][i]) { done[dev][i] = kern; break; }
   return true;
+}
+
+// Query-key pairs that take part in the softmax (masked pairs not counted), all heads.
+double core_pairs(const AttnArgs& a) {
+  const double s = a.S;
+  return (double)a.B * a.H * (a.causal ? s * (s + 1) / 2 : s * s);
 }
 
 AttnArgs make_args(int B, int S, int H, int dh, int t, int causal) {
@@ -832,7 +862,10 @@ tp_status fwd_launch(const uint16_t* qkv, uint16_t* o, float* lse, const AttnArg
   auto kern = attn_fwd_kernel<DH>;
   if (!set_smem((const void*)kern, FwdCfg<DH>::SMEM)) return TP_ERR_CUDA;
   const dim3 grid((a.S + 127) / 128, a.H, a.B);
-  kern<<<grid, 192, FwdCfg<DH>::SMEM, st>>>(tm, p);
+  {
+    TraceScope ts(st, TK_ATTN_FWD, 4.0 * DH * core_pairs(a));
+    kern<<<grid, 192, FwdCfg<DH>::SMEM, st>>>(tm, p);
+  }
   return cuda_status(cudaGetLastError());
 }
 
@@ -842,8 +875,11 @@ tp_status bwd_launch(const uint16_t* qkv, const uint16_t* o, const float* lse, c
   float* dvec = static_cast<float*>(scratch);
   float* lse2 = dvec + align_up((size_t)a.B * a.H * a.S, 64);
   const long long n = (long long)a.B * a.H * a.S;
-  attn_bwd_prep_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(o, dout, lse, dvec, lse2, a.B,
-                                                                     a.S, a.H, a.Ht, DH, a.Dt, a.T);
+  {
+    TraceScope ts(st, TK_ATTN_BWD_PREP);
+    attn_bwd_prep_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(o, dout, lse, dvec, lse2, a.B,
+                                                                       a.S, a.H, a.Ht, DH, a.Dt, a.T);
+  }
   if (cudaGetLastError() != cudaSuccess) return TP_ERR_CUDA;
   AttnArgs p = a;
   p.out = dqkv;
@@ -861,9 +897,16 @@ tp_status bwd_launch(const uint16_t* qkv, const uint16_t* o, const float* lse, c
   auto k2 = attn_bwd_dq_kernel<DH>;
   if (!set_smem((const void*)k1, DkdvCfg<DH>::SMEM) || !set_smem((const void*)k2, DqCfg<DH>::SMEM))
     return TP_ERR_CUDA;
-  k1<<<dim3((a.S + 127) / 128, a.H, a.B), 192, DkdvCfg<DH>::SMEM, st>>>(kv128, q64, do64, p);
+  {
+    // dP, dV and dK: three of the backward's four algorithmic products.
+    TraceScope ts(st, TK_ATTN_BWD_DKDV, 6.0 * DH * core_pairs(a));
+    k1<<<dim3((a.S + 127) / 128, a.H, a.B), 192, DkdvCfg<DH>::SMEM, st>>>(kv128, q64, do64, p);
+  }
   if (cudaGetLastError() != cudaSuccess) return TP_ERR_CUDA;
-  k2<<<dim3((a.S + 127) / 128, a.H, a.B), 192, DqCfg<DH>::SMEM, st>>>(q128, do128, kv64, p);
+  {
+    TraceScope ts(st, TK_ATTN_BWD_DQ, 2.0 * DH * core_pairs(a));
+    k2<<<dim3((a.S + 127) / 128, a.H, a.B), 192, DqCfg<DH>::SMEM, st>>>(q128, do128, kv64, p);
+  }
   return cuda_status(cudaGetLastError());
 }
 

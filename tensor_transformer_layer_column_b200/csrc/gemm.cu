@@ -26,7 +26,7 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// 3-D bf16 tensor map with 128-byte swizzle; out-of-range elements read as 0.
+// 3-D 16-bit tensor map with 128-byte swizzle; out-of-range elements read as 0.
 bool encode_operand(CUtensorMap* map, const OperandDesc& d, uint32_t box_outer) {
   auto fn = encode_fn();
   if (!fn) return false;
@@ -35,7 +35,7 @@ bool encode_operand(CUtensorMap* map, const OperandDesc& d, uint32_t box_outer) 
   const cuuint64_t strides[2] = {(cuuint64_t)d.ld * 2, (cuuint64_t)shard_stride * 2};
   const cuuint32_t box[3] = {64, box_outer, 1};
   const cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(d.ptr), dims, strides,
+  CUresult r = fn(map, d.f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(d.ptr), dims, strides,
                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
@@ -43,7 +43,7 @@ bool encode_operand(CUtensorMap* map, const OperandDesc& d, uint32_t box_outer) 
 
 template <bool A_MN, bool B_MN>
 tp_status launch_inst(const CUtensorMap& ta, const CUtensorMap& tb, const GemmArgs& args,
-                      int grid, cudaStream_t stream) {
+                      int grid, double flops, cudaStream_t stream) {
   static bool configured[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -54,7 +54,10 @@ tp_status launch_inst(const CUtensorMap& ta, const CUtensorMap& tb, const GemmAr
       return TP_ERR_CUDA;
     configured[dev] = true;
   }
-  kern<<<grid, GEMM_THREADS, GEMM_SMEM_BYTES, stream>>>(ta, tb, args);
+  {
+    TraceScope ts(stream, TK_GEMM, flops);
+    kern<<<grid, GEMM_THREADS, GEMM_SMEM_BYTES, stream>>>(ta, tb, args);
+  }
   return cuda_status(cudaGetLastError());
 }
 
@@ -62,6 +65,7 @@ tp_status launch_inst(const CUtensorMap& ta, const CUtensorMap& tb, const GemmAr
 
 tp_status launch_gemm(const GemmProblem& g, cudaStream_t stream) {
   if (g.Mt <= 0 || g.Nt <= 0 || g.Kt <= 0) return TP_OK;   // empty product: nothing to do
+  if (g.a.f16 != g.b.f16) return TP_ERR_INVALID_ARG;       // one MMA takes one operand type
   CUtensorMap ta, tb;
   if (!encode_operand(&ta, g.a, g.a.mn_major ? 64 : GEMM_BM)) return TP_ERR_CUDA;
   if (!encode_operand(&tb, g.b, g.b.mn_major ? 64 : GEMM_BN)) return TP_ERR_CUDA;
@@ -89,12 +93,16 @@ tp_status launch_gemm(const GemmProblem& g, cudaStream_t stream) {
   a.c_ns = g.c_ns;
   a.ldc = g.ldc;
   a.err = error_word();
+  a.idesc = idesc_f32acc(GEMM_BM, GEMM_BN, g.a.mn_major, g.b.mn_major, g.a.f16);
+  a.out_f16 = g.out_f16 ? 1 : 0;
   const int grid = (int)(tiles < sm_count() ? tiles : sm_count());
+  const double flops = 2.0 * g.m_shards * (double)g.Mt * g.n_shards * (double)g.Nt * g.k_shards *
+                       (double)g.Kt;
 
-  if (!g.a.mn_major && g.b.mn_major) return launch_inst<false, true>(ta, tb, a, grid, stream);
-  if (!g.a.mn_major && !g.b.mn_major) return launch_inst<false, false>(ta, tb, a, grid, stream);
-  if (g.a.mn_major && g.b.mn_major) return launch_inst<true, true>(ta, tb, a, grid, stream);
-  return launch_inst<true, false>(ta, tb, a, grid, stream);
+  if (!g.a.mn_major && g.b.mn_major) return launch_inst<false, true>(ta, tb, a, grid, flops, stream);
+  if (!g.a.mn_major && !g.b.mn_major) return launch_inst<false, false>(ta, tb, a, grid, flops, stream);
+  if (g.a.mn_major && g.b.mn_major) return launch_inst<true, true>(ta, tb, a, grid, flops, stream);
+  return launch_inst<true, false>(ta, tb, a, grid, flops, stream);
 }
 
 }  // namespace tp

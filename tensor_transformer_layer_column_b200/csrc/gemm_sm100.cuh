@@ -1,7 +1,7 @@
 // Persistent, warp-specialised tcgen05 GEMM for the sharded sublayer.
 //
-// C[m, n] = epilogue( sum_k A[m, k] * B[k, n] ), bf16 operands, fp32
-// accumulation in tensor memory, bf16 output.
+// C[m, n] = epilogue( sum_k A[m, k] * B[k, n] ), bf16 or fp16 operands (A and
+// B of one type), fp32 accumulation in tensor memory, bf16 or fp16 output.
 //
 // Tensor-parallel structure ("How transformer layers actually decompose",
 // "The attention heads split"): the t shards of a column-parallel product
@@ -57,6 +57,7 @@ enum : unsigned int {
   ERR_GEMM_MMA_WAIT = 0x102,
   ERR_GEMM_EPI_WAIT = 0x103,
   ERR_GEMM_DRAIN_WAIT = 0x104,
+  ERR_F16_RANGE = 0x301,          // a value stored as fp16 exceeded its range
 };
 
 struct GemmArgs {
@@ -75,6 +76,8 @@ struct GemmArgs {
   const __nv_bfloat16* aux;
   const __nv_bfloat16* bias;
   long long c_ms, c_ns, ldc;
+  uint32_t idesc;                  // tcgen05 instruction descriptor (operand type, shape, majors)
+  int out_f16;                     // C (and C2) stored as fp16 instead of bf16
   unsigned int* err;
 };
 
@@ -220,7 +223,7 @@ gemm_bf16_sm100(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32(GEMM_BM, GEMM_BN, A_MN, B_MN);
+      const uint32_t idesc = p.idesc;
       int it = 0, tcount = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x, ++tcount) {
@@ -327,15 +330,33 @@ gemm_bf16_sm100(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
           }
         }
         __nv_bfloat16* cp = p.c + base + n;
+        if (p.out_f16) {
+          bool over = false;
 #pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          if (g * 8 < nvalid) {
-            uint4 o;
-            o.x = pack_bf16x2(v[g * 8 + 0], v[g * 8 + 1]);
-            o.y = pack_bf16x2(v[g * 8 + 2], v[g * 8 + 3]);
-            o.z = pack_bf16x2(v[g * 8 + 4], v[g * 8 + 5]);
-            o.w = pack_bf16x2(v[g * 8 + 6], v[g * 8 + 7]);
-            *reinterpret_cast<uint4*>(cp + g * 8) = o;
+          for (int g = 0; g < 4; ++g) {
+            if (g * 8 < nvalid) {
+              uint4 o;
+              o.x = pack_f16x2(v[g * 8 + 0], v[g * 8 + 1]);
+              o.y = pack_f16x2(v[g * 8 + 2], v[g * 8 + 3]);
+              o.z = pack_f16x2(v[g * 8 + 4], v[g * 8 + 5]);
+              o.w = pack_f16x2(v[g * 8 + 6], v[g * 8 + 7]);
+              *reinterpret_cast<uint4*>(cp + g * 8) = o;
+#pragma unroll
+              for (int e = 0; e < 8; ++e) over |= fabsf(v[g * 8 + e]) > 65504.0f;
+            }
+          }
+          if (over && p.err) atomicCAS(p.err, 0u, ERR_F16_RANGE);
+        } else {
+#pragma unroll
+          for (int g = 0; g < 4; ++g) {
+            if (g * 8 < nvalid) {
+              uint4 o;
+              o.x = pack_bf16x2(v[g * 8 + 0], v[g * 8 + 1]);
+              o.y = pack_bf16x2(v[g * 8 + 2], v[g * 8 + 3]);
+              o.z = pack_bf16x2(v[g * 8 + 4], v[g * 8 + 5]);
+              o.w = pack_bf16x2(v[g * 8 + 6], v[g * 8 + 7]);
+              *reinterpret_cast<uint4*>(cp + g * 8) = o;
+            }
           }
         }
         if (p.epi == EPI_BIAS_GELU) {

@@ -17,6 +17,7 @@ namespace tp {
 struct OperandDesc {
   const void* ptr;
   bool mn_major;
+  bool f16;                  // element type: fp16 (true) or bf16 (false)
   int src;                   // ShardSrc
   long long inner, outer, shards;
   long long ld;              // elements between consecutive outer indices
@@ -33,6 +34,7 @@ struct GemmProblem {
   const void* aux;
   const void* bias;
   long long c_ms, c_ns, ldc;
+  bool out_f16;              // store C / C2 as fp16
 };
 
 tp_status launch_gemm(const GemmProblem& g, cudaStream_t stream);
@@ -46,11 +48,12 @@ int sm_count();
 // of colsum_partial_floats(S, rows, cols) floats).
 size_t colsum_partial_floats(long long S, long long rows, long long cols);
 tp_status launch_colsum_stacked(const uint16_t* x, long long S, long long rows, long long cols,
-                                uint16_t* out, float* partial, cudaStream_t stream);
+                                uint16_t* out, float* partial, cudaStream_t stream,
+                                bool in_f16 = false);
 
 tp_status launch_layernorm_fwd(const uint16_t* x, const uint16_t* g, const uint16_t* b,
                                long long rows, int D, float eps, uint16_t* y, float* mean,
-                               float* rstd, cudaStream_t stream);
+                               float* rstd, cudaStream_t stream, bool out_f16 = false);
 size_t layernorm_bwd_partial_floats(long long rows, int D);
 tp_status launch_layernorm_bwd(const uint16_t* dy, const uint16_t* x, const uint16_t* g,
                                const float* mean, const float* rstd, const uint16_t* dres,
@@ -70,6 +73,28 @@ tp_status launch_shard_cols(const uint16_t* src, int rows, int cols, int t, uint
 tp_status launch_shard_qkv(const uint16_t* src, int rows, int hidden, int t, uint16_t* dst,
                            bool inverse, cudaStream_t stream);
 tp_status launch_copy(const uint16_t* src, size_t n, uint16_t* dst, cudaStream_t stream);
+// bf16 -> fp16 element copy (n elements); values beyond the fp16 range set
+// the device error word to 0x301.
+tp_status launch_cast_f16(const uint16_t* src, size_t n, uint16_t* dst, cudaStream_t stream);
+
+// Kernel classes reported by the launch trace (tp_trace_begin).
+enum TraceKind : int {
+  TK_GEMM = 0, TK_ATTN_FWD = 1, TK_ATTN_BWD_PREP = 2, TK_ATTN_BWD_DKDV = 3, TK_ATTN_BWD_DQ = 4,
+  TK_LN_FWD = 5, TK_LN_BWD = 6, TK_LN_PARAM = 7, TK_COLSUM = 8, TK_LAYOUT = 9, TK_CAST = 10,
+};
+
+// Brackets one kernel launch with the trace's events when a trace is open.
+class TraceScope {
+ public:
+  TraceScope(cudaStream_t stream, int kind, double flops = 0.0);
+  ~TraceScope();
+  TraceScope(const TraceScope&) = delete;
+  TraceScope& operator=(const TraceScope&) = delete;
+
+ private:
+  cudaStream_t stream_;
+  int slot_;
+};
 
 inline tp_status cuda_status(cudaError_t e) { return e == cudaSuccess ? TP_OK : TP_ERR_CUDA; }
 

@@ -3,6 +3,7 @@
 // W1 split by columns as [W1_left | W1_right], W2 split by rows as
 // [W2_top; W2_bottom]; "The attention heads split": Q, K, V split by the
 // columns of each shard's heads).
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include "internal.h"
@@ -77,6 +78,27 @@ __global__ void copy_kernel(const uint16_t* __restrict__ src, uint16_t* __restri
   }
 }
 
+// bf16 -> fp16, 8 elements per thread step; out-of-range values flag `err`.
+__global__ void cast_f16_kernel(const uint16_t* __restrict__ src, uint16_t* __restrict__ dst,
+                                long long n8, unsigned int* err) {
+  bool over = false;
+  for (long long v = blockIdx.x * (long long)blockDim.x + threadIdx.x; v < n8;
+       v += (long long)gridDim.x * blockDim.x) {
+    const uint4 u = *reinterpret_cast<const uint4*>(src + v * 8);
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float lo = __uint_as_float(w[q] << 16), hi = __uint_as_float(w[q] & 0xFFFF0000u);
+      over |= fabsf(lo) > 65504.0f || fabsf(hi) > 65504.0f;
+      __half2 h = __floats2half2_rn(lo, hi);
+      o[q] = *reinterpret_cast<uint32_t*>(&h);
+    }
+    *reinterpret_cast<uint4*>(dst + v * 8) = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+  if (over && err) atomicCAS(err, 0u, 0x301u);
+}
+
 int grid_for(long long work) {
   const long long cap = (long long)sm_count() * 8;
   long long g = (work + 255) / 256;
@@ -93,6 +115,7 @@ tp_status launch_shard_cols(const uint16_t* src, int rows, int cols, int t, uint
   const long long ct = cols / t;
   const long long n = (long long)rows * cols;
   if (n == 0) return TP_OK;
+  TraceScope ts(stream, TK_LAYOUT);
   if (ct % 8 == 0 && aligned16(src) && aligned16(dst))
     shard_cols_kernel<8><<<grid_for(n / 8), 256, 0, stream>>>(src, dst, rows, ct, t, inverse);
   else
@@ -105,6 +128,7 @@ tp_status launch_shard_qkv(const uint16_t* src, int rows, int hidden, int t, uin
   const long long dt = hidden / t;
   const long long n = (long long)rows * 3 * hidden;
   if (n == 0) return TP_OK;
+  TraceScope ts(stream, TK_LAYOUT);
   if (dt % 8 == 0 && aligned16(src) && aligned16(dst))
     shard_qkv_kernel<8><<<grid_for(n / 8), 256, 0, stream>>>(src, dst, rows, dt, t, inverse);
   else
@@ -114,10 +138,20 @@ tp_status launch_shard_qkv(const uint16_t* src, int rows, int hidden, int t, uin
 
 tp_status launch_copy(const uint16_t* src, size_t n, uint16_t* dst, cudaStream_t stream) {
   if (n == 0) return TP_OK;
+  TraceScope ts(stream, TK_LAYOUT);
   if (n % 8 == 0 && aligned16(src) && aligned16(dst))
     copy_kernel<8><<<grid_for((long long)n / 8), 256, 0, stream>>>(src, dst, (long long)n);
   else
     copy_kernel<1><<<grid_for((long long)n), 256, 0, stream>>>(src, dst, (long long)n);
+  return cuda_status(cudaGetLastError());
+}
+
+tp_status launch_cast_f16(const uint16_t* src, size_t n, uint16_t* dst, cudaStream_t stream) {
+  if (n == 0) return TP_OK;
+  if (n % 8 || !aligned16(src) || !aligned16(dst)) return TP_ERR_MISALIGNED;
+  TraceScope ts(stream, TK_CAST);
+  cast_f16_kernel<<<grid_for((long long)n / 8), 256, 0, stream>>>(src, dst, (long long)n / 8,
+                                                                  error_word());
   return cuda_status(cudaGetLastError());
 }
 

@@ -3,6 +3,7 @@
 // column sums for bias gradients.  128-bit loads and stores throughout; fp32
 // statistics; every reduction order is fixed, so results repeat bit for bit.
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include "internal.h"
@@ -32,18 +33,44 @@ __device__ __forceinline__ uint4 pack8(const float (&f)[8]) {
   return u;
 }
 
+__device__ __forceinline__ void unpack8_f16(const uint4& u, float (&f)[8]) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const __half2 h = *reinterpret_cast<const __half2*>(&w[q]);
+    const float2 v = __half22float2(h);
+    f[2 * q] = v.x;
+    f[2 * q + 1] = v.y;
+  }
+}
+
+__device__ __forceinline__ uint4 pack8_f16(const float (&f)[8]) {
+  uint4 u;
+  uint32_t w[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    __half2 v = __floats2half2_rn(f[2 * q], f[2 * q + 1]);
+    w[q] = *reinterpret_cast<uint32_t*>(&v);
+  }
+  u.x = w[0]; u.y = w[1]; u.z = w[2]; u.w = w[3];
+  return u;
+}
+
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
   return v;
 }
 
-// One warp per row; lane owns 8-element chunks lane, lane+32, ...
-template <int CH>
+// One warp per row; lane owns 8-element chunks lane, lane+32, ...  The
+// output is bf16, or fp16 when F16OUT (values beyond the fp16 range set
+// `err` to 0x301).
+template <int CH, bool F16OUT>
 __global__ void __launch_bounds__(256)
 ln_fwd_kernel(const uint16_t* __restrict__ x, const uint16_t* __restrict__ g,
               const uint16_t* __restrict__ b, long long rows, int D, float eps,
-              uint16_t* __restrict__ y, float* __restrict__ mean, float* __restrict__ rstd) {
+              uint16_t* __restrict__ y, float* __restrict__ mean, float* __restrict__ rstd,
+              unsigned int* err) {
   const int lane = threadIdx.x & 31;
   const long long row = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (row >= rows) return;
@@ -82,7 +109,15 @@ ln_fwd_kernel(const uint16_t* __restrict__ x, const uint16_t* __restrict__ g,
       unpack8(*reinterpret_cast<const uint4*>(b + c * 8), bv);
 #pragma unroll
       for (int e = 0; e < 8; ++e) o[e] = (v[j][e] - mu) * rs * gv[e] + bv[e];
-      *reinterpret_cast<uint4*>(y + row * D + c * 8) = pack8(o);
+      if (F16OUT) {
+        *reinterpret_cast<uint4*>(y + row * D + c * 8) = pack8_f16(o);
+        bool over = false;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) over |= fabsf(o[e]) > 65504.0f;
+        if (over && err) atomicCAS(err, 0u, 0x301u);
+      } else {
+        *reinterpret_cast<uint4*>(y + row * D + c * 8) = pack8(o);
+      }
     }
   }
   if (lane == 0) {
@@ -200,6 +235,7 @@ __global__ void ln_param_reduce(const float* __restrict__ partial, int nblocks, 
 
 // Column sums of S stacked [rows][cols] matrices, pass 1: block (cx, cy, s)
 // sums rows [cy*rpc, (cy+1)*rpc) of columns [cx*2048, cx*2048+2048) of matrix s.
+template <bool F16IN>
 __global__ void __launch_bounds__(256)
 colsum_partial_kernel(const uint16_t* __restrict__ x, long long rows, long long cols,
                       int rows_per_chunk, float* __restrict__ partial) {
@@ -212,7 +248,8 @@ colsum_partial_kernel(const uint16_t* __restrict__ x, long long rows, long long 
   float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
   for (long long r = r0; r < r1; ++r) {
     float v[8];
-    unpack8(*reinterpret_cast<const uint4*>(base + r * cols), v);
+    if (F16IN) unpack8_f16(*reinterpret_cast<const uint4*>(base + r * cols), v);
+    else unpack8(*reinterpret_cast<const uint4*>(base + r * cols), v);
 #pragma unroll
     for (int e = 0; e < 8; ++e) acc[e] += v[e];
   }
@@ -255,34 +292,60 @@ size_t colsum_partial_floats(long long S, long long rows, long long cols) {
 }
 
 tp_status launch_colsum_stacked(const uint16_t* x, long long S, long long rows, long long cols,
-                                uint16_t* out, float* partial, cudaStream_t stream) {
+                                uint16_t* out, float* partial, cudaStream_t stream, bool in_f16) {
   if (out == nullptr || cols == 0 || S == 0) return TP_OK;
   if (rows == 0) {
     return cuda_status(cudaMemsetAsync(out, 0, (size_t)(S * cols) * 2, stream));
   }
   const int chunks = colsum_chunks(rows, cols, S);
   const dim3 grid((unsigned)((cols + 2047) / 2048), (unsigned)chunks, (unsigned)S);
-  colsum_partial_kernel<<<grid, 256, 0, stream>>>(x, rows, cols, (int)((rows + chunks - 1) / chunks),
-                                                  partial);
+  {
+    TraceScope ts(stream, TK_COLSUM);
+    const int rpc = (int)((rows + chunks - 1) / chunks);
+    if (in_f16)
+      colsum_partial_kernel<true><<<grid, 256, 0, stream>>>(x, rows, cols, rpc, partial);
+    else
+      colsum_partial_kernel<false><<<grid, 256, 0, stream>>>(x, rows, cols, rpc, partial);
+  }
   const long long n = S * cols;
-  colsum_reduce_kernel<<<(unsigned)((n + 255) / 256), 256, 0, stream>>>(partial, chunks, cols, S, out);
+  {
+    TraceScope ts(stream, TK_COLSUM);
+    colsum_reduce_kernel<<<(unsigned)((n + 255) / 256), 256, 0, stream>>>(partial, chunks, cols, S, out);
+  }
+  return cuda_status(cudaGetLastError());
+}
+
+template <bool F16OUT>
+tp_status ln_fwd_dispatch(const uint16_t* x, const uint16_t* g, const uint16_t* b, long long rows,
+                          int D, float eps, uint16_t* y, float* mean, float* rstd,
+                          cudaStream_t stream) {
+  const unsigned grid = (unsigned)((rows + 7) / 8);
+  const int per_lane = (D / 8 + 31) / 32;
+  unsigned int* err = error_word();
+  TraceScope ts(stream, TK_LN_FWD);
+  if (per_lane <= 1)
+    ln_fwd_kernel<1, F16OUT><<<grid, 256, 0, stream>>>(x, g, b, rows, D, eps, y, mean, rstd, err);
+  else if (per_lane <= 2)
+    ln_fwd_kernel<2, F16OUT><<<grid, 256, 0, stream>>>(x, g, b, rows, D, eps, y, mean, rstd, err);
+  else if (per_lane <= 4)
+    ln_fwd_kernel<4, F16OUT><<<grid, 256, 0, stream>>>(x, g, b, rows, D, eps, y, mean, rstd, err);
+  else if (per_lane <= 8)
+    ln_fwd_kernel<8, F16OUT><<<grid, 256, 0, stream>>>(x, g, b, rows, D, eps, y, mean, rstd, err);
+  else if (per_lane <= 16)
+    ln_fwd_kernel<16, F16OUT><<<grid, 256, 0, stream>>>(x, g, b, rows, D, eps, y, mean, rstd, err);
+  else if (per_lane <= 32)
+    ln_fwd_kernel<32, F16OUT><<<grid, 256, 0, stream>>>(x, g, b, rows, D, eps, y, mean, rstd, err);
+  else
+    return TP_ERR_UNSUPPORTED;
   return cuda_status(cudaGetLastError());
 }
 
 tp_status launch_layernorm_fwd(const uint16_t* x, const uint16_t* g, const uint16_t* b,
                                long long rows, int D, float eps, uint16_t* y, float* mean,
-                               float* rstd, cudaStream_t stream) {
+                               float* rstd, cudaStream_t stream, bool out_f16) {
   if (rows == 0) return TP_OK;
-  const unsigned grid = (unsigned)((rows + 7) / 8);
-  const int per_lane = (D / 8 + 31) / 32;
-  if (per_lane <= 1) ln_fwd_kernel<1><<<grid, 256, 0, stream>>>(x, g, b, rows, D, eps, y, mean, rstd);
-  else if (per_lane <= 2) ln_fwd_kernel<2><<<grid, 256, 0, stream>>>(x, g, b, rows, D, eps, y, mean, rstd);
-  else if (per_lane <= 4) ln_fwd_kernel<4><<<grid, 256, 0, stream>>>(x, g, b, rows, D, eps, y, mean, rstd);
-  else if (per_lane <= 8) ln_fwd_kernel<8><<<grid, 256, 0, stream>>>(x, g, b, rows, D, eps, y, mean, rstd);
-  else if (per_lane <= 16) ln_fwd_kernel<16><<<grid, 256, 0, stream>>>(x, g, b, rows, D, eps, y, mean, rstd);
-  else if (per_lane <= 32) ln_fwd_kernel<32><<<grid, 256, 0, stream>>>(x, g, b, rows, D, eps, y, mean, rstd);
-  else return TP_ERR_UNSUPPORTED;
-  return cuda_status(cudaGetLastError());
+  if (out_f16) return ln_fwd_dispatch<true>(x, g, b, rows, D, eps, y, mean, rstd, stream);
+  return ln_fwd_dispatch<false>(x, g, b, rows, D, eps, y, mean, rstd, stream);
 }
 
 size_t layernorm_bwd_partial_floats(long long rows, int D) {
@@ -301,6 +364,8 @@ tp_status launch_layernorm_bwd(const uint16_t* dy, const uint16_t* x, const uint
   const int nb = ln_bwd_blocks(rows);
   const int rpb = (int)((rows + nb - 1) / nb);
   const int per_thread = (D / 8 + LNB_THREADS - 1) / LNB_THREADS;
+  {
+  TraceScope ts(stream, TK_LN_BWD);
   if (per_thread <= 1)
     ln_bwd_kernel<1><<<nb, LNB_THREADS, 0, stream>>>(dy, x, g, mean, rstd, dres, rows, D, rpb, dx, partial);
   else if (per_thread <= 2)
@@ -309,8 +374,11 @@ tp_status launch_layernorm_bwd(const uint16_t* dy, const uint16_t* x, const uint
     ln_bwd_kernel<4><<<nb, LNB_THREADS, 0, stream>>>(dy, x, g, mean, rstd, dres, rows, D, rpb, dx, partial);
   else
     return TP_ERR_UNSUPPORTED;
-  if (dg != nullptr || db != nullptr)
+  }
+  if (dg != nullptr || db != nullptr) {
+    TraceScope ts(stream, TK_LN_PARAM);
     ln_param_reduce<<<(2 * D + 255) / 256, 256, 0, stream>>>(partial, nb, D, dg, db);
+  }
   return cuda_status(cudaGetLastError());
 }
 

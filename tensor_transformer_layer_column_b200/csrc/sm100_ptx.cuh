@@ -9,6 +9,7 @@
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 namespace tp {
 
@@ -247,12 +248,13 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo
   return d;
 }
 
-// Instruction descriptor for kind::f16 with bf16 A/B and fp32 D.
-__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn_major,
-                                                      bool b_mn_major) {
+// Instruction descriptor for kind::f16 with fp32 D; A and B share one type,
+// bf16 (f16 = false) or fp16 (f16 = true).
+__host__ __device__ constexpr uint32_t idesc_f32acc(int M, int N, bool a_mn_major, bool b_mn_major,
+                                                    bool f16 = false) {
   return (1u << 4)                                  // D format: f32
-       | (1u << 7)                                  // A format: bf16
-       | (1u << 10)                                 // B format: bf16
+       | ((f16 ? 0u : 1u) << 7)                     // A format: 0 = f16, 1 = bf16
+       | ((f16 ? 0u : 1u) << 10)                    // B format
        | (static_cast<uint32_t>(a_mn_major) << 15)  // A major: 0 = K, 1 = MN
        | (static_cast<uint32_t>(b_mn_major) << 16)  // B major
        | (static_cast<uint32_t>(N >> 3) << 17)      // N / 8
@@ -263,6 +265,18 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn_ma
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
+}
+
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  __half2 v = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+__device__ __forceinline__ float f16_lo(uint32_t v) {
+  return __half2float(__ushort_as_half(static_cast<unsigned short>(v & 0xFFFFu)));
+}
+__device__ __forceinline__ float f16_hi(uint32_t v) {
+  return __half2float(__ushort_as_half(static_cast<unsigned short>(v >> 16)));
 }
 
 __device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }

@@ -12,7 +12,8 @@ from typing import Dict, Optional
 
 import torch
 
-from . import (Dims, OP_ATTN_BWD, OP_LAYER_BWD, OP_MLP_BWD, attn_bwd, attn_fwd, layer_bwd,
+from . import (Dims, OP_ATTN_BWD, OP_ATTN_FWD, OP_LAYER_BWD, OP_LAYER_FWD, OP_MLP_BWD,
+               attn_bwd, attn_fwd, layer_bwd,
                layer_fwd, mlp_bwd, mlp_fwd, shard_cols, shard_qkv_heads, shard_rows,
                unshard_cols, unshard_qkv_heads, workspace_size)
 
@@ -118,17 +119,20 @@ class ShardedAttention:
         self.bout = None if bout is None else bout.contiguous()
         self.device = wqkv.device
         self.ws = None
+        self.ws_fwd = None
 
     def forward(self, x, resid=None, out: Optional[Dict] = None):
         d = self.dims
         T, D = d.batch * d.seq, d.hidden
         o = out if out is not None else {
             "y": _empty((T, D), device=self.device),
-            "qkv": _empty((d.t, T, 3 * D // d.t), device=self.device),
+            "qkv": _empty((d.t, T, 3 * D // d.t), dtype=torch.float16, device=self.device),
             "o": _empty((d.t, T, D // d.t), device=self.device),
             "lse": _empty((d.batch, d.heads, d.seq), dtype=torch.float32, device=self.device)}
+        if self.ws_fwd is None:
+            self.ws_fwd = _ws(OP_ATTN_FWD, d, self.device)
         attn_fwd(d, x, self.wqkv, self.bqkv, self.wout, self.bout, resid, o["y"], o["qkv"],
-                 o["o"], o["lse"])
+                 o["o"], o["lse"], self.ws_fwd)
         self.saved = (x, o["qkv"], o["o"], o["lse"])
         return o
 
@@ -173,14 +177,16 @@ class ShardedLayer:
             "b2": None if p.get("b2") is None else p["b2"].contiguous(),
         }
         self.ws = None
+        self.ws_fwd = None
 
     def alloc_acts(self):
         d = self.dims
         T, D, F, t = d.batch * d.seq, d.hidden, d.ffn, d.t
         f32 = torch.float32
         dev = self.device
-        return {"u1": _empty((T, D), device=dev), "mean1": _empty((T,), f32, dev),
-                "rstd1": _empty((T,), f32, dev), "qkv": _empty((t, T, 3 * D // t), device=dev),
+        f16 = torch.float16
+        return {"u1": _empty((T, D), f16, dev), "mean1": _empty((T,), f32, dev),
+                "rstd1": _empty((T,), f32, dev), "qkv": _empty((t, T, 3 * D // t), f16, dev),
                 "o": _empty((t, T, D // t), device=dev),
                 "lse": _empty((d.batch, d.heads, d.seq), f32, dev),
                 "h": _empty((T, D), device=dev), "u2": _empty((T, D), device=dev),
@@ -203,7 +209,9 @@ class ShardedLayer:
         d = self.dims
         acts = acts if acts is not None else self.alloc_acts()
         y = y if y is not None else _empty((d.batch * d.seq, d.hidden), device=self.device)
-        layer_fwd(d, x, self.p, acts, y)
+        if self.ws_fwd is None:
+            self.ws_fwd = _ws(OP_LAYER_FWD, d, self.device)
+        layer_fwd(d, x, self.p, acts, y, self.ws_fwd)
         self.saved = (x, acts)
         return y, acts
 

@@ -1,0 +1,78 @@
+"""The C-ABI library loads on any host and exports every symbol include/*.h declares.
+
+No compute calls: these run without a GPU.
+"""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+import tensor_transformer_layer_column_b200 as tl
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        src = open(h).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        for m in re.finditer(r"\b(tp_[a-z0-9_]+)\s*\(", src):
+            names.add(m.group(1))
+    return names
+
+
+def test_header_declares_the_boundary():
+    want = {"tp_mlp_fwd", "tp_mlp_bwd", "tp_attn_fwd", "tp_attn_bwd", "tp_layer_fwd",
+            "tp_layer_bwd", "tp_shard_cols", "tp_shard_rows", "tp_shard_qkv_heads",
+            "tp_workspace_size", "tp_status_string"}
+    assert want <= _declared()
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built_library():
+    if not os.path.exists(tl.lib_path):
+        from tensor_transformer_layer_column_b200 import build
+        build.build()
+
+
+def test_library_exports_every_declared_symbol():
+    handle = ctypes.CDLL(tl.lib_path)
+    missing = [n for n in sorted(_declared()) if not hasattr(handle, n)]
+    assert not missing, missing
+    assert set(tl.EXPORTED_SYMBOLS) == _declared()
+
+
+def test_host_validation_without_gpu():
+    lib = tl.lib()
+    assert tl.version().startswith("tplayer-b200")
+    assert lib.tp_status_string(4) == b"TP_ERR_WORKSPACE"
+    ok = tl.Dims.of(4, 2048, 4096, 16384, 32, 128, 8)
+    assert tl.workspace_size(tl.OP_LAYER_BWD, ok) > 0
+    assert tl.workspace_size(tl.OP_MLP_FWD, ok) == 0
+    # Invalid dims give size 0 (H % t, D != H*dh, unsupported t, dh).
+    for bad in (tl.Dims.of(1, 8, 4096, 16384, 30, 128, 8), tl.Dims.of(1, 8, 4096, 16384, 32, 64, 8),
+                tl.Dims.of(1, 8, 4096, 16384, 32, 128, 3), tl.Dims.of(1, 8, 4096, 16384, 16, 256, 8)):
+        assert tl.workspace_size(tl.OP_LAYER_BWD, bad) == 0
+    # Arguments are checked before anything touches a device: these return
+    # without a GPU.
+    d = tl.Dims.of(1, 8, 256, 1024, 0, 0, 2)
+    st = lib.tp_mlp_fwd(ctypes.byref(d), None, None, None, None, None, None, None, None, None,
+                        None, 0, None)
+    assert st == 1  # TP_ERR_INVALID_ARG: null pointers
+    d3 = tl.Dims.of(1, 8, 256, 1024, 0, 0, 3)
+    st = lib.tp_mlp_fwd(ctypes.byref(d3), 16, 16, None, 16, None, None, 16, 16, 16, None, 0, None)
+    assert st == 2  # TP_ERR_UNSUPPORTED: t = 3
+    st = lib.tp_mlp_fwd(ctypes.byref(d), 24, 16, None, 16, None, None, 16, 16, 16, None, 0, None)
+    assert st == 3  # TP_ERR_MISALIGNED: x not 16-byte aligned
+    st = lib.tp_mlp_bwd(ctypes.byref(d), 16, 16, 16, 16, 16, 16, None, 16, 16, 16, None, None,
+                        None, 0, None)
+    assert st == 4  # TP_ERR_WORKSPACE
+    da = tl.Dims.of(1, 8, 512, 0, 4, 128, 8)
+    st = lib.tp_attn_fwd(ctypes.byref(da), 16, 16, None, 16, None, None, 16, 16, 16, 16, None, 0,
+                         None)
+    assert st == 1  # TP_ERR_INVALID_ARG: heads % t != 0
+    assert lib.tp_trace_begin(None, None, None, -1) == 1
+    assert lib.tp_trace_end() == 0
