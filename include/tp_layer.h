@@ -262,6 +262,24 @@ tp_status tp_layernorm_bwd(const tp_bf16* dy, const tp_bf16* x, const tp_bf16* g
                            int D, tp_bf16* dx, tp_bf16* dgamma, tp_bf16* dbeta, void* ws,
                            size_t ws_bytes, tp_stream stream);
 
+/* tp_layernorm_bwd_noalloc: the same computation as tp_layernorm_bwd, for
+ * callers that cannot allocate device memory where they run it (allocator or
+ * memory-pool callbacks, runtimes with a fixed memory budget, hot paths where
+ * cudaMalloc is forbidden).  The pages have no counterpart to it: it exists
+ * for those callers only.  It takes no workspace and allocates nothing; its
+ * scratch (the dgamma/dbeta partial sums) is a 4 MiB device array inside the
+ * library that every GPU loading the library holds until exit.  All calls on
+ * a device share that array: calls whose kernels may overlap on the GPU race
+ * and must be serialised by the caller.  The first call on each device looks
+ * up the array's device address; make it outside stream capture.  D up to
+ * 8192 (wider rows: TP_ERR_UNSUPPORTED); row count unlimited.  dgamma/dbeta
+ * sums may group rows differently from tp_layernorm_bwd (fp32, deterministic);
+ * dx is identical. */
+tp_status tp_layernorm_bwd_noalloc(const tp_bf16* dy, const tp_bf16* x, const tp_bf16* gamma,
+                                   const float* mean, const float* rstd, const tp_bf16* dres,
+                                   int rows, int D, tp_bf16* dx, tp_bf16* dgamma, tp_bf16* dbeta,
+                                   tp_stream stream);
+
 /* ------------------------------------------------------------------ launch trace
  * Measurement support (the pages describe no tracing; this exists so that a
  * bench can time individual kernels inside a longer step on their own stream).

@@ -21,7 +21,8 @@ __all__ = [
     "workspace_size", "check_error", "version", "EXPORTED_SYMBOLS",
     "shard_cols", "unshard_cols", "shard_rows", "unshard_rows", "shard_qkv_heads",
     "unshard_qkv_heads", "mlp_fwd", "mlp_bwd", "attn_fwd", "attn_bwd", "layer_fwd", "layer_bwd",
-    "layernorm_fwd", "layernorm_bwd", "layernorm_bwd_workspace_size", "LaunchTrace",
+    "layernorm_fwd", "layernorm_bwd", "layernorm_bwd_workspace_size", "layernorm_bwd_noalloc",
+    "LaunchTrace",
     "TRACE_KINDS",
 ]
 
@@ -94,6 +95,8 @@ _SIGS = {
     "tp_layernorm_bwd_workspace_size": [ctypes.c_int, ctypes.c_int],
     "tp_layernorm_bwd": [_P, _P, _P, _P, _P, _P, ctypes.c_int, ctypes.c_int, _P, _P, _P, _P,
                          ctypes.c_size_t, _P],
+    "tp_layernorm_bwd_noalloc": [_P, _P, _P, _P, _P, _P, ctypes.c_int, ctypes.c_int, _P, _P, _P,
+                                 _P],
     "tp_trace_begin": [ctypes.POINTER(ctypes.c_void_p), ctypes.POINTER(ctypes.c_int),
                        ctypes.POINTER(ctypes.c_double), ctypes.c_int],
     "tp_trace_end": [],
@@ -270,6 +273,21 @@ def layernorm_bwd(dy, x, gamma, mean, rstd, dres, rows, D, dx, dgamma, dbeta, ws
                                   _ptr(dres), rows, D, _ptr(dx), _ptr(dgamma), _ptr(dbeta), wp,
                                   wn, _stream(stream, x)), "tp_layernorm_bwd")
 
+
+
+def layernorm_bwd_noalloc(dy, x, gamma, mean, rstd, dres, rows, D, dx, dgamma, dbeta,
+                          stream=None):
+    """LayerNorm backward without a workspace (scratch is a static array in the library).
+
+    For callers that cannot allocate device memory where they run the
+    backward.  Calls on one device share the scratch: do not let two of them
+    overlap on the GPU, and make the first call on a device outside stream
+    capture.
+    """
+    _check(lib().tp_layernorm_bwd_noalloc(_ptr(dy), _ptr(x), _ptr(gamma), _ptr(mean), _ptr(rstd),
+                                          _ptr(dres), rows, D, _ptr(dx), _ptr(dgamma),
+                                          _ptr(dbeta), _stream(stream, x)),
+           "tp_layernorm_bwd_noalloc")
 
 TRACE_KINDS = ("gemm", "attn_fwd", "attn_bwd_prep", "attn_bwd_dkdv", "attn_bwd_dq", "ln_fwd",
                "ln_bwd", "ln_param", "colsum", "layout", "cast")

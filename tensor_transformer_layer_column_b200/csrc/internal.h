@@ -60,6 +60,11 @@ tp_status launch_layernorm_bwd(const uint16_t* dy, const uint16_t* x, const uint
                                long long rows, int D, uint16_t* dx, uint16_t* dg, uint16_t* db,
                                float* partial, cudaStream_t stream);
 
+tp_status launch_layernorm_bwd_blocks(const uint16_t* dy, const uint16_t* x, const uint16_t* g,
+                                      const float* mean, const float* rstd, const uint16_t* dres,
+                                      long long rows, int D, uint16_t* dx, uint16_t* dg,
+                                      uint16_t* db, int nb, float* partial, cudaStream_t stream);
+
 // Per-head causal attention over the shard-packed qkv [t][T][3Dt].
 tp_status launch_attn_fwd(const uint16_t* qkv, uint16_t* o, float* lse, int B, int S, int H,
                           int dh, int t, int causal, cudaStream_t stream);

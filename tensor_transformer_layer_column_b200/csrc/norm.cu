@@ -382,4 +382,37 @@ tp_status launch_layernorm_bwd(const uint16_t* dy, const uint16_t* x, const uint
   return cuda_status(cudaGetLastError());
 }
 
+// LayerNorm backward with a caller-chosen number of row blocks `nb` (>= 1):
+// `partial` must hold nb * 2 * D floats.  Used by the entry point whose
+// scratch is a fixed-size static array.
+tp_status launch_layernorm_bwd_blocks(const uint16_t* dy, const uint16_t* x, const uint16_t* g,
+                                      const float* mean, const float* rstd, const uint16_t* dres,
+                                      long long rows, int D, uint16_t* dx, uint16_t* dg,
+                                      uint16_t* db, int nb, float* partial, cudaStream_t stream) {
+  if (rows == 0) {
+    if (dg) cudaMemsetAsync(dg, 0, (size_t)D * 2, stream);
+    if (db) cudaMemsetAsync(db, 0, (size_t)D * 2, stream);
+    return cuda_status(cudaGetLastError());
+  }
+  if (nb < 1) return TP_ERR_INVALID_ARG;
+  const int rpb = (int)((rows + nb - 1) / nb);
+  const int per_thread = (D / 8 + LNB_THREADS - 1) / LNB_THREADS;
+  {
+    TraceScope ts(stream, TK_LN_BWD);
+    if (per_thread <= 1)
+      ln_bwd_kernel<1><<<nb, LNB_THREADS, 0, stream>>>(dy, x, g, mean, rstd, dres, rows, D, rpb, dx, partial);
+    else if (per_thread <= 2)
+      ln_bwd_kernel<2><<<nb, LNB_THREADS, 0, stream>>>(dy, x, g, mean, rstd, dres, rows, D, rpb, dx, partial);
+    else if (per_thread <= 4)
+      ln_bwd_kernel<4><<<nb, LNB_THREADS, 0, stream>>>(dy, x, g, mean, rstd, dres, rows, D, rpb, dx, partial);
+    else
+      return TP_ERR_UNSUPPORTED;
+  }
+  if (dg != nullptr || db != nullptr) {
+    TraceScope ts(stream, TK_LN_PARAM);
+    ln_param_reduce<<<(2 * D + 255) / 256, 256, 0, stream>>>(partial, nb, D, dg, db);
+  }
+  return cuda_status(cudaGetLastError());
+}
+
 }  // namespace tp
