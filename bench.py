@@ -7,6 +7,7 @@ one GPU), the workload the headline metric is quoted on.  Prints ONE JSON
 line (rank 0).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                  [--workload NAME]   (any name in synth.WORKLOADS; default the layer)
 
 N > 1 (launched with torch.distributed.run): N independent replicas, one per
 GPU, each on its own batch; no collective on the data path (weak scaling);
@@ -31,7 +32,7 @@ if ROOT not in sys.path:
 import numpy as np  # noqa: E402
 import torch  # noqa: E402
 
-from synth import Workload, make_inputs, to_f64, workload  # noqa: E402
+from synth import WORKLOADS, Workload, make_inputs, to_f64, workload  # noqa: E402
 
 METRIC = "sharded-layer TFLOP/s (bf16 fwd+bwd, 1 B200) and % of dense BF16 peak"
 WORKLOAD = "layer_fwdbwd_B4_S2048_D4096_H32_F16384_t8"
@@ -55,6 +56,21 @@ def dist_env():
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     return world, rank, local
+
+
+def max_over_ranks(ms: float, device) -> float:
+    """The slowest rank's time: every rank returns the same maximum."""
+    import torch.distributed as dist
+    if not dist.is_available() or not dist.is_initialized() or dist.get_world_size() == 1:
+        return ms
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tflops(world: int, flops_per_step_per_rank: float, ms_per_step: float) -> float:
+    """Whole-job throughput: all ranks' work over the slowest rank's time."""
+    return world * flops_per_step_per_rank / (ms_per_step * 1e-3) / 1e12
 
 
 # ---------------------------------------------------------------- CPU oracle leg
@@ -138,7 +154,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
+                 "--format=csv,noheader,nounits", "-lms", "50"],
                 stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except OSError:
             self.proc = None
@@ -179,15 +195,48 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------- our arm
-def build_layer(w: Workload, device):
-    import tensor_transformer_layer_column_b200 as tl
-    from tensor_transformer_layer_column_b200.sublayer import ShardedLayer
-    tl.lib()
-    inp = make_inputs(w)
-    g = {k: v.to(device) for k, v in inp.items()}
-    dims = tl.Dims.of(w.batch, w.seq, w.hidden, w.ffn, w.heads, w.head_dim, w.t, 1, w.ln_eps)
-    layer = ShardedLayer(dims, {k: g[k] for k in PARAMS})
-    return layer, g, inp
+class Runner:
+    """One step of a workload through the public API, on preallocated buffers."""
+
+    def __init__(self, w: Workload, device):
+        import tensor_transformer_layer_column_b200 as tl
+        from tensor_transformer_layer_column_b200.sublayer import (ShardedAttention, ShardedLayer,
+                                                                   ShardedMLP)
+        tl.lib()
+        self.w = w
+        self.host = make_inputs(w, with_dy=w.backward)
+        g = {k: v.to(device) for k, v in self.host.items()}
+        self.g = g
+        dims = tl.Dims.of(w.batch, w.seq, w.hidden, w.ffn, w.heads, w.head_dim, w.t,
+                          1 if w.causal else 0, w.ln_eps)
+        if w.kind.startswith("layer"):
+            self.mod = ShardedLayer(dims, {k: g[k] for k in PARAMS})
+            self.acts = self.mod.alloc_acts()
+            self.grads = self.mod.alloc_grads()
+        elif w.kind.startswith("attn"):
+            self.mod = ShardedAttention(dims, g["wqkv"], g["bqkv"], g["wout"], g["bout"])
+        else:
+            self.mod = ShardedMLP(dims, g["w1"], g["b1"], g["w2"], g["b2"])
+        self.y = torch.empty_like(g["x"])
+        self.dx = torch.empty_like(g["x"]) if w.backward else None
+        self.fwd_out = None
+        self.bwd_out = None
+
+    def step(self, x, dy=None):
+        w = self.w
+        if w.kind.startswith("layer"):
+            self.mod.forward(x, acts=self.acts, y=self.y)
+            self.mod.backward(dy, dx=self.dx, grads=self.grads)
+            return
+        if self.fwd_out is None:
+            self.fwd_out = self.mod.forward(x)
+            self.fwd_out["y"] = self.y
+        self.mod.forward(x, out=self.fwd_out)
+        if w.backward:
+            if self.bwd_out is None:
+                self.bwd_out = self.mod.backward(dy)
+                self.bwd_out["dx"] = self.dx
+            self.mod.backward(dy, out=self.bwd_out)
 
 
 def run_ours(args):
@@ -200,20 +249,15 @@ def run_ours(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     device = torch.device("cuda", local if world > 1 else 0)
     torch.cuda.set_device(device)
-    w = workload(WORKLOAD)
-    layer, g, host_inp = build_layer(w, device)
-    acts = layer.alloc_acts()
-    grads = layer.alloc_grads()
-    y = torch.empty_like(g["x"])
-    dx = torch.empty_like(g["x"])
+    w = workload(args.workload)
+    run = Runner(w, device)
+    g, host_inp = run.g, run.host
+    y, dx = run.y, run.dx
     stream = torch.cuda.current_stream(device)
-
-    def step(x, dy):
-        layer.forward(x, acts=acts, y=y)
-        layer.backward(dy, dx=dx, grads=grads)
+    step = run.step
 
     for _ in range(args.warmup):
-        step(g["x"], g["dy"])
+        step(g["x"], g.get("dy"))
     torch.cuda.synchronize(device)
     if tl.check_error() != 0:
         raise RuntimeError("device error word set during warm-up")
@@ -232,54 +276,54 @@ def run_ours(args):
         with trace:
             start.record(stream)
             for _ in range(args.steps):
-                step(g["x"], g["dy"])
+                step(g["x"], g.get("dy"))
             end.record(stream)
         torch.cuda.synchronize(device)
         barrier()
-    ms_total = start.elapsed_time(end)
-    if world > 1:
-        t = torch.tensor([ms_total], device=device)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms_total = float(t.item())
+    ms_total = max_over_ranks(start.elapsed_time(end), device)
     clock = clocks.summary()
     records = trace.records()
     launches = trace.count
     ms_step = ms_total / args.steps
     flops_step = w.flops()
-    value = world * flops_step / (ms_step * 1e-3) / 1e12
+    in_bytes = sum(v.numel() * v.element_size() for v in host_inp.values())
+    value = job_tflops(world, flops_step, ms_step)
 
     # ---- end to end through the public API with host buffers
-    hx = host_inp["x"].pin_memory()
-    hdy = host_inp["dy"].pin_memory()
-    hy = torch.empty_like(hx).pin_memory()
-    hdx = torch.empty_like(hx).pin_memory()
-    dxin = torch.empty_like(g["x"])
-    dyin = torch.empty_like(g["dy"])
+    e2e = None
+    if not args.no_e2e:
+        hx = host_inp["x"].pin_memory()
+        hdy = host_inp["dy"].pin_memory() if w.backward else None
+        hy = torch.empty_like(hx).pin_memory()
+        hdx = torch.empty_like(hx).pin_memory() if w.backward else None
+        xin = torch.empty_like(g["x"])
+        dyin = torch.empty_like(g["dy"]) if w.backward else None
 
-    def e2e_step():
-        dxin.copy_(hx, non_blocking=True)
-        dyin.copy_(hdy, non_blocking=True)
-        step(dxin, dyin)
-        hy.copy_(y, non_blocking=True)
-        hdx.copy_(dx, non_blocking=True)
+        def e2e_step():
+            xin.copy_(hx, non_blocking=True)
+            if w.backward:
+                dyin.copy_(hdy, non_blocking=True)
+            step(xin, dyin)
+            hy.copy_(y, non_blocking=True)
+            if w.backward:
+                hdx.copy_(dx, non_blocking=True)
 
-    for _ in range(max(1, args.warmup)):
-        e2e_step()
-    barrier()
-    torch.cuda.synchronize(device)
-    s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    s2.record(stream)
-    for _ in range(args.steps):
-        e2e_step()
-    e2.record(stream)
-    torch.cuda.synchronize(device)
-    barrier()
-    e2e_ms = s2.elapsed_time(e2)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=device)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_value = world * flops_step / (e2e_ms / args.steps * 1e-3) / 1e12
+        for _ in range(args.warmup):
+            e2e_step()
+        barrier()
+        torch.cuda.synchronize(device)
+        s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s2.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        e2.record(stream)
+        torch.cuda.synchronize(device)
+        barrier()
+        e2e_ms = max_over_ranks(s2.elapsed_time(e2), device)
+        nb = 2 if w.backward else 1
+        e2e = {"value": job_tflops(world, flops_step, e2e_ms / args.steps),
+               "unit": "TFLOP/s", "h2d_bytes_per_step": nb * hx.numel() * 2,
+               "d2h_bytes_per_step": nb * hy.numel() * 2}
     if tl.check_error() != 0:
         raise RuntimeError("device error word set during the timed region")
 
@@ -309,7 +353,7 @@ def run_ours(args):
 
     # ---- CPU oracle baseline (rank 0, N = 1 only), after the GPU timing
     cpu = None
-    if world == 1 and not args.no_cpu_baseline:
+    if world == 1 and not args.no_cpu_baseline and args.workload == WORKLOAD:
         oseq = 512
         cv, csec, cs = time_oracle(oseq, 2)
         cpu = {"value": cv, "unit": "TFLOP/s", "cores": cores_used(), "kind": "oracle",
@@ -323,18 +367,18 @@ def run_ours(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": WORKLOAD, "batch": w.batch, "seq": w.seq,
+            "config": {"workload": w.name, "batch": w.batch, "seq": w.seq,
                        "hidden": w.hidden, "ffn": w.ffn, "heads": w.heads,
-                       "head_dim": w.head_dim, "t": w.t, "causal": True,
+                       "head_dim": w.head_dim, "t": w.t, "causal": w.causal,
                        "flop_per_step": flops_step,
-                       "l2": "inputs larger than L2 (weights 384 MiB, activations > 1 GiB per step)",
+                       "l2": (f"inputs larger than L2: {in_bytes / 2**20:.0f} MiB of inputs per "
+                              "step vs 120 MiB of L2, no flush" if in_bytes > 126e6
+                              else "L2 not flushed: inputs smaller than L2"),
                        "parallelism": f"t{w.t} shards on each GPU; {world} independent replica(s)"},
             "pct_dense_bf16_peak": 100.0 * value / world / NOMINAL_BF16_TFLOPS,
             "pct_measured_bf16_peak": 100.0 * value / world / peaks["bf16_tflops"],
             "peak_source": peak_src,
-            "e2e": {"value": e2e_value, "unit": "TFLOP/s",
-                    "h2d_bytes_per_step": hx.numel() * 2 + hdy.numel() * 2,
-                    "d2h_bytes_per_step": hy.numel() * 2 + hdx.numel() * 2},
+            "e2e": e2e,
             "gpu_launches": launches,
             "roofline": roofline,
             "kernels": breakdown,
@@ -352,8 +396,11 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", default=WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true",
                     help="skip the timed CPU oracle sample (for profiler runs)")
+    ap.add_argument("--no-e2e", action="store_true",
+                    help="skip the host-buffer end-to-end leg (for profiler runs)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
