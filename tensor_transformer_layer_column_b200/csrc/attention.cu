@@ -52,14 +52,15 @@ constexpr float kLn2 = 0.6931471805599453f;
 
 struct AttnArgs {
   int B, S, H, Ht, Dt, t;
+  int S_pad;            // bwd: row length of lse2 / dvec per (batch, head), a multiple of 128
   int causal;
   long long T;
   float scale_log2;     // log2(e) / sqrt(dh)
   float inv_sqrt_dh;
   uint16_t* out;        // fwd: o_save [t][T][Dt]; bwd: dqkv [t][T][3Dt]
   float* lse;           // fwd: lse [B][H][S]
-  const float* lse2;    // bwd: lse * log2(e), [B][H][S]
-  const float* dvec;    // bwd: rowsum(dO * O), [B][H][S]
+  const float* lse2;    // bwd: lse * log2(e), [B][H][S_pad]; +inf past S
+  const float* dvec;    // bwd: rowsum(dO * O), [B][H][S_pad]; 0 past S
   unsigned int* err;
 };
 
@@ -346,15 +347,23 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_qkv, const AttnArgs p) {
 // =====================================================================================
 // Backward
 // =====================================================================================
+// Dv = rowsum(dO * O) and lse2 = lse * log2(e) for every (batch, head, query),
+// written with rows padded to S_pad: padded queries get lse2 = +inf, Dv = 0.
 __global__ void attn_bwd_prep_kernel(const uint16_t* __restrict__ o, const uint16_t* __restrict__ dout,
                                      const float* __restrict__ lse, float* __restrict__ dvec,
-                                     float* __restrict__ lse2, int B, int S, int H, int Ht,
-                                     int dh, int Dt, long long T) {
+                                     float* __restrict__ lse2, int B, int S, int S_pad, int H,
+                                     int Ht, int dh, int Dt, long long T) {
   const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  if (idx >= (long long)B * H * S) return;
-  const int s = (int)(idx % S);
-  const int h = (int)((idx / S) % H);
-  const int b = (int)(idx / ((long long)S * H));
+  if (idx >= (long long)B * H * S_pad) return;
+  const int s = (int)(idx % S_pad);
+  const long long bh = idx / S_pad;
+  if (s >= S) {
+    dvec[idx] = 0.f;
+    lse2[idx] = INFINITY;
+    return;
+  }
+  const int h = (int)(bh % H);
+  const int b = (int)(bh / H);
   const int shard = h / Ht, hl = h - shard * Ht;
   const long long off = (long long)shard * T * Dt + ((long long)b * S + s) * Dt + hl * dh;
   float acc = 0.f;
@@ -367,20 +376,27 @@ __global__ void attn_bwd_prep_kernel(const uint16_t* __restrict__ o, const uint1
       acc += bf16_lo(wa[k]) * f16_lo(wg[k]) + bf16_hi(wa[k]) * f16_hi(wg[k]);
   }
   dvec[idx] = acc;
-  lse2[idx] = lse[idx] * kLog2e;
+  lse2[idx] = lse[bh * S + s] * kLog2e;
 }
 
 // ---------------------------------------------------------------- dK / dV
+// Per 128-key block, walk 64-query blocks.  Double-buffered S^T/dP^T in TMEM
+// and P^T/dS^T tiles in shared memory: the MMAs of block k+1 (S^T, dP^T) and
+// the dV/dK MMAs of block k-1 run while the compute warps work on block k.
 template <int DH>
 struct DkdvCfg {
   static constexpr int BK = 128, BQ = 64, CH = DH / 64;
   static constexpr int K_BYTES = BK * DH * 2;              // K and V tiles, each
   static constexpr int Q_BYTES = BQ * DH * 2;              // q and dO tiles, each (per stage)
+  static constexpr int VEC_BYTES = BQ * 4;                 // lse2 / dvec slice of one stage
+  static constexpr int STAGES = 3;                         // q / dO / lse2 / dvec ring depth
+  static constexpr int STAGE_BYTES = 2 * Q_BYTES;
   static constexpr int OFF_K = 0, OFF_V = K_BYTES;
-  static constexpr int OFF_ST = 2 * K_BYTES;               // stage s: q at +s*2*Q, dO at +Q
-  static constexpr int OFF_PT = OFF_ST + 4 * Q_BYTES;      // P^T  [128 keys][64 queries]
-  static constexpr int OFF_DST = OFF_PT + BK * BQ * 2;     // dS^T [128 keys][64 queries]
-  static constexpr int OFF_BAR = OFF_DST + BK * BQ * 2;
+  static constexpr int OFF_ST = 2 * K_BYTES;               // stage s: q | dO
+  static constexpr int T_BYTES = BK * BQ * 2;              // one P^T or dS^T tile
+  static constexpr int OFF_PT = OFF_ST + STAGES * STAGE_BYTES;  // buffer b: P^T at +2b*T, dS^T at +(2b+1)*T
+  static constexpr int OFF_VEC = OFF_PT + 4 * T_BYTES;     // stage s: lse2 at +2s*VEC, dvec at +(2s+1)*VEC
+  static constexpr int OFF_BAR = OFF_VEC + STAGES * 2 * VEC_BYTES;
   static constexpr int RAW = OFF_BAR + 256 + 1024;
   static constexpr int SMEM = RAW > 120 * 1024 ? RAW : 120 * 1024;
 };
@@ -396,14 +412,14 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_kv128,
   uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   uint64_t* kv_full = bars + 0;
-  uint64_t* qd_full = bars + 1;    // [2]
-  uint64_t* qd_empty = bars + 3;   // [2]
-  uint64_t* s_full = bars + 5;
-  uint64_t* s_free = bars + 6;
-  uint64_t* p_full = bars + 7;
-  uint64_t* mm2_done = bars + 8;
-  uint64_t* drain = bars + 9;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 10);
+  uint64_t* qd_full = bars + 1;    // [3] per stage
+  uint64_t* qd_empty = bars + 4;   // [3]
+  uint64_t* s_full = bars + 7;     // [2] per TMEM buffer
+  uint64_t* s_free = bars + 9;     // [2]
+  uint64_t* p_full = bars + 11;    // [2] per P^T/dS^T buffer
+  uint64_t* mm2_done = bars + 13;  // [2]
+  uint64_t* drain = bars + 15;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -414,18 +430,21 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_kv128,
   const int i0 = p.causal ? k0 / C::BQ : 0;
   const int nsteps = nqb - i0;
   const int colq = hl * DH, colk = p.Dt + hl * DH, colv = 2 * p.Dt + hl * DH, cold = hl * DH;
+  const long long hrow = ((long long)b * p.H + h) * p.S_pad;
   const Ctl ctl{abort_flag, p.err};
 
   if (threadIdx.x == 0) {
     mbar_init(kv_full, 1);
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < C::STAGES; ++i) {
       mbar_init(&qd_full[i], 1);
       mbar_init(&qd_empty[i], 1);
     }
-    mbar_init(s_full, 1);
-    mbar_init(s_free, 128);
-    mbar_init(p_full, 128);
-    mbar_init(mm2_done, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&s_free[i], 128);
+      mbar_init(&p_full[i], 128);
+      mbar_init(&mm2_done[i], 1);
+    }
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -438,7 +457,8 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_kv128,
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t t_s = tmem, t_dp = tmem + 64, t_dv = tmem + 128, t_dk = tmem + 128 + DH;
+  // buffer j: S^T at 128j, dP^T at 128j + 64; dV at 256, dK at 384 (DH <= 128)
+  const uint32_t t_dv = tmem + 256, t_dk = tmem + 256 + DH;
 
   if (warp == 0) {
     if (lane == 0) {
@@ -449,53 +469,67 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_kv128,
       }
       int k = 0;
       for (; k < nsteps; ++k) {
-        const int st = k & 1;
-        const uint32_t u = k >> 1;
+        const int st = k % C::STAGES;
+        const uint32_t u = k / C::STAGES;
         if (!wait_bar(&qd_empty[st], (u & 1) ^ 1, ctl, ERR_ATTN_DKDV_WAIT)) break;
-        uint8_t* sq = smem + C::OFF_ST + st * 2 * C::Q_BYTES;
+        uint8_t* sq = smem + C::OFF_ST + st * C::STAGE_BYTES;
         uint8_t* sd = sq + C::Q_BYTES;
+        uint8_t* sv = smem + C::OFF_VEC + st * 2 * C::VEC_BYTES;
         const int qs = (i0 + k) * C::BQ;
-        mbar_arrive_expect_tx(&qd_full[st], 2 * C::Q_BYTES);
+        mbar_arrive_expect_tx(&qd_full[st], 2 * C::Q_BYTES + 2 * C::VEC_BYTES);
         for (int c = 0; c < C::CH; ++c) {
           tma_load_4d(sq + c * C::BQ * 128, &tm_q64, &qd_full[st], colq + 64 * c, qs, b, shard);
           tma_load_4d(sd + c * C::BQ * 128, &tm_do64, &qd_full[st], cold + 64 * c, qs, b, shard);
         }
+        bulk_load(sv, p.lse2 + hrow + qs, C::VEC_BYTES, &qd_full[st]);
+        bulk_load(sv + C::VEC_BYTES, p.dvec + hrow + qs, C::VEC_BYTES, &qd_full[st]);
       }
       mbar_wait(kv_full, 0, 200000000ull);
-      for (int i = k - 1; i >= 0 && i >= k - 2; --i) mbar_wait(&qd_full[i & 1], (i >> 1) & 1, 200000000ull);
+      for (int i = k - 1; i >= 0 && i >= k - C::STAGES; --i)
+        mbar_wait(&qd_full[i % C::STAGES], (i / C::STAGES) & 1, 200000000ull);
     }
   } else if (warp == 1) {
     if (lane == 0) {
       constexpr uint32_t id_s = idesc_f32acc(128, C::BQ, false, false, true);
       constexpr uint32_t id_acc = idesc_f32acc(128, DH, false, true, true);
       const uint32_t sk = smem_u32(smem + C::OFF_K), sv = smem_u32(smem + C::OFF_V);
-      const uint32_t spt = smem_u32(smem + C::OFF_PT), sdst = smem_u32(smem + C::OFF_DST);
+      const uint32_t spt = smem_u32(smem + C::OFF_PT);
       bool ok = wait_bar(kv_full, 0, ctl, ERR_ATTN_DKDV_WAIT);
-      for (int k = 0; ok && k < nsteps; ++k) {
-        const int st = k & 1;
-        const uint32_t u = k >> 1;
-        if (!wait_bar(&qd_full[st], u & 1, ctl, ERR_ATTN_DKDV_WAIT)) break;
-        if (!wait_bar(s_free, (k & 1) ^ 1, ctl, ERR_ATTN_DKDV_WAIT)) break;
-        tc_fence_after();
-        const uint32_t sq = smem_u32(smem + C::OFF_ST + st * 2 * C::Q_BYTES);
-        const uint32_t sd = sq + C::Q_BYTES;
+      for (int k = 0; ok && k <= nsteps; ++k) {
+        if (k < nsteps) {
+          const int bf = k & 1, st = k % C::STAGES;
+          const uint32_t u = k >> 1;
+          if (!wait_bar(&qd_full[st], (k / C::STAGES) & 1, ctl, ERR_ATTN_DKDV_WAIT)) break;
+          if (!wait_bar(&s_free[bf], (u & 1) ^ 1, ctl, ERR_ATTN_DKDV_WAIT)) break;
+          tc_fence_after();
+          const uint32_t sq = smem_u32(smem + C::OFF_ST + st * C::STAGE_BYTES);
+          const uint32_t sd = sq + C::Q_BYTES;
 #pragma unroll
-        for (int kk = 0; kk < DH / 16; ++kk) {
-          tc_mma_f16(t_s, kmajor_desc(sk, C::BK, kk), kmajor_desc(sq, C::BQ, kk), id_s, kk > 0);
-          tc_mma_f16(t_dp, kmajor_desc(sv, C::BK, kk), kmajor_desc(sd, C::BQ, kk), id_s, kk > 0);
+          for (int kk = 0; kk < DH / 16; ++kk) {
+            tc_mma_f16(tmem + bf * 128, kmajor_desc(sk, C::BK, kk), kmajor_desc(sq, C::BQ, kk), id_s,
+                       kk > 0);
+            tc_mma_f16(tmem + bf * 128 + 64, kmajor_desc(sv, C::BK, kk), kmajor_desc(sd, C::BQ, kk),
+                       id_s, kk > 0);
+          }
+          tc_commit(&s_full[bf]);
         }
-        tc_commit(s_full);
-        if (!wait_bar(p_full, k & 1, ctl, ERR_ATTN_DKDV_WAIT)) break;
-        tc_fence_after();
+        if (k > 0) {
+          const int j = k - 1, bj = j & 1, sj = j % C::STAGES;
+          if (!wait_bar(&p_full[bj], (j >> 1) & 1, ctl, ERR_ATTN_DKDV_WAIT)) break;
+          tc_fence_after();
+          const uint32_t sq = smem_u32(smem + C::OFF_ST + sj * C::STAGE_BYTES);
+          const uint32_t sd = sq + C::Q_BYTES;
+          const uint32_t pt = spt + 2 * bj * C::T_BYTES, dst = pt + C::T_BYTES;
 #pragma unroll
-        for (int kk = 0; kk < C::BQ / 16; ++kk) {
-          tc_mma_f16(t_dv, kmajor_desc(spt, C::BK, kk), mnmajor_desc(sd, C::BQ, kk), id_acc,
-                     (k | kk) != 0);
-          tc_mma_f16(t_dk, kmajor_desc(sdst, C::BK, kk), mnmajor_desc(sq, C::BQ, kk), id_acc,
-                     (k | kk) != 0);
+          for (int kk = 0; kk < C::BQ / 16; ++kk) {
+            tc_mma_f16(t_dv, kmajor_desc(pt, C::BK, kk), mnmajor_desc(sd, C::BQ, kk), id_acc,
+                       (j | kk) != 0);
+            tc_mma_f16(t_dk, kmajor_desc(dst, C::BK, kk), mnmajor_desc(sq, C::BQ, kk), id_acc,
+                       (j | kk) != 0);
+          }
+          tc_commit(&mm2_done[bj]);
+          tc_commit(&qd_empty[sj]);
         }
-        tc_commit(mm2_done);
-        tc_commit(&qd_empty[st]);
       }
       tc_commit(drain);
       mbar_wait(drain, 0, 200000000ull);
@@ -505,46 +539,49 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_kv128,
     const int r = quad * 32 + lane;
     const int kpos = k0 + r;
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-    uint8_t* spt = smem + C::OFF_PT;
-    uint8_t* sdst = smem + C::OFF_DST;
-    const long long hrow = ((long long)b * p.H + h) * p.S;
     bool ok = true;
     for (int k = 0; k < nsteps; ++k) {
+      const int bf = k & 1;
+      const uint32_t u = k >> 1;
       const int qs = (i0 + k) * C::BQ;
-      if (!__all_sync(0xffffffffu, wait_bar(s_full, k & 1, ctl, ERR_ATTN_DKDV_WAIT))) { ok = false; break; }
-      if (k > 0 && !__all_sync(0xffffffffu, wait_bar(mm2_done, (k - 1) & 1, ctl, ERR_ATTN_DKDV_WAIT))) { ok = false; break; }
+      if (!__all_sync(0xffffffffu, wait_bar(&s_full[bf], u & 1, ctl, ERR_ATTN_DKDV_WAIT))) { ok = false; break; }
+      // The P^T/dS^T buffer bf was last read by the dV/dK MMAs of block k-2.
+      if (k >= 2 && !__all_sync(0xffffffffu, wait_bar(&mm2_done[bf], (u - 1) & 1, ctl, ERR_ATTN_DKDV_WAIT))) { ok = false; break; }
       tc_fence_after();
+      const float* vl = reinterpret_cast<const float*>(smem + C::OFF_VEC + (k % C::STAGES) * 2 * C::VEC_BYTES);
+      const float* vd = vl + C::BQ;
+      uint8_t* pt = smem + C::OFF_PT + 2 * bf * C::T_BYTES;
+      uint8_t* dst = pt + C::T_BYTES;
 #pragma unroll 1
       for (int c = 0; c < C::BQ / 32; ++c) {
         uint32_t rs[32], rd[32];
-        tmem_ld32(t_s + lane_off + c * 32, rs);
-        tmem_ld32(t_dp + lane_off + c * 32, rd);
+        tmem_ld32(tmem + bf * 128 + lane_off + c * 32, rs);
+        tmem_ld32(tmem + bf * 128 + 64 + lane_off + c * 32, rd);
         tc_wait_ld();
         float pv[32], dsv[32];
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
-          const int q = qs + c * 32 + e;
-          float pe = 0.f, de = 0.f;
-          if (q < p.S && !(p.causal && kpos > q)) {
-            pe = fast_exp2(__uint_as_float(rs[e]) * p.scale_log2 - __ldg(p.lse2 + hrow + q));
-            de = pe * (__uint_as_float(rd[e]) - __ldg(p.dvec + hrow + q));
-          }
+          const int qi = c * 32 + e;
+          // Padded queries carry lse2 = +inf and dvec = 0, so they give 0.
+          float pe = fast_exp2(__uint_as_float(rs[e]) * p.scale_log2 - vl[qi]);
+          if (p.causal && kpos > qs + qi) pe = 0.f;
           pv[e] = pe;
-          dsv[e] = de;
+          dsv[e] = pe * (__uint_as_float(rd[e]) - vd[qi]);
         }
 #pragma unroll
         for (int g = 0; g < 4; ++g) {
           const uint32_t off = sw128_offset(C::BK, r, c * 32 + g * 8);
-          *reinterpret_cast<uint4*>(spt + off) = pack8_f16(&pv[g * 8]);
-          *reinterpret_cast<uint4*>(sdst + off) = pack8_f16(&dsv[g * 8]);
+          *reinterpret_cast<uint4*>(pt + off) = pack8_f16(&pv[g * 8]);
+          *reinterpret_cast<uint4*>(dst + off) = pack8_f16(&dsv[g * 8]);
         }
       }
       tc_fence_before();
-      mbar_arrive(s_free);
+      mbar_arrive(&s_free[bf]);
       fence_proxy_async_smem();
-      mbar_arrive(p_full);
+      mbar_arrive(&p_full[bf]);
     }
-    if (ok && __all_sync(0xffffffffu, wait_bar(mm2_done, (nsteps - 1) & 1, ctl, ERR_ATTN_DKDV_WAIT))) {
+    const int last = nsteps - 1;
+    if (ok && __all_sync(0xffffffffu, wait_bar(&mm2_done[last & 1], (last >> 1) & 1, ctl, ERR_ATTN_DKDV_WAIT))) {
       tc_fence_after();
       const bool valid = kpos < p.S;
       const long long w3 = 3LL * p.Dt;
@@ -583,15 +620,18 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_kv128,
 }
 
 // ---------------------------------------------------------------- dQ
+// Per 128-query block, walk 64-key blocks, with the same double buffering.
 template <int DH>
 struct DqCfg {
   static constexpr int BQ = 128, BK = 64, CH = DH / 64;
   static constexpr int Q_BYTES = BQ * DH * 2;                // q and dO tiles, each
   static constexpr int K_BYTES = BK * DH * 2;                // K and V tiles, each (per stage)
   static constexpr int OFF_Q = 0, OFF_DO = Q_BYTES;
+  static constexpr int STAGES = 3;                           // K / V ring depth
   static constexpr int OFF_ST = 2 * Q_BYTES;                 // stage s: k at +s*2*K, v at +K
-  static constexpr int OFF_DS = OFF_ST + 4 * K_BYTES;        // dS [128 queries][64 keys]
-  static constexpr int OFF_BAR = OFF_DS + BQ * BK * 2;
+  static constexpr int DS_BYTES = BQ * BK * 2;
+  static constexpr int OFF_DS = OFF_ST + STAGES * 2 * K_BYTES;  // buffer b: dS at +b*DS
+  static constexpr int OFF_BAR = OFF_DS + 2 * DS_BYTES;
   static constexpr int RAW = OFF_BAR + 256 + 1024;
   static constexpr int SMEM = RAW > 120 * 1024 ? RAW : 120 * 1024;
 };
@@ -607,14 +647,14 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q128,
   uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   uint64_t* q_full = bars + 0;
-  uint64_t* kv_full = bars + 1;    // [2]
-  uint64_t* kv_empty = bars + 3;   // [2]
-  uint64_t* s_full = bars + 5;
-  uint64_t* s_free = bars + 6;
-  uint64_t* p_full = bars + 7;
-  uint64_t* mm2_done = bars + 8;
-  uint64_t* drain = bars + 9;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 10);
+  uint64_t* kv_full = bars + 1;    // [3] per stage
+  uint64_t* kv_empty = bars + 4;   // [3]
+  uint64_t* s_full = bars + 7;     // [2] per TMEM buffer
+  uint64_t* s_free = bars + 9;     // [2]
+  uint64_t* p_full = bars + 11;    // [2] per dS buffer
+  uint64_t* mm2_done = bars + 13;  // [2]
+  uint64_t* drain = bars + 15;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -630,27 +670,29 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q128,
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < C::STAGES; ++i) {
       mbar_init(&kv_full[i], 1);
       mbar_init(&kv_empty[i], 1);
     }
-    mbar_init(s_full, 1);
-    mbar_init(s_free, 128);
-    mbar_init(p_full, 128);
-    mbar_init(mm2_done, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&s_free[i], 128);
+      mbar_init(&p_full[i], 128);
+      mbar_init(&mm2_done[i], 1);
+    }
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, 256);
+    tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t t_s = tmem, t_dp = tmem + 64, t_dq = tmem + 128;
+  const uint32_t t_dq = tmem + 256;   // buffer j: S at 128j, dP at 128j + 64
 
   if (warp == 0) {
     if (lane == 0) {
@@ -661,8 +703,8 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q128,
       }
       int k = 0;
       for (; k < nsteps; ++k) {
-        const int st = k & 1;
-        const uint32_t u = k >> 1;
+        const int st = k % C::STAGES;
+        const uint32_t u = k / C::STAGES;
         if (!wait_bar(&kv_empty[st], (u & 1) ^ 1, ctl, ERR_ATTN_DQ_WAIT)) break;
         uint8_t* sk = smem + C::OFF_ST + st * 2 * C::K_BYTES;
         uint8_t* sv = sk + C::K_BYTES;
@@ -673,7 +715,8 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q128,
         }
       }
       mbar_wait(q_full, 0, 200000000ull);
-      for (int i = k - 1; i >= 0 && i >= k - 2; --i) mbar_wait(&kv_full[i & 1], (i >> 1) & 1, 200000000ull);
+      for (int i = k - 1; i >= 0 && i >= k - C::STAGES; --i)
+        mbar_wait(&kv_full[i % C::STAGES], (i / C::STAGES) & 1, 200000000ull);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -682,28 +725,36 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q128,
       const uint32_t sq = smem_u32(smem + C::OFF_Q), sd = smem_u32(smem + C::OFF_DO);
       const uint32_t sds = smem_u32(smem + C::OFF_DS);
       bool ok = wait_bar(q_full, 0, ctl, ERR_ATTN_DQ_WAIT);
-      for (int k = 0; ok && k < nsteps; ++k) {
-        const int st = k & 1;
-        const uint32_t u = k >> 1;
-        if (!wait_bar(&kv_full[st], u & 1, ctl, ERR_ATTN_DQ_WAIT)) break;
-        if (!wait_bar(s_free, (k & 1) ^ 1, ctl, ERR_ATTN_DQ_WAIT)) break;
-        tc_fence_after();
-        const uint32_t sk = smem_u32(smem + C::OFF_ST + st * 2 * C::K_BYTES);
-        const uint32_t sv = sk + C::K_BYTES;
+      for (int k = 0; ok && k <= nsteps; ++k) {
+        if (k < nsteps) {
+          const int bf = k & 1, st = k % C::STAGES;
+          const uint32_t u = k >> 1;
+          if (!wait_bar(&kv_full[st], (k / C::STAGES) & 1, ctl, ERR_ATTN_DQ_WAIT)) break;
+          if (!wait_bar(&s_free[bf], (u & 1) ^ 1, ctl, ERR_ATTN_DQ_WAIT)) break;
+          tc_fence_after();
+          const uint32_t sk = smem_u32(smem + C::OFF_ST + st * 2 * C::K_BYTES);
+          const uint32_t sv = sk + C::K_BYTES;
 #pragma unroll
-        for (int kk = 0; kk < DH / 16; ++kk) {
-          tc_mma_f16(t_s, kmajor_desc(sq, C::BQ, kk), kmajor_desc(sk, C::BK, kk), id_s, kk > 0);
-          tc_mma_f16(t_dp, kmajor_desc(sd, C::BQ, kk), kmajor_desc(sv, C::BK, kk), id_s, kk > 0);
+          for (int kk = 0; kk < DH / 16; ++kk) {
+            tc_mma_f16(tmem + bf * 128, kmajor_desc(sq, C::BQ, kk), kmajor_desc(sk, C::BK, kk), id_s,
+                       kk > 0);
+            tc_mma_f16(tmem + bf * 128 + 64, kmajor_desc(sd, C::BQ, kk), kmajor_desc(sv, C::BK, kk),
+                       id_s, kk > 0);
+          }
+          tc_commit(&s_full[bf]);
         }
-        tc_commit(s_full);
-        if (!wait_bar(p_full, k & 1, ctl, ERR_ATTN_DQ_WAIT)) break;
-        tc_fence_after();
+        if (k > 0) {
+          const int j = k - 1, bj = j & 1, sj = j % C::STAGES;
+          if (!wait_bar(&p_full[bj], (j >> 1) & 1, ctl, ERR_ATTN_DQ_WAIT)) break;
+          tc_fence_after();
+          const uint32_t sk = smem_u32(smem + C::OFF_ST + sj * 2 * C::K_BYTES);
 #pragma unroll
-        for (int kk = 0; kk < C::BK / 16; ++kk)
-          tc_mma_f16(t_dq, kmajor_desc(sds, C::BQ, kk), mnmajor_desc(sk, C::BK, kk), id_acc,
-                     (k | kk) != 0);
-        tc_commit(mm2_done);
-        tc_commit(&kv_empty[st]);
+          for (int kk = 0; kk < C::BK / 16; ++kk)
+            tc_mma_f16(t_dq, kmajor_desc(sds + bj * C::DS_BYTES, C::BQ, kk),
+                       mnmajor_desc(sk, C::BK, kk), id_acc, (j | kk) != 0);
+          tc_commit(&mm2_done[bj]);
+          tc_commit(&kv_empty[sj]);
+        }
       }
       tc_commit(drain);
       mbar_wait(drain, 0, 200000000ull);
@@ -713,44 +764,45 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q128,
     const int r = quad * 32 + lane;
     const int q = q0 + r;
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-    uint8_t* sds = smem + C::OFF_DS;
-    const long long hrow = ((long long)b * p.H + h) * p.S;
+    const long long hrow = ((long long)b * p.H + h) * p.S_pad;
     const bool qvalid = q < p.S;
-    const float l2 = qvalid ? p.lse2[hrow + q] : 0.f;
-    const float dv = qvalid ? p.dvec[hrow + q] : 0.f;
+    const float l2 = p.lse2[hrow + q];     // padded rows: +inf, so P = 0
+    const float dv = p.dvec[hrow + q];
     bool ok = true;
     for (int k = 0; k < nsteps; ++k) {
+      const int bf = k & 1;
+      const uint32_t u = k >> 1;
       const int ks = k * C::BK;
-      if (!__all_sync(0xffffffffu, wait_bar(s_full, k & 1, ctl, ERR_ATTN_DQ_WAIT))) { ok = false; break; }
-      if (k > 0 && !__all_sync(0xffffffffu, wait_bar(mm2_done, (k - 1) & 1, ctl, ERR_ATTN_DQ_WAIT))) { ok = false; break; }
+      if (!__all_sync(0xffffffffu, wait_bar(&s_full[bf], u & 1, ctl, ERR_ATTN_DQ_WAIT))) { ok = false; break; }
+      if (k >= 2 && !__all_sync(0xffffffffu, wait_bar(&mm2_done[bf], (u - 1) & 1, ctl, ERR_ATTN_DQ_WAIT))) { ok = false; break; }
       tc_fence_after();
+      uint8_t* sds = smem + C::OFF_DS + bf * C::DS_BYTES;
 #pragma unroll 1
       for (int c = 0; c < C::BK / 32; ++c) {
         uint32_t rs[32], rd[32];
-        tmem_ld32(t_s + lane_off + c * 32, rs);
-        tmem_ld32(t_dp + lane_off + c * 32, rd);
+        tmem_ld32(tmem + bf * 128 + lane_off + c * 32, rs);
+        tmem_ld32(tmem + bf * 128 + 64 + lane_off + c * 32, rd);
         tc_wait_ld();
         float dsv[32];
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
           const int kpos = ks + c * 32 + e;
-          float de = 0.f;
-          if (qvalid && kpos < p.S && !(p.causal && kpos > q)) {
-            const float pe = fast_exp2(__uint_as_float(rs[e]) * p.scale_log2 - l2);
-            de = pe * (__uint_as_float(rd[e]) - dv);
-          }
-          dsv[e] = de;
+          float pe = fast_exp2(__uint_as_float(rs[e]) * p.scale_log2 - l2);
+          if ((p.causal && kpos > q) || kpos >= p.S) pe = 0.f;
+          dsv[e] = pe * (__uint_as_float(rd[e]) - dv);
         }
 #pragma unroll
         for (int g = 0; g < 4; ++g)
           *reinterpret_cast<uint4*>(sds + sw128_offset(C::BQ, r, c * 32 + g * 8)) = pack8_f16(&dsv[g * 8]);
       }
       tc_fence_before();
-      mbar_arrive(s_free);
+      mbar_arrive(&s_free[bf]);
       fence_proxy_async_smem();
-      mbar_arrive(p_full);
+      mbar_arrive(&p_full[bf]);
     }
-    if (ok && nsteps > 0 && __all_sync(0xffffffffu, wait_bar(mm2_done, (nsteps - 1) & 1, ctl, ERR_ATTN_DQ_WAIT))) {
+    const int last = nsteps - 1;
+    if (ok && nsteps > 0 &&
+        __all_sync(0xffffffffu, wait_bar(&mm2_done[last & 1], (last >> 1) & 1, ctl, ERR_ATTN_DQ_WAIT))) {
       tc_fence_after();
       const long long w3 = 3LL * p.Dt;
       uint16_t* row = p.out + (long long)shard * p.T * w3 + ((long long)b * p.S + q) * w3 + colq;
@@ -779,7 +831,7 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q128,
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 256);
+    tmem_dealloc(tmem, 512);
   }
 }
 
@@ -844,6 +896,7 @@ AttnArgs make_args(int B, int S, int H, int dh, int t, int causal) {
   AttnArgs a{};
   a.B = B; a.S = S; a.H = H; a.Ht = H / t; a.Dt = (H / t) * dh; a.t = t;
   a.causal = causal;
+  a.S_pad = (S + 127) / 128 * 128;
   a.T = (long long)B * S;
   a.scale_log2 = kLog2e / sqrtf((float)dh);
   a.inv_sqrt_dh = 1.0f / sqrtf((float)dh);
@@ -873,12 +926,12 @@ template <int DH>
 tp_status bwd_launch(const uint16_t* qkv, const uint16_t* o, const float* lse, const uint16_t* dout,
                      uint16_t* dqkv, const AttnArgs& a, void* scratch, cudaStream_t st) {
   float* dvec = static_cast<float*>(scratch);
-  float* lse2 = dvec + align_up((size_t)a.B * a.H * a.S, 64);
-  const long long n = (long long)a.B * a.H * a.S;
+  float* lse2 = dvec + (size_t)a.B * a.H * a.S_pad;
+  const long long n = (long long)a.B * a.H * a.S_pad;
   {
     TraceScope ts(st, TK_ATTN_BWD_PREP);
-    attn_bwd_prep_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(o, dout, lse, dvec, lse2, a.B,
-                                                                       a.S, a.H, a.Ht, DH, a.Dt, a.T);
+    attn_bwd_prep_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(
+        o, dout, lse, dvec, lse2, a.B, a.S, a.S_pad, a.H, a.Ht, DH, a.Dt, a.T);
   }
   if (cudaGetLastError() != cudaSuccess) return TP_ERR_CUDA;
   AttnArgs p = a;
@@ -923,7 +976,8 @@ tp_status launch_attn_fwd(const uint16_t* qkv, uint16_t* o, float* lse, int B, i
 
 size_t attn_bwd_scratch_bytes(int B, int S, int H, int dh) {
   (void)dh;
-  return 2 * align_up((size_t)B * H * S, 64) * sizeof(float);
+  const size_t s_pad = ((size_t)S + 127) / 128 * 128;
+  return 2 * (size_t)B * H * s_pad * sizeof(float);
 }
 
 tp_status launch_attn_bwd(const uint16_t* qkv, const uint16_t* o, const float* lse,
