@@ -61,22 +61,63 @@ tp_status launch_inst(const CUtensorMap& ta, const CUtensorMap& tb, const GemmAr
   return cuda_status(cudaGetLastError());
 }
 
+// CTA-pair kernel: clusters of 2 CTAs, one 256 x 256 tile per cluster at a time.
+template <bool A_MN, bool B_MN>
+tp_status launch_pair(const CUtensorMap& ta, const CUtensorMap& tb, const GemmArgs& args,
+                      double flops, cudaStream_t stream) {
+  static int max_clusters[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  auto kern = gemm_pair_sm100<A_MN, B_MN>;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.blockDim = dim3(GEMM_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = GP_SMEM_BYTES;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (dev < 0 || dev >= 64) return TP_ERR_CUDA;
+  if (max_clusters[dev] == 0) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, GP_SMEM_BYTES) !=
+        cudaSuccess)
+      return TP_ERR_CUDA;
+    int n = 0;
+    cfg.gridDim = dim3(2 * (sm_count() / 2), 1, 1);
+    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0) return TP_ERR_CUDA;
+    max_clusters[dev] = n;
+  }
+  const int clusters = args.num_tiles < max_clusters[dev] ? args.num_tiles : max_clusters[dev];
+  cfg.gridDim = dim3(2 * clusters, 1, 1);
+  {
+    TraceScope ts(stream, TK_GEMM, flops);
+    if (cudaLaunchKernelEx(&cfg, kern, ta, tb, args) != cudaSuccess) return TP_ERR_CUDA;
+  }
+  return cuda_status(cudaGetLastError());
+}
+
 }  // namespace
 
 tp_status launch_gemm(const GemmProblem& g, cudaStream_t stream) {
   if (g.Mt <= 0 || g.Nt <= 0 || g.Kt <= 0) return TP_OK;   // empty product: nothing to do
   if (g.a.f16 != g.b.f16) return TP_ERR_INVALID_ARG;       // one MMA takes one operand type
+  // Pairs of CTAs (256-row tiles) unless one 128-row block covers M.
+  const bool pair = g.Mt > GEMM_BM;
   CUtensorMap ta, tb;
   if (!encode_operand(&ta, g.a, g.a.mn_major ? 64 : GEMM_BM)) return TP_ERR_CUDA;
-  if (!encode_operand(&tb, g.b, g.b.mn_major ? 64 : GEMM_BN)) return TP_ERR_CUDA;
+  if (!encode_operand(&tb, g.b, g.b.mn_major ? 64 : (pair ? 128 : GEMM_BN))) return TP_ERR_CUDA;
 
   GemmArgs a{};
   a.m_shards = g.m_shards;
   a.n_shards = g.n_shards;
   a.Mt = g.Mt;
   a.Nt = g.Nt;
-  a.mb_per_shard = (g.Mt + GEMM_BM - 1) / GEMM_BM;
-  a.nb_per_shard = (g.Nt + GEMM_BN - 1) / GEMM_BN;
+  const int bm = pair ? GP_BM : GEMM_BM, bn = pair ? GP_BN : GEMM_BN;
+  a.mb_per_shard = (g.Mt + bm - 1) / bm;
+  a.nb_per_shard = (g.Nt + bn - 1) / bn;
   a.k_shards = g.k_shards;
   a.kb_per_shard = (g.Kt + GEMM_BK - 1) / GEMM_BK;
   a.a_src = g.a.src;
@@ -93,12 +134,19 @@ tp_status launch_gemm(const GemmProblem& g, cudaStream_t stream) {
   a.c_ns = g.c_ns;
   a.ldc = g.ldc;
   a.err = error_word();
-  a.idesc = idesc_f32acc(GEMM_BM, GEMM_BN, g.a.mn_major, g.b.mn_major, g.a.f16);
+  a.idesc = idesc_f32acc(pair ? GP_BM : GEMM_BM, pair ? GP_BN : GEMM_BN, g.a.mn_major,
+                         g.b.mn_major, g.a.f16);
   a.out_f16 = g.out_f16 ? 1 : 0;
   const int grid = (int)(tiles < sm_count() ? tiles : sm_count());
   const double flops = 2.0 * g.m_shards * (double)g.Mt * g.n_shards * (double)g.Nt * g.k_shards *
                        (double)g.Kt;
 
+  if (pair) {
+    if (!g.a.mn_major && g.b.mn_major) return launch_pair<false, true>(ta, tb, a, flops, stream);
+    if (!g.a.mn_major && !g.b.mn_major) return launch_pair<false, false>(ta, tb, a, flops, stream);
+    if (g.a.mn_major && g.b.mn_major) return launch_pair<true, true>(ta, tb, a, flops, stream);
+    return launch_pair<true, false>(ta, tb, a, flops, stream);
+  }
   if (!g.a.mn_major && g.b.mn_major) return launch_inst<false, true>(ta, tb, a, grid, flops, stream);
   if (!g.a.mn_major && !g.b.mn_major) return launch_inst<false, false>(ta, tb, a, grid, flops, stream);
   if (g.a.mn_major && g.b.mn_major) return launch_inst<true, true>(ta, tb, a, grid, flops, stream);

@@ -92,6 +92,94 @@ __device__ __forceinline__ float gelu_tanh_grad_f(float a) {
   return 0.5f * (1.0f + th) + 0.5f * a * (1.0f - th * th) * k0 * (1.0f + 3.0f * k1 * a * a);
 }
 
+// Epilogue of 32 consecutive columns [n, n+32) of one output row: bias,
+// residual or GeLU', store (bf16 or fp16), and GeLU into C2.  `base` is the
+// row's element offset of C; columns past Nt are not touched.
+__device__ __forceinline__ void epilogue_store32(const GemmArgs& p, float (&v)[32], int ns,
+                                                 long long base, int n) {
+  const int nvalid = min(32, p.Nt - n);   // a multiple of 8
+  if (p.bias != nullptr && p.epi != EPI_DGELU) {
+    const __nv_bfloat16* bp = p.bias + (long long)ns * p.Nt + n;
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
+      if (g * 8 < nvalid) {
+        const uint4 bv = *reinterpret_cast<const uint4*>(bp + g * 8);
+        const uint32_t w[4] = {bv.x, bv.y, bv.z, bv.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          v[g * 8 + 2 * q] += bf16_lo(w[q]);
+          v[g * 8 + 2 * q + 1] += bf16_hi(w[q]);
+        }
+      }
+    }
+  }
+  if (p.aux != nullptr) {
+    const __nv_bfloat16* xp = p.aux + base + n;
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
+      if (g * 8 < nvalid) {
+        const uint4 av = *reinterpret_cast<const uint4*>(xp + g * 8);
+        const uint32_t w[4] = {av.x, av.y, av.z, av.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float lo = bf16_lo(w[q]), hi = bf16_hi(w[q]);
+          if (p.epi == EPI_DGELU) {
+            v[g * 8 + 2 * q] *= gelu_tanh_grad_f(lo);
+            v[g * 8 + 2 * q + 1] *= gelu_tanh_grad_f(hi);
+          } else {
+            v[g * 8 + 2 * q] += lo;
+            v[g * 8 + 2 * q + 1] += hi;
+          }
+        }
+      }
+    }
+  }
+  __nv_bfloat16* cp = p.c + base + n;
+  if (p.out_f16) {
+    bool over = false;
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
+      if (g * 8 < nvalid) {
+        uint4 o;
+        o.x = pack_f16x2(v[g * 8 + 0], v[g * 8 + 1]);
+        o.y = pack_f16x2(v[g * 8 + 2], v[g * 8 + 3]);
+        o.z = pack_f16x2(v[g * 8 + 4], v[g * 8 + 5]);
+        o.w = pack_f16x2(v[g * 8 + 6], v[g * 8 + 7]);
+        *reinterpret_cast<uint4*>(cp + g * 8) = o;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) over |= fabsf(v[g * 8 + e]) > 65504.0f;
+      }
+    }
+    if (over && p.err) atomicCAS(p.err, 0u, ERR_F16_RANGE);
+  } else {
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
+      if (g * 8 < nvalid) {
+        uint4 o;
+        o.x = pack_bf16x2(v[g * 8 + 0], v[g * 8 + 1]);
+        o.y = pack_bf16x2(v[g * 8 + 2], v[g * 8 + 3]);
+        o.z = pack_bf16x2(v[g * 8 + 4], v[g * 8 + 5]);
+        o.w = pack_bf16x2(v[g * 8 + 6], v[g * 8 + 7]);
+        *reinterpret_cast<uint4*>(cp + g * 8) = o;
+      }
+    }
+  }
+  if (p.epi == EPI_BIAS_GELU) {
+    __nv_bfloat16* hp = p.c2 + base + n;
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
+      if (g * 8 < nvalid) {
+        uint4 o;
+        o.x = pack_bf16x2(gelu_tanh_f(v[g * 8 + 0]), gelu_tanh_f(v[g * 8 + 1]));
+        o.y = pack_bf16x2(gelu_tanh_f(v[g * 8 + 2]), gelu_tanh_f(v[g * 8 + 3]));
+        o.z = pack_bf16x2(gelu_tanh_f(v[g * 8 + 4]), gelu_tanh_f(v[g * 8 + 5]));
+        o.w = pack_bf16x2(gelu_tanh_f(v[g * 8 + 6]), gelu_tanh_f(v[g * 8 + 7]));
+        *reinterpret_cast<uint4*>(hp + g * 8) = o;
+      }
+    }
+  }
+}
+
 struct TileCoord {
   int ms, m0, ns, n0;
 };
@@ -292,87 +380,7 @@ gemm_bf16_sm100(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
         float v[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-        const int nvalid = min(32, p.Nt - n);   // a multiple of 8
-        if (p.bias != nullptr && p.epi != EPI_DGELU) {
-          const __nv_bfloat16* bp = p.bias + (long long)tc.ns * p.Nt + n;
-#pragma unroll
-          for (int g = 0; g < 4; ++g) {
-            if (g * 8 < nvalid) {
-              const uint4 bv = *reinterpret_cast<const uint4*>(bp + g * 8);
-              const uint32_t w[4] = {bv.x, bv.y, bv.z, bv.w};
-#pragma unroll
-              for (int q = 0; q < 4; ++q) {
-                v[g * 8 + 2 * q] += bf16_lo(w[q]);
-                v[g * 8 + 2 * q + 1] += bf16_hi(w[q]);
-              }
-            }
-          }
-        }
-        if (p.aux != nullptr) {
-          const __nv_bfloat16* xp = p.aux + base + n;
-#pragma unroll
-          for (int g = 0; g < 4; ++g) {
-            if (g * 8 < nvalid) {
-              const uint4 av = *reinterpret_cast<const uint4*>(xp + g * 8);
-              const uint32_t w[4] = {av.x, av.y, av.z, av.w};
-#pragma unroll
-              for (int q = 0; q < 4; ++q) {
-                const float lo = bf16_lo(w[q]), hi = bf16_hi(w[q]);
-                if (p.epi == EPI_DGELU) {
-                  v[g * 8 + 2 * q] *= gelu_tanh_grad_f(lo);
-                  v[g * 8 + 2 * q + 1] *= gelu_tanh_grad_f(hi);
-                } else {
-                  v[g * 8 + 2 * q] += lo;
-                  v[g * 8 + 2 * q + 1] += hi;
-                }
-              }
-            }
-          }
-        }
-        __nv_bfloat16* cp = p.c + base + n;
-        if (p.out_f16) {
-          bool over = false;
-#pragma unroll
-          for (int g = 0; g < 4; ++g) {
-            if (g * 8 < nvalid) {
-              uint4 o;
-              o.x = pack_f16x2(v[g * 8 + 0], v[g * 8 + 1]);
-              o.y = pack_f16x2(v[g * 8 + 2], v[g * 8 + 3]);
-              o.z = pack_f16x2(v[g * 8 + 4], v[g * 8 + 5]);
-              o.w = pack_f16x2(v[g * 8 + 6], v[g * 8 + 7]);
-              *reinterpret_cast<uint4*>(cp + g * 8) = o;
-#pragma unroll
-              for (int e = 0; e < 8; ++e) over |= fabsf(v[g * 8 + e]) > 65504.0f;
-            }
-          }
-          if (over && p.err) atomicCAS(p.err, 0u, ERR_F16_RANGE);
-        } else {
-#pragma unroll
-          for (int g = 0; g < 4; ++g) {
-            if (g * 8 < nvalid) {
-              uint4 o;
-              o.x = pack_bf16x2(v[g * 8 + 0], v[g * 8 + 1]);
-              o.y = pack_bf16x2(v[g * 8 + 2], v[g * 8 + 3]);
-              o.z = pack_bf16x2(v[g * 8 + 4], v[g * 8 + 5]);
-              o.w = pack_bf16x2(v[g * 8 + 6], v[g * 8 + 7]);
-              *reinterpret_cast<uint4*>(cp + g * 8) = o;
-            }
-          }
-        }
-        if (p.epi == EPI_BIAS_GELU) {
-          __nv_bfloat16* hp = p.c2 + base + n;
-#pragma unroll
-          for (int g = 0; g < 4; ++g) {
-            if (g * 8 < nvalid) {
-              uint4 o;
-              o.x = pack_bf16x2(gelu_tanh_f(v[g * 8 + 0]), gelu_tanh_f(v[g * 8 + 1]));
-              o.y = pack_bf16x2(gelu_tanh_f(v[g * 8 + 2]), gelu_tanh_f(v[g * 8 + 3]));
-              o.z = pack_bf16x2(gelu_tanh_f(v[g * 8 + 4]), gelu_tanh_f(v[g * 8 + 5]));
-              o.w = pack_bf16x2(gelu_tanh_f(v[g * 8 + 6]), gelu_tanh_f(v[g * 8 + 7]));
-              *reinterpret_cast<uint4*>(hp + g * 8) = o;
-            }
-          }
-        }
+        epilogue_store32(p, v, tc.ns, base, n);
       }
       tc_fence_before();
       mbar_arrive(&tempty[acc]);
@@ -384,6 +392,227 @@ gemm_bf16_sm100(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, GEMM_TMEM_COLS);
+  }
+}
+
+// =====================================================================================
+// CTA-pair variant (tcgen05 cta_group::2): a cluster of two CTAs computes one
+// 256 x 256 tile.  Each CTA streams its own 128 rows of A and its own half
+// (128 columns) of B; one thread of the even CTA issues 256 x 256 x 16 MMAs
+// that read A and B from both CTAs' shared memory and write each CTA's 128
+// rows into that CTA's tensor memory.  Per SM this halves the B tile it has
+// to fetch and stage compared with the single-CTA kernel.
+// =====================================================================================
+constexpr int GP_BM = 256;                 // rows per pair tile (128 per CTA)
+constexpr int GP_BN = 256;                 // columns per pair tile (128 of B per CTA)
+constexpr int GP_STAGES = 6;
+constexpr int GP_A_BYTES = 128 * GEMM_BK * 2;   // 16 KiB per CTA
+constexpr int GP_B_BYTES = 128 * GEMM_BK * 2;   // 16 KiB per CTA
+constexpr int GP_STAGE_BYTES = GP_A_BYTES + GP_B_BYTES;
+constexpr int GP_SMEM_BYTES = GP_STAGES * GP_STAGE_BYTES + 1024 + 256;
+
+enum : unsigned int {
+  ERR_GEMMP_PRODUCER_WAIT = 0x111,
+  ERR_GEMMP_MMA_WAIT = 0x112,
+  ERR_GEMMP_EPI_WAIT = 0x113,
+};
+
+__device__ __forceinline__ TileCoord gemm_pair_tile(const GemmArgs& p, int tile) {
+  const int mbt = p.m_shards * p.mb_per_shard;
+  const int nbt = p.n_shards * p.nb_per_shard;
+  const int per_group = p.group_m * nbt;
+  const int g = tile / per_group;
+  const int first = g * p.group_m;
+  const int gsize = min(mbt - first, p.group_m);
+  const int r = tile - g * per_group;
+  const int mb = first + r % gsize;
+  const int nb = r / gsize;
+  TileCoord tc;
+  tc.ms = mb / p.mb_per_shard;
+  tc.m0 = (mb - tc.ms * p.mb_per_shard) * GP_BM;
+  tc.ns = nb / p.nb_per_shard;
+  tc.n0 = (nb - tc.ns * p.nb_per_shard) * GP_BN;
+  return tc;
+}
+
+template <bool A_MN, bool B_MN>
+__global__ void __launch_bounds__(GEMM_THREADS, 1)
+gemm_pair_sm100(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                const GemmArgs p) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + GP_STAGES * GP_STAGE_BYTES);
+  uint64_t* full = bars;                      // [STAGES], counted in the even CTA
+  uint64_t* empty = bars + GP_STAGES;         // [STAGES], one per CTA
+  uint64_t* tfull = bars + 2 * GP_STAGES;     // [2]
+  uint64_t* tempty = tfull + 2;               // [2], counted in the even CTA
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < GP_STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&tfull[i], 1);
+      mbar_init(&tempty[i], 8);     // one arrival per epilogue warp of both CTAs
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, GEMM_TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();                   // the peer's barriers exist before anyone signals them
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int num_kb = p.k_shards * p.kb_per_shard;
+  const int cid = (int)cluster_id_x(), ncl = (int)nclusters_x();
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int it = 0;
+      bool ok = true;
+      for (int tile = cid; tile < p.num_tiles && ok; tile += ncl) {
+        const TileCoord tc = gemm_pair_tile(p, tile);
+        const int am = tc.m0 + (int)rank * 128;
+        const int bn = tc.n0 + (int)rank * 128;
+        for (int kb = 0; kb < num_kb; ++kb, ++it) {
+          const int s = it % GP_STAGES;
+          const uint32_t round = it / GP_STAGES;
+          if (!wait_or_abort(&empty[s], (round & 1) ^ 1, abort_flag)) {
+            record_error(p.err, abort_flag, ERR_GEMMP_PRODUCER_WAIT);
+            ok = false;
+            break;
+          }
+          const int ks = kb / p.kb_per_shard;
+          const int k0 = (kb - ks * p.kb_per_shard) * GEMM_BK;
+          const int a_s = p.a_src == SHARD_K ? ks : (p.a_src == SHARD_MN ? tc.ms : 0);
+          const int b_s = p.b_src == SHARD_K ? ks : (p.b_src == SHARD_MN ? tc.ns : 0);
+          uint8_t* sa = smem + s * GP_STAGE_BYTES;
+          uint8_t* sb = sa + GP_A_BYTES;
+          if (leader) mbar_arrive_expect_tx(&full[s], 2 * GP_STAGE_BYTES);
+          if (A_MN) {
+            tma_load_3d_pair(sa, &tmA, &full[s], am, k0, a_s);
+            tma_load_3d_pair(sa + 8192, &tmA, &full[s], am + 64, k0, a_s);
+          } else {
+            tma_load_3d_pair(sa, &tmA, &full[s], k0, am, a_s);
+          }
+          if (B_MN) {
+            tma_load_3d_pair(sb, &tmB, &full[s], bn, k0, b_s);
+            tma_load_3d_pair(sb + 8192, &tmB, &full[s], bn + 64, k0, b_s);
+          } else {
+            tma_load_3d_pair(sb, &tmB, &full[s], k0, bn, b_s);
+          }
+        }
+      }
+      if (leader) {
+        const int issued = it;
+        for (int j = 0; j < GP_STAGES && j < issued; ++j) {
+          const int i = issued - 1 - j;
+          mbar_wait(&full[i % GP_STAGES], (i / GP_STAGES) & 1, 200000000ull);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      if (leader) {
+        const uint32_t idesc = p.idesc;
+        int it = 0, tcount = 0;
+        bool ok = true;
+        for (int tile = cid; tile < p.num_tiles && ok; tile += ncl, ++tcount) {
+          const int acc = tcount & 1;
+          const uint32_t use = tcount >> 1;
+          if (!wait_or_abort(&tempty[acc], (use & 1) ^ 1, abort_flag)) {
+            record_error(p.err, abort_flag, ERR_GEMMP_MMA_WAIT);
+            break;
+          }
+          tc_fence_after();
+          const uint32_t d_tmem = tmem_base + acc * GP_BN;
+          for (int kb = 0; kb < num_kb; ++kb, ++it) {
+            const int s = it % GP_STAGES;
+            const uint32_t round = it / GP_STAGES;
+            if (!wait_or_abort(&full[s], round & 1, abort_flag)) {
+              record_error(p.err, abort_flag, ERR_GEMMP_MMA_WAIT);
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t sa = smem_u32(smem + s * GP_STAGE_BYTES);
+            const uint32_t sb = sa + GP_A_BYTES;
+#pragma unroll
+            for (int kk = 0; kk < GEMM_BK / 16; ++kk) {
+              const uint64_t ad = A_MN ? smem_desc_sw128(sa + kk * 2048, 8192, 1024)
+                                       : smem_desc_sw128(sa + kk * 32, 16, 1024);
+              const uint64_t bd = B_MN ? smem_desc_sw128(sb + kk * 2048, 8192, 1024)
+                                       : smem_desc_sw128(sb + kk * 32, 16, 1024);
+              tc_mma_f16_pair(d_tmem, ad, bd, idesc, (kb | kk) != 0);
+            }
+            tc_commit_pair(&empty[s], 0x3);   // frees stage s in both CTAs
+          }
+          if (!ok) break;
+          tc_commit_pair(&tfull[acc], 0x3);   // both CTAs' accumulators ready
+        }
+        tc_commit_pair(drain, 0x3);
+      }
+      if (!mbar_wait(drain, 0, 200000000ull)) record_error(p.err, abort_flag, ERR_GEMM_DRAIN_WAIT);
+    }
+  } else {
+    const int quad = warp & 3;
+    const int row = quad * 32 + lane;
+    const uint32_t tempty_leader0 = map_to_rank(&tempty[0], 0);
+    int tcount = 0;
+    for (int tile = cid; tile < p.num_tiles; tile += ncl, ++tcount) {
+      const TileCoord tc = gemm_pair_tile(p, tile);
+      const int acc = tcount & 1;
+      const uint32_t use = tcount >> 1;
+      if (!__all_sync(0xffffffffu, wait_or_abort(&tfull[acc], use & 1, abort_flag))) {
+        record_error(p.err, abort_flag, ERR_GEMMP_EPI_WAIT);
+        break;
+      }
+      tc_fence_after();
+      const int m = tc.m0 + (int)rank * 128 + row;
+      const bool row_ok = m < p.Mt;
+      const long long base = tc.ms * p.c_ms + tc.ns * p.c_ns + (long long)m * p.ldc;
+      const uint32_t taddr = tmem_base + ((uint32_t)(quad * 32) << 16) + acc * GP_BN;
+#pragma unroll 1
+      for (int c = 0; c < GP_BN / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld32(taddr + c * 32, r);
+        tc_wait_ld();
+        const int n = tc.n0 + c * 32;
+        if (!row_ok || n >= p.Nt) continue;
+        float v[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+        epilogue_store32(p, v, tc.ns, base, n);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(tempty_leader0 + acc * 8);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();                   // no CTA leaves while its pair may still read its memory
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, GEMM_TMEM_COLS);
   }
 }
 
