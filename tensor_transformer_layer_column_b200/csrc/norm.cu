@@ -62,77 +62,90 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
-// One warp per row; lane owns 8-element chunks lane, lane+32, ...  The
-// output is bf16, or fp16 when F16OUT (values beyond the fp16 range set
-// `err` to 0x301).
+// One warp per row, rows walked grid-stride; lane owns 8-element chunks lane,
+// lane+32, ...  The row stays in registers as packed bf16 (4 registers per
+// chunk), so two 256-thread blocks fit per SM.  Statistics in fp32, two
+// passes over the registers (mean, then centred variance).  The output is
+// bf16, or fp16 when F16OUT (values beyond the fp16 range set `err` to 0x301).
 template <int CH, bool F16OUT>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256, 2)
 ln_fwd_kernel(const uint16_t* __restrict__ x, const uint16_t* __restrict__ g,
               const uint16_t* __restrict__ b, long long rows, int D, float eps,
               uint16_t* __restrict__ y, float* __restrict__ mean, float* __restrict__ rstd,
               unsigned int* err) {
   const int lane = threadIdx.x & 31;
-  const long long row = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  if (row >= rows) return;
   const int nch = D >> 3;
-  const uint16_t* xr = x + row * D;
-  float v[CH][8];
-  float s = 0.f;
+  const long long nwarps = (long long)gridDim.x * (blockDim.x >> 5);
+  bool over = false;
+  for (long long row = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); row < rows;
+       row += nwarps) {
+    const uint16_t* xr = x + row * D;
+    uint4 pk[CH];
+    float s = 0.f;
 #pragma unroll
-  for (int j = 0; j < CH; ++j) {
-    const int c = lane + 32 * j;
-    if (c < nch) {
-      unpack8(*reinterpret_cast<const uint4*>(xr + c * 8), v[j]);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) s += v[j][e];
+    for (int j = 0; j < CH; ++j) {
+      const int c = lane + 32 * j;
+      if (c < nch) pk[j] = *reinterpret_cast<const uint4*>(xr + c * 8);
     }
-  }
-  const float mu = warp_sum(s) / D;
-  float ss = 0.f;
 #pragma unroll
-  for (int j = 0; j < CH; ++j) {
-    if (lane + 32 * j < nch) {
+    for (int j = 0; j < CH; ++j) {
+      if (lane + 32 * j < nch) {
+        float v[8];
+        unpack8(pk[j], v);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const float d = v[j][e] - mu;
-        ss += d * d;
+        for (int e = 0; e < 8; ++e) s += v[e];
       }
     }
-  }
-  const float rs = rsqrtf(warp_sum(ss) / D + eps);
+    const float mu = warp_sum(s) / D;
+    float ss = 0.f;
 #pragma unroll
-  for (int j = 0; j < CH; ++j) {
-    const int c = lane + 32 * j;
-    if (c < nch) {
-      float gv[8], bv[8], o[8];
-      unpack8(*reinterpret_cast<const uint4*>(g + c * 8), gv);
-      unpack8(*reinterpret_cast<const uint4*>(b + c * 8), bv);
+    for (int j = 0; j < CH; ++j) {
+      if (lane + 32 * j < nch) {
+        float v[8];
+        unpack8(pk[j], v);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) o[e] = (v[j][e] - mu) * rs * gv[e] + bv[e];
-      if (F16OUT) {
-        *reinterpret_cast<uint4*>(y + row * D + c * 8) = pack8_f16(o);
-        bool over = false;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) over |= fabsf(o[e]) > 65504.0f;
-        if (over && err) atomicCAS(err, 0u, 0x301u);
-      } else {
-        *reinterpret_cast<uint4*>(y + row * D + c * 8) = pack8(o);
+        for (int e = 0; e < 8; ++e) {
+          const float d = v[e] - mu;
+          ss += d * d;
+        }
       }
     }
+    const float rs = rsqrtf(warp_sum(ss) / D + eps);
+#pragma unroll
+    for (int j = 0; j < CH; ++j) {
+      const int c = lane + 32 * j;
+      if (c < nch) {
+        float v[8], gv[8], bv[8], o[8];
+        unpack8(pk[j], v);
+        unpack8(*reinterpret_cast<const uint4*>(g + c * 8), gv);
+        unpack8(*reinterpret_cast<const uint4*>(b + c * 8), bv);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) o[e] = (v[e] - mu) * rs * gv[e] + bv[e];
+        if (F16OUT) {
+          *reinterpret_cast<uint4*>(y + row * D + c * 8) = pack8_f16(o);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) over |= fabsf(o[e]) > 65504.0f;
+        } else {
+          *reinterpret_cast<uint4*>(y + row * D + c * 8) = pack8(o);
+        }
+      }
+    }
+    if (lane == 0) {
+      mean[row] = mu;
+      rstd[row] = rs;
+    }
   }
-  if (lane == 0) {
-    mean[row] = mu;
-    rstd[row] = rs;
-  }
+  if (F16OUT && over && err) atomicCAS(err, 0u, 0x301u);
 }
 
 constexpr int LNB_THREADS = 256;
 
 // One block walks a contiguous chunk of rows; thread owns 8-element chunks
-// tid, tid+256, ...; per-block dgamma/dbeta partials go to `partial`
-// [gridDim.x][2][D] and are reduced by ln_param_reduce in block order.
+// tid, tid+256, ...; the next row's operands are loaded while the current
+// row goes through its block reduction.  Per-block dgamma/dbeta partials go to
+// `partial` [gridDim.x][2][D] and are reduced by ln_param_reduce in block order.
 template <int CH>
-__global__ void __launch_bounds__(LNB_THREADS)
+__global__ void __launch_bounds__(LNB_THREADS, 2)
 ln_bwd_kernel(const uint16_t* __restrict__ dy, const uint16_t* __restrict__ x,
               const uint16_t* __restrict__ g, const float* __restrict__ mean,
               const float* __restrict__ rstd, const uint16_t* __restrict__ dres, long long rows,
@@ -151,18 +164,32 @@ ln_bwd_kernel(const uint16_t* __restrict__ dy, const uint16_t* __restrict__ x,
   const long long r0 = (long long)blockIdx.x * rows_per_block;
   const long long r1 = min(rows, r0 + rows_per_block);
   const float invD = 1.0f / D;
+  uint4 cdy[CH], cx[CH], cres[CH];
+  auto load_row = [&](long long r, uint4 (&ody)[CH], uint4 (&ox)[CH], uint4 (&ores)[CH]) {
+#pragma unroll
+    for (int j = 0; j < CH; ++j) {
+      const int c = tid + LNB_THREADS * j;
+      if (c < nch) {
+        ody[j] = *reinterpret_cast<const uint4*>(dy + r * D + c * 8);
+        ox[j] = *reinterpret_cast<const uint4*>(x + r * D + c * 8);
+        if (dres != nullptr) ores[j] = *reinterpret_cast<const uint4*>(dres + r * D + c * 8);
+      }
+    }
+  };
+  if (r0 < r1) load_row(r0, cdy, cx, cres);
   int buf = 0;
   for (long long r = r0; r < r1; ++r, buf ^= 1) {
+    uint4 ndy[CH], nx[CH], nres[CH];
+    if (r + 1 < r1) load_row(r + 1, ndy, nx, nres);
     const float mu = mean[r], rs = rstd[r];
     float xh[CH][8], gv[CH][8];
     float s1 = 0.f, s2 = 0.f;
 #pragma unroll
     for (int j = 0; j < CH; ++j) {
-      const int c = tid + LNB_THREADS * j;
-      if (c < nch) {
+      if (tid + LNB_THREADS * j < nch) {
         float dv[8];
-        unpack8(*reinterpret_cast<const uint4*>(dy + r * D + c * 8), dv);
-        unpack8(*reinterpret_cast<const uint4*>(x + r * D + c * 8), xh[j]);
+        unpack8(cdy[j], dv);
+        unpack8(cx[j], xh[j]);
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           xh[j][e] = (xh[j][e] - mu) * rs;
@@ -198,12 +225,18 @@ ln_bwd_kernel(const uint16_t* __restrict__ dy, const uint16_t* __restrict__ x,
         for (int e = 0; e < 8; ++e) o[e] = rs * (gv[j][e] - m1 - xh[j][e] * m2);
         if (dres != nullptr) {
           float rv[8];
-          unpack8(*reinterpret_cast<const uint4*>(dres + r * D + c * 8), rv);
+          unpack8(cres[j], rv);
 #pragma unroll
           for (int e = 0; e < 8; ++e) o[e] += rv[e];
         }
         *reinterpret_cast<uint4*>(dx + r * D + c * 8) = pack8(o);
       }
+    }
+#pragma unroll
+    for (int j = 0; j < CH; ++j) {
+      cdy[j] = ndy[j];
+      cx[j] = nx[j];
+      cres[j] = nres[j];
     }
   }
   float* pg = partial + (long long)blockIdx.x * 2 * D;
@@ -220,21 +253,45 @@ ln_bwd_kernel(const uint16_t* __restrict__ dy, const uint16_t* __restrict__ x,
   }
 }
 
-// out_k[c] = sum over blocks b (in order) of partial[b][k][c], k = 0 (dgamma), 1 (dbeta).
-__global__ void ln_param_reduce(const float* __restrict__ partial, int nblocks, int D,
-                                uint16_t* __restrict__ dg, uint16_t* __restrict__ db) {
-  const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= 2 * D) return;
+// Fixed-order reduction of `n` partial rows of `width` floats: block x covers
+// 32 columns; warp w sums rows w, w+8, ... of its column (coalesced 128-byte
+// rows), then warp 0 adds the 8 warp sums in order.  Returns the total for
+// column blockIdx.x*32 + lane in warp 0 (valid when that column exists).
+__device__ __forceinline__ float reduce_rows_fixed(const float* __restrict__ rowsrc, int n,
+                                                   long long width, long long stride_rows,
+                                                   float (*red)[33]) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const long long c = (long long)blockIdx.x * 32 + lane;
   float s = 0.f;
-  for (int b = 0; b < nblocks; ++b) s += partial[(long long)b * 2 * D + i];
+  if (c < width)
+    for (int k = warp; k < n; k += 8) s += rowsrc[(long long)k * stride_rows + c];
+  red[warp][lane] = s;
+  __syncthreads();
+  float t = 0.f;
+  if (warp == 0) {
+#pragma unroll
+    for (int w = 0; w < 8; ++w) t += red[w][lane];
+  }
+  return t;
+}
+
+// out_k[c] = sum over blocks b (fixed order) of partial[b][k][c]; k = 0 dgamma, 1 dbeta.
+__global__ void __launch_bounds__(256)
+ln_param_reduce(const float* __restrict__ partial, int nblocks, int D, uint16_t* __restrict__ dg,
+                uint16_t* __restrict__ db) {
+  __shared__ float red[8][33];
+  const float t = reduce_rows_fixed(partial, nblocks, 2LL * D, 2LL * D, red);
+  const int i = blockIdx.x * 32 + (threadIdx.x & 31);
+  if ((threadIdx.x >> 5) != 0 || i >= 2 * D) return;
   uint16_t* out = i < D ? dg : db;
   if (out == nullptr) return;
-  __nv_bfloat16 v = __float2bfloat16_rn(s);
+  __nv_bfloat16 v = __float2bfloat16_rn(t);
   out[i < D ? i : i - D] = *reinterpret_cast<uint16_t*>(&v);
 }
 
 // Column sums of S stacked [rows][cols] matrices, pass 1: block (cx, cy, s)
-// sums rows [cy*rpc, (cy+1)*rpc) of columns [cx*2048, cx*2048+2048) of matrix s.
+// sums rows [cy*rpc, (cy+1)*rpc) of columns [cx*2048, cx*2048+2048) of matrix s,
+// four rows in flight per thread.
 template <bool F16IN>
 __global__ void __launch_bounds__(256)
 colsum_partial_kernel(const uint16_t* __restrict__ x, long long rows, long long cols,
@@ -245,28 +302,48 @@ colsum_partial_kernel(const uint16_t* __restrict__ x, long long rows, long long 
   const long long r0 = (long long)blockIdx.y * rows_per_chunk;
   const long long r1 = min(rows, r0 + rows_per_chunk);
   const uint16_t* base = x + s * rows * cols + c;
-  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-  for (long long r = r0; r < r1; ++r) {
+  float acc[4][8];
+#pragma unroll
+  for (int u = 0; u < 4; ++u)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[u][e] = 0.f;
+  long long r = r0;
+  for (; r + 4 <= r1; r += 4) {
+    uint4 q[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) q[u] = *reinterpret_cast<const uint4*>(base + (r + u) * cols);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      float v[8];
+      if (F16IN) unpack8_f16(q[u], v);
+      else unpack8(q[u], v);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[u][e] += v[e];
+    }
+  }
+  for (; r < r1; ++r) {
     float v[8];
     if (F16IN) unpack8_f16(*reinterpret_cast<const uint4*>(base + r * cols), v);
     else unpack8(*reinterpret_cast<const uint4*>(base + r * cols), v);
 #pragma unroll
-    for (int e = 0; e < 8; ++e) acc[e] += v[e];
+    for (int e = 0; e < 8; ++e) acc[0][e] += v[e];
   }
   float* p = partial + (s * gridDim.y + blockIdx.y) * cols + c;
 #pragma unroll
-  for (int e = 0; e < 8; ++e) p[e] = acc[e];
+  for (int e = 0; e < 8; ++e) p[e] = (acc[0][e] + acc[1][e]) + (acc[2][e] + acc[3][e]);
 }
 
-__global__ void colsum_reduce_kernel(const float* __restrict__ partial, int chunks, long long cols,
-                                     long long S, uint16_t* __restrict__ out) {
-  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= S * cols) return;
-  const long long s = i / cols, c = i - s * cols;
-  float acc = 0.f;
-  for (int k = 0; k < chunks; ++k) acc += partial[(s * chunks + k) * cols + c];
-  __nv_bfloat16 v = __float2bfloat16_rn(acc);
-  out[i] = *reinterpret_cast<uint16_t*>(&v);
+// Pass 2: out[s][c] = sum over chunks k (fixed order) of partial[s][k][c].
+__global__ void __launch_bounds__(256)
+colsum_reduce_kernel(const float* __restrict__ partial, int chunks, long long cols,
+                     uint16_t* __restrict__ out) {
+  __shared__ float red[8][33];
+  const long long s = blockIdx.y;
+  const float t = reduce_rows_fixed(partial + s * chunks * cols, chunks, cols, cols, red);
+  const long long c = (long long)blockIdx.x * 32 + (threadIdx.x & 31);
+  if ((threadIdx.x >> 5) != 0 || c >= cols) return;
+  __nv_bfloat16 v = __float2bfloat16_rn(t);
+  out[s * cols + c] = *reinterpret_cast<uint16_t*>(&v);
 }
 
 int colsum_chunks(long long rows, long long cols, long long S) {
@@ -279,7 +356,7 @@ int colsum_chunks(long long rows, long long cols, long long S) {
 }
 
 int ln_bwd_blocks(long long rows) {
-  long long b = 4LL * sm_count();
+  long long b = 2LL * sm_count();
   if (b > rows) b = rows;
   return (int)(b < 1 ? 1 : b);
 }
@@ -307,10 +384,10 @@ tp_status launch_colsum_stacked(const uint16_t* x, long long S, long long rows, 
     else
       colsum_partial_kernel<false><<<grid, 256, 0, stream>>>(x, rows, cols, rpc, partial);
   }
-  const long long n = S * cols;
   {
     TraceScope ts(stream, TK_COLSUM);
-    colsum_reduce_kernel<<<(unsigned)((n + 255) / 256), 256, 0, stream>>>(partial, chunks, cols, S, out);
+    const dim3 g2((unsigned)((cols + 31) / 32), (unsigned)S, 1);
+    colsum_reduce_kernel<<<g2, 256, 0, stream>>>(partial, chunks, cols, out);
   }
   return cuda_status(cudaGetLastError());
 }
@@ -319,7 +396,9 @@ template <bool F16OUT>
 tp_status ln_fwd_dispatch(const uint16_t* x, const uint16_t* g, const uint16_t* b, long long rows,
                           int D, float eps, uint16_t* y, float* mean, float* rstd,
                           cudaStream_t stream) {
-  const unsigned grid = (unsigned)((rows + 7) / 8);
+  long long nblk = (rows + 7) / 8;
+  if (nblk > 2LL * sm_count()) nblk = 2LL * sm_count();
+  const unsigned grid = (unsigned)nblk;
   const int per_lane = (D / 8 + 31) / 32;
   unsigned int* err = error_word();
   TraceScope ts(stream, TK_LN_FWD);
@@ -377,7 +456,7 @@ tp_status launch_layernorm_bwd(const uint16_t* dy, const uint16_t* x, const uint
   }
   if (dg != nullptr || db != nullptr) {
     TraceScope ts(stream, TK_LN_PARAM);
-    ln_param_reduce<<<(2 * D + 255) / 256, 256, 0, stream>>>(partial, nb, D, dg, db);
+    ln_param_reduce<<<(2 * D + 31) / 32, 256, 0, stream>>>(partial, nb, D, dg, db);
   }
   return cuda_status(cudaGetLastError());
 }
@@ -410,7 +489,7 @@ tp_status launch_layernorm_bwd_blocks(const uint16_t* dy, const uint16_t* x, con
   }
   if (dg != nullptr || db != nullptr) {
     TraceScope ts(stream, TK_LN_PARAM);
-    ln_param_reduce<<<(2 * D + 255) / 256, 256, 0, stream>>>(partial, nb, D, dg, db);
+    ln_param_reduce<<<(2 * D + 31) / 32, 256, 0, stream>>>(partial, nb, D, dg, db);
   }
   return cuda_status(cudaGetLastError());
 }
