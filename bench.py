@@ -32,7 +32,7 @@ if ROOT not in sys.path:
 import numpy as np  # noqa: E402
 import torch  # noqa: E402
 
-from synth import WORKLOADS, Workload, make_inputs, to_f64, workload  # noqa: E402
+from synth import PROFILING_WORKLOADS, WORKLOADS, Workload, make_inputs, to_f64, workload  # noqa: E402
 
 METRIC = "sharded-layer TFLOP/s (bf16 fwd+bwd, 1 B200) and % of dense BF16 peak"
 WORKLOAD = "layer_fwdbwd_B4_S2048_D4096_H32_F16384_t8"
@@ -396,7 +396,8 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
-    ap.add_argument("--workload", default=WORKLOAD, choices=sorted(WORKLOADS))
+    ap.add_argument("--workload", default=WORKLOAD,
+                    choices=sorted(WORKLOADS) + sorted(PROFILING_WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true",
                     help="skip the timed CPU oracle sample (for profiler runs)")
     ap.add_argument("--no-e2e", action="store_true",

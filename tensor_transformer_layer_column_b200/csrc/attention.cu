@@ -12,11 +12,11 @@
 // bf16 storage that alone puts the relative L2 error of O and of dWout near
 // 6e-3 at S = 2048, with fp16 near 2e-3.  The tensor-core rate is the same.
 //
-// Forward (per 128-query block, head, batch):
-//   S = q k^T (tcgen05, fp32 in TMEM, double-buffered), online softmax in
-//   fp32 by one thread per query row (base-2 exponent, scores pre-scaled by
-//   log2(e)/sqrt(dh)), P rounded to fp16 into swizzled shared memory,
-//   O += P v (tcgen05, fp32 in TMEM, rescaled in place when the row max moves).
+// Forward (per pair of 128-query tiles, head, batch; 64-key blocks):
+//   S = q k^T (tcgen05, fp32 in TMEM), online softmax in fp32 by one thread per
+//   query row (base-2 exponent, scores pre-scaled by log2(e)/sqrt(dh)), P
+//   rounded to fp16 into swizzled shared memory, O += P v (tcgen05, fp32 in
+//   TMEM, rescaled lazily).  The two tiles alternate on the tensor core.
 //   Writes O [t][T][Dt] (bf16) and the log-sum-exp [B][H][S] (fp32).
 // Backward (P recomputed from the log-sum-exp; no atomics, deterministic;
 // dO in and dqkv out are fp16):
@@ -115,64 +115,83 @@ __device__ __forceinline__ uint64_t mnmajor_desc(uint32_t base, int R, int kk) {
 // =====================================================================================
 // Forward
 // =====================================================================================
+// Two 128-query tiles per CTA take turns on the tensor core: while one tile's
+// softmax warpgroup works on its scores, the other tile's products run.  Keys
+// come in 64-wide blocks through a 3-stage ring; each tile has its own S (64
+// TMEM columns) and O (dh columns).  O is rescaled lazily: only when a row's
+// running max grows by more than 2^8 (log2 units), so P = 2^(s - m_used) stays
+// below 256 (exact in fp16) and the final O / l is unchanged.
 template <int DH>
 struct FwdCfg {
-  static constexpr int BM = 128, BN = 128, CH = DH / 64;
-  static constexpr int Q_BYTES = BM * DH * 2;
-  static constexpr int KV_BYTES = BN * DH * 2;
-  static constexpr int P_BYTES = BM * BN * 2;
-  static constexpr int OFF_K = Q_BYTES;                      // K[s] = OFF_K + s*2*KV, V[s] = +KV
-  static constexpr int OFF_P = Q_BYTES + 4 * KV_BYTES;
-  static constexpr int OFF_BAR = OFF_P + P_BYTES;
+  static constexpr int BM = 128, BN = 64, CH = DH / 64, STAGES = 3;
+  static constexpr int THREADS = 320;                   // producer, MMA, 2 x 4 softmax warps
+  static constexpr int Q_BYTES = BM * DH * 2;           // one query tile
+  static constexpr int KV_BYTES = BN * DH * 2;          // K or V of one stage
+  static constexpr int P_BYTES = BM * BN * 2;           // one P tile
+  static constexpr int OFF_Q = 0;                       // tile i at +i*Q
+  static constexpr int OFF_KV = 2 * Q_BYTES;            // stage s: K at +2s*KV, V at +(2s+1)*KV
+  static constexpr int OFF_P = OFF_KV + STAGES * 2 * KV_BYTES;   // tile i at +i*P
+  static constexpr int OFF_BAR = OFF_P + 2 * P_BYTES;
   static constexpr int RAW = OFF_BAR + 256 + 1024;
-  // One CTA per SM: the kernel holds all 512 TMEM columns.
-  static constexpr int SMEM = RAW > 120 * 1024 ? RAW : 120 * 1024;
+  static constexpr int SMEM = RAW > 120 * 1024 ? RAW : 120 * 1024;   // one CTA per SM (512 TMEM columns)
 };
 
+constexpr float kLazyRescaleLog2 = 8.0f;
+
 template <int DH>
-__global__ void __launch_bounds__(192, 1)
-attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_qkv, const AttnArgs p) {
+__global__ void __launch_bounds__(320, 1)
+attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q128,
+                const __grid_constant__ CUtensorMap tm_kv64, const AttnArgs p) {
   using C = FwdCfg<DH>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   uint64_t* q_full = bars + 0;
-  uint64_t* kv_full = bars + 1;     // [2]
-  uint64_t* kv_empty = bars + 3;    // [2]
-  uint64_t* s_full = bars + 5;      // [2]
-  uint64_t* s_free = bars + 7;      // [2]
-  uint64_t* p_full = bars + 9;
-  uint64_t* pv_done = bars + 10;
-  uint64_t* drain = bars + 11;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 12);
+  uint64_t* kv_full = bars + 1;     // [3]
+  uint64_t* kv_empty = bars + 4;    // [3]
+  uint64_t* s_full = bars + 7;      // [2] per tile
+  uint64_t* s_free = bars + 9;      // [2]
+  uint64_t* p_full = bars + 11;     // [2]
+  uint64_t* pv_done = bars + 13;    // [2]
+  uint64_t* drain = bars + 15;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nqb = (p.S + C::BM - 1) / C::BM;
+  const int nqb = (p.S + 2 * C::BM - 1) / (2 * C::BM);
   const int qb = p.causal ? nqb - 1 - (int)blockIdx.x : (int)blockIdx.x;
   const int h = blockIdx.y, b = blockIdx.z;
   const int shard = h / p.Ht, hl = h - shard * p.Ht;
-  const int q0 = qb * C::BM;
+  const int q0 = qb * 2 * C::BM;
   const int nkb = (p.S + C::BN - 1) / C::BN;
-  const int n_kv = p.causal ? min(nkb, qb + 1) : nkb;
+  int ntile[2];
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const int qs = q0 + i * C::BM;
+    ntile[i] = qs >= p.S ? 0 : (p.causal ? min(nkb, (qs + C::BM) / C::BN) : nkb);
+  }
+  const int nkv = max(ntile[0], ntile[1]);
   const int colq = hl * DH, colk = p.Dt + hl * DH, colv = 2 * p.Dt + hl * DH;
   const Ctl ctl{abort_flag, p.err};
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < C::STAGES; ++i) {
       mbar_init(&kv_full[i], 1);
       mbar_init(&kv_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
       mbar_init(&s_free[i], 128);
+      mbar_init(&p_full[i], 128);
+      mbar_init(&pv_done[i], 1);
     }
-    mbar_init(p_full, 128);
-    mbar_init(pv_done, 1);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
-    tma_prefetch_desc(&tm_qkv);
+    tma_prefetch_desc(&tm_q128);
+    tma_prefetch_desc(&tm_kv64);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, 512);
@@ -181,97 +200,122 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_qkv, const AttnArgs p) {
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
-  const uint32_t t_s0 = tmem, t_o = tmem + 256;
+  const uint32_t tmem = *tmem_slot;   // S of tile i at 64i; O of tile i at 128 + 128i
 
   if (warp == 0) {
     if (lane == 0) {
-      uint8_t* sq = smem;
-      mbar_arrive_expect_tx(q_full, C::Q_BYTES);
-      for (int c = 0; c < C::CH; ++c)
-        tma_load_4d(sq + c * C::BM * 128, &tm_qkv, q_full, colq + 64 * c, q0, b, shard);
+      mbar_arrive_expect_tx(q_full, 2 * C::Q_BYTES);
+      for (int i = 0; i < 2; ++i)
+        for (int c = 0; c < C::CH; ++c)
+          tma_load_4d(smem + C::OFF_Q + i * C::Q_BYTES + c * C::BM * 128, &tm_q128, q_full,
+                      colq + 64 * c, q0 + i * C::BM, b, shard);
       int j = 0;
-      for (; j < n_kv; ++j) {
-        const int st = j & 1;
-        const uint32_t u = j >> 1;
+      for (; j < nkv; ++j) {
+        const int st = j % C::STAGES;
+        const uint32_t u = j / C::STAGES;
         if (!wait_bar(&kv_empty[st], (u & 1) ^ 1, ctl, ERR_ATTN_FWD_WAIT)) break;
-        uint8_t* sk = smem + C::OFF_K + st * 2 * C::KV_BYTES;
+        uint8_t* sk = smem + C::OFF_KV + st * 2 * C::KV_BYTES;
         uint8_t* sv = sk + C::KV_BYTES;
         mbar_arrive_expect_tx(&kv_full[st], 2 * C::KV_BYTES);
         for (int c = 0; c < C::CH; ++c) {
-          tma_load_4d(sk + c * C::BN * 128, &tm_qkv, &kv_full[st], colk + 64 * c, j * C::BN, b, shard);
-          tma_load_4d(sv + c * C::BN * 128, &tm_qkv, &kv_full[st], colv + 64 * c, j * C::BN, b, shard);
+          tma_load_4d(sk + c * C::BN * 128, &tm_kv64, &kv_full[st], colk + 64 * c, j * C::BN, b, shard);
+          tma_load_4d(sv + c * C::BN * 128, &tm_kv64, &kv_full[st], colv + 64 * c, j * C::BN, b, shard);
         }
       }
-      // Let the copies this thread issued land before the CTA may exit.
       mbar_wait(q_full, 0, 200000000ull);
-      for (int i = j - 1; i >= 0 && i >= j - 2; --i) mbar_wait(&kv_full[i & 1], (i >> 1) & 1, 200000000ull);
+      for (int i = j - 1; i >= 0 && i >= j - C::STAGES; --i)
+        mbar_wait(&kv_full[i % C::STAGES], (i / C::STAGES) & 1, 200000000ull);
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      constexpr uint32_t id_qk = idesc_f32acc(128, 128, false, false, true);
+      constexpr uint32_t id_s = idesc_f32acc(128, C::BN, false, false, true);
       constexpr uint32_t id_pv = idesc_f32acc(128, DH, false, true, true);
-      const uint32_t sq = smem_u32(smem), sp = smem_u32(smem + C::OFF_P);
+      const uint32_t sq = smem_u32(smem + C::OFF_Q), sp = smem_u32(smem + C::OFF_P);
+      auto issue_s = [&](int i, uint32_t sk) {
+#pragma unroll
+        for (int kk = 0; kk < DH / 16; ++kk)
+          tc_mma_f16(tmem + 64 * i, kmajor_desc(sq + i * C::Q_BYTES, C::BM, kk),
+                     kmajor_desc(sk, C::BN, kk), id_s, kk > 0);
+        tc_commit(&s_full[i]);
+      };
+      auto issue_pv = [&](int i, int jj, uint32_t sv) {
+#pragma unroll
+        for (int kk = 0; kk < C::BN / 16; ++kk)
+          tc_mma_f16(tmem + 128 + 128 * i, kmajor_desc(sp + i * C::P_BYTES, C::BM, kk),
+                     mnmajor_desc(sv, C::BN, kk), id_pv, (jj | kk) != 0);
+        tc_commit(&pv_done[i]);
+      };
+      // Issue order: S of block j+1 for a tile goes out as soon as its softmax
+      // has copied S of block j out of tensor memory, so the next scores are
+      // computed while the current softmax runs; P V of block j follows once
+      // P is in shared memory.
       bool ok = wait_bar(q_full, 0, ctl, ERR_ATTN_FWD_WAIT);
-      for (int j = 0; ok && j <= n_kv; ++j) {
-        if (j < n_kv) {
-          const int st = j & 1;
-          const uint32_t u = j >> 1;
-          if (!wait_bar(&kv_full[st], u & 1, ctl, ERR_ATTN_FWD_WAIT)) break;
-          if (!wait_bar(&s_free[st], (u & 1) ^ 1, ctl, ERR_ATTN_FWD_WAIT)) break;
+      auto kv_addr = [&](int j) { return smem_u32(smem + C::OFF_KV + (j % C::STAGES) * 2 * C::KV_BYTES); };
+      if (ok && nkv > 0) {
+        ok = wait_bar(&kv_full[0], 0, ctl, ERR_ATTN_FWD_WAIT);
+        if (ok) {
           tc_fence_after();
-          const uint32_t sk = smem_u32(smem + C::OFF_K + st * 2 * C::KV_BYTES);
-#pragma unroll
-          for (int kk = 0; kk < DH / 16; ++kk)
-            tc_mma_f16(t_s0 + st * 128, kmajor_desc(sq, C::BM, kk), kmajor_desc(sk, C::BN, kk),
-                       id_qk, kk > 0);
-          tc_commit(&s_full[st]);
+          if (ntile[0] > 0) issue_s(0, kv_addr(0));
+          if (ntile[1] > 0) issue_s(1, kv_addr(0));
         }
-        if (j > 0) {
-          const int jj = j - 1, st = jj & 1;
-          if (!wait_bar(p_full, jj & 1, ctl, ERR_ATTN_FWD_WAIT)) break;
-          tc_fence_after();
-          const uint32_t sv = smem_u32(smem + C::OFF_K + st * 2 * C::KV_BYTES + C::KV_BYTES);
+      }
+      for (int j = 0; ok && j < nkv; ++j) {
+        const bool next = j + 1 < nkv;
+        if (next && !(ok = wait_bar(&kv_full[(j + 1) % C::STAGES], ((j + 1) / C::STAGES) & 1, ctl,
+                                    ERR_ATTN_FWD_WAIT)))
+          break;
 #pragma unroll
-          for (int kk = 0; kk < C::BN / 16; ++kk)
-            tc_mma_f16(t_o, kmajor_desc(sp, C::BM, kk), mnmajor_desc(sv, C::BN, kk), id_pv,
-                       (jj | kk) != 0);
-          tc_commit(pv_done);
-          tc_commit(&kv_empty[st]);
+        for (int i = 0; i < 2; ++i) {
+          if (j + 1 < ntile[i]) {
+            if (!(ok = wait_bar(&s_free[i], j & 1, ctl, ERR_ATTN_FWD_WAIT))) break;
+            tc_fence_after();
+            issue_s(i, kv_addr(j + 1));
+          }
+          if (j < ntile[i]) {
+            if (!(ok = wait_bar(&p_full[i], j & 1, ctl, ERR_ATTN_FWD_WAIT))) break;
+            tc_fence_after();
+            issue_pv(i, j, kv_addr(j) + C::KV_BYTES);
+          }
         }
+        if (!ok) break;
+        tc_commit(&kv_empty[j % C::STAGES]);   // every product that reads block j is issued
       }
       tc_commit(drain);
       mbar_wait(drain, 0, 200000000ull);
     }
   } else {
-    // ---------------------------------------------------------------- softmax warps
+    // ---------------------------------------------------------------- softmax warpgroups
+    const int tile = (warp - 2) >> 2;
     const int quad = warp & 3;
     const int r = quad * 32 + lane;
-    const int q = q0 + r;
+    const int qt = q0 + tile * C::BM;
+    const int q = qt + r;
+    const int n = ntile[tile];
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-    uint8_t* sp = smem + C::OFF_P;
-    float m = -1e30f, l = 0.f;
+    const uint32_t t_s = tmem + 64 * tile + lane_off;
+    const uint32_t t_o = tmem + 128 + 128 * tile + lane_off;
+    uint8_t* sp = smem + C::OFF_P + tile * C::P_BYTES;
+    float m_used = -1e30f, l = 0.f;
     bool ok = true;
-    for (int j = 0; j < n_kv; ++j) {
-      const int st = j & 1;
-      if (!__all_sync(0xffffffffu, wait_bar(&s_full[st], (j >> 1) & 1, ctl, ERR_ATTN_FWD_WAIT))) { ok = false; break; }
+    for (int j = 0; j < n; ++j) {
+      if (!__all_sync(0xffffffffu, wait_bar(&s_full[tile], j & 1, ctl, ERR_ATTN_FWD_WAIT))) { ok = false; break; }
       tc_fence_after();
-      float s[128];
+      float s[C::BN];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < C::BN / 32; ++c) {
         uint32_t rr[32];
-        tmem_ld32(t_s0 + st * 128 + lane_off + c * 32, rr);
+        tmem_ld32(t_s + c * 32, rr);
         tc_wait_ld();
 #pragma unroll
         for (int e = 0; e < 32; ++e) s[c * 32 + e] = __uint_as_float(rr[e]);
       }
       tc_fence_before();
-      mbar_arrive(&s_free[st]);
+      mbar_arrive(&s_free[tile]);
       const int k0 = j * C::BN;
-      const bool need_mask = (p.causal && k0 + C::BN - 1 > q0) || (k0 + C::BN > p.S);
-      float mx = m;
+      const bool need_mask = (p.causal && k0 + C::BN - 1 > qt) || (k0 + C::BN > p.S);
+      float mx = -1e30f;
 #pragma unroll
-      for (int c = 0; c < 128; ++c) {
+      for (int c = 0; c < C::BN; ++c) {
         float v = s[c] * p.scale_log2;
         if (need_mask) {
           const int kpos = k0 + c;
@@ -280,41 +324,48 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_qkv, const AttnArgs p) {
         s[c] = v;
         mx = fmaxf(mx, v);
       }
-      const float alpha = fast_exp2(m - mx);
-      m = mx;
+      float alpha = 1.0f;
+      if (j == 0) {
+        m_used = mx;
+      } else if (mx > m_used + kLazyRescaleLog2) {
+        alpha = fast_exp2(m_used - mx);
+        m_used = mx;
+        l *= alpha;
+      }
       float sum = 0.f;
 #pragma unroll
-      for (int c = 0; c < 128; ++c) {
-        const float e = fast_exp2(s[c] - m);
+      for (int c = 0; c < C::BN; ++c) {
+        const float e = fast_exp2(s[c] - m_used);
         s[c] = e;
         sum += e;
       }
-      l = l * alpha + sum;
+      l += sum;
       if (j > 0) {
-        // The previous P V has landed: P's buffer is free and O may be rescaled.
-        if (!__all_sync(0xffffffffu, wait_bar(pv_done, (j - 1) & 1, ctl, ERR_ATTN_FWD_WAIT))) { ok = false; break; }
+        // The previous P V of this tile has landed: P's buffer is free and O may be rescaled.
+        if (!__all_sync(0xffffffffu, wait_bar(&pv_done[tile], (j - 1) & 1, ctl, ERR_ATTN_FWD_WAIT))) { ok = false; break; }
         tc_fence_after();
         if (!__all_sync(0xffffffffu, alpha == 1.0f)) {
 #pragma unroll 1
           for (int c = 0; c < DH / 32; ++c) {
             uint32_t rr[32];
-            tmem_ld32(t_o + lane_off + c * 32, rr);
+            tmem_ld32(t_o + c * 32, rr);
             tc_wait_ld();
 #pragma unroll
             for (int e = 0; e < 32; ++e) rr[e] = __float_as_uint(__uint_as_float(rr[e]) * alpha);
-            tmem_st32(t_o + lane_off + c * 32, rr);
+            tmem_st32(t_o + c * 32, rr);
           }
           tc_wait_st();
         }
       }
 #pragma unroll
-      for (int g = 0; g < 16; ++g)
+      for (int g = 0; g < C::BN / 8; ++g)
         *reinterpret_cast<uint4*>(sp + sw128_offset(C::BM, r, g * 8)) = pack8_f16(&s[g * 8]);
       fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(p_full);
+      mbar_arrive(&p_full[tile]);
     }
-    if (ok && __all_sync(0xffffffffu, wait_bar(pv_done, (n_kv - 1) & 1, ctl, ERR_ATTN_FWD_WAIT))) {
+    if (ok && n > 0 &&
+        __all_sync(0xffffffffu, wait_bar(&pv_done[tile], (n - 1) & 1, ctl, ERR_ATTN_FWD_WAIT))) {
       tc_fence_after();
       const float inv_l = 1.0f / l;
       const bool valid = q < p.S;
@@ -322,7 +373,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_qkv, const AttnArgs p) {
 #pragma unroll 1
       for (int c = 0; c < DH / 32; ++c) {
         uint32_t rr[32];
-        tmem_ld32(t_o + lane_off + c * 32, rr);
+        tmem_ld32(t_o + c * 32, rr);
         tc_wait_ld();
         if (valid) {
           float v[32];
@@ -333,7 +384,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_qkv, const AttnArgs p) {
             *reinterpret_cast<uint4*>(orow + c * 32 + g * 8) = pack8_bf16(&v[g * 8]);
         }
       }
-      if (valid) p.lse[((long long)b * p.H + h) * p.S + q] = (m + __log2f(l)) * kLn2;
+      if (valid) p.lse[((long long)b * p.H + h) * p.S + q] = (m_used + __log2f(l)) * kLn2;
     }
   }
   tc_fence_before();
@@ -402,7 +453,7 @@ struct DkdvCfg {
 };
 
 template <int DH>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
 attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_kv128,
                      const __grid_constant__ CUtensorMap tm_q64,
                      const __grid_constant__ CUtensorMap tm_do64, const AttnArgs p) {
@@ -441,8 +492,8 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_kv128,
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&s_free[i], 128);
-      mbar_init(&p_full[i], 128);
+      mbar_init(&s_free[i], 256);   // both compute warpgroups
+      mbar_init(&p_full[i], 256);
       mbar_init(&mm2_done[i], 1);
     }
     mbar_init(drain, 1);
@@ -535,6 +586,9 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_kv128,
       mbar_wait(drain, 0, 200000000ull);
     }
   } else {
+    // Two compute warpgroups: warpgroup g takes columns [32g, 32g + 32) of each
+    // block and every other 32-column slice of the epilogue.
+    const int wg = (warp - 2) >> 2;
     const int quad = warp & 3;
     const int r = quad * 32 + lane;
     const int kpos = k0 + r;
@@ -553,7 +607,7 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_kv128,
       uint8_t* pt = smem + C::OFF_PT + 2 * bf * C::T_BYTES;
       uint8_t* dst = pt + C::T_BYTES;
 #pragma unroll 1
-      for (int c = 0; c < C::BQ / 32; ++c) {
+      for (int c = wg; c < C::BQ / 32; c += 2) {
         uint32_t rs[32], rd[32];
         tmem_ld32(tmem + bf * 128 + lane_off + c * 32, rs);
         tmem_ld32(tmem + bf * 128 + 64 + lane_off + c * 32, rd);
@@ -587,7 +641,7 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_kv128,
       const long long w3 = 3LL * p.Dt;
       uint16_t* row = p.out + (long long)shard * p.T * w3 + ((long long)b * p.S + kpos) * w3;
 #pragma unroll 1
-      for (int c = 0; c < DH / 32; ++c) {
+      for (int c = wg; c < DH / 32; c += 2) {
         uint32_t rv[32], rk[32];
         tmem_ld32(t_dv + lane_off + c * 32, rv);
         tmem_ld32(t_dk + lane_off + c * 32, rk);
@@ -637,7 +691,7 @@ struct DqCfg {
 };
 
 template <int DH>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
 attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q128,
                    const __grid_constant__ CUtensorMap tm_do128,
                    const __grid_constant__ CUtensorMap tm_kv64, const AttnArgs p) {
@@ -676,8 +730,8 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q128,
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&s_free[i], 128);
-      mbar_init(&p_full[i], 128);
+      mbar_init(&s_free[i], 256);   // both compute warpgroups
+      mbar_init(&p_full[i], 256);
       mbar_init(&mm2_done[i], 1);
     }
     mbar_init(drain, 1);
@@ -760,6 +814,9 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q128,
       mbar_wait(drain, 0, 200000000ull);
     }
   } else {
+    // Two compute warpgroups: warpgroup g takes columns [32g, 32g + 32) of each
+    // block and every other 32-column slice of the epilogue.
+    const int wg = (warp - 2) >> 2;
     const int quad = warp & 3;
     const int r = quad * 32 + lane;
     const int q = q0 + r;
@@ -778,7 +835,7 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q128,
       tc_fence_after();
       uint8_t* sds = smem + C::OFF_DS + bf * C::DS_BYTES;
 #pragma unroll 1
-      for (int c = 0; c < C::BK / 32; ++c) {
+      for (int c = wg; c < C::BK / 32; c += 2) {
         uint32_t rs[32], rd[32];
         tmem_ld32(tmem + bf * 128 + lane_off + c * 32, rs);
         tmem_ld32(tmem + bf * 128 + 64 + lane_off + c * 32, rd);
@@ -807,7 +864,7 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q128,
       const long long w3 = 3LL * p.Dt;
       uint16_t* row = p.out + (long long)shard * p.T * w3 + ((long long)b * p.S + q) * w3 + colq;
 #pragma unroll 1
-      for (int c = 0; c < DH / 32; ++c) {
+      for (int c = wg; c < DH / 32; c += 2) {
         uint32_t rq[32];
         tmem_ld32(t_dq + lane_off + c * 32, rq);
         tc_wait_ld();
@@ -907,17 +964,19 @@ AttnArgs make_args(int B, int S, int H, int dh, int t, int causal) {
 template <int DH>
 tp_status fwd_launch(const uint16_t* qkv, uint16_t* o, float* lse, const AttnArgs& a,
                      cudaStream_t st) {
-  CUtensorMap tm;
-  if (!encode_act(&tm, qkv, 3LL * a.Dt, a.S, a.B, a.t, a.T, 128)) return TP_ERR_CUDA;
+  CUtensorMap tq, tkv;
+  if (!encode_act(&tq, qkv, 3LL * a.Dt, a.S, a.B, a.t, a.T, 128) ||
+      !encode_act(&tkv, qkv, 3LL * a.Dt, a.S, a.B, a.t, a.T, 64))
+    return TP_ERR_CUDA;
   AttnArgs p = a;
   p.out = o;
   p.lse = lse;
   auto kern = attn_fwd_kernel<DH>;
   if (!set_smem((const void*)kern, FwdCfg<DH>::SMEM)) return TP_ERR_CUDA;
-  const dim3 grid((a.S + 127) / 128, a.H, a.B);
+  const dim3 grid((a.S + 255) / 256, a.H, a.B);
   {
     TraceScope ts(st, TK_ATTN_FWD, 4.0 * DH * core_pairs(a));
-    kern<<<grid, 192, FwdCfg<DH>::SMEM, st>>>(tm, p);
+    kern<<<grid, FwdCfg<DH>::THREADS, FwdCfg<DH>::SMEM, st>>>(tq, tkv, p);
   }
   return cuda_status(cudaGetLastError());
 }
@@ -953,12 +1012,12 @@ tp_status bwd_launch(const uint16_t* qkv, const uint16_t* o, const float* lse, c
   {
     // dP, dV and dK: three of the backward's four algorithmic products.
     TraceScope ts(st, TK_ATTN_BWD_DKDV, 6.0 * DH * core_pairs(a));
-    k1<<<dim3((a.S + 127) / 128, a.H, a.B), 192, DkdvCfg<DH>::SMEM, st>>>(kv128, q64, do64, p);
+    k1<<<dim3((a.S + 127) / 128, a.H, a.B), 320, DkdvCfg<DH>::SMEM, st>>>(kv128, q64, do64, p);
   }
   if (cudaGetLastError() != cudaSuccess) return TP_ERR_CUDA;
   {
     TraceScope ts(st, TK_ATTN_BWD_DQ, 2.0 * DH * core_pairs(a));
-    k2<<<dim3((a.S + 127) / 128, a.H, a.B), 192, DqCfg<DH>::SMEM, st>>>(q128, do128, kv64, p);
+    k2<<<dim3((a.S + 127) / 128, a.H, a.B), 320, DqCfg<DH>::SMEM, st>>>(q128, do128, kv64, p);
   }
   return cuda_status(cudaGetLastError());
 }

@@ -41,6 +41,31 @@ bool encode_operand(CUtensorMap* map, const OperandDesc& d, uint32_t box_outer) 
   return r == CUDA_SUCCESS;
 }
 
+// MN-major operand staged chunk-interleaved: a 5-D view (64 of MN, 8 K rows,
+// MN/64 chunks, K/8 groups, shards) whose box {64, 8, chunks, 8, 1} lands in
+// shared memory as [K group][chunk][8 rows x 128 B].  Needs MN % 64 == 0 and
+// K % 8 == 0 so that the view covers exactly the tensor.
+bool interleave_ok(const OperandDesc& d) {
+  return d.mn_major && d.inner % 64 == 0 && d.outer % 8 == 0;
+}
+
+bool encode_operand_il(CUtensorMap* map, const OperandDesc& d, uint32_t chunks) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const long long shard_stride = d.shards > 1 ? d.shard_stride : d.ld * d.outer;
+  const cuuint64_t dims[5] = {64, 8, (cuuint64_t)(d.inner / 64), (cuuint64_t)(d.outer / 8),
+                              (cuuint64_t)d.shards};
+  const cuuint64_t strides[4] = {(cuuint64_t)d.ld * 2, 128, (cuuint64_t)d.ld * 16,
+                                 (cuuint64_t)shard_stride * 2};
+  const cuuint32_t box[5] = {64, 8, chunks, 8, 1};
+  const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  CUresult r = fn(map, d.f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5,
+                  const_cast<void*>(d.ptr), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 template <bool A_MN, bool B_MN>
 tp_status launch_inst(const CUtensorMap& ta, const CUtensorMap& tb, const GemmArgs& args,
                       int grid, double flops, cudaStream_t stream) {
@@ -106,9 +131,15 @@ tp_status launch_gemm(const GemmProblem& g, cudaStream_t stream) {
   if (g.a.f16 != g.b.f16) return TP_ERR_INVALID_ARG;       // one MMA takes one operand type
   // Pairs of CTAs (256-row tiles) unless one 128-row block covers M.
   const bool pair = g.Mt > GEMM_BM;
+  const bool a_il = interleave_ok(g.a), b_il = interleave_ok(g.b);
   CUtensorMap ta, tb;
-  if (!encode_operand(&ta, g.a, g.a.mn_major ? 64 : GEMM_BM)) return TP_ERR_CUDA;
-  if (!encode_operand(&tb, g.b, g.b.mn_major ? 64 : (pair ? 128 : GEMM_BN))) return TP_ERR_CUDA;
+  if (a_il ? !encode_operand_il(&ta, g.a, GEMM_BM / 64)
+           : !encode_operand(&ta, g.a, g.a.mn_major ? 64 : GEMM_BM))
+    return TP_ERR_CUDA;
+  const uint32_t b_rows = pair ? 128 : GEMM_BN;
+  if (b_il ? !encode_operand_il(&tb, g.b, b_rows / 64)
+           : !encode_operand(&tb, g.b, g.b.mn_major ? 64 : b_rows))
+    return TP_ERR_CUDA;
 
   GemmArgs a{};
   a.m_shards = g.m_shards;
@@ -137,6 +168,8 @@ tp_status launch_gemm(const GemmProblem& g, cudaStream_t stream) {
   a.idesc = idesc_f32acc(pair ? GP_BM : GEMM_BM, pair ? GP_BN : GEMM_BN, g.a.mn_major,
                          g.b.mn_major, g.a.f16);
   a.out_f16 = g.out_f16 ? 1 : 0;
+  a.a_il = a_il ? 1 : 0;
+  a.b_il = b_il ? 1 : 0;
   const int grid = (int)(tiles < sm_count() ? tiles : sm_count());
   const double flops = 2.0 * g.m_shards * (double)g.Mt * g.n_shards * (double)g.Nt * g.k_shards *
                        (double)g.Kt;

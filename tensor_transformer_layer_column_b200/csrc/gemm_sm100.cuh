@@ -77,18 +77,29 @@ struct GemmArgs {
   const __nv_bfloat16* bias;
   long long c_ms, c_ns, ldc;
   uint32_t idesc;                  // tcgen05 instruction descriptor (operand type, shape, majors)
+  int a_il, b_il;                  // MN-major operand staged chunk-interleaved (see below)
   int out_f16;                     // C (and C2) stored as fp16 instead of bf16
   unsigned int* err;
 };
 
+// tanh(u) = 1 - 2 / (e^(2u) + 1), with e^(2u) = 2^(2u log2 e) from the hardware
+// base-2 exponential: two special-function operations instead of a full tanh
+// routine.  Saturates to +-1 for large |u| (e^(2u) -> inf or 0); absolute
+// error about 1e-7, far below the bf16/fp16 rounding of the stored results.
+__device__ __forceinline__ float tanh_via_exp2(float u) {
+  float e;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e) : "f"(u * 2.8853900817779268f));   // 2 log2(e)
+  return 1.0f - __fdividef(2.0f, e + 1.0f);
+}
+
 __device__ __forceinline__ float gelu_tanh_f(float a) {
   const float k0 = 0.7978845608028654f, k1 = 0.044715f;
-  return 0.5f * a * (1.0f + tanhf(k0 * (a + k1 * a * a * a)));
+  return 0.5f * a * (1.0f + tanh_via_exp2(k0 * (a + k1 * a * a * a)));
 }
 
 __device__ __forceinline__ float gelu_tanh_grad_f(float a) {
   const float k0 = 0.7978845608028654f, k1 = 0.044715f;
-  const float th = tanhf(k0 * (a + k1 * a * a * a));
+  const float th = tanh_via_exp2(k0 * (a + k1 * a * a * a));
   return 0.5f * (1.0f + th) + 0.5f * a * (1.0f - th * th) * k0 * (1.0f + 3.0f * k1 * a * a);
 }
 
@@ -178,6 +189,18 @@ __device__ __forceinline__ void epilogue_store32(const GemmArgs& p, float (&v)[3
       }
     }
   }
+}
+
+// Shared-memory descriptor of an MN-major operand tile of `chunks` 64-wide
+// M/N chunks at K step kk (16 rows of K).  Two staging layouts:
+//   interleaved (il): for each group of 8 K rows, the chunks' 1 KiB swizzle
+//     atoms sit side by side (the canonical order: LBO = 1 KiB between chunks,
+//     SBO = chunks KiB between 8-row K groups); one 5-D TMA box fills it;
+//   chunk-major: each chunk holds all 64 K rows (8 KiB); LBO = 8 KiB,
+//     SBO = 1 KiB; one 2-D box per chunk.
+__device__ __forceinline__ uint64_t mn_desc(uint32_t base, int chunks, int kk, bool il) {
+  return il ? smem_desc_sw128(base + kk * 2 * chunks * 1024, 1024, chunks * 1024)
+            : smem_desc_sw128(base + kk * 2048, 8192, 1024);
 }
 
 struct TileCoord {
@@ -285,14 +308,18 @@ gemm_bf16_sm100(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
           uint8_t* sa = smem + s * GEMM_STAGE_BYTES;
           uint8_t* sb = sa + GEMM_A_BYTES;
           mbar_arrive_expect_tx(&full[s], GEMM_STAGE_BYTES);
-          if (A_MN) {
+          if (A_MN && p.a_il) {
+            tma_load_5d(sa, &tmA, &full[s], 0, 0, tc.m0 / 64, k0 / 8, a_s);
+          } else if (A_MN) {
 #pragma unroll
             for (int j = 0; j < GEMM_BM / 64; ++j)
               tma_load_3d(sa + j * 8192, &tmA, &full[s], tc.m0 + 64 * j, k0, a_s);
           } else {
             tma_load_3d(sa, &tmA, &full[s], k0, tc.m0, a_s);
           }
-          if (B_MN) {
+          if (B_MN && p.b_il) {
+            tma_load_5d(sb, &tmB, &full[s], 0, 0, tc.n0 / 64, k0 / 8, b_s);
+          } else if (B_MN) {
 #pragma unroll
             for (int j = 0; j < GEMM_BN / 64; ++j)
               tma_load_3d(sb + j * 8192, &tmB, &full[s], tc.n0 + 64 * j, k0, b_s);
@@ -336,9 +363,9 @@ gemm_bf16_sm100(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
           const uint32_t sb = sa + GEMM_A_BYTES;
 #pragma unroll
           for (int kk = 0; kk < GEMM_BK / 16; ++kk) {
-            const uint64_t ad = A_MN ? smem_desc_sw128(sa + kk * 2048, 8192, 1024)
+            const uint64_t ad = A_MN ? mn_desc(sa, GEMM_BM / 64, kk, p.a_il)
                                      : smem_desc_sw128(sa + kk * 32, 16, 1024);
-            const uint64_t bd = B_MN ? smem_desc_sw128(sb + kk * 2048, 8192, 1024)
+            const uint64_t bd = B_MN ? mn_desc(sb, GEMM_BN / 64, kk, p.b_il)
                                      : smem_desc_sw128(sb + kk * 32, 16, 1024);
             tc_mma_f16(d_tmem, ad, bd, idesc, (kb | kk) != 0);
           }
@@ -506,13 +533,17 @@ gemm_pair_sm100(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
           uint8_t* sa = smem + s * GP_STAGE_BYTES;
           uint8_t* sb = sa + GP_A_BYTES;
           if (leader) mbar_arrive_expect_tx(&full[s], 2 * GP_STAGE_BYTES);
-          if (A_MN) {
+          if (A_MN && p.a_il) {
+            tma_load_5d_pair(sa, &tmA, &full[s], 0, 0, am / 64, k0 / 8, a_s);
+          } else if (A_MN) {
             tma_load_3d_pair(sa, &tmA, &full[s], am, k0, a_s);
             tma_load_3d_pair(sa + 8192, &tmA, &full[s], am + 64, k0, a_s);
           } else {
             tma_load_3d_pair(sa, &tmA, &full[s], k0, am, a_s);
           }
-          if (B_MN) {
+          if (B_MN && p.b_il) {
+            tma_load_5d_pair(sb, &tmB, &full[s], 0, 0, bn / 64, k0 / 8, b_s);
+          } else if (B_MN) {
             tma_load_3d_pair(sb, &tmB, &full[s], bn, k0, b_s);
             tma_load_3d_pair(sb + 8192, &tmB, &full[s], bn + 64, k0, b_s);
           } else {
@@ -556,9 +587,9 @@ gemm_pair_sm100(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
             const uint32_t sb = sa + GP_A_BYTES;
 #pragma unroll
             for (int kk = 0; kk < GEMM_BK / 16; ++kk) {
-              const uint64_t ad = A_MN ? smem_desc_sw128(sa + kk * 2048, 8192, 1024)
+              const uint64_t ad = A_MN ? mn_desc(sa, 2, kk, p.a_il)
                                        : smem_desc_sw128(sa + kk * 32, 16, 1024);
-              const uint64_t bd = B_MN ? smem_desc_sw128(sb + kk * 2048, 8192, 1024)
+              const uint64_t bd = B_MN ? mn_desc(sb, 2, kk, p.b_il)
                                        : smem_desc_sw128(sb + kk * 32, 16, 1024);
               tc_mma_f16_pair(d_tmem, ad, bd, idesc, (kb | kk) != 0);
             }
