@@ -492,8 +492,8 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_kv128,
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&s_free[i], 256);   // both compute warpgroups
-      mbar_init(&p_full[i], 256);
+      mbar_init(&s_free[i], 128);   // buffer i belongs to compute warpgroup i
+      mbar_init(&p_full[i], 128);
       mbar_init(&mm2_done[i], 1);
     }
     mbar_init(drain, 1);
@@ -586,15 +586,16 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_kv128,
       mbar_wait(drain, 0, 200000000ull);
     }
   } else {
-    // Two compute warpgroups: warpgroup g takes columns [32g, 32g + 32) of each
-    // block and every other 32-column slice of the epilogue.
+    // Two compute warpgroups: warpgroup g takes the blocks k with k % 2 == g (its
+    // own TMEM and shared buffers), so two blocks are in flight at once; the
+    // epilogue splits the 32-column slices between them.
     const int wg = (warp - 2) >> 2;
     const int quad = warp & 3;
     const int r = quad * 32 + lane;
     const int kpos = k0 + r;
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
     bool ok = true;
-    for (int k = 0; k < nsteps; ++k) {
+    for (int k = wg; k < nsteps; k += 2) {
       const int bf = k & 1;
       const uint32_t u = k >> 1;
       const int qs = (i0 + k) * C::BQ;
@@ -607,7 +608,7 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_kv128,
       uint8_t* pt = smem + C::OFF_PT + 2 * bf * C::T_BYTES;
       uint8_t* dst = pt + C::T_BYTES;
 #pragma unroll 1
-      for (int c = wg; c < C::BQ / 32; c += 2) {
+      for (int c = 0; c < C::BQ / 32; ++c) {
         uint32_t rs[32], rd[32];
         tmem_ld32(tmem + bf * 128 + lane_off + c * 32, rs);
         tmem_ld32(tmem + bf * 128 + 64 + lane_off + c * 32, rd);
@@ -634,8 +635,10 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_kv128,
       fence_proxy_async_smem();
       mbar_arrive(&p_full[bf]);
     }
-    const int last = nsteps - 1;
-    if (ok && __all_sync(0xffffffffu, wait_bar(&mm2_done[last & 1], (last >> 1) & 1, ctl, ERR_ATTN_DKDV_WAIT))) {
+    // Every product has completed once `drain` (committed after the last one)
+    // completes; waiting on the per-buffer barrier here could alias across its
+    // phases for the warpgroup that did not process the last block.
+    if (ok && __all_sync(0xffffffffu, wait_bar(drain, 0, ctl, ERR_ATTN_DKDV_WAIT))) {
       tc_fence_after();
       const bool valid = kpos < p.S;
       const long long w3 = 3LL * p.Dt;
@@ -730,8 +733,8 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q128,
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&s_free[i], 256);   // both compute warpgroups
-      mbar_init(&p_full[i], 256);
+      mbar_init(&s_free[i], 128);   // buffer i belongs to compute warpgroup i
+      mbar_init(&p_full[i], 128);
       mbar_init(&mm2_done[i], 1);
     }
     mbar_init(drain, 1);
@@ -814,8 +817,9 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q128,
       mbar_wait(drain, 0, 200000000ull);
     }
   } else {
-    // Two compute warpgroups: warpgroup g takes columns [32g, 32g + 32) of each
-    // block and every other 32-column slice of the epilogue.
+    // Two compute warpgroups: warpgroup g takes the blocks k with k % 2 == g (its
+    // own TMEM and shared buffers), so two blocks are in flight at once; the
+    // epilogue splits the 32-column slices between them.
     const int wg = (warp - 2) >> 2;
     const int quad = warp & 3;
     const int r = quad * 32 + lane;
@@ -826,7 +830,7 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q128,
     const float l2 = p.lse2[hrow + q];     // padded rows: +inf, so P = 0
     const float dv = p.dvec[hrow + q];
     bool ok = true;
-    for (int k = 0; k < nsteps; ++k) {
+    for (int k = wg; k < nsteps; k += 2) {
       const int bf = k & 1;
       const uint32_t u = k >> 1;
       const int ks = k * C::BK;
@@ -835,7 +839,7 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q128,
       tc_fence_after();
       uint8_t* sds = smem + C::OFF_DS + bf * C::DS_BYTES;
 #pragma unroll 1
-      for (int c = wg; c < C::BK / 32; c += 2) {
+      for (int c = 0; c < C::BK / 32; ++c) {
         uint32_t rs[32], rd[32];
         tmem_ld32(tmem + bf * 128 + lane_off + c * 32, rs);
         tmem_ld32(tmem + bf * 128 + 64 + lane_off + c * 32, rd);
@@ -857,9 +861,8 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q128,
       fence_proxy_async_smem();
       mbar_arrive(&p_full[bf]);
     }
-    const int last = nsteps - 1;
-    if (ok && nsteps > 0 &&
-        __all_sync(0xffffffffu, wait_bar(&mm2_done[last & 1], (last >> 1) & 1, ctl, ERR_ATTN_DQ_WAIT))) {
+    // As in the dK/dV kernel: `drain` completes after the last product.
+    if (ok && nsteps > 0 && __all_sync(0xffffffffu, wait_bar(drain, 0, ctl, ERR_ATTN_DQ_WAIT))) {
       tc_fence_after();
       const long long w3 = 3LL * p.Dt;
       uint16_t* row = p.out + (long long)shard * p.T * w3 + ((long long)b * p.S + q) * w3 + colq;
