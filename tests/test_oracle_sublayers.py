@@ -249,3 +249,69 @@ def test_layer_matches_torch_autograd():
     for name in p:
         np.testing.assert_allclose(g["d" + name], tp[name].grad.numpy(), atol=1e-10,
                                    err_msg=name)
+
+
+# ---------------------------------------------------------------- post-LN layer
+
+def test_postln_layer_structure():
+    x, p, B, H = _layer_case()
+    y, sv = layer.postln_layer_fwd(x, p, B, H)
+    from oracle import core
+    a, _ = attention.attn_fwd(x, p["wqkv"], p["bqkv"], p["wout"], p["bout"], B, H)
+    np.testing.assert_allclose(sv["z1"], x + a, atol=1e-13)
+    h, _, _ = core.layernorm_fwd(x + a, p["ln1_g"], p["ln1_b"])
+    np.testing.assert_allclose(sv["h"], h, atol=1e-13)
+    m, _, _ = mlp.mlp_fwd(h, p["w1"], p["b1"], p["w2"], p["b2"])
+    yy, _, _ = core.layernorm_fwd(h + m, p["ln2_g"], p["ln2_b"])
+    np.testing.assert_allclose(y, yy, atol=1e-13)
+    # With beta = 0 and gamma = 1 every output row is normalised: mean 0, variance ~ 1.
+    p1 = dict(p, ln2_g=np.ones_like(p["ln2_g"]), ln2_b=np.zeros_like(p["ln2_b"]))
+    y1, _ = layer.postln_layer_fwd(x, p1, B, H)
+    np.testing.assert_allclose(y1.mean(axis=1), 0, atol=1e-12)
+
+
+def test_postln_layer_bwd_finite_difference():
+    x, p, B, H = _layer_case()
+    dy = _rand(*x.shape)
+    g = layer.postln_layer_bwd(x, p, dy, B, H)
+
+    def J(xx, pp):
+        return (layer.postln_layer_fwd(xx, pp, B, H)[0] * dy).sum()
+
+    h = 1e-6
+    fd = np.zeros_like(x)
+    for idx in np.ndindex(x.shape):
+        xp, xm = x.copy(), x.copy()
+        xp[idx] += h
+        xm[idx] -= h
+        fd[idx] = (J(xp, p) - J(xm, p)) / (2 * h)
+    np.testing.assert_allclose(g["dx"], fd, rtol=0, atol=1e-7)
+    for name in p:
+        fd = np.zeros_like(p[name])
+        for idx in np.ndindex(p[name].shape):
+            pp = {k: v.copy() for k, v in p.items()}
+            pm = {k: v.copy() for k, v in p.items()}
+            pp[name][idx] += h
+            pm[name][idx] -= h
+            fd[idx] = (J(x, pp) - J(x, pm)) / (2 * h)
+        np.testing.assert_allclose(g["d" + name], fd, rtol=0, atol=1e-7, err_msg=name)
+
+
+def test_postln_layer_matches_torch_autograd():
+    x, p, B, H = _layer_case(B=2, S=5, H=4, dh=4, F_=64)
+    D = x.shape[1]
+    dy = _rand(*x.shape)
+    tx = torch.tensor(x, requires_grad=True)
+    tp = {k: torch.tensor(v, requires_grad=True) for k, v in p.items()}
+    z1 = tx + _torch_attn(tx, tp["wqkv"], tp["bqkv"], tp["wout"], tp["bout"], B, H)
+    h = F.layer_norm(z1, (D,), tp["ln1_g"], tp["ln1_b"], eps=1e-5)
+    z2 = h + F.gelu(h @ tp["w1"] + tp["b1"], approximate="tanh") @ tp["w2"] + tp["b2"]
+    y = F.layer_norm(z2, (D,), tp["ln2_g"], tp["ln2_b"], eps=1e-5)
+    y.backward(torch.tensor(dy))
+    y0, _ = layer.postln_layer_fwd(x, p, B, H)
+    np.testing.assert_allclose(y0, y.detach().numpy(), atol=1e-12)
+    g = layer.postln_layer_bwd(x, p, dy, B, H)
+    np.testing.assert_allclose(g["dx"], tx.grad.numpy(), atol=1e-10)
+    for name in p:
+        np.testing.assert_allclose(g["d" + name], tp[name].grad.numpy(), atol=1e-10,
+                                   err_msg=name)
