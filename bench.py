@@ -32,7 +32,7 @@ if ROOT not in sys.path:
 import numpy as np  # noqa: E402
 import torch  # noqa: E402
 
-from synth import PROFILING_WORKLOADS, WORKLOADS, Workload, make_inputs, to_f64, workload  # noqa: E402
+from synth import EXTRA_WORKLOADS, WORKLOADS, Workload, make_inputs, to_f64, workload  # noqa: E402
 
 METRIC = "sharded-layer TFLOP/s (bf16 fwd+bwd, 1 B200) and % of dense BF16 peak"
 WORKLOAD = "layer_fwdbwd_B4_S2048_D4096_H32_F16384_t8"
@@ -210,7 +210,8 @@ class Runner:
         dims = tl.Dims.of(w.batch, w.seq, w.hidden, w.ffn, w.heads, w.head_dim, w.t,
                           1 if w.causal else 0, w.ln_eps)
         if w.kind.startswith("layer"):
-            self.mod = ShardedLayer(dims, {k: g[k] for k in PARAMS})
+            self.mod = ShardedLayer(dims, {k: g[k] for k in PARAMS},
+                                    placement="post" if "postln" in w.kind else "pre")
             self.acts = self.mod.alloc_acts()
             self.grads = self.mod.alloc_grads()
         elif w.kind.startswith("attn"):
@@ -397,7 +398,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", default=WORKLOAD,
-                    choices=sorted(WORKLOADS) + sorted(PROFILING_WORKLOADS))
+                    choices=sorted(WORKLOADS) + sorted(EXTRA_WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true",
                     help="skip the timed CPU oracle sample (for profiler runs)")
     ap.add_argument("--no-e2e", action="store_true",

@@ -87,7 +87,9 @@ typedef enum {
   TP_OP_ATTN_FWD = 2,
   TP_OP_ATTN_BWD = 3,
   TP_OP_LAYER_FWD = 4,
-  TP_OP_LAYER_BWD = 5
+  TP_OP_LAYER_BWD = 5,
+  TP_OP_POSTLN_FWD = 6,
+  TP_OP_POSTLN_BWD = 7
 } tp_op;
 
 /* Version string of the library. */
@@ -244,6 +246,40 @@ tp_status tp_layer_fwd(const tp_dims* dims, const tp_bf16* x, const tp_layer_par
 tp_status tp_layer_bwd(const tp_dims* dims, const tp_bf16* x, const tp_layer_params* params,
                        const tp_layer_acts* acts, const tp_bf16* dy, tp_bf16* dx,
                        const tp_layer_grads* grads, void* ws, size_t ws_bytes, tp_stream stream);
+
+/* ------------------------------------------------------------------ post-LN layer
+ * The other placement in "The layernorm placement the paper flags as
+ * critical": LayerNorm after each residual addition (the original
+ * transformer's, the BERT ablation's other arm):
+ *   z1 = x + Attn(x);  h = LN1(z1);  z2 = h + MLP(h);  y = LN2(z2)
+ * Same parameters (tp_layer_params) and gradients (tp_layer_grads) as the
+ * pre-LN layer; the attention sublayer reads x itself. */
+typedef struct {
+  tp_bf16* z1;            /* x + attention output [T][D] (LN1 input) */
+  float *mean1, *rstd1;   /* [T] */
+  tp_bf16* qkv;           /* [t][T][3Dt], FP16 */
+  tp_bf16* o;             /* [t][T][Dt] */
+  float* lse;             /* [B][H][S] */
+  tp_bf16* h;             /* LN1(z1) [T][D] */
+  tp_bf16* z2;            /* h + MLP output [T][D] (LN2 input) */
+  float *mean2, *rstd2;   /* [T] */
+  tp_bf16* a;             /* MLP pre-activation [t][T][Ft] */
+  tp_bf16* hact;          /* MLP activation [t][T][Ft] */
+} tp_postln_acts;
+
+/* tp_postln_layer_fwd: x [T][D] -> y [T][D], filling *acts.
+ * Workspace: tp_workspace_size(TP_OP_POSTLN_FWD, dims) bytes. */
+tp_status tp_postln_layer_fwd(const tp_dims* dims, const tp_bf16* x, const tp_layer_params* params,
+                              const tp_postln_acts* acts, tp_bf16* y, void* ws, size_t ws_bytes,
+                              tp_stream stream);
+
+/* tp_postln_layer_bwd: dy -> dx and *grads:
+ *   dz2 = LN2^T(dy);  dh = dz2 + MLP^T(dz2);  dz1 = LN1^T(dh);  dx = dz1 + Attn^T(dz1)
+ * Workspace: tp_workspace_size(TP_OP_POSTLN_BWD, dims) bytes. */
+tp_status tp_postln_layer_bwd(const tp_dims* dims, const tp_bf16* x, const tp_layer_params* params,
+                              const tp_postln_acts* acts, const tp_bf16* dy, tp_bf16* dx,
+                              const tp_layer_grads* grads, void* ws, size_t ws_bytes,
+                              tp_stream stream);
 
 /* ------------------------------------------------------------------ LayerNorm
  * The pre-LN building block on its own ("The layernorm placement the paper

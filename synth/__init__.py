@@ -31,7 +31,7 @@ from typing import Dict, Optional
 
 import torch
 
-__all__ = ["Workload", "WORKLOADS", "PROFILING_WORKLOADS", "workload", "make_inputs", "to_f64"]
+__all__ = ["Workload", "WORKLOADS", "EXTRA_WORKLOADS", "workload", "make_inputs", "to_f64"]
 
 
 @dataclasses.dataclass(frozen=True)
@@ -96,16 +96,19 @@ WORKLOADS: Dict[str, Workload] = {w.name: w for w in [
              hidden=4096, ffn=16384, heads=32, head_dim=128, t=8),
 ]}
 
-# Profiling case (not one of the five): the layer's attention sublayer at half
-# the batch, forward + backward; its inputs exceed L2 but it holds < 1 GB.
-PROFILING_WORKLOADS: Dict[str, Workload] = {w.name: w for w in [
+# Beyond the five: a profiling case (the layer's attention sublayer at half the
+# batch; inputs exceed L2 but it holds < 1 GB) and the post-LN arm of the
+# layer-norm placement passage at the pre-LN layer's size.
+EXTRA_WORKLOADS: Dict[str, Workload] = {w.name: w for w in [
     Workload("attn_fwdbwd_B2_S2048_D4096_H32_t8", "attn_fwdbwd", batch=2, seq=2048, hidden=4096,
              heads=32, head_dim=128, t=8),
+    Workload("layer_postln_fwdbwd_B4_S2048_D4096_H32_F16384_t8", "layer_postln_fwdbwd", batch=4,
+             seq=2048, hidden=4096, ffn=16384, heads=32, head_dim=128, t=8),
 ]}
 
 
 def workload(name: str) -> Workload:
-    return WORKLOADS[name] if name in WORKLOADS else PROFILING_WORKLOADS[name]
+    return WORKLOADS[name] if name in WORKLOADS else EXTRA_WORKLOADS[name]
 
 
 def _normal(gen: torch.Generator, shape, std: float) -> torch.Tensor:

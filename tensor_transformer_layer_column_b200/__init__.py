@@ -16,8 +16,9 @@ import os
 from typing import Optional
 
 __all__ = [
-    "TpError", "Dims", "LayerParams", "LayerActs", "LayerGrads", "lib", "lib_path",
+    "TpError", "Dims", "LayerParams", "LayerActs", "PostLNActs", "LayerGrads", "lib", "lib_path",
     "OP_MLP_FWD", "OP_MLP_BWD", "OP_ATTN_FWD", "OP_ATTN_BWD", "OP_LAYER_FWD", "OP_LAYER_BWD",
+    "OP_POSTLN_FWD", "OP_POSTLN_BWD", "postln_layer_fwd", "postln_layer_bwd",
     "workspace_size", "check_error", "version", "EXPORTED_SYMBOLS",
     "shard_cols", "unshard_cols", "shard_rows", "unshard_rows", "shard_qkv_heads",
     "unshard_qkv_heads", "mlp_fwd", "mlp_bwd", "attn_fwd", "attn_bwd", "layer_fwd", "layer_bwd",
@@ -29,7 +30,8 @@ __all__ = [
 _HERE = os.path.dirname(os.path.abspath(__file__))
 lib_path = os.path.join(_HERE, "libtplayer.so")
 
-OP_MLP_FWD, OP_MLP_BWD, OP_ATTN_FWD, OP_ATTN_BWD, OP_LAYER_FWD, OP_LAYER_BWD = range(6)
+(OP_MLP_FWD, OP_MLP_BWD, OP_ATTN_FWD, OP_ATTN_BWD, OP_LAYER_FWD, OP_LAYER_BWD, OP_POSTLN_FWD,
+ OP_POSTLN_BWD) = range(8)
 
 STATUS_NAMES = {0: "TP_OK", 1: "TP_ERR_INVALID_ARG", 2: "TP_ERR_UNSUPPORTED",
                 3: "TP_ERR_MISALIGNED", 4: "TP_ERR_WORKSPACE", 5: "TP_ERR_CUDA",
@@ -65,6 +67,11 @@ class LayerActs(ctypes.Structure):
                                   "mean2", "rstd2", "a", "hact")]
 
 
+class PostLNActs(ctypes.Structure):
+    _fields_ = [(n, _P) for n in ("z1", "mean1", "rstd1", "qkv", "o", "lse", "h", "z2",
+                                  "mean2", "rstd2", "a", "hact")]
+
+
 class LayerGrads(ctypes.Structure):
     _fields_ = [(n, _P) for n in ("dln1_g", "dln1_b", "dwqkv", "dbqkv", "dwout", "dbout",
                                   "dln2_g", "dln2_b", "dw1", "db1", "dw2", "db2")]
@@ -91,6 +98,11 @@ _SIGS = {
     "tp_layer_bwd": [ctypes.POINTER(Dims), _P, ctypes.POINTER(LayerParams),
                      ctypes.POINTER(LayerActs), _P, _P, ctypes.POINTER(LayerGrads), _P,
                      ctypes.c_size_t, _P],
+    "tp_postln_layer_fwd": [ctypes.POINTER(Dims), _P, ctypes.POINTER(LayerParams),
+                            ctypes.POINTER(PostLNActs), _P, _P, ctypes.c_size_t, _P],
+    "tp_postln_layer_bwd": [ctypes.POINTER(Dims), _P, ctypes.POINTER(LayerParams),
+                            ctypes.POINTER(PostLNActs), _P, _P, ctypes.POINTER(LayerGrads), _P,
+                            ctypes.c_size_t, _P],
     "tp_layernorm_fwd": [_P, _P, _P, ctypes.c_int, ctypes.c_int, ctypes.c_float, _P, _P, _P, _P],
     "tp_layernorm_bwd_workspace_size": [ctypes.c_int, ctypes.c_int],
     "tp_layernorm_bwd": [_P, _P, _P, _P, _P, _P, ctypes.c_int, ctypes.c_int, _P, _P, _P, _P,
@@ -256,6 +268,24 @@ def layer_bwd(dims, x, params: dict, acts: dict, dy, dx, grads: dict, ws, stream
     _check(lib().tp_layer_bwd(ctypes.byref(dims), _ptr(x), ctypes.byref(p), ctypes.byref(a),
                               _ptr(dy), _ptr(dx), ctypes.byref(g), wp, wn, _stream(stream, x)),
            "tp_layer_bwd")
+
+
+def postln_layer_fwd(dims, x, params: dict, acts: dict, y, ws=None, stream=None):
+    wp, wn = _ws(ws)
+    p = _struct(LayerParams, params)
+    a = _struct(PostLNActs, acts)
+    _check(lib().tp_postln_layer_fwd(ctypes.byref(dims), _ptr(x), ctypes.byref(p), ctypes.byref(a),
+                                     _ptr(y), wp, wn, _stream(stream, x)), "tp_postln_layer_fwd")
+
+
+def postln_layer_bwd(dims, x, params: dict, acts: dict, dy, dx, grads: dict, ws, stream=None):
+    wp, wn = _ws(ws)
+    p = _struct(LayerParams, params)
+    a = _struct(PostLNActs, acts)
+    g = _struct(LayerGrads, grads)
+    _check(lib().tp_postln_layer_bwd(ctypes.byref(dims), _ptr(x), ctypes.byref(p), ctypes.byref(a),
+                                     _ptr(dy), _ptr(dx), ctypes.byref(g), wp, wn,
+                                     _stream(stream, x)), "tp_postln_layer_bwd")
 
 
 def layernorm_fwd(x, gamma, beta, rows, D, eps, y, mean, rstd, stream=None):

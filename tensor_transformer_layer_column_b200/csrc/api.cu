@@ -205,7 +205,8 @@ size_t mlp_bwd_ws(const Sizes& z) {
 
 tp_status mlp_bwd_impl(const Sizes& z, bf16p x, bf16p w1, bf16p w2, bf16p a_save, bf16p h_save,
                        bf16p dy, bf16p dres, uint16_t* dx, uint16_t* dw1, uint16_t* dw2,
-                       uint16_t* db1, uint16_t* db2, void* ws, cudaStream_t st) {
+                       uint16_t* db1, uint16_t* db2, void* ws, cudaStream_t st,
+                       const float* dres32 = nullptr, float* dx32 = nullptr) {
   if (z.T == 0) {
     // Sums over zero tokens: all parameter gradients are zero.
     cudaMemsetAsync(dw1, 0, (size_t)(z.D * z.F) * 2, st);
@@ -256,6 +257,8 @@ tp_status mlp_bwd_impl(const Sizes& z, bf16p x, bf16p w1, bf16p w2, bf16p a_save
   g7.a = op(da, false, SHARD_K, z.Ft, z.T, z.t, z.Ft, z.T * z.Ft);
   g7.b = op(w1, false, SHARD_K, z.Ft, z.D, z.t, z.Ft, z.D * z.Ft);
   g7.epi = EPI_LINEAR; g7.c = dx; g7.aux = dres;
+  if (dres32) { g7.aux = dres32; g7.aux_f32 = true; }
+  if (dx32) { g7.c = dx32; g7.out_f32 = true; }
   g7.c_ms = 0; g7.c_ns = 0; g7.ldc = z.D;
   if ((s = launch_gemm(g7, st)) != TP_OK) return s;
 
@@ -309,7 +312,7 @@ size_t attn_bwd_core_ws(const Sizes& z) {
 tp_status attn_bwd_impl(const Sizes& z, int causal, bf16p x16, bf16p wqkv16, bf16p wout,
                         bf16p qkv, bf16p o, const float* lse, bf16p dy, bf16p dres, uint16_t* dx,
                         uint16_t* dwqkv, uint16_t* dbqkv, uint16_t* dwout, uint16_t* dbout,
-                        void* ws, cudaStream_t st) {
+                        void* ws, cudaStream_t st, const float* dres32 = nullptr) {
   const long long w3 = 3 * z.Dt;
   if (z.T == 0) {
     cudaMemsetAsync(dwqkv, 0, (size_t)(z.D * 3 * z.D) * 2, st);
@@ -366,6 +369,7 @@ tp_status attn_bwd_impl(const Sizes& z, int causal, bf16p x16, bf16p wqkv16, bf1
   g4.a = op(dqkv, false, SHARD_K, w3, z.T, z.t, w3, z.T * w3, true);
   g4.b = op(wqkv16, false, SHARD_K, w3, z.D, z.t, w3, z.D * w3, true);
   g4.epi = EPI_LINEAR; g4.c = dx; g4.aux = dres;
+  if (dres32) { g4.aux = dres32; g4.aux_f32 = true; }
   g4.c_ms = 0; g4.c_ns = 0; g4.ldc = z.D;
   if ((s = launch_gemm(g4, st)) != TP_OK) return s;
 
@@ -396,6 +400,27 @@ size_t layer_bwd_ws(const Sizes& z) {
   c.take<uint16_t>((size_t)(z.D * 3 * z.D));   // fp16 copy of Wqkv
   c.take<uint16_t>((size_t)(z.T * z.D));       // du
   c.take<uint16_t>((size_t)(z.T * z.D));       // dh
+  c.take<float>(layernorm_bwd_partial_floats(z.T, (int)z.D));
+  const size_t sub = mlp_bwd_ws(z) > attn_bwd_core_ws(z) ? mlp_bwd_ws(z) : attn_bwd_core_ws(z);
+  c.take<uint8_t>(sub);
+  return align_up(c.off, 256);
+}
+
+// Post-LN layer workspaces: fp16 copies of x and Wqkv (forward and backward),
+// plus the gradient chain, LayerNorm partials and the sublayer workspace
+// (backward).  The chain dz2 -> dh -> dz1 passes through two LayerNorm
+// Jacobians and two residual additions; rounding each link to bf16 compounds
+// to about twice the per-element error of the pre-LN layer, so the links are
+// carried in fp32 and only the GEMM operands are bf16: one bf16 buffer (dz2,
+// then dz1), one fp32 buffer (dz2, then dz1) and fp32 dh.
+size_t postln_fwd_ws(const Sizes& z) { return attn_fwd_ws(z); }
+
+size_t postln_bwd_ws(const Sizes& z) {
+  Carver c(nullptr);
+  c.take<uint8_t>(attn_fwd_ws(z));
+  c.take<uint16_t>((size_t)(z.T * z.D));
+  c.take<float>((size_t)(z.T * z.D));
+  c.take<float>((size_t)(z.T * z.D));
   c.take<float>(layernorm_bwd_partial_floats(z.T, (int)z.D));
   const size_t sub = mlp_bwd_ws(z) > attn_bwd_core_ws(z) ? mlp_bwd_ws(z) : attn_bwd_core_ws(z);
   c.take<uint8_t>(sub);
@@ -439,6 +464,8 @@ size_t tp_workspace_size(int op_, const tp_dims* d) {
     case TP_OP_MLP_BWD: return check_mlp(d) == TP_OK ? mlp_bwd_ws(sizes_of(*d)) : 0;
     case TP_OP_ATTN_BWD: return check_attn(d) == TP_OK ? attn_bwd_ws(sizes_of(*d)) : 0;
     case TP_OP_LAYER_BWD: return check_layer(d) == TP_OK ? layer_bwd_ws(sizes_of(*d)) : 0;
+    case TP_OP_POSTLN_FWD: return check_layer(d) == TP_OK ? postln_fwd_ws(sizes_of(*d)) : 0;
+    case TP_OP_POSTLN_BWD: return check_layer(d) == TP_OK ? postln_bwd_ws(sizes_of(*d)) : 0;
   }
   return 0;
 }
@@ -711,6 +738,102 @@ tp_status tp_layer_bwd(const tp_dims* dims, const tp_bf16* x, const tp_layer_par
     return st;
   return launch_layernorm_bwd(du, x, p->ln1_g, a->mean1, a->rstd1, dh, z.T, (int)z.D, dx,
                               g->dln1_g, g->dln1_b, lnp, cs);
+}
+
+// ------------------------------------------------------------------ post-LN layer
+static tp_status check_postln_ptrs(const tp_layer_params* p, const tp_postln_acts* a) {
+  if (!p || !a) return TP_ERR_INVALID_ARG;
+  if (!all_set(p->ln1_g, p->ln1_b, p->wqkv, p->wout, p->ln2_g, p->ln2_b, p->w1, p->w2))
+    return TP_ERR_INVALID_ARG;
+  if (!all_set(a->z1, a->mean1, a->rstd1, a->qkv, a->o, a->lse, a->h, a->z2, a->mean2, a->rstd2,
+               a->a, a->hact))
+    return TP_ERR_INVALID_ARG;
+  if (!all_aligned(p->ln1_g, p->ln1_b, p->wqkv, p->bqkv, p->wout, p->bout, p->ln2_g, p->ln2_b,
+                   p->w1, p->b1, p->w2, p->b2))
+    return TP_ERR_MISALIGNED;
+  if (!all_aligned(a->z1, a->qkv, a->o, a->lse, a->h, a->z2, a->a, a->hact)) return TP_ERR_MISALIGNED;
+  return TP_OK;
+}
+
+tp_status tp_postln_layer_fwd(const tp_dims* dims, const tp_bf16* x, const tp_layer_params* p,
+                              const tp_postln_acts* a, tp_bf16* y, void* ws, size_t ws_bytes,
+                              tp_stream s) {
+  tp_status st = check_layer(dims);
+  if (st != TP_OK) return st;
+  if (!x || !y) return TP_ERR_INVALID_ARG;
+  if ((st = check_postln_ptrs(p, a)) != TP_OK) return st;
+  if (!all_aligned(x, y)) return TP_ERR_MISALIGNED;
+  const Sizes z = sizes_of(*dims);
+  cudaStream_t cs = (cudaStream_t)s;
+  if (z.T == 0) return TP_OK;
+  if ((st = check_ws(ws, ws_bytes, postln_fwd_ws(z))) != TP_OK) return st;
+  Carver c(ws);
+  uint16_t* x16 = c.take<uint16_t>((size_t)(z.T * z.D));
+  uint16_t* w16 = c.take<uint16_t>((size_t)(z.D * 3 * z.D));
+  if ((st = launch_cast_f16(x, (size_t)(z.T * z.D), x16, cs)) != TP_OK) return st;
+  if ((st = launch_cast_f16(p->wqkv, (size_t)(z.D * 3 * z.D), w16, cs)) != TP_OK) return st;
+  // z1 = x + Attn(x); h = LN1(z1); z2 = h + MLP(h); y = LN2(z2)
+  if ((st = attn_fwd_impl(z, dims->causal, x16, w16, p->bqkv, p->wout, p->bout, x, a->z1, a->qkv,
+                          a->o, a->lse, cs)) != TP_OK)
+    return st;
+  if ((st = launch_layernorm_fwd(a->z1, p->ln1_g, p->ln1_b, z.T, (int)z.D, dims->ln_eps, a->h,
+                                 a->mean1, a->rstd1, cs)) != TP_OK)
+    return st;
+  if ((st = mlp_fwd_impl(z, a->h, p->w1, p->b1, p->w2, p->b2, a->h, a->z2, a->a, a->hact, cs)) !=
+      TP_OK)
+    return st;
+  return launch_layernorm_fwd(a->z2, p->ln2_g, p->ln2_b, z.T, (int)z.D, dims->ln_eps, y, a->mean2,
+                              a->rstd2, cs);
+}
+
+tp_status tp_postln_layer_bwd(const tp_dims* dims, const tp_bf16* x, const tp_layer_params* p,
+                              const tp_postln_acts* a, const tp_bf16* dy, tp_bf16* dx,
+                              const tp_layer_grads* g, void* ws, size_t ws_bytes, tp_stream s) {
+  tp_status st = check_layer(dims);
+  if (st != TP_OK) return st;
+  if (!x || !dy || !dx || !g) return TP_ERR_INVALID_ARG;
+  if ((st = check_postln_ptrs(p, a)) != TP_OK) return st;
+  if (!all_set(g->dwqkv, g->dwout, g->dw1, g->dw2)) return TP_ERR_INVALID_ARG;
+  if (!all_aligned(x, dy, dx, g->dln1_g, g->dln1_b, g->dwqkv, g->dbqkv, g->dwout, g->dbout,
+                   g->dln2_g, g->dln2_b, g->dw1, g->db1, g->dw2, g->db2))
+    return TP_ERR_MISALIGNED;
+  const Sizes z = sizes_of(*dims);
+  cudaStream_t cs = (cudaStream_t)s;
+  if (z.T == 0) {
+    mlp_bwd_impl(z, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, g->dw1,
+                 g->dw2, g->db1, g->db2, nullptr, cs);
+    attn_bwd_impl(z, dims->causal, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
+                  nullptr, nullptr, g->dwqkv, g->dbqkv, g->dwout, g->dbout, nullptr, cs);
+    for (tp_bf16* q : {g->dln1_g, g->dln1_b, g->dln2_g, g->dln2_b})
+      if (q) cudaMemsetAsync(q, 0, (size_t)z.D * 2, cs);
+    return cuda_status(cudaGetLastError());
+  }
+  if ((st = check_ws(ws, ws_bytes, postln_bwd_ws(z))) != TP_OK) return st;
+  Carver c(ws);
+  uint16_t* x16 = c.take<uint16_t>((size_t)(z.T * z.D));
+  uint16_t* w16 = c.take<uint16_t>((size_t)(z.D * 3 * z.D));
+  c.off = align_up(attn_fwd_ws(z), 256);
+  uint16_t* d16 = c.take<uint16_t>((size_t)(z.T * z.D));   // dz2, then dz1 (GEMM operand)
+  float* d32 = c.take<float>((size_t)(z.T * z.D));          // dz2, then dz1 (residual carry)
+  float* dh32 = c.take<float>((size_t)(z.T * z.D));
+  float* lnp = c.take<float>(layernorm_bwd_partial_floats(z.T, (int)z.D));
+  const size_t sub = mlp_bwd_ws(z) > attn_bwd_core_ws(z) ? mlp_bwd_ws(z) : attn_bwd_core_ws(z);
+  void* subws = c.take<uint8_t>(sub);
+  // y = LN2(z2): dz2 = LN2^T(dy).  z2 = h + MLP(h): dh = dz2 + MLP^T(dz2).
+  if ((st = launch_layernorm_bwd(dy, a->z2, p->ln2_g, a->mean2, a->rstd2, nullptr, z.T, (int)z.D,
+                                 d16, g->dln2_g, g->dln2_b, lnp, cs, d32)) != TP_OK)
+    return st;
+  if ((st = mlp_bwd_impl(z, a->h, p->w1, p->w2, a->a, a->hact, d16, nullptr, nullptr, g->dw1,
+                         g->dw2, g->db1, g->db2, subws, cs, d32, dh32)) != TP_OK)
+    return st;
+  // h = LN1(z1): dz1 = LN1^T(dh).  z1 = x + Attn(x): dx = dz1 + Attn^T(dz1).
+  if ((st = launch_layernorm_bwd_f32(dh32, a->z1, p->ln1_g, a->mean1, a->rstd1, z.T, (int)z.D,
+                                     d16, d32, g->dln1_g, g->dln1_b, lnp, cs)) != TP_OK)
+    return st;
+  if ((st = launch_cast_f16(x, (size_t)(z.T * z.D), x16, cs)) != TP_OK) return st;
+  if ((st = launch_cast_f16(p->wqkv, (size_t)(z.D * 3 * z.D), w16, cs)) != TP_OK) return st;
+  return attn_bwd_impl(z, dims->causal, x16, w16, p->wout, a->qkv, a->o, a->lse, d16, nullptr, dx,
+                       g->dwqkv, g->dbqkv, g->dwout, g->dbout, subws, cs, d32);
 }
 
 }  // extern "C"

@@ -129,6 +129,8 @@ tp_status launch_pair(const CUtensorMap& ta, const CUtensorMap& tb, const GemmAr
 tp_status launch_gemm(const GemmProblem& g, cudaStream_t stream) {
   if (g.Mt <= 0 || g.Nt <= 0 || g.Kt <= 0) return TP_OK;   // empty product: nothing to do
   if (g.a.f16 != g.b.f16) return TP_ERR_INVALID_ARG;       // one MMA takes one operand type
+  // fp32 residual / output: plain linear epilogue, no fp16 store.
+  if ((g.out_f32 || g.aux_f32) && (g.epi != EPI_LINEAR || g.out_f16)) return TP_ERR_INVALID_ARG;
   // Pairs of CTAs (256-row tiles) unless one 128-row block covers M.
   const bool pair = g.Mt > GEMM_BM;
   const bool a_il = interleave_ok(g.a), b_il = interleave_ok(g.b);
@@ -168,6 +170,8 @@ tp_status launch_gemm(const GemmProblem& g, cudaStream_t stream) {
   a.idesc = idesc_f32acc(pair ? GP_BM : GEMM_BM, pair ? GP_BN : GEMM_BN, g.a.mn_major,
                          g.b.mn_major, g.a.f16);
   a.out_f16 = g.out_f16 ? 1 : 0;
+  a.out_f32 = g.out_f32 ? 1 : 0;
+  a.aux_f32 = g.aux_f32 ? 1 : 0;
   a.a_il = a_il ? 1 : 0;
   a.b_il = b_il ? 1 : 0;
   const int grid = (int)(tiles < sm_count() ? tiles : sm_count());

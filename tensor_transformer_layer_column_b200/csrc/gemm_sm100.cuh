@@ -79,6 +79,8 @@ struct GemmArgs {
   uint32_t idesc;                  // tcgen05 instruction descriptor (operand type, shape, majors)
   int a_il, b_il;                  // MN-major operand staged chunk-interleaved (see below)
   int out_f16;                     // C (and C2) stored as fp16 instead of bf16
+  int out_f32;                     // C stored as fp32 (EPI_LINEAR only; `c` then points at floats)
+  int aux_f32;                     // aux is an fp32 residual (EPI_LINEAR only)
   unsigned int* err;
 };
 
@@ -104,7 +106,7 @@ __device__ __forceinline__ float gelu_tanh_grad_f(float a) {
 }
 
 // Epilogue of 32 consecutive columns [n, n+32) of one output row: bias,
-// residual or GeLU', store (bf16 or fp16), and GeLU into C2.  `base` is the
+// residual (bf16 or fp32) or GeLU', store (bf16, fp16 or fp32), and GeLU into C2.  `base` is the
 // row's element offset of C; columns past Nt are not touched.
 __device__ __forceinline__ void epilogue_store32(const GemmArgs& p, float (&v)[32], int ns,
                                                  long long base, int n) {
@@ -124,7 +126,18 @@ __device__ __forceinline__ void epilogue_store32(const GemmArgs& p, float (&v)[3
       }
     }
   }
-  if (p.aux != nullptr) {
+  if (p.aux != nullptr && p.aux_f32) {
+    const float* xp = reinterpret_cast<const float*>(p.aux) + base + n;
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
+      if (g * 8 < nvalid) {
+        const float4 r0 = *reinterpret_cast<const float4*>(xp + g * 8);
+        const float4 r1 = *reinterpret_cast<const float4*>(xp + g * 8 + 4);
+        v[g * 8 + 0] += r0.x; v[g * 8 + 1] += r0.y; v[g * 8 + 2] += r0.z; v[g * 8 + 3] += r0.w;
+        v[g * 8 + 4] += r1.x; v[g * 8 + 5] += r1.y; v[g * 8 + 6] += r1.z; v[g * 8 + 7] += r1.w;
+      }
+    }
+  } else if (p.aux != nullptr) {
     const __nv_bfloat16* xp = p.aux + base + n;
 #pragma unroll
     for (int g = 0; g < 4; ++g) {
@@ -146,7 +159,18 @@ __device__ __forceinline__ void epilogue_store32(const GemmArgs& p, float (&v)[3
     }
   }
   __nv_bfloat16* cp = p.c + base + n;
-  if (p.out_f16) {
+  if (p.out_f32) {
+    float* fp = reinterpret_cast<float*>(p.c) + base + n;
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
+      if (g * 8 < nvalid) {
+        *reinterpret_cast<float4*>(fp + g * 8) =
+            make_float4(v[g * 8 + 0], v[g * 8 + 1], v[g * 8 + 2], v[g * 8 + 3]);
+        *reinterpret_cast<float4*>(fp + g * 8 + 4) =
+            make_float4(v[g * 8 + 4], v[g * 8 + 5], v[g * 8 + 6], v[g * 8 + 7]);
+      }
+    }
+  } else if (p.out_f16) {
     bool over = false;
 #pragma unroll
     for (int g = 0; g < 4; ++g) {

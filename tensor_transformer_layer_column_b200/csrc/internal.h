@@ -35,6 +35,8 @@ struct GemmProblem {
   const void* bias;
   long long c_ms, c_ns, ldc;
   bool out_f16;              // store C / C2 as fp16
+  bool out_f32;              // store C as fp32 (EPI_LINEAR only)
+  bool aux_f32;              // aux is an fp32 residual (EPI_LINEAR only)
 };
 
 tp_status launch_gemm(const GemmProblem& g, cudaStream_t stream);
@@ -58,7 +60,13 @@ size_t layernorm_bwd_partial_floats(long long rows, int D);
 tp_status launch_layernorm_bwd(const uint16_t* dy, const uint16_t* x, const uint16_t* g,
                                const float* mean, const float* rstd, const uint16_t* dres,
                                long long rows, int D, uint16_t* dx, uint16_t* dg, uint16_t* db,
-                               float* partial, cudaStream_t stream);
+                               float* partial, cudaStream_t stream, float* dx32 = nullptr);
+
+// fp32 upstream gradient dy; dx is written bf16 and, when dx32 is set, also fp32.
+tp_status launch_layernorm_bwd_f32(const float* dy, const uint16_t* x, const uint16_t* g,
+                                   const float* mean, const float* rstd, long long rows, int D,
+                                   uint16_t* dx, float* dx32, uint16_t* dg, uint16_t* db,
+                                   float* partial, cudaStream_t stream);
 
 tp_status launch_layernorm_bwd_blocks(const uint16_t* dy, const uint16_t* x, const uint16_t* g,
                                       const float* mean, const float* rstd, const uint16_t* dres,

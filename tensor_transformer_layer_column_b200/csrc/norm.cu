@@ -144,12 +144,37 @@ constexpr int LNB_THREADS = 256;
 // tid, tid+256, ...; the next row's operands are loaded while the current
 // row goes through its block reduction.  Per-block dgamma/dbeta partials go to
 // `partial` [gridDim.x][2][D] and are reduced by ln_param_reduce in block order.
-template <int CH>
+// Eight consecutive elements of the upstream gradient, bf16 or fp32.
+template <bool F32>
+struct DyChunk {
+  uint4 v;
+  __device__ __forceinline__ void load(const void* p, long long off) {
+    v = *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p) + off);
+  }
+  __device__ __forceinline__ void get(float (&o)[8]) const { unpack8(v, o); }
+};
+template <>
+struct DyChunk<true> {
+  float4 a, b;
+  __device__ __forceinline__ void load(const void* p, long long off) {
+    const float* q = static_cast<const float*>(p) + off;
+    a = *reinterpret_cast<const float4*>(q);
+    b = *reinterpret_cast<const float4*>(q + 4);
+  }
+  __device__ __forceinline__ void get(float (&o)[8]) const {
+    o[0] = a.x; o[1] = a.y; o[2] = a.z; o[3] = a.w;
+    o[4] = b.x; o[5] = b.y; o[6] = b.z; o[7] = b.w;
+  }
+};
+
+// DY32: dy is fp32.  dx32, when set, receives an fp32 copy of dx.
+template <int CH, bool DY32 = false>
 __global__ void __launch_bounds__(LNB_THREADS, 2)
-ln_bwd_kernel(const uint16_t* __restrict__ dy, const uint16_t* __restrict__ x,
+ln_bwd_kernel(const void* __restrict__ dy, const uint16_t* __restrict__ x,
               const uint16_t* __restrict__ g, const float* __restrict__ mean,
               const float* __restrict__ rstd, const uint16_t* __restrict__ dres, long long rows,
-              int D, int rows_per_block, uint16_t* __restrict__ dx, float* __restrict__ partial) {
+              int D, int rows_per_block, uint16_t* __restrict__ dx, float* __restrict__ partial,
+              float* __restrict__ dx32 = nullptr) {
   __shared__ float red[2][2][LNB_THREADS / 32];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int nch = D >> 3;
@@ -164,13 +189,14 @@ ln_bwd_kernel(const uint16_t* __restrict__ dy, const uint16_t* __restrict__ x,
   const long long r0 = (long long)blockIdx.x * rows_per_block;
   const long long r1 = min(rows, r0 + rows_per_block);
   const float invD = 1.0f / D;
-  uint4 cdy[CH], cx[CH], cres[CH];
-  auto load_row = [&](long long r, uint4 (&ody)[CH], uint4 (&ox)[CH], uint4 (&ores)[CH]) {
+  DyChunk<DY32> cdy[CH];
+  uint4 cx[CH], cres[CH];
+  auto load_row = [&](long long r, DyChunk<DY32> (&ody)[CH], uint4 (&ox)[CH], uint4 (&ores)[CH]) {
 #pragma unroll
     for (int j = 0; j < CH; ++j) {
       const int c = tid + LNB_THREADS * j;
       if (c < nch) {
-        ody[j] = *reinterpret_cast<const uint4*>(dy + r * D + c * 8);
+        ody[j].load(dy, r * D + c * 8);
         ox[j] = *reinterpret_cast<const uint4*>(x + r * D + c * 8);
         if (dres != nullptr) ores[j] = *reinterpret_cast<const uint4*>(dres + r * D + c * 8);
       }
@@ -179,7 +205,8 @@ ln_bwd_kernel(const uint16_t* __restrict__ dy, const uint16_t* __restrict__ x,
   if (r0 < r1) load_row(r0, cdy, cx, cres);
   int buf = 0;
   for (long long r = r0; r < r1; ++r, buf ^= 1) {
-    uint4 ndy[CH], nx[CH], nres[CH];
+    DyChunk<DY32> ndy[CH];
+    uint4 nx[CH], nres[CH];
     if (r + 1 < r1) load_row(r + 1, ndy, nx, nres);
     const float mu = mean[r], rs = rstd[r];
     float xh[CH][8], gv[CH][8];
@@ -188,7 +215,7 @@ ln_bwd_kernel(const uint16_t* __restrict__ dy, const uint16_t* __restrict__ x,
     for (int j = 0; j < CH; ++j) {
       if (tid + LNB_THREADS * j < nch) {
         float dv[8];
-        unpack8(cdy[j], dv);
+        cdy[j].get(dv);
         unpack8(cx[j], xh[j]);
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
@@ -230,6 +257,11 @@ ln_bwd_kernel(const uint16_t* __restrict__ dy, const uint16_t* __restrict__ x,
           for (int e = 0; e < 8; ++e) o[e] += rv[e];
         }
         *reinterpret_cast<uint4*>(dx + r * D + c * 8) = pack8(o);
+        if (dx32 != nullptr) {
+          float* q = dx32 + r * D + c * 8;
+          *reinterpret_cast<float4*>(q) = make_float4(o[0], o[1], o[2], o[3]);
+          *reinterpret_cast<float4*>(q + 4) = make_float4(o[4], o[5], o[6], o[7]);
+        }
       }
     }
 #pragma unroll
@@ -431,43 +463,12 @@ size_t layernorm_bwd_partial_floats(long long rows, int D) {
   return (size_t)ln_bwd_blocks(rows < 1 ? 1 : rows) * 2 * (size_t)D;
 }
 
-tp_status launch_layernorm_bwd(const uint16_t* dy, const uint16_t* x, const uint16_t* g,
-                               const float* mean, const float* rstd, const uint16_t* dres,
-                               long long rows, int D, uint16_t* dx, uint16_t* dg, uint16_t* db,
-                               float* partial, cudaStream_t stream) {
-  if (rows == 0) {
-    if (dg) cudaMemsetAsync(dg, 0, (size_t)D * 2, stream);
-    if (db) cudaMemsetAsync(db, 0, (size_t)D * 2, stream);
-    return cuda_status(cudaGetLastError());
-  }
-  const int nb = ln_bwd_blocks(rows);
-  const int rpb = (int)((rows + nb - 1) / nb);
-  const int per_thread = (D / 8 + LNB_THREADS - 1) / LNB_THREADS;
-  {
-  TraceScope ts(stream, TK_LN_BWD);
-  if (per_thread <= 1)
-    ln_bwd_kernel<1><<<nb, LNB_THREADS, 0, stream>>>(dy, x, g, mean, rstd, dres, rows, D, rpb, dx, partial);
-  else if (per_thread <= 2)
-    ln_bwd_kernel<2><<<nb, LNB_THREADS, 0, stream>>>(dy, x, g, mean, rstd, dres, rows, D, rpb, dx, partial);
-  else if (per_thread <= 4)
-    ln_bwd_kernel<4><<<nb, LNB_THREADS, 0, stream>>>(dy, x, g, mean, rstd, dres, rows, D, rpb, dx, partial);
-  else
-    return TP_ERR_UNSUPPORTED;
-  }
-  if (dg != nullptr || db != nullptr) {
-    TraceScope ts(stream, TK_LN_PARAM);
-    ln_param_reduce<<<(2 * D + 31) / 32, 256, 0, stream>>>(partial, nb, D, dg, db);
-  }
-  return cuda_status(cudaGetLastError());
-}
-
-// LayerNorm backward with a caller-chosen number of row blocks `nb` (>= 1):
-// `partial` must hold nb * 2 * D floats.  Used by the entry point whose
-// scratch is a fixed-size static array.
-tp_status launch_layernorm_bwd_blocks(const uint16_t* dy, const uint16_t* x, const uint16_t* g,
-                                      const float* mean, const float* rstd, const uint16_t* dres,
-                                      long long rows, int D, uint16_t* dx, uint16_t* dg,
-                                      uint16_t* db, int nb, float* partial, cudaStream_t stream) {
+namespace {
+template <bool DY32>
+tp_status ln_bwd_launch(const void* dy, const uint16_t* x, const uint16_t* g, const float* mean,
+                        const float* rstd, const uint16_t* dres, long long rows, int D,
+                        uint16_t* dx, float* dx32, uint16_t* dg, uint16_t* db, int nb,
+                        float* partial, cudaStream_t stream) {
   if (rows == 0) {
     if (dg) cudaMemsetAsync(dg, 0, (size_t)D * 2, stream);
     if (db) cudaMemsetAsync(db, 0, (size_t)D * 2, stream);
@@ -479,11 +480,14 @@ tp_status launch_layernorm_bwd_blocks(const uint16_t* dy, const uint16_t* x, con
   {
     TraceScope ts(stream, TK_LN_BWD);
     if (per_thread <= 1)
-      ln_bwd_kernel<1><<<nb, LNB_THREADS, 0, stream>>>(dy, x, g, mean, rstd, dres, rows, D, rpb, dx, partial);
+      ln_bwd_kernel<1, DY32><<<nb, LNB_THREADS, 0, stream>>>(dy, x, g, mean, rstd, dres, rows, D,
+                                                              rpb, dx, partial, dx32);
     else if (per_thread <= 2)
-      ln_bwd_kernel<2><<<nb, LNB_THREADS, 0, stream>>>(dy, x, g, mean, rstd, dres, rows, D, rpb, dx, partial);
+      ln_bwd_kernel<2, DY32><<<nb, LNB_THREADS, 0, stream>>>(dy, x, g, mean, rstd, dres, rows, D,
+                                                              rpb, dx, partial, dx32);
     else if (per_thread <= 4)
-      ln_bwd_kernel<4><<<nb, LNB_THREADS, 0, stream>>>(dy, x, g, mean, rstd, dres, rows, D, rpb, dx, partial);
+      ln_bwd_kernel<4, DY32><<<nb, LNB_THREADS, 0, stream>>>(dy, x, g, mean, rstd, dres, rows, D,
+                                                              rpb, dx, partial, dx32);
     else
       return TP_ERR_UNSUPPORTED;
   }
@@ -492,6 +496,34 @@ tp_status launch_layernorm_bwd_blocks(const uint16_t* dy, const uint16_t* x, con
     ln_param_reduce<<<(2 * D + 31) / 32, 256, 0, stream>>>(partial, nb, D, dg, db);
   }
   return cuda_status(cudaGetLastError());
+}
+}  // namespace
+
+tp_status launch_layernorm_bwd(const uint16_t* dy, const uint16_t* x, const uint16_t* g,
+                               const float* mean, const float* rstd, const uint16_t* dres,
+                               long long rows, int D, uint16_t* dx, uint16_t* dg, uint16_t* db,
+                               float* partial, cudaStream_t stream, float* dx32) {
+  return ln_bwd_launch<false>(dy, x, g, mean, rstd, dres, rows, D, dx, dx32, dg, db,
+                              ln_bwd_blocks(rows < 1 ? 1 : rows), partial, stream);
+}
+
+tp_status launch_layernorm_bwd_f32(const float* dy, const uint16_t* x, const uint16_t* g,
+                                   const float* mean, const float* rstd, long long rows, int D,
+                                   uint16_t* dx, float* dx32, uint16_t* dg, uint16_t* db,
+                                   float* partial, cudaStream_t stream) {
+  return ln_bwd_launch<true>(dy, x, g, mean, rstd, nullptr, rows, D, dx, dx32, dg, db,
+                             ln_bwd_blocks(rows < 1 ? 1 : rows), partial, stream);
+}
+
+// LayerNorm backward with a caller-chosen number of row blocks `nb` (>= 1):
+// `partial` must hold nb * 2 * D floats.  Used by the entry point whose
+// scratch is a fixed-size static array.
+tp_status launch_layernorm_bwd_blocks(const uint16_t* dy, const uint16_t* x, const uint16_t* g,
+                                      const float* mean, const float* rstd, const uint16_t* dres,
+                                      long long rows, int D, uint16_t* dx, uint16_t* dg,
+                                      uint16_t* db, int nb, float* partial, cudaStream_t stream) {
+  return ln_bwd_launch<false>(dy, x, g, mean, rstd, dres, rows, D, dx, nullptr, dg, db, nb,
+                              partial, stream);
 }
 
 }  // namespace tp

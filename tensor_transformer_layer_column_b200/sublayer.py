@@ -13,7 +13,8 @@ from typing import Dict, Optional
 import torch
 
 from . import (Dims, OP_ATTN_BWD, OP_ATTN_FWD, OP_LAYER_BWD, OP_LAYER_FWD, OP_MLP_BWD,
-               attn_bwd, attn_fwd, layer_bwd,
+               OP_POSTLN_BWD, OP_POSTLN_FWD, attn_bwd, attn_fwd, layer_bwd, postln_layer_bwd,
+               postln_layer_fwd,
                layer_fwd, mlp_bwd, mlp_fwd, shard_cols, shard_qkv_heads, shard_rows,
                unshard_cols, unshard_qkv_heads, workspace_size)
 
@@ -158,9 +159,13 @@ LAYER_PARAM_NAMES = ("ln1_g", "ln1_b", "wqkv", "bqkv", "wout", "bout", "ln2_g", 
 
 
 class ShardedLayer:
-    """Pre-LN layer: h = x + Attn(LN1(x)); y = h + MLP(LN2(h))."""
+    """Pre-LN layer h = x + Attn(LN1(x)); y = h + MLP(LN2(h)), or with
+    placement="post" the post-LN layer h = LN1(x + Attn(x)); y = LN2(h + MLP(h))."""
 
-    def __init__(self, dims: Dims, p: Dict[str, torch.Tensor]):
+    def __init__(self, dims: Dims, p: Dict[str, torch.Tensor], placement: str = "pre"):
+        if placement not in ("pre", "post"):
+            raise ValueError("placement is 'pre' or 'post'")
+        self.post = placement == "post"
         self.dims = dims
         t, H = dims.t, dims.heads
         self.device = p["w1"].device
@@ -185,6 +190,15 @@ class ShardedLayer:
         f32 = torch.float32
         dev = self.device
         f16 = torch.float16
+        if self.post:
+            return {"z1": _empty((T, D), device=dev), "mean1": _empty((T,), f32, dev),
+                    "rstd1": _empty((T,), f32, dev), "qkv": _empty((t, T, 3 * D // t), f16, dev),
+                    "o": _empty((t, T, D // t), device=dev),
+                    "lse": _empty((d.batch, d.heads, d.seq), f32, dev),
+                    "h": _empty((T, D), device=dev), "z2": _empty((T, D), device=dev),
+                    "mean2": _empty((T,), f32, dev), "rstd2": _empty((T,), f32, dev),
+                    "a": _empty((t, T, F // t), device=dev),
+                    "hact": _empty((t, T, F // t), device=dev)}
         return {"u1": _empty((T, D), f16, dev), "mean1": _empty((T,), f32, dev),
                 "rstd1": _empty((T,), f32, dev), "qkv": _empty((t, T, 3 * D // t), f16, dev),
                 "o": _empty((t, T, D // t), device=dev),
@@ -210,8 +224,8 @@ class ShardedLayer:
         acts = acts if acts is not None else self.alloc_acts()
         y = y if y is not None else _empty((d.batch * d.seq, d.hidden), device=self.device)
         if self.ws_fwd is None:
-            self.ws_fwd = _ws(OP_LAYER_FWD, d, self.device)
-        layer_fwd(d, x, self.p, acts, y, self.ws_fwd)
+            self.ws_fwd = _ws(OP_POSTLN_FWD if self.post else OP_LAYER_FWD, d, self.device)
+        (postln_layer_fwd if self.post else layer_fwd)(d, x, self.p, acts, y, self.ws_fwd)
         self.saved = (x, acts)
         return y, acts
 
@@ -219,8 +233,8 @@ class ShardedLayer:
         d = self.dims
         x, acts = self.saved
         if self.ws is None:
-            self.ws = _ws(OP_LAYER_BWD, d, self.device)
+            self.ws = _ws(OP_POSTLN_BWD if self.post else OP_LAYER_BWD, d, self.device)
         dx = dx if dx is not None else torch.empty_like(x)
         grads = grads if grads is not None else self.alloc_grads(bias_grads)
-        layer_bwd(d, x, self.p, acts, dy, dx, grads, self.ws)
+        (postln_layer_bwd if self.post else layer_bwd)(d, x, self.p, acts, dy, dx, grads, self.ws)
         return dx, grads

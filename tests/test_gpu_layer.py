@@ -68,3 +68,52 @@ def test_layer_full_size_B4_S2048_D4096_H32_F16384_t8():
     require_gpu()
     w = workload("layer_fwdbwd_B4_S2048_D4096_H32_F16384_t8")
     _run_and_compare(w, make_inputs(w))
+
+
+# ---------------------------------------------------------------- post-LN layer
+
+def _run_and_compare_postln(w, inp):
+    d = dims_of(w)
+    g = dev(inp)
+    layer = ShardedLayer(d, {k: g[k] for k in PARAMS}, placement="post")
+    y, acts = layer.forward(g["x"])
+    dx, grads = layer.backward(g["dy"])
+    torch.cuda.synchronize()
+    assert_no_device_error()
+    t = w.t
+    p = {k: to_f64(inp[k]) for k in PARAMS}
+    x = to_f64(inp["x"])
+    yr, sv = olayer.postln_layer_fwd(x, p, w.batch, w.heads, w.causal, w.ln_eps)
+    check("y", y, yr)
+    for k in ("z1", "h", "z2"):
+        check(k, acts[k], sv[k])
+    check("a", acts["a"], olay.shard_cols(sv["a"], t))
+    gr = olayer.postln_layer_bwd(x, p, to_f64(inp["dy"]), w.batch, w.heads, w.causal, w.ln_eps)
+    check("dx", dx, gr["dx"])
+    check("dwqkv", grads["dwqkv"], olay.shard_qkv(gr["dwqkv"], t))
+    check("dbqkv", grads["dbqkv"], olay.shard_qkv(gr["dbqkv"][None, :], t))
+    check("dwout", grads["dwout"], olay.shard_rows(gr["dwout"], t))
+    check("dbout", grads["dbout"], gr["dbout"])
+    check("dw1", grads["dw1"], olay.shard_cols(gr["dw1"], t))
+    check("db1", grads["db1"], gr["db1"])
+    check("dw2", grads["dw2"], olay.shard_rows(gr["dw2"], t))
+    check("db2", grads["db2"], gr["db2"])
+    for k in ("dln1_g", "dln1_b", "dln2_g", "dln2_b"):
+        check(k, grads[k], gr[k])
+
+
+@pytest.mark.parametrize("B,S,H,dh,F,t", [(2, 128, 4, 64, 1024, 2), (1, 200, 2, 128, 1024, 2),
+                                          (2, 96, 8, 64, 2048, 8)])
+@pytest.mark.parametrize("affine", [False, True])
+def test_postln_layer_fwd_bwd_small(B, S, H, dh, F, t, affine):
+    require_gpu()
+    w = Workload("postln_test", "layer_fwdbwd", batch=B, seq=S, hidden=H * dh, ffn=F, heads=H,
+                 head_dim=dh, t=t)
+    _run_and_compare_postln(w, make_inputs(w, seed=17, random_affine=affine))
+
+
+def test_postln_layer_full_size_B4_S2048_D4096_H32_F16384_t8():
+    """The post-LN arm at the pre-LN layer's full size, every output and gradient."""
+    require_gpu()
+    w = workload("layer_fwdbwd_B4_S2048_D4096_H32_F16384_t8")
+    _run_and_compare_postln(w, make_inputs(w))
