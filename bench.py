@@ -211,7 +211,8 @@ class Runner:
                           1 if w.causal else 0, w.ln_eps)
         if w.kind.startswith("layer"):
             self.mod = ShardedLayer(dims, {k: g[k] for k in PARAMS},
-                                    placement="post" if "postln" in w.kind else "pre")
+                                    placement="post" if "postln" in w.kind else "pre",
+                                    recompute="recompute" in w.kind)
             self.acts = self.mod.alloc_acts()
             self.grads = self.mod.alloc_grads()
         elif w.kind.startswith("attn"):
@@ -238,6 +239,25 @@ class Runner:
                 self.bwd_out = self.mod.backward(dy)
                 self.bwd_out["dx"] = self.dx
             self.mod.backward(dy, out=self.bwd_out)
+
+
+def recompute_flops(w: Workload) -> int:
+    """FLOPs the recomputing backward adds: the forward without the MLP's
+    second product (QKV and output projections, causal core, W1 product)."""
+    pairs = w.seq * (w.seq + 1) // 2 if w.causal else w.seq * w.seq
+    return (8 * w.tokens * w.hidden * w.hidden + 4 * w.head_dim * w.batch * w.heads * pairs
+            + 2 * w.tokens * w.hidden * w.ffn)
+
+
+def activation_report(w: Workload, mod) -> dict:
+    """Activation memory held from forward to backward, and the recomputation cost."""
+    rec = bool(getattr(mod, "recompute", False))
+    out = {"held_bytes_per_layer": mod.saved_bytes(), "recompute": rec}
+    if rec:
+        out["recompute_flop_per_step"] = recompute_flops(w)
+        out["note"] = ("value counts algorithmic FLOPs only; the recomputed forward's FLOPs "
+                       "are extra work inside the timed step")
+    return out
 
 
 def run_ours(args):
@@ -386,6 +406,8 @@ def run_ours(args):
             "clocks": clock,
             "cpu_baseline": cpu,
         }
+        if w.kind.startswith("layer"):
+            line["activations"] = activation_report(w, run.mod)
         print(json.dumps(line), flush=True)
     if world > 1:
         torch.distributed.destroy_process_group()

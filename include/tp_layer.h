@@ -89,7 +89,9 @@ typedef enum {
   TP_OP_LAYER_FWD = 4,
   TP_OP_LAYER_BWD = 5,
   TP_OP_POSTLN_FWD = 6,
-  TP_OP_POSTLN_BWD = 7
+  TP_OP_POSTLN_BWD = 7,
+  TP_OP_LAYER_FWD_NOSAVE = 8,
+  TP_OP_LAYER_BWD_RECOMPUTE = 9
 } tp_op;
 
 /* Version string of the library. */
@@ -246,6 +248,33 @@ tp_status tp_layer_fwd(const tp_dims* dims, const tp_bf16* x, const tp_layer_par
 tp_status tp_layer_bwd(const tp_dims* dims, const tp_bf16* x, const tp_layer_params* params,
                        const tp_layer_acts* acts, const tp_bf16* dy, tp_bf16* dx,
                        const tp_layer_grads* grads, void* ws, size_t ws_bytes, tp_stream stream);
+
+/* ------------------------------------------------------------------ activation recomputation
+ * "What actually limits throughput in production", the activation memory vs.
+ * recomputation trade-off: instead of keeping the layer's activations from
+ * the forward to the backward pass, keep only the layer input x and compute
+ * them again at the start of the backward pass.
+ *
+ * tp_layer_fwd_nosave: the pre-LN forward (same result as tp_layer_fwd, bit
+ *   for bit) with every intermediate in the workspace; nothing outlives the
+ *   call but y.  Workspace: tp_workspace_size(TP_OP_LAYER_FWD_NOSAVE, dims),
+ *   about T*(10D + 4F) bytes + the fp16 copy of Wqkv; callers running many
+ *   layers can share one workspace between them.
+ * tp_layer_bwd_recompute: recomputes the activations of tp_layer_fwd from x
+ *   and params into the workspace, then runs tp_layer_bwd on them.  The
+ *   recomputed forward leaves out the MLP's second product (y is not needed
+ *   for any gradient): 2*T*D*F + 8*T*D^2 + the causal core's forward FLOPs on
+ *   top of the backward's.  dx and *grads equal tp_layer_bwd's bit for bit
+ *   (same kernels on the same inputs; the library is deterministic).
+ *   Workspace: tp_workspace_size(TP_OP_LAYER_BWD_RECOMPUTE, dims) bytes.
+ * Arguments, layouts and errors as tp_layer_fwd / tp_layer_bwd. */
+tp_status tp_layer_fwd_nosave(const tp_dims* dims, const tp_bf16* x,
+                              const tp_layer_params* params, tp_bf16* y, void* ws,
+                              size_t ws_bytes, tp_stream stream);
+tp_status tp_layer_bwd_recompute(const tp_dims* dims, const tp_bf16* x,
+                                 const tp_layer_params* params, const tp_bf16* dy, tp_bf16* dx,
+                                 const tp_layer_grads* grads, void* ws, size_t ws_bytes,
+                                 tp_stream stream);
 
 /* ------------------------------------------------------------------ post-LN layer
  * The other placement in "The layernorm placement the paper flags as

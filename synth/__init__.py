@@ -97,13 +97,16 @@ WORKLOADS: Dict[str, Workload] = {w.name: w for w in [
 ]}
 
 # Beyond the five: a profiling case (the layer's attention sublayer at half the
-# batch; inputs exceed L2 but it holds < 1 GB) and the post-LN arm of the
-# layer-norm placement passage at the pre-LN layer's size.
+# batch; inputs exceed L2 but it holds < 1 GB), the post-LN arm of the
+# layer-norm placement passage at the pre-LN layer's size, and the pre-LN layer
+# with activation recomputation (nothing kept between forward and backward).
 EXTRA_WORKLOADS: Dict[str, Workload] = {w.name: w for w in [
     Workload("attn_fwdbwd_B2_S2048_D4096_H32_t8", "attn_fwdbwd", batch=2, seq=2048, hidden=4096,
              heads=32, head_dim=128, t=8),
     Workload("layer_postln_fwdbwd_B4_S2048_D4096_H32_F16384_t8", "layer_postln_fwdbwd", batch=4,
              seq=2048, hidden=4096, ffn=16384, heads=32, head_dim=128, t=8),
+    Workload("layer_recompute_fwdbwd_B4_S2048_D4096_H32_F16384_t8", "layer_recompute_fwdbwd",
+             batch=4, seq=2048, hidden=4096, ffn=16384, heads=32, head_dim=128, t=8),
 ]}
 
 

@@ -19,6 +19,7 @@ __all__ = [
     "TpError", "Dims", "LayerParams", "LayerActs", "PostLNActs", "LayerGrads", "lib", "lib_path",
     "OP_MLP_FWD", "OP_MLP_BWD", "OP_ATTN_FWD", "OP_ATTN_BWD", "OP_LAYER_FWD", "OP_LAYER_BWD",
     "OP_POSTLN_FWD", "OP_POSTLN_BWD", "postln_layer_fwd", "postln_layer_bwd",
+    "OP_LAYER_FWD_NOSAVE", "OP_LAYER_BWD_RECOMPUTE", "layer_fwd_nosave", "layer_bwd_recompute",
     "workspace_size", "check_error", "version", "EXPORTED_SYMBOLS",
     "shard_cols", "unshard_cols", "shard_rows", "unshard_rows", "shard_qkv_heads",
     "unshard_qkv_heads", "mlp_fwd", "mlp_bwd", "attn_fwd", "attn_bwd", "layer_fwd", "layer_bwd",
@@ -31,7 +32,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 lib_path = os.path.join(_HERE, "libtplayer.so")
 
 (OP_MLP_FWD, OP_MLP_BWD, OP_ATTN_FWD, OP_ATTN_BWD, OP_LAYER_FWD, OP_LAYER_BWD, OP_POSTLN_FWD,
- OP_POSTLN_BWD) = range(8)
+ OP_POSTLN_BWD, OP_LAYER_FWD_NOSAVE, OP_LAYER_BWD_RECOMPUTE) = range(10)
 
 STATUS_NAMES = {0: "TP_OK", 1: "TP_ERR_INVALID_ARG", 2: "TP_ERR_UNSUPPORTED",
                 3: "TP_ERR_MISALIGNED", 4: "TP_ERR_WORKSPACE", 5: "TP_ERR_CUDA",
@@ -103,6 +104,10 @@ _SIGS = {
     "tp_postln_layer_bwd": [ctypes.POINTER(Dims), _P, ctypes.POINTER(LayerParams),
                             ctypes.POINTER(PostLNActs), _P, _P, ctypes.POINTER(LayerGrads), _P,
                             ctypes.c_size_t, _P],
+    "tp_layer_fwd_nosave": [ctypes.POINTER(Dims), _P, ctypes.POINTER(LayerParams), _P, _P,
+                            ctypes.c_size_t, _P],
+    "tp_layer_bwd_recompute": [ctypes.POINTER(Dims), _P, ctypes.POINTER(LayerParams), _P, _P,
+                               ctypes.POINTER(LayerGrads), _P, ctypes.c_size_t, _P],
     "tp_layernorm_fwd": [_P, _P, _P, ctypes.c_int, ctypes.c_int, ctypes.c_float, _P, _P, _P, _P],
     "tp_layernorm_bwd_workspace_size": [ctypes.c_int, ctypes.c_int],
     "tp_layernorm_bwd": [_P, _P, _P, _P, _P, _P, ctypes.c_int, ctypes.c_int, _P, _P, _P, _P,
@@ -286,6 +291,22 @@ def postln_layer_bwd(dims, x, params: dict, acts: dict, dy, dx, grads: dict, ws,
     _check(lib().tp_postln_layer_bwd(ctypes.byref(dims), _ptr(x), ctypes.byref(p), ctypes.byref(a),
                                      _ptr(dy), _ptr(dx), ctypes.byref(g), wp, wn,
                                      _stream(stream, x)), "tp_postln_layer_bwd")
+
+
+def layer_fwd_nosave(dims, x, params: dict, y, ws, stream=None):
+    wp, wn = _ws(ws)
+    p = _struct(LayerParams, params)
+    _check(lib().tp_layer_fwd_nosave(ctypes.byref(dims), _ptr(x), ctypes.byref(p), _ptr(y), wp, wn,
+                                     _stream(stream, x)), "tp_layer_fwd_nosave")
+
+
+def layer_bwd_recompute(dims, x, params: dict, dy, dx, grads: dict, ws, stream=None):
+    wp, wn = _ws(ws)
+    p = _struct(LayerParams, params)
+    g = _struct(LayerGrads, grads)
+    _check(lib().tp_layer_bwd_recompute(ctypes.byref(dims), _ptr(x), ctypes.byref(p), _ptr(dy),
+                                        _ptr(dx), ctypes.byref(g), wp, wn, _stream(stream, x)),
+           "tp_layer_bwd_recompute")
 
 
 def layernorm_fwd(x, gamma, beta, rows, D, eps, y, mean, rstd, stream=None):

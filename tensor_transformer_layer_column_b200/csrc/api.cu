@@ -184,7 +184,7 @@ tp_status mlp_fwd_impl(const Sizes& z, bf16p x, bf16p w1, bf16p b1, bf16p w2, bf
   g1.epi = EPI_BIAS_GELU; g1.c = a_save; g1.c2 = h_save; g1.bias = b1;
   g1.c_ms = 0; g1.c_ns = z.T * z.Ft; g1.ldc = z.Ft;
   tp_status s = launch_gemm(g1, st);
-  if (s != TP_OK) return s;
+  if (s != TP_OK || y == nullptr) return s;   // y == nullptr: A and H only (recomputation)
 
   GemmProblem g2{};
   g2.m_shards = 1; g2.n_shards = 1; g2.Mt = (int)z.T; g2.Nt = (int)z.D;
@@ -406,6 +406,34 @@ size_t layer_bwd_ws(const Sizes& z) {
   return align_up(c.off, 256);
 }
 
+// The pre-LN layer's saved activations carved out of a workspace (the
+// recomputation entry points keep them there instead of in caller buffers).
+tp_layer_acts carve_layer_acts(Carver& c, const Sizes& z) {
+  tp_layer_acts a{};
+  a.u1 = c.take<uint16_t>((size_t)(z.T * z.D));
+  a.mean1 = c.take<float>((size_t)z.T);
+  a.rstd1 = c.take<float>((size_t)z.T);
+  a.qkv = c.take<uint16_t>((size_t)(z.T * 3 * z.D));
+  a.o = c.take<uint16_t>((size_t)(z.T * z.D));
+  a.lse = c.take<float>((size_t)(z.B * z.H * z.S));
+  a.h = c.take<uint16_t>((size_t)(z.T * z.D));
+  a.u2 = c.take<uint16_t>((size_t)(z.T * z.D));
+  a.mean2 = c.take<float>((size_t)z.T);
+  a.rstd2 = c.take<float>((size_t)z.T);
+  a.a = c.take<uint16_t>((size_t)(z.T * z.F));
+  a.hact = c.take<uint16_t>((size_t)(z.T * z.F));
+  return a;
+}
+
+size_t layer_acts_ws(const Sizes& z) {
+  Carver c(nullptr);
+  carve_layer_acts(c, z);
+  return align_up(c.off, 256);
+}
+
+size_t layer_fwd_nosave_ws(const Sizes& z) { return layer_fwd_ws(z) + layer_acts_ws(z); }
+size_t layer_bwd_recompute_ws(const Sizes& z) { return layer_acts_ws(z) + layer_bwd_ws(z); }
+
 // Post-LN layer workspaces: fp16 copies of x and Wqkv (forward and backward),
 // plus the gradient chain, LayerNorm partials and the sublayer workspace
 // (backward).  The chain dz2 -> dh -> dz1 passes through two LayerNorm
@@ -466,6 +494,10 @@ size_t tp_workspace_size(int op_, const tp_dims* d) {
     case TP_OP_LAYER_BWD: return check_layer(d) == TP_OK ? layer_bwd_ws(sizes_of(*d)) : 0;
     case TP_OP_POSTLN_FWD: return check_layer(d) == TP_OK ? postln_fwd_ws(sizes_of(*d)) : 0;
     case TP_OP_POSTLN_BWD: return check_layer(d) == TP_OK ? postln_bwd_ws(sizes_of(*d)) : 0;
+    case TP_OP_LAYER_FWD_NOSAVE:
+      return check_layer(d) == TP_OK ? layer_fwd_nosave_ws(sizes_of(*d)) : 0;
+    case TP_OP_LAYER_BWD_RECOMPUTE:
+      return check_layer(d) == TP_OK ? layer_bwd_recompute_ws(sizes_of(*d)) : 0;
   }
   return 0;
 }
@@ -666,19 +698,17 @@ static tp_status check_layer_ptrs(const tp_layer_params* p, const tp_layer_acts*
   return TP_OK;
 }
 
-tp_status tp_layer_fwd(const tp_dims* dims, const tp_bf16* x, const tp_layer_params* p,
-                       const tp_layer_acts* a, tp_bf16* y, void* ws, size_t ws_bytes, tp_stream s) {
-  tp_status st = check_layer(dims);
-  if (st != TP_OK) return st;
-  if (!x || !y) return TP_ERR_INVALID_ARG;
-  if ((st = check_layer_ptrs(p, a)) != TP_OK) return st;
-  if (!all_aligned(x, y)) return TP_ERR_MISALIGNED;
-  const Sizes z = sizes_of(*dims);
-  cudaStream_t cs = (cudaStream_t)s;
-  if (z.T == 0) return TP_OK;
-  if ((st = check_ws(ws, ws_bytes, layer_fwd_ws(z))) != TP_OK) return st;
-  uint16_t* w16 = static_cast<uint16_t*>(ws);
-  if ((st = launch_cast_f16(p->wqkv, (size_t)(z.D * 3 * z.D), w16, cs)) != TP_OK) return st;
+}  // extern "C"
+
+namespace tp {
+namespace {
+
+// Pre-LN forward on activations `a`, with the fp16 copy of Wqkv already in
+// w16.  y == nullptr leaves out the MLP's second product (recomputation).
+tp_status layer_fwd_core(const Sizes& z, const tp_dims* dims, const tp_bf16* x,
+                         const tp_layer_params* p, const tp_layer_acts* a, tp_bf16* y,
+                         const uint16_t* w16, cudaStream_t cs) {
+  tp_status st;
   // LN1 writes u1 in fp16: it only feeds the attention sublayer's fp16 products.
   if ((st = launch_layernorm_fwd(x, p->ln1_g, p->ln1_b, z.T, (int)z.D, dims->ln_eps, a->u1,
                                  a->mean1, a->rstd1, cs, true)) != TP_OK)
@@ -692,30 +722,12 @@ tp_status tp_layer_fwd(const tp_dims* dims, const tp_bf16* x, const tp_layer_par
   return mlp_fwd_impl(z, a->u2, p->w1, p->b1, p->w2, p->b2, a->h, y, a->a, a->hact, cs);
 }
 
-tp_status tp_layer_bwd(const tp_dims* dims, const tp_bf16* x, const tp_layer_params* p,
-                       const tp_layer_acts* a, const tp_bf16* dy, tp_bf16* dx,
-                       const tp_layer_grads* g, void* ws, size_t ws_bytes, tp_stream s) {
-  tp_status st = check_layer(dims);
-  if (st != TP_OK) return st;
-  if (!x || !dy || !dx || !g) return TP_ERR_INVALID_ARG;
-  if ((st = check_layer_ptrs(p, a)) != TP_OK) return st;
-  if (!all_set(g->dwqkv, g->dwout, g->dw1, g->dw2)) return TP_ERR_INVALID_ARG;
-  if (!all_aligned(x, dy, dx, g->dln1_g, g->dln1_b, g->dwqkv, g->dbqkv, g->dwout, g->dbout,
-                   g->dln2_g, g->dln2_b, g->dw1, g->db1, g->dw2, g->db2))
-    return TP_ERR_MISALIGNED;
-  const Sizes z = sizes_of(*dims);
-  const size_t need = z.T ? layer_bwd_ws(z) : 0;
-  if ((st = check_ws(ws, ws_bytes, need)) != TP_OK) return st;
-  cudaStream_t cs = (cudaStream_t)s;
-  if (z.T == 0) {
-    mlp_bwd_impl(z, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, g->dw1,
-                 g->dw2, g->db1, g->db2, nullptr, cs);
-    attn_bwd_impl(z, dims->causal, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
-                  nullptr, nullptr, g->dwqkv, g->dbqkv, g->dwout, g->dbout, nullptr, cs);
-    for (tp_bf16* q : {g->dln1_g, g->dln1_b, g->dln2_g, g->dln2_b})
-      if (q) cudaMemsetAsync(q, 0, (size_t)z.D * 2, cs);
-    return cuda_status(cudaGetLastError());
-  }
+// Pre-LN backward; `ws` is laid out as layer_bwd_ws describes and its first
+// slice already holds the fp16 copy of Wqkv.
+tp_status layer_bwd_core(const Sizes& z, const tp_dims* dims, const tp_bf16* x,
+                         const tp_layer_params* p, const tp_layer_acts* a, const tp_bf16* dy,
+                         tp_bf16* dx, const tp_layer_grads* g, void* ws, cudaStream_t cs) {
+  tp_status st;
   Carver c(ws);
   uint16_t* w16 = c.take<uint16_t>((size_t)(z.D * 3 * z.D));
   uint16_t* du = c.take<uint16_t>((size_t)(z.T * z.D));
@@ -723,7 +735,6 @@ tp_status tp_layer_bwd(const tp_dims* dims, const tp_bf16* x, const tp_layer_par
   float* lnp = c.take<float>(layernorm_bwd_partial_floats(z.T, (int)z.D));
   const size_t sub = mlp_bwd_ws(z) > attn_bwd_core_ws(z) ? mlp_bwd_ws(z) : attn_bwd_core_ws(z);
   void* subws = c.take<uint8_t>(sub);
-  if ((st = launch_cast_f16(p->wqkv, (size_t)(z.D * 3 * z.D), w16, cs)) != TP_OK) return st;
 
   // y = h + MLP(LN2(h)):  du2 = MLP^T(dy);  dh = dy + LN2^T(du2).
   if ((st = mlp_bwd_impl(z, a->u2, p->w1, p->w2, a->a, a->hact, dy, nullptr, du, g->dw1, g->dw2,
@@ -738,6 +749,118 @@ tp_status tp_layer_bwd(const tp_dims* dims, const tp_bf16* x, const tp_layer_par
     return st;
   return launch_layernorm_bwd(du, x, p->ln1_g, a->mean1, a->rstd1, dh, z.T, (int)z.D, dx,
                               g->dln1_g, g->dln1_b, lnp, cs);
+}
+
+tp_status check_layer_params(const tp_layer_params* p) {
+  if (!p) return TP_ERR_INVALID_ARG;
+  if (!all_set(p->ln1_g, p->ln1_b, p->wqkv, p->wout, p->ln2_g, p->ln2_b, p->w1, p->w2))
+    return TP_ERR_INVALID_ARG;
+  if (!all_aligned(p->ln1_g, p->ln1_b, p->wqkv, p->bqkv, p->wout, p->bout, p->ln2_g, p->ln2_b,
+                   p->w1, p->b1, p->w2, p->b2))
+    return TP_ERR_MISALIGNED;
+  return TP_OK;
+}
+
+// Activations (x, dy, dx) may be NULL when the layer has zero tokens.
+tp_status check_layer_grads(const tp_dims* d, const tp_bf16* x, const tp_bf16* dy,
+                            const tp_bf16* dx, const tp_layer_grads* g) {
+  const bool tok = (long long)d->batch * d->seq > 0;
+  if (!g || (tok && !all_set(x, dy, dx))) return TP_ERR_INVALID_ARG;
+  if (!all_set(g->dwqkv, g->dwout, g->dw1, g->dw2)) return TP_ERR_INVALID_ARG;
+  if (!all_aligned(x, dy, dx, g->dln1_g, g->dln1_b, g->dwqkv, g->dbqkv, g->dwout, g->dbout,
+                   g->dln2_g, g->dln2_b, g->dw1, g->db1, g->dw2, g->db2))
+    return TP_ERR_MISALIGNED;
+  return TP_OK;
+}
+
+// Gradients of a layer over zero tokens: every parameter gradient is zero.
+tp_status layer_bwd_empty(const Sizes& z, int causal, const tp_layer_grads* g, cudaStream_t cs) {
+  mlp_bwd_impl(z, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, g->dw1,
+               g->dw2, g->db1, g->db2, nullptr, cs);
+  attn_bwd_impl(z, causal, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
+                nullptr, nullptr, g->dwqkv, g->dbqkv, g->dwout, g->dbout, nullptr, cs);
+  for (tp_bf16* q : {g->dln1_g, g->dln1_b, g->dln2_g, g->dln2_b})
+    if (q) cudaMemsetAsync(q, 0, (size_t)z.D * 2, cs);
+  return cuda_status(cudaGetLastError());
+}
+
+}  // namespace
+}  // namespace tp
+
+extern "C" {
+
+tp_status tp_layer_fwd(const tp_dims* dims, const tp_bf16* x, const tp_layer_params* p,
+                       const tp_layer_acts* a, tp_bf16* y, void* ws, size_t ws_bytes, tp_stream s) {
+  tp_status st = check_layer(dims);
+  if (st != TP_OK) return st;
+  if (!x || !y) return TP_ERR_INVALID_ARG;
+  if ((st = check_layer_ptrs(p, a)) != TP_OK) return st;
+  if (!all_aligned(x, y)) return TP_ERR_MISALIGNED;
+  const Sizes z = sizes_of(*dims);
+  cudaStream_t cs = (cudaStream_t)s;
+  if (z.T == 0) return TP_OK;
+  if ((st = check_ws(ws, ws_bytes, layer_fwd_ws(z))) != TP_OK) return st;
+  uint16_t* w16 = static_cast<uint16_t*>(ws);
+  if ((st = launch_cast_f16(p->wqkv, (size_t)(z.D * 3 * z.D), w16, cs)) != TP_OK) return st;
+  return layer_fwd_core(z, dims, x, p, a, y, w16, cs);
+}
+
+tp_status tp_layer_bwd(const tp_dims* dims, const tp_bf16* x, const tp_layer_params* p,
+                       const tp_layer_acts* a, const tp_bf16* dy, tp_bf16* dx,
+                       const tp_layer_grads* g, void* ws, size_t ws_bytes, tp_stream s) {
+  tp_status st = check_layer(dims);
+  if (st != TP_OK) return st;
+  if ((st = check_layer_ptrs(p, a)) != TP_OK) return st;
+  if ((st = check_layer_grads(dims, x, dy, dx, g)) != TP_OK) return st;
+  const Sizes z = sizes_of(*dims);
+  const size_t need = z.T ? layer_bwd_ws(z) : 0;
+  if ((st = check_ws(ws, ws_bytes, need)) != TP_OK) return st;
+  cudaStream_t cs = (cudaStream_t)s;
+  if (z.T == 0) return layer_bwd_empty(z, dims->causal, g, cs);
+  uint16_t* w16 = static_cast<uint16_t*>(ws);
+  if ((st = launch_cast_f16(p->wqkv, (size_t)(z.D * 3 * z.D), w16, cs)) != TP_OK) return st;
+  return layer_bwd_core(z, dims, x, p, a, dy, dx, g, ws, cs);
+}
+
+tp_status tp_layer_fwd_nosave(const tp_dims* dims, const tp_bf16* x, const tp_layer_params* p,
+                              tp_bf16* y, void* ws, size_t ws_bytes, tp_stream s) {
+  tp_status st = check_layer(dims);
+  if (st != TP_OK) return st;
+  if ((long long)dims->batch * dims->seq > 0 && !all_set(x, y)) return TP_ERR_INVALID_ARG;
+  if ((st = check_layer_params(p)) != TP_OK) return st;
+  if (!all_aligned(x, y)) return TP_ERR_MISALIGNED;
+  const Sizes z = sizes_of(*dims);
+  cudaStream_t cs = (cudaStream_t)s;
+  if (z.T == 0) return TP_OK;
+  if ((st = check_ws(ws, ws_bytes, layer_fwd_nosave_ws(z))) != TP_OK) return st;
+  Carver c(ws);
+  uint16_t* w16 = c.take<uint16_t>((size_t)(z.D * 3 * z.D));
+  c.off = align_up(layer_fwd_ws(z), 256);
+  const tp_layer_acts a = carve_layer_acts(c, z);
+  if ((st = launch_cast_f16(p->wqkv, (size_t)(z.D * 3 * z.D), w16, cs)) != TP_OK) return st;
+  return layer_fwd_core(z, dims, x, p, &a, y, w16, cs);
+}
+
+tp_status tp_layer_bwd_recompute(const tp_dims* dims, const tp_bf16* x, const tp_layer_params* p,
+                                 const tp_bf16* dy, tp_bf16* dx, const tp_layer_grads* g,
+                                 void* ws, size_t ws_bytes, tp_stream s) {
+  tp_status st = check_layer(dims);
+  if (st != TP_OK) return st;
+  if ((st = check_layer_params(p)) != TP_OK) return st;
+  if ((st = check_layer_grads(dims, x, dy, dx, g)) != TP_OK) return st;
+  const Sizes z = sizes_of(*dims);
+  const size_t need = z.T ? layer_bwd_recompute_ws(z) : 0;
+  if ((st = check_ws(ws, ws_bytes, need)) != TP_OK) return st;
+  cudaStream_t cs = (cudaStream_t)s;
+  if (z.T == 0) return layer_bwd_empty(z, dims->causal, g, cs);
+  Carver c(ws);
+  const tp_layer_acts a = carve_layer_acts(c, z);
+  c.off = align_up(layer_acts_ws(z), 256);
+  void* bws = c.take<uint8_t>(layer_bwd_ws(z));
+  uint16_t* w16 = static_cast<uint16_t*>(bws);
+  if ((st = launch_cast_f16(p->wqkv, (size_t)(z.D * 3 * z.D), w16, cs)) != TP_OK) return st;
+  if ((st = layer_fwd_core(z, dims, x, p, &a, nullptr, w16, cs)) != TP_OK) return st;
+  return layer_bwd_core(z, dims, x, p, &a, dy, dx, g, bws, cs);
 }
 
 // ------------------------------------------------------------------ post-LN layer

@@ -74,7 +74,7 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, const C
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait_sleep(bar, parity, 20000)) return true;
     if (*c.abort_flag || globaltimer_ns() - t0 > 2000000000ull) {
       *c.abort_flag = 1;
       if (c.err) atomicCAS(c.err, 0u, code);
@@ -117,14 +117,14 @@ __device__ __forceinline__ uint64_t mnmajor_desc(uint32_t base, int R, int kk) {
 // =====================================================================================
 // Two 128-query tiles per CTA take turns on the tensor core: while one tile's
 // softmax warpgroup works on its scores, the other tile's products run.  Keys
-// come in 64-wide blocks through a 3-stage ring; each tile has its own S (64
+// come in 64-wide blocks through a 4-stage ring; each tile has its own S (64
 // TMEM columns) and O (dh columns).  O is rescaled lazily: only when a row's
 // running max grows by more than 2^8 (log2 units), so P = 2^(s - m_used) stays
 // below 256 (exact in fp16) and the final O / l is unchanged.
 template <int DH>
 struct FwdCfg {
-  static constexpr int BM = 128, BN = 64, CH = DH / 64, STAGES = 3;
-  static constexpr int THREADS = 320;                   // producer, MMA, 2 x 4 softmax warps
+  static constexpr int BM = 128, BN = 64, CH = DH / 64, STAGES = 4;
+  static constexpr int THREADS = 352;                   // producer, S issuer, 2 x 4 softmax warps, P V issuer
   static constexpr int Q_BYTES = BM * DH * 2;           // one query tile
   static constexpr int KV_BYTES = BN * DH * 2;          // K or V of one stage
   static constexpr int P_BYTES = BM * BN * 2;           // one P tile
@@ -136,10 +136,12 @@ struct FwdCfg {
   static constexpr int SMEM = RAW > 120 * 1024 ? RAW : 120 * 1024;   // one CTA per SM (512 TMEM columns)
 };
 
+static_assert(FwdCfg<128>::SMEM <= 227 * 1024, "forward tile exceeds shared memory");
+
 constexpr float kLazyRescaleLog2 = 8.0f;
 
 template <int DH>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(352, 1)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q128,
                 const __grid_constant__ CUtensorMap tm_kv64, const AttnArgs p) {
   using C = FwdCfg<DH>;
@@ -148,14 +150,14 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q128,
   uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   uint64_t* q_full = bars + 0;
-  uint64_t* kv_full = bars + 1;     // [3]
-  uint64_t* kv_empty = bars + 4;    // [3]
-  uint64_t* s_full = bars + 7;      // [2] per tile
-  uint64_t* s_free = bars + 9;      // [2]
-  uint64_t* p_full = bars + 11;     // [2]
-  uint64_t* pv_done = bars + 13;    // [2]
-  uint64_t* drain = bars + 15;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
+  uint64_t* kv_full = bars + 1;     // [STAGES <= 4]
+  uint64_t* kv_empty = bars + 5;    // [STAGES]
+  uint64_t* s_full = bars + 9;      // [2] per tile
+  uint64_t* s_free = bars + 11;     // [2]
+  uint64_t* p_full = bars + 13;     // [2]
+  uint64_t* pv_done = bars + 15;    // [2]
+  uint64_t* drain = bars + 17;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 18);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -226,62 +228,62 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q128,
       for (int i = j - 1; i >= 0 && i >= j - C::STAGES; --i)
         mbar_wait(&kv_full[i % C::STAGES], (i / C::STAGES) & 1, 200000000ull);
     }
-  } else if (warp == 1) {
+  } else if (warp == 1 || warp == 10) {
+    // Two issuers, each blocking only on its own barriers: warp 1 issues the
+    // scores S = q k^T of both tiles (block j+1 once the tile's softmax has
+    // copied S of block j out of tensor memory), warp 10 the products P V
+    // (once P is in shared memory) and releases each K/V stage.  Neither
+    // stream waits behind the other.
     if (lane == 0) {
       constexpr uint32_t id_s = idesc_f32acc(128, C::BN, false, false, true);
       constexpr uint32_t id_pv = idesc_f32acc(128, DH, false, true, true);
       const uint32_t sq = smem_u32(smem + C::OFF_Q), sp = smem_u32(smem + C::OFF_P);
-      auto issue_s = [&](int i, uint32_t sk) {
-#pragma unroll
-        for (int kk = 0; kk < DH / 16; ++kk)
-          tc_mma_f16(tmem + 64 * i, kmajor_desc(sq + i * C::Q_BYTES, C::BM, kk),
-                     kmajor_desc(sk, C::BN, kk), id_s, kk > 0);
-        tc_commit(&s_full[i]);
-      };
-      auto issue_pv = [&](int i, int jj, uint32_t sv) {
-#pragma unroll
-        for (int kk = 0; kk < C::BN / 16; ++kk)
-          tc_mma_f16(tmem + 128 + 128 * i, kmajor_desc(sp + i * C::P_BYTES, C::BM, kk),
-                     mnmajor_desc(sv, C::BN, kk), id_pv, (jj | kk) != 0);
-        tc_commit(&pv_done[i]);
-      };
-      // Issue order: S of block j+1 for a tile goes out as soon as its softmax
-      // has copied S of block j out of tensor memory, so the next scores are
-      // computed while the current softmax runs; P V of block j follows once
-      // P is in shared memory.
-      bool ok = wait_bar(q_full, 0, ctl, ERR_ATTN_FWD_WAIT);
       auto kv_addr = [&](int j) { return smem_u32(smem + C::OFF_KV + (j % C::STAGES) * 2 * C::KV_BYTES); };
-      if (ok && nkv > 0) {
-        ok = wait_bar(&kv_full[0], 0, ctl, ERR_ATTN_FWD_WAIT);
-        if (ok) {
-          tc_fence_after();
-          if (ntile[0] > 0) issue_s(0, kv_addr(0));
-          if (ntile[1] > 0) issue_s(1, kv_addr(0));
-        }
-      }
-      for (int j = 0; ok && j < nkv; ++j) {
-        const bool next = j + 1 < nkv;
-        if (next && !(ok = wait_bar(&kv_full[(j + 1) % C::STAGES], ((j + 1) / C::STAGES) & 1, ctl,
-                                    ERR_ATTN_FWD_WAIT)))
-          break;
+      bool ok = wait_bar(q_full, 0, ctl, ERR_ATTN_FWD_WAIT);
+      if (warp == 1) {
+        for (int j = 0; ok && j < nkv; ++j) {
+          bool kv_in = false;   // block j has landed (waited for once)
 #pragma unroll
-        for (int i = 0; i < 2; ++i) {
-          if (j + 1 < ntile[i]) {
-            if (!(ok = wait_bar(&s_free[i], j & 1, ctl, ERR_ATTN_FWD_WAIT))) break;
-            tc_fence_after();
-            issue_s(i, kv_addr(j + 1));
-          }
-          if (j < ntile[i]) {
-            if (!(ok = wait_bar(&p_full[i], j & 1, ctl, ERR_ATTN_FWD_WAIT))) break;
-            tc_fence_after();
-            issue_pv(i, j, kv_addr(j) + C::KV_BYTES);
+          for (int i = 0; i < 2; ++i) {
+            if (ok && j < ntile[i]) {
+              if (j > 0 && !(ok = wait_bar(&s_free[i], (j - 1) & 1, ctl, ERR_ATTN_FWD_WAIT))) break;
+              if (!kv_in && !(ok = wait_bar(&kv_full[j % C::STAGES], (j / C::STAGES) & 1, ctl,
+                                            ERR_ATTN_FWD_WAIT)))
+                break;
+              kv_in = true;
+              tc_fence_after();
+              const uint32_t sk = kv_addr(j);
+#pragma unroll
+              for (int kk = 0; kk < DH / 16; ++kk)
+                tc_mma_f16(tmem + 64 * i, kmajor_desc(sq + i * C::Q_BYTES, C::BM, kk),
+                           kmajor_desc(sk, C::BN, kk), id_s, kk > 0);
+              tc_commit(&s_full[i]);
+            }
           }
         }
-        if (!ok) break;
-        tc_commit(&kv_empty[j % C::STAGES]);   // every product that reads block j is issued
+      } else {
+        for (int j = 0; ok && j < nkv; ++j) {
+#pragma unroll
+          for (int i = 0; i < 2; ++i) {
+            if (ok && j < ntile[i]) {
+              if (!(ok = wait_bar(&p_full[i], j & 1, ctl, ERR_ATTN_FWD_WAIT))) break;
+              tc_fence_after();
+              const uint32_t sv = kv_addr(j) + C::KV_BYTES;
+#pragma unroll
+              for (int kk = 0; kk < C::BN / 16; ++kk)
+                tc_mma_f16(tmem + 128 + 128 * i, kmajor_desc(sp + i * C::P_BYTES, C::BM, kk),
+                           mnmajor_desc(sv, C::BN, kk), id_pv, (j | kk) != 0);
+              tc_commit(&pv_done[i]);
+            }
+          }
+          if (!ok) break;
+          // The scores of block j completed before its softmax produced P, so
+          // once these products complete nothing reads the stage any more.
+          tc_commit(&kv_empty[j % C::STAGES]);
+        }
+        tc_commit(drain);
+        mbar_wait(drain, 0, 200000000ull);
       }
-      tc_commit(drain);
-      mbar_wait(drain, 0, 200000000ull);
     }
   } else {
     // ---------------------------------------------------------------- softmax warpgroups
@@ -301,19 +303,26 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q128,
       if (!__all_sync(0xffffffffu, wait_bar(&s_full[tile], j & 1, ctl, ERR_ATTN_FWD_WAIT))) { ok = false; break; }
       tc_fence_after();
       float s[C::BN];
-#pragma unroll
-      for (int c = 0; c < C::BN / 32; ++c) {
-        uint32_t rr[32];
-        tmem_ld32(t_s + c * 32, rr);
+      {
+        uint32_t ra[32], rb[32];
+        tmem_ld32(t_s, ra);
+        tmem_ld32(t_s + 32, rb);
         tc_wait_ld();
 #pragma unroll
-        for (int e = 0; e < 32; ++e) s[c * 32 + e] = __uint_as_float(rr[e]);
+        for (int e = 0; e < 32; ++e) {
+          s[e] = __uint_as_float(ra[e]);
+          s[32 + e] = __uint_as_float(rb[e]);
+        }
       }
       tc_fence_before();
       mbar_arrive(&s_free[tile]);
       const int k0 = j * C::BN;
       const bool need_mask = (p.causal && k0 + C::BN - 1 > qt) || (k0 + C::BN > p.S);
-      float mx = -1e30f;
+      // Row max and (below) row sum over 8 interleaved partials: short
+      // dependency chains instead of one chain through all 64 columns.
+      float m8[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) m8[e] = -1e30f;
 #pragma unroll
       for (int c = 0; c < C::BN; ++c) {
         float v = s[c] * p.scale_log2;
@@ -322,8 +331,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q128,
           if ((p.causal && kpos > q) || kpos >= p.S) v = -INFINITY;
         }
         s[c] = v;
-        mx = fmaxf(mx, v);
+        m8[c & 7] = fmaxf(m8[c & 7], v);
       }
+      const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                             fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
       float alpha = 1.0f;
       if (j == 0) {
         m_used = mx;
@@ -332,14 +343,16 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q128,
         m_used = mx;
         l *= alpha;
       }
-      float sum = 0.f;
+      float l8[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) l8[e] = 0.f;
 #pragma unroll
       for (int c = 0; c < C::BN; ++c) {
         const float e = fast_exp2(s[c] - m_used);
         s[c] = e;
-        sum += e;
+        l8[c & 7] += e;
       }
-      l += sum;
+      l += ((l8[0] + l8[1]) + (l8[2] + l8[3])) + ((l8[4] + l8[5]) + (l8[6] + l8[7]));
       if (j > 0) {
         // The previous P V of this tile has landed: P's buffer is free and O may be rescaled.
         if (!__all_sync(0xffffffffu, wait_bar(&pv_done[tile], (j - 1) & 1, ctl, ERR_ATTN_FWD_WAIT))) { ok = false; break; }
@@ -451,9 +464,10 @@ struct DkdvCfg {
   static constexpr int RAW = OFF_BAR + 256 + 1024;
   static constexpr int SMEM = RAW > 120 * 1024 ? RAW : 120 * 1024;
 };
+static_assert(DkdvCfg<128>::SMEM <= 227 * 1024, "dK/dV tile exceeds shared memory");
 
 template <int DH>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(352, 1)
 attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_kv128,
                      const __grid_constant__ CUtensorMap tm_q64,
                      const __grid_constant__ CUtensorMap tm_do64, const AttnArgs p) {
@@ -539,19 +553,23 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_kv128,
       for (int i = k - 1; i >= 0 && i >= k - C::STAGES; --i)
         mbar_wait(&qd_full[i % C::STAGES], (i / C::STAGES) & 1, 200000000ull);
     }
-  } else if (warp == 1) {
+  } else if (warp == 1 || warp == 10) {
+    // Two issuers, each blocking only on its own barriers: warp 1 issues
+    // S^T/dP^T of block k (once its q/dO stage has landed and the compute of
+    // block k-2 has copied its scores out of tensor memory), warp 10 issues
+    // dV/dK of block k (once its P^T/dS^T are in shared memory) and releases
+    // the stage.  Neither stream waits behind the other.
     if (lane == 0) {
       constexpr uint32_t id_s = idesc_f32acc(128, C::BQ, false, false, true);
       constexpr uint32_t id_acc = idesc_f32acc(128, DH, false, true, true);
       const uint32_t sk = smem_u32(smem + C::OFF_K), sv = smem_u32(smem + C::OFF_V);
       const uint32_t spt = smem_u32(smem + C::OFF_PT);
       bool ok = wait_bar(kv_full, 0, ctl, ERR_ATTN_DKDV_WAIT);
-      for (int k = 0; ok && k <= nsteps; ++k) {
-        if (k < nsteps) {
+      if (warp == 1) {
+        for (int k = 0; ok && k < nsteps; ++k) {
           const int bf = k & 1, st = k % C::STAGES;
-          const uint32_t u = k >> 1;
-          if (!wait_bar(&qd_full[st], (k / C::STAGES) & 1, ctl, ERR_ATTN_DKDV_WAIT)) break;
-          if (!wait_bar(&s_free[bf], (u & 1) ^ 1, ctl, ERR_ATTN_DKDV_WAIT)) break;
+          if (!(ok = wait_bar(&qd_full[st], (k / C::STAGES) & 1, ctl, ERR_ATTN_DKDV_WAIT))) break;
+          if (!(ok = wait_bar(&s_free[bf], ((k >> 1) & 1) ^ 1, ctl, ERR_ATTN_DKDV_WAIT))) break;
           tc_fence_after();
           const uint32_t sq = smem_u32(smem + C::OFF_ST + st * C::STAGE_BYTES);
           const uint32_t sd = sq + C::Q_BYTES;
@@ -564,9 +582,10 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_kv128,
           }
           tc_commit(&s_full[bf]);
         }
-        if (k > 0) {
-          const int j = k - 1, bj = j & 1, sj = j % C::STAGES;
-          if (!wait_bar(&p_full[bj], (j >> 1) & 1, ctl, ERR_ATTN_DKDV_WAIT)) break;
+      } else {
+        for (int k = 0; ok && k < nsteps; ++k) {
+          const int bj = k & 1, sj = k % C::STAGES;
+          if (!(ok = wait_bar(&p_full[bj], (k >> 1) & 1, ctl, ERR_ATTN_DKDV_WAIT))) break;
           tc_fence_after();
           const uint32_t sq = smem_u32(smem + C::OFF_ST + sj * C::STAGE_BYTES);
           const uint32_t sd = sq + C::Q_BYTES;
@@ -574,16 +593,16 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_kv128,
 #pragma unroll
           for (int kk = 0; kk < C::BQ / 16; ++kk) {
             tc_mma_f16(t_dv, kmajor_desc(pt, C::BK, kk), mnmajor_desc(sd, C::BQ, kk), id_acc,
-                       (j | kk) != 0);
+                       (k | kk) != 0);
             tc_mma_f16(t_dk, kmajor_desc(dst, C::BK, kk), mnmajor_desc(sq, C::BQ, kk), id_acc,
-                       (j | kk) != 0);
+                       (k | kk) != 0);
           }
           tc_commit(&mm2_done[bj]);
-          tc_commit(&qd_empty[sj]);
+          tc_commit(&qd_empty[sj]);   // the scores of block k completed before its P^T existed
         }
+        tc_commit(drain);
+        mbar_wait(drain, 0, 200000000ull);
       }
-      tc_commit(drain);
-      mbar_wait(drain, 0, 200000000ull);
     }
   } else {
     // Two compute warpgroups: warpgroup g takes the blocks k with k % 2 == g (its
@@ -600,38 +619,58 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_kv128,
       const uint32_t u = k >> 1;
       const int qs = (i0 + k) * C::BQ;
       if (!__all_sync(0xffffffffu, wait_bar(&s_full[bf], u & 1, ctl, ERR_ATTN_DKDV_WAIT))) { ok = false; break; }
-      // The P^T/dS^T buffer bf was last read by the dV/dK MMAs of block k-2.
-      if (k >= 2 && !__all_sync(0xffffffffu, wait_bar(&mm2_done[bf], (u - 1) & 1, ctl, ERR_ATTN_DKDV_WAIT))) { ok = false; break; }
       tc_fence_after();
       const float* vl = reinterpret_cast<const float*>(smem + C::OFF_VEC + (k % C::STAGES) * 2 * C::VEC_BYTES);
       const float* vd = vl + C::BQ;
       uint8_t* pt = smem + C::OFF_PT + 2 * bf * C::T_BYTES;
       uint8_t* dst = pt + C::T_BYTES;
-#pragma unroll 1
-      for (int c = 0; c < C::BQ / 32; ++c) {
+      // S^T and dP^T leave tensor memory in two 32-column halves; the buffer is
+      // handed back right after the second half is copied, so the scores of
+      // block k+2 are computed while this block's P^T and dS^T are finished.
+      // Each half goes to shared memory as soon as it is done (register budget
+      // of 320 threads).
+      const bool diag = p.causal && kpos > qs;   // some query of this block precedes key kpos
+      bool fail = false;
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
         uint32_t rs[32], rd[32];
         tmem_ld32(tmem + bf * 128 + lane_off + c * 32, rs);
         tmem_ld32(tmem + bf * 128 + 64 + lane_off + c * 32, rd);
         tc_wait_ld();
-        float pv[32], dsv[32];
+        if (c == 1) {
+          tc_fence_before();
+          mbar_arrive(&s_free[bf]);
+        }
+        uint32_t pk[16], dk[16];   // fp16 pairs of P^T and dS^T
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const int qi = c * 32 + e;
-          // Padded queries carry lse2 = +inf and dvec = 0, so they give 0.
-          float pe = fast_exp2(__uint_as_float(rs[e]) * p.scale_log2 - vl[qi]);
-          if (p.causal && kpos > qs + qi) pe = 0.f;
-          pv[e] = pe;
-          dsv[e] = pe * (__uint_as_float(rd[e]) - vd[qi]);
+        for (int e = 0; e < 32; e += 2) {
+          float pe[2], de[2];
+#pragma unroll
+          for (int h2 = 0; h2 < 2; ++h2) {
+            const int qi = c * 32 + e + h2;
+            // Padded queries carry lse2 = +inf and dvec = 0, so they give 0.
+            float x = fast_exp2(__uint_as_float(rs[e + h2]) * p.scale_log2 - vl[qi]);
+            if (diag && kpos > qs + qi) x = 0.f;
+            pe[h2] = x;
+            de[h2] = x * (__uint_as_float(rd[e + h2]) - vd[qi]);
+          }
+          pk[e / 2] = pack_f16x2(pe[0], pe[1]);
+          dk[e / 2] = pack_f16x2(de[0], de[1]);
+        }
+        // The P^T/dS^T buffer bf was last read by the dV/dK MMAs of block k-2.
+        if (c == 0 && k >= 2 &&
+            !__all_sync(0xffffffffu, wait_bar(&mm2_done[bf], (u - 1) & 1, ctl, ERR_ATTN_DKDV_WAIT))) {
+          fail = true;
+          break;
         }
 #pragma unroll
         for (int g = 0; g < 4; ++g) {
           const uint32_t off = sw128_offset(C::BK, r, c * 32 + g * 8);
-          *reinterpret_cast<uint4*>(pt + off) = pack8_f16(&pv[g * 8]);
-          *reinterpret_cast<uint4*>(dst + off) = pack8_f16(&dsv[g * 8]);
+          *reinterpret_cast<uint4*>(pt + off) = make_uint4(pk[4 * g], pk[4 * g + 1], pk[4 * g + 2], pk[4 * g + 3]);
+          *reinterpret_cast<uint4*>(dst + off) = make_uint4(dk[4 * g], dk[4 * g + 1], dk[4 * g + 2], dk[4 * g + 3]);
         }
       }
-      tc_fence_before();
-      mbar_arrive(&s_free[bf]);
+      if (fail) { ok = false; break; }
       fence_proxy_async_smem();
       mbar_arrive(&p_full[bf]);
     }
@@ -684,7 +723,7 @@ struct DqCfg {
   static constexpr int Q_BYTES = BQ * DH * 2;                // q and dO tiles, each
   static constexpr int K_BYTES = BK * DH * 2;                // K and V tiles, each (per stage)
   static constexpr int OFF_Q = 0, OFF_DO = Q_BYTES;
-  static constexpr int STAGES = 3;                           // K / V ring depth
+  static constexpr int STAGES = 4;                           // K / V ring depth
   static constexpr int OFF_ST = 2 * Q_BYTES;                 // stage s: k at +s*2*K, v at +K
   static constexpr int DS_BYTES = BQ * BK * 2;
   static constexpr int OFF_DS = OFF_ST + STAGES * 2 * K_BYTES;  // buffer b: dS at +b*DS
@@ -692,9 +731,10 @@ struct DqCfg {
   static constexpr int RAW = OFF_BAR + 256 + 1024;
   static constexpr int SMEM = RAW > 120 * 1024 ? RAW : 120 * 1024;
 };
+static_assert(DqCfg<128>::SMEM <= 227 * 1024, "dQ tile exceeds shared memory");
 
 template <int DH>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(352, 1)
 attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q128,
                    const __grid_constant__ CUtensorMap tm_do128,
                    const __grid_constant__ CUtensorMap tm_kv64, const AttnArgs p) {
@@ -704,14 +744,14 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q128,
   uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   uint64_t* q_full = bars + 0;
-  uint64_t* kv_full = bars + 1;    // [3] per stage
-  uint64_t* kv_empty = bars + 4;   // [3]
-  uint64_t* s_full = bars + 7;     // [2] per TMEM buffer
-  uint64_t* s_free = bars + 9;     // [2]
-  uint64_t* p_full = bars + 11;    // [2] per dS buffer
-  uint64_t* mm2_done = bars + 13;  // [2]
-  uint64_t* drain = bars + 15;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
+  uint64_t* kv_full = bars + 1;    // [STAGES <= 4] per stage
+  uint64_t* kv_empty = bars + 5;   // [STAGES]
+  uint64_t* s_full = bars + 9;     // [2] per TMEM buffer
+  uint64_t* s_free = bars + 11;    // [2]
+  uint64_t* p_full = bars + 13;    // [2] per dS buffer
+  uint64_t* mm2_done = bars + 15;  // [2]
+  uint64_t* drain = bars + 17;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 18);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -775,19 +815,20 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q128,
       for (int i = k - 1; i >= 0 && i >= k - C::STAGES; --i)
         mbar_wait(&kv_full[i % C::STAGES], (i / C::STAGES) & 1, 200000000ull);
     }
-  } else if (warp == 1) {
+  } else if (warp == 1 || warp == 10) {
+    // Two issuers as in the dK/dV kernel: warp 1 issues S/dP of block k,
+    // warp 10 dQ += dS K of block k and releases the K/V stage.
     if (lane == 0) {
       constexpr uint32_t id_s = idesc_f32acc(128, C::BK, false, false, true);
       constexpr uint32_t id_acc = idesc_f32acc(128, DH, false, true, true);
       const uint32_t sq = smem_u32(smem + C::OFF_Q), sd = smem_u32(smem + C::OFF_DO);
       const uint32_t sds = smem_u32(smem + C::OFF_DS);
       bool ok = wait_bar(q_full, 0, ctl, ERR_ATTN_DQ_WAIT);
-      for (int k = 0; ok && k <= nsteps; ++k) {
-        if (k < nsteps) {
+      if (warp == 1) {
+        for (int k = 0; ok && k < nsteps; ++k) {
           const int bf = k & 1, st = k % C::STAGES;
-          const uint32_t u = k >> 1;
-          if (!wait_bar(&kv_full[st], (k / C::STAGES) & 1, ctl, ERR_ATTN_DQ_WAIT)) break;
-          if (!wait_bar(&s_free[bf], (u & 1) ^ 1, ctl, ERR_ATTN_DQ_WAIT)) break;
+          if (!(ok = wait_bar(&kv_full[st], (k / C::STAGES) & 1, ctl, ERR_ATTN_DQ_WAIT))) break;
+          if (!(ok = wait_bar(&s_free[bf], ((k >> 1) & 1) ^ 1, ctl, ERR_ATTN_DQ_WAIT))) break;
           tc_fence_after();
           const uint32_t sk = smem_u32(smem + C::OFF_ST + st * 2 * C::K_BYTES);
           const uint32_t sv = sk + C::K_BYTES;
@@ -800,21 +841,22 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q128,
           }
           tc_commit(&s_full[bf]);
         }
-        if (k > 0) {
-          const int j = k - 1, bj = j & 1, sj = j % C::STAGES;
-          if (!wait_bar(&p_full[bj], (j >> 1) & 1, ctl, ERR_ATTN_DQ_WAIT)) break;
+      } else {
+        for (int k = 0; ok && k < nsteps; ++k) {
+          const int bj = k & 1, sj = k % C::STAGES;
+          if (!(ok = wait_bar(&p_full[bj], (k >> 1) & 1, ctl, ERR_ATTN_DQ_WAIT))) break;
           tc_fence_after();
           const uint32_t sk = smem_u32(smem + C::OFF_ST + sj * 2 * C::K_BYTES);
 #pragma unroll
           for (int kk = 0; kk < C::BK / 16; ++kk)
             tc_mma_f16(t_dq, kmajor_desc(sds + bj * C::DS_BYTES, C::BQ, kk),
-                       mnmajor_desc(sk, C::BK, kk), id_acc, (j | kk) != 0);
+                       mnmajor_desc(sk, C::BK, kk), id_acc, (k | kk) != 0);
           tc_commit(&mm2_done[bj]);
-          tc_commit(&kv_empty[sj]);
+          tc_commit(&kv_empty[sj]);   // the scores of block k completed before its dS existed
         }
+        tc_commit(drain);
+        mbar_wait(drain, 0, 200000000ull);
       }
-      tc_commit(drain);
-      mbar_wait(drain, 0, 200000000ull);
     }
   } else {
     // Two compute warpgroups: warpgroup g takes the blocks k with k % 2 == g (its
@@ -835,29 +877,38 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q128,
       const uint32_t u = k >> 1;
       const int ks = k * C::BK;
       if (!__all_sync(0xffffffffu, wait_bar(&s_full[bf], u & 1, ctl, ERR_ATTN_DQ_WAIT))) { ok = false; break; }
-      if (k >= 2 && !__all_sync(0xffffffffu, wait_bar(&mm2_done[bf], (u - 1) & 1, ctl, ERR_ATTN_DQ_WAIT))) { ok = false; break; }
       tc_fence_after();
       uint8_t* sds = smem + C::OFF_DS + bf * C::DS_BYTES;
-#pragma unroll 1
-      for (int c = 0; c < C::BK / 32; ++c) {
-        uint32_t rs[32], rd[32];
-        tmem_ld32(tmem + bf * 128 + lane_off + c * 32, rs);
-        tmem_ld32(tmem + bf * 128 + 64 + lane_off + c * 32, rd);
-        tc_wait_ld();
-        float dsv[32];
+      // Copy S and dP out of tensor memory and hand the buffer back first.
+      uint32_t rs0[32], rs1[32], rd0[32], rd1[32];
+      tmem_ld32(tmem + bf * 128 + lane_off, rs0);
+      tmem_ld32(tmem + bf * 128 + lane_off + 32, rs1);
+      tmem_ld32(tmem + bf * 128 + 64 + lane_off, rd0);
+      tmem_ld32(tmem + bf * 128 + 64 + lane_off + 32, rd1);
+      tc_wait_ld();
+      tc_fence_before();
+      mbar_arrive(&s_free[bf]);
+      const bool edge = (p.causal && ks + C::BK - 1 > q) || ks + C::BK > p.S;
+      auto ds = [&](const uint32_t (&rs)[32], uint32_t (&rd)[32], int c) {
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
           const int kpos = ks + c * 32 + e;
           float pe = fast_exp2(__uint_as_float(rs[e]) * p.scale_log2 - l2);
-          if ((p.causal && kpos > q) || kpos >= p.S) pe = 0.f;
-          dsv[e] = pe * (__uint_as_float(rd[e]) - dv);
+          if (edge && ((p.causal && kpos > q) || kpos >= p.S)) pe = 0.f;
+          rd[e] = __float_as_uint(pe * (__uint_as_float(rd[e]) - dv));
         }
+      };
+      ds(rs0, rd0, 0);
+      ds(rs1, rd1, 1);
+      // The dS buffer bf was last read by the dQ MMAs of block k-2.
+      if (k >= 2 && !__all_sync(0xffffffffu, wait_bar(&mm2_done[bf], (u - 1) & 1, ctl, ERR_ATTN_DQ_WAIT))) { ok = false; break; }
 #pragma unroll
-        for (int g = 0; g < 4; ++g)
-          *reinterpret_cast<uint4*>(sds + sw128_offset(C::BQ, r, c * 32 + g * 8)) = pack8_f16(&dsv[g * 8]);
+      for (int g = 0; g < 4; ++g) {
+        *reinterpret_cast<uint4*>(sds + sw128_offset(C::BQ, r, g * 8)) =
+            pack8_f16(reinterpret_cast<const float*>(&rd0[g * 8]));
+        *reinterpret_cast<uint4*>(sds + sw128_offset(C::BQ, r, 32 + g * 8)) =
+            pack8_f16(reinterpret_cast<const float*>(&rd1[g * 8]));
       }
-      tc_fence_before();
-      mbar_arrive(&s_free[bf]);
       fence_proxy_async_smem();
       mbar_arrive(&p_full[bf]);
     }
@@ -1015,12 +1066,12 @@ tp_status bwd_launch(const uint16_t* qkv, const uint16_t* o, const float* lse, c
   {
     // dP, dV and dK: three of the backward's four algorithmic products.
     TraceScope ts(st, TK_ATTN_BWD_DKDV, 6.0 * DH * core_pairs(a));
-    k1<<<dim3((a.S + 127) / 128, a.H, a.B), 320, DkdvCfg<DH>::SMEM, st>>>(kv128, q64, do64, p);
+    k1<<<dim3((a.S + 127) / 128, a.H, a.B), 352, DkdvCfg<DH>::SMEM, st>>>(kv128, q64, do64, p);
   }
   if (cudaGetLastError() != cudaSuccess) return TP_ERR_CUDA;
   {
     TraceScope ts(st, TK_ATTN_BWD_DQ, 2.0 * DH * core_pairs(a));
-    k2<<<dim3((a.S + 127) / 128, a.H, a.B), 320, DqCfg<DH>::SMEM, st>>>(q128, do128, kv64, p);
+    k2<<<dim3((a.S + 127) / 128, a.H, a.B), 352, DqCfg<DH>::SMEM, st>>>(q128, do128, kv64, p);
   }
   return cuda_status(cudaGetLastError());
 }

@@ -12,11 +12,11 @@ from typing import Dict, Optional
 
 import torch
 
-from . import (Dims, OP_ATTN_BWD, OP_ATTN_FWD, OP_LAYER_BWD, OP_LAYER_FWD, OP_MLP_BWD,
-               OP_POSTLN_BWD, OP_POSTLN_FWD, attn_bwd, attn_fwd, layer_bwd, postln_layer_bwd,
-               postln_layer_fwd,
-               layer_fwd, mlp_bwd, mlp_fwd, shard_cols, shard_qkv_heads, shard_rows,
-               unshard_cols, unshard_qkv_heads, workspace_size)
+from . import (Dims, OP_ATTN_BWD, OP_ATTN_FWD, OP_LAYER_BWD, OP_LAYER_BWD_RECOMPUTE,
+               OP_LAYER_FWD, OP_LAYER_FWD_NOSAVE, OP_MLP_BWD, OP_POSTLN_BWD, OP_POSTLN_FWD,
+               attn_bwd, attn_fwd, layer_bwd, layer_bwd_recompute, layer_fwd, layer_fwd_nosave,
+               mlp_bwd, mlp_fwd, postln_layer_bwd, postln_layer_fwd, shard_cols,
+               shard_qkv_heads, shard_rows, unshard_cols, unshard_qkv_heads, workspace_size)
 
 BF16 = torch.bfloat16
 
@@ -160,12 +160,20 @@ LAYER_PARAM_NAMES = ("ln1_g", "ln1_b", "wqkv", "bqkv", "wout", "bout", "ln2_g", 
 
 class ShardedLayer:
     """Pre-LN layer h = x + Attn(LN1(x)); y = h + MLP(LN2(h)), or with
-    placement="post" the post-LN layer h = LN1(x + Attn(x)); y = LN2(h + MLP(h))."""
+    placement="post" the post-LN layer h = LN1(x + Attn(x)); y = LN2(h + MLP(h)).
 
-    def __init__(self, dims: Dims, p: Dict[str, torch.Tensor], placement: str = "pre"):
+    recompute=True (pre-LN only) keeps nothing but x between forward and
+    backward: the forward's intermediates live in its workspace, and the
+    backward computes them again before using them."""
+
+    def __init__(self, dims: Dims, p: Dict[str, torch.Tensor], placement: str = "pre",
+                 recompute: bool = False):
         if placement not in ("pre", "post"):
             raise ValueError("placement is 'pre' or 'post'")
+        if recompute and placement != "pre":
+            raise ValueError("recompute is available for the pre-LN layer")
         self.post = placement == "post"
+        self.recompute = recompute
         self.dims = dims
         t, H = dims.t, dims.heads
         self.device = p["w1"].device
@@ -219,10 +227,22 @@ class ShardedLayer:
                 "dw1": _empty((t, D, F // t), device=dev), "db1": opt((F,)),
                 "dw2": _empty((t, F // t, D), device=dev), "db2": opt((D,))}
 
+    def saved_bytes(self) -> int:
+        """Bytes of activations held from the forward to the backward (x excluded)."""
+        if self.recompute:
+            return 0
+        return sum(v.numel() * v.element_size() for v in self.alloc_acts().values())
+
     def forward(self, x, acts=None, y=None):
         d = self.dims
-        acts = acts if acts is not None else self.alloc_acts()
         y = y if y is not None else _empty((d.batch * d.seq, d.hidden), device=self.device)
+        if self.recompute:
+            if self.ws_fwd is None:
+                self.ws_fwd = _ws(OP_LAYER_FWD_NOSAVE, d, self.device)
+            layer_fwd_nosave(d, x, self.p, y, self.ws_fwd)
+            self.saved = (x, None)
+            return y, None
+        acts = acts if acts is not None else self.alloc_acts()
         if self.ws_fwd is None:
             self.ws_fwd = _ws(OP_POSTLN_FWD if self.post else OP_LAYER_FWD, d, self.device)
         (postln_layer_fwd if self.post else layer_fwd)(d, x, self.p, acts, y, self.ws_fwd)
@@ -232,9 +252,14 @@ class ShardedLayer:
     def backward(self, dy, dx=None, grads=None, bias_grads=True):
         d = self.dims
         x, acts = self.saved
-        if self.ws is None:
-            self.ws = _ws(OP_POSTLN_BWD if self.post else OP_LAYER_BWD, d, self.device)
         dx = dx if dx is not None else torch.empty_like(x)
         grads = grads if grads is not None else self.alloc_grads(bias_grads)
+        if self.recompute:
+            if self.ws is None:
+                self.ws = _ws(OP_LAYER_BWD_RECOMPUTE, d, self.device)
+            layer_bwd_recompute(d, x, self.p, dy, dx, grads, self.ws)
+            return dx, grads
+        if self.ws is None:
+            self.ws = _ws(OP_POSTLN_BWD if self.post else OP_LAYER_BWD, d, self.device)
         (postln_layer_bwd if self.post else layer_bwd)(d, x, self.p, acts, dy, dx, grads, self.ws)
         return dx, grads

@@ -76,3 +76,34 @@ def test_host_validation_without_gpu():
     assert st == 1  # TP_ERR_INVALID_ARG: heads % t != 0
     assert lib.tp_trace_begin(None, None, None, -1) == 1
     assert lib.tp_trace_end() == 0
+
+
+def test_recompute_entry_points_host_side():
+    """Workspace sizes and argument checks of the recomputation entry points (no GPU).
+
+    The recomputing backward needs the saved activations' bytes on top of the
+    ordinary backward workspace, since it rebuilds them there; the forward
+    that saves nothing holds them in its workspace instead of caller buffers.
+    """
+    lib = tl.lib()
+    B, S, D, F, H, dh, t = 4, 2048, 4096, 16384, 32, 128, 8
+    d = tl.Dims.of(B, S, D, F, H, dh, t)
+    T = B * S
+    acts = (T * D * 2 + 2 * T * 4 + T * 3 * D * 2 + T * D * 2 + B * H * S * 4 + 2 * T * D * 2
+            + 2 * T * 4 + 2 * T * F * 2)
+    bwd = tl.workspace_size(tl.OP_LAYER_BWD, d)
+    rec = tl.workspace_size(tl.OP_LAYER_BWD_RECOMPUTE, d)
+    assert acts <= rec - bwd <= acts + 16 * 256
+    fwd = tl.workspace_size(tl.OP_LAYER_FWD, d)
+    nos = tl.workspace_size(tl.OP_LAYER_FWD_NOSAVE, d)
+    assert acts <= nos - fwd <= acts + 16 * 256
+    bad = tl.Dims.of(1, 8, 4096, 16384, 30, 128, 8)
+    assert tl.workspace_size(tl.OP_LAYER_BWD_RECOMPUTE, bad) == 0
+    small = tl.Dims.of(1, 8, 256, 1024, 2, 128, 2)
+    p = tl.LayerParams()
+    st = lib.tp_layer_fwd_nosave(ctypes.byref(small), 16, ctypes.byref(p), 16, None, 0, None)
+    assert st == 1  # TP_ERR_INVALID_ARG: parameter pointers missing
+    g = tl.LayerGrads()
+    st = lib.tp_layer_bwd_recompute(ctypes.byref(small), 16, ctypes.byref(p), 16, 16,
+                                    ctypes.byref(g), None, 0, None)
+    assert st == 1
