@@ -15,8 +15,9 @@
 // Forward (per pair of 128-query tiles, head, batch; 64-key blocks):
 //   S = q k^T (tcgen05, fp32 in TMEM), online softmax in fp32 by one thread per
 //   query row (base-2 exponent, scores pre-scaled by log2(e)/sqrt(dh)), P
-//   rounded to fp16 into swizzled shared memory, O += P v (tcgen05, fp32 in
-//   TMEM, rescaled lazily).  The two tiles alternate on the tensor core.
+//   rounded to fp16 into tensor memory, O += P v (tcgen05 with P as the
+//   A operand read from tensor memory, fp32 in TMEM, rescaled lazily).  The
+//   two tiles alternate on the tensor core.
 //   Writes O [t][T][Dt] (bf16) and the log-sum-exp [B][H][S] (fp32).
 // Backward (P recomputed from the log-sum-exp; no atomics, deterministic;
 // dO in and dqkv out are fp16):
@@ -26,6 +27,10 @@
 //           dV += P^T dO, dK += dS^T q
 //   dQ:     per 128-query block, walk 64-key blocks: S = q k^T, dP = dO v^T,
 //           dS = P * (dP - Dv), dQ += dS k
+// P, P^T, dS^T and dS go from registers to tensor memory (fp16) and are the
+// A operands of the products that consume them, read from there: shared
+// memory, whose bandwidth the score products already use up, carries only
+// the TMA tiles and the B operands.
 // Every wait is bounded (about 2 s); a timeout records an error code and the
 // kernel drains its copies and MMAs, frees TMEM and returns.
 #include <cuda.h>
@@ -118,7 +123,7 @@ __device__ __forceinline__ uint64_t mnmajor_desc(uint32_t base, int R, int kk) {
 // Two 128-query tiles per CTA take turns on the tensor core: while one tile's
 // softmax warpgroup works on its scores, the other tile's products run.  Keys
 // come in 64-wide blocks through a 4-stage ring; each tile has its own S (64
-// TMEM columns) and O (dh columns).  O is rescaled lazily: only when a row's
+// TMEM columns), P (32 columns of fp16 pairs) and O (dh columns).  O is rescaled lazily: only when a row's
 // running max grows by more than 2^8 (log2 units), so P = 2^(s - m_used) stays
 // below 256 (exact in fp16) and the final O / l is unchanged.
 template <int DH>
@@ -127,11 +132,9 @@ struct FwdCfg {
   static constexpr int THREADS = 352;                   // producer, S issuer, 2 x 4 softmax warps, P V issuer
   static constexpr int Q_BYTES = BM * DH * 2;           // one query tile
   static constexpr int KV_BYTES = BN * DH * 2;          // K or V of one stage
-  static constexpr int P_BYTES = BM * BN * 2;           // one P tile
   static constexpr int OFF_Q = 0;                       // tile i at +i*Q
   static constexpr int OFF_KV = 2 * Q_BYTES;            // stage s: K at +2s*KV, V at +(2s+1)*KV
-  static constexpr int OFF_P = OFF_KV + STAGES * 2 * KV_BYTES;   // tile i at +i*P
-  static constexpr int OFF_BAR = OFF_P + 2 * P_BYTES;
+  static constexpr int OFF_BAR = OFF_KV + STAGES * 2 * KV_BYTES;
   static constexpr int RAW = OFF_BAR + 256 + 1024;
   static constexpr int SMEM = RAW > 120 * 1024 ? RAW : 120 * 1024;   // one CTA per SM (512 TMEM columns)
 };
@@ -202,7 +205,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q128,
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = *tmem_slot;   // S of tile i at 64i; O of tile i at 128 + 128i
+  // TMEM columns: S of tile i at 64i, O of tile i at 128 + 128i, P of tile i at 384 + 32i.
+  const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
     if (lane == 0) {
@@ -232,12 +236,12 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q128,
     // Two issuers, each blocking only on its own barriers: warp 1 issues the
     // scores S = q k^T of both tiles (block j+1 once the tile's softmax has
     // copied S of block j out of tensor memory), warp 10 the products P V
-    // (once P is in shared memory) and releases each K/V stage.  Neither
+    // (once P is in tensor memory) and releases each K/V stage.  Neither
     // stream waits behind the other.
     if (lane == 0) {
       constexpr uint32_t id_s = idesc_f32acc(128, C::BN, false, false, true);
       constexpr uint32_t id_pv = idesc_f32acc(128, DH, false, true, true);
-      const uint32_t sq = smem_u32(smem + C::OFF_Q), sp = smem_u32(smem + C::OFF_P);
+      const uint32_t sq = smem_u32(smem + C::OFF_Q);
       auto kv_addr = [&](int j) { return smem_u32(smem + C::OFF_KV + (j % C::STAGES) * 2 * C::KV_BYTES); };
       bool ok = wait_bar(q_full, 0, ctl, ERR_ATTN_FWD_WAIT);
       if (warp == 1) {
@@ -270,9 +274,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q128,
               tc_fence_after();
               const uint32_t sv = kv_addr(j) + C::KV_BYTES;
 #pragma unroll
-              for (int kk = 0; kk < C::BN / 16; ++kk)
-                tc_mma_f16(tmem + 128 + 128 * i, kmajor_desc(sp + i * C::P_BYTES, C::BM, kk),
-                           mnmajor_desc(sv, C::BN, kk), id_pv, (j | kk) != 0);
+              for (int kk = 0; kk < C::BN / 16; ++kk)   // 16 keys = 8 columns of P per step
+                tc_mma_f16_ts(tmem + 128 + 128 * i, tmem + 384 + 32 * i + 8 * kk,
+                              mnmajor_desc(sv, C::BN, kk), id_pv, (j | kk) != 0);
               tc_commit(&pv_done[i]);
             }
           }
@@ -296,7 +300,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q128,
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
     const uint32_t t_s = tmem + 64 * tile + lane_off;
     const uint32_t t_o = tmem + 128 + 128 * tile + lane_off;
-    uint8_t* sp = smem + C::OFF_P + tile * C::P_BYTES;
+    const uint32_t t_p = tmem + 384 + 32 * tile + lane_off;
     float m_used = -1e30f, l = 0.f;
     bool ok = true;
     for (int j = 0; j < n; ++j) {
@@ -316,8 +320,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q128,
       }
       tc_fence_before();
       mbar_arrive(&s_free[tile]);
-      const int k0 = j * C::BN;
-      const bool need_mask = (p.causal && k0 + C::BN - 1 > qt) || (k0 + C::BN > p.S);
+      // Keys past the last visible one (after the query, or past S) are masked: a select
+      // per element against a bound fixed once per block, no branches.
+      const int kmax = (p.causal ? min(q, p.S - 1) : p.S - 1) - j * C::BN;
       // Row max and (below) row sum over 8 interleaved partials: short
       // dependency chains instead of one chain through all 64 columns.
       float m8[8];
@@ -325,11 +330,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q128,
       for (int e = 0; e < 8; ++e) m8[e] = -1e30f;
 #pragma unroll
       for (int c = 0; c < C::BN; ++c) {
-        float v = s[c] * p.scale_log2;
-        if (need_mask) {
-          const int kpos = k0 + c;
-          if ((p.causal && kpos > q) || kpos >= p.S) v = -INFINITY;
-        }
+        const float v = c > kmax ? -INFINITY : s[c] * p.scale_log2;
         s[c] = v;
         m8[c & 7] = fmaxf(m8[c & 7], v);
       }
@@ -354,7 +355,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q128,
       }
       l += ((l8[0] + l8[1]) + (l8[2] + l8[3])) + ((l8[4] + l8[5]) + (l8[6] + l8[7]));
       if (j > 0) {
-        // The previous P V of this tile has landed: P's buffer is free and O may be rescaled.
+        // The previous P V of this tile has completed: P's columns are free and O may be rescaled.
         if (!__all_sync(0xffffffffu, wait_bar(&pv_done[tile], (j - 1) & 1, ctl, ERR_ATTN_FWD_WAIT))) { ok = false; break; }
         tc_fence_after();
         if (!__all_sync(0xffffffffu, alpha == 1.0f)) {
@@ -370,10 +371,13 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q128,
           tc_wait_st();
         }
       }
+      {
+        uint32_t pk[C::BN / 2];
 #pragma unroll
-      for (int g = 0; g < C::BN / 8; ++g)
-        *reinterpret_cast<uint4*>(sp + sw128_offset(C::BM, r, g * 8)) = pack8_f16(&s[g * 8]);
-      fence_proxy_async_smem();
+        for (int g = 0; g < C::BN / 2; ++g) pk[g] = pack_f16x2(s[2 * g], s[2 * g + 1]);
+        tmem_st32(t_p, pk);
+        tc_wait_st();
+      }
       tc_fence_before();
       mbar_arrive(&p_full[tile]);
     }
@@ -444,22 +448,23 @@ __global__ void attn_bwd_prep_kernel(const uint16_t* __restrict__ o, const uint1
 }
 
 // ---------------------------------------------------------------- dK / dV
-// Per 128-key block, walk 64-query blocks.  Double-buffered S^T/dP^T in TMEM
-// and P^T/dS^T tiles in shared memory: the MMAs of block k+1 (S^T, dP^T) and
-// the dV/dK MMAs of block k-1 run while the compute warps work on block k.
+// Per 128-key block, walk 64-query blocks.  Two S^T/dP^T buffers in TMEM,
+// one per compute warpgroup (block k uses buffer k % 2): the score MMAs of
+// block k+1 and the dV/dK MMAs of block k-1 run while the compute warps work
+// on block k.  P^T and dS^T (fp16) replace, in place, the halves of S^T and
+// dP^T that have been copied out, and are the A operands of dV += P^T dO and
+// dK += dS^T q.
 template <int DH>
 struct DkdvCfg {
   static constexpr int BK = 128, BQ = 64, CH = DH / 64;
   static constexpr int K_BYTES = BK * DH * 2;              // K and V tiles, each
   static constexpr int Q_BYTES = BQ * DH * 2;              // q and dO tiles, each (per stage)
   static constexpr int VEC_BYTES = BQ * 4;                 // lse2 / dvec slice of one stage
-  static constexpr int STAGES = 3;                         // q / dO / lse2 / dvec ring depth
+  static constexpr int STAGES = 4;                         // q / dO / lse2 / dvec ring depth
   static constexpr int STAGE_BYTES = 2 * Q_BYTES;
   static constexpr int OFF_K = 0, OFF_V = K_BYTES;
   static constexpr int OFF_ST = 2 * K_BYTES;               // stage s: q | dO
-  static constexpr int T_BYTES = BK * BQ * 2;              // one P^T or dS^T tile
-  static constexpr int OFF_PT = OFF_ST + STAGES * STAGE_BYTES;  // buffer b: P^T at +2b*T, dS^T at +(2b+1)*T
-  static constexpr int OFF_VEC = OFF_PT + 4 * T_BYTES;     // stage s: lse2 at +2s*VEC, dvec at +(2s+1)*VEC
+  static constexpr int OFF_VEC = OFF_ST + STAGES * STAGE_BYTES;  // stage s: lse2 at +2s*VEC, dvec at +(2s+1)*VEC
   static constexpr int OFF_BAR = OFF_VEC + STAGES * 2 * VEC_BYTES;
   static constexpr int RAW = OFF_BAR + 256 + 1024;
   static constexpr int SMEM = RAW > 120 * 1024 ? RAW : 120 * 1024;
@@ -477,11 +482,10 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_kv128,
   uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   uint64_t* kv_full = bars + 0;
-  uint64_t* qd_full = bars + 1;    // [3] per stage
-  uint64_t* qd_empty = bars + 4;   // [3]
-  uint64_t* s_full = bars + 7;     // [2] per TMEM buffer
-  uint64_t* s_free = bars + 9;     // [2]
-  uint64_t* p_full = bars + 11;    // [2] per P^T/dS^T buffer
+  uint64_t* qd_full = bars + 1;    // [STAGES <= 4] per stage
+  uint64_t* qd_empty = bars + 5;   // [STAGES]
+  uint64_t* s_full = bars + 9;     // [2] per TMEM buffer
+  uint64_t* p_full = bars + 11;    // [2]
   uint64_t* mm2_done = bars + 13;  // [2]
   uint64_t* drain = bars + 15;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
@@ -506,8 +510,7 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_kv128,
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&s_free[i], 128);   // buffer i belongs to compute warpgroup i
-      mbar_init(&p_full[i], 128);
+      mbar_init(&p_full[i], 128);   // buffer i belongs to compute warpgroup i
       mbar_init(&mm2_done[i], 1);
     }
     mbar_init(drain, 1);
@@ -555,21 +558,20 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_kv128,
     }
   } else if (warp == 1 || warp == 10) {
     // Two issuers, each blocking only on its own barriers: warp 1 issues
-    // S^T/dP^T of block k (once its q/dO stage has landed and the compute of
-    // block k-2 has copied its scores out of tensor memory), warp 10 issues
-    // dV/dK of block k (once its P^T/dS^T are in shared memory) and releases
+    // S^T/dP^T of block k (once its q/dO stage has landed and the dV/dK MMAs
+    // of block k-2 have read P^T/dS^T out of the same buffer), warp 10 issues
+    // dV/dK of block k (once its P^T/dS^T are in tensor memory) and releases
     // the stage.  Neither stream waits behind the other.
     if (lane == 0) {
       constexpr uint32_t id_s = idesc_f32acc(128, C::BQ, false, false, true);
       constexpr uint32_t id_acc = idesc_f32acc(128, DH, false, true, true);
       const uint32_t sk = smem_u32(smem + C::OFF_K), sv = smem_u32(smem + C::OFF_V);
-      const uint32_t spt = smem_u32(smem + C::OFF_PT);
       bool ok = wait_bar(kv_full, 0, ctl, ERR_ATTN_DKDV_WAIT);
       if (warp == 1) {
         for (int k = 0; ok && k < nsteps; ++k) {
           const int bf = k & 1, st = k % C::STAGES;
           if (!(ok = wait_bar(&qd_full[st], (k / C::STAGES) & 1, ctl, ERR_ATTN_DKDV_WAIT))) break;
-          if (!(ok = wait_bar(&s_free[bf], ((k >> 1) & 1) ^ 1, ctl, ERR_ATTN_DKDV_WAIT))) break;
+          if (!(ok = wait_bar(&mm2_done[bf], ((k >> 1) & 1) ^ 1, ctl, ERR_ATTN_DKDV_WAIT))) break;
           tc_fence_after();
           const uint32_t sq = smem_u32(smem + C::OFF_ST + st * C::STAGE_BYTES);
           const uint32_t sd = sq + C::Q_BYTES;
@@ -589,13 +591,12 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_kv128,
           tc_fence_after();
           const uint32_t sq = smem_u32(smem + C::OFF_ST + sj * C::STAGE_BYTES);
           const uint32_t sd = sq + C::Q_BYTES;
-          const uint32_t pt = spt + 2 * bj * C::T_BYTES, dst = pt + C::T_BYTES;
 #pragma unroll
-          for (int kk = 0; kk < C::BQ / 16; ++kk) {
-            tc_mma_f16(t_dv, kmajor_desc(pt, C::BK, kk), mnmajor_desc(sd, C::BQ, kk), id_acc,
-                       (k | kk) != 0);
-            tc_mma_f16(t_dk, kmajor_desc(dst, C::BK, kk), mnmajor_desc(sq, C::BQ, kk), id_acc,
-                       (k | kk) != 0);
+          for (int kk = 0; kk < C::BQ / 16; ++kk) {   // 16 queries = 8 columns per step
+            tc_mma_f16_ts(t_dv, tmem + bj * 128 + 8 * kk, mnmajor_desc(sd, C::BQ, kk), id_acc,
+                          (k | kk) != 0);
+            tc_mma_f16_ts(t_dk, tmem + bj * 128 + 64 + 8 * kk, mnmajor_desc(sq, C::BQ, kk), id_acc,
+                          (k | kk) != 0);
           }
           tc_commit(&mm2_done[bj]);
           tc_commit(&qd_empty[sj]);   // the scores of block k completed before its P^T existed
@@ -622,25 +623,21 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_kv128,
       tc_fence_after();
       const float* vl = reinterpret_cast<const float*>(smem + C::OFF_VEC + (k % C::STAGES) * 2 * C::VEC_BYTES);
       const float* vd = vl + C::BQ;
-      uint8_t* pt = smem + C::OFF_PT + 2 * bf * C::T_BYTES;
-      uint8_t* dst = pt + C::T_BYTES;
-      // S^T and dP^T leave tensor memory in two 32-column halves; the buffer is
-      // handed back right after the second half is copied, so the scores of
-      // block k+2 are computed while this block's P^T and dS^T are finished.
-      // Each half goes to shared memory as soon as it is done (register budget
-      // of 320 threads).
-      const bool diag = p.causal && kpos > qs;   // some query of this block precedes key kpos
-      bool fail = false;
-#pragma unroll
+      // S^T and dP^T leave tensor memory in two 32-column halves; P^T and dS^T
+      // of each half (fp16 pairs, 16 columns) are written back over the half
+      // of S^T / dP^T just copied out.  The buffer was free once the dV/dK
+      // MMAs of block k-2 completed, which the score MMAs of this block
+      // already waited for.
+      const uint32_t t_st = tmem + bf * 128 + lane_off;
+      // Queries qs + qi with qi < qmin precede key kpos and are masked (causal):
+      // a select per element, no branches.
+      const int qmin = p.causal ? kpos - qs : 0;
+#pragma unroll 1
       for (int c = 0; c < 2; ++c) {
         uint32_t rs[32], rd[32];
-        tmem_ld32(tmem + bf * 128 + lane_off + c * 32, rs);
-        tmem_ld32(tmem + bf * 128 + 64 + lane_off + c * 32, rd);
+        tmem_ld32(t_st + c * 32, rs);
+        tmem_ld32(t_st + 64 + c * 32, rd);
         tc_wait_ld();
-        if (c == 1) {
-          tc_fence_before();
-          mbar_arrive(&s_free[bf]);
-        }
         uint32_t pk[16], dk[16];   // fp16 pairs of P^T and dS^T
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
@@ -650,28 +647,18 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_kv128,
             const int qi = c * 32 + e + h2;
             // Padded queries carry lse2 = +inf and dvec = 0, so they give 0.
             float x = fast_exp2(__uint_as_float(rs[e + h2]) * p.scale_log2 - vl[qi]);
-            if (diag && kpos > qs + qi) x = 0.f;
+            x = qi < qmin ? 0.f : x;
             pe[h2] = x;
             de[h2] = x * (__uint_as_float(rd[e + h2]) - vd[qi]);
           }
           pk[e / 2] = pack_f16x2(pe[0], pe[1]);
           dk[e / 2] = pack_f16x2(de[0], de[1]);
         }
-        // The P^T/dS^T buffer bf was last read by the dV/dK MMAs of block k-2.
-        if (c == 0 && k >= 2 &&
-            !__all_sync(0xffffffffu, wait_bar(&mm2_done[bf], (u - 1) & 1, ctl, ERR_ATTN_DKDV_WAIT))) {
-          fail = true;
-          break;
-        }
-#pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          const uint32_t off = sw128_offset(C::BK, r, c * 32 + g * 8);
-          *reinterpret_cast<uint4*>(pt + off) = make_uint4(pk[4 * g], pk[4 * g + 1], pk[4 * g + 2], pk[4 * g + 3]);
-          *reinterpret_cast<uint4*>(dst + off) = make_uint4(dk[4 * g], dk[4 * g + 1], dk[4 * g + 2], dk[4 * g + 3]);
-        }
+        tmem_st16(t_st + c * 16, pk);
+        tmem_st16(t_st + 64 + c * 16, dk);
       }
-      if (fail) { ok = false; break; }
-      fence_proxy_async_smem();
+      tc_wait_st();
+      tc_fence_before();
       mbar_arrive(&p_full[bf]);
     }
     // Every product has completed once `drain` (committed after the last one)
@@ -725,9 +712,7 @@ struct DqCfg {
   static constexpr int OFF_Q = 0, OFF_DO = Q_BYTES;
   static constexpr int STAGES = 4;                           // K / V ring depth
   static constexpr int OFF_ST = 2 * Q_BYTES;                 // stage s: k at +s*2*K, v at +K
-  static constexpr int DS_BYTES = BQ * BK * 2;
-  static constexpr int OFF_DS = OFF_ST + STAGES * 2 * K_BYTES;  // buffer b: dS at +b*DS
-  static constexpr int OFF_BAR = OFF_DS + 2 * DS_BYTES;
+  static constexpr int OFF_BAR = OFF_ST + STAGES * 2 * K_BYTES;
   static constexpr int RAW = OFF_BAR + 256 + 1024;
   static constexpr int SMEM = RAW > 120 * 1024 ? RAW : 120 * 1024;
 };
@@ -789,7 +774,9 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q128,
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t t_dq = tmem + 256;   // buffer j: S at 128j, dP at 128j + 64
+  // TMEM columns: buffer j holds S at 128j, dP at 128j + 64 and dS (fp16 pairs)
+  // at 384 + 32j; dQ accumulates at 256.
+  const uint32_t t_dq = tmem + 256;
 
   if (warp == 0) {
     if (lane == 0) {
@@ -822,7 +809,6 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q128,
       constexpr uint32_t id_s = idesc_f32acc(128, C::BK, false, false, true);
       constexpr uint32_t id_acc = idesc_f32acc(128, DH, false, true, true);
       const uint32_t sq = smem_u32(smem + C::OFF_Q), sd = smem_u32(smem + C::OFF_DO);
-      const uint32_t sds = smem_u32(smem + C::OFF_DS);
       bool ok = wait_bar(q_full, 0, ctl, ERR_ATTN_DQ_WAIT);
       if (warp == 1) {
         for (int k = 0; ok && k < nsteps; ++k) {
@@ -848,9 +834,9 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q128,
           tc_fence_after();
           const uint32_t sk = smem_u32(smem + C::OFF_ST + sj * 2 * C::K_BYTES);
 #pragma unroll
-          for (int kk = 0; kk < C::BK / 16; ++kk)
-            tc_mma_f16(t_dq, kmajor_desc(sds + bj * C::DS_BYTES, C::BQ, kk),
-                       mnmajor_desc(sk, C::BK, kk), id_acc, (k | kk) != 0);
+          for (int kk = 0; kk < C::BK / 16; ++kk)   // 16 keys = 8 columns of dS per step
+            tc_mma_f16_ts(t_dq, tmem + 384 + 32 * bj + 8 * kk, mnmajor_desc(sk, C::BK, kk),
+                          id_acc, (k | kk) != 0);
           tc_commit(&mm2_done[bj]);
           tc_commit(&kv_empty[sj]);   // the scores of block k completed before its dS existed
         }
@@ -878,7 +864,6 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q128,
       const int ks = k * C::BK;
       if (!__all_sync(0xffffffffu, wait_bar(&s_full[bf], u & 1, ctl, ERR_ATTN_DQ_WAIT))) { ok = false; break; }
       tc_fence_after();
-      uint8_t* sds = smem + C::OFF_DS + bf * C::DS_BYTES;
       // Copy S and dP out of tensor memory and hand the buffer back first.
       uint32_t rs0[32], rs1[32], rd0[32], rd1[32];
       tmem_ld32(tmem + bf * 128 + lane_off, rs0);
@@ -888,28 +873,30 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q128,
       tc_wait_ld();
       tc_fence_before();
       mbar_arrive(&s_free[bf]);
-      const bool edge = (p.causal && ks + C::BK - 1 > q) || ks + C::BK > p.S;
+      // Keys past the last visible one (after the query, or past S) are
+      // masked: a select per element against a bound fixed once per block.
+      const int kmax = (p.causal ? min(q, p.S - 1) : p.S - 1) - ks;
       auto ds = [&](const uint32_t (&rs)[32], uint32_t (&rd)[32], int c) {
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
-          const int kpos = ks + c * 32 + e;
           float pe = fast_exp2(__uint_as_float(rs[e]) * p.scale_log2 - l2);
-          if (edge && ((p.causal && kpos > q) || kpos >= p.S)) pe = 0.f;
+          pe = c * 32 + e > kmax ? 0.f : pe;
           rd[e] = __float_as_uint(pe * (__uint_as_float(rd[e]) - dv));
         }
       };
       ds(rs0, rd0, 0);
       ds(rs1, rd1, 1);
-      // The dS buffer bf was last read by the dQ MMAs of block k-2.
-      if (k >= 2 && !__all_sync(0xffffffffu, wait_bar(&mm2_done[bf], (u - 1) & 1, ctl, ERR_ATTN_DQ_WAIT))) { ok = false; break; }
+      uint32_t pk[32];   // dS as fp16 pairs, 64 keys
 #pragma unroll
-      for (int g = 0; g < 4; ++g) {
-        *reinterpret_cast<uint4*>(sds + sw128_offset(C::BQ, r, g * 8)) =
-            pack8_f16(reinterpret_cast<const float*>(&rd0[g * 8]));
-        *reinterpret_cast<uint4*>(sds + sw128_offset(C::BQ, r, 32 + g * 8)) =
-            pack8_f16(reinterpret_cast<const float*>(&rd1[g * 8]));
+      for (int e = 0; e < 16; ++e) {
+        pk[e] = pack_f16x2(__uint_as_float(rd0[2 * e]), __uint_as_float(rd0[2 * e + 1]));
+        pk[16 + e] = pack_f16x2(__uint_as_float(rd1[2 * e]), __uint_as_float(rd1[2 * e + 1]));
       }
-      fence_proxy_async_smem();
+      // The dS columns of buffer bf were last read by the dQ MMAs of block k-2.
+      if (k >= 2 && !__all_sync(0xffffffffu, wait_bar(&mm2_done[bf], (u - 1) & 1, ctl, ERR_ATTN_DQ_WAIT))) { ok = false; break; }
+      tmem_st32(tmem + 384 + 32 * bf + lane_off, pk);
+      tc_wait_st();
+      tc_fence_before();
       mbar_arrive(&p_full[bf]);
     }
     // As in the dK/dV kernel: `drain` completes after the last product.
