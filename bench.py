@@ -38,6 +38,11 @@ METRIC = "sharded-layer TFLOP/s (bf16 fwd+bwd, 1 B200) and % of dense BF16 peak"
 WORKLOAD = "layer_fwdbwd_B4_S2048_D4096_H32_F16384_t8"
 NOMINAL_BF16_TFLOPS = 2250.0
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per GEMM launch,
+# averaged over the 12 GEMM launches of one layer step, from an ncu capture of
+# the current GEMM kernel (the launch-by-launch table is kept with the ncu
+# summaries).  To be re-measured whenever the GEMM kernel changes.
+GEMM_DRAM_BYTES_PER_LAUNCH = {"layer_fwdbwd_B4_S2048_D4096_H32_F16384_t8": 953.7e6}
 PARAMS = ("ln1_g", "ln1_b", "wqkv", "bqkv", "wout", "bout", "ln2_g", "ln2_b", "w1", "b1", "w2", "b2")
 
 
@@ -362,9 +367,10 @@ def run_ours(args):
         n, fl, ms = by_kind[dom]
         achieved = fl / (ms * 1e-3) / 1e12 if ms > 0 else 0.0
         peak = peaks["bf16_tflops_sustained"]
+        traffic = GEMM_DRAM_BYTES_PER_LAUNCH.get(w.name) if dom == "gemm" else None
         roofline = {"bound": "tensor", "kernel": f"{dom} (tcgen05)", "achieved": achieved,
                     "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
-                    "peak_source": f"{peak_src} bf16_tflops_sustained", "traffic": None,
+                    "peak_source": f"{peak_src} bf16_tflops_sustained", "traffic": traffic,
                     "launches": n, "avg_launch_ms": ms / n,
                     "avg_launch_gflop": fl / n / 1e9}
     breakdown = {k: {"launches": v[0], "ms_per_step": v[2] / args.steps,
@@ -375,7 +381,7 @@ def run_ours(args):
     # ---- CPU oracle baseline (rank 0, N = 1 only), after the GPU timing
     cpu = None
     if world == 1 and not args.no_cpu_baseline and args.workload == WORKLOAD:
-        oseq = 512
+        oseq = 1024
         cv, csec, cs = time_oracle(oseq, 2)
         cpu = {"value": cv, "unit": "TFLOP/s", "cores": cores_used(), "kind": "oracle",
                "sample": (f"one sequence of {oseq} tokens of the workload (batch 1, full widths), "
