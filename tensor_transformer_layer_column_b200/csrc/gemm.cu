@@ -37,7 +37,7 @@ bool encode_operand(CUtensorMap* map, const OperandDesc& d, uint32_t box_outer) 
   const cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = fn(map, d.f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(d.ptr), dims, strides,
                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
@@ -62,7 +62,7 @@ bool encode_operand_il(CUtensorMap* map, const OperandDesc& d, uint32_t chunks) 
   CUresult r = fn(map, d.f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5,
                   const_cast<void*>(d.ptr), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
@@ -157,7 +157,7 @@ tp_status launch_gemm(const GemmProblem& g, cudaStream_t stream) {
   a.b_src = g.b.src;
   const long long tiles = (long long)a.m_shards * a.mb_per_shard * a.n_shards * a.nb_per_shard;
   a.num_tiles = (int)tiles;
-  a.group_m = 16;
+  a.group_m = 8;
   a.epi = g.epi;
   a.c = static_cast<__nv_bfloat16*>(g.c);
   a.c2 = static_cast<__nv_bfloat16*>(g.c2);
