@@ -417,34 +417,44 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q128,
 // =====================================================================================
 // Dv = rowsum(dO * O) and lse2 = lse * log2(e) for every (batch, head, query),
 // written with rows padded to S_pad: padded queries get lse2 = +inf, Dv = 0.
-__global__ void attn_bwd_prep_kernel(const uint16_t* __restrict__ o, const uint16_t* __restrict__ dout,
-                                     const float* __restrict__ lse, float* __restrict__ dvec,
-                                     float* __restrict__ lse2, int B, int S, int S_pad, int H,
-                                     int Ht, int dh, int Dt, long long T) {
-  const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  if (idx >= (long long)B * H * S_pad) return;
-  const int s = (int)(idx % S_pad);
-  const long long bh = idx / S_pad;
-  if (s >= S) {
-    dvec[idx] = 0.f;
-    lse2[idx] = INFINITY;
-    return;
-  }
-  const int h = (int)(bh % H);
-  const int b = (int)(bh / H);
-  const int shard = h / Ht, hl = h - shard * Ht;
-  const long long off = (long long)shard * T * Dt + ((long long)b * S + s) * Dt + hl * dh;
+// dh/8 consecutive threads share one row (8 elements each, one 16-byte load
+// of O and of dO) and reduce with shuffles, so a warp reads whole rows.
+__global__ void __launch_bounds__(256)
+attn_bwd_prep_kernel(const uint16_t* __restrict__ o, const uint16_t* __restrict__ dout,
+                     const float* __restrict__ lse, float* __restrict__ dvec,
+                     float* __restrict__ lse2, int B, int S, int S_pad, int H, int Ht, int dh,
+                     int Dt, long long T) {
+  const int tpr = dh >> 3;                    // threads per row: 8 or 16
+  const int rpb = blockDim.x / tpr;
+  const long long row = (long long)blockIdx.x * rpb + threadIdx.x / tpr;
+  const int sub = threadIdx.x % tpr;
+  const bool in = row < (long long)B * H * S_pad;
+  const int s = in ? (int)(row % S_pad) : 0;
+  const long long bh = in ? row / S_pad : 0;
   float acc = 0.f;
-  for (int d = 0; d < dh; d += 8) {
-    const uint4 a = *reinterpret_cast<const uint4*>(o + off + d);
-    const uint4 g = *reinterpret_cast<const uint4*>(dout + off + d);
+  if (in && s < S) {
+    const int h = (int)(bh % H);
+    const int b = (int)(bh / H);
+    const int shard = h / Ht, hl = h - shard * Ht;
+    const long long off =
+        (long long)shard * T * Dt + ((long long)b * S + s) * Dt + hl * dh + sub * 8;
+    const uint4 a = *reinterpret_cast<const uint4*>(o + off);
+    const uint4 g = *reinterpret_cast<const uint4*>(dout + off);
     const uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wg[4] = {g.x, g.y, g.z, g.w};
 #pragma unroll
     for (int k = 0; k < 4; ++k)
       acc += bf16_lo(wa[k]) * f16_lo(wg[k]) + bf16_hi(wa[k]) * f16_hi(wg[k]);
   }
-  dvec[idx] = acc;
-  lse2[idx] = lse[bh * S + s] * kLog2e;
+  for (int m = tpr >> 1; m > 0; m >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, m);
+  if (in && sub == 0) {
+    if (s >= S) {
+      dvec[row] = 0.f;
+      lse2[row] = INFINITY;
+    } else {
+      dvec[row] = acc;
+      lse2[row] = lse[bh * S + s] * kLog2e;
+    }
+  }
 }
 
 // ---------------------------------------------------------------- dK / dV
@@ -1030,7 +1040,8 @@ tp_status bwd_launch(const uint16_t* qkv, const uint16_t* o, const float* lse, c
   const long long n = (long long)a.B * a.H * a.S_pad;
   {
     TraceScope ts(st, TK_ATTN_BWD_PREP);
-    attn_bwd_prep_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(
+    const long long rows_per_block = 256 / (DH / 8);
+    attn_bwd_prep_kernel<<<(unsigned)((n + rows_per_block - 1) / rows_per_block), 256, 0, st>>>(
         o, dout, lse, dvec, lse2, a.B, a.S, a.S_pad, a.H, a.Ht, DH, a.Dt, a.T);
   }
   if (cudaGetLastError() != cudaSuccess) return TP_ERR_CUDA;
