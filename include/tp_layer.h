@@ -345,6 +345,17 @@ tp_status tp_layernorm_bwd_noalloc(const tp_bf16* dy, const tp_bf16* x, const tp
                                    int rows, int D, tp_bf16* dx, tp_bf16* dgamma, tp_bf16* dbeta,
                                    tp_stream stream);
 
+/* ------------------------------------------------------------------ failure-detection self-test
+ * Not an operation of the pages: a check of the library's bounded device
+ * waits.  tp_selftest_wait_timeout enqueues one small kernel whose thread
+ * waits on a barrier that nothing completes, through the same bounded wait
+ * every kernel here uses, with limit limit_ns (1 ms to 10 s); when the limit
+ * expires it records code 0x0F1 in the device error word and returns.  A
+ * following tp_check_error then reports TP_ERR_TIMEOUT with *code == 0x0F1 and
+ * clears the word.  Nothing faults or hangs; the context stays usable.
+ * INVALID_ARG for a limit outside that range. */
+tp_status tp_selftest_wait_timeout(unsigned long long limit_ns, tp_stream stream);
+
 /* ------------------------------------------------------------------ launch trace
  * Measurement support (the pages describe no tracing; this exists so that a
  * bench can time individual kernels inside a longer step on their own stream).

@@ -25,7 +25,7 @@ __all__ = [
     "unshard_qkv_heads", "mlp_fwd", "mlp_bwd", "attn_fwd", "attn_bwd", "layer_fwd", "layer_bwd",
     "layernorm_fwd", "layernorm_bwd", "layernorm_bwd_workspace_size", "layernorm_bwd_noalloc",
     "LaunchTrace",
-    "TRACE_KINDS",
+    "TRACE_KINDS", "selftest_wait_timeout",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -114,6 +114,7 @@ _SIGS = {
                          ctypes.c_size_t, _P],
     "tp_layernorm_bwd_noalloc": [_P, _P, _P, _P, _P, _P, ctypes.c_int, ctypes.c_int, _P, _P, _P,
                                  _P],
+    "tp_selftest_wait_timeout": [ctypes.c_ulonglong, _P],
     "tp_trace_begin": [ctypes.POINTER(ctypes.c_void_p), ctypes.POINTER(ctypes.c_int),
                        ctypes.POINTER(ctypes.c_double), ctypes.c_int],
     "tp_trace_end": [],
@@ -307,6 +308,15 @@ def layer_bwd_recompute(dims, x, params: dict, dy, dx, grads: dict, ws, stream=N
     _check(lib().tp_layer_bwd_recompute(ctypes.byref(dims), _ptr(x), ctypes.byref(p), _ptr(dy),
                                         _ptr(dx), ctypes.byref(g), wp, wn, _stream(stream, x)),
            "tp_layer_bwd_recompute")
+
+
+def selftest_wait_timeout(limit_ns: int, stream=None):
+    """Enqueue the bounded-wait self-test (see include/tp_layer.h); read the
+    outcome with check_error() afterwards."""
+    import torch
+    s = stream if stream is not None else torch.cuda.current_stream()
+    _check(lib().tp_selftest_wait_timeout(int(limit_ns), ctypes.c_void_p(s.cuda_stream)),
+           "tp_selftest_wait_timeout")
 
 
 def layernorm_fwd(x, gamma, beta, rows, D, eps, y, mean, rstd, stream=None):

@@ -107,3 +107,9 @@ def test_recompute_entry_points_host_side():
     st = lib.tp_layer_bwd_recompute(ctypes.byref(small), 16, ctypes.byref(p), 16, 16,
                                     ctypes.byref(g), None, 0, None)
     assert st == 1
+
+
+def test_selftest_limit_checked_on_host():
+    lib = tl.lib()
+    assert lib.tp_selftest_wait_timeout(0, None) == 1            # below 1 ms
+    assert lib.tp_selftest_wait_timeout(20_000_000_000, None) == 1   # above 10 s
