@@ -110,6 +110,14 @@ def cores_used():
         return os.cpu_count() or 1
 
 
+def base_config(w: Workload, world: int) -> dict:
+    """The workload identity both arms report in their JSON line."""
+    return {"workload": w.name, "batch": w.batch, "seq": w.seq, "hidden": w.hidden,
+            "ffn": w.ffn, "heads": w.heads, "head_dim": w.head_dim, "t": w.t,
+            "causal": w.causal, "flop_per_step": w.flops(),
+            "parallelism": f"t{w.t} shards on each GPU; {world} independent replica(s)"}
+
+
 def run_reference(args):
     world, rank, _ = dist_env()
     if rank != 0:
@@ -131,7 +139,7 @@ def run_reference(args):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": sec * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "sample_seq": seq},
+        "config": base_config(workload(WORKLOAD), world),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores_used(),
                          "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
@@ -394,14 +402,10 @@ def run_ours(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": w.name, "batch": w.batch, "seq": w.seq,
-                       "hidden": w.hidden, "ffn": w.ffn, "heads": w.heads,
-                       "head_dim": w.head_dim, "t": w.t, "causal": w.causal,
-                       "flop_per_step": flops_step,
+            "config": {**base_config(w, world),
                        "l2": (f"inputs larger than L2: {in_bytes / 2**20:.0f} MiB of inputs per "
                               "step vs 120 MiB of L2, no flush" if in_bytes > 126e6
-                              else "L2 not flushed: inputs smaller than L2"),
-                       "parallelism": f"t{w.t} shards on each GPU; {world} independent replica(s)"},
+                              else "L2 not flushed: inputs smaller than L2")},
             "pct_dense_bf16_peak": 100.0 * value / world / NOMINAL_BF16_TFLOPS,
             "pct_measured_bf16_peak": 100.0 * value / world / peaks["bf16_tflops"],
             "peak_source": peak_src,
