@@ -713,7 +713,9 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_kv128,
 }
 
 // ---------------------------------------------------------------- dQ
-// Per 128-query block, walk 64-key blocks, with the same double buffering.
+// Per 128-query block, walk 64-key blocks through a 4-stage K/V ring.  Two
+// S/dP buffers in TMEM, one per compute warpgroup; dS (fp16 pairs) goes to
+// its own TMEM columns and is the A operand of dQ += dS k.
 template <int DH>
 struct DqCfg {
   static constexpr int BQ = 128, BK = 64, CH = DH / 64;
