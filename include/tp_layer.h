@@ -60,7 +60,8 @@ typedef void* tp_stream;   /* cudaStream_t */
 typedef enum {
   TP_OK = 0,
   TP_ERR_INVALID_ARG = 1,  /* null pointer, non-positive size, t not dividing H or F, D != H*dh */
-  TP_ERR_UNSUPPORTED = 2,  /* valid but not provided: t not in {1,2,4,8}, dh not in {64,128} */
+  TP_ERR_UNSUPPORTED = 2,  /* valid but not provided: t not in {1,2,4,8}, dh not in {64,128},
+                              batch*seq >= 2^31, layer entry points with hidden > 8192 */
   TP_ERR_MISALIGNED = 3,   /* pointer not 16-byte aligned or a row not a multiple of 8 elements */
   TP_ERR_WORKSPACE = 4,    /* workspace pointer null or smaller than tp_workspace_size */
   TP_ERR_CUDA = 5,         /* a CUDA runtime call or kernel launch failed */

@@ -109,6 +109,8 @@ tp_status check_common(const tp_dims* d) {
   if (!d) return TP_ERR_INVALID_ARG;
   if (d->batch < 0 || d->seq < 0 || d->hidden <= 0 || d->t <= 0) return TP_ERR_INVALID_ARG;
   if (!supported_t(d->t)) return TP_ERR_UNSUPPORTED;
+  // Row counts and tensor-map coordinates are 32-bit.
+  if ((long long)d->batch * d->seq > 0x7FFFFFFFLL) return TP_ERR_UNSUPPORTED;
   if (d->hidden % d->t) return TP_ERR_INVALID_ARG;
   if (d->hidden % 8) return TP_ERR_MISALIGNED;
   return TP_OK;

@@ -113,3 +113,15 @@ def test_selftest_limit_checked_on_host():
     lib = tl.lib()
     assert lib.tp_selftest_wait_timeout(0, None) == 1            # below 1 ms
     assert lib.tp_selftest_wait_timeout(20_000_000_000, None) == 1   # above 10 s
+
+
+def test_size_limits_reported_on_host():
+    lib = tl.lib()
+    big = tl.Dims.of(65536, 32768, 4096, 16384, 32, 128, 8)      # batch*seq = 2^31
+    assert tl.workspace_size(tl.OP_LAYER_BWD, big) == 0
+    st = lib.tp_mlp_fwd(ctypes.byref(big), 16, 16, None, 16, None, None, 16, 16, 16, None, 0, None)
+    assert st == 2  # TP_ERR_UNSUPPORTED
+    wide = tl.Dims.of(1, 8, 16384, 65536, 128, 128, 8)             # layer LayerNorm limit
+    p = tl.LayerParams()
+    st = lib.tp_layer_fwd_nosave(ctypes.byref(wide), 16, ctypes.byref(p), 16, None, 0, None)
+    assert st == 2
