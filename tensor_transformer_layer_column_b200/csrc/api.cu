@@ -685,12 +685,15 @@ tp_status tp_layernorm_bwd(const tp_bf16* dy, const tp_bf16* x, const tp_bf16* g
 }
 
 // ------------------------------------------------------------------ pre-LN layer
-static tp_status check_layer_ptrs(const tp_layer_params* p, const tp_layer_acts* a) {
+// Saved activations (and x, y) may be NULL when the layer has zero tokens.
+static bool has_tokens(const tp_dims* d) { return (long long)d->batch * d->seq > 0; }
+
+static tp_status check_layer_ptrs(const tp_layer_params* p, const tp_layer_acts* a, bool tok) {
   if (!p || !a) return TP_ERR_INVALID_ARG;
   if (!all_set(p->ln1_g, p->ln1_b, p->wqkv, p->wout, p->ln2_g, p->ln2_b, p->w1, p->w2))
     return TP_ERR_INVALID_ARG;
-  if (!all_set(a->u1, a->mean1, a->rstd1, a->qkv, a->o, a->lse, a->h, a->u2, a->mean2, a->rstd2,
-               a->a, a->hact))
+  if (tok && !all_set(a->u1, a->mean1, a->rstd1, a->qkv, a->o, a->lse, a->h, a->u2, a->mean2,
+                      a->rstd2, a->a, a->hact))
     return TP_ERR_INVALID_ARG;
   if (!all_aligned(p->ln1_g, p->ln1_b, p->wqkv, p->bqkv, p->wout, p->bout, p->ln2_g, p->ln2_b,
                    p->w1, p->b1, p->w2, p->b2))
@@ -795,8 +798,8 @@ tp_status tp_layer_fwd(const tp_dims* dims, const tp_bf16* x, const tp_layer_par
                        const tp_layer_acts* a, tp_bf16* y, void* ws, size_t ws_bytes, tp_stream s) {
   tp_status st = check_layer(dims);
   if (st != TP_OK) return st;
-  if (!x || !y) return TP_ERR_INVALID_ARG;
-  if ((st = check_layer_ptrs(p, a)) != TP_OK) return st;
+  if (has_tokens(dims) && !all_set(x, y)) return TP_ERR_INVALID_ARG;
+  if ((st = check_layer_ptrs(p, a, has_tokens(dims))) != TP_OK) return st;
   if (!all_aligned(x, y)) return TP_ERR_MISALIGNED;
   const Sizes z = sizes_of(*dims);
   cudaStream_t cs = (cudaStream_t)s;
@@ -812,7 +815,7 @@ tp_status tp_layer_bwd(const tp_dims* dims, const tp_bf16* x, const tp_layer_par
                        const tp_layer_grads* g, void* ws, size_t ws_bytes, tp_stream s) {
   tp_status st = check_layer(dims);
   if (st != TP_OK) return st;
-  if ((st = check_layer_ptrs(p, a)) != TP_OK) return st;
+  if ((st = check_layer_ptrs(p, a, has_tokens(dims))) != TP_OK) return st;
   if ((st = check_layer_grads(dims, x, dy, dx, g)) != TP_OK) return st;
   const Sizes z = sizes_of(*dims);
   const size_t need = z.T ? layer_bwd_ws(z) : 0;
@@ -866,12 +869,12 @@ tp_status tp_layer_bwd_recompute(const tp_dims* dims, const tp_bf16* x, const tp
 }
 
 // ------------------------------------------------------------------ post-LN layer
-static tp_status check_postln_ptrs(const tp_layer_params* p, const tp_postln_acts* a) {
+static tp_status check_postln_ptrs(const tp_layer_params* p, const tp_postln_acts* a, bool tok) {
   if (!p || !a) return TP_ERR_INVALID_ARG;
   if (!all_set(p->ln1_g, p->ln1_b, p->wqkv, p->wout, p->ln2_g, p->ln2_b, p->w1, p->w2))
     return TP_ERR_INVALID_ARG;
-  if (!all_set(a->z1, a->mean1, a->rstd1, a->qkv, a->o, a->lse, a->h, a->z2, a->mean2, a->rstd2,
-               a->a, a->hact))
+  if (tok && !all_set(a->z1, a->mean1, a->rstd1, a->qkv, a->o, a->lse, a->h, a->z2, a->mean2,
+                      a->rstd2, a->a, a->hact))
     return TP_ERR_INVALID_ARG;
   if (!all_aligned(p->ln1_g, p->ln1_b, p->wqkv, p->bqkv, p->wout, p->bout, p->ln2_g, p->ln2_b,
                    p->w1, p->b1, p->w2, p->b2))
@@ -885,8 +888,8 @@ tp_status tp_postln_layer_fwd(const tp_dims* dims, const tp_bf16* x, const tp_la
                               tp_stream s) {
   tp_status st = check_layer(dims);
   if (st != TP_OK) return st;
-  if (!x || !y) return TP_ERR_INVALID_ARG;
-  if ((st = check_postln_ptrs(p, a)) != TP_OK) return st;
+  if (has_tokens(dims) && !all_set(x, y)) return TP_ERR_INVALID_ARG;
+  if ((st = check_postln_ptrs(p, a, has_tokens(dims))) != TP_OK) return st;
   if (!all_aligned(x, y)) return TP_ERR_MISALIGNED;
   const Sizes z = sizes_of(*dims);
   cudaStream_t cs = (cudaStream_t)s;
@@ -916,12 +919,8 @@ tp_status tp_postln_layer_bwd(const tp_dims* dims, const tp_bf16* x, const tp_la
                               const tp_layer_grads* g, void* ws, size_t ws_bytes, tp_stream s) {
   tp_status st = check_layer(dims);
   if (st != TP_OK) return st;
-  if (!x || !dy || !dx || !g) return TP_ERR_INVALID_ARG;
-  if ((st = check_postln_ptrs(p, a)) != TP_OK) return st;
-  if (!all_set(g->dwqkv, g->dwout, g->dw1, g->dw2)) return TP_ERR_INVALID_ARG;
-  if (!all_aligned(x, dy, dx, g->dln1_g, g->dln1_b, g->dwqkv, g->dbqkv, g->dwout, g->dbout,
-                   g->dln2_g, g->dln2_b, g->dw1, g->db1, g->dw2, g->db2))
-    return TP_ERR_MISALIGNED;
+  if ((st = check_postln_ptrs(p, a, has_tokens(dims))) != TP_OK) return st;
+  if ((st = check_layer_grads(dims, x, dy, dx, g)) != TP_OK) return st;
   const Sizes z = sizes_of(*dims);
   cudaStream_t cs = (cudaStream_t)s;
   if (z.T == 0) {

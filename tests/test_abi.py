@@ -125,3 +125,18 @@ def test_size_limits_reported_on_host():
     p = tl.LayerParams()
     st = lib.tp_layer_fwd_nosave(ctypes.byref(wide), 16, ctypes.byref(p), 16, None, 0, None)
     assert st == 2
+
+
+def test_layer_forward_accepts_null_activations_at_zero_tokens():
+    """torch gives NULL for empty tensors: with batch*seq == 0 the layer
+    forwards need no activation buffers and return before touching a device."""
+    lib = tl.lib()
+    d = tl.Dims.of(0, 64, 256, 1024, 2, 128, 2)
+    p = tl.LayerParams(ln1_g=16, ln1_b=16, wqkv=16, wout=16, ln2_g=16, ln2_b=16, w1=16, w2=16)
+    assert lib.tp_layer_fwd(ctypes.byref(d), None, ctypes.byref(p), ctypes.byref(tl.LayerActs()),
+                            None, None, 0, None) == 0
+    assert lib.tp_postln_layer_fwd(ctypes.byref(d), None, ctypes.byref(p),
+                                   ctypes.byref(tl.PostLNActs()), None, None, 0, None) == 0
+    d1 = tl.Dims.of(1, 64, 256, 1024, 2, 128, 2)   # with tokens the buffers are required
+    assert lib.tp_layer_fwd(ctypes.byref(d1), None, ctypes.byref(p), ctypes.byref(tl.LayerActs()),
+                            None, None, 0, None) == 1

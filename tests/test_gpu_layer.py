@@ -117,3 +117,23 @@ def test_postln_layer_full_size_B4_S2048_D4096_H32_F16384_t8():
     require_gpu()
     w = workload("layer_fwdbwd_B4_S2048_D4096_H32_F16384_t8")
     _run_and_compare_postln(w, make_inputs(w))
+
+
+@pytest.mark.parametrize("placement", ["pre", "post"])
+def test_layer_zero_tokens(placement):
+    """batch 0: the forward does nothing and every parameter gradient is zero."""
+    require_gpu()
+    w = Workload("layer_test", "layer_fwdbwd", batch=0, seq=64, hidden=256, ffn=1024, heads=2,
+                 head_dim=128, t=2)
+    inp = make_inputs(w, seed=5)
+    g = dev(inp)
+    layer = ShardedLayer(dims_of(w), {k: g[k] for k in PARAMS}, placement=placement)
+    layer.forward(g["x"])
+    grads = layer.alloc_grads()
+    for v in grads.values():
+        v.fill_(1.0)
+    layer.backward(g["dy"], grads=grads)
+    torch.cuda.synchronize()
+    assert_no_device_error()
+    for k, v in grads.items():
+        assert not v.float().abs().any(), k
