@@ -257,6 +257,29 @@ class Runner:
             self.mod.backward(dy, out=self.bwd_out)
 
 
+def hbm_bytes_per_step(w: Workload) -> dict:
+    """Algorithmic DRAM bytes per step of the HBM-bound kernel classes of the
+    pre-LN layer (each tensor read or written once; bf16/fp16 activations,
+    fp32 statistics).  Empty for other workloads."""
+    if w.kind != "layer_fwdbwd":
+        return {}
+    T, D, F = w.tokens, w.hidden, w.ffn
+    BHS = w.batch * w.heads * w.seq
+    BHS_pad = w.batch * w.heads * ((w.seq + 127) // 128 * 128)
+    return {
+        # LN1, LN2: read x, write u (2 bytes each), write mean and rstd
+        "ln_fwd": 2 * (4 * T * D + 8 * T),
+        # LN2, LN1 backward: read du, the LN input and the residual gradient, write dx
+        "ln_bwd": 2 * (8 * T * D + 8 * T),
+        # bias gradients: read dA, dqkv, dy and dh once
+        "colsum": 2 * T * F + 2 * T * 3 * D + 2 * T * D + 2 * T * D,
+        # Wqkv to fp16, forward and backward: read bf16, write fp16
+        "cast": 2 * (4 * D * 3 * D),
+        # Dv and lse2: read O and dO, read lse, write both padded rows
+        "attn_bwd_prep": 4 * T * D + 4 * BHS + 8 * BHS_pad,
+    }
+
+
 def recompute_flops(w: Workload) -> int:
     """FLOPs the recomputing backward adds: the forward without the MLP's
     second product (QKV and output projections, causal core, W1 product)."""
@@ -420,9 +443,14 @@ def run_ours(args):
                     "peak_source": f"{peak_src} bf16_tflops_sustained", "traffic": traffic,
                     "launches": n, "avg_launch_ms": ms / n,
                     "avg_launch_gflop": fl / n / 1e9}
+    hbm = hbm_bytes_per_step(w)
     breakdown = {k: {"launches": v[0], "ms_per_step": v[2] / args.steps,
                      "share": v[2] / max(1e-9, sum(x[2] for x in by_kind.values())),
-                     **({"tflops": v[1] / (v[2] * 1e-3) / 1e12} if v[1] > 0 and v[2] > 0 else {})}
+                     **({"tflops": v[1] / (v[2] * 1e-3) / 1e12} if v[1] > 0 and v[2] > 0 else {}),
+                     **({"algorithmic_bytes_per_step": hbm[k],
+                         "gbs": hbm[k] / (v[2] / args.steps * 1e-3) / 1e9,
+                         "frac_of_hbm": hbm[k] / (v[2] / args.steps * 1e-3) / 1e9 / peaks["hbm_gbs"]}
+                        if k in hbm and v[2] > 0 else {})}
                  for k, v in sorted(by_kind.items(), key=lambda kv: -kv[1][2])}
 
     # ---- CPU oracle baseline (rank 0, N = 1 only), after the GPU timing

@@ -8,6 +8,7 @@ streams only; all arithmetic happens in libtplayer.so.
 """
 from __future__ import annotations
 
+import functools
 from typing import Dict, Optional
 
 import torch
@@ -62,6 +63,20 @@ def unpack_qkv(p: torch.Tensor, heads: int) -> torch.Tensor:
     return out
 
 
+def _nvtx(name: str):
+    """Wrap a sublayer call in an NVTX range (for timeline profilers)."""
+    def deco(fn):
+        @functools.wraps(fn)
+        def wrapper(*args, **kwargs):
+            torch.cuda.nvtx.range_push(name)
+            try:
+                return fn(*args, **kwargs)
+            finally:
+                torch.cuda.nvtx.range_pop()
+        return wrapper
+    return deco
+
+
 def _ws(op: int, dims: Dims, device) -> Optional[torch.Tensor]:
     n = workspace_size(op, dims)
     return torch.empty(max(n, 1), dtype=torch.uint8, device=device) if n else None
@@ -80,6 +95,7 @@ class ShardedMLP:
         self.device = w1.device
         self.ws = None
 
+    @_nvtx("tp.mlp.forward")
     def forward(self, x, resid=None, out: Optional[Dict] = None):
         d = self.dims
         T, D, F = d.batch * d.seq, d.hidden, d.ffn
@@ -91,6 +107,7 @@ class ShardedMLP:
         self.saved = (x, o["a"], o["h"])
         return o
 
+    @_nvtx("tp.mlp.backward")
     def backward(self, dy, dres=None, bias_grads=True, out: Optional[Dict] = None):
         d = self.dims
         T, D, F = d.batch * d.seq, d.hidden, d.ffn
@@ -122,6 +139,7 @@ class ShardedAttention:
         self.ws = None
         self.ws_fwd = None
 
+    @_nvtx("tp.attn.forward")
     def forward(self, x, resid=None, out: Optional[Dict] = None):
         d = self.dims
         T, D = d.batch * d.seq, d.hidden
@@ -137,6 +155,7 @@ class ShardedAttention:
         self.saved = (x, o["qkv"], o["o"], o["lse"])
         return o
 
+    @_nvtx("tp.attn.backward")
     def backward(self, dy, dres=None, bias_grads=True, out: Optional[Dict] = None):
         d = self.dims
         T, D = d.batch * d.seq, d.hidden
@@ -233,6 +252,7 @@ class ShardedLayer:
             return 0
         return sum(v.numel() * v.element_size() for v in self.alloc_acts().values())
 
+    @_nvtx("tp.layer.forward")
     def forward(self, x, acts=None, y=None):
         d = self.dims
         y = y if y is not None else _empty((d.batch * d.seq, d.hidden), device=self.device)
@@ -249,6 +269,7 @@ class ShardedLayer:
         self.saved = (x, acts)
         return y, acts
 
+    @_nvtx("tp.layer.backward")
     def backward(self, dy, dx=None, grads=None, bias_grads=True):
         d = self.dims
         x, acts = self.saved

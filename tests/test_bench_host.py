@@ -32,3 +32,15 @@ def test_both_arms_report_the_same_workload_identity():
     # Counted work of the layer step: MLP 12TDF = 6.597 T, projections 24TD^2 =
     # 3.299 T, causal core 3 x 4 dh B H S(S+1)/2 = 0.413 T.
     assert c["flop_per_step"] == 10_308_122_836_992
+
+
+def test_hbm_bytes_of_the_layer_step():
+    w = workload(LAYER)
+    b = bench.hbm_bytes_per_step(w)
+    T, D, F = w.tokens, w.hidden, w.ffn
+    assert b["ln_fwd"] == 2 * 4 * T * D + 16 * T                # 2 x (64 MiB in + 64 MiB out) + stats
+    assert b["ln_bwd"] == 16 * T * D + 16 * T                   # 2 x (3 reads + 1 write of [T][D])
+    assert b["colsum"] == 2 * T * (F + 5 * D)                   # dA, dqkv (3D), dy, dh
+    assert b["cast"] == 24 * D * D                              # Wqkv read + written, twice
+    assert abs(b["ln_bwd"] / 2**20 - 512.125) < 1e-9            # 512 MiB of rows + 128 KiB of stats
+    assert bench.hbm_bytes_per_step(workload("mlp_fwdbwd_T8192_D3072_F12288_t8")) == {}
