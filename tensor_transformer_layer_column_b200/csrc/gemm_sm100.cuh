@@ -1,7 +1,8 @@
 // Persistent, warp-specialised tcgen05 GEMM for the sharded sublayer.
 //
 // C[m, n] = epilogue( sum_k A[m, k] * B[k, n] ), bf16 or fp16 operands (A and
-// B of one type), fp32 accumulation in tensor memory, bf16 or fp16 output.
+// B of one type), fp32 accumulation in tensor memory, bf16, fp16 or fp32
+// output.
 //
 // Tensor-parallel structure ("How transformer layers actually decompose",
 // "The attention heads split"): the t shards of a column-parallel product
@@ -9,17 +10,24 @@
 // row-parallel product appear as K shards, walked one after the other into
 // the SAME tensor-memory accumulator, so the cross-shard sum that the pages
 // perform with an all-reduce happens in fp32 inside the MMA, in shard order
-// 0..t-1, with a single bf16 rounding in the epilogue.  Weight-gradient
-// products shard M or N the same way.
+// 0..t-1, with a single rounding in the epilogue.  Weight-gradient products
+// shard M or N the same way.
 //
-// Roles (192 threads, one CTA per SM):
-//   warp 0      TMA producer: streams A/B k-blocks into a 4-stage ring;
-//   warp 1      TMEM owner and MMA issuer (one thread): 4 x (128x256x16) MMAs
-//               per k-block into one of two 256-column accumulators;
-//   warps 2..5  epilogue: tcgen05.ld of their 32-lane quarter, bias / GeLU /
-//               GeLU-backward / residual, bf16 stores.  The second
-//               accumulator lets the epilogue of tile i overlap the MMAs of
-//               tile i+1.
+// Two kernels, both persistent with 192 threads (6 warps) per CTA:
+//   gemm_pair_sm100 (M > 128): clusters of two CTAs on two SMs compute
+//     256 x 256 tiles with tcgen05.mma.cta_group::2 (M = 256 split across the
+//     pair).  Each CTA's producer stages its half of A and of B through a
+//     6-stage TMA ring; the even CTA's single MMA thread issues 4 MMAs of
+//     256 x 256 x 16 per 64-wide k-block into one of two 256-column TMEM
+//     accumulators and commits stage releases to both CTAs.
+//   gemm_bf16_sm100 (M <= 128): one CTA per 128 x 256 tile, 4-stage ring,
+//     4 MMAs of 128 x 256 x 16 per k-block.
+// Roles in both: warp 0 TMA producer; warp 1 TMEM owner and MMA issuer (one
+// thread); warps 2..5 epilogue: tcgen05.ld of their 32-lane quarter, bias /
+// GeLU (writing A and H) / GeLU-backward / residual (bf16 or fp32), then the
+// stores.  The second accumulator lets the epilogue of tile i overlap the
+// MMAs of tile i+1.  Tiles are visited in groups of 8 M-blocks per N sweep so
+// that concurrently running tiles share A and B panels in L2.
 // Every wait is bounded; a timeout records an error code and the kernel
 // drains its own copies and MMAs, frees TMEM and returns.
 #pragma once
