@@ -26,6 +26,31 @@ def _empty(shape, dtype=BF16, device="cuda"):
     return torch.empty(shape, dtype=dtype, device=device)
 
 
+def _expect(name, t, shape, dtype=BF16, device=None, optional=False):
+    """Check a tensor argument before any library call: the C ABI takes raw
+    pointers, so a wrong shape or dtype would otherwise be read as garbage or
+    past the end of the buffer."""
+    if t is None:
+        if optional:
+            return
+        raise ValueError(f"{name} is required")
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name}: dtype {t.dtype}, expected {dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if device is not None and t.device != torch.device(device):
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+
+
+def _expect_all(given: Dict, spec: Dict, device, what: str, optional=()):
+    """Every tensor of a caller-provided buffer dict against its (shape, dtype);
+    keys in `optional` may be absent or None."""
+    for k, (shape, dtype) in spec.items():
+        _expect(f"{what}[{k!r}]", given.get(k), shape, dtype, device, optional=k in optional)
+
+
 def pack_cols(w: torch.Tensor, t: int) -> torch.Tensor:
     rows, cols = w.shape
     out = _empty((t, rows, cols // t), device=w.device)
@@ -88,6 +113,14 @@ class ShardedMLP:
     def __init__(self, dims: Dims, w1, b1, w2, b2):
         self.dims = dims
         t = dims.t
+        D, F = dims.hidden, dims.ffn
+        dev = w1.device if isinstance(w1, torch.Tensor) else None
+        _expect("w1", w1, (D, F), device=dev)
+        _expect("b1", b1, (F,), device=dev, optional=True)
+        _expect("w2", w2, (F, D), device=dev)
+        _expect("b2", b2, (D,), device=dev, optional=True)
+        if not w1.is_cuda:
+            raise ValueError("weights must live on a CUDA device")
         self.w1 = pack_cols(w1, t)           # [t][D][Ft]
         self.w2 = pack_rows(w2, t)           # [t][Ft][D]
         self.b1 = None if b1 is None else b1.contiguous()   # [F] == [t][Ft]
@@ -99,6 +132,11 @@ class ShardedMLP:
     def forward(self, x, resid=None, out: Optional[Dict] = None):
         d = self.dims
         T, D, F = d.batch * d.seq, d.hidden, d.ffn
+        _expect("x", x, (T, D), device=self.device)
+        _expect("resid", resid, (T, D), device=self.device, optional=True)
+        if out is not None:
+            _expect_all(out, {"y": ((T, D), BF16), "a": ((d.t, T, F // d.t), BF16),
+                              "h": ((d.t, T, F // d.t), BF16)}, self.device, "out")
         o = out if out is not None else {
             "y": _empty((T, D), device=self.device),
             "a": _empty((d.t, T, F // d.t), device=self.device),
@@ -112,6 +150,12 @@ class ShardedMLP:
         d = self.dims
         T, D, F = d.batch * d.seq, d.hidden, d.ffn
         x, a, h = self.saved
+        _expect("dy", dy, (T, D), device=self.device)
+        _expect("dres", dres, (T, D), device=self.device, optional=True)
+        if out is not None:
+            _expect_all(out, {"dx": ((T, D), BF16), "dw1": ((d.t, D, F // d.t), BF16),
+                              "dw2": ((d.t, F // d.t, D), BF16), "db1": ((F,), BF16),
+                              "db2": ((D,), BF16)}, self.device, "out", optional=("db1", "db2"))
         if self.ws is None:
             self.ws = _ws(OP_MLP_BWD, d, self.device)
         g = out if out is not None else {
@@ -131,6 +175,14 @@ class ShardedAttention:
     def __init__(self, dims: Dims, wqkv, bqkv, wout, bout):
         self.dims = dims
         t, H = dims.t, dims.heads
+        D = dims.hidden
+        dev = wqkv.device if isinstance(wqkv, torch.Tensor) else None
+        _expect("wqkv", wqkv, (D, 3 * D), device=dev)
+        _expect("bqkv", bqkv, (3 * D,), device=dev, optional=True)
+        _expect("wout", wout, (D, D), device=dev)
+        _expect("bout", bout, (D,), device=dev, optional=True)
+        if not wqkv.is_cuda:
+            raise ValueError("weights must live on a CUDA device")
         self.wqkv = pack_qkv(wqkv, H, t)                                  # [t][D][3Dt]
         self.bqkv = None if bqkv is None else pack_qkv(bqkv, H, t)        # [t][1][3Dt]
         self.wout = pack_rows(wout, t)                                    # [t][Dt][D]
@@ -143,6 +195,13 @@ class ShardedAttention:
     def forward(self, x, resid=None, out: Optional[Dict] = None):
         d = self.dims
         T, D = d.batch * d.seq, d.hidden
+        _expect("x", x, (T, D), device=self.device)
+        _expect("resid", resid, (T, D), device=self.device, optional=True)
+        if out is not None:
+            _expect_all(out, {"y": ((T, D), BF16), "qkv": ((d.t, T, 3 * D // d.t), torch.float16),
+                              "o": ((d.t, T, D // d.t), BF16),
+                              "lse": ((d.batch, d.heads, d.seq), torch.float32)},
+                        self.device, "out")
         o = out if out is not None else {
             "y": _empty((T, D), device=self.device),
             "qkv": _empty((d.t, T, 3 * D // d.t), dtype=torch.float16, device=self.device),
@@ -160,6 +219,13 @@ class ShardedAttention:
         d = self.dims
         T, D = d.batch * d.seq, d.hidden
         x, qkv, o, lse = self.saved
+        _expect("dy", dy, (T, D), device=self.device)
+        _expect("dres", dres, (T, D), device=self.device, optional=True)
+        if out is not None:
+            _expect_all(out, {"dx": ((T, D), BF16), "dwqkv": ((d.t, D, 3 * D // d.t), BF16),
+                              "dwout": ((d.t, D // d.t, D), BF16),
+                              "dbqkv": ((d.t, 1, 3 * D // d.t), BF16), "dbout": ((D,), BF16)},
+                        self.device, "out", optional=("dbqkv", "dbout"))
         if self.ws is None:
             self.ws = _ws(OP_ATTN_BWD, d, self.device)
         g = out if out is not None else {
@@ -195,7 +261,11 @@ class ShardedLayer:
         self.recompute = recompute
         self.dims = dims
         t, H = dims.t, dims.heads
-        self.device = p["w1"].device
+        self.device = p["w1"].device if isinstance(p.get("w1"), torch.Tensor) else None
+        _expect_all(p, self._param_spec(), self.device, "p",
+                    optional=("bqkv", "bout", "b1", "b2"))
+        if not p["w1"].is_cuda:
+            raise ValueError("parameters must live on a CUDA device")
         self.p = {
             "ln1_g": p["ln1_g"].contiguous(), "ln1_b": p["ln1_b"].contiguous(),
             "wqkv": pack_qkv(p["wqkv"], H, t),
@@ -211,11 +281,24 @@ class ShardedLayer:
         self.ws = None
         self.ws_fwd = None
 
-    def alloc_acts(self):
+    def _param_spec(self):
+        D, F = self.dims.hidden, self.dims.ffn
+        return {"ln1_g": ((D,), BF16), "ln1_b": ((D,), BF16), "wqkv": ((D, 3 * D), BF16),
+                "bqkv": ((3 * D,), BF16), "wout": ((D, D), BF16), "bout": ((D,), BF16),
+                "ln2_g": ((D,), BF16), "ln2_b": ((D,), BF16), "w1": ((D, F), BF16),
+                "b1": ((F,), BF16), "w2": ((F, D), BF16), "b2": ((D,), BF16)}
+
+    def _acts_spec(self):
+        return {k: (tuple(v.shape), v.dtype) for k, v in self.alloc_acts(meta=True).items()}
+
+    def _grads_spec(self):
+        return {k: (tuple(v.shape), v.dtype) for k, v in self.alloc_grads(meta=True).items()}
+
+    def alloc_acts(self, meta=False):
         d = self.dims
         T, D, F, t = d.batch * d.seq, d.hidden, d.ffn, d.t
         f32 = torch.float32
-        dev = self.device
+        dev = "meta" if meta else self.device
         f16 = torch.float16
         if self.post:
             return {"z1": _empty((T, D), device=dev), "mean1": _empty((T,), f32, dev),
@@ -234,10 +317,10 @@ class ShardedLayer:
                 "mean2": _empty((T,), f32, dev), "rstd2": _empty((T,), f32, dev),
                 "a": _empty((t, T, F // t), device=dev), "hact": _empty((t, T, F // t), device=dev)}
 
-    def alloc_grads(self, bias_grads=True):
+    def alloc_grads(self, bias_grads=True, meta=False):
         d = self.dims
         D, F, t = d.hidden, d.ffn, d.t
-        dev = self.device
+        dev = "meta" if meta else self.device
         opt = (lambda s: _empty(s, device=dev)) if bias_grads else (lambda s: None)
         return {"dln1_g": opt((D,)), "dln1_b": opt((D,)),
                 "dwqkv": _empty((t, D, 3 * D // t), device=dev), "dbqkv": opt((t, 1, 3 * D // t)),
@@ -250,11 +333,16 @@ class ShardedLayer:
         """Bytes of activations held from the forward to the backward (x excluded)."""
         if self.recompute:
             return 0
-        return sum(v.numel() * v.element_size() for v in self.alloc_acts().values())
+        return sum(v.numel() * v.element_size() for v in self.alloc_acts(meta=True).values())
 
     @_nvtx("tp.layer.forward")
     def forward(self, x, acts=None, y=None):
         d = self.dims
+        T, D = d.batch * d.seq, d.hidden
+        _expect("x", x, (T, D), device=self.device)
+        _expect("y", y, (T, D), device=self.device, optional=True)
+        if acts is not None:
+            _expect_all(acts, self._acts_spec(), self.device, "acts")
         y = y if y is not None else _empty((d.batch * d.seq, d.hidden), device=self.device)
         if self.recompute:
             if self.ws_fwd is None:
@@ -273,6 +361,13 @@ class ShardedLayer:
     def backward(self, dy, dx=None, grads=None, bias_grads=True):
         d = self.dims
         x, acts = self.saved
+        T, D = d.batch * d.seq, d.hidden
+        _expect("dy", dy, (T, D), device=self.device)
+        _expect("dx", dx, (T, D), device=self.device, optional=True)
+        if grads is not None:
+            _expect_all(grads, self._grads_spec(), self.device, "grads",
+                        optional=("dln1_g", "dln1_b", "dbqkv", "dbout", "dln2_g", "dln2_b",
+                                  "db1", "db2"))
         dx = dx if dx is not None else torch.empty_like(x)
         grads = grads if grads is not None else self.alloc_grads(bias_grads)
         if self.recompute:
