@@ -21,8 +21,11 @@
  *  - Element type: bf16, passed as raw 16-bit patterns (tp_bf16); fp16 or fp32
  *    where stated.  Accumulation is fp32; outputs are rounded to nearest even once.
  *  - Pointers: DEVICE pointers owned by the caller, 16-byte aligned, dense
- *    row-major, unless stated otherwise.  The library allocates nothing and
- *    keeps no state apart from cached per-device attributes.
+ *    row-major, unless stated otherwise.  The library allocates nothing on the
+ *    compute path.  Its only state: cached per-device attributes and kernel
+ *    settings, one device error word per device (tp_check_error), the
+ *    optional launch trace (tp_trace_begin) and the static scratch array of
+ *    tp_layernorm_bwd_noalloc.
  *  - Shapes: T = batch*seq tokens (batch outer), D = hidden, F = ffn,
  *    H = heads, dh = head_dim (D = H*dh), t = tensor-parallel degree,
  *    Ft = F/t, Dt = D/t.  Activations x, y: [T][D].
@@ -71,15 +74,17 @@ typedef enum {
 /* Sizes of one problem.  Fields an operation does not use are ignored
  * (e.g. heads/head_dim for the MLP, ffn for attention). */
 typedef struct {
-  int batch;     /* B >= 1 */
-  int seq;       /* S >= 1; T = B*S */
+  int batch;     /* B >= 0 */
+  int seq;       /* S >= 0; T = B*S < 2^31.  T = 0 is an empty problem: nothing is
+                    computed, parameter gradients are zeroed, and activation
+                    pointers may be NULL */
   int hidden;    /* D, multiple of 8*t */
   int ffn;       /* F, multiple of 8*t */
   int heads;     /* H, multiple of t */
   int head_dim;  /* dh in {64, 128}, D = H*dh */
   int t;         /* tensor-parallel degree in {1, 2, 4, 8} */
   int causal;    /* attention mask: 1 = key s' visible to query s iff s' <= s; 0 = none */
-  float ln_eps;  /* LayerNorm epsilon (pre-LN layer only), > 0 */
+  float ln_eps;  /* LayerNorm epsilon (layer entry points only), > 0 */
 } tp_dims;
 
 typedef enum {
