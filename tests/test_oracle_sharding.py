@@ -118,3 +118,65 @@ def test_30b_ffn_weight_size_from_the_pages():
     assert nbytes == 411_041_792
     assert round(nbytes / 1e6) == g["approx_mb_per_matrix"]
     assert abs(2 * nbytes / 1e6 - g["approx_mb_per_layer"]) < 1.0
+
+
+def _layer_params(D, F_):
+    p = {"ln1_g": 1 + 0.1 * RNG.normal(size=D), "ln1_b": 0.1 * RNG.normal(size=D),
+         "wqkv": 0.4 * RNG.normal(size=(D, 3 * D)), "bqkv": 0.1 * RNG.normal(size=3 * D),
+         "wout": 0.4 * RNG.normal(size=(D, D)), "bout": 0.1 * RNG.normal(size=D),
+         "ln2_g": 1 + 0.1 * RNG.normal(size=D), "ln2_b": 0.1 * RNG.normal(size=D),
+         "w1": 0.3 * RNG.normal(size=(D, F_)), "b1": 0.1 * RNG.normal(size=F_),
+         "w2": 0.3 * RNG.normal(size=(F_, D)), "b2": 0.1 * RNG.normal(size=D)}
+    return p
+
+
+@pytest.mark.parametrize("t", [1, 2, 4, 8])
+@pytest.mark.parametrize("placement", ["pre", "post"])
+def test_layer_built_from_sharded_sublayers(t, placement):
+    """Both layer placements composed from the sharded sublayers (each with its
+    own shard sums) equal the unsharded layers, forward and backward."""
+    from oracle import layer as olayer
+    B, S, H, dh, F_ = 2, 5, 8, 3, 64
+    D = H * dh
+    p = _layer_params(D, F_)
+    x = RNG.normal(size=(B * S, D))
+    dy = RNG.normal(size=(B * S, D))
+
+    def attn_s(u):
+        return sharded.attn_fwd_sharded(u, p["wqkv"], p["bqkv"], p["wout"], p["bout"], B, H, t)
+
+    def mlp_s(u):
+        return sharded.mlp_fwd_sharded(u, p["w1"], p["b1"], p["w2"], p["b2"], t)
+
+    ln = core.layernorm_fwd
+    if placement == "pre":
+        u1, m1, r1 = ln(x, p["ln1_g"], p["ln1_b"], 1e-5)
+        h = x + attn_s(u1)
+        u2, m2, r2 = ln(h, p["ln2_g"], p["ln2_b"], 1e-5)
+        y = h + mlp_s(u2)
+        yr, _ = olayer.layer_fwd(x, p, B, H)
+        gm = sharded.mlp_bwd_sharded(u2, p["w1"], p["b1"], p["w2"], dy, t)
+        du2, _, _ = core.layernorm_bwd(gm["dx"], h, p["ln2_g"], m2, r2)
+        dh = dy + du2
+        ga = sharded.attn_bwd_sharded(u1, p["wqkv"], p["bqkv"], p["wout"], dh, B, H, t)
+        du1, _, _ = core.layernorm_bwd(ga["dx"], x, p["ln1_g"], m1, r1)
+        dx = dh + du1
+        gr = olayer.layer_bwd(x, p, dy, B, H)
+    else:
+        z1 = x + attn_s(x)
+        h, m1, r1 = ln(z1, p["ln1_g"], p["ln1_b"], 1e-5)
+        z2 = h + mlp_s(h)
+        y, m2, r2 = ln(z2, p["ln2_g"], p["ln2_b"], 1e-5)
+        yr, _ = olayer.postln_layer_fwd(x, p, B, H)
+        dz2, _, _ = core.layernorm_bwd(dy, z2, p["ln2_g"], m2, r2)
+        gm = sharded.mlp_bwd_sharded(h, p["w1"], p["b1"], p["w2"], dz2, t)
+        dh = dz2 + gm["dx"]
+        dz1, _, _ = core.layernorm_bwd(dh, z1, p["ln1_g"], m1, r1)
+        ga = sharded.attn_bwd_sharded(x, p["wqkv"], p["bqkv"], p["wout"], dz1, B, H, t)
+        dx = dz1 + ga["dx"]
+        gr = olayer.postln_layer_bwd(x, p, dy, B, H)
+    assert _rel(y, yr) < 1e-12
+    assert _rel(dx, gr["dx"]) < 1e-12
+    for k, v in (("dw1", gm["dw1"]), ("dw2", gm["dw2"]), ("dwqkv", ga["dwqkv"]),
+                 ("dwout", ga["dwout"]), ("db1", gm["db1"]), ("dbqkv", ga["dbqkv"])):
+        assert _rel(v, gr[k]) < 1e-12, k
