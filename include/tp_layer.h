@@ -58,6 +58,8 @@ extern "C" {
 #endif
 
 typedef uint16_t tp_bf16;  /* raw bfloat16 bits */
+typedef uint16_t tp_f16;   /* raw IEEE binary16 (fp16) bits: the buffers inside the attention
+                              sublayer that hold fp16, never bf16 (qkv, LN1's output u1) */
 typedef void* tp_stream;   /* cudaStream_t */
 
 typedef enum {
@@ -68,8 +70,19 @@ typedef enum {
   TP_ERR_MISALIGNED = 3,   /* pointer not 16-byte aligned or a row not a multiple of 8 elements */
   TP_ERR_WORKSPACE = 4,    /* workspace pointer null or smaller than tp_workspace_size */
   TP_ERR_CUDA = 5,         /* a CUDA runtime call or kernel launch failed */
-  TP_ERR_TIMEOUT = 6       /* a bounded device wait expired (from tp_check_error) */
+  TP_ERR_TIMEOUT = 6,      /* a bounded device wait expired (from tp_check_error) */
+  TP_ERR_RANGE = 7         /* a value stored as fp16 exceeded +-65504 (from tp_check_error) */
 } tp_status;
+
+/* Codes of the device error word (read by tp_check_error):
+ *   0x0F1          the bounded-wait self-test (tp_selftest_wait_timeout)     -> TP_ERR_TIMEOUT
+ *   0x101 - 0x1FF  a GEMM kernel's wait expired                              -> TP_ERR_TIMEOUT
+ *   0x201 - 0x2FF  an attention kernel's wait expired                        -> TP_ERR_TIMEOUT
+ *   0x301          a value written as fp16 (qkv, u1, dO, dqkv, the fp16
+ *                  copies of x or Wqkv) was beyond the fp16 range; it is
+ *                  stored as +-inf and everything computed from it is
+ *                  meaningless                                               -> TP_ERR_RANGE
+ * The word keeps the first code recorded since it was last cleared. */
 
 /* Sizes of one problem.  Fields an operation does not use are ignored
  * (e.g. heads/head_dim for the MLP, ffn for attention). */
@@ -113,9 +126,10 @@ const char* tp_status_string(tp_status s);
 size_t tp_workspace_size(int op, const tp_dims* dims);
 
 /* Synchronises the current device, then reads and clears the library's
- * device error word.  TP_ERR_TIMEOUT if a bounded wait expired since the
- * last call (the code is stored in *code if code != NULL), TP_ERR_CUDA if
- * the synchronisation failed, TP_OK otherwise. */
+ * device error word.  The code (0 if none) is stored in *code if code != NULL.
+ * TP_ERR_RANGE for code 0x301 (an fp16 overflow), TP_ERR_TIMEOUT for any
+ * other nonzero code (a bounded wait expired), TP_ERR_CUDA if the
+ * synchronisation or the read failed, TP_OK otherwise. */
 tp_status tp_check_error(unsigned int* code);
 
 /* ------------------------------------------------------------------ layout
@@ -174,7 +188,7 @@ tp_status tp_mlp_bwd(const tp_dims* dims, const tp_bf16* x, const tp_bf16* w1, c
  * "The attention heads split": shard i owns heads i*H/t .. (i+1)*H/t-1.
  *
  * tp_attn_fwd:
- *   qkv_save[i] = x Wqkv_i + bqkv_i        [t][T][3*Dt], FP16; within shard i,
+ *   qkv_save[i] = x Wqkv_i + bqkv_i        [t][T][3*Dt], fp16 (tp_f16); within shard i,
  *                 columns [0,Dt) are q, [Dt,2Dt) k, [2Dt,3Dt) v, local head j at j*dh
  *   per head:  O = softmax(q k^T / sqrt(dh) + mask) v, softmax in fp32;
  *              lse_save = log-sum-exp of the scaled masked scores, fp32 [B][H][S]
@@ -185,12 +199,12 @@ tp_status tp_mlp_bwd(const tp_dims* dims, const tp_bf16* x, const tp_bf16* w1, c
  * storage the softmax over long causal rows amplifies the rounding of q and k
  * to a relative error near 6e-3 in O at S = 2048, with fp16 near 2e-3.  A value
  * beyond the fp16 range (|v| > 65504) sets device error code 0x301
- * (tp_check_error reports TP_ERR_TIMEOUT with that code).
+ * (tp_check_error reports TP_ERR_RANGE with that code).
  * bqkv, bout, resid may be NULL.  Uses batch, seq, hidden, heads, head_dim, t,
  * causal.  Workspace: tp_workspace_size(TP_OP_ATTN_FWD, dims) bytes. */
 tp_status tp_attn_fwd(const tp_dims* dims, const tp_bf16* x, const tp_bf16* wqkv,
                       const tp_bf16* bqkv, const tp_bf16* wout, const tp_bf16* bout,
-                      const tp_bf16* resid, tp_bf16* y, tp_bf16* qkv_save, tp_bf16* o_save,
+                      const tp_bf16* resid, tp_bf16* y, tp_f16* qkv_save, tp_bf16* o_save,
                       float* lse_save, void* ws, size_t ws_bytes, tp_stream stream);
 
 /* tp_attn_bwd: vector-Jacobian product of tp_attn_fwd for dy [T][D]:
@@ -201,7 +215,7 @@ tp_status tp_attn_fwd(const tp_dims* dims, const tp_bf16* x, const tp_bf16* wqkv
  *   dbqkv = column sums of dqkv [t][3*Dt], dbout = column sums of dy [D]
  * dres, dbqkv, dbout may be NULL.  Workspace: tp_workspace_size(TP_OP_ATTN_BWD). */
 tp_status tp_attn_bwd(const tp_dims* dims, const tp_bf16* x, const tp_bf16* wqkv,
-                      const tp_bf16* wout, const tp_bf16* qkv_save, const tp_bf16* o_save,
+                      const tp_bf16* wout, const tp_f16* qkv_save, const tp_bf16* o_save,
                       const float* lse_save, const tp_bf16* dy, const tp_bf16* dres, tp_bf16* dx,
                       tp_bf16* dwqkv, tp_bf16* dbqkv, tp_bf16* dwout, tp_bf16* dbout, void* ws,
                       size_t ws_bytes, tp_stream stream);
@@ -222,9 +236,9 @@ typedef struct {
 
 /* Activations saved by tp_layer_fwd for tp_layer_bwd (all caller-owned). */
 typedef struct {
-  tp_bf16* u1;            /* LN1(x) [T][D], FP16 (it feeds only the fp16 attention products) */
+  tp_f16* u1;             /* LN1(x) [T][D], fp16 (it feeds only the fp16 attention products) */
   float *mean1, *rstd1;   /* [T] */
-  tp_bf16* qkv;           /* [t][T][3Dt], FP16 */
+  tp_f16* qkv;            /* [t][T][3Dt], fp16 */
   tp_bf16* o;             /* [t][T][Dt] */
   float* lse;             /* [B][H][S] */
   tp_bf16* h;             /* x + attention output [T][D] */
@@ -292,7 +306,7 @@ tp_status tp_layer_bwd_recompute(const tp_dims* dims, const tp_bf16* x,
 typedef struct {
   tp_bf16* z1;            /* x + attention output [T][D] (LN1 input) */
   float *mean1, *rstd1;   /* [T] */
-  tp_bf16* qkv;           /* [t][T][3Dt], FP16 */
+  tp_f16* qkv;            /* [t][T][3Dt], fp16 */
   tp_bf16* o;             /* [t][T][Dt] */
   float* lse;             /* [B][H][S] */
   tp_bf16* h;             /* LN1(z1) [T][D] */
@@ -343,9 +357,11 @@ tp_status tp_layernorm_bwd(const tp_bf16* dy, const tp_bf16* x, const tp_bf16* g
  * a device share that array: calls whose kernels may overlap on the GPU race
  * and must be serialised by the caller.  The first call on each device looks
  * up the array's device address; make it outside stream capture.  D up to
- * 8192 (wider rows: TP_ERR_UNSUPPORTED); row count unlimited.  dgamma/dbeta
- * sums may group rows differently from tp_layernorm_bwd (fp32, deterministic);
- * dx is identical. */
+ * 8192 (wider rows: TP_ERR_UNSUPPORTED); row count unlimited.  dx is
+ * identical to tp_layernorm_bwd's; dgamma/dbeta are too while 2 * D * (row
+ * blocks, 2 per SM) floats fit the array (D up to 1771 on a 148-SM GPU);
+ * wider rows use fewer blocks, which groups the fp32 sums differently
+ * (still deterministic). */
 tp_status tp_layernorm_bwd_noalloc(const tp_bf16* dy, const tp_bf16* x, const tp_bf16* gamma,
                                    const float* mean, const float* rstd, const tp_bf16* dres,
                                    int rows, int D, tp_bf16* dx, tp_bf16* dgamma, tp_bf16* dbeta,

@@ -20,7 +20,7 @@ __all__ = [
     "OP_MLP_FWD", "OP_MLP_BWD", "OP_ATTN_FWD", "OP_ATTN_BWD", "OP_LAYER_FWD", "OP_LAYER_BWD",
     "OP_POSTLN_FWD", "OP_POSTLN_BWD", "postln_layer_fwd", "postln_layer_bwd",
     "OP_LAYER_FWD_NOSAVE", "OP_LAYER_BWD_RECOMPUTE", "layer_fwd_nosave", "layer_bwd_recompute",
-    "workspace_size", "check_error", "version", "EXPORTED_SYMBOLS",
+    "workspace_size", "check_error", "check_status", "version", "EXPORTED_SYMBOLS",
     "shard_cols", "unshard_cols", "shard_rows", "unshard_rows", "shard_qkv_heads",
     "unshard_qkv_heads", "mlp_fwd", "mlp_bwd", "attn_fwd", "attn_bwd", "layer_fwd", "layer_bwd",
     "layernorm_fwd", "layernorm_bwd", "layernorm_bwd_workspace_size", "layernorm_bwd_noalloc",
@@ -36,7 +36,7 @@ lib_path = os.path.join(_HERE, "libtplayer.so")
 
 STATUS_NAMES = {0: "TP_OK", 1: "TP_ERR_INVALID_ARG", 2: "TP_ERR_UNSUPPORTED",
                 3: "TP_ERR_MISALIGNED", 4: "TP_ERR_WORKSPACE", 5: "TP_ERR_CUDA",
-                6: "TP_ERR_TIMEOUT"}
+                6: "TP_ERR_TIMEOUT", 7: "TP_ERR_RANGE"}
 
 
 class TpError(RuntimeError):
@@ -178,13 +178,21 @@ def workspace_size(op: int, dims: Dims) -> int:
     return lib().tp_workspace_size(op, ctypes.byref(dims))
 
 
-def check_error() -> int:
-    """Synchronise and return the device error word (0 if no bounded wait expired)."""
+def check_status():
+    """Synchronise, read and clear the device error word: (status, code).
+
+    status is 0 (TP_OK), 6 (TP_ERR_TIMEOUT: a bounded wait expired) or 7
+    (TP_ERR_RANGE: a value stored as fp16 overflowed); code is the word."""
     code = ctypes.c_uint(0)
     st = lib().tp_check_error(ctypes.byref(code))
-    if st not in (0, 6):
+    if st not in (0, 6, 7):
         raise TpError(st, "tp_check_error")
-    return code.value
+    return st, code.value
+
+
+def check_error() -> int:
+    """Synchronise and return the device error word (0 if nothing was recorded)."""
+    return check_status()[1]
 
 
 def _ws(ws):

@@ -482,6 +482,7 @@ const char* tp_status_string(tp_status s) {
     case TP_ERR_WORKSPACE: return "TP_ERR_WORKSPACE";
     case TP_ERR_CUDA: return "TP_ERR_CUDA";
     case TP_ERR_TIMEOUT: return "TP_ERR_TIMEOUT";
+    case TP_ERR_RANGE: return "TP_ERR_RANGE";
   }
   return "TP_ERR_UNKNOWN";
 }
@@ -515,7 +516,8 @@ tp_status tp_check_error(unsigned int* code) {
     cudaMemcpy(p, &zero, sizeof(zero), cudaMemcpyHostToDevice);
   }
   if (code) *code = v;
-  return v ? TP_ERR_TIMEOUT : TP_OK;
+  if (v == 0) return TP_OK;
+  return (v & 0xF00u) == 0x300u ? TP_ERR_RANGE : TP_ERR_TIMEOUT;
 }
 
 // ------------------------------------------------------------------ layout
@@ -604,7 +606,7 @@ tp_status tp_mlp_bwd(const tp_dims* dims, const tp_bf16* x, const tp_bf16* w1, c
 // ------------------------------------------------------------------ attention
 tp_status tp_attn_fwd(const tp_dims* dims, const tp_bf16* x, const tp_bf16* wqkv,
                       const tp_bf16* bqkv, const tp_bf16* wout, const tp_bf16* bout,
-                      const tp_bf16* resid, tp_bf16* y, tp_bf16* qkv_save, tp_bf16* o_save,
+                      const tp_bf16* resid, tp_bf16* y, tp_f16* qkv_save, tp_bf16* o_save,
                       float* lse_save, void* ws, size_t ws_bytes, tp_stream s) {
   tp_status st = check_attn(dims);
   if (st != TP_OK) return st;
@@ -627,7 +629,7 @@ tp_status tp_attn_fwd(const tp_dims* dims, const tp_bf16* x, const tp_bf16* wqkv
 }
 
 tp_status tp_attn_bwd(const tp_dims* dims, const tp_bf16* x, const tp_bf16* wqkv,
-                      const tp_bf16* wout, const tp_bf16* qkv_save, const tp_bf16* o_save,
+                      const tp_bf16* wout, const tp_f16* qkv_save, const tp_bf16* o_save,
                       const float* lse_save, const tp_bf16* dy, const tp_bf16* dres, tp_bf16* dx,
                       tp_bf16* dwqkv, tp_bf16* dbqkv, tp_bf16* dwout, tp_bf16* dbout, void* ws,
                       size_t ws_bytes, tp_stream s) {

@@ -56,6 +56,9 @@ tp_status launch_colsum_stacked(const uint16_t* x, long long S, long long rows, 
 tp_status launch_layernorm_fwd(const uint16_t* x, const uint16_t* g, const uint16_t* b,
                                long long rows, int D, float eps, uint16_t* y, float* mean,
                                float* rstd, cudaStream_t stream, bool out_f16 = false);
+// Row blocks of the LayerNorm backward (2 per SM, at most one per row); the
+// dgamma/dbeta partials hold 2 * D floats per block.
+int layernorm_bwd_blocks(long long rows);
 size_t layernorm_bwd_partial_floats(long long rows, int D);
 tp_status launch_layernorm_bwd(const uint16_t* dy, const uint16_t* x, const uint16_t* g,
                                const float* mean, const float* rstd, const uint16_t* dres,

@@ -74,10 +74,11 @@ extern "C" tp_status tp_layernorm_bwd_noalloc(const tp_bf16* dy, const tp_bf16* 
   float* scratch = nullptr;
   tp_status st = scratch_for_current_device(&scratch);
   if (st != TP_OK) return st;
-  // Row blocks: as many as the regular entry point uses (4 per SM), capped by
-  // what the array holds (2 * D partial floats per block; >= 64 blocks at D = 8192).
-  long long nb = 4LL * sm_count();
-  if (nb > rows) nb = rows;
+  // Row blocks: the same count as the workspace entry point (2 per SM, at
+  // most one per row), so both group rows alike and give identical dgamma /
+  // dbeta; capped by what the array holds (2 * D partial floats per block,
+  // 64 blocks at D = 8192, where the two may group rows differently).
+  long long nb = layernorm_bwd_blocks(rows < 1 ? 1 : rows);
   const long long cap = (long long)(kStaticScratchFloats / (2 * (size_t)D));
   if (nb > cap) nb = cap;
   if (nb < 1) nb = 1;

@@ -387,13 +387,13 @@ int colsum_chunks(long long rows, long long cols, long long S) {
   return (int)(chunks < 1 ? 1 : chunks);
 }
 
-int ln_bwd_blocks(long long rows) {
+}  // namespace
+
+int layernorm_bwd_blocks(long long rows) {
   long long b = 2LL * sm_count();
   if (b > rows) b = rows;
   return (int)(b < 1 ? 1 : b);
 }
-
-}  // namespace
 
 size_t colsum_partial_floats(long long S, long long rows, long long cols) {
   if (rows < 1) rows = 1;
@@ -460,7 +460,7 @@ tp_status launch_layernorm_fwd(const uint16_t* x, const uint16_t* g, const uint1
 }
 
 size_t layernorm_bwd_partial_floats(long long rows, int D) {
-  return (size_t)ln_bwd_blocks(rows < 1 ? 1 : rows) * 2 * (size_t)D;
+  return (size_t)layernorm_bwd_blocks(rows < 1 ? 1 : rows) * 2 * (size_t)D;
 }
 
 namespace {
@@ -504,7 +504,7 @@ tp_status launch_layernorm_bwd(const uint16_t* dy, const uint16_t* x, const uint
                                long long rows, int D, uint16_t* dx, uint16_t* dg, uint16_t* db,
                                float* partial, cudaStream_t stream, float* dx32) {
   return ln_bwd_launch<false>(dy, x, g, mean, rstd, dres, rows, D, dx, dx32, dg, db,
-                              ln_bwd_blocks(rows < 1 ? 1 : rows), partial, stream);
+                              layernorm_bwd_blocks(rows < 1 ? 1 : rows), partial, stream);
 }
 
 tp_status launch_layernorm_bwd_f32(const float* dy, const uint16_t* x, const uint16_t* g,
@@ -512,7 +512,7 @@ tp_status launch_layernorm_bwd_f32(const float* dy, const uint16_t* x, const uin
                                    uint16_t* dx, float* dx32, uint16_t* dg, uint16_t* db,
                                    float* partial, cudaStream_t stream) {
   return ln_bwd_launch<true>(dy, x, g, mean, rstd, nullptr, rows, D, dx, dx32, dg, db,
-                             ln_bwd_blocks(rows < 1 ? 1 : rows), partial, stream);
+                             layernorm_bwd_blocks(rows < 1 ? 1 : rows), partial, stream);
 }
 
 // LayerNorm backward with a caller-chosen number of row blocks `nb` (>= 1):

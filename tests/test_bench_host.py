@@ -44,3 +44,42 @@ def test_hbm_bytes_of_the_layer_step():
     assert b["cast"] == 24 * D * D                              # Wqkv read + written, twice
     assert abs(b["ln_bwd"] / 2**20 - 512.125) < 1e-9            # 512 MiB of rows + 128 KiB of stats
     assert bench.hbm_bytes_per_step(workload("mlp_fwdbwd_T8192_D3072_F12288_t8")) == {}
+
+
+PEAKS = {"hbm_gbs": 6425.6, "bf16_tflops": 1713.1, "bf16_tflops_sustained": 1430.5}
+
+
+def test_peak_follows_the_sampled_clock():
+    """Burst figure when the SM clock held at its maximum, sustained when it sagged."""
+    at_max = {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0}
+    sagged = {"sm_mhz": 1455.0, "sm_max_mhz": 1965.0}
+    assert bench.choose_peak(PEAKS, at_max) == (1713.1, "bf16_tflops")
+    assert bench.choose_peak(PEAKS, {"sm_mhz": 1890.0, "sm_max_mhz": 1965.0})[0] == 1713.1
+    assert bench.choose_peak(PEAKS, sagged) == (1430.5, "bf16_tflops_sustained")
+    # No clock record: the larger denominator.
+    assert bench.choose_peak(PEAKS, {"sm_mhz": None, "sm_max_mhz": None})[0] == 1713.1
+
+
+def test_roofline_fraction_of_a_recorded_run():
+    """The first round's c5 line: 9.896 TFLOP of GEMM work per step in 7.587 ms
+    at 1965 MHz is 1304 TFLOP/s, 0.76 of the burst figure (not 0.91 of the
+    sustained one)."""
+    gemm_flop = 12 * 8192 * 4096 * 16384 + 24 * 8192 * 4096 * 4096
+    achieved = gemm_flop / 7.586649605631829e-3 / 1e12
+    peak, name = bench.choose_peak(PEAKS, {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0})
+    assert abs(achieved - 1304.3) < 0.1
+    assert abs(achieved / peak - 0.761) < 1e-3 and name == "bf16_tflops"
+    assert bench.clock_normalised(achieved, {"sm_mhz": 1455.0, "sm_max_mhz": 1965.0}) == \
+        achieved * 1965.0 / 1455.0
+
+
+def test_step_time_is_the_median_of_per_step_durations():
+    class Ev:
+        def __init__(self, t):
+            self.t = t
+
+        def elapsed_time(self, other):
+            return other.t - self.t
+
+    evs = [Ev(t) for t in (0.0, 9.0, 18.5, 27.0, 45.0)]   # steps 9, 9.5, 8.5, 18
+    assert bench.median_step_ms(evs) == 9.25
