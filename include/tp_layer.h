@@ -341,6 +341,12 @@ tp_status tp_postln_layer_bwd(const tp_dims* dims, const tp_bf16* x, const tp_la
  *                     Workspace: tp_layernorm_bwd_workspace_size(rows, D). */
 tp_status tp_layernorm_fwd(const tp_bf16* x, const tp_bf16* gamma, const tp_bf16* beta, int rows,
                            int D, float eps, tp_bf16* y, float* mean, float* rstd, tp_stream stream);
+/* tp_layernorm_fwd_f16: tp_layernorm_fwd with an fp16 output y, for a LayerNorm
+ * that feeds the attention sublayer's fp16 products (tp_attn_fwd_rank's x16);
+ * values beyond the fp16 range set device error 0x301. */
+tp_status tp_layernorm_fwd_f16(const tp_bf16* x, const tp_bf16* gamma, const tp_bf16* beta,
+                               int rows, int D, float eps, tp_f16* y, float* mean, float* rstd,
+                               tp_stream stream);
 size_t tp_layernorm_bwd_workspace_size(int rows, int D);
 tp_status tp_layernorm_bwd(const tp_bf16* dy, const tp_bf16* x, const tp_bf16* gamma,
                            const float* mean, const float* rstd, const tp_bf16* dres, int rows,
@@ -367,6 +373,91 @@ tp_status tp_layernorm_bwd_noalloc(const tp_bf16* dy, const tp_bf16* x, const tp
                                    int rows, int D, tp_bf16* dx, tp_bf16* dgamma, tp_bf16* dbeta,
                                    tp_stream stream);
 
+/* ------------------------------------------------------------------ one shard per GPU
+ * The pages' own deployment ("One Idea, Two Insertions" on the explainer;
+ * "How transformer layers actually decompose" and "Why TP must stay within a
+ * node" on the blog): GPU i of a t-GPU group holds shard i of every weight and
+ * the shards meet in one all-reduce per sublayer per direction.  Each call
+ * below runs one shard between two exchange points on the calling GPU and
+ * writes that shard's PARTIAL of the exchanged tensor, fp32 [T][D], without
+ * bias.  The caller sums the t partials (an all-reduce among the ranks, or
+ * reads of the peers' buffers) and finishes with tp_rowpar_finish, which adds
+ * the row-parallel product's bias once and the residual and rounds once.
+ *
+ * Every pointer is shard-local (what GPU i holds): W1_i [D][Ft], b1_i [Ft],
+ * W2_i [Ft][D], Wqkv_i [D][3Dt] = [Wq_i | Wk_i | Wv_i], bqkv_i [3Dt],
+ * Wout_i [Dt][D]; activations of the shard: A_i, H_i [T][Ft], qkv_i [T][3Dt]
+ * (fp16), O_i [T][Dt], lse_i [B][H/t][S].  x, dy, the full-width biases b2,
+ * bout and the residuals are replicated on every rank.  dims->t is the
+ * tensor-parallel degree (the number of ranks); dims describes the WHOLE
+ * layer (hidden, ffn, heads), from which the shard widths Ft = F/t,
+ * Dt = D/t and the local head count H/t follow.  Workspaces:
+ * tp_rank_workspace_size.  Errors and streams as for the other entry points. */
+typedef enum {
+  TP_RANK_MLP_FWD = 0,
+  TP_RANK_MLP_BWD = 1,
+  TP_RANK_ATTN_FWD = 2,
+  TP_RANK_ATTN_BWD = 3
+} tp_rank_op;
+
+/* Bytes of device workspace rank-local operation `op` needs (0 if none or invalid dims). */
+size_t tp_rank_workspace_size(int op, const tp_dims* dims);
+
+/* tp_mlp_fwd_rank: a_i = x W1_i + b1_i, h_i = GeLU(a_i) [T][Ft] (saved for the
+ * backward); partial = h_i W2_i, fp32 [T][D].  b1_i may be NULL.  No workspace.
+ * Finish: y = tp_rowpar_finish(sum of the t partials, b2, resid). */
+tp_status tp_mlp_fwd_rank(const tp_dims* dims, const tp_bf16* x, const tp_bf16* w1_i,
+                          const tp_bf16* b1_i, const tp_bf16* w2_i, tp_bf16* a_i, tp_bf16* h_i,
+                          float* partial, tp_stream stream);
+
+/* tp_mlp_bwd_rank, for the upstream gradient dy [T][D] (replicated):
+ *   dA_i = (dy W2_i^T) * GeLU'(a_i);  dw2_i = h_i^T dy [Ft][D];  dw1_i = x^T dA_i [D][Ft];
+ *   db1_i = column sums of dA_i [Ft];  db2 = column sums of dy [D] (the same on
+ *   every rank; NULL to skip);  partial = dA_i W1_i^T, fp32 [T][D].
+ * Finish: dx = tp_rowpar_finish(sum of the t partials, NULL, dres). */
+tp_status tp_mlp_bwd_rank(const tp_dims* dims, const tp_bf16* x, const tp_bf16* w1_i,
+                          const tp_bf16* w2_i, const tp_bf16* a_i, const tp_bf16* h_i,
+                          const tp_bf16* dy, tp_bf16* dw1_i, tp_bf16* dw2_i, tp_bf16* db1_i,
+                          tp_bf16* db2, float* partial, void* ws, size_t ws_bytes,
+                          tp_stream stream);
+
+/* tp_attn_fwd_rank: the sublayer input as bf16 x or, when the caller already
+ * holds it in fp16 (a LayerNorm with fp16 output, tp_layernorm_fwd_f16), as
+ * x16; exactly one of the two is non-NULL.  Inside, the products run on fp16
+ * operands as in tp_attn_fwd.
+ *   qkv_i = x Wqkv_i + bqkv_i [T][3Dt] (fp16; columns [0,Dt) q, [Dt,2Dt) k,
+ *   [2Dt,3Dt) v, local head j at j*dh);  per local head: O = softmax(q k^T /
+ *   sqrt(dh) + mask) v (fp32 softmax), o_i [T][Dt], lse_i [B][H/t][S];
+ *   partial = o_i Wout_i, fp32 [T][D].  bqkv_i may be NULL.
+ * Finish: y = tp_rowpar_finish(sum of the t partials, bout, resid). */
+tp_status tp_attn_fwd_rank(const tp_dims* dims, const tp_bf16* x, const tp_f16* x16,
+                           const tp_bf16* wqkv_i, const tp_bf16* bqkv_i, const tp_bf16* wout_i,
+                           tp_f16* qkv_i, tp_bf16* o_i, float* lse_i, float* partial, void* ws,
+                           size_t ws_bytes, tp_stream stream);
+
+/* tp_attn_bwd_rank, for dy [T][D] (replicated); x or x16 as in the forward:
+ *   dO_i = dy Wout_i^T;  dwout_i = o_i^T dy [Dt][D];  the attention backward of
+ *   the local heads (P recomputed from lse_i) gives dqkv_i;  dwqkv_i = x^T dqkv_i
+ *   [D][3Dt];  dbqkv_i = column sums of dqkv_i [3Dt];  dbout = column sums of
+ *   dy [D] (NULL to skip);  partial = dqkv_i Wqkv_i^T, fp32 [T][D].
+ * Finish: dx = tp_rowpar_finish(sum of the t partials, NULL, dres). */
+tp_status tp_attn_bwd_rank(const tp_dims* dims, const tp_bf16* x, const tp_f16* x16,
+                           const tp_bf16* wqkv_i, const tp_bf16* wout_i, const tp_f16* qkv_i,
+                           const tp_bf16* o_i, const float* lse_i, const tp_bf16* dy,
+                           tp_bf16* dwqkv_i, tp_bf16* dbqkv_i, tp_bf16* dwout_i, tp_bf16* dbout,
+                           float* partial, void* ws, size_t ws_bytes, tp_stream stream);
+
+/* tp_rowpar_finish: out = bf16( parts[0] + parts[1] + ... + parts[nparts-1]
+ * + bias + resid ), summed in fp32 in that order and rounded once; out32, when
+ * not NULL, receives the same values in fp32.  parts is a HOST array of
+ * nparts (1..8) device pointers to fp32 [rows][cols] buffers: one buffer that
+ * an all-reduce has already summed, or the t ranks' partials themselves (for
+ * example peers' buffers reachable through peer access, read with plain
+ * loads).  bias [cols] and resid [rows][cols] may be NULL.  cols % 8 == 0. */
+tp_status tp_rowpar_finish(const float* const* parts, int nparts, const tp_bf16* bias,
+                           const tp_bf16* resid, int rows, int cols, tp_bf16* out, float* out32,
+                           tp_stream stream);
+
 /* ------------------------------------------------------------------ failure-detection self-test
  * Not an operation of the pages: a check of the library's bounded device
  * waits.  tp_selftest_wait_timeout enqueues one small kernel whose thread
@@ -386,7 +477,8 @@ tp_status tp_selftest_wait_timeout(unsigned long long limit_ns, tp_stream stream
  * events[2i+1] just after it, store its class in kinds[i] (0 GEMM, 1 attention
  * forward, 2 attention-backward prep, 3 attention dK/dV, 4 attention dQ,
  * 5 LayerNorm forward, 6 LayerNorm backward, 7 LayerNorm parameter reduce,
- * 8 column sum, 9 layout copy, 10 bf16-to-fp16 conversion) and, if flops != NULL, its algorithmic FLOP
+ * 8 column sum, 9 layout copy, 10 bf16-to-fp16 conversion, 11 row-parallel finish) and, if
+ * flops != NULL, its algorithmic FLOP
  * count in flops[i] (0 for non-contraction kernels).  events are cudaEvent_t
  * handles created by the caller on the current device; arrays are host memory
  * owned by the caller and must stay valid until tp_trace_end.  capacity 0

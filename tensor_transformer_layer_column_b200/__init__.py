@@ -24,7 +24,9 @@ __all__ = [
     "shard_cols", "unshard_cols", "shard_rows", "unshard_rows", "shard_qkv_heads",
     "unshard_qkv_heads", "mlp_fwd", "mlp_bwd", "attn_fwd", "attn_bwd", "layer_fwd", "layer_bwd",
     "layernorm_fwd", "layernorm_bwd", "layernorm_bwd_workspace_size", "layernorm_bwd_noalloc",
-    "LaunchTrace",
+    "LaunchTrace", "RANK_MLP_FWD", "RANK_MLP_BWD", "RANK_ATTN_FWD", "RANK_ATTN_BWD",
+    "rank_workspace_size", "mlp_fwd_rank", "mlp_bwd_rank", "attn_fwd_rank", "attn_bwd_rank",
+    "rowpar_finish", "layernorm_fwd_f16",
     "TRACE_KINDS", "selftest_wait_timeout",
 ]
 
@@ -33,6 +35,8 @@ lib_path = os.path.join(_HERE, "libtplayer.so")
 
 (OP_MLP_FWD, OP_MLP_BWD, OP_ATTN_FWD, OP_ATTN_BWD, OP_LAYER_FWD, OP_LAYER_BWD, OP_POSTLN_FWD,
  OP_POSTLN_BWD, OP_LAYER_FWD_NOSAVE, OP_LAYER_BWD_RECOMPUTE) = range(10)
+
+RANK_MLP_FWD, RANK_MLP_BWD, RANK_ATTN_FWD, RANK_ATTN_BWD = range(4)
 
 STATUS_NAMES = {0: "TP_OK", 1: "TP_ERR_INVALID_ARG", 2: "TP_ERR_UNSUPPORTED",
                 3: "TP_ERR_MISALIGNED", 4: "TP_ERR_WORKSPACE", 5: "TP_ERR_CUDA",
@@ -115,13 +119,23 @@ _SIGS = {
     "tp_layernorm_bwd_noalloc": [_P, _P, _P, _P, _P, _P, ctypes.c_int, ctypes.c_int, _P, _P, _P,
                                  _P],
     "tp_selftest_wait_timeout": [ctypes.c_ulonglong, _P],
+    "tp_rank_workspace_size": [ctypes.c_int, ctypes.POINTER(Dims)],
+    "tp_mlp_fwd_rank": [ctypes.POINTER(Dims)] + [_P] * 7 + [_P],
+    "tp_mlp_bwd_rank": [ctypes.POINTER(Dims)] + [_P] * 11 + [_P, ctypes.c_size_t, _P],
+    "tp_attn_fwd_rank": [ctypes.POINTER(Dims)] + [_P] * 9 + [_P, ctypes.c_size_t, _P],
+    "tp_attn_bwd_rank": [ctypes.POINTER(Dims)] + [_P] * 13 + [_P, ctypes.c_size_t, _P],
+    "tp_rowpar_finish": [ctypes.POINTER(ctypes.c_void_p), ctypes.c_int, _P, _P, ctypes.c_int,
+                         ctypes.c_int, _P, _P, _P],
+    "tp_layernorm_fwd_f16": [_P, _P, _P, ctypes.c_int, ctypes.c_int, ctypes.c_float, _P, _P, _P,
+                             _P],
     "tp_trace_begin": [ctypes.POINTER(ctypes.c_void_p), ctypes.POINTER(ctypes.c_int),
                        ctypes.POINTER(ctypes.c_double), ctypes.c_int],
     "tp_trace_end": [],
 }
 _RESTYPES = {"tp_version": ctypes.c_char_p, "tp_status_string": ctypes.c_char_p,
              "tp_workspace_size": ctypes.c_size_t,
-             "tp_layernorm_bwd_workspace_size": ctypes.c_size_t, "tp_trace_end": ctypes.c_int}
+             "tp_layernorm_bwd_workspace_size": ctypes.c_size_t, "tp_trace_end": ctypes.c_int,
+             "tp_rank_workspace_size": ctypes.c_size_t}
 EXPORTED_SYMBOLS = tuple(_SIGS)
 
 _lib: Optional[ctypes.CDLL] = None
@@ -358,8 +372,60 @@ def layernorm_bwd_noalloc(dy, x, gamma, mean, rstd, dres, rows, D, dx, dgamma, d
                                           _ptr(dbeta), _stream(stream, x)),
            "tp_layernorm_bwd_noalloc")
 
+# ---------------------------------------------------------------- one shard per GPU
+def rank_workspace_size(op: int, dims: Dims) -> int:
+    return lib().tp_rank_workspace_size(op, ctypes.byref(dims))
+
+
+def mlp_fwd_rank(dims, x, w1_i, b1_i, w2_i, a_i, h_i, partial, stream=None):
+    _check(lib().tp_mlp_fwd_rank(ctypes.byref(dims), _ptr(x), _ptr(w1_i), _ptr(b1_i), _ptr(w2_i),
+                                 _ptr(a_i), _ptr(h_i), _ptr(partial), _stream(stream, x)),
+           "tp_mlp_fwd_rank")
+
+
+def mlp_bwd_rank(dims, x, w1_i, w2_i, a_i, h_i, dy, dw1_i, dw2_i, db1_i, db2, partial, ws,
+                 stream=None):
+    wp, wn = _ws(ws)
+    _check(lib().tp_mlp_bwd_rank(ctypes.byref(dims), _ptr(x), _ptr(w1_i), _ptr(w2_i), _ptr(a_i),
+                                 _ptr(h_i), _ptr(dy), _ptr(dw1_i), _ptr(dw2_i), _ptr(db1_i),
+                                 _ptr(db2), _ptr(partial), wp, wn, _stream(stream, dy)),
+           "tp_mlp_bwd_rank")
+
+
+def attn_fwd_rank(dims, x, x16, wqkv_i, bqkv_i, wout_i, qkv_i, o_i, lse_i, partial, ws,
+                  stream=None):
+    wp, wn = _ws(ws)
+    _check(lib().tp_attn_fwd_rank(ctypes.byref(dims), _ptr(x), _ptr(x16), _ptr(wqkv_i),
+                                  _ptr(bqkv_i), _ptr(wout_i), _ptr(qkv_i), _ptr(o_i), _ptr(lse_i),
+                                  _ptr(partial), wp, wn, _stream(stream, wqkv_i)),
+           "tp_attn_fwd_rank")
+
+
+def attn_bwd_rank(dims, x, x16, wqkv_i, wout_i, qkv_i, o_i, lse_i, dy, dwqkv_i, dbqkv_i, dwout_i,
+                  dbout, partial, ws, stream=None):
+    wp, wn = _ws(ws)
+    _check(lib().tp_attn_bwd_rank(ctypes.byref(dims), _ptr(x), _ptr(x16), _ptr(wqkv_i),
+                                  _ptr(wout_i), _ptr(qkv_i), _ptr(o_i), _ptr(lse_i), _ptr(dy),
+                                  _ptr(dwqkv_i), _ptr(dbqkv_i), _ptr(dwout_i), _ptr(dbout),
+                                  _ptr(partial), wp, wn, _stream(stream, dy)),
+           "tp_attn_bwd_rank")
+
+
+def rowpar_finish(parts, bias, resid, rows, cols, out, out32=None, stream=None):
+    """out = bf16(sum of the fp32 buffers in `parts`, in order, + bias + resid)."""
+    arr = (ctypes.c_void_p * len(parts))(*[_ptr(q) for q in parts])
+    _check(lib().tp_rowpar_finish(arr, len(parts), _ptr(bias), _ptr(resid), rows, cols, _ptr(out),
+                                  _ptr(out32), _stream(stream, out)), "tp_rowpar_finish")
+
+
+def layernorm_fwd_f16(x, gamma, beta, rows, D, eps, y, mean, rstd, stream=None):
+    _check(lib().tp_layernorm_fwd_f16(_ptr(x), _ptr(gamma), _ptr(beta), rows, D, eps, _ptr(y),
+                                      _ptr(mean), _ptr(rstd), _stream(stream, x)),
+           "tp_layernorm_fwd_f16")
+
+
 TRACE_KINDS = ("gemm", "attn_fwd", "attn_bwd_prep", "attn_bwd_dkdv", "attn_bwd_dq", "ln_fwd",
-               "ln_bwd", "ln_param", "colsum", "layout", "cast")
+               "ln_bwd", "ln_param", "colsum", "layout", "cast", "finish")
 
 
 class LaunchTrace:

@@ -60,48 +60,6 @@ int sm_count() {
   return g_sms[d];
 }
 
-namespace {
-
-using bf16p = const uint16_t*;
-
-bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
-
-// Every non-null pointer 16-byte aligned.
-template <typename... P>
-bool all_aligned(P... ps) {
-  bool ok = true;
-  ((ok = ok && (ps == nullptr || al16(ps))), ...);
-  return ok;
-}
-
-template <typename... P>
-bool all_set(P... ps) {
-  bool ok = true;
-  ((ok = ok && ps != nullptr), ...);
-  return ok;
-}
-
-bool supported_t(int t) { return t == 1 || t == 2 || t == 4 || t == 8; }
-
-struct Sizes {
-  long long B, S, T, D, F, H, dh, t, Ft, Dt;
-};
-
-Sizes sizes_of(const tp_dims& d) {
-  Sizes s{};
-  s.B = d.batch;
-  s.S = d.seq;
-  s.T = (long long)d.batch * d.seq;
-  s.D = d.hidden;
-  s.F = d.ffn;
-  s.H = d.heads;
-  s.dh = d.head_dim;
-  s.t = d.t;
-  s.Ft = d.t > 0 ? d.ffn / d.t : 0;
-  s.Dt = d.t > 0 ? d.hidden / d.t : 0;
-  return s;
-}
-
 // Shape rules shared by every op: "What determines your tensor parallel
 // degree" requires H % t == 0 (and the FFN width divisible by t); the
 // library provides t in {1, 2, 4, 8} ("doesn't recommend going above 8").
@@ -145,24 +103,33 @@ tp_status check_layer(const tp_dims* d) {
   return TP_OK;
 }
 
+namespace {
+
+using bf16p = const uint16_t*;
+
+struct Sizes {
+  long long B, S, T, D, F, H, dh, t, Ft, Dt;
+};
+
+Sizes sizes_of(const tp_dims& d) {
+  Sizes s{};
+  s.B = d.batch;
+  s.S = d.seq;
+  s.T = (long long)d.batch * d.seq;
+  s.D = d.hidden;
+  s.F = d.ffn;
+  s.H = d.heads;
+  s.dh = d.head_dim;
+  s.t = d.t;
+  s.Ft = d.t > 0 ? d.ffn / d.t : 0;
+  s.Dt = d.t > 0 ? d.hidden / d.t : 0;
+  return s;
+}
+
 OperandDesc op(const void* p, bool mn, int src, long long inner, long long outer,
                long long shards, long long ld, long long shard_stride, bool f16 = false) {
   return OperandDesc{p, mn, f16, src, inner, outer, shards, ld, shard_stride};
 }
-
-// Workspace carving: consecutive 256-byte aligned slices.
-struct Carver {
-  uint8_t* base;
-  size_t off = 0;
-  explicit Carver(void* p) : base(static_cast<uint8_t*>(p)) {}
-  template <typename T>
-  T* take(size_t count) {
-    off = align_up(off, 256);
-    T* p = base ? reinterpret_cast<T*>(base + off) : nullptr;
-    off += count * sizeof(T);
-    return p;
-  }
-};
 
 size_t colsum_scratch_floats_max(long long T, std::initializer_list<std::pair<long long, long long>> sc) {
   size_t m = 0;
@@ -457,13 +424,6 @@ size_t postln_bwd_ws(const Sizes& z) {
   return align_up(c.off, 256);
 }
 
-tp_status check_ws(void* ws, size_t have, size_t need) {
-  if (need == 0) return TP_OK;
-  if (ws == nullptr || have < need) return TP_ERR_WORKSPACE;
-  if (!al16(ws)) return TP_ERR_MISALIGNED;
-  return TP_OK;
-}
-
 }  // namespace
 }  // namespace tp
 
@@ -666,6 +626,16 @@ tp_status tp_layernorm_fwd(const tp_bf16* x, const tp_bf16* gamma, const tp_bf16
   if (D > 8192) return TP_ERR_UNSUPPORTED;
   if (D % 8 || !all_aligned(x, gamma, beta, y)) return TP_ERR_MISALIGNED;
   return launch_layernorm_fwd(x, gamma, beta, rows, D, eps, y, mean, rstd, (cudaStream_t)s);
+}
+
+tp_status tp_layernorm_fwd_f16(const tp_bf16* x, const tp_bf16* gamma, const tp_bf16* beta,
+                               int rows, int D, float eps, tp_f16* y, float* mean, float* rstd,
+                               tp_stream s) {
+  if (!all_set(x, gamma, beta, y, mean, rstd) || rows < 0 || D <= 0 || !(eps > 0.f))
+    return TP_ERR_INVALID_ARG;
+  if (D > 8192) return TP_ERR_UNSUPPORTED;
+  if (D % 8 || !all_aligned(x, gamma, beta, y)) return TP_ERR_MISALIGNED;
+  return launch_layernorm_fwd(x, gamma, beta, rows, D, eps, y, mean, rstd, (cudaStream_t)s, true);
 }
 
 size_t tp_layernorm_bwd_workspace_size(int rows, int D) {

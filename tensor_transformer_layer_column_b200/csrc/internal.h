@@ -41,6 +41,12 @@ struct GemmProblem {
 
 tp_status launch_gemm(const GemmProblem& g, cudaStream_t stream);
 
+// Host validation of tp_dims shared by the entry points (status before any launch).
+tp_status check_common(const tp_dims* d);
+tp_status check_mlp(const tp_dims* d);
+tp_status check_attn(const tp_dims* d);
+tp_status check_layer(const tp_dims* d);
+
 // Device error word of the current device (bounded-wait timeouts).
 unsigned int* error_word();
 int sm_count();
@@ -97,6 +103,7 @@ tp_status launch_cast_f16(const uint16_t* src, size_t n, uint16_t* dst, cudaStre
 enum TraceKind : int {
   TK_GEMM = 0, TK_ATTN_FWD = 1, TK_ATTN_BWD_PREP = 2, TK_ATTN_BWD_DKDV = 3, TK_ATTN_BWD_DQ = 4,
   TK_LN_FWD = 5, TK_LN_BWD = 6, TK_LN_PARAM = 7, TK_COLSUM = 8, TK_LAYOUT = 9, TK_CAST = 10,
+  TK_FINISH = 11,
 };
 
 // Brackets one kernel launch with the trace's events when a trace is open.
@@ -115,5 +122,46 @@ class TraceScope {
 inline tp_status cuda_status(cudaError_t e) { return e == cudaSuccess ? TP_OK : TP_ERR_CUDA; }
 
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// ---------------------------------------------------------------- host-side argument checks
+inline bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+// Every non-null pointer 16-byte aligned.
+template <typename... P>
+bool all_aligned(P... ps) {
+  bool ok = true;
+  ((ok = ok && (ps == nullptr || al16(ps))), ...);
+  return ok;
+}
+
+template <typename... P>
+bool all_set(P... ps) {
+  bool ok = true;
+  ((ok = ok && ps != nullptr), ...);
+  return ok;
+}
+
+inline bool supported_t(int t) { return t == 1 || t == 2 || t == 4 || t == 8; }
+
+// Workspace carving: consecutive 256-byte aligned slices.
+struct Carver {
+  uint8_t* base;
+  size_t off = 0;
+  explicit Carver(void* p) : base(static_cast<uint8_t*>(p)) {}
+  template <typename T>
+  T* take(size_t count) {
+    off = align_up(off, 256);
+    T* p = base ? reinterpret_cast<T*>(base + off) : nullptr;
+    off += count * sizeof(T);
+    return p;
+  }
+};
+
+inline tp_status check_ws(void* ws, size_t have, size_t need) {
+  if (need == 0) return TP_OK;
+  if (ws == nullptr || have < need) return TP_ERR_WORKSPACE;
+  if (!al16(ws)) return TP_ERR_MISALIGNED;
+  return TP_OK;
+}
 
 }  // namespace tp

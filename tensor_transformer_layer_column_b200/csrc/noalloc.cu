@@ -53,8 +53,6 @@ tp_status scratch_for_current_device(float** out) {
   return TP_OK;
 }
 
-bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
-
 }  // namespace
 
 }  // namespace tp

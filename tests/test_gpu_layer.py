@@ -19,7 +19,7 @@ pytestmark = pytest.mark.gpu
 PARAMS = ("ln1_g", "ln1_b", "wqkv", "bqkv", "wout", "bout", "ln2_g", "ln2_b", "w1", "b1", "w2", "b2")
 
 
-def _run_and_compare(w, inp):
+def _run_and_compare(w, inp, reference=None):
     d = dims_of(w)
     g = dev(inp)
     layer = ShardedLayer(d, {k: g[k] for k in PARAMS})
@@ -30,7 +30,10 @@ def _run_and_compare(w, inp):
     t = w.t
     p = {k: to_f64(inp[k]) for k in PARAMS}
     x = to_f64(inp["x"])
-    yr, sv = olayer.layer_fwd(x, p, w.batch, w.heads, w.causal, w.ln_eps)
+    if reference is None:
+        yr, sv = olayer.layer_fwd(x, p, w.batch, w.heads, w.causal, w.ln_eps)
+    else:
+        yr, sv, gr = reference
     check("y", y, yr)
     check("h", acts["h"], sv["h"])
     check("u1", acts["u1"], sv["u1"])
@@ -39,7 +42,8 @@ def _run_and_compare(w, inp):
     check("lse", acts["lse"], sv["lse"])
     check("a", acts["a"], olay.shard_cols(sv["a"], t))
     check("hact", acts["hact"], olay.shard_cols(sv["hact"], t))
-    gr = olayer.layer_bwd(x, p, to_f64(inp["dy"]), w.batch, w.heads, w.causal, w.ln_eps)
+    if reference is None:
+        gr = olayer.layer_bwd(x, p, to_f64(inp["dy"]), w.batch, w.heads, w.causal, w.ln_eps)
     check("dx", dx, gr["dx"])
     check("dwqkv", grads["dwqkv"], olay.shard_qkv(gr["dwqkv"], t))
     check("dbqkv", grads["dbqkv"], olay.shard_qkv(gr["dbqkv"][None, :], t))
@@ -66,8 +70,9 @@ def test_layer_fwd_bwd_small(B, S, H, dh, F, t, affine):
 def test_layer_full_size_B4_S2048_D4096_H32_F16384_t8():
     """The pre-LN GPT layer at full size, every output and gradient against the full oracle."""
     require_gpu()
-    w = workload("layer_fwdbwd_B4_S2048_D4096_H32_F16384_t8")
-    _run_and_compare(w, make_inputs(w))
+    from full_size_reference import pre_ln_layer
+    w, inp, yr, sv, gr = pre_ln_layer()
+    _run_and_compare(w, inp, reference=(yr, sv, gr))
 
 
 # ---------------------------------------------------------------- post-LN layer
