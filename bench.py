@@ -9,9 +9,12 @@ line (rank 0).
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                   [--workload NAME]   (any name in synth.WORKLOADS; default the layer)
 
-N > 1 (launched with torch.distributed.run): N independent replicas, one per
-GPU, each on its own batch; no collective on the data path (weak scaling);
-the time is the max over ranks.  --impl reference times the fp64 CPU oracle
+N > 1 (launched with torch.distributed.run): N data-parallel replicas, one per
+GPU, each on its own batch (weak scaling), whose parameter gradients are
+all-reduced over NCCL bucket by bucket, each bucket as soon as the backward
+has produced it, beside the rest of the backward (--no-dp-allreduce: pure
+replicas); the time is the max over ranks.  --dp-allreduce turns the
+reduction on at N = 1 too (a one-rank group: it exercises the path).  --impl reference times the fp64 CPU oracle
 on the host cores on a bounded sample of the same workload.
 """
 from __future__ import annotations
@@ -239,7 +242,7 @@ class ClockSampler:
 class Runner:
     """One step of a workload through the public API, on preallocated buffers."""
 
-    def __init__(self, w: Workload, device):
+    def __init__(self, w: Workload, device, dp: bool = False):
         import tensor_transformer_layer_column_b200 as tl
         from tensor_transformer_layer_column_b200.sublayer import (ShardedAttention, ShardedLayer,
                                                                    ShardedMLP)
@@ -256,6 +259,15 @@ class Runner:
                                     recompute="recompute" in w.kind)
             self.acts = self.mod.alloc_acts()
             self.grads = self.mod.alloc_grads()
+            self.reducer = None
+            if dp:
+                from tensor_transformer_layer_column_b200.data_parallel import (
+                    GradientAllReduce, sharded_layer_buckets)
+                if self.mod.post or self.mod.recompute:
+                    raise ValueError("the data-parallel reduction is wired for the pre-LN layer")
+                self.buckets, self.grads = sharded_layer_buckets(self.mod, device)
+                self.reducer = GradientAllReduce(self.buckets)
+                self.ready = self.reducer.events()
         elif w.kind.startswith("attn"):
             self.mod = ShardedAttention(dims, g["wqkv"], g["bqkv"], g["wout"], g["bout"])
         else:
@@ -272,7 +284,16 @@ class Runner:
         dx = self.dx if dx is None else dx
         if w.kind.startswith("layer"):
             self.mod.forward(x, acts=self.acts, y=y)
-            self.mod.backward(dy, dx=dx, grads=self.grads)
+            if self.reducer is None:
+                self.mod.backward(dy, dx=dx, grads=self.grads)
+                return
+            # Each gradient group's all-reduce waits on its event on a side
+            # stream, so it overlaps the rest of the backward; the step ends
+            # when the last reduction has landed.
+            self.mod.backward(dy, dx=dx, grads=self.grads, ready=self.ready)
+            for group in ("mlp", "attn", "ln1"):
+                self.reducer.launch(group, self.ready[group])
+            self.reducer.finish()
             return
         if self.fwd_out is None:
             self.fwd_out = self.mod.forward(x)
@@ -330,15 +351,24 @@ def activation_report(w: Workload, mod) -> dict:
 def run_ours(args):
     import tensor_transformer_layer_column_b200 as tl
     world, rank, local = dist_env()
-    if world > 1:
+    w = workload(args.workload)
+    dp = args.dp_allreduce if args.dp_allreduce is not None else world > 1
+    dp = dp and w.kind == "layer_fwdbwd"
+    if world > 1 or dp:
         import datetime
+        import socket
         import torch.distributed as dist
         torch.cuda.set_device(local)
+        if world == 1 and "MASTER_PORT" not in os.environ:
+            with socket.socket() as sk:
+                sk.bind(("127.0.0.1", 0))
+                port = sk.getsockname()[1]
+            os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK="0",
+                              WORLD_SIZE="1")
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     device = torch.device("cuda", local if world > 1 else 0)
     torch.cuda.set_device(device)
-    w = workload(args.workload)
-    run = Runner(w, device)
+    run = Runner(w, device, dp=dp)
     g, host_inp = run.g, run.host
     y, dx = run.y, run.dx
     stream = torch.cuda.current_stream(device)
@@ -352,7 +382,7 @@ def run_ours(args):
 
     def barrier():
         if world > 1:
-            torch.distributed.barrier()
+            torch.distributed.barrier(device_ids=[device.index])
 
     # ---- device-resident timed region: K steps, launch trace closed, one
     # event at every step boundary; the step time is the median of the K
@@ -532,8 +562,18 @@ def run_ours(args):
         }
         if w.kind.startswith("layer"):
             line["activations"] = activation_report(w, run.mod)
+        if dp:
+            line["config"]["parallelism"] = (
+                f"t{w.t} shards on each GPU; {world} data-parallel replica(s), parameter "
+                "gradients all-reduced (NCCL, sum) in 3 buckets, each issued on a side stream "
+                "as soon as the backward has produced it")
+            line["dp_allreduce"] = {
+                "buckets": {g: int(b.numel() * b.element_size())
+                            for g, b in run.buckets.flat.items()},
+                "bytes_per_step": int(sum(b.numel() * b.element_size()
+                                          for b in run.buckets.flat.values()))}
         print(json.dumps(line), flush=True)
-    if world > 1:
+    if torch.distributed.is_initialized():
         torch.distributed.destroy_process_group()
 
 
@@ -549,6 +589,11 @@ def main():
                     help="skip the timed CPU oracle sample (for profiler runs)")
     ap.add_argument("--no-e2e", action="store_true",
                     help="skip the host-buffer end-to-end leg (for profiler runs)")
+    ap.add_argument("--dp-allreduce", dest="dp_allreduce", action="store_true", default=None,
+                    help="all-reduce the layer's parameter gradients over the replicas "
+                         "(default with --gpus > 1; at 1 GPU a one-rank group)")
+    ap.add_argument("--no-dp-allreduce", dest="dp_allreduce", action="store_false",
+                    help="pure replicas: no gradient reduction")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

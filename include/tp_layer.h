@@ -269,6 +269,31 @@ tp_status tp_layer_bwd(const tp_dims* dims, const tp_bf16* x, const tp_layer_par
                        const tp_layer_acts* acts, const tp_bf16* dy, tp_bf16* dx,
                        const tp_layer_grads* grads, void* ws, size_t ws_bytes, tp_stream stream);
 
+/* tp_layer_bwd_notify: tp_layer_bwd (same arguments and results, bit for bit),
+ * for data-parallel training, where each replica's parameter gradients are
+ * all-reduced over the replicas ("3D decomposition in practice" and "What
+ * actually limits throughput in production": that reduction runs off the
+ * critical path, beside the rest of the backward pass).  Each non-NULL
+ * member of *ready is a cudaEvent_t (created by the caller on the current
+ * device) that is recorded on `stream` as soon as the kernels writing a
+ * group of gradients have been enqueued:
+ *   mlp   dw1, db1, dw2, db2       (first: the MLP backward runs first)
+ *   attn  dwqkv, dbqkv, dwout, dbout, dln2_g, dln2_b
+ *   ln1   dln1_g, dln1_b           (last)
+ * A stream that waits on an event may reduce that group while the later
+ * kernels of the backward still run.  ready may be NULL (then this is
+ * tp_layer_bwd). */
+typedef struct {
+  void* mlp;    /* cudaEvent_t or NULL */
+  void* attn;   /* cudaEvent_t or NULL */
+  void* ln1;    /* cudaEvent_t or NULL */
+} tp_grad_ready;
+
+tp_status tp_layer_bwd_notify(const tp_dims* dims, const tp_bf16* x, const tp_layer_params* params,
+                              const tp_layer_acts* acts, const tp_bf16* dy, tp_bf16* dx,
+                              const tp_layer_grads* grads, const tp_grad_ready* ready, void* ws,
+                              size_t ws_bytes, tp_stream stream);
+
 /* ------------------------------------------------------------------ activation recomputation
  * "What actually limits throughput in production", the activation memory vs.
  * recomputation trade-off: instead of keeping the layer's activations from

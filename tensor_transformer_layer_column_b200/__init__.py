@@ -24,7 +24,7 @@ __all__ = [
     "shard_cols", "unshard_cols", "shard_rows", "unshard_rows", "shard_qkv_heads",
     "unshard_qkv_heads", "mlp_fwd", "mlp_bwd", "attn_fwd", "attn_bwd", "layer_fwd", "layer_bwd",
     "layernorm_fwd", "layernorm_bwd", "layernorm_bwd_workspace_size", "layernorm_bwd_noalloc",
-    "LaunchTrace", "RANK_MLP_FWD", "RANK_MLP_BWD", "RANK_ATTN_FWD", "RANK_ATTN_BWD",
+    "LaunchTrace", "GradReady", "layer_bwd_notify", "RANK_MLP_FWD", "RANK_MLP_BWD", "RANK_ATTN_FWD", "RANK_ATTN_BWD",
     "rank_workspace_size", "mlp_fwd_rank", "mlp_bwd_rank", "attn_fwd_rank", "attn_bwd_rank",
     "rowpar_finish", "layernorm_fwd_f16",
     "TRACE_KINDS", "selftest_wait_timeout",
@@ -82,6 +82,10 @@ class LayerGrads(ctypes.Structure):
                                   "dln2_g", "dln2_b", "dw1", "db1", "dw2", "db2")]
 
 
+class GradReady(ctypes.Structure):
+    _fields_ = [(n, _P) for n in ("mlp", "attn", "ln1")]
+
+
 # name -> argument types (all return tp_status unless listed in _RESTYPES)
 _SIGS = {
     "tp_version": [],
@@ -103,6 +107,9 @@ _SIGS = {
     "tp_layer_bwd": [ctypes.POINTER(Dims), _P, ctypes.POINTER(LayerParams),
                      ctypes.POINTER(LayerActs), _P, _P, ctypes.POINTER(LayerGrads), _P,
                      ctypes.c_size_t, _P],
+    "tp_layer_bwd_notify": [ctypes.POINTER(Dims), _P, ctypes.POINTER(LayerParams),
+                            ctypes.POINTER(LayerActs), _P, _P, ctypes.POINTER(LayerGrads),
+                            ctypes.POINTER(GradReady), _P, ctypes.c_size_t, _P],
     "tp_postln_layer_fwd": [ctypes.POINTER(Dims), _P, ctypes.POINTER(LayerParams),
                             ctypes.POINTER(PostLNActs), _P, _P, ctypes.c_size_t, _P],
     "tp_postln_layer_bwd": [ctypes.POINTER(Dims), _P, ctypes.POINTER(LayerParams),
@@ -296,6 +303,22 @@ def layer_bwd(dims, x, params: dict, acts: dict, dy, dx, grads: dict, ws, stream
     _check(lib().tp_layer_bwd(ctypes.byref(dims), _ptr(x), ctypes.byref(p), ctypes.byref(a),
                               _ptr(dy), _ptr(dx), ctypes.byref(g), wp, wn, _stream(stream, x)),
            "tp_layer_bwd")
+
+
+def layer_bwd_notify(dims, x, params: dict, acts: dict, dy, dx, grads: dict, ready: dict, ws,
+                     stream=None):
+    """tp_layer_bwd that records ready["mlp"], ready["attn"], ready["ln1"]
+    (torch.cuda.Event, already recorded once so that their handles exist) as
+    each group of parameter gradients is enqueued."""
+    wp, wn = _ws(ws)
+    p = _struct(LayerParams, params)
+    a = _struct(LayerActs, acts)
+    g = _struct(LayerGrads, grads)
+    r = GradReady(**{k: (None if ready.get(k) is None else ready[k].cuda_event)
+                     for k in ("mlp", "attn", "ln1")})
+    _check(lib().tp_layer_bwd_notify(ctypes.byref(dims), _ptr(x), ctypes.byref(p), ctypes.byref(a),
+                                     _ptr(dy), _ptr(dx), ctypes.byref(g), ctypes.byref(r), wp, wn,
+                                     _stream(stream, x)), "tp_layer_bwd_notify")
 
 
 def postln_layer_fwd(dims, x, params: dict, acts: dict, y, ws=None, stream=None):

@@ -701,9 +701,16 @@ tp_status layer_fwd_core(const Sizes& z, const tp_dims* dims, const tp_bf16* x,
 
 // Pre-LN backward; `ws` is laid out as layer_bwd_ws describes and its first
 // slice already holds the fp16 copy of Wqkv.
+// Records `ev` (a caller's cudaEvent_t, may be NULL) on the stream.
+tp_status record_ready(void* ev, cudaStream_t cs) {
+  if (ev == nullptr) return TP_OK;
+  return cuda_status(cudaEventRecord(static_cast<cudaEvent_t>(ev), cs));
+}
+
 tp_status layer_bwd_core(const Sizes& z, const tp_dims* dims, const tp_bf16* x,
                          const tp_layer_params* p, const tp_layer_acts* a, const tp_bf16* dy,
-                         tp_bf16* dx, const tp_layer_grads* g, void* ws, cudaStream_t cs) {
+                         tp_bf16* dx, const tp_layer_grads* g, void* ws, cudaStream_t cs,
+                         const tp_grad_ready* ready = nullptr) {
   tp_status st;
   Carver c(ws);
   uint16_t* w16 = c.take<uint16_t>((size_t)(z.D * 3 * z.D));
@@ -717,6 +724,7 @@ tp_status layer_bwd_core(const Sizes& z, const tp_dims* dims, const tp_bf16* x,
   if ((st = mlp_bwd_impl(z, a->u2, p->w1, p->w2, a->a, a->hact, dy, nullptr, du, g->dw1, g->dw2,
                          g->db1, g->db2, subws, cs)) != TP_OK)
     return st;
+  if (ready && (st = record_ready(ready->mlp, cs)) != TP_OK) return st;
   if ((st = launch_layernorm_bwd(du, a->h, p->ln2_g, a->mean2, a->rstd2, dy, z.T, (int)z.D, dh,
                                  g->dln2_g, g->dln2_b, lnp, cs)) != TP_OK)
     return st;
@@ -724,8 +732,11 @@ tp_status layer_bwd_core(const Sizes& z, const tp_dims* dims, const tp_bf16* x,
   if ((st = attn_bwd_impl(z, dims->causal, a->u1, w16, p->wout, a->qkv, a->o, a->lse, dh,
                           nullptr, du, g->dwqkv, g->dbqkv, g->dwout, g->dbout, subws, cs)) != TP_OK)
     return st;
-  return launch_layernorm_bwd(du, x, p->ln1_g, a->mean1, a->rstd1, dh, z.T, (int)z.D, dx,
-                              g->dln1_g, g->dln1_b, lnp, cs);
+  if (ready && (st = record_ready(ready->attn, cs)) != TP_OK) return st;
+  if ((st = launch_layernorm_bwd(du, x, p->ln1_g, a->mean1, a->rstd1, dh, z.T, (int)z.D, dx,
+                                 g->dln1_g, g->dln1_b, lnp, cs)) != TP_OK)
+    return st;
+  return ready ? record_ready(ready->ln1, cs) : TP_OK;
 }
 
 tp_status check_layer_params(const tp_layer_params* p) {
@@ -797,6 +808,31 @@ tp_status tp_layer_bwd(const tp_dims* dims, const tp_bf16* x, const tp_layer_par
   uint16_t* w16 = static_cast<uint16_t*>(ws);
   if ((st = launch_cast_f16(p->wqkv, (size_t)(z.D * 3 * z.D), w16, cs)) != TP_OK) return st;
   return layer_bwd_core(z, dims, x, p, a, dy, dx, g, ws, cs);
+}
+
+tp_status tp_layer_bwd_notify(const tp_dims* dims, const tp_bf16* x, const tp_layer_params* p,
+                              const tp_layer_acts* a, const tp_bf16* dy, tp_bf16* dx,
+                              const tp_layer_grads* g, const tp_grad_ready* ready, void* ws,
+                              size_t ws_bytes, tp_stream s) {
+  tp_status st = check_layer(dims);
+  if (st != TP_OK) return st;
+  if ((st = check_layer_ptrs(p, a, has_tokens(dims))) != TP_OK) return st;
+  if ((st = check_layer_grads(dims, x, dy, dx, g)) != TP_OK) return st;
+  const Sizes z = sizes_of(*dims);
+  const size_t need = z.T ? layer_bwd_ws(z) : 0;
+  if ((st = check_ws(ws, ws_bytes, need)) != TP_OK) return st;
+  cudaStream_t cs = (cudaStream_t)s;
+  if (z.T == 0) {
+    if ((st = layer_bwd_empty(z, dims->causal, g, cs)) != TP_OK) return st;
+    if (ready) {
+      for (void* ev : {ready->mlp, ready->attn, ready->ln1})
+        if ((st = record_ready(ev, cs)) != TP_OK) return st;
+    }
+    return TP_OK;
+  }
+  uint16_t* w16 = static_cast<uint16_t*>(ws);
+  if ((st = launch_cast_f16(p->wqkv, (size_t)(z.D * 3 * z.D), w16, cs)) != TP_OK) return st;
+  return layer_bwd_core(z, dims, x, p, a, dy, dx, g, ws, cs, ready);
 }
 
 tp_status tp_layer_fwd_nosave(const tp_dims* dims, const tp_bf16* x, const tp_layer_params* p,

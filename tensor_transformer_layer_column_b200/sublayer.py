@@ -15,7 +15,8 @@ import torch
 
 from . import (Dims, OP_ATTN_BWD, OP_ATTN_FWD, OP_LAYER_BWD, OP_LAYER_BWD_RECOMPUTE,
                OP_LAYER_FWD, OP_LAYER_FWD_NOSAVE, OP_MLP_BWD, OP_POSTLN_BWD, OP_POSTLN_FWD,
-               attn_bwd, attn_fwd, layer_bwd, layer_bwd_recompute, layer_fwd, layer_fwd_nosave,
+               attn_bwd, attn_fwd, layer_bwd, layer_bwd_notify, layer_bwd_recompute, layer_fwd,
+               layer_fwd_nosave,
                mlp_bwd, mlp_fwd, postln_layer_bwd, postln_layer_fwd, shard_cols,
                shard_qkv_heads, shard_rows, unshard_cols, unshard_qkv_heads, workspace_size)
 
@@ -358,7 +359,9 @@ class ShardedLayer:
         return y, acts
 
     @_nvtx("tp.layer.backward")
-    def backward(self, dy, dx=None, grads=None, bias_grads=True):
+    def backward(self, dy, dx=None, grads=None, bias_grads=True, ready=None):
+        """ready (pre-LN, saving layer only): {"mlp", "attn", "ln1"} -> torch.cuda.Event,
+        recorded as each group of parameter gradients is enqueued (tp_layer_bwd_notify)."""
         d = self.dims
         x, acts = self.saved
         T, D = d.batch * d.seq, d.hidden
@@ -377,5 +380,10 @@ class ShardedLayer:
             return dx, grads
         if self.ws is None:
             self.ws = _ws(OP_POSTLN_BWD if self.post else OP_LAYER_BWD, d, self.device)
+        if ready is not None:
+            if self.post:
+                raise ValueError("gradient-ready events are provided for the pre-LN layer")
+            layer_bwd_notify(d, x, self.p, acts, dy, dx, grads, ready, self.ws)
+            return dx, grads
         (postln_layer_bwd if self.post else layer_bwd)(d, x, self.p, acts, dy, dx, grads, self.ws)
         return dx, grads
