@@ -277,9 +277,9 @@ tp_status tp_layer_bwd(const tp_dims* dims, const tp_bf16* x, const tp_layer_par
  * member of *ready is a cudaEvent_t (created by the caller on the current
  * device) that is recorded on `stream` as soon as the kernels writing a
  * group of gradients have been enqueued:
- *   mlp   dw1, db1, dw2, db2       (first: the MLP backward runs first)
- *   attn  dwqkv, dbqkv, dwout, dbout, dln2_g, dln2_b
- *   ln1   dln1_g, dln1_b           (last)
+ *   mlp   dw1, db1, dw2, db2, dln2_g, dln2_b   (first: the MLP backward runs first)
+ *   attn  dwqkv, dbqkv, dwout
+ *   ln1   dln1_g, dln1_b, dbout               (last: LN1's backward also sums dbout)
  * A stream that waits on an event may reduce that group while the later
  * kernels of the backward still run.  ready may be NULL (then this is
  * tp_layer_bwd). */

@@ -369,7 +369,7 @@ size_t layer_bwd_ws(const Sizes& z) {
   c.take<uint16_t>((size_t)(z.D * 3 * z.D));   // fp16 copy of Wqkv
   c.take<uint16_t>((size_t)(z.T * z.D));       // du
   c.take<uint16_t>((size_t)(z.T * z.D));       // dh
-  c.take<float>(layernorm_bwd_partial_floats(z.T, (int)z.D));
+  c.take<float>(layernorm_bwd_partial_floats(z.T, (int)z.D, 3));
   const size_t sub = mlp_bwd_ws(z) > attn_bwd_core_ws(z) ? mlp_bwd_ws(z) : attn_bwd_core_ws(z);
   c.take<uint8_t>(sub);
   return align_up(c.off, 256);
@@ -716,25 +716,27 @@ tp_status layer_bwd_core(const Sizes& z, const tp_dims* dims, const tp_bf16* x,
   uint16_t* w16 = c.take<uint16_t>((size_t)(z.D * 3 * z.D));
   uint16_t* du = c.take<uint16_t>((size_t)(z.T * z.D));
   uint16_t* dh = c.take<uint16_t>((size_t)(z.T * z.D));
-  float* lnp = c.take<float>(layernorm_bwd_partial_floats(z.T, (int)z.D));
+  float* lnp = c.take<float>(layernorm_bwd_partial_floats(z.T, (int)z.D, 3));
   const size_t sub = mlp_bwd_ws(z) > attn_bwd_core_ws(z) ? mlp_bwd_ws(z) : attn_bwd_core_ws(z);
   void* subws = c.take<uint8_t>(sub);
 
-  // y = h + MLP(LN2(h)):  du2 = MLP^T(dy);  dh = dy + LN2^T(du2).
+  // y = h + MLP(LN2(h)):  du2 = MLP^T(dy);  dh = dy + LN2^T(du2).  db2 = column
+  // sums of dy, which LN2's backward reads as the residual gradient anyway.
   if ((st = mlp_bwd_impl(z, a->u2, p->w1, p->w2, a->a, a->hact, dy, nullptr, du, g->dw1, g->dw2,
-                         g->db1, g->db2, subws, cs)) != TP_OK)
+                         g->db1, nullptr, subws, cs)) != TP_OK)
+    return st;
+  if ((st = launch_layernorm_bwd(du, a->h, p->ln2_g, a->mean2, a->rstd2, dy, z.T, (int)z.D, dh,
+                                 g->dln2_g, g->dln2_b, lnp, cs, nullptr, g->db2)) != TP_OK)
     return st;
   if (ready && (st = record_ready(ready->mlp, cs)) != TP_OK) return st;
-  if ((st = launch_layernorm_bwd(du, a->h, p->ln2_g, a->mean2, a->rstd2, dy, z.T, (int)z.D, dh,
-                                 g->dln2_g, g->dln2_b, lnp, cs)) != TP_OK)
-    return st;
-  // h = x + Attn(LN1(x)):  du1 = Attn^T(dh);  dx = dh + LN1^T(du1).
+  // h = x + Attn(LN1(x)):  du1 = Attn^T(dh);  dx = dh + LN1^T(du1).  dbout =
+  // column sums of dh, read by LN1's backward as its residual gradient.
   if ((st = attn_bwd_impl(z, dims->causal, a->u1, w16, p->wout, a->qkv, a->o, a->lse, dh,
-                          nullptr, du, g->dwqkv, g->dbqkv, g->dwout, g->dbout, subws, cs)) != TP_OK)
+                          nullptr, du, g->dwqkv, g->dbqkv, g->dwout, nullptr, subws, cs)) != TP_OK)
     return st;
   if (ready && (st = record_ready(ready->attn, cs)) != TP_OK) return st;
   if ((st = launch_layernorm_bwd(du, x, p->ln1_g, a->mean1, a->rstd1, dh, z.T, (int)z.D, dx,
-                                 g->dln1_g, g->dln1_b, lnp, cs)) != TP_OK)
+                                 g->dln1_g, g->dln1_b, lnp, cs, nullptr, g->dbout)) != TP_OK)
     return st;
   return ready ? record_ready(ready->ln1, cs) : TP_OK;
 }

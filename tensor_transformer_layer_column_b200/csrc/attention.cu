@@ -52,6 +52,13 @@ enum : unsigned int {
   ERR_ATTN_DQ_WAIT = 0x203,
 };
 
+// Compile-time flag for generic lambdas: one code path with the causal
+// select, one without, chosen per block.
+template <bool B>
+struct BoolTag {
+  static constexpr bool value = B;
+};
+
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
@@ -321,21 +328,23 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q128,
       tc_fence_before();
       mbar_arrive(&s_free[tile]);
       // Keys past the last visible one (after the query, or past S) are masked: a select
-      // per element against a bound fixed once per block, no branches.
+      // per element against a bound fixed once per block, taken only in blocks where
+      // some row of the warp has a masked key (the causal diagonal, the sequence end).
       const int kmax = (p.causal ? min(q, p.S - 1) : p.S - 1) - j * C::BN;
-      // Row max and (below) row sum over 8 interleaved partials: short
-      // dependency chains instead of one chain through all 64 columns.
+      if (!__all_sync(0xffffffffu, kmax >= C::BN - 1)) {
+#pragma unroll
+        for (int c = 0; c < C::BN; ++c) s[c] = c > kmax ? -INFINITY : s[c];
+      }
+      // Row max of the raw scores (the scale is positive, so scaling after the
+      // max gives the max of the scaled scores), over 8 interleaved partials:
+      // short dependency chains instead of one chain through all 64 columns.
       float m8[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) m8[e] = -1e30f;
 #pragma unroll
-      for (int c = 0; c < C::BN; ++c) {
-        const float v = c > kmax ? -INFINITY : s[c] * p.scale_log2;
-        s[c] = v;
-        m8[c & 7] = fmaxf(m8[c & 7], v);
-      }
+      for (int c = 0; c < C::BN; ++c) m8[c & 7] = fmaxf(m8[c & 7], s[c]);
       const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                             fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+                             fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7]))) * p.scale_log2;
       float alpha = 1.0f;
       if (j == 0) {
         m_used = mx;
@@ -349,7 +358,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q128,
       for (int e = 0; e < 8; ++e) l8[e] = 0.f;
 #pragma unroll
       for (int c = 0; c < C::BN; ++c) {
-        const float e = fast_exp2(s[c] - m_used);
+        const float e = fast_exp2(fmaf(s[c], p.scale_log2, -m_used));   // masked: 2^-inf = 0
         s[c] = e;
         l8[c & 7] += e;
       }
@@ -640,32 +649,44 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_kv128,
       // already waited for.
       const uint32_t t_st = tmem + bf * 128 + lane_off;
       // Queries qs + qi with qi < qmin precede key kpos and are masked (causal):
-      // a select per element, no branches.
+      // a select per element, taken only in blocks where some key row of the
+      // warp has a masked query (the causal diagonal).
       const int qmin = p.causal ? kpos - qs : 0;
-#pragma unroll 1
-      for (int c = 0; c < 2; ++c) {
+      const bool masked = !__all_sync(0xffffffffu, qmin <= 0);
+      auto half = [&](int c, auto mask_tag) {
+        constexpr bool MASK = decltype(mask_tag)::value;
         uint32_t rs[32], rd[32];
         tmem_ld32(t_st + c * 32, rs);
         tmem_ld32(t_st + 64 + c * 32, rd);
         tc_wait_ld();
         uint32_t pk[16], dk[16];   // fp16 pairs of P^T and dS^T
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          float pe[2], de[2];
+        for (int e = 0; e < 32; e += 4) {
+          // lse2 and Dv of four queries in one shared-memory load each.
+          const float4 l4 = *reinterpret_cast<const float4*>(vl + c * 32 + e);
+          const float4 d4 = *reinterpret_cast<const float4*>(vd + c * 32 + e);
+          const float la[4] = {l4.x, l4.y, l4.z, l4.w}, da[4] = {d4.x, d4.y, d4.z, d4.w};
+          float pe[4], de[4];
 #pragma unroll
-          for (int h2 = 0; h2 < 2; ++h2) {
-            const int qi = c * 32 + e + h2;
+          for (int h4 = 0; h4 < 4; ++h4) {
             // Padded queries carry lse2 = +inf and dvec = 0, so they give 0.
-            float x = fast_exp2(__uint_as_float(rs[e + h2]) * p.scale_log2 - vl[qi]);
-            x = qi < qmin ? 0.f : x;
-            pe[h2] = x;
-            de[h2] = x * (__uint_as_float(rd[e + h2]) - vd[qi]);
+            float x = fast_exp2(fmaf(__uint_as_float(rs[e + h4]), p.scale_log2, -la[h4]));
+            if (MASK) x = c * 32 + e + h4 < qmin ? 0.f : x;
+            pe[h4] = x;
+            de[h4] = x * (__uint_as_float(rd[e + h4]) - da[h4]);
           }
           pk[e / 2] = pack_f16x2(pe[0], pe[1]);
+          pk[e / 2 + 1] = pack_f16x2(pe[2], pe[3]);
           dk[e / 2] = pack_f16x2(de[0], de[1]);
+          dk[e / 2 + 1] = pack_f16x2(de[2], de[3]);
         }
         tmem_st16(t_st + c * 16, pk);
         tmem_st16(t_st + 64 + c * 16, dk);
+      };
+#pragma unroll 1
+      for (int c = 0; c < 2; ++c) {
+        if (masked) half(c, BoolTag<true>{});
+        else half(c, BoolTag<false>{});
       }
       tc_wait_st();
       tc_fence_before();
@@ -888,16 +909,23 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q128,
       // Keys past the last visible one (after the query, or past S) are
       // masked: a select per element against a bound fixed once per block.
       const int kmax = (p.causal ? min(q, p.S - 1) : p.S - 1) - ks;
-      auto ds = [&](const uint32_t (&rs)[32], uint32_t (&rd)[32], int c) {
+      auto ds = [&](const uint32_t (&rs)[32], uint32_t (&rd)[32], int c, auto mask_tag) {
+        constexpr bool MASK = decltype(mask_tag)::value;
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
-          float pe = fast_exp2(__uint_as_float(rs[e]) * p.scale_log2 - l2);
-          pe = c * 32 + e > kmax ? 0.f : pe;
+          float pe = fast_exp2(fmaf(__uint_as_float(rs[e]), p.scale_log2, -l2));
+          if (MASK) pe = c * 32 + e > kmax ? 0.f : pe;
           rd[e] = __float_as_uint(pe * (__uint_as_float(rd[e]) - dv));
         }
       };
-      ds(rs0, rd0, 0);
-      ds(rs1, rd1, 1);
+      // The select only where some row of the warp has a masked key.
+      if (!__all_sync(0xffffffffu, kmax >= C::BK - 1)) {
+        ds(rs0, rd0, 0, BoolTag<true>{});
+        ds(rs1, rd1, 1, BoolTag<true>{});
+      } else {
+        ds(rs0, rd0, 0, BoolTag<false>{});
+        ds(rs1, rd1, 1, BoolTag<false>{});
+      }
       uint32_t pk[32];   // dS as fp16 pairs, 64 keys
 #pragma unroll
       for (int e = 0; e < 16; ++e) {

@@ -65,11 +65,16 @@ tp_status launch_layernorm_fwd(const uint16_t* x, const uint16_t* g, const uint1
 // Row blocks of the LayerNorm backward (2 per SM, at most one per row); the
 // dgamma/dbeta partials hold 2 * D floats per block.
 int layernorm_bwd_blocks(long long rows);
-size_t layernorm_bwd_partial_floats(long long rows, int D);
+// Partial floats of the LayerNorm backward: nk rows of D per block (2: dgamma,
+// dbeta; 3: also the column sums of dres, see launch_layernorm_bwd).
+size_t layernorm_bwd_partial_floats(long long rows, int D, int nk = 2);
+// dres_sum (needs dres; partial sized with nk = 3): the column sums of dres,
+// bf16 [D] -- the bias gradient of the product whose output gradient dres is.
 tp_status launch_layernorm_bwd(const uint16_t* dy, const uint16_t* x, const uint16_t* g,
                                const float* mean, const float* rstd, const uint16_t* dres,
                                long long rows, int D, uint16_t* dx, uint16_t* dg, uint16_t* db,
-                               float* partial, cudaStream_t stream, float* dx32 = nullptr);
+                               float* partial, cudaStream_t stream, float* dx32 = nullptr,
+                               uint16_t* dres_sum = nullptr);
 
 // fp32 upstream gradient dy; dx is written bf16 and, when dx32 is set, also fp32.
 tp_status launch_layernorm_bwd_f32(const float* dy, const uint16_t* x, const uint16_t* g,

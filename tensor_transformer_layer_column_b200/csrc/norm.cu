@@ -167,8 +167,11 @@ struct DyChunk<true> {
   }
 };
 
-// DY32: dy is fp32.  dx32, when set, receives an fp32 copy of dx.
-template <int CH, bool DY32 = false>
+// DY32: dy is fp32.  dx32, when set, receives an fp32 copy of dx.  RSUM: the
+// block also sums the rows of dres (a third partial row, [gridDim.x][3][D]):
+// the column sums of a residual gradient that passes through, e.g. the bias
+// gradient of the row-parallel product that produced it.
+template <int CH, bool DY32 = false, bool RSUM = false>
 __global__ void __launch_bounds__(LNB_THREADS, 2)
 ln_bwd_kernel(const void* __restrict__ dy, const uint16_t* __restrict__ x,
               const uint16_t* __restrict__ g, const float* __restrict__ mean,
@@ -178,13 +181,19 @@ ln_bwd_kernel(const void* __restrict__ dy, const uint16_t* __restrict__ x,
   __shared__ float red[2][2][LNB_THREADS / 32];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int nch = D >> 3;
-  float gam[CH][8], adg[CH][8], adb[CH][8];
+  // gamma stays packed (bf16); xhat and g = dy * gamma are recomputed from the
+  // packed row in the output pass instead of being held in fp32 registers.
+  uint4 gpk[CH];
+  float adg[CH][8], adb[CH][8], adr[RSUM ? CH : 1][8];
 #pragma unroll
   for (int j = 0; j < CH; ++j) {
     const int c = tid + LNB_THREADS * j;
 #pragma unroll
-    for (int e = 0; e < 8; ++e) adg[j][e] = adb[j][e] = 0.f;
-    if (c < nch) unpack8(*reinterpret_cast<const uint4*>(g + c * 8), gam[j]);
+    for (int e = 0; e < 8; ++e) {
+      adg[j][e] = adb[j][e] = 0.f;
+      if (RSUM) adr[j][e] = 0.f;
+    }
+    if (c < nch) gpk[j] = *reinterpret_cast<const uint4*>(g + c * 8);
   }
   const long long r0 = (long long)blockIdx.x * rows_per_block;
   const long long r1 = min(rows, r0 + rows_per_block);
@@ -209,21 +218,21 @@ ln_bwd_kernel(const void* __restrict__ dy, const uint16_t* __restrict__ x,
     uint4 nx[CH], nres[CH];
     if (r + 1 < r1) load_row(r + 1, ndy, nx, nres);
     const float mu = mean[r], rs = rstd[r];
-    float xh[CH][8], gv[CH][8];
     float s1 = 0.f, s2 = 0.f;
 #pragma unroll
     for (int j = 0; j < CH; ++j) {
       if (tid + LNB_THREADS * j < nch) {
-        float dv[8];
+        float dv[8], xv[8], gm[8];
         cdy[j].get(dv);
-        unpack8(cx[j], xh[j]);
+        unpack8(cx[j], xv);
+        unpack8(gpk[j], gm);
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          xh[j][e] = (xh[j][e] - mu) * rs;
-          gv[j][e] = dv[e] * gam[j][e];
-          s1 += gv[j][e];
-          s2 += gv[j][e] * xh[j][e];
-          adg[j][e] += dv[e] * xh[j][e];
+          const float xh = (xv[e] - mu) * rs;
+          const float gv = dv[e] * gm[e];
+          s1 += gv;
+          s2 += gv * xh;
+          adg[j][e] += dv[e] * xh;
           adb[j][e] += dv[e];
         }
       }
@@ -247,14 +256,23 @@ ln_bwd_kernel(const void* __restrict__ dy, const uint16_t* __restrict__ x,
     for (int j = 0; j < CH; ++j) {
       const int c = tid + LNB_THREADS * j;
       if (c < nch) {
-        float o[8];
+        float dv[8], xv[8], gm[8], o[8];
+        cdy[j].get(dv);
+        unpack8(cx[j], xv);
+        unpack8(gpk[j], gm);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) o[e] = rs * (gv[j][e] - m1 - xh[j][e] * m2);
+        for (int e = 0; e < 8; ++e) {
+          const float xh = (xv[e] - mu) * rs;
+          o[e] = rs * (dv[e] * gm[e] - m1 - xh * m2);
+        }
         if (dres != nullptr) {
           float rv[8];
           unpack8(cres[j], rv);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) o[e] += rv[e];
+          for (int e = 0; e < 8; ++e) {
+            o[e] += rv[e];
+            if (RSUM) adr[j][e] += rv[e];
+          }
         }
         *reinterpret_cast<uint4*>(dx + r * D + c * 8) = pack8(o);
         if (dx32 != nullptr) {
@@ -271,7 +289,7 @@ ln_bwd_kernel(const void* __restrict__ dy, const uint16_t* __restrict__ x,
       cres[j] = nres[j];
     }
   }
-  float* pg = partial + (long long)blockIdx.x * 2 * D;
+  float* pg = partial + (long long)blockIdx.x * (RSUM ? 3 : 2) * D;
 #pragma unroll
   for (int j = 0; j < CH; ++j) {
     const int c = tid + LNB_THREADS * j;
@@ -280,6 +298,7 @@ ln_bwd_kernel(const void* __restrict__ dy, const uint16_t* __restrict__ x,
       for (int e = 0; e < 8; ++e) {
         pg[c * 8 + e] = adg[j][e];
         pg[D + c * 8 + e] = adb[j][e];
+        if (RSUM) pg[2 * D + c * 8 + e] = adr[j][e];
       }
     }
   }
@@ -307,18 +326,21 @@ __device__ __forceinline__ float reduce_rows_fixed(const float* __restrict__ row
   return t;
 }
 
-// out_k[c] = sum over blocks b (fixed order) of partial[b][k][c]; k = 0 dgamma, 1 dbeta.
+// out_k[c] = sum over blocks b (fixed order) of partial[b][k][c], k < nk:
+// 0 dgamma, 1 dbeta, 2 the column sums of dres.
 __global__ void __launch_bounds__(256)
-ln_param_reduce(const float* __restrict__ partial, int nblocks, int D, uint16_t* __restrict__ dg,
-                uint16_t* __restrict__ db) {
+ln_param_reduce(const float* __restrict__ partial, int nblocks, int D, int nk,
+                uint16_t* __restrict__ dg, uint16_t* __restrict__ db, uint16_t* __restrict__ dr) {
   __shared__ float red[8][33];
-  const float t = reduce_rows_fixed(partial, nblocks, 2LL * D, 2LL * D, red);
+  const long long width = (long long)nk * D;
+  const float t = reduce_rows_fixed(partial, nblocks, width, width, red);
   const int i = blockIdx.x * 32 + (threadIdx.x & 31);
-  if ((threadIdx.x >> 5) != 0 || i >= 2 * D) return;
-  uint16_t* out = i < D ? dg : db;
+  if ((threadIdx.x >> 5) != 0 || i >= width) return;
+  const int k = i / D;
+  uint16_t* out = k == 0 ? dg : (k == 1 ? db : dr);
   if (out == nullptr) return;
   __nv_bfloat16 v = __float2bfloat16_rn(t);
-  out[i < D ? i : i - D] = *reinterpret_cast<uint16_t*>(&v);
+  out[i - k * D] = *reinterpret_cast<uint16_t*>(&v);
 }
 
 // Column sums of S stacked [rows][cols] matrices, pass 1: block (cx, cy, s)
@@ -459,41 +481,58 @@ tp_status launch_layernorm_fwd(const uint16_t* x, const uint16_t* g, const uint1
   return ln_fwd_dispatch<false>(x, g, b, rows, D, eps, y, mean, rstd, stream);
 }
 
-size_t layernorm_bwd_partial_floats(long long rows, int D) {
-  return (size_t)layernorm_bwd_blocks(rows < 1 ? 1 : rows) * 2 * (size_t)D;
+size_t layernorm_bwd_partial_floats(long long rows, int D, int nk) {
+  return (size_t)layernorm_bwd_blocks(rows < 1 ? 1 : rows) * (size_t)nk * (size_t)D;
 }
 
 namespace {
+template <int CH, bool DY32>
+void ln_bwd_kernel_launch(bool rsum, int nb, const void* dy, const uint16_t* x, const uint16_t* g,
+                          const float* mean, const float* rstd, const uint16_t* dres,
+                          long long rows, int D, int rpb, uint16_t* dx, float* partial,
+                          float* dx32, cudaStream_t stream) {
+  if (rsum)
+    ln_bwd_kernel<CH, DY32, true><<<nb, LNB_THREADS, 0, stream>>>(dy, x, g, mean, rstd, dres, rows,
+                                                                   D, rpb, dx, partial, dx32);
+  else
+    ln_bwd_kernel<CH, DY32, false><<<nb, LNB_THREADS, 0, stream>>>(dy, x, g, mean, rstd, dres,
+                                                                    rows, D, rpb, dx, partial, dx32);
+}
+
+// dr (may be NULL; needs dres): column sums of dres, from a third partial row.
 template <bool DY32>
 tp_status ln_bwd_launch(const void* dy, const uint16_t* x, const uint16_t* g, const float* mean,
                         const float* rstd, const uint16_t* dres, long long rows, int D,
                         uint16_t* dx, float* dx32, uint16_t* dg, uint16_t* db, int nb,
-                        float* partial, cudaStream_t stream) {
+                        float* partial, cudaStream_t stream, uint16_t* dr = nullptr) {
+  if (dres == nullptr) dr = nullptr;
   if (rows == 0) {
-    if (dg) cudaMemsetAsync(dg, 0, (size_t)D * 2, stream);
-    if (db) cudaMemsetAsync(db, 0, (size_t)D * 2, stream);
+    for (uint16_t* o : {dg, db, dr})
+      if (o) cudaMemsetAsync(o, 0, (size_t)D * 2, stream);
     return cuda_status(cudaGetLastError());
   }
   if (nb < 1) return TP_ERR_INVALID_ARG;
   const int rpb = (int)((rows + nb - 1) / nb);
   const int per_thread = (D / 8 + LNB_THREADS - 1) / LNB_THREADS;
+  const bool rsum = dr != nullptr;
   {
     TraceScope ts(stream, TK_LN_BWD);
     if (per_thread <= 1)
-      ln_bwd_kernel<1, DY32><<<nb, LNB_THREADS, 0, stream>>>(dy, x, g, mean, rstd, dres, rows, D,
-                                                              rpb, dx, partial, dx32);
+      ln_bwd_kernel_launch<1, DY32>(rsum, nb, dy, x, g, mean, rstd, dres, rows, D, rpb, dx,
+                                    partial, dx32, stream);
     else if (per_thread <= 2)
-      ln_bwd_kernel<2, DY32><<<nb, LNB_THREADS, 0, stream>>>(dy, x, g, mean, rstd, dres, rows, D,
-                                                              rpb, dx, partial, dx32);
+      ln_bwd_kernel_launch<2, DY32>(rsum, nb, dy, x, g, mean, rstd, dres, rows, D, rpb, dx,
+                                    partial, dx32, stream);
     else if (per_thread <= 4)
-      ln_bwd_kernel<4, DY32><<<nb, LNB_THREADS, 0, stream>>>(dy, x, g, mean, rstd, dres, rows, D,
-                                                              rpb, dx, partial, dx32);
+      ln_bwd_kernel_launch<4, DY32>(rsum, nb, dy, x, g, mean, rstd, dres, rows, D, rpb, dx,
+                                    partial, dx32, stream);
     else
       return TP_ERR_UNSUPPORTED;
   }
-  if (dg != nullptr || db != nullptr) {
+  if (dg != nullptr || db != nullptr || dr != nullptr) {
     TraceScope ts(stream, TK_LN_PARAM);
-    ln_param_reduce<<<(2 * D + 31) / 32, 256, 0, stream>>>(partial, nb, D, dg, db);
+    const int nk = rsum ? 3 : 2;
+    ln_param_reduce<<<(nk * D + 31) / 32, 256, 0, stream>>>(partial, nb, D, nk, dg, db, dr);
   }
   return cuda_status(cudaGetLastError());
 }
@@ -502,9 +541,11 @@ tp_status ln_bwd_launch(const void* dy, const uint16_t* x, const uint16_t* g, co
 tp_status launch_layernorm_bwd(const uint16_t* dy, const uint16_t* x, const uint16_t* g,
                                const float* mean, const float* rstd, const uint16_t* dres,
                                long long rows, int D, uint16_t* dx, uint16_t* dg, uint16_t* db,
-                               float* partial, cudaStream_t stream, float* dx32) {
+                               float* partial, cudaStream_t stream, float* dx32,
+                               uint16_t* dres_sum) {
   return ln_bwd_launch<false>(dy, x, g, mean, rstd, dres, rows, D, dx, dx32, dg, db,
-                              layernorm_bwd_blocks(rows < 1 ? 1 : rows), partial, stream);
+                              layernorm_bwd_blocks(rows < 1 ? 1 : rows), partial, stream,
+                              dres_sum);
 }
 
 tp_status launch_layernorm_bwd_f32(const float* dy, const uint16_t* x, const uint16_t* g,

@@ -9,9 +9,9 @@ while the rest of the backward pass computes.
 The layer's backward finishes its parameter gradients in three groups, in
 this order (tp_layer_bwd_notify records one event per group; the
 one-shard-per-GPU driver calls back at the same points):
-  "mlp"   w1, b1, w2, b2                       (the MLP backward runs first)
-  "attn"  wqkv, bqkv, wout, bout, ln2_g, ln2_b
-  "ln1"   ln1_g, ln1_b
+  "mlp"   w1, b1, w2, b2, ln2_g, ln2_b   (the MLP backward and LN2's run first)
+  "attn"  wqkv, bqkv, wout
+  "ln1"   ln1_g, ln1_b, bout             (LN1's backward, last, also sums bout)
 ``GradBuckets`` lays each group's gradients out in one flat buffer, so one
 collective reduces a group; ``GradientAllReduce`` issues that collective on
 a side stream that first waits on the group's event, so the MLP gradients
@@ -32,9 +32,9 @@ import torch
 
 # Gradient groups of the pre-LN layer, in the order the backward completes them.
 LAYER_GROUPS = {
-    "mlp": ("w1", "b1", "w2", "b2"),
-    "attn": ("wqkv", "bqkv", "wout", "bout", "ln2_g", "ln2_b"),
-    "ln1": ("ln1_g", "ln1_b"),
+    "mlp": ("w1", "b1", "w2", "b2", "ln2_g", "ln2_b"),
+    "attn": ("wqkv", "bqkv", "wout"),
+    "ln1": ("ln1_g", "ln1_b", "bout"),
 }
 ALIGN = 128    # elements between views: every gradient starts 256-byte aligned
 

@@ -269,8 +269,10 @@ def layer_backward(ranks: Sequence[RankLayer], dy, exchange: Exchange, on_grads_
     """Backward; returns dx per rank (equal on every rank).  Each rank's
     parameter gradients land in ``rank.grads``.  ``on_grads_ready(group)``,
     if given, is called as soon as the kernels producing a group of gradients
-    are enqueued: "mlp" (w1, b1, w2, b2), "attn" (wqkv, bqkv, wout, bout, ln2),
-    "ln1" -- the points where a data-parallel reduction of them can start."""
+    are enqueued -- the points where a data-parallel reduction of them can
+    start: "mlp" after the MLP shard's backward (w1, b1, w2, b2), "attn" after
+    LN2's and the attention shard's (ln2, wqkv, bqkv, wout, bout), "ln1" at the
+    end.  Each call covers at least the groups of data_parallel.LAYER_GROUPS."""
     sources = exchange([r.bwd_mlp(dy) for r in ranks])          # MLP input-gradient all-reduce
     if on_grads_ready:
         on_grads_ready("mlp")
