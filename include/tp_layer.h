@@ -246,6 +246,10 @@ typedef struct {
   float *mean2, *rstd2;   /* [T] */
   tp_bf16* a;             /* MLP pre-activation [t][T][Ft] */
   tp_bf16* hact;          /* MLP activation [t][T][Ft] */
+  tp_f16* wqkv16;         /* optional (may be NULL): [t][D][3Dt] fp16 copy of params->wqkv.
+                             tp_layer_fwd writes it and tp_layer_bwd reads it instead of
+                             converting Wqkv again; the weights must not change between the
+                             two calls.  NULL: each call converts into its workspace. */
 } tp_layer_acts;
 
 /* Parameter gradients written by tp_layer_bwd (same layouts as the parameters;

@@ -69,7 +69,7 @@ class LayerParams(ctypes.Structure):
 
 class LayerActs(ctypes.Structure):
     _fields_ = [(n, _P) for n in ("u1", "mean1", "rstd1", "qkv", "o", "lse", "h", "u2",
-                                  "mean2", "rstd2", "a", "hact")]
+                                  "mean2", "rstd2", "a", "hact", "wqkv16")]
 
 
 class PostLNActs(ctypes.Structure):

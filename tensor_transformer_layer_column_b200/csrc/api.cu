@@ -670,7 +670,7 @@ static tp_status check_layer_ptrs(const tp_layer_params* p, const tp_layer_acts*
   if (!all_aligned(p->ln1_g, p->ln1_b, p->wqkv, p->bqkv, p->wout, p->bout, p->ln2_g, p->ln2_b,
                    p->w1, p->b1, p->w2, p->b2))
     return TP_ERR_MISALIGNED;
-  if (!all_aligned(a->u1, a->qkv, a->o, a->lse, a->h, a->u2, a->a, a->hact))
+  if (!all_aligned(a->u1, a->qkv, a->o, a->lse, a->h, a->u2, a->a, a->hact, a->wqkv16))
     return TP_ERR_MISALIGNED;
   return TP_OK;
 }
@@ -699,14 +699,15 @@ tp_status layer_fwd_core(const Sizes& z, const tp_dims* dims, const tp_bf16* x,
   return mlp_fwd_impl(z, a->u2, p->w1, p->b1, p->w2, p->b2, a->h, y, a->a, a->hact, cs);
 }
 
-// Pre-LN backward; `ws` is laid out as layer_bwd_ws describes and its first
-// slice already holds the fp16 copy of Wqkv.
 // Records `ev` (a caller's cudaEvent_t, may be NULL) on the stream.
 tp_status record_ready(void* ev, cudaStream_t cs) {
   if (ev == nullptr) return TP_OK;
   return cuda_status(cudaEventRecord(static_cast<cudaEvent_t>(ev), cs));
 }
 
+// Pre-LN backward; `ws` is laid out as layer_bwd_ws describes.  The fp16 copy
+// of Wqkv is the forward's (a->wqkv16) when the caller kept it, otherwise it
+// is made here in the workspace's first slice.
 tp_status layer_bwd_core(const Sizes& z, const tp_dims* dims, const tp_bf16* x,
                          const tp_layer_params* p, const tp_layer_acts* a, const tp_bf16* dy,
                          tp_bf16* dx, const tp_layer_grads* g, void* ws, cudaStream_t cs,
@@ -714,6 +715,11 @@ tp_status layer_bwd_core(const Sizes& z, const tp_dims* dims, const tp_bf16* x,
   tp_status st;
   Carver c(ws);
   uint16_t* w16 = c.take<uint16_t>((size_t)(z.D * 3 * z.D));
+  if (a->wqkv16 != nullptr) {
+    w16 = a->wqkv16;
+  } else if ((st = launch_cast_f16(p->wqkv, (size_t)(z.D * 3 * z.D), w16, cs)) != TP_OK) {
+    return st;
+  }
   uint16_t* du = c.take<uint16_t>((size_t)(z.T * z.D));
   uint16_t* dh = c.take<uint16_t>((size_t)(z.T * z.D));
   float* lnp = c.take<float>(layernorm_bwd_partial_floats(z.T, (int)z.D, 3));
@@ -790,7 +796,7 @@ tp_status tp_layer_fwd(const tp_dims* dims, const tp_bf16* x, const tp_layer_par
   cudaStream_t cs = (cudaStream_t)s;
   if (z.T == 0) return TP_OK;
   if ((st = check_ws(ws, ws_bytes, layer_fwd_ws(z))) != TP_OK) return st;
-  uint16_t* w16 = static_cast<uint16_t*>(ws);
+  uint16_t* w16 = a->wqkv16 != nullptr ? a->wqkv16 : static_cast<uint16_t*>(ws);
   if ((st = launch_cast_f16(p->wqkv, (size_t)(z.D * 3 * z.D), w16, cs)) != TP_OK) return st;
   return layer_fwd_core(z, dims, x, p, a, y, w16, cs);
 }
@@ -807,8 +813,6 @@ tp_status tp_layer_bwd(const tp_dims* dims, const tp_bf16* x, const tp_layer_par
   if ((st = check_ws(ws, ws_bytes, need)) != TP_OK) return st;
   cudaStream_t cs = (cudaStream_t)s;
   if (z.T == 0) return layer_bwd_empty(z, dims->causal, g, cs);
-  uint16_t* w16 = static_cast<uint16_t*>(ws);
-  if ((st = launch_cast_f16(p->wqkv, (size_t)(z.D * 3 * z.D), w16, cs)) != TP_OK) return st;
   return layer_bwd_core(z, dims, x, p, a, dy, dx, g, ws, cs);
 }
 
@@ -832,8 +836,6 @@ tp_status tp_layer_bwd_notify(const tp_dims* dims, const tp_bf16* x, const tp_la
     }
     return TP_OK;
   }
-  uint16_t* w16 = static_cast<uint16_t*>(ws);
-  if ((st = launch_cast_f16(p->wqkv, (size_t)(z.D * 3 * z.D), w16, cs)) != TP_OK) return st;
   return layer_bwd_core(z, dims, x, p, a, dy, dx, g, ws, cs, ready);
 }
 
@@ -875,7 +877,9 @@ tp_status tp_layer_bwd_recompute(const tp_dims* dims, const tp_bf16* x, const tp
   uint16_t* w16 = static_cast<uint16_t*>(bws);
   if ((st = launch_cast_f16(p->wqkv, (size_t)(z.D * 3 * z.D), w16, cs)) != TP_OK) return st;
   if ((st = layer_fwd_core(z, dims, x, p, &a, nullptr, w16, cs)) != TP_OK) return st;
-  return layer_bwd_core(z, dims, x, p, &a, dy, dx, g, bws, cs);
+  tp_layer_acts ar = a;
+  ar.wqkv16 = w16;   // the recomputed forward's copy serves the backward
+  return layer_bwd_core(z, dims, x, p, &ar, dy, dx, g, bws, cs);
 }
 
 // ------------------------------------------------------------------ post-LN layer

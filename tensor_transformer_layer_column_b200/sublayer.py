@@ -316,7 +316,9 @@ class ShardedLayer:
                 "lse": _empty((d.batch, d.heads, d.seq), f32, dev),
                 "h": _empty((T, D), device=dev), "u2": _empty((T, D), device=dev),
                 "mean2": _empty((T,), f32, dev), "rstd2": _empty((T,), f32, dev),
-                "a": _empty((t, T, F // t), device=dev), "hact": _empty((t, T, F // t), device=dev)}
+                "a": _empty((t, T, F // t), device=dev), "hact": _empty((t, T, F // t), device=dev),
+                # the forward's fp16 copy of Wqkv, reused by the backward
+                "wqkv16": _empty((t, D, 3 * D // t), f16, dev)}
 
     def alloc_grads(self, bias_grads=True, meta=False):
         d = self.dims

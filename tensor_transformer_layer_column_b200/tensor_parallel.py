@@ -237,15 +237,19 @@ class RankLayer:
         return self.ops.mlp_bwd(s["u2"], self.p["w1"], self.p["w2"], s["a"], s["hact"], dy,
                                 self.grads)
 
-    def bwd_attention(self, sources):
-        """du2 = the summed MLP input gradient; dh = dy + LN2^T(du2); the
-        attention shard's gradients (dbout replicated) and the partial dqkv_i Wqkv_i^T."""
+    def bwd_ln2(self, sources):
+        """du2 = the summed MLP input gradient; dh = dy + LN2^T(du2) (and LN2's
+        parameter gradients, replicated)."""
         p, s, g = self.p, self.s, self.grads
         du2 = self.ops.finish("du2", sources, None, None)
         s["dh"] = self.ops.layernorm_bwd("dh", du2, s["h"], p["ln2_g"], s["mean2"], s["rstd2"],
                                          s["dy"], g.get("ln2_g"), g.get("ln2_b"))
+
+    def bwd_attention(self):
+        """The attention shard's gradients (dbout replicated) and the partial dqkv_i Wqkv_i^T."""
+        p, s = self.p, self.s
         return self.ops.attn_bwd(s["u1"], p["wqkv"], p["wout"], s["qkv"], s["o"], s["lse"],
-                                 s["dh"], g)
+                                 s["dh"], self.grads)
 
     def bwd_input(self, sources):
         """du1 = the summed attention input gradient; dx = dh + LN1^T(du1)."""
@@ -270,13 +274,15 @@ def layer_backward(ranks: Sequence[RankLayer], dy, exchange: Exchange, on_grads_
     parameter gradients land in ``rank.grads``.  ``on_grads_ready(group)``,
     if given, is called as soon as the kernels producing a group of gradients
     are enqueued -- the points where a data-parallel reduction of them can
-    start: "mlp" after the MLP shard's backward (w1, b1, w2, b2), "attn" after
-    LN2's and the attention shard's (ln2, wqkv, bqkv, wout, bout), "ln1" at the
-    end.  Each call covers at least the groups of data_parallel.LAYER_GROUPS."""
+    start: "mlp" after the MLP shard's and LN2's backward (w1, b1, w2, b2, ln2),
+    "attn" after the attention shard's (wqkv, bqkv, wout, bout), "ln1" at the
+    end: the groups of data_parallel.LAYER_GROUPS, or earlier."""
     sources = exchange([r.bwd_mlp(dy) for r in ranks])          # MLP input-gradient all-reduce
+    for r in ranks:
+        r.bwd_ln2(sources)
     if on_grads_ready:
         on_grads_ready("mlp")
-    sources = exchange([r.bwd_attention(sources) for r in ranks])   # attention all-reduce
+    sources = exchange([r.bwd_attention() for r in ranks])      # attention all-reduce
     if on_grads_ready:
         on_grads_ready("attn")
     dx = [r.bwd_input(sources) for r in ranks]

@@ -142,3 +142,39 @@ def test_layer_zero_tokens(placement):
     assert_no_device_error()
     for k, v in grads.items():
         assert not v.float().abs().any(), k
+
+
+def test_layer_kept_fp16_wqkv_equals_converting_again():
+    """acts["wqkv16"] (the forward's fp16 copy of Wqkv, reused by the backward)
+    gives the same y, dx and gradients, bit for bit, as leaving it NULL."""
+    require_gpu()
+    w = Workload("layer_test", "layer_fwdbwd", batch=2, seq=96, hidden=512, ffn=1024, heads=4,
+                 head_dim=128, t=4)
+    inp = make_inputs(w, seed=19, random_affine=True)
+    g = dev(inp)
+    out = []
+    for keep in (True, False):
+        layer = ShardedLayer(dims_of(w), {k: g[k] for k in PARAMS})
+        acts = layer.alloc_acts()
+        if not keep:
+            acts["wqkv16"] = None
+        y, _ = layer.forward(g["x"], acts=acts) if keep else _forward_without_copy(layer, g, acts)
+        dx, grads = layer.backward(g["dy"])
+        torch.cuda.synchronize()
+        assert_no_device_error()
+        out.append((y.clone(), dx.clone(), {k: v.clone() for k, v in grads.items()}))
+    assert torch.equal(out[0][0], out[1][0]) and torch.equal(out[0][1], out[1][1])
+    for k in out[0][2]:
+        assert torch.equal(out[0][2][k], out[1][2][k]), k
+
+
+def _forward_without_copy(layer, g, acts):
+    """The layer forward through the binding with acts["wqkv16"] = NULL."""
+    import tensor_transformer_layer_column_b200 as tl
+    from tensor_transformer_layer_column_b200.sublayer import OP_LAYER_FWD, _ws
+    d = layer.dims
+    y = torch.empty_like(g["x"])
+    layer.ws_fwd = _ws(OP_LAYER_FWD, d, layer.device)
+    tl.layer_fwd(d, g["x"], layer.p, acts, y, layer.ws_fwd)
+    layer.saved = (g["x"], acts)
+    return y, acts
