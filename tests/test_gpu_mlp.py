@@ -139,20 +139,40 @@ def test_mlp_full_size_T8192_D3072_F12288_t8():
     _compare(w, o, grads, y, a, h, g)
 
 
+def c4_sample_rows_cols(T, F, t):
+    """Rows: every 16th token and the last row of every 128-row block (both
+    sides of every tile edge of the 128- and 256-row tiles).  FFN columns:
+    every 16th, plus the first and last column of every 256-wide tile of every
+    shard (the column tiles restart at each shard's boundary)."""
+    rows = set(range(0, T, 16)) | set(range(127, T, 128))
+    ft = F // t
+    cols = set(range(0, F, 16))
+    for i in range(t):
+        for n0 in range(0, ft, 256):
+            cols |= {i * ft + n0, i * ft + min(n0 + 255, ft - 1)}
+    return np.array(sorted(rows)), np.array(sorted(cols))
+
+
+def test_c4_sample_covers_every_tile_edge():
+    T, F, t = 8192, 28672, 8
+    R, J = c4_sample_rows_cols(T, F, t)
+    assert len(R) == 8192 // 16 + 64 and {0, 127, 128, 255, 256, T - 1} <= set(R)
+    ft = F // t
+    assert {0, 255, 256, ft - 1, ft, ft + 255, F - 1} <= set(J) and len(J) > F // 16
+
+
 def test_mlp_full_size_T8192_D7168_F28672_t8_sampled():
-    """The 30B FFN shape, checked on sampled rows (y, dx, saved activations) and
-    sampled ffn columns (dW1 columns, dW2 rows, db1): the MLP decomposes exactly
-    over rows of x and over columns of W1 / rows of W2, so the oracle computes
-    each sample from the same definition on a slice."""
+    """The 30B FFN shape, checked on ~600 rows (y, dx, saved activations) and
+    ~2000 ffn columns (dW1 columns, dW2 rows, db1) that include every tile edge:
+    the MLP decomposes exactly over rows of x and over columns of W1 / rows of
+    W2, so the oracle computes each sample from the same definition on a slice."""
     require_gpu()
     w = workload("mlp_fwdbwd_T8192_D7168_F28672_t8")
     inp = make_inputs(w)
     o, grads = _run(w, inp)
     T, D, F, t = w.tokens, w.hidden, w.ffn, w.t
     ft = F // t
-    rs = np.random.default_rng(0)
-    R = np.sort(rs.choice(T, 48, replace=False))
-    J = np.sort(rs.choice(F, 48, replace=False))
+    R, J = c4_sample_rows_cols(T, F, t)
     x, w1, b1, w2, b2, dy = (to_f64(inp[k]) for k in ("x", "w1", "b1", "w2", "b2", "dy"))
     y, a, h = omlp.mlp_fwd(x[R], w1, b1, w2, b2)
     check("y[rows]", f64(o["y"])[R], y)
