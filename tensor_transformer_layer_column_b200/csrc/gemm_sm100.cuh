@@ -13,7 +13,7 @@
 // 0..t-1, with a single rounding in the epilogue.  Weight-gradient products
 // shard M or N the same way.
 //
-// Two kernels, both persistent with 192 threads (6 warps) per CTA:
+// Two kernels, both persistent with 320 threads (10 warps) per CTA:
 //   gemm_pair_sm100 (M > 128): clusters of two CTAs on two SMs compute
 //     256 x 256 tiles with tcgen05.mma.cta_group::2 (M = 256 split across the
 //     pair).  Each CTA's producer stages its half of A and of B through a
@@ -23,9 +23,10 @@
 //   gemm_bf16_sm100 (M <= 128): one CTA per 128 x 256 tile, 4-stage ring,
 //     4 MMAs of 128 x 256 x 16 per k-block.
 // Roles in both: warp 0 TMA producer; warp 1 TMEM owner and MMA issuer (one
-// thread); warps 2..5 epilogue: tcgen05.ld of their 32-lane quarter, bias /
-// GeLU (writing A and H) / GeLU-backward / residual (bf16 or fp32), then the
-// stores.  The second accumulator lets the epilogue of tile i overlap the
+// thread); warps 2..9 epilogue, two per 32-lane quarter of tensor memory (a
+// warp may only read its own quarter), each taking half of the tile's
+// columns: tcgen05.ld, bias / GeLU (writing A and H) / GeLU-backward /
+// residual (bf16 or fp32), then the stores.  The second accumulator lets the epilogue of tile i overlap the
 // MMAs of tile i+1.  Tiles are visited in groups of 8 M-blocks per N sweep so
 // that concurrently running tiles share A and B panels in L2.
 // Every wait is bounded; a timeout records an error code and the kernel
@@ -44,7 +45,8 @@ constexpr int GEMM_BM = 128;
 constexpr int GEMM_BN = 256;
 constexpr int GEMM_BK = 64;        // one 128-byte swizzle row of bf16
 constexpr int GEMM_STAGES = 4;
-constexpr int GEMM_THREADS = 192;
+constexpr int GEMM_EPI_WARPS = 8;   // two per TMEM lane quarter, each draining half the columns
+constexpr int GEMM_THREADS = 64 + 32 * GEMM_EPI_WARPS;
 constexpr int GEMM_A_BYTES = GEMM_BM * GEMM_BK * 2;   // 16 KiB
 constexpr int GEMM_B_BYTES = GEMM_BN * GEMM_BK * 2;   // 32 KiB
 constexpr int GEMM_STAGE_BYTES = GEMM_A_BYTES + GEMM_B_BYTES;
@@ -300,7 +302,7 @@ gemm_bf16_sm100(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&tfull[i], 1);
-      mbar_init(&tempty[i], 128);
+      mbar_init(&tempty[i], 32 * GEMM_EPI_WARPS);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -414,6 +416,8 @@ gemm_bf16_sm100(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
     // ------------------------------------------------------------ epilogue
     const int quad = warp & 3;                 // TMEM lane quarter this warp may access
     const int row = quad * 32 + lane;          // row within the tile
+    constexpr int CPW = GEMM_BN / 32 / (GEMM_EPI_WARPS / 4);   // 32-column chunks per warp
+    const int c0 = ((warp - 2) / 4) * CPW;
     int tcount = 0;
     for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++tcount) {
       const TileCoord tc = gemm_tile(p, tile);
@@ -430,7 +434,7 @@ gemm_bf16_sm100(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
       const long long base = tc.ms * p.c_ms + tc.ns * p.c_ns + (long long)m * p.ldc;
       const uint32_t taddr = tmem_base + ((uint32_t)(quad * 32) << 16) + acc * GEMM_BN;
 #pragma unroll 1
-      for (int c = 0; c < GEMM_BN / 32; ++c) {
+      for (int c = c0; c < c0 + CPW; ++c) {
         uint32_t r[32];
         tmem_ld32(taddr + c * 32, r);
         tc_wait_ld();
@@ -522,7 +526,7 @@ gemm_pair_sm100(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&tfull[i], 1);
-      mbar_init(&tempty[i], 8);     // one arrival per epilogue warp of both CTAs
+      mbar_init(&tempty[i], 2 * GEMM_EPI_WARPS);   // one arrival per epilogue warp of both CTAs
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -637,6 +641,8 @@ gemm_pair_sm100(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
   } else {
     const int quad = warp & 3;
     const int row = quad * 32 + lane;
+    constexpr int CPW = GP_BN / 32 / (GEMM_EPI_WARPS / 4);     // 32-column chunks per warp
+    const int c0 = ((warp - 2) / 4) * CPW;
     const uint32_t tempty_leader0 = map_to_rank(&tempty[0], 0);
     int tcount = 0;
     for (int tile = cid; tile < p.num_tiles; tile += ncl, ++tcount) {
@@ -653,7 +659,7 @@ gemm_pair_sm100(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
       const long long base = tc.ms * p.c_ms + tc.ns * p.c_ns + (long long)m * p.ldc;
       const uint32_t taddr = tmem_base + ((uint32_t)(quad * 32) << 16) + acc * GP_BN;
 #pragma unroll 1
-      for (int c = 0; c < GP_BN / 32; ++c) {
+      for (int c = c0; c < c0 + CPW; ++c) {
         uint32_t r[32];
         tmem_ld32(taddr + c * 32, r);
         tc_wait_ld();
