@@ -165,10 +165,14 @@ tp_status mlp_fwd_impl(const Sizes& z, bf16p x, bf16p w1, bf16p b1, bf16p w2, bf
   return launch_gemm(g2, st);
 }
 
+// Column-sum partial rows of dA that the GeLU' product writes for db1: one per 32 rows.
+long long db1_groups(const Sizes& z) { return (z.T + 31) / 32; }
+
 size_t mlp_bwd_ws(const Sizes& z) {
   Carver c(nullptr);
   c.take<uint16_t>((size_t)(z.T * z.F));
-  c.take<float>(colsum_scratch_floats_max(z.T, {{z.t, z.Ft}, {1, z.D}}));
+  c.take<float>(colsum_scratch_floats_max(z.T, {{1, z.D}}));
+  c.take<float>((size_t)(db1_groups(z) * z.F));
   return align_up(c.off, 256);
 }
 
@@ -186,9 +190,11 @@ tp_status mlp_bwd_impl(const Sizes& z, bf16p x, bf16p w1, bf16p w2, bf16p a_save
   }
   Carver c(ws);
   uint16_t* da = c.take<uint16_t>((size_t)(z.T * z.F));
-  float* part = c.take<float>(colsum_scratch_floats_max(z.T, {{z.t, z.Ft}, {1, z.D}}));
+  float* part = c.take<float>(colsum_scratch_floats_max(z.T, {{1, z.D}}));
+  float* dapart = c.take<float>((size_t)(db1_groups(z) * z.F));
 
   // dA_i = (dY W2_i^T) * GeLU'(A_i): B = W2_i read as [n = Ft][k = D], K-major.
+  // db1 = column sums of dA: the epilogue writes one partial row per 32 rows.
   GemmProblem g4{};
   g4.m_shards = 1; g4.n_shards = (int)z.t; g4.Mt = (int)z.T; g4.Nt = (int)z.Ft;
   g4.k_shards = 1; g4.Kt = (int)z.D;
@@ -196,8 +202,10 @@ tp_status mlp_bwd_impl(const Sizes& z, bf16p x, bf16p w1, bf16p w2, bf16p a_save
   g4.b = op(w2, false, SHARD_MN, z.D, z.Ft, z.t, z.D, z.Ft * z.D);
   g4.epi = EPI_DGELU; g4.c = da; g4.aux = a_save;
   g4.c_ms = 0; g4.c_ns = z.T * z.Ft; g4.ldc = z.Ft;
+  if (db1) g4.colpart = dapart;
   tp_status s = launch_gemm(g4, st);
   if (s != TP_OK) return s;
+  if (db1 && (s = launch_colsum_reduce(dapart, db1_groups(z), z.F, db1, st)) != TP_OK) return s;
 
   // dW2_i = H_i^T dY: A = H_i^T (M-major), M shards.
   GemmProblem g5{};
@@ -231,7 +239,6 @@ tp_status mlp_bwd_impl(const Sizes& z, bf16p x, bf16p w1, bf16p w2, bf16p a_save
   g7.c_ms = 0; g7.c_ns = 0; g7.ldc = z.D;
   if ((s = launch_gemm(g7, st)) != TP_OK) return s;
 
-  if (db1 && (s = launch_colsum_stacked(da, z.t, z.T, z.Ft, db1, part, st)) != TP_OK) return s;
   if (db2 && (s = launch_colsum_stacked(dy, 1, z.T, z.D, db2, part, st)) != TP_OK) return s;
   return TP_OK;
 }

@@ -131,6 +131,7 @@ tp_status launch_gemm(const GemmProblem& g, cudaStream_t stream) {
   if (g.a.f16 != g.b.f16) return TP_ERR_INVALID_ARG;       // one MMA takes one operand type
   // fp32 residual / output: plain linear epilogue, no fp16 store.
   if ((g.out_f32 || g.aux_f32) && (g.epi != EPI_LINEAR || g.out_f16)) return TP_ERR_INVALID_ARG;
+  if (g.colpart != nullptr && g.m_shards != 1) return TP_ERR_INVALID_ARG;
   // Pairs of CTAs (256-row tiles) unless one 128-row block covers M.
   const bool pair = g.Mt > GEMM_BM;
   const bool a_il = interleave_ok(g.a), b_il = interleave_ok(g.b);
@@ -174,6 +175,8 @@ tp_status launch_gemm(const GemmProblem& g, cudaStream_t stream) {
   a.aux_f32 = g.aux_f32 ? 1 : 0;
   a.a_il = a_il ? 1 : 0;
   a.b_il = b_il ? 1 : 0;
+  a.colpart = g.colpart;
+  a.colpart_ld = (long long)g.n_shards * g.Nt;
   const int grid = (int)(tiles < sm_count() ? tiles : sm_count());
   const double flops = 2.0 * g.m_shards * (double)g.Mt * g.n_shards * (double)g.Nt * g.k_shards *
                        (double)g.Kt;

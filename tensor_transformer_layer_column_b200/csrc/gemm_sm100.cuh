@@ -91,6 +91,10 @@ struct GemmArgs {
   int out_f16;                     // C (and C2) stored as fp16 instead of bf16
   int out_f32;                     // C stored as fp32 (EPI_LINEAR only; `c` then points at floats)
   int aux_f32;                     // aux is an fp32 residual (EPI_LINEAR only)
+  // Column sums of C (its fp32 values, before rounding), one partial row per
+  // 32-row group: colpart[(m / 32) * colpart_ld + ns * Nt + n].  One M shard only.
+  float* colpart;
+  long long colpart_ld;
   unsigned int* err;
 };
 
@@ -222,6 +226,43 @@ __device__ __forceinline__ void epilogue_store32(const GemmArgs& p, float (&v)[3
         *reinterpret_cast<uint4*>(hp + g * 8) = o;
       }
     }
+  }
+}
+
+// Sum over the warp's 32 lanes of each of the 32 columns in v: a transposing
+// butterfly (at each of 5 stages a lane keeps one half of its columns, sends
+// the other half to its partner and adds what it receives), after which lane
+// l holds the sum of column l.  The order of the additions is fixed.
+__device__ __forceinline__ float warp_colsum32(float (&v)[32]) {
+#pragma unroll
+  for (int s = 16; s >= 1; s >>= 1) {
+    const bool upper = (threadIdx.x & s) != 0;
+#pragma unroll
+    for (int i = 0; i < s; ++i) {
+      const float send = upper ? v[i] : v[i + s];
+      const float keep = upper ? v[i + s] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, s);
+    }
+  }
+  return v[0];
+}
+
+// One 32-column chunk of an epilogue warp: the epilogue for rows inside the
+// tensor, then (when asked) the warp's column sums.  `group` is the 32-row
+// group of the warp's rows; rows past Mt contribute zero, and a group wholly
+// past Mt (the tail of the last tile) writes nothing: the partial buffer holds
+// ceil(Mt / 32) rows.
+__device__ __forceinline__ void epilogue_chunk(const GemmArgs& p, const uint32_t (&r)[32], int ns,
+                                               long long base, int n, bool row_ok, int group) {
+  float v[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = row_ok ? __uint_as_float(r[i]) : 0.f;
+  if (row_ok) epilogue_store32(p, v, ns, base, n);
+  if (p.colpart != nullptr) {
+    const float s = warp_colsum32(v);
+    const int col = n + (int)(threadIdx.x & 31);
+    if (col < p.Nt && group * 32 < p.Mt)
+      p.colpart[(long long)group * p.colpart_ld + (long long)ns * p.Nt + col] = s;
   }
 }
 
@@ -439,11 +480,8 @@ gemm_bf16_sm100(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
         tmem_ld32(taddr + c * 32, r);
         tc_wait_ld();
         const int n = tc.n0 + c * 32;
-        if (!row_ok || n >= p.Nt) continue;
-        float v[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-        epilogue_store32(p, v, tc.ns, base, n);
+        if (n >= p.Nt) continue;   // the same for every lane of the warp
+        epilogue_chunk(p, r, tc.ns, base, n, row_ok, (tc.m0 + quad * 32) / 32);
       }
       tc_fence_before();
       mbar_arrive(&tempty[acc]);
@@ -664,11 +702,8 @@ gemm_pair_sm100(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
         tmem_ld32(taddr + c * 32, r);
         tc_wait_ld();
         const int n = tc.n0 + c * 32;
-        if (!row_ok || n >= p.Nt) continue;
-        float v[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-        epilogue_store32(p, v, tc.ns, base, n);
+        if (n >= p.Nt) continue;   // the same for every lane of the warp
+        epilogue_chunk(p, r, tc.ns, base, n, row_ok, (tc.m0 + (int)rank * 128 + quad * 32) / 32);
       }
       tc_fence_before();
       __syncwarp();

@@ -37,6 +37,9 @@ struct GemmProblem {
   bool out_f16;              // store C / C2 as fp16
   bool out_f32;              // store C as fp32 (EPI_LINEAR only)
   bool aux_f32;              // aux is an fp32 residual (EPI_LINEAR only)
+  // When set (one M shard only): per 32-row group column sums of C, fp32
+  // [ceil(Mt / 32)][n_shards * Nt]; reduce them with launch_colsum_reduce.
+  float* colpart = nullptr;
 };
 
 tp_status launch_gemm(const GemmProblem& g, cudaStream_t stream);
@@ -58,6 +61,9 @@ size_t colsum_partial_floats(long long S, long long rows, long long cols);
 tp_status launch_colsum_stacked(const uint16_t* x, long long S, long long rows, long long cols,
                                 uint16_t* out, float* partial, cudaStream_t stream,
                                 bool in_f16 = false);
+// out[c] = bf16( sum over r of partial[r][c] ), r = 0..rows-1 in order.
+tp_status launch_colsum_reduce(const float* partial, long long rows, long long cols, uint16_t* out,
+                               cudaStream_t stream);
 
 tp_status launch_layernorm_fwd(const uint16_t* x, const uint16_t* g, const uint16_t* b,
                                long long rows, int D, float eps, uint16_t* y, float* mean,

@@ -502,6 +502,16 @@ tp_status launch_colsum_stacked(const uint16_t* x, long long S, long long rows, 
   return cuda_status(cudaGetLastError());
 }
 
+tp_status launch_colsum_reduce(const float* partial, long long rows, long long cols, uint16_t* out,
+                               cudaStream_t stream) {
+  if (out == nullptr || cols == 0) return TP_OK;
+  if (rows == 0) return cuda_status(cudaMemsetAsync(out, 0, (size_t)cols * 2, stream));
+  TraceScope ts(stream, TK_COLSUM);
+  const dim3 g2((unsigned)((cols + 31) / 32), 1, 1);
+  colsum_reduce_kernel<<<g2, 256, 0, stream>>>(partial, (int)rows, cols, out);
+  return cuda_status(cudaGetLastError());
+}
+
 template <bool F16OUT>
 tp_status ln_fwd_dispatch(const uint16_t* x, const uint16_t* g, const uint16_t* b, long long rows,
                           int D, float eps, uint16_t* y, float* mean, float* rstd,

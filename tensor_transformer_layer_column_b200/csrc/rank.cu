@@ -70,7 +70,8 @@ size_t colsum_floats(long long T, long long cols_a, long long cols_b) {
 size_t mlp_bwd_rank_ws(const RankSizes& z) {
   Carver c(nullptr);
   c.take<uint16_t>((size_t)(z.T * z.Ft));                 // dA_i
-  c.take<float>(colsum_floats(z.T, z.Ft, z.D));
+  c.take<float>(colsum_partial_floats(1, z.T, z.D));      // db2
+  c.take<float>((size_t)((z.T + 31) / 32 * z.Ft));        // db1_i: a partial row per 32 rows
   return align_up(c.off, 256);
 }
 
@@ -255,13 +256,18 @@ tp_status tp_mlp_bwd_rank(const tp_dims* dims, const tp_bf16* x, const tp_bf16* 
   if ((st = check_ws(ws, ws_bytes, mlp_bwd_rank_ws(z))) != TP_OK) return st;
   Carver c(ws);
   uint16_t* da = c.take<uint16_t>((size_t)(z.T * z.Ft));
-  float* part = c.take<float>(colsum_floats(z.T, z.Ft, z.D));
-  // dA_i = (dy W2_i^T) * GeLU'(A_i): W2_i [Ft][D] read as [n = Ft][k = D], K-major.
+  float* part = c.take<float>(colsum_partial_floats(1, z.T, z.D));
+  float* dapart = c.take<float>((size_t)((z.T + 31) / 32 * z.Ft));
+  // dA_i = (dy W2_i^T) * GeLU'(A_i): W2_i [Ft][D] read as [n = Ft][k = D], K-major;
+  // its epilogue also writes the column-sum partials of dA_i for db1_i.
   GemmProblem g4 = problem(z.T, z.Ft, z.D);
   g4.a = opnd(dy, false, z.D, z.T);
   g4.b = opnd(w2_i, false, z.D, z.Ft);
   g4.epi = EPI_DGELU; g4.c = da; g4.aux = a_i;
+  if (db1_i) g4.colpart = dapart;
   if ((st = launch_gemm(g4, cs)) != TP_OK) return st;
+  if (db1_i && (st = launch_colsum_reduce(dapart, (z.T + 31) / 32, z.Ft, db1_i, cs)) != TP_OK)
+    return st;
   // dW2_i = H_i^T dy.
   GemmProblem g5 = problem(z.Ft, z.D, z.T);
   g5.a = opnd(h_i, true, z.Ft, z.T);
@@ -280,7 +286,6 @@ tp_status tp_mlp_bwd_rank(const tp_dims* dims, const tp_bf16* x, const tp_bf16* 
   g7.b = opnd(w1_i, false, z.Ft, z.D);
   g7.c = partial; g7.out_f32 = true;
   if ((st = launch_gemm(g7, cs)) != TP_OK) return st;
-  if (db1_i && (st = launch_colsum_stacked(da, 1, z.T, z.Ft, db1_i, part, cs)) != TP_OK) return st;
   if (db2 && (st = launch_colsum_stacked(dy, 1, z.T, z.D, db2, part, cs)) != TP_OK) return st;
   return TP_OK;
 }
