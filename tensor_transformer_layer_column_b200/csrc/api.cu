@@ -275,13 +275,15 @@ tp_status attn_fwd_impl(const Sizes& z, int causal, bf16p x16, bf16p wqkv16, bf1
   return launch_gemm(g2, st);
 }
 
-// Workspace of attn_bwd_impl: dO (fp16), dqkv (fp16), attention scratch, colsum partials.
+// Workspace of attn_bwd_impl: dO (fp16), dqkv (fp16), attention scratch, colsum
+// partials of dy (dbout) and the dqkv column partials the attention kernels write (dbqkv).
 size_t attn_bwd_core_ws(const Sizes& z) {
   Carver c(nullptr);
   c.take<uint16_t>((size_t)(z.T * z.D));
   c.take<uint16_t>((size_t)(z.T * 3 * z.D));
   c.take<uint8_t>(attn_bwd_scratch_bytes((int)z.B, (int)z.S, (int)z.H, (int)z.dh));
-  c.take<float>(colsum_scratch_floats_max(z.T, {{z.t, 3 * z.Dt}, {1, z.D}}));
+  c.take<float>(colsum_scratch_floats_max(z.T, {{1, z.D}}));
+  c.take<float>((size_t)(attn_colpart_rows(z.B, z.S) * 3 * z.D));
   return align_up(c.off, 256);
 }
 
@@ -301,7 +303,8 @@ tp_status attn_bwd_impl(const Sizes& z, int causal, bf16p x16, bf16p wqkv16, bf1
   uint16_t* dout = c.take<uint16_t>((size_t)(z.T * z.D));
   uint16_t* dqkv = c.take<uint16_t>((size_t)(z.T * 3 * z.D));
   void* scratch = c.take<uint8_t>(attn_bwd_scratch_bytes((int)z.B, (int)z.S, (int)z.H, (int)z.dh));
-  float* part = c.take<float>(colsum_scratch_floats_max(z.T, {{z.t, w3}, {1, z.D}}));
+  float* part = c.take<float>(colsum_scratch_floats_max(z.T, {{1, z.D}}));
+  float* qkvpart = c.take<float>((size_t)(attn_colpart_rows(z.B, z.S) * 3 * z.D));
 
   // dO_i = dY Wout_i^T: B = Wout_i read as [n = Dt][k = D], K-major, N shards; fp16 out.
   GemmProblem g1{};
@@ -324,9 +327,13 @@ tp_status attn_bwd_impl(const Sizes& z, int causal, bf16p x16, bf16p wqkv16, bf1
   g2.c_ms = z.Dt * z.D; g2.c_ns = 0; g2.ldc = z.D;
   if ((s = launch_gemm(g2, st)) != TP_OK) return s;
 
+  // dbqkv = column sums of dqkv: the attention kernels' epilogues write partials.
   s = launch_attn_bwd(qkv, o, lse, dout, dqkv, (int)z.B, (int)z.S, (int)z.H, (int)z.dh, (int)z.t,
-                      causal, scratch, st);
+                      causal, scratch, st, dbqkv ? qkvpart : nullptr);
   if (s != TP_OK) return s;
+  if (dbqkv && (s = launch_colsum_reduce(qkvpart, attn_colpart_rows(z.B, z.S), 3 * z.D, dbqkv,
+                                         st)) != TP_OK)
+    return s;
 
   // dWqkv_i = x^T dqkv_i, N shards (fp16 operands).
   GemmProblem g3{};
@@ -349,8 +356,6 @@ tp_status attn_bwd_impl(const Sizes& z, int causal, bf16p x16, bf16p wqkv16, bf1
   g4.c_ms = 0; g4.c_ns = 0; g4.ldc = z.D;
   if ((s = launch_gemm(g4, st)) != TP_OK) return s;
 
-  if (dbqkv && (s = launch_colsum_stacked(dqkv, z.t, z.T, w3, dbqkv, part, st, true)) != TP_OK)
-    return s;
   if (dbout && (s = launch_colsum_stacked(dy, 1, z.T, z.D, dbout, part, st)) != TP_OK) return s;
   return TP_OK;
 }

@@ -73,8 +73,39 @@ struct AttnArgs {
   float* lse;           // fwd: lse [B][H][S]
   const float* lse2;    // bwd: lse * log2(e), [B][H][S_pad]; +inf past S
   const float* dvec;    // bwd: rowsum(dO * O), [B][H][S_pad]; 0 past S
+  // bwd (may be null): column sums of dqkv for its bias gradient, one fp32
+  // partial row per 32 rows of one batch element: colpart[(b * G + s / 32) *
+  // (t * 3Dt) + shard * 3Dt + column], G = ceil(S / 32).
+  float* colpart;
   unsigned int* err;
 };
+
+// Sum over the warp's 32 lanes of each of the 32 columns in v (a transposing
+// butterfly; lane l ends with column l).  The order of additions is fixed.
+__device__ __forceinline__ float warp_colsum32(float (&v)[32]) {
+#pragma unroll
+  for (int s = 16; s >= 1; s >>= 1) {
+    const bool upper = (threadIdx.x & s) != 0;
+#pragma unroll
+    for (int i = 0; i < s; ++i) {
+      const float send = upper ? v[i] : v[i + s];
+      const float keep = upper ? v[i + s] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, s);
+    }
+  }
+  return v[0];
+}
+
+// Writes the warp's column sums of 32 columns starting at shard column `col0`
+// (rows of the warp: s0 .. s0 + 31 of batch element b; rows past S hold 0).
+__device__ __forceinline__ void colpart_store(const AttnArgs& p, float (&v)[32], int b, int s0,
+                                              int shard, int col0) {
+  const float sum = warp_colsum32(v);
+  const long long w3 = 3LL * p.Dt;
+  const long long slot = (long long)b * ((p.S + 31) / 32) + s0 / 32;
+  if (s0 < p.S)
+    p.colpart[slot * (p.t * w3) + shard * w3 + col0 + (threadIdx.x & 31)] = sum;
+}
 
 struct Ctl {
   volatile int* abort_flag;
@@ -728,21 +759,27 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_kv128,
         tmem_ld32(t_dv + lane_off + c * 32, rv);
         tmem_ld32(t_dk + lane_off + c * 32, rk);
         tc_wait_ld();
+        float v[32], kx[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          v[e] = valid ? __uint_as_float(rv[e]) : 0.f;
+          kx[e] = valid ? __uint_as_float(rk[e]) * p.inv_sqrt_dh : 0.f;
+        }
         if (valid) {
-          float v[32], kx[32];
           bool over = false;
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            v[e] = __uint_as_float(rv[e]);
-            kx[e] = __uint_as_float(rk[e]) * p.inv_sqrt_dh;
-            over |= fabsf(v[e]) > 65504.0f || fabsf(kx[e]) > 65504.0f;
-          }
+          for (int e = 0; e < 32; ++e) over |= fabsf(v[e]) > 65504.0f || fabsf(kx[e]) > 65504.0f;
 #pragma unroll
           for (int g = 0; g < 4; ++g) {
             *reinterpret_cast<uint4*>(row + colv + c * 32 + g * 8) = pack8_f16(&v[g * 8]);
             *reinterpret_cast<uint4*>(row + colk + c * 32 + g * 8) = pack8_f16(&kx[g * 8]);
           }
           if (over && p.err) atomicCAS(p.err, 0u, 0x301u);
+        }
+        if (p.colpart != nullptr) {
+          const int s0 = k0 + quad * 32;
+          colpart_store(p, v, b, s0, shard, colv + c * 32);
+          colpart_store(p, kx, b, s0, shard, colk + c * 32);
         }
       }
     }
@@ -971,19 +1008,19 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q128,
         uint32_t rq[32];
         tmem_ld32(t_dq + lane_off + c * 32, rq);
         tc_wait_ld();
+        float v[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) v[e] = qvalid ? __uint_as_float(rq[e]) * p.inv_sqrt_dh : 0.f;
         if (qvalid) {
-          float v[32];
           bool over = false;
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            v[e] = __uint_as_float(rq[e]) * p.inv_sqrt_dh;
-            over |= fabsf(v[e]) > 65504.0f;
-          }
+          for (int e = 0; e < 32; ++e) over |= fabsf(v[e]) > 65504.0f;
 #pragma unroll
           for (int g = 0; g < 4; ++g)
             *reinterpret_cast<uint4*>(row + c * 32 + g * 8) = pack8_f16(&v[g * 8]);
           if (over && p.err) atomicCAS(p.err, 0u, 0x301u);
         }
+        if (p.colpart != nullptr) colpart_store(p, v, b, q0 + quad * 32, shard, colq + c * 32);
       }
     }
   }
@@ -1147,9 +1184,10 @@ size_t attn_bwd_scratch_bytes(int B, int S, int H, int dh) {
 
 tp_status launch_attn_bwd(const uint16_t* qkv, const uint16_t* o, const float* lse,
                           const uint16_t* dout, uint16_t* dqkv, int B, int S, int H, int dh, int t,
-                          int causal, void* scratch, cudaStream_t stream) {
+                          int causal, void* scratch, cudaStream_t stream, float* colpart) {
   if ((long long)B * S == 0) return TP_OK;
-  const AttnArgs a = make_args(B, S, H, dh, t, causal);
+  AttnArgs a = make_args(B, S, H, dh, t, causal);
+  a.colpart = colpart;
   if (dh == 64) return bwd_launch<64>(qkv, o, lse, dout, dqkv, a, scratch, stream);
   if (dh == 128) return bwd_launch<128>(qkv, o, lse, dout, dqkv, a, scratch, stream);
   return TP_ERR_UNSUPPORTED;

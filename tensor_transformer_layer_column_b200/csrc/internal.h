@@ -97,9 +97,13 @@ tp_status launch_layernorm_bwd_blocks(const uint16_t* dy, const uint16_t* x, con
 tp_status launch_attn_fwd(const uint16_t* qkv, uint16_t* o, float* lse, int B, int S, int H,
                           int dh, int t, int causal, cudaStream_t stream);
 size_t attn_bwd_scratch_bytes(int B, int S, int H, int dh);
+// colpart (may be null): column sums of dqkv, fp32 [B * ceil(S / 32)][t * 3Dt] (one
+// partial row per 32 rows of a batch element), for launch_colsum_reduce.
 tp_status launch_attn_bwd(const uint16_t* qkv, const uint16_t* o, const float* lse,
                           const uint16_t* dout, uint16_t* dqkv, int B, int S, int H, int dh, int t,
-                          int causal, void* scratch, cudaStream_t stream);
+                          int causal, void* scratch, cudaStream_t stream,
+                          float* colpart = nullptr);
+inline long long attn_colpart_rows(long long B, long long S) { return B * ((S + 31) / 32); }
 
 tp_status launch_shard_cols(const uint16_t* src, int rows, int cols, int t, uint16_t* dst,
                             bool inverse, cudaStream_t stream);

@@ -62,11 +62,6 @@ RankSizes rank_sizes(const tp_dims& d) {
   return z;
 }
 
-size_t colsum_floats(long long T, long long cols_a, long long cols_b) {
-  const size_t a = colsum_partial_floats(1, T, cols_a), b = colsum_partial_floats(1, T, cols_b);
-  return a > b ? a : b;
-}
-
 size_t mlp_bwd_rank_ws(const RankSizes& z) {
   Carver c(nullptr);
   c.take<uint16_t>((size_t)(z.T * z.Ft));                 // dA_i
@@ -90,7 +85,8 @@ size_t attn_bwd_rank_ws(const RankSizes& z) {
   c.take<uint16_t>((size_t)(z.T * z.Dt));                 // dO_i (fp16)
   c.take<uint16_t>((size_t)(z.T * 3 * z.Dt));             // dqkv_i (fp16)
   c.take<uint8_t>(attn_bwd_scratch_bytes((int)z.B, (int)z.S, (int)z.Hl, (int)z.dh));
-  c.take<float>(colsum_floats(z.T, 3 * z.Dt, z.D));
+  c.take<float>(colsum_partial_floats(1, z.T, z.D));                  // dbout
+  c.take<float>((size_t)(attn_colpart_rows(z.B, z.S) * 3 * z.Dt));    // dbqkv_i
   return align_up(c.off, 256);
 }
 
@@ -380,7 +376,8 @@ tp_status tp_attn_bwd_rank(const tp_dims* dims, const tp_bf16* x, const tp_f16* 
   uint16_t* dout = c.take<uint16_t>((size_t)(z.T * z.Dt));
   uint16_t* dqkv = c.take<uint16_t>((size_t)(z.T * w3));
   void* scratch = c.take<uint8_t>(attn_bwd_scratch_bytes((int)z.B, (int)z.S, (int)z.Hl, (int)z.dh));
-  float* part = c.take<float>(colsum_floats(z.T, w3, z.D));
+  float* part = c.take<float>(colsum_partial_floats(1, z.T, z.D));
+  float* qkvpart = c.take<float>((size_t)(attn_colpart_rows(z.B, z.S) * w3));
   // dO_i = dy Wout_i^T (fp16): Wout_i [Dt][D] read as [n = Dt][k = D].
   GemmProblem g1 = problem(z.T, z.Dt, z.D);
   g1.a = opnd(dy, false, z.D, z.T);
@@ -394,7 +391,11 @@ tp_status tp_attn_bwd_rank(const tp_dims* dims, const tp_bf16* x, const tp_f16* 
   g2.c = dwout_i;
   if ((st = launch_gemm(g2, cs)) != TP_OK) return st;
   if ((st = launch_attn_bwd(qkv_i, o_i, lse_i, dout, dqkv, (int)z.B, (int)z.S, (int)z.Hl,
-                            (int)z.dh, 1, dims->causal, scratch, cs)) != TP_OK)
+                            (int)z.dh, 1, dims->causal, scratch, cs,
+                            dbqkv_i ? qkvpart : nullptr)) != TP_OK)
+    return st;
+  if (dbqkv_i && (st = launch_colsum_reduce(qkvpart, attn_colpart_rows(z.B, z.S), w3, dbqkv_i,
+                                            cs)) != TP_OK)
     return st;
   // dWqkv_i = x^T dqkv_i (fp16 operands).
   GemmProblem g3 = problem(z.D, w3, z.T);
@@ -408,8 +409,6 @@ tp_status tp_attn_bwd_rank(const tp_dims* dims, const tp_bf16* x, const tp_f16* 
   g4.b = opnd(w16, false, w3, z.D, true);
   g4.c = partial; g4.out_f32 = true;
   if ((st = launch_gemm(g4, cs)) != TP_OK) return st;
-  if (dbqkv_i && (st = launch_colsum_stacked(dqkv, 1, z.T, w3, dbqkv_i, part, cs, true)) != TP_OK)
-    return st;
   if (dbout && (st = launch_colsum_stacked(dy, 1, z.T, z.D, dbout, part, cs)) != TP_OK) return st;
   return TP_OK;
 }
