@@ -320,10 +320,13 @@ def hbm_bytes_per_step(w: Workload) -> dict:
         "ln_fwd": 2 * (4 * T * D + 8 * T),
         # LN2, LN1 backward: read du, the LN input and the residual gradient, write dx
         "ln_bwd": 2 * (8 * T * D + 8 * T),
-        # bias gradients: read dA, dqkv, dy and dh once
-        "colsum": 2 * T * F + 2 * T * 3 * D + 2 * T * D + 2 * T * D,
-        # Wqkv to fp16, forward and backward: read bf16, write fp16
-        "cast": 2 * (4 * D * 3 * D),
+        # bias gradients db1 and dbqkv: the fp32 column partials that the GeLU'
+        # product and the attention backward write (one row per 32 rows), read
+        # once, and the bf16 sums written (db2 and dbout come from the LayerNorm
+        # backwards)
+        "colsum": 4 * (T // 32) * F + 4 * w.batch * ((w.seq + 31) // 32) * 3 * D + 2 * (F + 3 * D),
+        # Wqkv to fp16 once per step (the backward reuses the forward's copy)
+        "cast": 4 * D * 3 * D,
         # Dv and lse2: read O and dO, read lse, write both padded rows
         "attn_bwd_prep": 4 * T * D + 4 * BHS + 8 * BHS_pad,
     }

@@ -40,8 +40,9 @@ def test_hbm_bytes_of_the_layer_step():
     T, D, F = w.tokens, w.hidden, w.ffn
     assert b["ln_fwd"] == 2 * 4 * T * D + 16 * T                # 2 x (64 MiB in + 64 MiB out) + stats
     assert b["ln_bwd"] == 16 * T * D + 16 * T                   # 2 x (3 reads + 1 write of [T][D])
-    assert b["colsum"] == 2 * T * (F + 5 * D)                   # dA, dqkv (3D), dy, dh
-    assert b["cast"] == 24 * D * D                              # Wqkv read + written, twice
+    # db1 / dbqkv partial rows (one per 32 rows, fp32) read, the sums written
+    assert b["colsum"] == 4 * (T // 32) * (F + 3 * D) + 2 * (F + 3 * D)
+    assert b["cast"] == 12 * D * D                              # Wqkv read + written, once
     assert abs(b["ln_bwd"] / 2**20 - 512.125) < 1e-9            # 512 MiB of rows + 128 KiB of stats
     assert bench.hbm_bytes_per_step(workload("mlp_fwdbwd_T8192_D3072_F12288_t8")) == {}
 
