@@ -13,11 +13,13 @@
 // 6e-3 at S = 2048, with fp16 near 2e-3.  The tensor-core rate is the same.
 //
 // Forward (per pair of 128-query tiles, head, batch; 64-key blocks):
-//   S = q k^T (tcgen05, fp32 in TMEM), online softmax in fp32 by one thread per
-//   query row (base-2 exponent, scores pre-scaled by log2(e)/sqrt(dh)), P
-//   rounded to fp16 into tensor memory, O += P v (tcgen05 with P as the
-//   A operand read from tensor memory, fp32 in TMEM, rescaled lazily).  The
-//   two tiles alternate on the tensor core.
+//   q is copied once into tensor memory and is the A operand of S = q k^T
+//   (tcgen05, fp32 in TMEM), so the score products read only k from shared
+//   memory; online softmax in fp32 by one thread per query row (base-2
+//   exponent, scores scaled by log2(e)/sqrt(dh) inside the exponent), P
+//   rounded to fp16 and written into tensor memory over the scores it came
+//   from, O += P v (tcgen05 with P as the A operand read from tensor memory,
+//   fp32 in TMEM, rescaled lazily).  The two tiles alternate on the tensor core.
 //   Writes O [t][T][Dt] (bf16) and the log-sum-exp [B][H][S] (fp32).
 // Backward (P recomputed from the log-sum-exp; no atomics, deterministic;
 // dO in and dqkv out are fp16):
@@ -160,10 +162,14 @@ __device__ __forceinline__ uint64_t mnmajor_desc(uint32_t base, int R, int kk) {
 // =====================================================================================
 // Two 128-query tiles per CTA take turns on the tensor core: while one tile's
 // softmax warpgroup works on its scores, the other tile's products run.  Keys
-// come in 64-wide blocks through a 4-stage ring; each tile has its own S (64
-// TMEM columns), P (32 columns of fp16 pairs) and O (dh columns).  O is rescaled lazily: only when a row's
-// running max grows by more than 2^8 (log2 units), so P = 2^(s - m_used) stays
-// below 256 (exact in fp16) and the final O / l is unchanged.
+// come in 64-wide blocks through a 4-stage ring.  Tensor memory per tile: q
+// (dh/2 columns of fp16 pairs, written once by the tile's softmax warps), S
+// (64 columns; P, 32 columns of fp16 pairs, is written over its first half)
+// and O (dh columns).  Because P lives in S's columns, the scores of block
+// j+1 wait for the P v product of block j; the other tile fills the tensor
+// core meanwhile.  O is rescaled lazily: only when a row's running max grows
+// by more than 2^8 (log2 units), so P = 2^(s - m_used) stays below 256 (exact
+// in fp16) and the final O / l is unchanged.
 template <int DH>
 struct FwdCfg {
   static constexpr int BM = 128, BN = 64, CH = DH / 64, STAGES = 4;
@@ -194,7 +200,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q128,
   uint64_t* kv_full = bars + 1;     // [STAGES <= 4]
   uint64_t* kv_empty = bars + 5;    // [STAGES]
   uint64_t* s_full = bars + 9;      // [2] per tile
-  uint64_t* s_free = bars + 11;     // [2]
+  uint64_t* q_tmem = bars + 11;     // [2] the tile's q is in tensor memory
   uint64_t* p_full = bars + 13;     // [2]
   uint64_t* pv_done = bars + 15;    // [2]
   uint64_t* drain = bars + 17;
@@ -226,7 +232,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q128,
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&s_free[i], 128);
+      mbar_init(&q_tmem[i], 128);
       mbar_init(&p_full[i], 128);
       mbar_init(&pv_done[i], 1);
     }
@@ -243,7 +249,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q128,
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  // TMEM columns: S of tile i at 64i, O of tile i at 128 + 128i, P of tile i at 384 + 32i.
+  // TMEM columns: S (then P) of tile i at 64i, O of tile i at 128 + 128i, q of tile i at
+  // 384 + 64i (dh/2 columns).
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
@@ -272,14 +279,12 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q128,
     }
   } else if (warp == 1 || warp == 10) {
     // Two issuers, each blocking only on its own barriers: warp 1 issues the
-    // scores S = q k^T of both tiles (block j+1 once the tile's softmax has
-    // copied S of block j out of tensor memory), warp 10 the products P V
-    // (once P is in tensor memory) and releases each K/V stage.  Neither
-    // stream waits behind the other.
+    // scores S = q k^T of both tiles (block j+1 once the tile's P v of block j
+    // has read P out of S's columns), warp 10 the products P V (once P is in
+    // tensor memory) and releases each K/V stage.
     if (lane == 0) {
       constexpr uint32_t id_s = idesc_f32acc(128, C::BN, false, false, true);
       constexpr uint32_t id_pv = idesc_f32acc(128, DH, false, true, true);
-      const uint32_t sq = smem_u32(smem + C::OFF_Q);
       auto kv_addr = [&](int j) { return smem_u32(smem + C::OFF_KV + (j % C::STAGES) * 2 * C::KV_BYTES); };
       bool ok = wait_bar(q_full, 0, ctl, ERR_ATTN_FWD_WAIT);
       if (warp == 1) {
@@ -288,7 +293,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q128,
 #pragma unroll
           for (int i = 0; i < 2; ++i) {
             if (ok && j < ntile[i]) {
-              if (j > 0 && !(ok = wait_bar(&s_free[i], (j - 1) & 1, ctl, ERR_ATTN_FWD_WAIT))) break;
+              if (j == 0 && !(ok = wait_bar(&q_tmem[i], 0, ctl, ERR_ATTN_FWD_WAIT))) break;
+              if (j > 0 && !(ok = wait_bar(&pv_done[i], (j - 1) & 1, ctl, ERR_ATTN_FWD_WAIT))) break;
               if (!kv_in && !(ok = wait_bar(&kv_full[j % C::STAGES], (j / C::STAGES) & 1, ctl,
                                             ERR_ATTN_FWD_WAIT)))
                 break;
@@ -296,9 +302,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q128,
               tc_fence_after();
               const uint32_t sk = kv_addr(j);
 #pragma unroll
-              for (int kk = 0; kk < DH / 16; ++kk)
-                tc_mma_f16(tmem + 64 * i, kmajor_desc(sq + i * C::Q_BYTES, C::BM, kk),
-                           kmajor_desc(sk, C::BN, kk), id_s, kk > 0);
+              for (int kk = 0; kk < DH / 16; ++kk)   // 16 of dh = 8 columns of q per step
+                tc_mma_f16_ts(tmem + 64 * i, tmem + 384 + 64 * i + 8 * kk,
+                              kmajor_desc(sk, C::BN, kk), id_s, kk > 0);
               tc_commit(&s_full[i]);
             }
           }
@@ -313,7 +319,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q128,
               const uint32_t sv = kv_addr(j) + C::KV_BYTES;
 #pragma unroll
               for (int kk = 0; kk < C::BN / 16; ++kk)   // 16 keys = 8 columns of P per step
-                tc_mma_f16_ts(tmem + 128 + 128 * i, tmem + 384 + 32 * i + 8 * kk,
+                tc_mma_f16_ts(tmem + 128 + 128 * i, tmem + 64 * i + 8 * kk,
                               mnmajor_desc(sv, C::BN, kk), id_pv, (j | kk) != 0);
               tc_commit(&pv_done[i]);
             }
@@ -338,10 +344,32 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q128,
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
     const uint32_t t_s = tmem + 64 * tile + lane_off;
     const uint32_t t_o = tmem + 128 + 128 * tile + lane_off;
-    const uint32_t t_p = tmem + 384 + 32 * tile + lane_off;
+    const uint32_t t_q = tmem + 384 + 64 * tile + lane_off;
     float m_used = -1e30f, l = 0.f;
     bool ok = true;
-    for (int j = 0; j < n; ++j) {
+    // q of this row into tensor memory, once: dh fp16 values as dh/2 pairs,
+    // read from the tile's 128-byte-swizzled shared-memory copy (16-byte unit u
+    // of row r of a 64-wide chunk sits at unit u ^ (r % 8)).
+    if (__all_sync(0xffffffffu, wait_bar(q_full, 0, ctl, ERR_ATTN_FWD_WAIT))) {
+      const uint8_t* qrow = smem + C::OFF_Q + tile * C::Q_BYTES + r * 128;
+#pragma unroll
+      for (int h = 0; h < DH / 64; ++h) {
+        uint32_t w[32];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const uint4 v = *reinterpret_cast<const uint4*>(qrow + h * C::BM * 128 +
+                                                          ((u ^ (r & 7)) << 4));
+          w[4 * u] = v.x; w[4 * u + 1] = v.y; w[4 * u + 2] = v.z; w[4 * u + 3] = v.w;
+        }
+        tmem_st32(t_q + 32 * h, w);
+      }
+      tc_wait_st();
+      tc_fence_before();
+      mbar_arrive(&q_tmem[tile]);
+    } else {
+      ok = false;
+    }
+    for (int j = 0; ok && j < n; ++j) {
       if (!__all_sync(0xffffffffu, wait_bar(&s_full[tile], j & 1, ctl, ERR_ATTN_FWD_WAIT))) { ok = false; break; }
       tc_fence_after();
       float s[C::BN];
@@ -356,8 +384,6 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q128,
           s[32 + e] = __uint_as_float(rb[e]);
         }
       }
-      tc_fence_before();
-      mbar_arrive(&s_free[tile]);
       // Keys past the last visible one (after the query, or past S) are masked: a select
       // per element against a bound fixed once per block, taken only in blocks where
       // some row of the warp has a masked key (the causal diagonal, the sequence end).
@@ -412,10 +438,11 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q128,
         }
       }
       {
+        // P over the first half of this block's S columns (already in registers).
         uint32_t pk[C::BN / 2];
 #pragma unroll
         for (int g = 0; g < C::BN / 2; ++g) pk[g] = pack_f16x2(s[2 * g], s[2 * g + 1]);
-        tmem_st32(t_p, pk);
+        tmem_st32(t_s, pk);
         tc_wait_st();
       }
       tc_fence_before();
