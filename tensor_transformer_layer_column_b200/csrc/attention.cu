@@ -820,9 +820,13 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_kv128,
 }
 
 // ---------------------------------------------------------------- dQ
-// Per 128-query block, walk 64-key blocks through a 4-stage K/V ring.  Two
-// S/dP buffers in TMEM, one per compute warpgroup; dS (fp16 pairs) goes to
-// its own TMEM columns and is the A operand of dQ += dS k.
+// Per 128-query block, walk 64-key blocks through a 4-stage K/V ring.  q and
+// dO (fixed per block) are copied once into tensor memory and are the A
+// operands of S = q k^T and dP = dO v^T, so those products read only k and v
+// from shared memory.  Two S/dP buffers in TMEM, one per compute warpgroup;
+// dS (fp16 pairs) is written over the first half of its S columns and is the
+// A operand of dQ += dS k, so the next scores into a buffer wait for the dQ
+// product that reads it.
 template <int DH>
 struct DqCfg {
   static constexpr int BQ = 128, BK = 64, CH = DH / 64;
@@ -851,7 +855,7 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q128,
   uint64_t* kv_full = bars + 1;    // [STAGES <= 4] per stage
   uint64_t* kv_empty = bars + 5;   // [STAGES]
   uint64_t* s_full = bars + 9;     // [2] per TMEM buffer
-  uint64_t* s_free = bars + 11;    // [2]
+  uint64_t* qd_tmem = bars + 11;   // [1] q and dO are in tensor memory
   uint64_t* p_full = bars + 13;    // [2] per dS buffer
   uint64_t* mm2_done = bars + 15;  // [2]
   uint64_t* drain = bars + 17;
@@ -877,10 +881,10 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q128,
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&s_free[i], 128);   // buffer i belongs to compute warpgroup i
-      mbar_init(&p_full[i], 128);
+      mbar_init(&p_full[i], 128);   // buffer i belongs to compute warpgroup i
       mbar_init(&mm2_done[i], 1);
     }
+    mbar_init(qd_tmem, 256);        // both compute warpgroups
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -893,8 +897,9 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q128,
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  // TMEM columns: buffer j holds S at 128j, dP at 128j + 64 and dS (fp16 pairs)
-  // at 384 + 32j; dQ accumulates at 256.
+  // TMEM columns: buffer j holds S (then dS, fp16 pairs, over its first half)
+  // at 128j and dP at 128j + 64; dQ accumulates at 256; q at 384 and dO at
+  // 448 (dh/2 columns each).
   const uint32_t t_dq = tmem + 256;
 
   if (warp == 0) {
@@ -927,22 +932,24 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q128,
     if (lane == 0) {
       constexpr uint32_t id_s = idesc_f32acc(128, C::BK, false, false, true);
       constexpr uint32_t id_acc = idesc_f32acc(128, DH, false, true, true);
-      const uint32_t sq = smem_u32(smem + C::OFF_Q), sd = smem_u32(smem + C::OFF_DO);
       bool ok = wait_bar(q_full, 0, ctl, ERR_ATTN_DQ_WAIT);
       if (warp == 1) {
+        ok = ok && wait_bar(qd_tmem, 0, ctl, ERR_ATTN_DQ_WAIT);
         for (int k = 0; ok && k < nsteps; ++k) {
           const int bf = k & 1, st = k % C::STAGES;
           if (!(ok = wait_bar(&kv_full[st], (k / C::STAGES) & 1, ctl, ERR_ATTN_DQ_WAIT))) break;
-          if (!(ok = wait_bar(&s_free[bf], ((k >> 1) & 1) ^ 1, ctl, ERR_ATTN_DQ_WAIT))) break;
+          // dS of block k-2 (over this buffer's S columns) has been read by its dQ product.
+          if (k >= 2 && !(ok = wait_bar(&mm2_done[bf], ((k >> 1) - 1) & 1, ctl, ERR_ATTN_DQ_WAIT)))
+            break;
           tc_fence_after();
           const uint32_t sk = smem_u32(smem + C::OFF_ST + st * 2 * C::K_BYTES);
           const uint32_t sv = sk + C::K_BYTES;
 #pragma unroll
-          for (int kk = 0; kk < DH / 16; ++kk) {
-            tc_mma_f16(tmem + bf * 128, kmajor_desc(sq, C::BQ, kk), kmajor_desc(sk, C::BK, kk), id_s,
-                       kk > 0);
-            tc_mma_f16(tmem + bf * 128 + 64, kmajor_desc(sd, C::BQ, kk), kmajor_desc(sv, C::BK, kk),
-                       id_s, kk > 0);
+          for (int kk = 0; kk < DH / 16; ++kk) {   // 16 of dh = 8 columns of q / dO per step
+            tc_mma_f16_ts(tmem + bf * 128, tmem + 384 + 8 * kk, kmajor_desc(sk, C::BK, kk), id_s,
+                          kk > 0);
+            tc_mma_f16_ts(tmem + bf * 128 + 64, tmem + 448 + 8 * kk, kmajor_desc(sv, C::BK, kk),
+                          id_s, kk > 0);
           }
           tc_commit(&s_full[bf]);
         }
@@ -954,7 +961,7 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q128,
           const uint32_t sk = smem_u32(smem + C::OFF_ST + sj * 2 * C::K_BYTES);
 #pragma unroll
           for (int kk = 0; kk < C::BK / 16; ++kk)   // 16 keys = 8 columns of dS per step
-            tc_mma_f16_ts(t_dq, tmem + 384 + 32 * bj + 8 * kk, mnmajor_desc(sk, C::BK, kk),
+            tc_mma_f16_ts(t_dq, tmem + 128 * bj + 8 * kk, mnmajor_desc(sk, C::BK, kk),
                           id_acc, (k | kk) != 0);
           tc_commit(&mm2_done[bj]);
           tc_commit(&kv_empty[sj]);   // the scores of block k completed before its dS existed
@@ -977,7 +984,29 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q128,
     const float l2 = p.lse2[hrow + q];     // padded rows: +inf, so P = 0
     const float dv = p.dvec[hrow + q];
     bool ok = true;
-    for (int k = wg; k < nsteps; k += 2) {
+    // q (warpgroup 0) or dO (warpgroup 1) of this row into tensor memory, once:
+    // dh fp16 values as dh/2 pairs from the 128-byte-swizzled shared-memory
+    // tile (16-byte unit u of row r of a 64-wide chunk sits at unit u ^ (r % 8)).
+    if (__all_sync(0xffffffffu, wait_bar(q_full, 0, ctl, ERR_ATTN_DQ_WAIT))) {
+      const uint8_t* src = smem + (wg == 0 ? C::OFF_Q : C::OFF_DO) + r * 128;
+      const uint32_t dst = tmem + (wg == 0 ? 384 : 448) + lane_off;
+#pragma unroll
+      for (int h = 0; h < DH / 64; ++h) {
+        uint32_t w[32];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const uint4 v = *reinterpret_cast<const uint4*>(src + h * C::BQ * 128 + ((u ^ (r & 7)) << 4));
+          w[4 * u] = v.x; w[4 * u + 1] = v.y; w[4 * u + 2] = v.z; w[4 * u + 3] = v.w;
+        }
+        tmem_st32(dst + 32 * h, w);
+      }
+      tc_wait_st();
+      tc_fence_before();
+      mbar_arrive(qd_tmem);
+    } else {
+      ok = false;
+    }
+    for (int k = wg; ok && k < nsteps; k += 2) {
       const int bf = k & 1;
       const uint32_t u = k >> 1;
       const int ks = k * C::BK;
@@ -990,8 +1019,6 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q128,
       tmem_ld32(tmem + bf * 128 + 64 + lane_off, rd0);
       tmem_ld32(tmem + bf * 128 + 64 + lane_off + 32, rd1);
       tc_wait_ld();
-      tc_fence_before();
-      mbar_arrive(&s_free[bf]);
       // Keys past the last visible one (after the query, or past S) are
       // masked: a select per element against a bound fixed once per block.
       const int kmax = (p.causal ? min(q, p.S - 1) : p.S - 1) - ks;
@@ -1018,9 +1045,10 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q128,
         pk[e] = pack_f16x2(__uint_as_float(rd0[2 * e]), __uint_as_float(rd0[2 * e + 1]));
         pk[16 + e] = pack_f16x2(__uint_as_float(rd1[2 * e]), __uint_as_float(rd1[2 * e + 1]));
       }
-      // The dS columns of buffer bf were last read by the dQ MMAs of block k-2.
-      if (k >= 2 && !__all_sync(0xffffffffu, wait_bar(&mm2_done[bf], (u - 1) & 1, ctl, ERR_ATTN_DQ_WAIT))) { ok = false; break; }
-      tmem_st32(tmem + 384 + 32 * bf + lane_off, pk);
+      // dS over the first half of this block's S columns (already in registers);
+      // the dQ product of block k-2, which read this buffer, completed before
+      // the scores of block k were issued.
+      tmem_st32(tmem + bf * 128 + lane_off, pk);
       tc_wait_st();
       tc_fence_before();
       mbar_arrive(&p_full[bf]);
