@@ -41,3 +41,27 @@ def test_layernorm_fwd_bwd(rows, D):
     check("dgamma", dg, dgr)
     check("dbeta", db, dbr)
     assert tl.check_error() == 0
+
+
+@pytest.mark.parametrize("rows,D,offset", [(300, 4096, 0.0), (77, 1000, 100.0), (5, 8192, -30.0)])
+def test_layernorm_fwd_f16_output_and_offset_rows(rows, D, offset):
+    """tp_layernorm_fwd_f16 (the fp16 output that feeds the attention
+    products) against the oracle, on rows whose mean is far from zero: the
+    per-thread mean / M2 combination must not lose the variance to
+    cancellation."""
+    require_gpu()
+    g = torch.Generator().manual_seed(rows * 7 + D)
+    bf = torch.bfloat16
+    x = (torch.randn(rows, D, generator=g) + offset).to(bf)
+    gam = (1 + 0.1 * torch.randn(D, generator=g)).to(bf)
+    bet = (0.1 * torch.randn(D, generator=g)).to(bf)
+    y = torch.empty(rows, D, dtype=torch.float16, device="cuda")
+    mean = torch.empty(rows, dtype=torch.float32, device="cuda")
+    rstd = torch.empty_like(mean)
+    tl.layernorm_fwd_f16(x.cuda(), gam.cuda(), bet.cuda(), rows, D, 1e-5, y, mean, rstd)
+    f = lambda v: v.to(torch.float64).numpy()
+    yr, mr, rr = core.layernorm_fwd(f(x), f(gam), f(bet), 1e-5)
+    check("y", y, yr)
+    check("mean", mean, mr)
+    check("rstd", rstd, rr)
+    assert tl.check_error() == 0
