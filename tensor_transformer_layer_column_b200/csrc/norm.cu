@@ -62,139 +62,83 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
-constexpr int LNB_THREADS = 256;
-
-// Mean and sum of squared deviations (M2) of a group of n values; two groups
-// combine exactly (Chan, Golub and LeVeque's pairwise update), so every
-// thread reduces its own values in two passes and the block combines the
-// per-thread triples in a fixed order.
-struct MeanM2 {
-  float n, mean, m2;
-};
-
-__device__ __forceinline__ MeanM2 combine(const MeanM2& a, const MeanM2& b) {
-  const float n = a.n + b.n;
-  if (n == 0.f) return a;
-  const float d = b.mean - a.mean;
-  const float wb = b.n / n;
-  return {n, a.mean + d * wb, a.m2 + b.m2 + d * d * a.n * wb};
-}
-
-__device__ __forceinline__ MeanM2 warp_combine(MeanM2 v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    MeanM2 w;
-    w.n = __shfl_xor_sync(0xffffffffu, v.n, o);
-    w.mean = __shfl_xor_sync(0xffffffffu, v.mean, o);
-    w.m2 = __shfl_xor_sync(0xffffffffu, v.m2, o);
-    // Both partners combine (lower lane's group first), so they agree bit for bit.
-    v = (threadIdx.x & o) ? combine(w, v) : combine(v, w);
-  }
-  return v;
-}
-
-// One 256-thread block per row, blocks walking contiguous runs of rows; thread
-// owns 8-element chunks tid, tid + 256, ... (CH of them), with its gamma and
-// beta chunks held in registers (packed bf16) for the whole kernel and the
-// next row's chunks loaded while the current row is reduced and written.
-// Statistics in fp32: per-thread two-pass mean / M2, one block combination.
-// The output is bf16, or fp16 when F16OUT (values beyond the fp16 range set
-// `err` to 0x301).
+// One warp per row, rows walked grid-stride; lane owns 8-element chunks lane,
+// lane+32, ...  The row stays in registers as packed bf16 (4 registers per
+// chunk), so two 256-thread blocks fit per SM.  Statistics in fp32, two
+// passes over the registers (mean, then centred variance).  The output is
+// bf16, or fp16 when F16OUT (values beyond the fp16 range set `err` to 0x301).
 template <int CH, bool F16OUT>
-__global__ void __launch_bounds__(LNB_THREADS, CH >= 4 ? 2 : 3)
+__global__ void __launch_bounds__(256, 2)
 ln_fwd_kernel(const uint16_t* __restrict__ x, const uint16_t* __restrict__ g,
-              const uint16_t* __restrict__ b, long long rows, int D, int rows_per_block,
-              float eps, uint16_t* __restrict__ y, float* __restrict__ mean,
-              float* __restrict__ rstd, unsigned int* err) {
-  __shared__ MeanM2 red[2][LNB_THREADS / 32];
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+              const uint16_t* __restrict__ b, long long rows, int D, float eps,
+              uint16_t* __restrict__ y, float* __restrict__ mean, float* __restrict__ rstd,
+              unsigned int* err) {
+  const int lane = threadIdx.x & 31;
   const int nch = D >> 3;
-  uint4 gpk[CH], bpk[CH];
-#pragma unroll
-  for (int j = 0; j < CH; ++j) {
-    const int c = tid + LNB_THREADS * j;
-    if (c < nch) {
-      gpk[j] = *reinterpret_cast<const uint4*>(g + c * 8);
-      bpk[j] = *reinterpret_cast<const uint4*>(b + c * 8);
-    }
-  }
-  const long long r0 = (long long)blockIdx.x * rows_per_block;
-  const long long r1 = min(rows, r0 + rows_per_block);
-  uint4 cur[CH], nxt[CH];
-  auto load_row = [&](long long r, uint4 (&o)[CH]) {
-#pragma unroll
-    for (int j = 0; j < CH; ++j) {
-      const int c = tid + LNB_THREADS * j;
-      if (c < nch) o[j] = *reinterpret_cast<const uint4*>(x + r * D + c * 8);
-    }
-  };
-  if (r0 < r1) load_row(r0, cur);
+  const long long nwarps = (long long)gridDim.x * (blockDim.x >> 5);
   bool over = false;
-  int buf = 0;
-  for (long long r = r0; r < r1; ++r, buf ^= 1) {
-    if (r + 1 < r1) load_row(r + 1, nxt);
-    // Per-thread mean and M2 of its (up to 8 * CH) values, two passes over registers.
-    float s = 0.f, cnt = 0.f;
+  for (long long row = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); row < rows;
+       row += nwarps) {
+    const uint16_t* xr = x + row * D;
+    uint4 pk[CH];
+    float s = 0.f;
 #pragma unroll
     for (int j = 0; j < CH; ++j) {
-      if (tid + LNB_THREADS * j < nch) {
+      const int c = lane + 32 * j;
+      if (c < nch) pk[j] = *reinterpret_cast<const uint4*>(xr + c * 8);
+    }
+#pragma unroll
+    for (int j = 0; j < CH; ++j) {
+      if (lane + 32 * j < nch) {
         float v[8];
-        unpack8(cur[j], v);
+        unpack8(pk[j], v);
 #pragma unroll
         for (int e = 0; e < 8; ++e) s += v[e];
-        cnt += 8.f;
       }
     }
-    MeanM2 st{cnt, cnt > 0.f ? s / cnt : 0.f, 0.f};
+    const float mu = warp_sum(s) / D;
+    float ss = 0.f;
 #pragma unroll
     for (int j = 0; j < CH; ++j) {
-      if (tid + LNB_THREADS * j < nch) {
+      if (lane + 32 * j < nch) {
         float v[8];
-        unpack8(cur[j], v);
+        unpack8(pk[j], v);
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          const float d = v[e] - st.mean;
-          st.m2 += d * d;
+          const float d = v[e] - mu;
+          ss += d * d;
         }
       }
     }
-    st = warp_combine(st);
-    if (lane == 0) red[buf][warp] = st;
-    __syncthreads();
-    MeanM2 tot = red[buf][0];
-#pragma unroll
-    for (int w = 1; w < LNB_THREADS / 32; ++w) tot = combine(tot, red[buf][w]);
-    const float mu = tot.mean;
-    const float rs = rsqrtf(tot.m2 / D + eps);
+    const float rs = rsqrtf(warp_sum(ss) / D + eps);
 #pragma unroll
     for (int j = 0; j < CH; ++j) {
-      const int c = tid + LNB_THREADS * j;
+      const int c = lane + 32 * j;
       if (c < nch) {
         float v[8], gv[8], bv[8], o[8];
-        unpack8(cur[j], v);
-        unpack8(gpk[j], gv);
-        unpack8(bpk[j], bv);
+        unpack8(pk[j], v);
+        unpack8(*reinterpret_cast<const uint4*>(g + c * 8), gv);
+        unpack8(*reinterpret_cast<const uint4*>(b + c * 8), bv);
 #pragma unroll
         for (int e = 0; e < 8; ++e) o[e] = (v[e] - mu) * rs * gv[e] + bv[e];
         if (F16OUT) {
-          *reinterpret_cast<uint4*>(y + r * D + c * 8) = pack8_f16(o);
+          *reinterpret_cast<uint4*>(y + row * D + c * 8) = pack8_f16(o);
 #pragma unroll
           for (int e = 0; e < 8; ++e) over |= fabsf(o[e]) > 65504.0f;
         } else {
-          *reinterpret_cast<uint4*>(y + r * D + c * 8) = pack8(o);
+          *reinterpret_cast<uint4*>(y + row * D + c * 8) = pack8(o);
         }
       }
     }
-    if (tid == 0) {
-      mean[r] = mu;
-      rstd[r] = rs;
+    if (lane == 0) {
+      mean[row] = mu;
+      rstd[row] = rs;
     }
-#pragma unroll
-    for (int j = 0; j < CH; ++j) cur[j] = nxt[j];
   }
   if (F16OUT && over && err) atomicCAS(err, 0u, 0x301u);
 }
 
+constexpr int LNB_THREADS = 256;
 
 // One block walks a contiguous chunk of rows; thread owns 8-element chunks
 // tid, tid+256, ...; the next row's operands are loaded while the current
@@ -516,22 +460,24 @@ template <bool F16OUT>
 tp_status ln_fwd_dispatch(const uint16_t* x, const uint16_t* g, const uint16_t* b, long long rows,
                           int D, float eps, uint16_t* y, float* mean, float* rstd,
                           cudaStream_t stream) {
-  const int per_thread = (D / 8 + LNB_THREADS - 1) / LNB_THREADS;
-  long long nblk = (per_thread >= 4 ? 2LL : 3LL) * sm_count();   // resident blocks
-  if (nblk > rows) nblk = rows;
-  const int rpb = (int)((rows + nblk - 1) / nblk);
+  long long nblk = (rows + 7) / 8;
+  if (nblk > 2LL * sm_count()) nblk = 2LL * sm_count();
   const unsigned grid = (unsigned)nblk;
+  const int per_lane = (D / 8 + 31) / 32;
   unsigned int* err = error_word();
   TraceScope ts(stream, TK_LN_FWD);
-  if (per_thread <= 1)
-    ln_fwd_kernel<1, F16OUT><<<grid, LNB_THREADS, 0, stream>>>(x, g, b, rows, D, rpb, eps, y, mean,
-                                                                rstd, err);
-  else if (per_thread <= 2)
-    ln_fwd_kernel<2, F16OUT><<<grid, LNB_THREADS, 0, stream>>>(x, g, b, rows, D, rpb, eps, y, mean,
-                                                                rstd, err);
-  else if (per_thread <= 4)
-    ln_fwd_kernel<4, F16OUT><<<grid, LNB_THREADS, 0, stream>>>(x, g, b, rows, D, rpb, eps, y, mean,
-                                                                rstd, err);
+  if (per_lane <= 1)
+    ln_fwd_kernel<1, F16OUT><<<grid, 256, 0, stream>>>(x, g, b, rows, D, eps, y, mean, rstd, err);
+  else if (per_lane <= 2)
+    ln_fwd_kernel<2, F16OUT><<<grid, 256, 0, stream>>>(x, g, b, rows, D, eps, y, mean, rstd, err);
+  else if (per_lane <= 4)
+    ln_fwd_kernel<4, F16OUT><<<grid, 256, 0, stream>>>(x, g, b, rows, D, eps, y, mean, rstd, err);
+  else if (per_lane <= 8)
+    ln_fwd_kernel<8, F16OUT><<<grid, 256, 0, stream>>>(x, g, b, rows, D, eps, y, mean, rstd, err);
+  else if (per_lane <= 16)
+    ln_fwd_kernel<16, F16OUT><<<grid, 256, 0, stream>>>(x, g, b, rows, D, eps, y, mean, rstd, err);
+  else if (per_lane <= 32)
+    ln_fwd_kernel<32, F16OUT><<<grid, 256, 0, stream>>>(x, g, b, rows, D, eps, y, mean, rstd, err);
   else
     return TP_ERR_UNSUPPORTED;
   return cuda_status(cudaGetLastError());

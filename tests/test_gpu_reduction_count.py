@@ -58,9 +58,10 @@ def test_launch_sequence_independent_of_t(kind):
 
 def test_mlp_one_shard_sum_per_direction():
     """MLP: forward = column-parallel product + row-parallel product (shard sum
-    in its K walk); backward = dA, dW2, dW1 and the input-gradient product
-    (shard sum in its K walk), plus the two bias column sums.  No other kernel."""
+    in its K walk); backward = dA (its epilogue also writes db1's column
+    partials, reduced right after), dW2, dW1 and the input-gradient product
+    (shard sum in its K walk), then db2's two-pass column sum.  No other kernel."""
     require_gpu()
     seq = _launches("mlp", 8)
-    assert seq == ["gemm", "gemm", "gemm", "gemm", "gemm", "gemm",
-                   "colsum", "colsum", "colsum", "colsum"]
+    assert seq == ["gemm", "gemm", "gemm", "colsum", "gemm", "gemm", "gemm",
+                   "colsum", "colsum"]
