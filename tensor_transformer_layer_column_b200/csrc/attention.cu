@@ -13,13 +13,11 @@
 // 6e-3 at S = 2048, with fp16 near 2e-3.  The tensor-core rate is the same.
 //
 // Forward (per pair of 128-query tiles, head, batch; 64-key blocks):
-//   q is copied once into tensor memory and is the A operand of S = q k^T
-//   (tcgen05, fp32 in TMEM), so the score products read only k from shared
-//   memory; online softmax in fp32 by one thread per query row (base-2
-//   exponent, scores scaled by log2(e)/sqrt(dh) inside the exponent), P
-//   rounded to fp16 and written into tensor memory over the scores it came
-//   from, O += P v (tcgen05 with P as the A operand read from tensor memory,
-//   fp32 in TMEM, rescaled lazily).  The two tiles alternate on the tensor core.
+//   S = q k^T (tcgen05, fp32 in TMEM), online softmax in fp32 by one thread per
+//   query row (base-2 exponent, scores pre-scaled by log2(e)/sqrt(dh)), P
+//   rounded to fp16 into tensor memory, O += P v (tcgen05 with P as the
+//   A operand read from tensor memory, fp32 in TMEM, rescaled lazily).  The
+//   two tiles alternate on the tensor core.
 //   Writes O [t][T][Dt] (bf16) and the log-sum-exp [B][H][S] (fp32).
 // Backward (P recomputed from the log-sum-exp; no atomics, deterministic;
 // dO in and dqkv out are fp16):
@@ -162,14 +160,10 @@ __device__ __forceinline__ uint64_t mnmajor_desc(uint32_t base, int R, int kk) {
 // =====================================================================================
 // Two 128-query tiles per CTA take turns on the tensor core: while one tile's
 // softmax warpgroup works on its scores, the other tile's products run.  Keys
-// come in 64-wide blocks through a 4-stage ring.  Tensor memory per tile: q
-// (dh/2 columns of fp16 pairs, written once by the tile's softmax warps), S
-// (64 columns; P, 32 columns of fp16 pairs, is written over its first half)
-// and O (dh columns).  Because P lives in S's columns, the scores of block
-// j+1 wait for the P v product of block j; the other tile fills the tensor
-// core meanwhile.  O is rescaled lazily: only when a row's running max grows
-// by more than 2^8 (log2 units), so P = 2^(s - m_used) stays below 256 (exact
-// in fp16) and the final O / l is unchanged.
+// come in 64-wide blocks through a 4-stage ring; each tile has its own S (64
+// TMEM columns), P (32 columns of fp16 pairs) and O (dh columns).  O is rescaled lazily: only when a row's
+// running max grows by more than 2^8 (log2 units), so P = 2^(s - m_used) stays
+// below 256 (exact in fp16) and the final O / l is unchanged.
 template <int DH>
 struct FwdCfg {
   static constexpr int BM = 128, BN = 64, CH = DH / 64, STAGES = 4;
@@ -200,7 +194,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q128,
   uint64_t* kv_full = bars + 1;     // [STAGES <= 4]
   uint64_t* kv_empty = bars + 5;    // [STAGES]
   uint64_t* s_full = bars + 9;      // [2] per tile
-  uint64_t* q_tmem = bars + 11;     // [2] the tile's q is in tensor memory
+  uint64_t* s_free = bars + 11;     // [2]
   uint64_t* p_full = bars + 13;     // [2]
   uint64_t* pv_done = bars + 15;    // [2]
   uint64_t* drain = bars + 17;
@@ -232,7 +226,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q128,
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&q_tmem[i], 128);
+      mbar_init(&s_free[i], 128);
       mbar_init(&p_full[i], 128);
       mbar_init(&pv_done[i], 1);
     }
@@ -249,8 +243,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q128,
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  // TMEM columns: S (then P) of tile i at 64i, O of tile i at 128 + 128i, q of tile i at
-  // 384 + 64i (dh/2 columns).
+  // TMEM columns: S of tile i at 64i, O of tile i at 128 + 128i, P of tile i at 384 + 32i.
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
@@ -279,12 +272,14 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q128,
     }
   } else if (warp == 1 || warp == 10) {
     // Two issuers, each blocking only on its own barriers: warp 1 issues the
-    // scores S = q k^T of both tiles (block j+1 once the tile's P v of block j
-    // has read P out of S's columns), warp 10 the products P V (once P is in
-    // tensor memory) and releases each K/V stage.
+    // scores S = q k^T of both tiles (block j+1 once the tile's softmax has
+    // copied S of block j out of tensor memory), warp 10 the products P V
+    // (once P is in tensor memory) and releases each K/V stage.  Neither
+    // stream waits behind the other.
     if (lane == 0) {
       constexpr uint32_t id_s = idesc_f32acc(128, C::BN, false, false, true);
       constexpr uint32_t id_pv = idesc_f32acc(128, DH, false, true, true);
+      const uint32_t sq = smem_u32(smem + C::OFF_Q);
       auto kv_addr = [&](int j) { return smem_u32(smem + C::OFF_KV + (j % C::STAGES) * 2 * C::KV_BYTES); };
       bool ok = wait_bar(q_full, 0, ctl, ERR_ATTN_FWD_WAIT);
       if (warp == 1) {
@@ -293,8 +288,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q128,
 #pragma unroll
           for (int i = 0; i < 2; ++i) {
             if (ok && j < ntile[i]) {
-              if (j == 0 && !(ok = wait_bar(&q_tmem[i], 0, ctl, ERR_ATTN_FWD_WAIT))) break;
-              if (j > 0 && !(ok = wait_bar(&pv_done[i], (j - 1) & 1, ctl, ERR_ATTN_FWD_WAIT))) break;
+              if (j > 0 && !(ok = wait_bar(&s_free[i], (j - 1) & 1, ctl, ERR_ATTN_FWD_WAIT))) break;
               if (!kv_in && !(ok = wait_bar(&kv_full[j % C::STAGES], (j / C::STAGES) & 1, ctl,
                                             ERR_ATTN_FWD_WAIT)))
                 break;
@@ -302,9 +296,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q128,
               tc_fence_after();
               const uint32_t sk = kv_addr(j);
 #pragma unroll
-              for (int kk = 0; kk < DH / 16; ++kk)   // 16 of dh = 8 columns of q per step
-                tc_mma_f16_ts(tmem + 64 * i, tmem + 384 + 64 * i + 8 * kk,
-                              kmajor_desc(sk, C::BN, kk), id_s, kk > 0);
+              for (int kk = 0; kk < DH / 16; ++kk)
+                tc_mma_f16(tmem + 64 * i, kmajor_desc(sq + i * C::Q_BYTES, C::BM, kk),
+                           kmajor_desc(sk, C::BN, kk), id_s, kk > 0);
               tc_commit(&s_full[i]);
             }
           }
@@ -319,7 +313,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q128,
               const uint32_t sv = kv_addr(j) + C::KV_BYTES;
 #pragma unroll
               for (int kk = 0; kk < C::BN / 16; ++kk)   // 16 keys = 8 columns of P per step
-                tc_mma_f16_ts(tmem + 128 + 128 * i, tmem + 64 * i + 8 * kk,
+                tc_mma_f16_ts(tmem + 128 + 128 * i, tmem + 384 + 32 * i + 8 * kk,
                               mnmajor_desc(sv, C::BN, kk), id_pv, (j | kk) != 0);
               tc_commit(&pv_done[i]);
             }
@@ -344,32 +338,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q128,
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
     const uint32_t t_s = tmem + 64 * tile + lane_off;
     const uint32_t t_o = tmem + 128 + 128 * tile + lane_off;
-    const uint32_t t_q = tmem + 384 + 64 * tile + lane_off;
+    const uint32_t t_p = tmem + 384 + 32 * tile + lane_off;
     float m_used = -1e30f, l = 0.f;
     bool ok = true;
-    // q of this row into tensor memory, once: dh fp16 values as dh/2 pairs,
-    // read from the tile's 128-byte-swizzled shared-memory copy (16-byte unit u
-    // of row r of a 64-wide chunk sits at unit u ^ (r % 8)).
-    if (__all_sync(0xffffffffu, wait_bar(q_full, 0, ctl, ERR_ATTN_FWD_WAIT))) {
-      const uint8_t* qrow = smem + C::OFF_Q + tile * C::Q_BYTES + r * 128;
-#pragma unroll
-      for (int h = 0; h < DH / 64; ++h) {
-        uint32_t w[32];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const uint4 v = *reinterpret_cast<const uint4*>(qrow + h * C::BM * 128 +
-                                                          ((u ^ (r & 7)) << 4));
-          w[4 * u] = v.x; w[4 * u + 1] = v.y; w[4 * u + 2] = v.z; w[4 * u + 3] = v.w;
-        }
-        tmem_st32(t_q + 32 * h, w);
-      }
-      tc_wait_st();
-      tc_fence_before();
-      mbar_arrive(&q_tmem[tile]);
-    } else {
-      ok = false;
-    }
-    for (int j = 0; ok && j < n; ++j) {
+    for (int j = 0; j < n; ++j) {
       if (!__all_sync(0xffffffffu, wait_bar(&s_full[tile], j & 1, ctl, ERR_ATTN_FWD_WAIT))) { ok = false; break; }
       tc_fence_after();
       float s[C::BN];
@@ -384,6 +356,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q128,
           s[32 + e] = __uint_as_float(rb[e]);
         }
       }
+      tc_fence_before();
+      mbar_arrive(&s_free[tile]);
       // Keys past the last visible one (after the query, or past S) are masked: a select
       // per element against a bound fixed once per block, taken only in blocks where
       // some row of the warp has a masked key (the causal diagonal, the sequence end).
@@ -438,11 +412,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q128,
         }
       }
       {
-        // P over the first half of this block's S columns (already in registers).
         uint32_t pk[C::BN / 2];
 #pragma unroll
         for (int g = 0; g < C::BN / 2; ++g) pk[g] = pack_f16x2(s[2 * g], s[2 * g + 1]);
-        tmem_st32(t_s, pk);
+        tmem_st32(t_p, pk);
         tc_wait_st();
       }
       tc_fence_before();
@@ -820,13 +793,9 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_kv128,
 }
 
 // ---------------------------------------------------------------- dQ
-// Per 128-query block, walk 64-key blocks through a 4-stage K/V ring.  q and
-// dO (fixed per block) are copied once into tensor memory and are the A
-// operands of S = q k^T and dP = dO v^T, so those products read only k and v
-// from shared memory.  Two S/dP buffers in TMEM, one per compute warpgroup;
-// dS (fp16 pairs) is written over the first half of its S columns and is the
-// A operand of dQ += dS k, so the next scores into a buffer wait for the dQ
-// product that reads it.
+// Per 128-query block, walk 64-key blocks through a 4-stage K/V ring.  Two
+// S/dP buffers in TMEM, one per compute warpgroup; dS (fp16 pairs) goes to
+// its own TMEM columns and is the A operand of dQ += dS k.
 template <int DH>
 struct DqCfg {
   static constexpr int BQ = 128, BK = 64, CH = DH / 64;
@@ -855,7 +824,7 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q128,
   uint64_t* kv_full = bars + 1;    // [STAGES <= 4] per stage
   uint64_t* kv_empty = bars + 5;   // [STAGES]
   uint64_t* s_full = bars + 9;     // [2] per TMEM buffer
-  uint64_t* qd_tmem = bars + 11;   // [1] q and dO are in tensor memory
+  uint64_t* s_free = bars + 11;    // [2]
   uint64_t* p_full = bars + 13;    // [2] per dS buffer
   uint64_t* mm2_done = bars + 15;  // [2]
   uint64_t* drain = bars + 17;
@@ -881,10 +850,10 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q128,
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&p_full[i], 128);   // buffer i belongs to compute warpgroup i
+      mbar_init(&s_free[i], 128);   // buffer i belongs to compute warpgroup i
+      mbar_init(&p_full[i], 128);
       mbar_init(&mm2_done[i], 1);
     }
-    mbar_init(qd_tmem, 256);        // both compute warpgroups
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -897,9 +866,8 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q128,
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  // TMEM columns: buffer j holds S (then dS, fp16 pairs, over its first half)
-  // at 128j and dP at 128j + 64; dQ accumulates at 256; q at 384 and dO at
-  // 448 (dh/2 columns each).
+  // TMEM columns: buffer j holds S at 128j, dP at 128j + 64 and dS (fp16 pairs)
+  // at 384 + 32j; dQ accumulates at 256.
   const uint32_t t_dq = tmem + 256;
 
   if (warp == 0) {
@@ -932,24 +900,22 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q128,
     if (lane == 0) {
       constexpr uint32_t id_s = idesc_f32acc(128, C::BK, false, false, true);
       constexpr uint32_t id_acc = idesc_f32acc(128, DH, false, true, true);
+      const uint32_t sq = smem_u32(smem + C::OFF_Q), sd = smem_u32(smem + C::OFF_DO);
       bool ok = wait_bar(q_full, 0, ctl, ERR_ATTN_DQ_WAIT);
       if (warp == 1) {
-        ok = ok && wait_bar(qd_tmem, 0, ctl, ERR_ATTN_DQ_WAIT);
         for (int k = 0; ok && k < nsteps; ++k) {
           const int bf = k & 1, st = k % C::STAGES;
           if (!(ok = wait_bar(&kv_full[st], (k / C::STAGES) & 1, ctl, ERR_ATTN_DQ_WAIT))) break;
-          // dS of block k-2 (over this buffer's S columns) has been read by its dQ product.
-          if (k >= 2 && !(ok = wait_bar(&mm2_done[bf], ((k >> 1) - 1) & 1, ctl, ERR_ATTN_DQ_WAIT)))
-            break;
+          if (!(ok = wait_bar(&s_free[bf], ((k >> 1) & 1) ^ 1, ctl, ERR_ATTN_DQ_WAIT))) break;
           tc_fence_after();
           const uint32_t sk = smem_u32(smem + C::OFF_ST + st * 2 * C::K_BYTES);
           const uint32_t sv = sk + C::K_BYTES;
 #pragma unroll
-          for (int kk = 0; kk < DH / 16; ++kk) {   // 16 of dh = 8 columns of q / dO per step
-            tc_mma_f16_ts(tmem + bf * 128, tmem + 384 + 8 * kk, kmajor_desc(sk, C::BK, kk), id_s,
-                          kk > 0);
-            tc_mma_f16_ts(tmem + bf * 128 + 64, tmem + 448 + 8 * kk, kmajor_desc(sv, C::BK, kk),
-                          id_s, kk > 0);
+          for (int kk = 0; kk < DH / 16; ++kk) {
+            tc_mma_f16(tmem + bf * 128, kmajor_desc(sq, C::BQ, kk), kmajor_desc(sk, C::BK, kk), id_s,
+                       kk > 0);
+            tc_mma_f16(tmem + bf * 128 + 64, kmajor_desc(sd, C::BQ, kk), kmajor_desc(sv, C::BK, kk),
+                       id_s, kk > 0);
           }
           tc_commit(&s_full[bf]);
         }
@@ -961,7 +927,7 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q128,
           const uint32_t sk = smem_u32(smem + C::OFF_ST + sj * 2 * C::K_BYTES);
 #pragma unroll
           for (int kk = 0; kk < C::BK / 16; ++kk)   // 16 keys = 8 columns of dS per step
-            tc_mma_f16_ts(t_dq, tmem + 128 * bj + 8 * kk, mnmajor_desc(sk, C::BK, kk),
+            tc_mma_f16_ts(t_dq, tmem + 384 + 32 * bj + 8 * kk, mnmajor_desc(sk, C::BK, kk),
                           id_acc, (k | kk) != 0);
           tc_commit(&mm2_done[bj]);
           tc_commit(&kv_empty[sj]);   // the scores of block k completed before its dS existed
@@ -984,29 +950,7 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q128,
     const float l2 = p.lse2[hrow + q];     // padded rows: +inf, so P = 0
     const float dv = p.dvec[hrow + q];
     bool ok = true;
-    // q (warpgroup 0) or dO (warpgroup 1) of this row into tensor memory, once:
-    // dh fp16 values as dh/2 pairs from the 128-byte-swizzled shared-memory
-    // tile (16-byte unit u of row r of a 64-wide chunk sits at unit u ^ (r % 8)).
-    if (__all_sync(0xffffffffu, wait_bar(q_full, 0, ctl, ERR_ATTN_DQ_WAIT))) {
-      const uint8_t* src = smem + (wg == 0 ? C::OFF_Q : C::OFF_DO) + r * 128;
-      const uint32_t dst = tmem + (wg == 0 ? 384 : 448) + lane_off;
-#pragma unroll
-      for (int h = 0; h < DH / 64; ++h) {
-        uint32_t w[32];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const uint4 v = *reinterpret_cast<const uint4*>(src + h * C::BQ * 128 + ((u ^ (r & 7)) << 4));
-          w[4 * u] = v.x; w[4 * u + 1] = v.y; w[4 * u + 2] = v.z; w[4 * u + 3] = v.w;
-        }
-        tmem_st32(dst + 32 * h, w);
-      }
-      tc_wait_st();
-      tc_fence_before();
-      mbar_arrive(qd_tmem);
-    } else {
-      ok = false;
-    }
-    for (int k = wg; ok && k < nsteps; k += 2) {
+    for (int k = wg; k < nsteps; k += 2) {
       const int bf = k & 1;
       const uint32_t u = k >> 1;
       const int ks = k * C::BK;
@@ -1019,6 +963,8 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q128,
       tmem_ld32(tmem + bf * 128 + 64 + lane_off, rd0);
       tmem_ld32(tmem + bf * 128 + 64 + lane_off + 32, rd1);
       tc_wait_ld();
+      tc_fence_before();
+      mbar_arrive(&s_free[bf]);
       // Keys past the last visible one (after the query, or past S) are
       // masked: a select per element against a bound fixed once per block.
       const int kmax = (p.causal ? min(q, p.S - 1) : p.S - 1) - ks;
@@ -1045,10 +991,9 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q128,
         pk[e] = pack_f16x2(__uint_as_float(rd0[2 * e]), __uint_as_float(rd0[2 * e + 1]));
         pk[16 + e] = pack_f16x2(__uint_as_float(rd1[2 * e]), __uint_as_float(rd1[2 * e + 1]));
       }
-      // dS over the first half of this block's S columns (already in registers);
-      // the dQ product of block k-2, which read this buffer, completed before
-      // the scores of block k were issued.
-      tmem_st32(tmem + bf * 128 + lane_off, pk);
+      // The dS columns of buffer bf were last read by the dQ MMAs of block k-2.
+      if (k >= 2 && !__all_sync(0xffffffffu, wait_bar(&mm2_done[bf], (u - 1) & 1, ctl, ERR_ATTN_DQ_WAIT))) { ok = false; break; }
+      tmem_st32(tmem + 384 + 32 * bf + lane_off, pk);
       tc_wait_st();
       tc_fence_before();
       mbar_arrive(&p_full[bf]);

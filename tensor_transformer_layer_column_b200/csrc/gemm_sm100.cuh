@@ -511,11 +511,6 @@ constexpr int GP_A_BYTES = 128 * GEMM_BK * 2;   // 16 KiB per CTA
 constexpr int GP_B_BYTES = 128 * GEMM_BK * 2;   // 16 KiB per CTA
 constexpr int GP_STAGE_BYTES = GP_A_BYTES + GP_B_BYTES;
 constexpr int GP_SMEM_BYTES = GP_STAGES * GP_STAGE_BYTES + 1024 + 256;
-// The producer prefetches into L2 the operand tiles of the k-block GEMM_PF
-// blocks ahead of the one it loads: most stages then hit in L2 instead of
-// waiting on DRAM misses, whose latency under load is close to what the
-// shared-memory ring covers.
-constexpr int GEMM_PF = 8;
 
 enum : unsigned int {
   ERR_GEMMP_PRODUCER_WAIT = 0x111,
@@ -609,29 +604,6 @@ gemm_pair_sm100(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
           const int k0 = (kb - ks * p.kb_per_shard) * GEMM_BK;
           const int a_s = p.a_src == SHARD_K ? ks : (p.a_src == SHARD_MN ? tc.ms : 0);
           const int b_s = p.b_src == SHARD_K ? ks : (p.b_src == SHARD_MN ? tc.ns : 0);
-          if (kb + GEMM_PF < num_kb) {
-            const int kbp = kb + GEMM_PF;
-            const int ksp = kbp / p.kb_per_shard;
-            const int k0p = (kbp - ksp * p.kb_per_shard) * GEMM_BK;
-            const int a_p = p.a_src == SHARD_K ? ksp : a_s;
-            const int b_p = p.b_src == SHARD_K ? ksp : b_s;
-            if (A_MN && p.a_il) {
-              tma_prefetch_5d(&tmA, 0, 0, am / 64, k0p / 8, a_p);
-            } else if (A_MN) {
-              tma_prefetch_3d(&tmA, am, k0p, a_p);
-              tma_prefetch_3d(&tmA, am + 64, k0p, a_p);
-            } else {
-              tma_prefetch_3d(&tmA, k0p, am, a_p);
-            }
-            if (B_MN && p.b_il) {
-              tma_prefetch_5d(&tmB, 0, 0, bn / 64, k0p / 8, b_p);
-            } else if (B_MN) {
-              tma_prefetch_3d(&tmB, bn, k0p, b_p);
-              tma_prefetch_3d(&tmB, bn + 64, k0p, b_p);
-            } else {
-              tma_prefetch_3d(&tmB, k0p, bn, b_p);
-            }
-          }
           uint8_t* sa = smem + s * GP_STAGE_BYTES;
           uint8_t* sb = sa + GP_A_BYTES;
           if (leader) mbar_arrive_expect_tx(&full[s], 2 * GP_STAGE_BYTES);
