@@ -457,10 +457,11 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q128,
 // =====================================================================================
 // Dv = rowsum(dO * O) and lse2 = lse * log2(e) for every (batch, head, query),
 // written with rows padded to S_pad: padded queries get lse2 = +inf, Dv = 0.
-// dh/8 consecutive threads share one row (8 elements each, one 16-byte load
-// of O and of dO) and reduce with shuffles, so a warp reads whole rows.  The
-// grid strides over groups of PREP_ROWS rows per thread group, whose loads
-// are all issued before any of them is reduced.
+// Block (x, y) covers queries [x * 16 * PREP_ROWS, ...) of batch-head y (b =
+// y / H, h = y % H), so the head's shard and column offset are computed once
+// per block.  dh/8 consecutive threads share one row (8 elements each, one
+// 16-byte load of O and of dO) and reduce with shuffles, so a warp reads whole
+// rows; a thread group's PREP_ROWS rows are loaded before any is reduced.
 constexpr int PREP_ROWS = 4;
 
 __global__ void __launch_bounds__(256)
@@ -469,52 +470,39 @@ attn_bwd_prep_kernel(const uint16_t* __restrict__ o, const uint16_t* __restrict_
                      float* __restrict__ lse2, int B, int S, int S_pad, int H, int Ht, int dh,
                      int Dt, long long T) {
   const int tpr = dh >> 3;                    // threads per row: 8 or 16
-  const int rpb = blockDim.x / tpr;           // rows per block and group
-  const int sub = threadIdx.x % tpr;
-  const long long nrows = (long long)B * H * S_pad;
-  for (long long base = (long long)blockIdx.x * rpb * PREP_ROWS; base < nrows;
-       base += (long long)gridDim.x * rpb * PREP_ROWS) {
-    uint4 av[PREP_ROWS], gv[PREP_ROWS];
-    long long row[PREP_ROWS];
-    bool live[PREP_ROWS];
+  const int rpb = blockDim.x / tpr;           // rows per group
+  const int sub = threadIdx.x & (tpr - 1);
+  const int bh = blockIdx.y;
+  const int b = bh / H, h = bh - b * H;
+  const int shard = h / Ht, hl = h - shard * Ht;
+  const long long head_base = (long long)shard * T * Dt + (long long)b * S * Dt + hl * dh + sub * 8;
+  const long long vrow = (long long)bh * S_pad;
+  const int s0 = blockIdx.x * rpb * PREP_ROWS + threadIdx.x / tpr;
+  uint4 av[PREP_ROWS], gv[PREP_ROWS];
 #pragma unroll
-    for (int u = 0; u < PREP_ROWS; ++u) {
-      row[u] = base + (long long)u * rpb + threadIdx.x / tpr;
-      const bool in = row[u] < nrows;
-      const int s = in ? (int)(row[u] % S_pad) : 0;
-      live[u] = in && s < S;
-      if (live[u]) {
-        const long long bh = row[u] / S_pad;
-        const int h = (int)(bh % H);
-        const int b = (int)(bh / H);
-        const int shard = h / Ht, hl = h - shard * Ht;
-        const long long off =
-            (long long)shard * T * Dt + ((long long)b * S + s) * Dt + hl * dh + sub * 8;
-        av[u] = *reinterpret_cast<const uint4*>(o + off);
-        gv[u] = *reinterpret_cast<const uint4*>(dout + off);
-      }
+  for (int u = 0; u < PREP_ROWS; ++u) {
+    const int s = s0 + u * rpb;
+    if (s < S) {
+      const long long off = head_base + (long long)s * Dt;
+      av[u] = *reinterpret_cast<const uint4*>(o + off);
+      gv[u] = *reinterpret_cast<const uint4*>(dout + off);
     }
+  }
 #pragma unroll
-    for (int u = 0; u < PREP_ROWS; ++u) {
-      float acc = 0.f;
-      if (live[u]) {
-        const uint32_t wa[4] = {av[u].x, av[u].y, av[u].z, av[u].w};
-        const uint32_t wg[4] = {gv[u].x, gv[u].y, gv[u].z, gv[u].w};
+  for (int u = 0; u < PREP_ROWS; ++u) {
+    const int s = s0 + u * rpb;
+    float acc = 0.f;
+    if (s < S) {
+      const uint32_t wa[4] = {av[u].x, av[u].y, av[u].z, av[u].w};
+      const uint32_t wg[4] = {gv[u].x, gv[u].y, gv[u].z, gv[u].w};
 #pragma unroll
-        for (int k = 0; k < 4; ++k)
-          acc += bf16_lo(wa[k]) * f16_lo(wg[k]) + bf16_hi(wa[k]) * f16_hi(wg[k]);
-      }
-      for (int m = tpr >> 1; m > 0; m >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, m);
-      if (row[u] < nrows && sub == 0) {
-        if (!live[u]) {
-          dvec[row[u]] = 0.f;
-          lse2[row[u]] = INFINITY;
-        } else {
-          const long long bh = row[u] / S_pad;
-          dvec[row[u]] = acc;
-          lse2[row[u]] = lse[bh * S + row[u] % S_pad] * kLog2e;
-        }
-      }
+      for (int k = 0; k < 4; ++k)
+        acc += bf16_lo(wa[k]) * f16_lo(wg[k]) + bf16_hi(wa[k]) * f16_hi(wg[k]);
+    }
+    for (int m = tpr >> 1; m > 0; m >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, m);
+    if (s < S_pad && sub == 0) {
+      dvec[vrow + s] = s < S ? acc : 0.f;
+      lse2[vrow + s] = s < S ? lse[(long long)bh * S + s] * kLog2e : INFINITY;
     }
   }
 }
@@ -1126,14 +1114,12 @@ tp_status bwd_launch(const uint16_t* qkv, const uint16_t* o, const float* lse, c
                      uint16_t* dqkv, const AttnArgs& a, void* scratch, cudaStream_t st) {
   float* dvec = static_cast<float*>(scratch);
   float* lse2 = dvec + (size_t)a.B * a.H * a.S_pad;
-  const long long n = (long long)a.B * a.H * a.S_pad;
   {
     TraceScope ts(st, TK_ATTN_BWD_PREP);
-    const long long rows_per_group = 256 / (DH / 8) * PREP_ROWS;
-    long long blocks = (n + rows_per_group - 1) / rows_per_group;
-    if (blocks > 8LL * sm_count()) blocks = 8LL * sm_count();
-    attn_bwd_prep_kernel<<<(unsigned)blocks, 256, 0, st>>>(o, dout, lse, dvec, lse2, a.B, a.S,
-                                                           a.S_pad, a.H, a.Ht, DH, a.Dt, a.T);
+    const int rows_per_block = 256 / (DH / 8) * PREP_ROWS;
+    const dim3 grid((unsigned)((a.S_pad + rows_per_block - 1) / rows_per_block), (unsigned)(a.B * a.H));
+    attn_bwd_prep_kernel<<<grid, 256, 0, st>>>(o, dout, lse, dvec, lse2, a.B, a.S, a.S_pad, a.H,
+                                               a.Ht, DH, a.Dt, a.T);
   }
   if (cudaGetLastError() != cudaSuccess) return TP_ERR_CUDA;
   AttnArgs p = a;
