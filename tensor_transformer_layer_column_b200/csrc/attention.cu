@@ -117,7 +117,7 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, const C
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   while (true) {
-    if (mbar_try_wait_sleep(bar, parity, 20000)) return true;
+    if (mbar_try_wait(bar, parity)) return true;
     if (*c.abort_flag || globaltimer_ns() - t0 > 2000000000ull) {
       *c.abort_flag = 1;
       if (c.err) atomicCAS(c.err, 0u, code);
