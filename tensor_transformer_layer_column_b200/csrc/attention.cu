@@ -181,6 +181,25 @@ static_assert(FwdCfg<128>::SMEM <= 227 * 1024, "forward tile exceeds shared memo
 
 constexpr float kLazyRescaleLog2 = 8.0f;
 
+// Work item of a CTA in a (length index, head, batch) grid, longest first.
+// Blocks start in linear order (x fastest); read as one index, the length
+// index varies slowest, so every CTA of the first length index (the longest
+// causal items) starts before any of the next, and the CTAs that start last,
+// filling the tail of the launch, are the shortest.
+struct AttnItem {
+  int x, h, b;
+};
+__device__ __forceinline__ AttnItem attn_item() {
+  const unsigned hb = gridDim.y * gridDim.z;
+  const unsigned lin = blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z);
+  AttnItem it;
+  it.x = (int)(lin / hb);
+  const unsigned r = lin - (unsigned)it.x * hb;
+  it.h = (int)(r % gridDim.y);
+  it.b = (int)(r / gridDim.y);
+  return it;
+}
+
 template <int DH>
 __global__ void __launch_bounds__(352, 1)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q128,
@@ -203,8 +222,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q128,
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nqb = (p.S + 2 * C::BM - 1) / (2 * C::BM);
-  const int qb = p.causal ? nqb - 1 - (int)blockIdx.x : (int)blockIdx.x;
-  const int h = blockIdx.y, b = blockIdx.z;
+  const AttnItem item = attn_item();
+  const int qb = p.causal ? nqb - 1 - item.x : item.x;
+  const int h = item.h, b = item.b;
   const int shard = h / p.Ht, hl = h - shard * p.Ht;
   const int q0 = qb * 2 * C::BM;
   const int nkb = (p.S + C::BN - 1) / C::BN;
@@ -552,7 +572,8 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_kv128,
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int kb = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const AttnItem item = attn_item();   // key block 0 (the longest causal item) first
+  const int kb = item.x, h = item.h, b = item.b;
   const int shard = h / p.Ht, hl = h - shard * p.Ht;
   const int k0 = kb * C::BK;
   const int nqb = (p.S + C::BQ - 1) / C::BQ;
@@ -821,8 +842,9 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q128,
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nqb = (p.S + C::BQ - 1) / C::BQ;
-  const int qb = p.causal ? nqb - 1 - (int)blockIdx.x : (int)blockIdx.x;
-  const int h = blockIdx.y, b = blockIdx.z;
+  const AttnItem item = attn_item();
+  const int qb = p.causal ? nqb - 1 - item.x : item.x;
+  const int h = item.h, b = item.b;
   const int shard = h / p.Ht, hl = h - shard * p.Ht;
   const int q0 = qb * C::BQ;
   const int nkb = (p.S + C::BK - 1) / C::BK;
