@@ -265,6 +265,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q128,
   tc_fence_after();
   // TMEM columns: S of tile i at 64i, O of tile i at 128 + 128i, P of tile i at 384 + 32i.
   const uint32_t tmem = *tmem_slot;
+  grid_dep_wait();   // inputs and outputs: the previous kernels have completed
+  grid_dep_launch();
 
   if (warp == 0) {
     if (lane == 0) {
@@ -489,6 +491,8 @@ attn_bwd_prep_kernel(const uint16_t* __restrict__ o, const uint16_t* __restrict_
                      const float* __restrict__ lse, float* __restrict__ dvec,
                      float* __restrict__ lse2, int B, int S, int S_pad, int H, int Ht, int dh,
                      int Dt, long long T) {
+  grid_dep_wait();
+  grid_dep_launch();
   const int tpr = dh >> 3;                    // threads per row: 8 or 16
   const int rpb = blockDim.x / tpr;           // rows per group
   const int sub = threadIdx.x & (tpr - 1);
@@ -606,6 +610,8 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_kv128,
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  grid_dep_wait();   // inputs and outputs: the previous kernels have completed
+  grid_dep_launch();
   // buffer j: S^T at 128j, dP^T at 128j + 64; dV at 256, dK at 384 (DH <= 128)
   const uint32_t t_dv = tmem + 256, t_dk = tmem + 256 + DH;
 
@@ -876,6 +882,8 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q128,
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  grid_dep_wait();   // inputs and outputs: the previous kernels have completed
+  grid_dep_launch();
   // TMEM columns: buffer j holds S at 128j, dP at 128j + 64 and dS (fp16 pairs)
   // at 384 + 32j; dQ accumulates at 256.
   const uint32_t t_dq = tmem + 256;
@@ -1126,7 +1134,9 @@ tp_status fwd_launch(const uint16_t* qkv, uint16_t* o, float* lse, const AttnArg
   const dim3 grid((a.S + 255) / 256, a.H, a.B);
   {
     TraceScope ts(st, TK_ATTN_FWD, 4.0 * DH * core_pairs(a));
-    kern<<<grid, FwdCfg<DH>::THREADS, FwdCfg<DH>::SMEM, st>>>(tq, tkv, p);
+    if (launch_pdl(kern, grid, dim3(FwdCfg<DH>::THREADS), FwdCfg<DH>::SMEM, st, tq, tkv, p) !=
+        cudaSuccess)
+      return TP_ERR_CUDA;
   }
   return cuda_status(cudaGetLastError());
 }
@@ -1140,8 +1150,9 @@ tp_status bwd_launch(const uint16_t* qkv, const uint16_t* o, const float* lse, c
     TraceScope ts(st, TK_ATTN_BWD_PREP);
     const int rows_per_block = 256 / (DH / 8) * PREP_ROWS;
     const dim3 grid((unsigned)((a.S_pad + rows_per_block - 1) / rows_per_block), (unsigned)(a.B * a.H));
-    attn_bwd_prep_kernel<<<grid, 256, 0, st>>>(o, dout, lse, dvec, lse2, a.B, a.S, a.S_pad, a.H,
-                                               a.Ht, DH, a.Dt, a.T);
+    if (launch_pdl(attn_bwd_prep_kernel, grid, dim3(256), 0, st, o, dout, lse, dvec, lse2, a.B, a.S,
+                   a.S_pad, a.H, a.Ht, DH, a.Dt, a.T) != cudaSuccess)
+      return TP_ERR_CUDA;
   }
   if (cudaGetLastError() != cudaSuccess) return TP_ERR_CUDA;
   AttnArgs p = a;
@@ -1163,12 +1174,16 @@ tp_status bwd_launch(const uint16_t* qkv, const uint16_t* o, const float* lse, c
   {
     // dP, dV and dK: three of the backward's four algorithmic products.
     TraceScope ts(st, TK_ATTN_BWD_DKDV, 6.0 * DH * core_pairs(a));
-    k1<<<dim3((a.S + 127) / 128, a.H, a.B), 352, DkdvCfg<DH>::SMEM, st>>>(kv128, q64, do64, p);
+    if (launch_pdl(k1, dim3((a.S + 127) / 128, a.H, a.B), dim3(352), DkdvCfg<DH>::SMEM, st, kv128,
+                   q64, do64, p) != cudaSuccess)
+      return TP_ERR_CUDA;
   }
   if (cudaGetLastError() != cudaSuccess) return TP_ERR_CUDA;
   {
     TraceScope ts(st, TK_ATTN_BWD_DQ, 2.0 * DH * core_pairs(a));
-    k2<<<dim3((a.S + 127) / 128, a.H, a.B), 352, DqCfg<DH>::SMEM, st>>>(q128, do128, kv64, p);
+    if (launch_pdl(k2, dim3((a.S + 127) / 128, a.H, a.B), dim3(352), DqCfg<DH>::SMEM, st, q128,
+                   do128, kv64, p) != cudaSuccess)
+      return TP_ERR_CUDA;
   }
   return cuda_status(cudaGetLastError());
 }

@@ -95,11 +95,13 @@ tp_status launch_pair(const CUtensorMap& ta, const CUtensorMap& tb, const GemmAr
   cudaGetDevice(&dev);
   auto kern = gemm_pair_sm100<A_MN, B_MN>;
   cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;   // see launch_pdl
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.blockDim = dim3(GEMM_THREADS, 1, 1);
   cfg.dynamicSmemBytes = GP_SMEM_BYTES;
   cfg.stream = stream;
@@ -117,6 +119,7 @@ tp_status launch_pair(const CUtensorMap& ta, const CUtensorMap& tb, const GemmAr
   }
   const int clusters = args.num_tiles < max_clusters[dev] ? args.num_tiles : max_clusters[dev];
   cfg.gridDim = dim3(2 * clusters, 1, 1);
+  cfg.numAttrs = 2;
   {
     TraceScope ts(stream, TK_GEMM, flops);
     if (cudaLaunchKernelEx(&cfg, kern, ta, tb, args) != cudaSuccess) return TP_ERR_CUDA;

@@ -37,6 +37,7 @@
 #include <cuda_bf16.h>
 #include <cstdint>
 
+#include "pdl.cuh"
 #include "sm100_ptx.cuh"
 
 namespace tp {
@@ -583,6 +584,8 @@ gemm_pair_sm100(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
   const uint32_t tmem_base = *tmem_slot;
   const int num_kb = p.k_shards * p.kb_per_shard;
   const int cid = (int)cluster_id_x(), ncl = (int)nclusters_x();
+  grid_dep_wait();                  // operands and outputs: the previous kernels have completed
+  grid_dep_launch();
 
   if (warp == 0) {
     if (lane == 0) {

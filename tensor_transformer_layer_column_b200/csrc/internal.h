@@ -4,7 +4,9 @@
 #include <cuda_runtime.h>
 #include <cstddef>
 #include <cstdint>
+#include <utility>
 
+#include "pdl.cuh"
 #include "tp_layer.h"
 
 namespace tp {
@@ -43,6 +45,23 @@ struct GemmProblem {
 };
 
 tp_status launch_gemm(const GemmProblem& g, cudaStream_t stream);
+
+// Launch with the programmatic-serialization attribute (see pdl.cuh).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t st, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
 
 // Host validation of tp_dims shared by the entry points (status before any launch).
 tp_status check_common(const tp_dims* d);

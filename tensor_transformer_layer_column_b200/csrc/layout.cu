@@ -81,6 +81,8 @@ __global__ void copy_kernel(const uint16_t* __restrict__ src, uint16_t* __restri
 // bf16 -> fp16, 8 elements per thread step; out-of-range values flag `err`.
 __global__ void cast_f16_kernel(const uint16_t* __restrict__ src, uint16_t* __restrict__ dst,
                                 long long n8, unsigned int* err) {
+  grid_dep_wait();
+  grid_dep_launch();
   bool over = false;
   for (long long v = blockIdx.x * (long long)blockDim.x + threadIdx.x; v < n8;
        v += (long long)gridDim.x * blockDim.x) {
@@ -150,8 +152,9 @@ tp_status launch_cast_f16(const uint16_t* src, size_t n, uint16_t* dst, cudaStre
   if (n == 0) return TP_OK;
   if (n % 8 || !aligned16(src) || !aligned16(dst)) return TP_ERR_MISALIGNED;
   TraceScope ts(stream, TK_CAST);
-  cast_f16_kernel<<<grid_for((long long)n / 8), 256, 0, stream>>>(src, dst, (long long)n / 8,
-                                                                  error_word());
+  if (launch_pdl(cast_f16_kernel, dim3(grid_for((long long)n / 8)), dim3(256), 0, stream, src, dst,
+                 (long long)n / 8, error_word()) != cudaSuccess)
+    return TP_ERR_CUDA;
   return cuda_status(cudaGetLastError());
 }
 

@@ -73,6 +73,8 @@ ln_fwd_kernel(const uint16_t* __restrict__ x, const uint16_t* __restrict__ g,
               const uint16_t* __restrict__ b, long long rows, int D, float eps,
               uint16_t* __restrict__ y, float* __restrict__ mean, float* __restrict__ rstd,
               unsigned int* err) {
+  grid_dep_wait();
+  grid_dep_launch();
   const int lane = threadIdx.x & 31;
   const int nch = D >> 3;
   const long long nwarps = (long long)gridDim.x * (blockDim.x >> 5);
@@ -178,6 +180,8 @@ ln_bwd_kernel(const void* __restrict__ dy, const uint16_t* __restrict__ x,
               const float* __restrict__ rstd, const uint16_t* __restrict__ dres, long long rows,
               int D, int rows_per_block, uint16_t* __restrict__ dx, float* __restrict__ partial,
               float* __restrict__ dx32 = nullptr) {
+  grid_dep_wait();
+  grid_dep_launch();
   __shared__ float red[2][2][LNB_THREADS / 32];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int nch = D >> 3;
@@ -331,6 +335,8 @@ __device__ __forceinline__ float reduce_rows_fixed(const float* __restrict__ row
 __global__ void __launch_bounds__(256)
 ln_param_reduce(const float* __restrict__ partial, int nblocks, int D, int nk,
                 uint16_t* __restrict__ dg, uint16_t* __restrict__ db, uint16_t* __restrict__ dr) {
+  grid_dep_wait();
+  grid_dep_launch();
   __shared__ float red[8][33];
   const long long width = (long long)nk * D;
   const float t = reduce_rows_fixed(partial, nblocks, width, width, red);
@@ -391,6 +397,8 @@ colsum_partial_kernel(const uint16_t* __restrict__ x, long long rows, long long 
 __global__ void __launch_bounds__(256)
 colsum_reduce_kernel(const float* __restrict__ partial, int chunks, long long cols,
                      uint16_t* __restrict__ out) {
+  grid_dep_wait();
+  grid_dep_launch();
   __shared__ float red[8][33];
   const long long s = blockIdx.y;
   const float t = reduce_rows_fixed(partial + s * chunks * cols, chunks, cols, cols, red);
@@ -452,7 +460,8 @@ tp_status launch_colsum_reduce(const float* partial, long long rows, long long c
   if (rows == 0) return cuda_status(cudaMemsetAsync(out, 0, (size_t)cols * 2, stream));
   TraceScope ts(stream, TK_COLSUM);
   const dim3 g2((unsigned)((cols + 31) / 32), 1, 1);
-  colsum_reduce_kernel<<<g2, 256, 0, stream>>>(partial, (int)rows, cols, out);
+  launch_pdl(colsum_reduce_kernel, g2, dim3(256), 0, stream, (const float*)partial, (int)rows, cols,
+             out);
   return cuda_status(cudaGetLastError());
 }
 
@@ -467,17 +476,23 @@ tp_status ln_fwd_dispatch(const uint16_t* x, const uint16_t* g, const uint16_t* 
   unsigned int* err = error_word();
   TraceScope ts(stream, TK_LN_FWD);
   if (per_lane <= 1)
-    ln_fwd_kernel<1, F16OUT><<<grid, 256, 0, stream>>>(x, g, b, rows, D, eps, y, mean, rstd, err);
+    launch_pdl(ln_fwd_kernel<1, F16OUT>, dim3(grid), dim3(256), 0, stream, x, g, b, rows, D, eps, y,
+               mean, rstd, err);
   else if (per_lane <= 2)
-    ln_fwd_kernel<2, F16OUT><<<grid, 256, 0, stream>>>(x, g, b, rows, D, eps, y, mean, rstd, err);
+    launch_pdl(ln_fwd_kernel<2, F16OUT>, dim3(grid), dim3(256), 0, stream, x, g, b, rows, D, eps, y,
+               mean, rstd, err);
   else if (per_lane <= 4)
-    ln_fwd_kernel<4, F16OUT><<<grid, 256, 0, stream>>>(x, g, b, rows, D, eps, y, mean, rstd, err);
+    launch_pdl(ln_fwd_kernel<4, F16OUT>, dim3(grid), dim3(256), 0, stream, x, g, b, rows, D, eps, y,
+               mean, rstd, err);
   else if (per_lane <= 8)
-    ln_fwd_kernel<8, F16OUT><<<grid, 256, 0, stream>>>(x, g, b, rows, D, eps, y, mean, rstd, err);
+    launch_pdl(ln_fwd_kernel<8, F16OUT>, dim3(grid), dim3(256), 0, stream, x, g, b, rows, D, eps, y,
+               mean, rstd, err);
   else if (per_lane <= 16)
-    ln_fwd_kernel<16, F16OUT><<<grid, 256, 0, stream>>>(x, g, b, rows, D, eps, y, mean, rstd, err);
+    launch_pdl(ln_fwd_kernel<16, F16OUT>, dim3(grid), dim3(256), 0, stream, x, g, b, rows, D, eps, y,
+               mean, rstd, err);
   else if (per_lane <= 32)
-    ln_fwd_kernel<32, F16OUT><<<grid, 256, 0, stream>>>(x, g, b, rows, D, eps, y, mean, rstd, err);
+    launch_pdl(ln_fwd_kernel<32, F16OUT>, dim3(grid), dim3(256), 0, stream, x, g, b, rows, D, eps, y,
+               mean, rstd, err);
   else
     return TP_ERR_UNSUPPORTED;
   return cuda_status(cudaGetLastError());
@@ -502,11 +517,11 @@ void ln_bwd_kernel_launch(bool rsum, int nb, const void* dy, const uint16_t* x, 
                           long long rows, int D, int rpb, uint16_t* dx, float* partial,
                           float* dx32, cudaStream_t stream) {
   if (rsum)
-    ln_bwd_kernel<CH, DY32, true><<<nb, LNB_THREADS, 0, stream>>>(dy, x, g, mean, rstd, dres, rows,
-                                                                   D, rpb, dx, partial, dx32);
+    launch_pdl(ln_bwd_kernel<CH, DY32, true>, dim3(nb), dim3(LNB_THREADS), 0, stream, dy, x, g, mean,
+               rstd, dres, rows, D, rpb, dx, partial, dx32);
   else
-    ln_bwd_kernel<CH, DY32, false><<<nb, LNB_THREADS, 0, stream>>>(dy, x, g, mean, rstd, dres,
-                                                                    rows, D, rpb, dx, partial, dx32);
+    launch_pdl(ln_bwd_kernel<CH, DY32, false>, dim3(nb), dim3(LNB_THREADS), 0, stream, dy, x, g,
+               mean, rstd, dres, rows, D, rpb, dx, partial, dx32);
 }
 
 // dr (may be NULL; needs dres): column sums of dres, from a third partial row.
@@ -542,7 +557,8 @@ tp_status ln_bwd_launch(const void* dy, const uint16_t* x, const uint16_t* g, co
   if (dg != nullptr || db != nullptr || dr != nullptr) {
     TraceScope ts(stream, TK_LN_PARAM);
     const int nk = rsum ? 3 : 2;
-    ln_param_reduce<<<(nk * D + 31) / 32, 256, 0, stream>>>(partial, nb, D, nk, dg, db, dr);
+    launch_pdl(ln_param_reduce, dim3((nk * D + 31) / 32), dim3(256), 0, stream, (const float*)partial,
+               nb, D, nk, dg, db, dr);
   }
   return cuda_status(cudaGetLastError());
 }
