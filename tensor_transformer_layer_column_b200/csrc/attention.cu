@@ -555,8 +555,38 @@ struct DkdvCfg {
 };
 static_assert(DkdvCfg<128>::SMEM <= 227 * 1024, "dK/dV tile exceeds shared memory");
 
+// Work item i of the dK/dV launch: (key block, head, batch), the key block
+// varying slowest, so that in item order the longest causal items come first.
+struct DkdvItem {
+  int kb, h, b;
+};
+__device__ __forceinline__ DkdvItem dkdv_item(int i, int H, int B) {
+  const int hb = H * B;
+  DkdvItem it;
+  it.kb = i / hb;
+  const int r = i - it.kb * hb;
+  it.h = r % H;
+  it.b = r / H;
+  return it;
+}
+
+constexpr int DKDV_THREADS = 480;
+
+// Persistent: one CTA per SM walks the items i = blockIdx.x, +gridDim.x, ...
+// Warp roles: 0 loads (K/V per item, q/dO/lse2/Dv per 64-query block), 1
+// issues the score products S^T = K q^T and dP^T = V dO^T, 2-9 are two
+// compute warpgroups (P^T, dS^T), 10 issues dV += P^T dO and dK += dS^T q,
+// 11-14 are the epilogue (dV, dK out of tensor memory to global, and their
+// column partials).  The block counter g runs over all items of the CTA, so
+// the stage ring and the two score buffers carry on from one item to the
+// next: the next item's K/V load and first score products overlap the
+// current item's last products and its epilogue, and the epilogue overlaps
+// the next item's first blocks.  Per item: kv_full / kv_empty guard K and V
+// (reloaded once the item's last score products completed), acc_full /
+// acc_empty guard the dV/dK accumulators (the next item's first products wait
+// until the epilogue warps have read them out).
 template <int DH>
-__global__ void __launch_bounds__(352, 1)
+__global__ void __launch_bounds__(DKDV_THREADS, 1)
 attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_kv128,
                      const __grid_constant__ CUtensorMap tm_q64,
                      const __grid_constant__ CUtensorMap tm_do64, const AttnArgs p) {
@@ -571,21 +601,39 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_kv128,
   uint64_t* s_full = bars + 9;     // [2] per TMEM buffer
   uint64_t* p_full = bars + 11;    // [2]
   uint64_t* mm2_done = bars + 13;  // [2]
-  uint64_t* drain = bars + 15;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
+  uint64_t* kv_empty = bars + 15;  // the item's score products completed: K/V reusable
+  uint64_t* acc_full = bars + 16;  // the item's dV/dK complete
+  uint64_t* acc_empty = bars + 17; // the epilogue has read dV/dK out
+  uint64_t* drain = bars + 18;     // [2] each issuer's products completed
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 20);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const AttnItem item = attn_item();   // key block 0 (the longest causal item) first
-  const int kb = item.x, h = item.h, b = item.b;
-  const int shard = h / p.Ht, hl = h - shard * p.Ht;
-  const int k0 = kb * C::BK;
+  const int nkb = (p.S + C::BK - 1) / C::BK;
+  const int nitems = nkb * p.H * p.B;
   const int nqb = (p.S + C::BQ - 1) / C::BQ;
-  const int i0 = p.causal ? k0 / C::BQ : 0;
-  const int nsteps = nqb - i0;
-  const int colq = hl * DH, colk = p.Dt + hl * DH, colv = 2 * p.Dt + hl * DH, cold = hl * DH;
-  const long long hrow = ((long long)b * p.H + h) * p.S_pad;
   const Ctl ctl{abort_flag, p.err};
+  // Per-item geometry.
+  struct Geo {
+    int b, shard, k0, i0, nsteps, colq, colk, colv, cold;
+    long long hrow;
+  };
+  auto geo = [&](int i) {
+    const DkdvItem it = dkdv_item(i, p.H, p.B);
+    Geo g;
+    g.b = it.b;
+    g.shard = it.h / p.Ht;
+    const int hl = it.h - g.shard * p.Ht;
+    g.k0 = it.kb * C::BK;
+    g.i0 = p.causal ? g.k0 / C::BQ : 0;
+    g.nsteps = nqb - g.i0;
+    g.colq = hl * DH;
+    g.colk = p.Dt + hl * DH;
+    g.colv = 2 * p.Dt + hl * DH;
+    g.cold = hl * DH;
+    g.hrow = ((long long)it.b * p.H + it.h) * p.S_pad;
+    return g;
+  };
 
   if (threadIdx.x == 0) {
     mbar_init(kv_full, 1);
@@ -597,8 +645,11 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_kv128,
       mbar_init(&s_full[i], 1);
       mbar_init(&p_full[i], 128);   // buffer i belongs to compute warpgroup i
       mbar_init(&mm2_done[i], 1);
+      mbar_init(&drain[i], 1);
     }
-    mbar_init(drain, 1);
+    mbar_init(kv_empty, 1);
+    mbar_init(acc_full, 1);
+    mbar_init(acc_empty, 4);        // one arrival per epilogue warp
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -617,159 +668,206 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_kv128,
 
   if (warp == 0) {
     if (lane == 0) {
-      mbar_arrive_expect_tx(kv_full, 2 * C::K_BYTES);
-      for (int c = 0; c < C::CH; ++c) {
-        tma_load_4d(smem + C::OFF_K + c * C::BK * 128, &tm_kv128, kv_full, colk + 64 * c, k0, b, shard);
-        tma_load_4d(smem + C::OFF_V + c * C::BK * 128, &tm_kv128, kv_full, colv + 64 * c, k0, b, shard);
-      }
-      int k = 0;
-      for (; k < nsteps; ++k) {
-        const int st = k % C::STAGES;
-        const uint32_t u = k / C::STAGES;
-        if (!wait_bar(&qd_empty[st], (u & 1) ^ 1, ctl, ERR_ATTN_DKDV_WAIT)) break;
-        uint8_t* sq = smem + C::OFF_ST + st * C::STAGE_BYTES;
-        uint8_t* sd = sq + C::Q_BYTES;
-        uint8_t* sv = smem + C::OFF_VEC + st * 2 * C::VEC_BYTES;
-        const int qs = (i0 + k) * C::BQ;
-        mbar_arrive_expect_tx(&qd_full[st], 2 * C::Q_BYTES + 2 * C::VEC_BYTES);
+      int g = 0, n = 0, nkv = 0;
+      bool ok = true;
+      for (int it = blockIdx.x; ok && it < nitems; it += gridDim.x, ++n) {
+        const Geo q = geo(it);
+        // K and V of the previous item are free once its score products completed.
+        if (!(ok = wait_bar(kv_empty, (n & 1) ^ 1, ctl, ERR_ATTN_DKDV_WAIT))) break;
+        mbar_arrive_expect_tx(kv_full, 2 * C::K_BYTES);
         for (int c = 0; c < C::CH; ++c) {
-          tma_load_4d(sq + c * C::BQ * 128, &tm_q64, &qd_full[st], colq + 64 * c, qs, b, shard);
-          tma_load_4d(sd + c * C::BQ * 128, &tm_do64, &qd_full[st], cold + 64 * c, qs, b, shard);
+          tma_load_4d(smem + C::OFF_K + c * C::BK * 128, &tm_kv128, kv_full, q.colk + 64 * c, q.k0,
+                      q.b, q.shard);
+          tma_load_4d(smem + C::OFF_V + c * C::BK * 128, &tm_kv128, kv_full, q.colv + 64 * c, q.k0,
+                      q.b, q.shard);
         }
-        bulk_load(sv, p.lse2 + hrow + qs, C::VEC_BYTES, &qd_full[st]);
-        bulk_load(sv + C::VEC_BYTES, p.dvec + hrow + qs, C::VEC_BYTES, &qd_full[st]);
+        ++nkv;
+        for (int k = 0; k < q.nsteps; ++k, ++g) {
+          const int st = g % C::STAGES;
+          const uint32_t u = g / C::STAGES;
+          if (!(ok = wait_bar(&qd_empty[st], (u & 1) ^ 1, ctl, ERR_ATTN_DKDV_WAIT))) break;
+          uint8_t* sq = smem + C::OFF_ST + st * C::STAGE_BYTES;
+          uint8_t* sd = sq + C::Q_BYTES;
+          uint8_t* sv = smem + C::OFF_VEC + st * 2 * C::VEC_BYTES;
+          const int qs = (q.i0 + k) * C::BQ;
+          mbar_arrive_expect_tx(&qd_full[st], 2 * C::Q_BYTES + 2 * C::VEC_BYTES);
+          for (int c = 0; c < C::CH; ++c) {
+            tma_load_4d(sq + c * C::BQ * 128, &tm_q64, &qd_full[st], q.colq + 64 * c, qs, q.b,
+                        q.shard);
+            tma_load_4d(sd + c * C::BQ * 128, &tm_do64, &qd_full[st], q.cold + 64 * c, qs, q.b,
+                        q.shard);
+          }
+          bulk_load(sv, p.lse2 + q.hrow + qs, C::VEC_BYTES, &qd_full[st]);
+          bulk_load(sv + C::VEC_BYTES, p.dvec + q.hrow + qs, C::VEC_BYTES, &qd_full[st]);
+        }
       }
-      mbar_wait(kv_full, 0, 200000000ull);
-      for (int i = k - 1; i >= 0 && i >= k - C::STAGES; --i)
+      // Copies still in flight land in this CTA's shared memory: wait for them
+      // (bounded) before the CTA may exit: nkv K/V loads and stages 0 .. g-1.
+      if (nkv > 0) mbar_wait(kv_full, (uint32_t)((nkv - 1) & 1), 200000000ull);
+      for (int i = g - 1; i >= 0 && i >= g - C::STAGES; --i)
         mbar_wait(&qd_full[i % C::STAGES], (i / C::STAGES) & 1, 200000000ull);
     }
   } else if (warp == 1 || warp == 10) {
     // Two issuers, each blocking only on its own barriers: warp 1 issues
-    // S^T/dP^T of block k (once its q/dO stage has landed and the dV/dK MMAs
-    // of block k-2 have read P^T/dS^T out of the same buffer), warp 10 issues
-    // dV/dK of block k (once its P^T/dS^T are in tensor memory) and releases
+    // S^T/dP^T of block g (once its q/dO stage has landed and the dV/dK MMAs
+    // of block g-2 have read P^T/dS^T out of the same buffer), warp 10 issues
+    // dV/dK of block g (once its P^T/dS^T are in tensor memory) and releases
     // the stage.  Neither stream waits behind the other.
     if (lane == 0) {
       constexpr uint32_t id_s = idesc_f32acc(128, C::BQ, false, false, true);
       constexpr uint32_t id_acc = idesc_f32acc(128, DH, false, true, true);
       const uint32_t sk = smem_u32(smem + C::OFF_K), sv = smem_u32(smem + C::OFF_V);
-      bool ok = wait_bar(kv_full, 0, ctl, ERR_ATTN_DKDV_WAIT);
+      int g = 0, n = 0;
+      bool ok = true;
       if (warp == 1) {
-        for (int k = 0; ok && k < nsteps; ++k) {
-          const int bf = k & 1, st = k % C::STAGES;
-          if (!(ok = wait_bar(&qd_full[st], (k / C::STAGES) & 1, ctl, ERR_ATTN_DKDV_WAIT))) break;
-          if (!(ok = wait_bar(&mm2_done[bf], ((k >> 1) & 1) ^ 1, ctl, ERR_ATTN_DKDV_WAIT))) break;
-          tc_fence_after();
-          const uint32_t sq = smem_u32(smem + C::OFF_ST + st * C::STAGE_BYTES);
-          const uint32_t sd = sq + C::Q_BYTES;
+        for (int it = blockIdx.x; ok && it < nitems; it += gridDim.x, ++n) {
+          const int nsteps = geo(it).nsteps;
+          if (!(ok = wait_bar(kv_full, n & 1, ctl, ERR_ATTN_DKDV_WAIT))) break;
+          for (int k = 0; k < nsteps; ++k, ++g) {
+            const int bf = g & 1, st = g % C::STAGES;
+            if (!(ok = wait_bar(&qd_full[st], (g / C::STAGES) & 1, ctl, ERR_ATTN_DKDV_WAIT))) break;
+            if (!(ok = wait_bar(&mm2_done[bf], ((g >> 1) & 1) ^ 1, ctl, ERR_ATTN_DKDV_WAIT))) break;
+            tc_fence_after();
+            const uint32_t sq = smem_u32(smem + C::OFF_ST + st * C::STAGE_BYTES);
+            const uint32_t sd = sq + C::Q_BYTES;
 #pragma unroll
-          for (int kk = 0; kk < DH / 16; ++kk) {
-            tc_mma_f16(tmem + bf * 128, kmajor_desc(sk, C::BK, kk), kmajor_desc(sq, C::BQ, kk), id_s,
-                       kk > 0);
-            tc_mma_f16(tmem + bf * 128 + 64, kmajor_desc(sv, C::BK, kk), kmajor_desc(sd, C::BQ, kk),
-                       id_s, kk > 0);
+            for (int kk = 0; kk < DH / 16; ++kk) {
+              tc_mma_f16(tmem + bf * 128, kmajor_desc(sk, C::BK, kk), kmajor_desc(sq, C::BQ, kk),
+                         id_s, kk > 0);
+              tc_mma_f16(tmem + bf * 128 + 64, kmajor_desc(sv, C::BK, kk),
+                         kmajor_desc(sd, C::BQ, kk), id_s, kk > 0);
+            }
+            tc_commit(&s_full[bf]);
           }
-          tc_commit(&s_full[bf]);
+          if (!ok) break;
+          tc_commit(kv_empty);   // K/V may be reloaded once this item's score products completed
         }
+        tc_commit(&drain[0]);
+        mbar_wait(&drain[0], 0, 200000000ull);
       } else {
-        for (int k = 0; ok && k < nsteps; ++k) {
-          const int bj = k & 1, sj = k % C::STAGES;
-          if (!(ok = wait_bar(&p_full[bj], (k >> 1) & 1, ctl, ERR_ATTN_DKDV_WAIT))) break;
-          tc_fence_after();
-          const uint32_t sq = smem_u32(smem + C::OFF_ST + sj * C::STAGE_BYTES);
-          const uint32_t sd = sq + C::Q_BYTES;
+        for (int it = blockIdx.x; ok && it < nitems; it += gridDim.x, ++n) {
+          const int nsteps = geo(it).nsteps;
+          // The first products of an item overwrite dV/dK: the epilogue has read the last item's.
+          if (!(ok = wait_bar(acc_empty, (n & 1) ^ 1, ctl, ERR_ATTN_DKDV_WAIT))) break;
+          for (int k = 0; k < nsteps; ++k, ++g) {
+            const int bj = g & 1, sj = g % C::STAGES;
+            if (!(ok = wait_bar(&p_full[bj], (g >> 1) & 1, ctl, ERR_ATTN_DKDV_WAIT))) break;
+            tc_fence_after();
+            const uint32_t sq = smem_u32(smem + C::OFF_ST + sj * C::STAGE_BYTES);
+            const uint32_t sd = sq + C::Q_BYTES;
 #pragma unroll
-          for (int kk = 0; kk < C::BQ / 16; ++kk) {   // 16 queries = 8 columns per step
-            tc_mma_f16_ts(t_dv, tmem + bj * 128 + 8 * kk, mnmajor_desc(sd, C::BQ, kk), id_acc,
-                          (k | kk) != 0);
-            tc_mma_f16_ts(t_dk, tmem + bj * 128 + 64 + 8 * kk, mnmajor_desc(sq, C::BQ, kk), id_acc,
-                          (k | kk) != 0);
+            for (int kk = 0; kk < C::BQ / 16; ++kk) {   // 16 queries = 8 columns per step
+              tc_mma_f16_ts(t_dv, tmem + bj * 128 + 8 * kk, mnmajor_desc(sd, C::BQ, kk), id_acc,
+                            (k | kk) != 0);
+              tc_mma_f16_ts(t_dk, tmem + bj * 128 + 64 + 8 * kk, mnmajor_desc(sq, C::BQ, kk),
+                            id_acc, (k | kk) != 0);
+            }
+            tc_commit(&mm2_done[bj]);
+            tc_commit(&qd_empty[sj]);   // the scores of block g completed before its P^T existed
           }
-          tc_commit(&mm2_done[bj]);
-          tc_commit(&qd_empty[sj]);   // the scores of block k completed before its P^T existed
+          if (!ok) break;
+          tc_commit(acc_full);
         }
-        tc_commit(drain);
-        mbar_wait(drain, 0, 200000000ull);
+        tc_commit(&drain[1]);
+        mbar_wait(&drain[1], 0, 200000000ull);
       }
     }
-  } else {
-    // Two compute warpgroups: warpgroup g takes the blocks k with k % 2 == g (its
-    // own TMEM and shared buffers), so two blocks are in flight at once; the
-    // epilogue splits the 32-column slices between them.
+  } else if (warp < 10) {
+    // Two compute warpgroups: warpgroup w takes the blocks g with g % 2 == w
+    // (its own TMEM buffer), so two blocks are in flight at once.
     const int wg = (warp - 2) >> 2;
     const int quad = warp & 3;
     const int r = quad * 32 + lane;
-    const int kpos = k0 + r;
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+    int g0 = 0;   // first block counter of the current item
     bool ok = true;
-    for (int k = wg; k < nsteps; k += 2) {
-      const int bf = k & 1;
-      const uint32_t u = k >> 1;
-      const int qs = (i0 + k) * C::BQ;
-      if (!__all_sync(0xffffffffu, wait_bar(&s_full[bf], u & 1, ctl, ERR_ATTN_DKDV_WAIT))) { ok = false; break; }
-      tc_fence_after();
-      const float* vl = reinterpret_cast<const float*>(smem + C::OFF_VEC + (k % C::STAGES) * 2 * C::VEC_BYTES);
-      const float* vd = vl + C::BQ;
-      // S^T and dP^T leave tensor memory in two 32-column halves; P^T and dS^T
-      // of each half (fp16 pairs, 16 columns) are written back over the half
-      // of S^T / dP^T just copied out.  The buffer was free once the dV/dK
-      // MMAs of block k-2 completed, which the score MMAs of this block
-      // already waited for.
-      const uint32_t t_st = tmem + bf * 128 + lane_off;
-      // Queries qs + qi with qi < qmin precede key kpos and are masked (causal):
-      // a select per element, taken only in blocks where some key row of the
-      // warp has a masked query (the causal diagonal).
-      const int qmin = p.causal ? kpos - qs : 0;
-      const bool masked = !__all_sync(0xffffffffu, qmin <= 0);
-      auto half = [&](int c, auto mask_tag) {
-        constexpr bool MASK = decltype(mask_tag)::value;
-        uint32_t rs[32], rd[32];
-        tmem_ld32(t_st + c * 32, rs);
-        tmem_ld32(t_st + 64 + c * 32, rd);
-        tc_wait_ld();
-        uint32_t pk[16], dk[16];   // fp16 pairs of P^T and dS^T
-#pragma unroll
-        for (int e = 0; e < 32; e += 4) {
-          // lse2 and Dv of four queries in one shared-memory load each.
-          const float4 l4 = *reinterpret_cast<const float4*>(vl + c * 32 + e);
-          const float4 d4 = *reinterpret_cast<const float4*>(vd + c * 32 + e);
-          const float la[4] = {l4.x, l4.y, l4.z, l4.w}, da[4] = {d4.x, d4.y, d4.z, d4.w};
-          float pe[4], de[4];
-#pragma unroll
-          for (int h4 = 0; h4 < 4; ++h4) {
-            // Padded queries carry lse2 = +inf and dvec = 0, so they give 0.
-            float x = fast_exp2(fmaf(__uint_as_float(rs[e + h4]), p.scale_log2, -la[h4]));
-            if (MASK) x = c * 32 + e + h4 < qmin ? 0.f : x;
-            pe[h4] = x;
-            de[h4] = x * (__uint_as_float(rd[e + h4]) - da[h4]);
-          }
-          pk[e / 2] = pack_f16x2(pe[0], pe[1]);
-          pk[e / 2 + 1] = pack_f16x2(pe[2], pe[3]);
-          dk[e / 2] = pack_f16x2(de[0], de[1]);
-          dk[e / 2 + 1] = pack_f16x2(de[2], de[3]);
+    for (int it = blockIdx.x; ok && it < nitems; it += gridDim.x) {
+      const Geo q = geo(it);
+      const int kpos = q.k0 + r;
+      for (int k = ((g0 & 1) == wg) ? 0 : 1; k < q.nsteps; k += 2) {
+        const int g = g0 + k;
+        const int bf = g & 1;
+        const uint32_t u = g >> 1;
+        const int qs = (q.i0 + k) * C::BQ;
+        if (!__all_sync(0xffffffffu, wait_bar(&s_full[bf], u & 1, ctl, ERR_ATTN_DKDV_WAIT))) {
+          ok = false;
+          break;
         }
-        tmem_st16(t_st + c * 16, pk);
-        tmem_st16(t_st + 64 + c * 16, dk);
-      };
+        tc_fence_after();
+        const float* vl =
+            reinterpret_cast<const float*>(smem + C::OFF_VEC + (g % C::STAGES) * 2 * C::VEC_BYTES);
+        const float* vd = vl + C::BQ;
+        // S^T and dP^T leave tensor memory in two 32-column halves; P^T and dS^T
+        // of each half (fp16 pairs, 16 columns) are written back over the half
+        // of S^T / dP^T just copied out.  The buffer was free once the dV/dK
+        // MMAs of block g-2 completed, which the score MMAs of this block
+        // already waited for.
+        const uint32_t t_st = tmem + bf * 128 + lane_off;
+        // Queries qs + qi with qi < qmin precede key kpos and are masked (causal):
+        // a select per element, taken only in blocks where some key row of the
+        // warp has a masked query (the causal diagonal).
+        const int qmin = p.causal ? kpos - qs : 0;
+        const bool masked = !__all_sync(0xffffffffu, qmin <= 0);
+        auto half = [&](int c, auto mask_tag) {
+          constexpr bool MASK = decltype(mask_tag)::value;
+          uint32_t rs[32], rd[32];
+          tmem_ld32(t_st + c * 32, rs);
+          tmem_ld32(t_st + 64 + c * 32, rd);
+          tc_wait_ld();
+          uint32_t pk[16], dk[16];   // fp16 pairs of P^T and dS^T
+#pragma unroll
+          for (int e = 0; e < 32; e += 4) {
+            // lse2 and Dv of four queries in one shared-memory load each.
+            const float4 l4 = *reinterpret_cast<const float4*>(vl + c * 32 + e);
+            const float4 d4 = *reinterpret_cast<const float4*>(vd + c * 32 + e);
+            const float la[4] = {l4.x, l4.y, l4.z, l4.w}, da[4] = {d4.x, d4.y, d4.z, d4.w};
+            float pe[4], de[4];
+#pragma unroll
+            for (int h4 = 0; h4 < 4; ++h4) {
+              // Padded queries carry lse2 = +inf and dvec = 0, so they give 0.
+              float x = fast_exp2(fmaf(__uint_as_float(rs[e + h4]), p.scale_log2, -la[h4]));
+              if (MASK) x = c * 32 + e + h4 < qmin ? 0.f : x;
+              pe[h4] = x;
+              de[h4] = x * (__uint_as_float(rd[e + h4]) - da[h4]);
+            }
+            pk[e / 2] = pack_f16x2(pe[0], pe[1]);
+            pk[e / 2 + 1] = pack_f16x2(pe[2], pe[3]);
+            dk[e / 2] = pack_f16x2(de[0], de[1]);
+            dk[e / 2 + 1] = pack_f16x2(de[2], de[3]);
+          }
+          tmem_st16(t_st + c * 16, pk);
+          tmem_st16(t_st + 64 + c * 16, dk);
+        };
 #pragma unroll 1
-      for (int c = 0; c < 2; ++c) {
-        if (masked) half(c, BoolTag<true>{});
-        else half(c, BoolTag<false>{});
+        for (int c = 0; c < 2; ++c) {
+          if (masked) half(c, BoolTag<true>{});
+          else half(c, BoolTag<false>{});
+        }
+        tc_wait_st();
+        tc_fence_before();
+        mbar_arrive(&p_full[bf]);
       }
-      tc_wait_st();
-      tc_fence_before();
-      mbar_arrive(&p_full[bf]);
+      g0 += q.nsteps;
     }
-    // Every product has completed once `drain` (committed after the last one)
-    // completes; waiting on the per-buffer barrier here could alias across its
-    // phases for the warpgroup that did not process the last block.
-    if (ok && __all_sync(0xffffffffu, wait_bar(drain, 0, ctl, ERR_ATTN_DKDV_WAIT))) {
+  } else {
+    // Epilogue warps 11-14 (TMEM lane quarter warp % 4): dV and dK of each
+    // item, once its last products completed, to global memory (fp16, dK
+    // scaled by 1/sqrt(dh)) with their column partials for dbqkv; then the
+    // accumulators are released to the next item.
+    const int quad = warp & 3;
+    const int r = quad * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+    const long long w3 = 3LL * p.Dt;
+    int n = 0;
+    for (int it = blockIdx.x; it < nitems; it += gridDim.x, ++n) {
+      const Geo q = geo(it);
+      if (!__all_sync(0xffffffffu, wait_bar(acc_full, n & 1, ctl, ERR_ATTN_DKDV_WAIT))) break;
       tc_fence_after();
+      const int kpos = q.k0 + r;
       const bool valid = kpos < p.S;
-      const long long w3 = 3LL * p.Dt;
-      uint16_t* row = p.out + (long long)shard * p.T * w3 + ((long long)b * p.S + kpos) * w3;
+      uint16_t* row = p.out + (long long)q.shard * p.T * w3 + ((long long)q.b * p.S + kpos) * w3;
 #pragma unroll 1
-      for (int c = wg; c < DH / 32; c += 2) {
+      for (int c = 0; c < DH / 32; ++c) {
         uint32_t rv[32], rk[32];
         tmem_ld32(t_dv + lane_off + c * 32, rv);
         tmem_ld32(t_dk + lane_off + c * 32, rk);
@@ -786,17 +884,20 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_kv128,
           for (int e = 0; e < 32; ++e) over |= fabsf(v[e]) > 65504.0f || fabsf(kx[e]) > 65504.0f;
 #pragma unroll
           for (int g = 0; g < 4; ++g) {
-            *reinterpret_cast<uint4*>(row + colv + c * 32 + g * 8) = pack8_f16(&v[g * 8]);
-            *reinterpret_cast<uint4*>(row + colk + c * 32 + g * 8) = pack8_f16(&kx[g * 8]);
+            *reinterpret_cast<uint4*>(row + q.colv + c * 32 + g * 8) = pack8_f16(&v[g * 8]);
+            *reinterpret_cast<uint4*>(row + q.colk + c * 32 + g * 8) = pack8_f16(&kx[g * 8]);
           }
           if (over && p.err) atomicCAS(p.err, 0u, 0x301u);
         }
         if (p.colpart != nullptr) {
-          const int s0 = k0 + quad * 32;
-          colpart_store(p, v, b, s0, shard, colv + c * 32);
-          colpart_store(p, kx, b, s0, shard, colk + c * 32);
+          const int s0 = q.k0 + quad * 32;
+          colpart_store(p, v, q.b, s0, q.shard, q.colv + c * 32);
+          colpart_store(p, kx, q.b, s0, q.shard, q.colk + c * 32);
         }
       }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acc_empty);
     }
   }
   tc_fence_before();
@@ -1174,8 +1275,11 @@ tp_status bwd_launch(const uint16_t* qkv, const uint16_t* o, const float* lse, c
   {
     // dP, dV and dK: three of the backward's four algorithmic products.
     TraceScope ts(st, TK_ATTN_BWD_DKDV, 6.0 * DH * core_pairs(a));
-    if (launch_pdl(k1, dim3((a.S + 127) / 128, a.H, a.B), dim3(352), DkdvCfg<DH>::SMEM, st, kv128,
-                   q64, do64, p) != cudaSuccess)
+    // Persistent: one CTA per SM (at most one per work item).
+    const long long items = (long long)((a.S + DkdvCfg<DH>::BK - 1) / DkdvCfg<DH>::BK) * a.H * a.B;
+    const unsigned grid = (unsigned)(items < sm_count() ? items : sm_count());
+    if (launch_pdl(k1, dim3(grid), dim3(DKDV_THREADS), DkdvCfg<DH>::SMEM, st, kv128, q64, do64, p) !=
+        cudaSuccess)
       return TP_ERR_CUDA;
   }
   if (cudaGetLastError() != cudaSuccess) return TP_ERR_CUDA;
