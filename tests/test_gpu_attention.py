@@ -78,6 +78,26 @@ def test_attn_fwd_bwd_small(B, S, H, dh, t, causal, affine):
     _compare(w, inp, o, grads)
 
 
+# More (key block, head, batch) items than SMs, so that each CTA of the
+# persistent dK/dV kernel walks several items of different lengths (causal:
+# 5, 3 and 1 query blocks of 64 at S = 300) and the stage ring, the score
+# buffers and the accumulator hand-over carry from one item to the next.
+MANY_ITEMS = [
+    (4, 300, 32, 64, 4, True),
+    (2, 200, 48, 128, 8, False),
+]
+
+
+@pytest.mark.parametrize("B,S,H,dh,t,causal", MANY_ITEMS)
+def test_attn_fwd_bwd_more_items_than_sms(B, S, H, dh, t, causal):
+    require_gpu()
+    w = Workload("attn_test", "attn_fwdbwd", batch=B, seq=S, hidden=H * dh, heads=H,
+                 head_dim=dh, t=t, causal=causal)
+    inp = make_inputs(w, seed=13, random_affine=True)
+    o, grads = _run(w, inp, backward=True)
+    _compare(w, inp, o, grads)
+
+
 def test_attn_deterministic_run_to_run():
     require_gpu()
     w = Workload("attn_test", "attn_fwdbwd", batch=2, seq=384, hidden=512, heads=4, head_dim=128,
