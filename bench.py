@@ -517,6 +517,10 @@ def run_ours(args):
                     "avg_launch_gflop": fl / n / 1e9,
                     "achieved_at_max_clock": clock_normalised(achieved, clock),
                     "frac_of_nominal": achieved / NOMINAL_BF16_TFLOPS,
+                    # Against the burst and the sustained figure alike, whichever
+                    # the clock record selected for `frac`.
+                    "frac_of_burst": achieved / peaks["bf16_tflops"],
+                    "frac_of_sustained": achieved / peaks["bf16_tflops_sustained"],
                     "traced_steps": traced_steps}
     hbm = hbm_bytes_per_step(w)
     breakdown = {k: {"launches": v[0], "ms_per_step": v[2] / traced_steps,
