@@ -912,6 +912,14 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_kv128,
 // Per 128-query block, walk 64-key blocks through a 4-stage K/V ring.  Two
 // S/dP buffers in TMEM, one per compute warpgroup; dS (fp16 pairs) goes to
 // its own TMEM columns and is the A operand of dQ += dS k.
+//
+// Persistent like the dK/dV kernel: one CTA per SM walks the (query block,
+// head, batch) items longest first (item i, i + #CTAs, ...).  The block
+// counter g runs across the CTA's items, so the K/V ring, the two S/dP
+// buffers and the two dS buffers carry on from item to item; q/dO of the next
+// item load once the item's last score products completed (q_empty), and the
+// next item's first dQ products wait until four epilogue warps have read the
+// accumulator out (acc_full / acc_empty).
 template <int DH>
 struct DqCfg {
   static constexpr int BQ = 128, BK = 64, CH = DH / 64;
@@ -926,8 +934,10 @@ struct DqCfg {
 };
 static_assert(DqCfg<128>::SMEM <= 227 * 1024, "dQ tile exceeds shared memory");
 
+constexpr int DQ_THREADS = 480;
+
 template <int DH>
-__global__ void __launch_bounds__(352, 1)
+__global__ void __launch_bounds__(DQ_THREADS, 1)
 attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q128,
                    const __grid_constant__ CUtensorMap tm_do128,
                    const __grid_constant__ CUtensorMap tm_kv64, const AttnArgs p) {
@@ -943,21 +953,41 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q128,
   uint64_t* s_free = bars + 11;    // [2]
   uint64_t* p_full = bars + 13;    // [2] per dS buffer
   uint64_t* mm2_done = bars + 15;  // [2]
-  uint64_t* drain = bars + 17;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 18);
+  uint64_t* q_empty = bars + 17;   // the item's score products completed: q/dO reusable
+  uint64_t* acc_full = bars + 18;  // the item's dQ complete
+  uint64_t* acc_empty = bars + 19; // the epilogue has read dQ out
+  uint64_t* drain = bars + 20;     // [2] each issuer's products completed
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 22);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nqb = (p.S + C::BQ - 1) / C::BQ;
-  const AttnItem item = attn_item();
-  const int qb = p.causal ? nqb - 1 - item.x : item.x;
-  const int h = item.h, b = item.b;
-  const int shard = h / p.Ht, hl = h - shard * p.Ht;
-  const int q0 = qb * C::BQ;
   const int nkb = (p.S + C::BK - 1) / C::BK;
-  const int nsteps = p.causal ? min(nkb, (q0 + C::BQ) / C::BK) : nkb;
-  const int colq = hl * DH, colk = p.Dt + hl * DH, colv = 2 * p.Dt + hl * DH, cold = hl * DH;
+  const int nitems = nqb * p.H * p.B;
   const Ctl ctl{abort_flag, p.err};
+  // Per-item geometry; items in (query block, head, batch) order with the
+  // length index slowest, longest causal item first.
+  struct Geo {
+    int b, h, shard, q0, nsteps, colq, colk, colv, cold;
+  };
+  auto geo = [&](int i) {
+    const int hb = p.H * p.B;
+    const int x = i / hb;
+    const int r = i - x * hb;
+    Geo g;
+    g.h = r % p.H;
+    g.b = r / p.H;
+    g.shard = g.h / p.Ht;
+    const int hl = g.h - g.shard * p.Ht;
+    const int qb = p.causal ? nqb - 1 - x : x;
+    g.q0 = qb * C::BQ;
+    g.nsteps = p.causal ? min(nkb, (g.q0 + C::BQ) / C::BK) : nkb;
+    g.colq = hl * DH;
+    g.colk = p.Dt + hl * DH;
+    g.colv = 2 * p.Dt + hl * DH;
+    g.cold = hl * DH;
+    return g;
+  };
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
@@ -970,8 +1000,11 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q128,
       mbar_init(&s_free[i], 128);   // buffer i belongs to compute warpgroup i
       mbar_init(&p_full[i], 128);
       mbar_init(&mm2_done[i], 1);
+      mbar_init(&drain[i], 1);
     }
-    mbar_init(drain, 1);
+    mbar_init(q_empty, 1);
+    mbar_init(acc_full, 1);
+    mbar_init(acc_empty, 4);        // one arrival per epilogue warp
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -991,139 +1024,192 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q128,
 
   if (warp == 0) {
     if (lane == 0) {
-      mbar_arrive_expect_tx(q_full, 2 * C::Q_BYTES);
-      for (int c = 0; c < C::CH; ++c) {
-        tma_load_4d(smem + C::OFF_Q + c * C::BQ * 128, &tm_q128, q_full, colq + 64 * c, q0, b, shard);
-        tma_load_4d(smem + C::OFF_DO + c * C::BQ * 128, &tm_do128, q_full, cold + 64 * c, q0, b, shard);
-      }
-      int k = 0;
-      for (; k < nsteps; ++k) {
-        const int st = k % C::STAGES;
-        const uint32_t u = k / C::STAGES;
-        if (!wait_bar(&kv_empty[st], (u & 1) ^ 1, ctl, ERR_ATTN_DQ_WAIT)) break;
-        uint8_t* sk = smem + C::OFF_ST + st * 2 * C::K_BYTES;
-        uint8_t* sv = sk + C::K_BYTES;
-        mbar_arrive_expect_tx(&kv_full[st], 2 * C::K_BYTES);
+      int g = 0, n = 0, nq = 0;
+      bool ok = true;
+      for (int it = blockIdx.x; ok && it < nitems; it += gridDim.x, ++n) {
+        const Geo q = geo(it);
+        // q and dO of the previous item are free once its score products completed.
+        if (!(ok = wait_bar(q_empty, (n & 1) ^ 1, ctl, ERR_ATTN_DQ_WAIT))) break;
+        mbar_arrive_expect_tx(q_full, 2 * C::Q_BYTES);
         for (int c = 0; c < C::CH; ++c) {
-          tma_load_4d(sk + c * C::BK * 128, &tm_kv64, &kv_full[st], colk + 64 * c, k * C::BK, b, shard);
-          tma_load_4d(sv + c * C::BK * 128, &tm_kv64, &kv_full[st], colv + 64 * c, k * C::BK, b, shard);
+          tma_load_4d(smem + C::OFF_Q + c * C::BQ * 128, &tm_q128, q_full, q.colq + 64 * c, q.q0,
+                      q.b, q.shard);
+          tma_load_4d(smem + C::OFF_DO + c * C::BQ * 128, &tm_do128, q_full, q.cold + 64 * c, q.q0,
+                      q.b, q.shard);
+        }
+        ++nq;
+        for (int k = 0; k < q.nsteps; ++k, ++g) {
+          const int st = g % C::STAGES;
+          const uint32_t u = g / C::STAGES;
+          if (!(ok = wait_bar(&kv_empty[st], (u & 1) ^ 1, ctl, ERR_ATTN_DQ_WAIT))) break;
+          uint8_t* sk = smem + C::OFF_ST + st * 2 * C::K_BYTES;
+          uint8_t* sv = sk + C::K_BYTES;
+          mbar_arrive_expect_tx(&kv_full[st], 2 * C::K_BYTES);
+          for (int c = 0; c < C::CH; ++c) {
+            tma_load_4d(sk + c * C::BK * 128, &tm_kv64, &kv_full[st], q.colk + 64 * c, k * C::BK,
+                        q.b, q.shard);
+            tma_load_4d(sv + c * C::BK * 128, &tm_kv64, &kv_full[st], q.colv + 64 * c, k * C::BK,
+                        q.b, q.shard);
+          }
         }
       }
-      mbar_wait(q_full, 0, 200000000ull);
-      for (int i = k - 1; i >= 0 && i >= k - C::STAGES; --i)
+      // Copies still in flight land in this CTA's shared memory: wait for them
+      // (bounded) before the CTA may exit: nq q/dO loads and stages 0 .. g-1.
+      if (nq > 0) mbar_wait(q_full, (uint32_t)((nq - 1) & 1), 200000000ull);
+      for (int i = g - 1; i >= 0 && i >= g - C::STAGES; --i)
         mbar_wait(&kv_full[i % C::STAGES], (i / C::STAGES) & 1, 200000000ull);
     }
   } else if (warp == 1 || warp == 10) {
-    // Two issuers as in the dK/dV kernel: warp 1 issues S/dP of block k,
-    // warp 10 dQ += dS K of block k and releases the K/V stage.
+    // Two issuers as in the dK/dV kernel: warp 1 issues S/dP of block g,
+    // warp 10 dQ += dS K of block g and releases the K/V stage.
     if (lane == 0) {
       constexpr uint32_t id_s = idesc_f32acc(128, C::BK, false, false, true);
       constexpr uint32_t id_acc = idesc_f32acc(128, DH, false, true, true);
       const uint32_t sq = smem_u32(smem + C::OFF_Q), sd = smem_u32(smem + C::OFF_DO);
-      bool ok = wait_bar(q_full, 0, ctl, ERR_ATTN_DQ_WAIT);
+      int g = 0, n = 0;
+      bool ok = true;
       if (warp == 1) {
-        for (int k = 0; ok && k < nsteps; ++k) {
-          const int bf = k & 1, st = k % C::STAGES;
-          if (!(ok = wait_bar(&kv_full[st], (k / C::STAGES) & 1, ctl, ERR_ATTN_DQ_WAIT))) break;
-          if (!(ok = wait_bar(&s_free[bf], ((k >> 1) & 1) ^ 1, ctl, ERR_ATTN_DQ_WAIT))) break;
-          tc_fence_after();
-          const uint32_t sk = smem_u32(smem + C::OFF_ST + st * 2 * C::K_BYTES);
-          const uint32_t sv = sk + C::K_BYTES;
+        for (int it = blockIdx.x; ok && it < nitems; it += gridDim.x, ++n) {
+          const int nsteps = geo(it).nsteps;
+          if (!(ok = wait_bar(q_full, n & 1, ctl, ERR_ATTN_DQ_WAIT))) break;
+          for (int k = 0; k < nsteps; ++k, ++g) {
+            const int bf = g & 1, st = g % C::STAGES;
+            if (!(ok = wait_bar(&kv_full[st], (g / C::STAGES) & 1, ctl, ERR_ATTN_DQ_WAIT))) break;
+            if (!(ok = wait_bar(&s_free[bf], ((g >> 1) & 1) ^ 1, ctl, ERR_ATTN_DQ_WAIT))) break;
+            tc_fence_after();
+            const uint32_t sk = smem_u32(smem + C::OFF_ST + st * 2 * C::K_BYTES);
+            const uint32_t sv = sk + C::K_BYTES;
 #pragma unroll
-          for (int kk = 0; kk < DH / 16; ++kk) {
-            tc_mma_f16(tmem + bf * 128, kmajor_desc(sq, C::BQ, kk), kmajor_desc(sk, C::BK, kk), id_s,
-                       kk > 0);
-            tc_mma_f16(tmem + bf * 128 + 64, kmajor_desc(sd, C::BQ, kk), kmajor_desc(sv, C::BK, kk),
-                       id_s, kk > 0);
+            for (int kk = 0; kk < DH / 16; ++kk) {
+              tc_mma_f16(tmem + bf * 128, kmajor_desc(sq, C::BQ, kk), kmajor_desc(sk, C::BK, kk),
+                         id_s, kk > 0);
+              tc_mma_f16(tmem + bf * 128 + 64, kmajor_desc(sd, C::BQ, kk),
+                         kmajor_desc(sv, C::BK, kk), id_s, kk > 0);
+            }
+            tc_commit(&s_full[bf]);
           }
-          tc_commit(&s_full[bf]);
+          if (!ok) break;
+          tc_commit(q_empty);   // q/dO may be reloaded once this item's score products completed
         }
+        tc_commit(&drain[0]);
+        mbar_wait(&drain[0], 0, 200000000ull);
       } else {
-        for (int k = 0; ok && k < nsteps; ++k) {
-          const int bj = k & 1, sj = k % C::STAGES;
-          if (!(ok = wait_bar(&p_full[bj], (k >> 1) & 1, ctl, ERR_ATTN_DQ_WAIT))) break;
-          tc_fence_after();
-          const uint32_t sk = smem_u32(smem + C::OFF_ST + sj * 2 * C::K_BYTES);
+        for (int it = blockIdx.x; ok && it < nitems; it += gridDim.x, ++n) {
+          const int nsteps = geo(it).nsteps;
+          // The first products of an item overwrite dQ: the epilogue has read the last item's.
+          if (!(ok = wait_bar(acc_empty, (n & 1) ^ 1, ctl, ERR_ATTN_DQ_WAIT))) break;
+          for (int k = 0; k < nsteps; ++k, ++g) {
+            const int bj = g & 1, sj = g % C::STAGES;
+            if (!(ok = wait_bar(&p_full[bj], (g >> 1) & 1, ctl, ERR_ATTN_DQ_WAIT))) break;
+            tc_fence_after();
+            const uint32_t sk = smem_u32(smem + C::OFF_ST + sj * 2 * C::K_BYTES);
 #pragma unroll
-          for (int kk = 0; kk < C::BK / 16; ++kk)   // 16 keys = 8 columns of dS per step
-            tc_mma_f16_ts(t_dq, tmem + 384 + 32 * bj + 8 * kk, mnmajor_desc(sk, C::BK, kk),
-                          id_acc, (k | kk) != 0);
-          tc_commit(&mm2_done[bj]);
-          tc_commit(&kv_empty[sj]);   // the scores of block k completed before its dS existed
+            for (int kk = 0; kk < C::BK / 16; ++kk)   // 16 keys = 8 columns of dS per step
+              tc_mma_f16_ts(t_dq, tmem + 384 + 32 * bj + 8 * kk, mnmajor_desc(sk, C::BK, kk),
+                            id_acc, (k | kk) != 0);
+            tc_commit(&mm2_done[bj]);
+            tc_commit(&kv_empty[sj]);   // the scores of block g completed before its dS existed
+          }
+          if (!ok) break;
+          tc_commit(acc_full);
         }
-        tc_commit(drain);
-        mbar_wait(drain, 0, 200000000ull);
+        tc_commit(&drain[1]);
+        mbar_wait(&drain[1], 0, 200000000ull);
       }
     }
-  } else {
-    // Two compute warpgroups: warpgroup g takes the blocks k with k % 2 == g (its
-    // own TMEM and shared buffers), so two blocks are in flight at once; the
-    // epilogue splits the 32-column slices between them.
+  } else if (warp < 10) {
+    // Two compute warpgroups: warpgroup w takes the blocks g with g % 2 == w
+    // (its own S/dP and dS buffers), so two blocks are in flight at once.
     const int wg = (warp - 2) >> 2;
     const int quad = warp & 3;
     const int r = quad * 32 + lane;
-    const int q = q0 + r;
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-    const long long hrow = ((long long)b * p.H + h) * p.S_pad;
-    const bool qvalid = q < p.S;
-    const float l2 = p.lse2[hrow + q];     // padded rows: +inf, so P = 0
-    const float dv = p.dvec[hrow + q];
+    int g0 = 0;   // first block counter of the current item
     bool ok = true;
-    for (int k = wg; k < nsteps; k += 2) {
-      const int bf = k & 1;
-      const uint32_t u = k >> 1;
-      const int ks = k * C::BK;
-      if (!__all_sync(0xffffffffu, wait_bar(&s_full[bf], u & 1, ctl, ERR_ATTN_DQ_WAIT))) { ok = false; break; }
-      tc_fence_after();
-      // Copy S and dP out of tensor memory and hand the buffer back first.
-      uint32_t rs0[32], rs1[32], rd0[32], rd1[32];
-      tmem_ld32(tmem + bf * 128 + lane_off, rs0);
-      tmem_ld32(tmem + bf * 128 + lane_off + 32, rs1);
-      tmem_ld32(tmem + bf * 128 + 64 + lane_off, rd0);
-      tmem_ld32(tmem + bf * 128 + 64 + lane_off + 32, rd1);
-      tc_wait_ld();
-      tc_fence_before();
-      mbar_arrive(&s_free[bf]);
-      // Keys past the last visible one (after the query, or past S) are
-      // masked: a select per element against a bound fixed once per block.
-      const int kmax = (p.causal ? min(q, p.S - 1) : p.S - 1) - ks;
-      auto ds = [&](const uint32_t (&rs)[32], uint32_t (&rd)[32], int c, auto mask_tag) {
-        constexpr bool MASK = decltype(mask_tag)::value;
-#pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          float pe = fast_exp2(fmaf(__uint_as_float(rs[e]), p.scale_log2, -l2));
-          if (MASK) pe = c * 32 + e > kmax ? 0.f : pe;
-          rd[e] = __float_as_uint(pe * (__uint_as_float(rd[e]) - dv));
+    for (int it = blockIdx.x; ok && it < nitems; it += gridDim.x) {
+      const Geo q = geo(it);
+      const int qr = q.q0 + r;
+      const long long hrow = ((long long)q.b * p.H + q.h) * p.S_pad;
+      const float l2 = p.lse2[hrow + qr];     // padded rows: +inf, so P = 0
+      const float dv = p.dvec[hrow + qr];
+      // Keys past the last visible one (after the query, or past S) are masked.
+      const int klast = p.causal ? min(qr, p.S - 1) : p.S - 1;
+      for (int k = ((g0 & 1) == wg) ? 0 : 1; k < q.nsteps; k += 2) {
+        const int g = g0 + k;
+        const int bf = g & 1;
+        const uint32_t u = g >> 1;
+        const int kmax = klast - k * C::BK;
+        if (!__all_sync(0xffffffffu, wait_bar(&s_full[bf], u & 1, ctl, ERR_ATTN_DQ_WAIT))) {
+          ok = false;
+          break;
         }
-      };
-      // The select only where some row of the warp has a masked key.
-      if (!__all_sync(0xffffffffu, kmax >= C::BK - 1)) {
-        ds(rs0, rd0, 0, BoolTag<true>{});
-        ds(rs1, rd1, 1, BoolTag<true>{});
-      } else {
-        ds(rs0, rd0, 0, BoolTag<false>{});
-        ds(rs1, rd1, 1, BoolTag<false>{});
-      }
-      uint32_t pk[32];   // dS as fp16 pairs, 64 keys
+        // The dS columns of buffer bf were last read by the dQ MMAs of block g-2.
+        if (g >= 2 && !__all_sync(0xffffffffu, wait_bar(&mm2_done[bf], (u - 1) & 1, ctl,
+                                                        ERR_ATTN_DQ_WAIT))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t tb = tmem + bf * 128 + lane_off;
+        // The select only where some row of the warp has a masked key.
+        const bool masked = !__all_sync(0xffffffffu, kmax >= C::BK - 1);
+        // S and dP leave tensor memory in two 32-key halves; the buffer goes
+        // back to the score issuer once both halves are in registers, and dS of
+        // each half (fp16 pairs, 16 columns) goes to this block's dS buffer.
+        auto half = [&](int c, auto mask_tag) {
+          constexpr bool MASK = decltype(mask_tag)::value;
+          uint32_t rs[32], rd[32];
+          tmem_ld32(tb + 32 * c, rs);
+          tmem_ld32(tb + 64 + 32 * c, rd);
+          tc_wait_ld();
+          if (c == 1) {
+            tc_fence_before();
+            mbar_arrive(&s_free[bf]);
+          }
+          uint32_t pk[16];
 #pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        pk[e] = pack_f16x2(__uint_as_float(rd0[2 * e]), __uint_as_float(rd0[2 * e + 1]));
-        pk[16 + e] = pack_f16x2(__uint_as_float(rd1[2 * e]), __uint_as_float(rd1[2 * e + 1]));
-      }
-      // The dS columns of buffer bf were last read by the dQ MMAs of block k-2.
-      if (k >= 2 && !__all_sync(0xffffffffu, wait_bar(&mm2_done[bf], (u - 1) & 1, ctl, ERR_ATTN_DQ_WAIT))) { ok = false; break; }
-      tmem_st32(tmem + 384 + 32 * bf + lane_off, pk);
-      tc_wait_st();
-      tc_fence_before();
-      mbar_arrive(&p_full[bf]);
-    }
-    // As in the dK/dV kernel: `drain` completes after the last product.
-    if (ok && nsteps > 0 && __all_sync(0xffffffffu, wait_bar(drain, 0, ctl, ERR_ATTN_DQ_WAIT))) {
-      tc_fence_after();
-      const long long w3 = 3LL * p.Dt;
-      uint16_t* row = p.out + (long long)shard * p.T * w3 + ((long long)b * p.S + q) * w3 + colq;
+          for (int e = 0; e < 32; e += 2) {
+            float pe0 = fast_exp2(fmaf(__uint_as_float(rs[e]), p.scale_log2, -l2));
+            float pe1 = fast_exp2(fmaf(__uint_as_float(rs[e + 1]), p.scale_log2, -l2));
+            if (MASK) {
+              pe0 = c * 32 + e > kmax ? 0.f : pe0;
+              pe1 = c * 32 + e + 1 > kmax ? 0.f : pe1;
+            }
+            pk[e / 2] = pack_f16x2(pe0 * (__uint_as_float(rd[e]) - dv),
+                                   pe1 * (__uint_as_float(rd[e + 1]) - dv));
+          }
+          tmem_st16(tmem + 384 + 32 * bf + lane_off + 16 * c, pk);
+        };
 #pragma unroll 1
-      for (int c = wg; c < DH / 32; c += 2) {
+        for (int c = 0; c < 2; ++c) {
+          if (masked) half(c, BoolTag<true>{});
+          else half(c, BoolTag<false>{});
+        }
+        tc_wait_st();
+        tc_fence_before();
+        mbar_arrive(&p_full[bf]);
+      }
+      g0 += q.nsteps;
+    }
+  } else {
+    // Epilogue warps 11-14 (TMEM lane quarter warp % 4): dQ of each item,
+    // once its last products completed, to global memory (fp16, scaled by
+    // 1/sqrt(dh)) with its column partials for dbqkv; then the accumulator is
+    // released to the next item.
+    const int quad = warp & 3;
+    const int r = quad * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+    const long long w3 = 3LL * p.Dt;
+    int n = 0;
+    for (int it = blockIdx.x; it < nitems; it += gridDim.x, ++n) {
+      const Geo q = geo(it);
+      if (!__all_sync(0xffffffffu, wait_bar(acc_full, n & 1, ctl, ERR_ATTN_DQ_WAIT))) break;
+      tc_fence_after();
+      const int qr = q.q0 + r;
+      const bool qvalid = qr < p.S;
+      uint16_t* row = p.out + (long long)q.shard * p.T * w3 + ((long long)q.b * p.S + qr) * w3 + q.colq;
+#pragma unroll 1
+      for (int c = 0; c < DH / 32; ++c) {
         uint32_t rq[32];
         tmem_ld32(t_dq + lane_off + c * 32, rq);
         tc_wait_ld();
@@ -1135,12 +1221,15 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q128,
 #pragma unroll
           for (int e = 0; e < 32; ++e) over |= fabsf(v[e]) > 65504.0f;
 #pragma unroll
-          for (int g = 0; g < 4; ++g)
-            *reinterpret_cast<uint4*>(row + c * 32 + g * 8) = pack8_f16(&v[g * 8]);
+          for (int gg = 0; gg < 4; ++gg)
+            *reinterpret_cast<uint4*>(row + c * 32 + gg * 8) = pack8_f16(&v[gg * 8]);
           if (over && p.err) atomicCAS(p.err, 0u, 0x301u);
         }
-        if (p.colpart != nullptr) colpart_store(p, v, b, q0 + quad * 32, shard, colq + c * 32);
+        if (p.colpart != nullptr) colpart_store(p, v, q.b, q.q0 + quad * 32, q.shard, q.colq + c * 32);
       }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acc_empty);
     }
   }
   tc_fence_before();
@@ -1285,8 +1374,11 @@ tp_status bwd_launch(const uint16_t* qkv, const uint16_t* o, const float* lse, c
   if (cudaGetLastError() != cudaSuccess) return TP_ERR_CUDA;
   {
     TraceScope ts(st, TK_ATTN_BWD_DQ, 2.0 * DH * core_pairs(a));
-    if (launch_pdl(k2, dim3((a.S + 127) / 128, a.H, a.B), dim3(352), DqCfg<DH>::SMEM, st, q128,
-                   do128, kv64, p) != cudaSuccess)
+    // Persistent: one CTA per SM (at most one per work item).
+    const long long items = (long long)((a.S + DqCfg<DH>::BQ - 1) / DqCfg<DH>::BQ) * a.H * a.B;
+    const unsigned grid = (unsigned)(items < sm_count() ? items : sm_count());
+    if (launch_pdl(k2, dim3(grid), dim3(DQ_THREADS), DqCfg<DH>::SMEM, st, q128, do128, kv64, p) !=
+        cudaSuccess)
       return TP_ERR_CUDA;
   }
   return cuda_status(cudaGetLastError());
