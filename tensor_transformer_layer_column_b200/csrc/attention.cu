@@ -27,6 +27,9 @@
 //           dV += P^T dO, dK += dS^T q
 //   dQ:     per 128-query block, walk 64-key blocks: S = q k^T, dP = dO v^T,
 //           dS = P * (dP - Dv), dQ += dS k
+//   Both are persistent: one CTA per SM walks its work items (snake order,
+//   longest first) with the pipelines carried from item to item and four
+//   epilogue warps writing an item's dK/dV or dQ while the next one starts.
 // P, P^T, dS^T and dS go from registers to tensor memory (fp16) and are the
 // A operands of the products that consume them, read from there: shared
 // memory, whose bandwidth the score products already use up, carries only
