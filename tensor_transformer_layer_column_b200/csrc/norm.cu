@@ -318,8 +318,18 @@ __device__ __forceinline__ float reduce_rows_fixed(const float* __restrict__ row
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const long long c = (long long)blockIdx.x * 32 + lane;
   float s = 0.f;
-  if (c < width)
-    for (int k = warp; k < n; k += 8) s += rowsrc[(long long)k * stride_rows + c];
+  if (c < width) {
+    // Eight rows' loads issued ahead of their (in-order) additions.
+    int k = warp;
+    for (; k + 56 < n; k += 64) {
+      float v[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) v[j] = rowsrc[(long long)(k + 8 * j) * stride_rows + c];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) s += v[j];
+    }
+    for (; k < n; k += 8) s += rowsrc[(long long)k * stride_rows + c];
+  }
   red[warp][lane] = s;
   __syncthreads();
   float t = 0.f;
