@@ -586,7 +586,7 @@ __device__ __forceinline__ DkdvItem dkdv_item(int i, int H, int B) {
 
 constexpr int DKDV_THREADS = 480;
 
-// Persistent: one CTA per SM walks the items i = blockIdx.x, +gridDim.x, ...
+// Persistent: one CTA per SM walks its items in snake order (snake_item).
 // Warp roles: 0 loads (K/V per item, q/dO/lse2/Dv per 64-query block), 1
 // issues the score products S^T = K q^T and dP^T = V dO^T, 2-9 are two
 // compute warpgroups (P^T, dS^T), 10 issues dV += P^T dO and dK += dS^T q,
@@ -938,7 +938,7 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_kv128,
 // its own TMEM columns and is the A operand of dQ += dS k.
 //
 // Persistent like the dK/dV kernel: one CTA per SM walks the (query block,
-// head, batch) items longest first (item i, i + #CTAs, ...).  The block
+// head, batch) items longest first, in snake order (snake_item).  The block
 // counter g runs across the CTA's items, so the K/V ring, the two S/dP
 // buffers and the two dS buffers carry on from item to item; q/dO of the next
 // item load once the item's last score products completed (q_empty), and the
