@@ -220,6 +220,20 @@ tp_status tp_attn_bwd(const tp_dims* dims, const tp_bf16* x, const tp_bf16* wqkv
                       tp_bf16* dwqkv, tp_bf16* dbqkv, tp_bf16* dwout, tp_bf16* dbout, void* ws,
                       size_t ws_bytes, tp_stream stream);
 
+/* tp_attn_set_ds_limit: how the attention backward forms dq = dS k.  When the
+ * fp16 array dS^T of all heads, B*H*S_pad*S_pad*2 bytes with S_pad = seq
+ * rounded up to 128, takes at most max_bytes, the kernel that forms dk and dv
+ * also stores dS^T in the workspace and the dq kernel reads it back; above the
+ * limit the dq kernel recomputes the scores q k^T and dP = dO v^T from the
+ * saved lse instead.  The two give dq equal up to fp32 rounding order.  The
+ * limit is process-wide, 4 GiB by default (0: always recompute), and enters
+ * tp_workspace_size and tp_rank_workspace_size for TP_OP_ATTN_BWD and the
+ * layer backward ops: set it while no such call is running and size
+ * workspaces after setting it (a smaller workspace gives TP_ERR_WORKSPACE).
+ * Returns the previous limit.  Not an operation of the pages: a choice of
+ * how to run the backward of their attention. */
+size_t tp_attn_set_ds_limit(size_t max_bytes);
+
 /* ------------------------------------------------------------------ pre-LN layer
  * "The layernorm placement the paper flags as critical":
  *   h = x + Attn(LN1(x));  y = h + MLP(LN2(h))

@@ -138,11 +138,12 @@ _SIGS = {
     "tp_trace_begin": [ctypes.POINTER(ctypes.c_void_p), ctypes.POINTER(ctypes.c_int),
                        ctypes.POINTER(ctypes.c_double), ctypes.c_int],
     "tp_trace_end": [],
+    "tp_attn_set_ds_limit": [ctypes.c_size_t],
 }
 _RESTYPES = {"tp_version": ctypes.c_char_p, "tp_status_string": ctypes.c_char_p,
              "tp_workspace_size": ctypes.c_size_t,
              "tp_layernorm_bwd_workspace_size": ctypes.c_size_t, "tp_trace_end": ctypes.c_int,
-             "tp_rank_workspace_size": ctypes.c_size_t}
+             "tp_rank_workspace_size": ctypes.c_size_t, "tp_attn_set_ds_limit": ctypes.c_size_t}
 EXPORTED_SYMBOLS = tuple(_SIGS)
 
 _lib: Optional[ctypes.CDLL] = None
@@ -353,6 +354,12 @@ def layer_bwd_recompute(dims, x, params: dict, dy, dx, grads: dict, ws, stream=N
     _check(lib().tp_layer_bwd_recompute(ctypes.byref(dims), _ptr(x), ctypes.byref(p), _ptr(dy),
                                         _ptr(dx), ctypes.byref(g), wp, wn, _stream(stream, x)),
            "tp_layer_bwd_recompute")
+
+
+def attn_set_ds_limit(max_bytes: int) -> int:
+    """Largest dS^T array (bytes) the attention backward keeps for its dq
+    kernel (see include/tp_layer.h); returns the previous limit."""
+    return int(lib().tp_attn_set_ds_limit(int(max_bytes)))
 
 
 def selftest_wait_timeout(limit_ns: int, stream=None):

@@ -459,6 +459,8 @@ const char* tp_status_string(tp_status s) {
   return "TP_ERR_UNKNOWN";
 }
 
+size_t tp_attn_set_ds_limit(size_t max_bytes) { return attn_set_dst_limit(max_bytes); }
+
 size_t tp_workspace_size(int op_, const tp_dims* d) {
   switch (op_) {
     case TP_OP_MLP_FWD: return 0;

@@ -24,12 +24,15 @@
 //   prep:   Dv = rowsum(dO * O), lse2 = lse * log2(e)
 //   dK/dV:  per 128-key block, walk 64-query blocks:  S^T = k q^T, dP^T = v dO^T,
 //           P^T, dS^T = P^T * (dP^T - Dv) by one thread per key row,
-//           dV += P^T dO, dK += dS^T q
-//   dQ:     per 128-query block, walk 64-key blocks: S = q k^T, dP = dO v^T,
-//           dS = P * (dP - Dv), dQ += dS k
-//   Both are persistent: one CTA per SM walks its work items (snake order,
-//   longest first) with the pipelines carried from item to item and four
-//   epilogue warps writing an item's dK/dV or dQ while the next one starts.
+//           dV += P^T dO, dK += dS^T q; also stores dS^T (fp16) when the
+//           array fits under the limit attn_set_dst_limit sets
+//   dQ:     per 128-query block, walk 64-key blocks: dQ += dS k, dS read
+//           back from that array; above the limit the dQ kernel recomputes
+//           S = q k^T, dP = dO v^T, dS = P * (dP - Dv) instead
+//   dK/dV and the recomputing dQ are persistent: one CTA per SM walks its
+//   work items (snake order, longest first) with the pipelines carried from
+//   item to item and four epilogue warps writing an item's dK/dV or dQ while
+//   the next one starts.
 // P, P^T, dS^T and dS go from registers to tensor memory (fp16) and are the
 // A operands of the products that consume them, read from there: shared
 // memory, whose bandwidth the score products already use up, carries only
@@ -40,6 +43,7 @@
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "internal.h"
@@ -80,6 +84,14 @@ struct AttnArgs {
   // partial row per 32 rows of one batch element: colpart[(b * G + s / 32) *
   // (t * 3Dt) + shard * 3Dt + column], G = ceil(S / 32).
   float* colpart;
+  // bwd (may be null): dS^T in fp16, written by the dK/dV kernel for the dQ
+  // kernel that reads it (attn_bwd_dq_ds_kernel), in 4 KiB pieces of 32 keys x
+  // 64 queries: piece (bh, j, i) holds keys 32i .. 32i+31 and queries 64j ..
+  // 64j+63 of head bh = b*H + h at element ((bh * S_pad/64 + j) * S_pad/32 + i)
+  // * 2048, one 128-byte row per key with its 16-byte chunks in the 128-byte
+  // swizzle (chunk c of row r at position c ^ (r % 8)) -- the image of an
+  // MN-major tensor-core operand tile, copied as is both ways.
+  uint16_t* dst;
   unsigned int* err;
 };
 
@@ -558,11 +570,13 @@ struct DkdvCfg {
   static constexpr int K_BYTES = BK * DH * 2;              // K and V tiles, each
   static constexpr int Q_BYTES = BQ * DH * 2;              // q and dO tiles, each (per stage)
   static constexpr int VEC_BYTES = BQ * 4;                 // lse2 / dvec slice of one stage
-  static constexpr int STAGES = 4;                         // q / dO / lse2 / dvec ring depth
+  static constexpr int STAGES = 3;                         // q / dO / lse2 / dvec ring depth
   static constexpr int STAGE_BYTES = 2 * Q_BYTES;
   static constexpr int OFF_K = 0, OFF_V = K_BYTES;
   static constexpr int OFF_ST = 2 * K_BYTES;               // stage s: q | dO
-  static constexpr int OFF_VEC = OFF_ST + STAGES * STAGE_BYTES;  // stage s: lse2 at +2s*VEC, dvec at +(2s+1)*VEC
+  static constexpr int DS_BYTES = 32 * BQ * 2;             // one compute warp's dS^T block (32 keys)
+  static constexpr int OFF_DS = OFF_ST + STAGES * STAGE_BYTES;   // compute warp w at +w*DS_BYTES
+  static constexpr int OFF_VEC = OFF_DS + 8 * DS_BYTES;    // stage s: lse2 at +2s*VEC, dvec at +(2s+1)*VEC
   static constexpr int OFF_BAR = OFF_VEC + STAGES * 2 * VEC_BYTES;
   static constexpr int RAW = OFF_BAR + 256 + 1024;
   static constexpr int SMEM = RAW > 120 * 1024 ? RAW : 120 * 1024;
@@ -629,13 +643,14 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_kv128,
   const Ctl ctl{abort_flag, p.err};
   // Per-item geometry.
   struct Geo {
-    int b, shard, k0, i0, nsteps, colq, colk, colv, cold;
+    int b, bh, shard, k0, i0, nsteps, colq, colk, colv, cold;
     long long hrow;
   };
   auto geo = [&](int i) {
     const DkdvItem it = dkdv_item(i, p.H, p.B);
     Geo g;
     g.b = it.b;
+    g.bh = it.b * p.H + it.h;
     g.shard = it.h / p.Ht;
     const int hl = it.h - g.shard * p.Ht;
     g.k0 = it.kb * C::BK;
@@ -799,6 +814,8 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_kv128,
     const int quad = warp & 3;
     const int r = quad * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+    uint8_t* ds_buf = smem + C::OFF_DS + (warp - 2) * C::DS_BYTES;
+    uint8_t* ds_row = ds_buf + lane * 128;
     int g0 = 0;   // first block counter of the current item
     bool ok = true;
     for (int rnd = 0; ok && (int)gridDim.x * rnd < nitems; ++rnd) {
@@ -806,6 +823,7 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_kv128,
       if (it >= nitems) continue;
       const Geo q = geo(it);
       const int kpos = q.k0 + r;
+      const bool kvalid = kpos < p.S;
       for (int k = ((g0 & 1) == wg) ? 0 : 1; k < q.nsteps; k += 2) {
         const int g = g0 + k;
         const int bf = g & 1;
@@ -825,6 +843,11 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_kv128,
         // MMAs of block g-2 completed, which the score MMAs of this block
         // already waited for.
         const uint32_t t_st = tmem + bf * 128 + lane_off;
+        // The warp's dS^T buffer: its previous block's store has read it out.
+        if (p.dst != nullptr) {
+          if (lane == 0) bulk_wait_read0();
+          __syncwarp();
+        }
         // Queries qs + qi with qi < qmin precede key kpos and are masked (causal):
         // a select per element, taken only in blocks where some key row of the
         // warp has a masked query (the causal diagonal).
@@ -859,6 +882,16 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_kv128,
           }
           tmem_st16(t_st + c * 16, pk);
           tmem_st16(t_st + 64 + c * 16, dk);
+          if (p.dst != nullptr) {
+            // dS^T row kpos (lane), queries 32c .. 32c+31 of the block: 16-byte
+            // chunks 4c .. 4c+3 of the lane's 128-byte row, swizzled (zeros
+            // for padded keys).
+#pragma unroll
+            for (int g4 = 0; g4 < 4; ++g4)
+              *reinterpret_cast<uint4*>(ds_row + (((4 * c + g4) ^ (lane & 7)) << 4)) =
+                  kvalid ? make_uint4(dk[4 * g4], dk[4 * g4 + 1], dk[4 * g4 + 2], dk[4 * g4 + 3])
+                         : make_uint4(0u, 0u, 0u, 0u);
+          }
         };
 #pragma unroll 1
         for (int c = 0; c < 2; ++c) {
@@ -868,9 +901,21 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_kv128,
         tc_wait_st();
         tc_fence_before();
         mbar_arrive(&p_full[bf]);
+        if (p.dst != nullptr) {
+          // The block's dS^T piece (32 keys x 64 queries) to global by one bulk copy.
+          fence_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            const long long piece =
+                ((long long)q.bh * (p.S_pad / 64) + qs / 64) * (p.S_pad / 32) + q.k0 / 32 + quad;
+            bulk_store(p.dst + piece * 2048, ds_buf, C::DS_BYTES);
+            bulk_commit();
+          }
+        }
       }
       g0 += q.nsteps;
     }
+    if (p.dst != nullptr && lane == 0) bulk_wait0();
   } else {
     // Epilogue warps 11-14 (TMEM lane quarter warp % 4): dV and dK of each
     // item, once its last products completed, to global memory (fp16, dK
@@ -1274,6 +1319,156 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q128,
   }
 }
 
+// ---------------------------------------------------------------- dQ from stored dS
+// When the dK/dV kernel also stores dS^T (fp16, the same values it feeds to
+// dK += dS^T q; AttnArgs::dst gives the layout), dQ = dS k needs no
+// recomputation of S and dP: per 128-query block, walk 64-key blocks through
+// a 3-stage ring of (dS^T tile, k tile) and accumulate dQ += dS k with dS as
+// an MN-major A operand (queries contiguous in each key row; two bulk copies
+// of 8 KiB, contiguous in global memory) and k as an MN-major B operand (TMA).  Warp 0 loads, warp 1 issues the
+// products, warps 2-5 (one per TMEM lane quarter) write dQ.  128 TMEM
+// columns and 96 KB of shared memory: two CTAs share an SM, so one's
+// epilogue overlaps the other's products.
+template <int DH>
+struct DqdsCfg {
+  static constexpr int BQ = 128, BK = 64, CH = DH / 64, STAGES = 3;
+  static constexpr int A_BYTES = BQ * BK * 2;                // dS^T tile: 64 key rows x 128 queries
+  static constexpr int K_BYTES = BK * DH * 2;                // k tile
+  static constexpr int STAGE_BYTES = A_BYTES + K_BYTES;
+  static constexpr int OFF_BAR = STAGES * STAGE_BYTES;
+  static constexpr int SMEM = OFF_BAR + 256 + 1024;
+  static constexpr int THREADS = 192;
+};
+
+template <int DH>
+__global__ void __launch_bounds__(192, 2)
+attn_bwd_dq_ds_kernel(const __grid_constant__ CUtensorMap tm_kv64, const AttnArgs p) {
+  using C = DqdsCfg<DH>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint64_t* full = bars + 0;       // [STAGES]
+  uint64_t* empty = bars + 3;      // [STAGES]
+  uint64_t* acc_full = bars + 6;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 7);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nqb = (p.S + C::BQ - 1) / C::BQ;
+  const AttnItem item = attn_item();
+  const int qb = p.causal ? nqb - 1 - item.x : item.x;
+  const int h = item.h, b = item.b;
+  const int shard = h / p.Ht, hl = h - shard * p.Ht;
+  const int q0 = qb * C::BQ;
+  const int nkb = (p.S + C::BK - 1) / C::BK;
+  const int nsteps = p.causal ? min(nkb, (q0 + C::BQ) / C::BK) : nkb;
+  const int colq = hl * DH, colk = p.Dt + hl * DH;
+  const int bh = b * p.H + h;
+  // dS^T pieces of this query block (its first 64-query column, key piece 0).
+  const uint16_t* ds_col = p.dst + ((long long)bh * (p.S_pad / 64) + 2 * qb) * (p.S_pad / 32) * 2048;
+  const Ctl ctl{abort_flag, p.err};
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < C::STAGES; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    mbar_init(acc_full, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tm_kv64);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 128);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t t_dq = *tmem_slot;
+  grid_dep_wait();   // inputs and outputs: the previous kernels have completed
+  grid_dep_launch();
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int k = 0;
+      for (; k < nsteps; ++k) {
+        const int st = k % C::STAGES;
+        const uint32_t u = k / C::STAGES;
+        if (!wait_bar(&empty[st], (u & 1) ^ 1, ctl, ERR_ATTN_DQ_WAIT)) break;
+        uint8_t* sa = smem + st * C::STAGE_BYTES;
+        uint8_t* sk = sa + C::A_BYTES;
+        mbar_arrive_expect_tx(&full[st], C::STAGE_BYTES);
+        // Two 64-query chunks of 64 key rows: two consecutive 32-key pieces each.
+        for (int c = 0; c < C::BQ / 64; ++c)
+          bulk_load(sa + c * C::BK * 128, ds_col + (long long)c * (p.S_pad / 32) * 2048 + k * 4096,
+                    C::BK * 128, &full[st]);
+        for (int c = 0; c < C::CH; ++c)
+          tma_load_4d(sk + c * C::BK * 128, &tm_kv64, &full[st], colk + 64 * c, k * C::BK, b, shard);
+      }
+      for (int i = k - 1; i >= 0 && i >= k - C::STAGES; --i)
+        mbar_wait(&full[i % C::STAGES], (i / C::STAGES) & 1, 200000000ull);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t id_acc = idesc_f32acc(128, DH, true, true, true);
+      bool ok = true;
+      for (int k = 0; ok && k < nsteps; ++k) {
+        const int st = k % C::STAGES;
+        if (!(ok = wait_bar(&full[st], (k / C::STAGES) & 1, ctl, ERR_ATTN_DQ_WAIT))) break;
+        tc_fence_after();
+        const uint32_t sa = smem_u32(smem + st * C::STAGE_BYTES);
+        const uint32_t sk = sa + C::A_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < C::BK / 16; ++kk)   // 16 keys per product
+          tc_mma_f16(t_dq, mnmajor_desc(sa, C::BK, kk),
+                     mnmajor_desc(sk, C::BK, kk), id_acc, (k | kk) != 0);
+        tc_commit(&empty[st]);
+      }
+      tc_commit(acc_full);   // also after an early stop: every issued product completes
+      mbar_wait(acc_full, 0, 200000000ull);
+    }
+  } else {
+    // Epilogue warps 2-5 (TMEM lane quarter warp % 4).
+    const int quad = warp & 3;
+    const int r = quad * 32 + lane;
+    const int q = q0 + r;
+    const bool qvalid = q < p.S;
+    const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+    if (nsteps > 0 && __all_sync(0xffffffffu, wait_bar(acc_full, 0, ctl, ERR_ATTN_DQ_WAIT))) {
+      tc_fence_after();
+      const long long w3 = 3LL * p.Dt;
+      uint16_t* row = p.out + (long long)shard * p.T * w3 + ((long long)b * p.S + q) * w3 + colq;
+#pragma unroll 1
+      for (int c = 0; c < DH / 32; ++c) {
+        uint32_t rq[32];
+        tmem_ld32(t_dq + lane_off + c * 32, rq);
+        tc_wait_ld();
+        float v[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) v[e] = qvalid ? __uint_as_float(rq[e]) * p.inv_sqrt_dh : 0.f;
+        if (qvalid) {
+          bool over = false;
+#pragma unroll
+          for (int e = 0; e < 32; ++e) over |= fabsf(v[e]) > 65504.0f;
+#pragma unroll
+          for (int g = 0; g < 4; ++g)
+            *reinterpret_cast<uint4*>(row + c * 32 + g * 8) = pack8_f16(&v[g * 8]);
+          if (over && p.err) atomicCAS(p.err, 0u, 0x301u);
+        }
+        if (p.colpart != nullptr) colpart_store(p, v, b, q0 + quad * 32, shard, colq + c * 32);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(t_dq, 128);
+  }
+}
+
 // =====================================================================================
 // Host side
 // =====================================================================================
@@ -1306,6 +1501,18 @@ bool encode_act(CUtensorMap* m, const void* base, long long width, int S, int B,
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
+
+// dS^T is kept for the dQ kernel when it takes at most this many bytes
+// (attn_set_dst_limit; 4 GiB by default); larger problems recompute S and dP
+// in the dQ kernel instead.
+std::atomic<size_t> g_dst_max{size_t(4) << 30};
+
+size_t dst_bytes(int B, int S, int H) {
+  const size_t s_pad = ((size_t)S + 127) / 128 * 128;
+  return (size_t)B * H * s_pad * s_pad * 2;
+}
+
+bool keep_dst(int B, int S, int H) { return dst_bytes(B, S, H) <= g_dst_max.load(); }
 
 // Opt the kernel into `bytes` of dynamic shared memory once per device.
 bool set_smem(const void* kern, int bytes) {
@@ -1391,9 +1598,14 @@ tp_status bwd_launch(const uint16_t* qkv, const uint16_t* o, const float* lse, c
       !encode_act(&do128, dout, a.Dt, a.S, a.B, a.t, a.T, 128) ||
       !encode_act(&kv64, qkv, 3LL * a.Dt, a.S, a.B, a.t, a.T, 64))
     return TP_ERR_CUDA;
+  const bool with_dst = keep_dst(a.B, a.S, a.H);
+  if (with_dst) p.dst = reinterpret_cast<uint16_t*>(lse2 + (size_t)a.B * a.H * a.S_pad);
   auto k1 = attn_bwd_dkdv_kernel<DH>;
   auto k2 = attn_bwd_dq_kernel<DH>;
-  if (!set_smem((const void*)k1, DkdvCfg<DH>::SMEM) || !set_smem((const void*)k2, DqCfg<DH>::SMEM))
+  auto k3 = attn_bwd_dq_ds_kernel<DH>;
+  if (!set_smem((const void*)k1, DkdvCfg<DH>::SMEM) ||
+      !set_smem((const void*)(with_dst ? (const void*)k3 : (const void*)k2),
+                with_dst ? DqdsCfg<DH>::SMEM : DqCfg<DH>::SMEM))
     return TP_ERR_CUDA;
   {
     // dP, dV and dK: three of the backward's four algorithmic products.
@@ -1406,6 +1618,14 @@ tp_status bwd_launch(const uint16_t* qkv, const uint16_t* o, const float* lse, c
       return TP_ERR_CUDA;
   }
   if (cudaGetLastError() != cudaSuccess) return TP_ERR_CUDA;
+  if (with_dst) {
+    TraceScope ts(st, TK_ATTN_BWD_DQ, 2.0 * DH * core_pairs(a));
+    const dim3 grid((unsigned)((a.S + DqdsCfg<DH>::BQ - 1) / DqdsCfg<DH>::BQ), a.H, a.B);
+    if (launch_pdl(k3, grid, dim3(DqdsCfg<DH>::THREADS), DqdsCfg<DH>::SMEM, st, kv64, p) !=
+        cudaSuccess)
+      return TP_ERR_CUDA;
+    return cuda_status(cudaGetLastError());
+  }
   {
     TraceScope ts(st, TK_ATTN_BWD_DQ, 2.0 * DH * core_pairs(a));
     // Persistent: one CTA per SM (at most one per work item).
@@ -1429,10 +1649,12 @@ tp_status launch_attn_fwd(const uint16_t* qkv, uint16_t* o, float* lse, int B, i
   return TP_ERR_UNSUPPORTED;
 }
 
+size_t attn_set_dst_limit(size_t max_bytes) { return g_dst_max.exchange(max_bytes); }
+
 size_t attn_bwd_scratch_bytes(int B, int S, int H, int dh) {
   (void)dh;
   const size_t s_pad = ((size_t)S + 127) / 128 * 128;
-  return 2 * (size_t)B * H * s_pad * sizeof(float);
+  return 2 * (size_t)B * H * s_pad * sizeof(float) + (keep_dst(B, S, H) ? dst_bytes(B, S, H) : 0);
 }
 
 tp_status launch_attn_bwd(const uint16_t* qkv, const uint16_t* o, const float* lse,

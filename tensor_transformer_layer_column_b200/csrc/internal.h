@@ -116,6 +116,9 @@ tp_status launch_layernorm_bwd_blocks(const uint16_t* dy, const uint16_t* x, con
 tp_status launch_attn_fwd(const uint16_t* qkv, uint16_t* o, float* lse, int B, int S, int H,
                           int dh, int t, int causal, cudaStream_t stream);
 size_t attn_bwd_scratch_bytes(int B, int S, int H, int dh);
+// Largest dS^T array (bytes) the attention backward keeps for its dQ kernel;
+// returns the previous limit.
+size_t attn_set_dst_limit(size_t max_bytes);
 // colpart (may be null): column sums of dqkv, fp32 [B * ceil(S / 32)][t * 3Dt] (one
 // partial row per 32 rows of a batch element), for launch_colsum_reduce.
 tp_status launch_attn_bwd(const uint16_t* qkv, const uint16_t* o, const float* lse,

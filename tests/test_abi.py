@@ -140,3 +140,22 @@ def test_layer_forward_accepts_null_activations_at_zero_tokens():
     d1 = tl.Dims.of(1, 64, 256, 1024, 2, 128, 2)   # with tokens the buffers are required
     assert lib.tp_layer_fwd(ctypes.byref(d1), None, ctypes.byref(p), ctypes.byref(tl.LayerActs()),
                             None, None, 0, None) == 1
+
+
+def test_ds_limit_sizes_the_attention_backward_workspace():
+    # dS^T of all heads (fp16, S rounded up to 128) is part of the attention
+    # backward's workspace exactly when it fits under the limit.
+    d = tl.Dims.of(2, 300, 512, 0, 4, 128, 4)
+    prev = tl.attn_set_ds_limit(0)
+    try:
+        assert prev == 4 << 30
+        without = tl.workspace_size(tl.OP_ATTN_BWD, d)
+        s_pad = 384
+        need = 2 * 4 * s_pad * s_pad * 2
+        assert tl.attn_set_ds_limit(need) == 0
+        with_ds = tl.workspace_size(tl.OP_ATTN_BWD, d)
+        assert with_ds - without == need
+        tl.attn_set_ds_limit(need - 1)
+        assert tl.workspace_size(tl.OP_ATTN_BWD, d) == without
+    finally:
+        tl.attn_set_ds_limit(prev)

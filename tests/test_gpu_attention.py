@@ -12,6 +12,7 @@ from oracle import attention as oatt
 from oracle import layout as olay
 from parity import check
 from synth import Workload, make_inputs, to_f64, workload
+import tensor_transformer_layer_column_b200 as tl
 from tensor_transformer_layer_column_b200.sublayer import ShardedAttention
 
 pytestmark = pytest.mark.gpu
@@ -115,3 +116,22 @@ def test_attn_deterministic_run_to_run():
         assert torch.equal(o1[k], o2[k]), k
     for k in g1:
         assert torch.equal(g1[k], g2[k]), k
+
+
+@pytest.fixture
+def recompute_dq():
+    prev = tl.attn_set_ds_limit(0)
+    yield
+    tl.attn_set_ds_limit(prev)
+
+
+# With the dS^T limit at 0 the dq kernel recomputes q k^T and dO v^T instead
+# of reading dS^T back (the path problems too large to keep dS^T take).
+@pytest.mark.parametrize("B,S,H,dh,t,causal", SMALL[:6] + MANY_ITEMS)
+def test_attn_bwd_recomputed_scores_dq(B, S, H, dh, t, causal, recompute_dq):
+    require_gpu()
+    w = Workload("attn_test", "attn_fwdbwd", batch=B, seq=S, hidden=H * dh, heads=H,
+                 head_dim=dh, t=t, causal=causal)
+    inp = make_inputs(w, seed=11, random_affine=True)
+    o, grads = _run(w, inp, backward=True)
+    _compare(w, inp, o, grads)
