@@ -317,7 +317,8 @@ tp_status attn_bwd_impl(const Sizes& z, int causal, bf16p x16, bf16p wqkv16, bf1
   tp_status s = launch_gemm(g1, st);
   if (s != TP_OK) return s;
 
-  // dWout_i = O_i^T dY, M shards.
+  // dWout_i = O_i^T dY, M shards (launched below together with dWqkv: its
+  // 16 x 16 tiles alone leave the last round of clusters half empty).
   GemmProblem g2{};
   g2.m_shards = (int)z.t; g2.n_shards = 1; g2.Mt = (int)z.Dt; g2.Nt = (int)z.D;
   g2.k_shards = 1; g2.Kt = (int)z.T;
@@ -325,7 +326,6 @@ tp_status attn_bwd_impl(const Sizes& z, int causal, bf16p x16, bf16p wqkv16, bf1
   g2.b = op(dy, true, SHARD_NONE, z.D, z.T, 1, z.D, 0);
   g2.epi = EPI_LINEAR; g2.c = dwout;
   g2.c_ms = z.Dt * z.D; g2.c_ns = 0; g2.ldc = z.D;
-  if ((s = launch_gemm(g2, st)) != TP_OK) return s;
 
   // dbqkv = column sums of dqkv: the attention kernels' epilogues write partials.
   s = launch_attn_bwd(qkv, o, lse, dout, dqkv, (int)z.B, (int)z.S, (int)z.H, (int)z.dh, (int)z.t,
@@ -343,7 +343,7 @@ tp_status attn_bwd_impl(const Sizes& z, int causal, bf16p x16, bf16p wqkv16, bf1
   g3.b = op(dqkv, true, SHARD_MN, w3, z.T, z.t, w3, z.T * w3, true);
   g3.epi = EPI_LINEAR; g3.c = dwqkv;
   g3.c_ms = 0; g3.c_ns = z.D * w3; g3.ldc = w3;
-  if ((s = launch_gemm(g3, st)) != TP_OK) return s;
+  if ((s = launch_gemm2(g2, g3, st)) != TP_OK) return s;
 
   // dX = sum_i dqkv_i Wqkv_i^T (+ dres): the backward shard reduction (fp16 operands).
   GemmProblem g4{};

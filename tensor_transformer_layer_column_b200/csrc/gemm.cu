@@ -86,9 +86,11 @@ tp_status launch_inst(const CUtensorMap& ta, const CUtensorMap& tb, const GemmAr
   return cuda_status(cudaGetLastError());
 }
 
-// CTA-pair kernel: clusters of 2 CTAs, one 256 x 256 tile per cluster at a time.
+// CTA-pair kernel: clusters of 2 CTAs, one 256 x 256 tile per cluster at a
+// time, over the tiles of `args` and then of `args2` (num_tiles 0: none).
 template <bool A_MN, bool B_MN>
 tp_status launch_pair(const CUtensorMap& ta, const CUtensorMap& tb, const GemmArgs& args,
+                      const CUtensorMap& ta2, const CUtensorMap& tb2, const GemmArgs& args2,
                       double flops, cudaStream_t stream) {
   static int max_clusters[64] = {};
   int dev = 0;
@@ -117,34 +119,36 @@ tp_status launch_pair(const CUtensorMap& ta, const CUtensorMap& tb, const GemmAr
     if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0) return TP_ERR_CUDA;
     max_clusters[dev] = n;
   }
-  const int clusters = args.num_tiles < max_clusters[dev] ? args.num_tiles : max_clusters[dev];
+  const int tiles = args.num_tiles + args2.num_tiles;
+  const int clusters = tiles < max_clusters[dev] ? tiles : max_clusters[dev];
   cfg.gridDim = dim3(2 * clusters, 1, 1);
   cfg.numAttrs = 2;
   {
     TraceScope ts(stream, TK_GEMM, flops);
-    if (cudaLaunchKernelEx(&cfg, kern, ta, tb, args) != cudaSuccess) return TP_ERR_CUDA;
+    if (cudaLaunchKernelEx(&cfg, kern, ta, tb, args, ta2, tb2, args2) != cudaSuccess)
+      return TP_ERR_CUDA;
   }
   return cuda_status(cudaGetLastError());
 }
 
-}  // namespace
-
-tp_status launch_gemm(const GemmProblem& g, cudaStream_t stream) {
-  if (g.Mt <= 0 || g.Nt <= 0 || g.Kt <= 0) return TP_OK;   // empty product: nothing to do
+// Tensor maps and kernel arguments of one product; *pair: the CTA-pair
+// kernel runs it (one 128-row block does not cover M).
+tp_status prepare(const GemmProblem& g, CUtensorMap* ta, CUtensorMap* tb, GemmArgs* out,
+                  bool* pair_out, double* flops, bool force_pair = false) {
   if (g.a.f16 != g.b.f16) return TP_ERR_INVALID_ARG;       // one MMA takes one operand type
   // fp32 residual / output: plain linear epilogue, no fp16 store.
   if ((g.out_f32 || g.aux_f32) && (g.epi != EPI_LINEAR || g.out_f16)) return TP_ERR_INVALID_ARG;
   if (g.colpart != nullptr && g.m_shards != 1) return TP_ERR_INVALID_ARG;
-  // Pairs of CTAs (256-row tiles) unless one 128-row block covers M.
-  const bool pair = g.Mt > GEMM_BM;
+  // Pairs of CTAs (256-row tiles) unless one 128-row block covers M (or the
+  // caller asks for the pair kernel: rows past Mt read as zero and are not stored).
+  const bool pair = force_pair || g.Mt > GEMM_BM;
   const bool a_il = interleave_ok(g.a), b_il = interleave_ok(g.b);
-  CUtensorMap ta, tb;
-  if (a_il ? !encode_operand_il(&ta, g.a, GEMM_BM / 64)
-           : !encode_operand(&ta, g.a, g.a.mn_major ? 64 : GEMM_BM))
+  if (a_il ? !encode_operand_il(ta, g.a, GEMM_BM / 64)
+           : !encode_operand(ta, g.a, g.a.mn_major ? 64 : GEMM_BM))
     return TP_ERR_CUDA;
   const uint32_t b_rows = pair ? 128 : GEMM_BN;
-  if (b_il ? !encode_operand_il(&tb, g.b, b_rows / 64)
-           : !encode_operand(&tb, g.b, g.b.mn_major ? 64 : b_rows))
+  if (b_il ? !encode_operand_il(tb, g.b, b_rows / 64)
+           : !encode_operand(tb, g.b, g.b.mn_major ? 64 : b_rows))
     return TP_ERR_CUDA;
 
   GemmArgs a{};
@@ -180,20 +184,63 @@ tp_status launch_gemm(const GemmProblem& g, cudaStream_t stream) {
   a.b_il = b_il ? 1 : 0;
   a.colpart = g.colpart;
   a.colpart_ld = (long long)g.n_shards * g.Nt;
-  const int grid = (int)(tiles < sm_count() ? tiles : sm_count());
-  const double flops = 2.0 * g.m_shards * (double)g.Mt * g.n_shards * (double)g.Nt * g.k_shards *
-                       (double)g.Kt;
+  *out = a;
+  *pair_out = pair;
+  *flops = 2.0 * g.m_shards * (double)g.Mt * g.n_shards * (double)g.Nt * g.k_shards * (double)g.Kt;
+  return TP_OK;
+}
 
+tp_status pair_dispatch(bool a_mn, bool b_mn, const CUtensorMap& ta, const CUtensorMap& tb,
+                        const GemmArgs& a, const CUtensorMap& ta2, const CUtensorMap& tb2,
+                        const GemmArgs& a2, double flops, cudaStream_t stream) {
+  if (!a_mn && b_mn) return launch_pair<false, true>(ta, tb, a, ta2, tb2, a2, flops, stream);
+  if (!a_mn && !b_mn) return launch_pair<false, false>(ta, tb, a, ta2, tb2, a2, flops, stream);
+  if (a_mn && b_mn) return launch_pair<true, true>(ta, tb, a, ta2, tb2, a2, flops, stream);
+  return launch_pair<true, false>(ta, tb, a, ta2, tb2, a2, flops, stream);
+}
+
+}  // namespace
+
+tp_status launch_gemm(const GemmProblem& g, cudaStream_t stream) {
+  if (g.Mt <= 0 || g.Nt <= 0 || g.Kt <= 0) return TP_OK;   // empty product: nothing to do
+  CUtensorMap ta, tb;
+  GemmArgs a;
+  bool pair = false;
+  double flops = 0;
+  tp_status s = prepare(g, &ta, &tb, &a, &pair, &flops);
+  if (s != TP_OK) return s;
   if (pair) {
-    if (!g.a.mn_major && g.b.mn_major) return launch_pair<false, true>(ta, tb, a, flops, stream);
-    if (!g.a.mn_major && !g.b.mn_major) return launch_pair<false, false>(ta, tb, a, flops, stream);
-    if (g.a.mn_major && g.b.mn_major) return launch_pair<true, true>(ta, tb, a, flops, stream);
-    return launch_pair<true, false>(ta, tb, a, flops, stream);
+    GemmArgs none = a;
+    none.num_tiles = 0;
+    return pair_dispatch(g.a.mn_major, g.b.mn_major, ta, tb, a, ta, tb, none, flops, stream);
   }
+  const long long tiles = a.num_tiles;
+  const int grid = (int)(tiles < sm_count() ? tiles : sm_count());
   if (!g.a.mn_major && g.b.mn_major) return launch_inst<false, true>(ta, tb, a, grid, flops, stream);
   if (!g.a.mn_major && !g.b.mn_major) return launch_inst<false, false>(ta, tb, a, grid, flops, stream);
   if (g.a.mn_major && g.b.mn_major) return launch_inst<true, true>(ta, tb, a, grid, flops, stream);
   return launch_inst<true, false>(ta, tb, a, grid, flops, stream);
+}
+
+tp_status launch_gemm2(const GemmProblem& g1, const GemmProblem& g2, cudaStream_t stream) {
+  const bool e1 = g1.Mt <= 0 || g1.Nt <= 0 || g1.Kt <= 0;
+  const bool e2 = g2.Mt <= 0 || g2.Nt <= 0 || g2.Kt <= 0;
+  // One launch of the pair kernel when the operand majors agree (each tile's
+  // products take its own problem's operand type; a product with M <= 128
+  // runs on 256-row tiles here), so that the launch sequence does not depend
+  // on the sizes; otherwise one after the other.
+  if (e1 || e2 || g1.a.mn_major != g2.a.mn_major || g1.b.mn_major != g2.b.mn_major) {
+    tp_status s = launch_gemm(g1, stream);
+    return s != TP_OK ? s : launch_gemm(g2, stream);
+  }
+  CUtensorMap ta1, tb1, ta2, tb2;
+  GemmArgs a1, a2;
+  bool p1 = false, p2 = false;
+  double f1 = 0, f2 = 0;
+  tp_status s = prepare(g1, &ta1, &tb1, &a1, &p1, &f1, true);
+  if (s != TP_OK) return s;
+  if ((s = prepare(g2, &ta2, &tb2, &a2, &p2, &f2, true)) != TP_OK) return s;
+  return pair_dispatch(g1.a.mn_major, g1.b.mn_major, ta1, tb1, a1, ta2, tb2, a2, f1 + f2, stream);
 }
 
 }  // namespace tp

@@ -19,7 +19,10 @@
 //     pair).  Each CTA's producer stages its half of A and of B through a
 //     6-stage TMA ring; the even CTA's single MMA thread issues 4 MMAs of
 //     256 x 256 x 16 per 64-wide k-block into one of two 256-column TMEM
-//     accumulators and commits stage releases to both CTAs.
+//     accumulators and commits stage releases to both CTAs.  One launch may
+//     carry two independent products (their tiles one after the other in the
+//     clusters' walk), so that two short products fill each other's partial
+//     last round.
 //   gemm_bf16_sm100 (M <= 128): one CTA per 128 x 256 tile, 4-stage ring,
 //     4 MMAs of 128 x 256 x 16 per k-block.
 // Roles in both: warp 0 TMA producer; warp 1 TMEM owner and MMA issuer (one
@@ -538,10 +541,16 @@ __device__ __forceinline__ TileCoord gemm_pair_tile(const GemmArgs& p, int tile)
   return tc;
 }
 
+// Two products in one launch: tiles 0 .. p.num_tiles-1 are product p (maps
+// tmA, tmB), the next p2.num_tiles are product p2 (maps tmA2, tmB2; same
+// operand majors and type).  One launch of two products whose tile counts
+// leave partial last rounds of clusters fills those rounds with each other's
+// tiles.  p2.num_tiles = 0 for a single product.
 template <bool A_MN, bool B_MN>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
 gemm_pair_sm100(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                const GemmArgs p) {
+                const __grid_constant__ GemmArgs p, const __grid_constant__ CUtensorMap tmA2,
+                const __grid_constant__ CUtensorMap tmB2, const __grid_constant__ GemmArgs p2) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
@@ -573,6 +582,10 @@ gemm_pair_sm100(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
     fence_mbar_init();
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
+    if (p2.num_tiles > 0) {
+      tma_prefetch_desc(&tmA2);
+      tma_prefetch_desc(&tmB2);
+    }
   }
   if (warp == 1) {
     tmem_alloc_pair(tmem_slot, GEMM_TMEM_COLS);
@@ -583,8 +596,8 @@ gemm_pair_sm100(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
   cluster_sync();                   // the peer's barriers exist before anyone signals them
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const int num_kb = p.k_shards * p.kb_per_shard;
   const int cid = (int)cluster_id_x(), ncl = (int)nclusters_x();
+  const int ntiles = p.num_tiles + p2.num_tiles;
   grid_dep_wait();                  // operands and outputs: the previous kernels have completed
   grid_dep_launch();
 
@@ -592,43 +605,50 @@ gemm_pair_sm100(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
     if (lane == 0) {
       int it = 0;
       bool ok = true;
-      for (int tile = cid; tile < p.num_tiles && ok; tile += ncl) {
-        const TileCoord tc = gemm_pair_tile(p, tile);
+      // One tile's k-blocks; called with the kernel parameter of its product
+      // itself, so that every field is read from the parameter space.
+      auto produce = [&](const GemmArgs& q, const CUtensorMap* ta, const CUtensorMap* tb,
+                         int ltile) {
+        const TileCoord tc = gemm_pair_tile(q, ltile);
         const int am = tc.m0 + (int)rank * 128;
         const int bn = tc.n0 + (int)rank * 128;
+        const int num_kb = q.k_shards * q.kb_per_shard;
         for (int kb = 0; kb < num_kb; ++kb, ++it) {
           const int s = it % GP_STAGES;
           const uint32_t round = it / GP_STAGES;
           if (!wait_or_abort(&empty[s], (round & 1) ^ 1, abort_flag)) {
             record_error(p.err, abort_flag, ERR_GEMMP_PRODUCER_WAIT);
-            ok = false;
-            break;
+            return false;
           }
-          const int ks = kb / p.kb_per_shard;
-          const int k0 = (kb - ks * p.kb_per_shard) * GEMM_BK;
-          const int a_s = p.a_src == SHARD_K ? ks : (p.a_src == SHARD_MN ? tc.ms : 0);
-          const int b_s = p.b_src == SHARD_K ? ks : (p.b_src == SHARD_MN ? tc.ns : 0);
+          const int ks = kb / q.kb_per_shard;
+          const int k0 = (kb - ks * q.kb_per_shard) * GEMM_BK;
+          const int a_s = q.a_src == SHARD_K ? ks : (q.a_src == SHARD_MN ? tc.ms : 0);
+          const int b_s = q.b_src == SHARD_K ? ks : (q.b_src == SHARD_MN ? tc.ns : 0);
           uint8_t* sa = smem + s * GP_STAGE_BYTES;
           uint8_t* sb = sa + GP_A_BYTES;
           if (leader) mbar_arrive_expect_tx(&full[s], 2 * GP_STAGE_BYTES);
-          if (A_MN && p.a_il) {
-            tma_load_5d_pair(sa, &tmA, &full[s], 0, 0, am / 64, k0 / 8, a_s);
+          if (A_MN && q.a_il) {
+            tma_load_5d_pair(sa, ta, &full[s], 0, 0, am / 64, k0 / 8, a_s);
           } else if (A_MN) {
-            tma_load_3d_pair(sa, &tmA, &full[s], am, k0, a_s);
-            tma_load_3d_pair(sa + 8192, &tmA, &full[s], am + 64, k0, a_s);
+            tma_load_3d_pair(sa, ta, &full[s], am, k0, a_s);
+            tma_load_3d_pair(sa + 8192, ta, &full[s], am + 64, k0, a_s);
           } else {
-            tma_load_3d_pair(sa, &tmA, &full[s], k0, am, a_s);
+            tma_load_3d_pair(sa, ta, &full[s], k0, am, a_s);
           }
-          if (B_MN && p.b_il) {
-            tma_load_5d_pair(sb, &tmB, &full[s], 0, 0, bn / 64, k0 / 8, b_s);
+          if (B_MN && q.b_il) {
+            tma_load_5d_pair(sb, tb, &full[s], 0, 0, bn / 64, k0 / 8, b_s);
           } else if (B_MN) {
-            tma_load_3d_pair(sb, &tmB, &full[s], bn, k0, b_s);
-            tma_load_3d_pair(sb + 8192, &tmB, &full[s], bn + 64, k0, b_s);
+            tma_load_3d_pair(sb, tb, &full[s], bn, k0, b_s);
+            tma_load_3d_pair(sb + 8192, tb, &full[s], bn + 64, k0, b_s);
           } else {
-            tma_load_3d_pair(sb, &tmB, &full[s], k0, bn, b_s);
+            tma_load_3d_pair(sb, tb, &full[s], k0, bn, b_s);
           }
         }
-      }
+        return true;
+      };
+      for (int tile = cid; tile < ntiles && ok; tile += ncl)
+        ok = tile < p.num_tiles ? produce(p, &tmA, &tmB, tile)
+                                : produce(p2, &tmA2, &tmB2, tile - p.num_tiles);
       if (leader) {
         const int issued = it;
         for (int j = 0; j < GP_STAGES && j < issued; ++j) {
@@ -640,10 +660,13 @@ gemm_pair_sm100(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
   } else if (warp == 1) {
     if (lane == 0) {
       if (leader) {
-        const uint32_t idesc = p.idesc;
         int it = 0, tcount = 0;
         bool ok = true;
-        for (int tile = cid; tile < p.num_tiles && ok; tile += ncl, ++tcount) {
+        for (int tile = cid; tile < ntiles && ok; tile += ncl, ++tcount) {
+          const bool sec = tile >= p.num_tiles;
+          const uint32_t idesc = sec ? p2.idesc : p.idesc;
+          const int num_kb = sec ? p2.k_shards * p2.kb_per_shard : p.k_shards * p.kb_per_shard;
+          const bool a_il = sec ? p2.a_il : p.a_il, b_il = sec ? p2.b_il : p.b_il;
           const int acc = tcount & 1;
           const uint32_t use = tcount >> 1;
           if (!wait_or_abort(&tempty[acc], (use & 1) ^ 1, abort_flag)) {
@@ -665,9 +688,9 @@ gemm_pair_sm100(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
             const uint32_t sb = sa + GP_A_BYTES;
 #pragma unroll
             for (int kk = 0; kk < GEMM_BK / 16; ++kk) {
-              const uint64_t ad = A_MN ? mn_desc(sa, 2, kk, p.a_il)
+              const uint64_t ad = A_MN ? mn_desc(sa, 2, kk, a_il)
                                        : smem_desc_sw128(sa + kk * 32, 16, 1024);
-              const uint64_t bd = B_MN ? mn_desc(sb, 2, kk, p.b_il)
+              const uint64_t bd = B_MN ? mn_desc(sb, 2, kk, b_il)
                                        : smem_desc_sw128(sb + kk * 32, 16, 1024);
               tc_mma_f16_pair(d_tmem, ad, bd, idesc, (kb | kk) != 0);
             }
@@ -687,18 +710,13 @@ gemm_pair_sm100(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
     const int c0 = ((warp - 2) / 4) * CPW;
     const uint32_t tempty_leader0 = map_to_rank(&tempty[0], 0);
     int tcount = 0;
-    for (int tile = cid; tile < p.num_tiles; tile += ncl, ++tcount) {
-      const TileCoord tc = gemm_pair_tile(p, tile);
-      const int acc = tcount & 1;
-      const uint32_t use = tcount >> 1;
-      if (!__all_sync(0xffffffffu, wait_or_abort(&tfull[acc], use & 1, abort_flag))) {
-        record_error(p.err, abort_flag, ERR_GEMMP_EPI_WAIT);
-        break;
-      }
-      tc_fence_after();
+    // One tile's epilogue, called like the producer's with its product's
+    // kernel parameter itself.
+    auto drain_tile = [&](const GemmArgs& q, int ltile, int acc) {
+      const TileCoord tc = gemm_pair_tile(q, ltile);
       const int m = tc.m0 + (int)rank * 128 + row;
-      const bool row_ok = m < p.Mt;
-      const long long base = tc.ms * p.c_ms + tc.ns * p.c_ns + (long long)m * p.ldc;
+      const bool row_ok = m < q.Mt;
+      const long long base = tc.ms * q.c_ms + tc.ns * q.c_ns + (long long)m * q.ldc;
       const uint32_t taddr = tmem_base + ((uint32_t)(quad * 32) << 16) + acc * GP_BN;
 #pragma unroll 1
       for (int c = c0; c < c0 + CPW; ++c) {
@@ -706,9 +724,20 @@ gemm_pair_sm100(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
         tmem_ld32(taddr + c * 32, r);
         tc_wait_ld();
         const int n = tc.n0 + c * 32;
-        if (n >= p.Nt) continue;   // the same for every lane of the warp
-        epilogue_chunk(p, r, tc.ns, base, n, row_ok, (tc.m0 + (int)rank * 128 + quad * 32) / 32);
+        if (n >= q.Nt) continue;   // the same for every lane of the warp
+        epilogue_chunk(q, r, tc.ns, base, n, row_ok, (tc.m0 + (int)rank * 128 + quad * 32) / 32);
       }
+    };
+    for (int tile = cid; tile < ntiles; tile += ncl, ++tcount) {
+      const int acc = tcount & 1;
+      const uint32_t use = tcount >> 1;
+      if (!__all_sync(0xffffffffu, wait_or_abort(&tfull[acc], use & 1, abort_flag))) {
+        record_error(p.err, abort_flag, ERR_GEMMP_EPI_WAIT);
+        break;
+      }
+      tc_fence_after();
+      if (tile < p.num_tiles) drain_tile(p, tile, acc);
+      else drain_tile(p2, tile - p.num_tiles, acc);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(tempty_leader0 + acc * 8);

@@ -45,6 +45,11 @@ struct GemmProblem {
 };
 
 tp_status launch_gemm(const GemmProblem& g, cudaStream_t stream);
+// g1 then g2 in one launch of the CTA-pair kernel when both run on it with
+// the same operand majors (the tiles of both fill the clusters' rounds
+// together; each keeps its own operand type); otherwise two launches.  The
+// products must not depend on each other.
+tp_status launch_gemm2(const GemmProblem& g1, const GemmProblem& g2, cudaStream_t stream);
 
 // Launch with the programmatic-serialization attribute (see pdl.cuh).
 template <typename... KArgs, typename... Args>
