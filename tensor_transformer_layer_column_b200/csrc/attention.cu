@@ -1322,33 +1322,38 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q128,
 // ---------------------------------------------------------------- dQ from stored dS
 // When the dK/dV kernel also stores dS^T (fp16, the same values it feeds to
 // dK += dS^T q; AttnArgs::dst gives the layout), dQ = dS k needs no
-// recomputation of S and dP: per 128-query block, walk 64-key blocks through
-// a 3-stage ring of (dS^T tile, k tile) and accumulate dQ += dS k with dS as
-// an MN-major A operand (queries contiguous in each key row; two bulk copies
-// of 8 KiB, contiguous in global memory) and k as an MN-major B operand (TMA).  Warp 0 loads, warp 1 issues the
-// products, warps 2-5 (one per TMEM lane quarter) write dQ.  128 TMEM
-// columns and 96 KB of shared memory: two CTAs share an SM, so one's
-// epilogue overlaps the other's products.
+// recomputation of S and dP: per 256-query block (two 128-row halves, each
+// with its own accumulator), walk 64-key blocks through a 2-stage ring of
+// (dS^T tile, k tile) and accumulate dQ += dS k with dS as an MN-major A
+// operand (queries contiguous in each key row; bulk copies of 8 KiB,
+// contiguous in global memory) and k as an MN-major B operand (TMA), each k
+// tile serving both halves.  Under the causal mask the first half stops two
+// key blocks before the second (dS^T past its diagonal was never written).
+// Warp 0 loads, warp 1 issues the products, warps 2-9 (two per TMEM lane
+// quarter, one per half) write dQ.  256 TMEM columns and 96 KB of shared
+// memory: two CTAs share an SM, so one's epilogue overlaps the other's
+// products.
 template <int DH>
 struct DqdsCfg {
-  static constexpr int BQ = 128, BK = 64, CH = DH / 64, STAGES = 3;
-  static constexpr int A_BYTES = BQ * BK * 2;                // dS^T tile: 64 key rows x 128 queries
+  static constexpr int BQ = 256, BK = 64, CH = DH / 64, STAGES = 2;
+  static constexpr int HALF_BYTES = 128 * BK * 2;            // dS^T of one half: 64 key rows x 128 queries
+  static constexpr int A_BYTES = 2 * HALF_BYTES;
   static constexpr int K_BYTES = BK * DH * 2;                // k tile
   static constexpr int STAGE_BYTES = A_BYTES + K_BYTES;
   static constexpr int OFF_BAR = STAGES * STAGE_BYTES;
   static constexpr int SMEM = OFF_BAR + 256 + 1024;
-  static constexpr int THREADS = 192;
+  static constexpr int THREADS = 320;
 };
 
 template <int DH>
-__global__ void __launch_bounds__(192, 2)
+__global__ void __launch_bounds__(320, 2)
 attn_bwd_dq_ds_kernel(const __grid_constant__ CUtensorMap tm_kv64, const AttnArgs p) {
   using C = DqdsCfg<DH>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
-  uint64_t* full = bars + 0;       // [STAGES]
+  uint64_t* full = bars + 0;       // [STAGES <= 3]
   uint64_t* empty = bars + 3;      // [STAGES]
   uint64_t* acc_full = bars + 6;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 7);
@@ -1362,11 +1367,17 @@ attn_bwd_dq_ds_kernel(const __grid_constant__ CUtensorMap tm_kv64, const AttnArg
   const int shard = h / p.Ht, hl = h - shard * p.Ht;
   const int q0 = qb * C::BQ;
   const int nkb = (p.S + C::BK - 1) / C::BK;
-  const int nsteps = p.causal ? min(nkb, (q0 + C::BQ) / C::BK) : nkb;
+  // Key blocks of each half (a half wholly past S has none); the second
+  // half's count is the block's.
+  auto half_blocks = [&](int qs) {
+    return qs >= p.S ? 0 : (p.causal ? min(nkb, (qs + 128) / C::BK) : nkb);
+  };
+  const int nk0 = half_blocks(q0), nk1 = half_blocks(q0 + 128);
+  const int nsteps = max(nk0, nk1);
   const int colq = hl * DH, colk = p.Dt + hl * DH;
   const int bh = b * p.H + h;
   // dS^T pieces of this query block (its first 64-query column, key piece 0).
-  const uint16_t* ds_col = p.dst + ((long long)bh * (p.S_pad / 64) + 2 * qb) * (p.S_pad / 32) * 2048;
+  const uint16_t* ds_col = p.dst + ((long long)bh * (p.S_pad / 64) + 4 * qb) * (p.S_pad / 32) * 2048;
   const Ctl ctl{abort_flag, p.err};
 
   if (threadIdx.x == 0) {
@@ -1380,13 +1391,13 @@ attn_bwd_dq_ds_kernel(const __grid_constant__ CUtensorMap tm_kv64, const AttnArg
     tma_prefetch_desc(&tm_kv64);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, 128);
+    tmem_alloc(tmem_slot, 256);
     tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t t_dq = *tmem_slot;
+  const uint32_t t_dq = *tmem_slot;   // half j at column 128 j
   grid_dep_wait();   // inputs and outputs: the previous kernels have completed
   grid_dep_launch();
 
@@ -1399,11 +1410,18 @@ attn_bwd_dq_ds_kernel(const __grid_constant__ CUtensorMap tm_kv64, const AttnArg
         if (!wait_bar(&empty[st], (u & 1) ^ 1, ctl, ERR_ATTN_DQ_WAIT)) break;
         uint8_t* sa = smem + st * C::STAGE_BYTES;
         uint8_t* sk = sa + C::A_BYTES;
-        mbar_arrive_expect_tx(&full[st], C::STAGE_BYTES);
-        // Two 64-query chunks of 64 key rows: two consecutive 32-key pieces each.
-        for (int c = 0; c < C::BQ / 64; ++c)
-          bulk_load(sa + c * C::BK * 128, ds_col + (long long)c * (p.S_pad / 32) * 2048 + k * 4096,
-                    C::BK * 128, &full[st]);
+        const bool a0 = k < nk0, a1 = k < nk1;
+        mbar_arrive_expect_tx(&full[st], ((int)a0 + (int)a1) * C::HALF_BYTES + C::K_BYTES);
+        // Each active half: two 64-query chunks of 64 key rows, two
+        // consecutive 32-key pieces each.
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          if (!(j == 0 ? a0 : a1)) continue;
+          for (int c = 0; c < 2; ++c)
+            bulk_load(sa + j * C::HALF_BYTES + c * C::BK * 128,
+                      ds_col + (long long)(2 * j + c) * (p.S_pad / 32) * 2048 + k * 4096,
+                      C::BK * 128, &full[st]);
+        }
         for (int c = 0; c < C::CH; ++c)
           tma_load_4d(sk + c * C::BK * 128, &tm_kv64, &full[st], colk + 64 * c, k * C::BK, b, shard);
       }
@@ -1421,29 +1439,34 @@ attn_bwd_dq_ds_kernel(const __grid_constant__ CUtensorMap tm_kv64, const AttnArg
         const uint32_t sa = smem_u32(smem + st * C::STAGE_BYTES);
         const uint32_t sk = sa + C::A_BYTES;
 #pragma unroll
-        for (int kk = 0; kk < C::BK / 16; ++kk)   // 16 keys per product
-          tc_mma_f16(t_dq, mnmajor_desc(sa, C::BK, kk),
-                     mnmajor_desc(sk, C::BK, kk), id_acc, (k | kk) != 0);
+        for (int j = 0; j < 2; ++j) {
+          if (k >= (j == 0 ? nk0 : nk1)) continue;
+#pragma unroll
+          for (int kk = 0; kk < C::BK / 16; ++kk)   // 16 keys per product
+            tc_mma_f16(t_dq + 128 * j, mnmajor_desc(sa + j * C::HALF_BYTES, C::BK, kk),
+                       mnmajor_desc(sk, C::BK, kk), id_acc, (k | kk) != 0);
+        }
         tc_commit(&empty[st]);
       }
       tc_commit(acc_full);   // also after an early stop: every issued product completes
       mbar_wait(acc_full, 0, 200000000ull);
     }
   } else {
-    // Epilogue warps 2-5 (TMEM lane quarter warp % 4).
+    // Epilogue warps 2-9: half j = (warp - 2) / 4, TMEM lane quarter warp % 4.
+    const int j = (warp - 2) >> 2;
     const int quad = warp & 3;
     const int r = quad * 32 + lane;
-    const int q = q0 + r;
+    const int q = q0 + 128 * j + r;
     const bool qvalid = q < p.S;
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-    if (nsteps > 0 && __all_sync(0xffffffffu, wait_bar(acc_full, 0, ctl, ERR_ATTN_DQ_WAIT))) {
+    if ((j == 0 ? nk0 : nk1) > 0 && __all_sync(0xffffffffu, wait_bar(acc_full, 0, ctl, ERR_ATTN_DQ_WAIT))) {
       tc_fence_after();
       const long long w3 = 3LL * p.Dt;
       uint16_t* row = p.out + (long long)shard * p.T * w3 + ((long long)b * p.S + q) * w3 + colq;
 #pragma unroll 1
       for (int c = 0; c < DH / 32; ++c) {
         uint32_t rq[32];
-        tmem_ld32(t_dq + lane_off + c * 32, rq);
+        tmem_ld32(t_dq + 128 * j + lane_off + c * 32, rq);
         tc_wait_ld();
         float v[32];
 #pragma unroll
@@ -1457,7 +1480,8 @@ attn_bwd_dq_ds_kernel(const __grid_constant__ CUtensorMap tm_kv64, const AttnArg
             *reinterpret_cast<uint4*>(row + c * 32 + g * 8) = pack8_f16(&v[g * 8]);
           if (over && p.err) atomicCAS(p.err, 0u, 0x301u);
         }
-        if (p.colpart != nullptr) colpart_store(p, v, b, q0 + quad * 32, shard, colq + c * 32);
+        if (p.colpart != nullptr)
+          colpart_store(p, v, b, q0 + 128 * j + quad * 32, shard, colq + c * 32);
       }
     }
   }
@@ -1465,7 +1489,7 @@ attn_bwd_dq_ds_kernel(const __grid_constant__ CUtensorMap tm_kv64, const AttnArg
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(t_dq, 128);
+    tmem_dealloc(t_dq, 256);
   }
 }
 
