@@ -26,9 +26,10 @@
 //           P^T, dS^T = P^T * (dP^T - Dv) by one thread per key row,
 //           dV += P^T dO, dK += dS^T q; also stores dS^T (fp16) when the
 //           array fits under the limit attn_set_dst_limit sets
-//   dQ:     per 128-query block, walk 64-key blocks: dQ += dS k, dS read
-//           back from that array; above the limit the dQ kernel recomputes
-//           S = q k^T, dP = dO v^T, dS = P * (dP - Dv) instead
+//   dQ:     per 256-query block, walk 64-key blocks: dQ += dS k, dS read
+//           back from that array; above the limit a dQ kernel over 128-query
+//           blocks recomputes S = q k^T, dP = dO v^T, dS = P * (dP - Dv)
+//           instead
 //   dK/dV and the recomputing dQ are persistent: one CTA per SM walks its
 //   work items (snake order, longest first) with the pipelines carried from
 //   item to item and four epilogue warps writing an item's dK/dV or dQ while
