@@ -159,3 +159,20 @@ def test_ds_limit_sizes_the_attention_backward_workspace():
         assert tl.workspace_size(tl.OP_ATTN_BWD, d) == without
     finally:
         tl.attn_set_ds_limit(prev)
+
+
+def test_ds_limit_enters_the_layer_backward_workspace():
+    # The layer backward shares one region between the MLP and attention
+    # backwards (the larger of the two); at c5 the attention part with dS^T
+    # (1.07 GB) is the larger, without it the MLP's.
+    d = tl.Dims.of(4, 2048, 4096, 16384, 32, 128, 8)
+    prev = tl.attn_set_ds_limit(0)
+    try:
+        without = tl.workspace_size(tl.OP_LAYER_BWD, d)
+        tl.attn_set_ds_limit(prev)
+        with_ds = tl.workspace_size(tl.OP_LAYER_BWD, d)
+    finally:
+        tl.attn_set_ds_limit(prev)
+    dst = 4 * 32 * 2048 * 2048 * 2
+    assert without < with_ds <= without + dst
+    assert tl.workspace_size(tl.OP_LAYER_FWD, d) > 0
