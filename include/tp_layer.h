@@ -228,9 +228,10 @@ tp_status tp_attn_bwd(const tp_dims* dims, const tp_bf16* x, const tp_bf16* wqkv
  * saved lse instead.  The two give dq equal up to fp32 rounding order.  The
  * limit is process-wide, 4 GiB by default (0: always recompute), and enters
  * tp_workspace_size and tp_rank_workspace_size for TP_OP_ATTN_BWD and the
- * layer backward ops: set it while no such call is running and size
- * workspaces after setting it (a smaller workspace gives TP_ERR_WORKSPACE).
- * Returns the previous limit.  Not an operation of the pages: a choice of
+ * layer backward ops: size workspaces after setting it (a smaller workspace
+ * gives TP_ERR_WORKSPACE).  A call already running keeps the value it read
+ * when it started, so setting the limit from another thread never changes
+ * the workspace a running call expects.  Returns the previous limit.  Not an operation of the pages: a choice of
  * how to run the backward of their attention. */
 size_t tp_attn_set_ds_limit(size_t max_bytes);
 

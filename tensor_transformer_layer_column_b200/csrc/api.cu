@@ -462,6 +462,7 @@ const char* tp_status_string(tp_status s) {
 size_t tp_attn_set_ds_limit(size_t max_bytes) { return attn_set_dst_limit(max_bytes); }
 
 size_t tp_workspace_size(int op_, const tp_dims* d) {
+  DstLimitPin pin;   // one dS^T limit for the whole call
   switch (op_) {
     case TP_OP_MLP_FWD: return 0;
     case TP_OP_ATTN_FWD: return check_attn(d) == TP_OK ? attn_fwd_ws(sizes_of(*d)) : 0;
@@ -607,6 +608,7 @@ tp_status tp_attn_bwd(const tp_dims* dims, const tp_bf16* x, const tp_bf16* wqkv
                       const float* lse_save, const tp_bf16* dy, const tp_bf16* dres, tp_bf16* dx,
                       tp_bf16* dwqkv, tp_bf16* dbqkv, tp_bf16* dwout, tp_bf16* dbout, void* ws,
                       size_t ws_bytes, tp_stream s) {
+  DstLimitPin pin;   // one dS^T limit for the whole call
   tp_status st = check_attn(dims);
   if (st != TP_OK) return st;
   const bool tok = (long long)dims->batch * dims->seq > 0;
@@ -818,6 +820,7 @@ tp_status tp_layer_fwd(const tp_dims* dims, const tp_bf16* x, const tp_layer_par
 tp_status tp_layer_bwd(const tp_dims* dims, const tp_bf16* x, const tp_layer_params* p,
                        const tp_layer_acts* a, const tp_bf16* dy, tp_bf16* dx,
                        const tp_layer_grads* g, void* ws, size_t ws_bytes, tp_stream s) {
+  DstLimitPin pin;   // one dS^T limit for the whole call
   tp_status st = check_layer(dims);
   if (st != TP_OK) return st;
   if ((st = check_layer_ptrs(p, a, has_tokens(dims))) != TP_OK) return st;
@@ -834,6 +837,7 @@ tp_status tp_layer_bwd_notify(const tp_dims* dims, const tp_bf16* x, const tp_la
                               const tp_layer_acts* a, const tp_bf16* dy, tp_bf16* dx,
                               const tp_layer_grads* g, const tp_grad_ready* ready, void* ws,
                               size_t ws_bytes, tp_stream s) {
+  DstLimitPin pin;   // one dS^T limit for the whole call
   tp_status st = check_layer(dims);
   if (st != TP_OK) return st;
   if ((st = check_layer_ptrs(p, a, has_tokens(dims))) != TP_OK) return st;
@@ -875,6 +879,7 @@ tp_status tp_layer_fwd_nosave(const tp_dims* dims, const tp_bf16* x, const tp_la
 tp_status tp_layer_bwd_recompute(const tp_dims* dims, const tp_bf16* x, const tp_layer_params* p,
                                  const tp_bf16* dy, tp_bf16* dx, const tp_layer_grads* g,
                                  void* ws, size_t ws_bytes, tp_stream s) {
+  DstLimitPin pin;   // one dS^T limit for the whole call
   tp_status st = check_layer(dims);
   if (st != TP_OK) return st;
   if ((st = check_layer_params(p)) != TP_OK) return st;
@@ -945,6 +950,7 @@ tp_status tp_postln_layer_fwd(const tp_dims* dims, const tp_bf16* x, const tp_la
 tp_status tp_postln_layer_bwd(const tp_dims* dims, const tp_bf16* x, const tp_layer_params* p,
                               const tp_postln_acts* a, const tp_bf16* dy, tp_bf16* dx,
                               const tp_layer_grads* g, void* ws, size_t ws_bytes, tp_stream s) {
+  DstLimitPin pin;   // one dS^T limit for the whole call
   tp_status st = check_layer(dims);
   if (st != TP_OK) return st;
   if ((st = check_postln_ptrs(p, a, has_tokens(dims))) != TP_OK) return st;

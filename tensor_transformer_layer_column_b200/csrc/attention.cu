@@ -1537,7 +1537,14 @@ size_t dst_bytes(int B, int S, int H) {
   return (size_t)B * H * s_pad * s_pad * 2;
 }
 
-bool keep_dst(int B, int S, int H) { return dst_bytes(B, S, H) <= g_dst_max.load(); }
+// A library call pins the limit for its thread (DstLimitPin), so that its
+// workspace check, its carving and its launches all see one value.
+thread_local bool t_dst_pinned = false;
+thread_local size_t t_dst_limit = 0;
+
+size_t dst_limit_now() { return t_dst_pinned ? t_dst_limit : g_dst_max.load(); }
+
+bool keep_dst(int B, int S, int H) { return dst_bytes(B, S, H) <= dst_limit_now(); }
 
 // Opt the kernel into `bytes` of dynamic shared memory once per device.
 bool set_smem(const void* kern, int bytes) {
@@ -1675,6 +1682,17 @@ tp_status launch_attn_fwd(const uint16_t* qkv, uint16_t* o, float* lse, int B, i
 }
 
 size_t attn_set_dst_limit(size_t max_bytes) { return g_dst_max.exchange(max_bytes); }
+
+DstLimitPin::DstLimitPin() : outer_(!t_dst_pinned) {
+  if (outer_) {
+    t_dst_limit = g_dst_max.load();
+    t_dst_pinned = true;
+  }
+}
+
+DstLimitPin::~DstLimitPin() {
+  if (outer_) t_dst_pinned = false;
+}
 
 size_t attn_bwd_scratch_bytes(int B, int S, int H, int dh) {
   (void)dh;

@@ -124,6 +124,17 @@ size_t attn_bwd_scratch_bytes(int B, int S, int H, int dh);
 // Largest dS^T array (bytes) the attention backward keeps for its dQ kernel;
 // returns the previous limit.
 size_t attn_set_dst_limit(size_t max_bytes);
+// While one is in scope, the calling thread reads the limit as it was when
+// the outermost one was made: a library call that sizes, checks and carves a
+// workspace and then launches into it sees one value, whatever another
+// thread sets meanwhile.
+struct DstLimitPin {
+  DstLimitPin();
+  ~DstLimitPin();
+  DstLimitPin(const DstLimitPin&) = delete;
+  DstLimitPin& operator=(const DstLimitPin&) = delete;
+  bool outer_;
+};
 // colpart (may be null): column sums of dqkv, fp32 [B * ceil(S / 32)][t * 3Dt] (one
 // partial row per 32 rows of a batch element), for launch_colsum_reduce.
 tp_status launch_attn_bwd(const uint16_t* qkv, const uint16_t* o, const float* lse,

@@ -161,6 +161,7 @@ using namespace tp;
 extern "C" {
 
 size_t tp_rank_workspace_size(int op, const tp_dims* dims) {
+  DstLimitPin pin;   // one dS^T limit for the whole call
   switch (op) {
     case TP_RANK_MLP_FWD: return 0;
     case TP_RANK_MLP_BWD: return check_mlp(dims) == TP_OK ? mlp_bwd_rank_ws(rank_sizes(*dims)) : 0;
@@ -349,6 +350,7 @@ tp_status tp_attn_bwd_rank(const tp_dims* dims, const tp_bf16* x, const tp_f16* 
                            const tp_bf16* o_i, const float* lse_i, const tp_bf16* dy,
                            tp_bf16* dwqkv_i, tp_bf16* dbqkv_i, tp_bf16* dwout_i, tp_bf16* dbout,
                            float* partial, void* ws, size_t ws_bytes, tp_stream stream) {
+  DstLimitPin pin;   // one dS^T limit for the whole call
   tp_status st = check_attn(dims);
   if (st != TP_OK) return st;
   const RankSizes z = rank_sizes(*dims);
